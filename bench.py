@@ -1,0 +1,340 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA sequence-mixing hot path on B200.
+
+One step = one kda_prefill over the long-context workload (1 sequence x
+T = 65,536 tokens, 64 heads x 128, bf16 inputs, fp32 state, gates near the -5
+floor on 10 % of channels).  `value` is prefill tokens/s over the whole job
+(all ranks), timed on the device with CUDA events, inputs resident in HBM.
+The same line carries the decode-step state bandwidth (256 sequences x 64
+heads, 1 GiB of fp32 state read and written in place) with its own roofline,
+the end-to-end number through the C ABI with host buffers, the oracle's CPU
+throughput, and the SM clocks sampled during the timed region.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own
+independent sequence (the path shards by sequence/head with no exchange), so
+scaling is weak; time = max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_inputs as ki  # noqa: E402
+
+METRIC = "KDA prefill tokens/s (64 heads, T=64k) and decode state GB/s vs HBM peak"
+WORKLOAD = "kda_prefill long-context: 1 x T=65536, 64 heads x 128, bf16 in / fp32 state, chunk 64"
+H, D, T_LONG = 64, 128, 65536
+# algorithmic bytes (what the method must move): per token-head q,k,v,g (4 x 256 B bf16)
+# + beta (2 B) + o (256 B); per (sequence, head) the final state (64 KiB; no initial
+# state in this workload).
+BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 2 + D * 2
+STATE_BYTES = D * D * 4
+# decode: per (sequence, head) the state read + written, q/k/v/g in, o out, beta,
+# the conv cache (3 tokens x q/k/v read, 3 written)
+DEC_BYTES_PER_PAIR = 2 * STATE_BYTES + 4 * D * 2 + D * 2 + 2 + 2 * 9 * D * 2
+# kernels launched per call: kda_prefill bf16 = main kernel + conv-tail kernel
+PREFILL_LAUNCHES = 2
+DECODE_LAUNCHES = 1
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "linear_attention_sequence_kda_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, x in enumerate(r) if x.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, steps, warmup, world, stream):
+    """W untimed steps, then K steps bracketed by barrier + synchronize, with
+    a CUDA event pair per step on the launching stream.  Returns (total ms,
+    per-step ms list), the total being the max over ranks."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    total = max_over_ranks(start.elapsed_time(stop), world)
+    return total, [a.elapsed_time(b) for a, b in evs]
+
+
+def cpu_baseline(tokens: int = 8192):
+    """The fp64 oracle as it stands on this host's cores: all 64 heads of the
+    long-context workload over its first `tokens` tokens."""
+    import oracle  # test infrastructure; only this leg of the benchmark runs it
+    inp = ki.make_prefill([tokens], H, torch.bfloat16, ki.BASE_SEED + 2, gate="bimodal")
+    probs = [oracle.prefill_problem(inp, 0, h) for h in range(H)]
+    cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    used = oracle.run_problems(probs, cores)
+    dt = time.perf_counter() - t0
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"first {tokens} tokens x all {H} heads of the T=65536 workload (fp64 C recurrence, "
+                      f"{used} threads, {dt:.2f} s wall)"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    steps, warmup = args.steps, args.warmup
+    tokens = 1024
+    for _ in range(warmup):
+        cpu_baseline(tokens)
+    t0 = time.perf_counter()
+    results = [cpu_baseline(tokens) for _ in range(steps)]
+    dt = time.perf_counter() - t0
+    value = steps * tokens / dt
+    cb = dict(results[-1])
+    cb["value"] = value
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": warmup, "ms_per_step": 1e3 * dt / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "heads": H, "seq_len": T_LONG, "batch": 1,
+                       "sample_tokens_per_step": tokens},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    world, rank, local = dist_setup()
+    import linear_attention_sequence_kda_b200 as kda
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    hbm_peak, bf16_peak, peak_src = peaks()
+
+    # ---------------- prefill: long-context workload, resident in HBM ----------
+    inp = ki.workload(2)
+    d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "g", "beta", "conv_w")}
+    cu_dev = torch.from_numpy(inp.cu_seqlens).to(dev)
+    o = torch.empty_like(d["q"])
+    S = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    tail = torch.empty((1, 3, 3, H * D), dtype=torch.bfloat16, device=dev)
+    ws_bytes = kda.workspace_size(1, T_LONG, H, T_LONG)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["conv_w"], inp.cu_seqlens, cu_dev,
+                    None, None, o=o, final_state=S, conv_tail=tail, workspace=ws, stream=stream)
+
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        total_ms, per_step = timed(step, args.steps, args.warmup, world, stream)
+    assert kda.check_async_status(stream) == 0
+    ms = total_ms / args.steps
+    tokens_per_rank = T_LONG
+    value = world * tokens_per_rank * args.steps / (total_ms / 1e3)
+    alg_bytes = T_LONG * H * BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+    launch_ms = statistics.mean(per_step)
+    achieved = alg_bytes / (launch_ms / 1e3) / 1e9
+    kernel_name = "kda_chunked_prefill"
+    traffic = recorded_traffic(kernel_name)
+
+    # ---------------- end to end: host buffers through the C ABI ----------------
+    pin = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    S_host = torch.empty(S.shape, dtype=S.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
+
+    def e2e_step():
+        for n, t in pin.items():
+            d[n].copy_(t, non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+        S_host.copy_(S, non_blocking=True)
+
+    e2e_ms, _ = timed(e2e_step, args.e2e_steps, 1, world, stream)
+    e2e_value = world * tokens_per_rank * args.e2e_steps / (e2e_ms / 1e3)
+    del pin, o_host, S_host
+
+    # ---------------- decode step: 256 sequences, state in place ----------------
+    dec = ki.workload(4)
+    dd = {n: getattr(dec, n).to(dev) for n in ("state", "conv_cache", "q", "k", "v", "g", "beta", "conv_w")}
+    o_dec = torch.empty_like(dd["q"])
+
+    def dstep():
+        kda.decode_step(dd["state"], dd["conv_cache"], dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
+                        dd["conv_w"], o=o_dec, stream=stream)
+
+    dec_total, dec_steps = timed(dstep, args.steps, args.warmup, world, stream)
+    npairs = dec.num_seqs * H
+    dec_ms = statistics.mean(dec_steps)
+    dec_state_gbs = npairs * 2 * STATE_BYTES / (dec_ms / 1e3) / 1e9
+    dec_alg_gbs = npairs * DEC_BYTES_PER_PAIR / (dec_ms / 1e3) / 1e9
+    dec_traffic = recorded_traffic("kda_decode")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "heads": H, "head_dim": D, "seq_len": T_LONG, "batch_per_gpu": 1,
+                   "chunk": 64, "parallelism": f"dp{world} (independent sequences per GPU)",
+                   "l2": "inputs larger than L2 (4.3 GB read per step), no flush"},
+        "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst)",
+                     "traffic": traffic, "algorithmic_bytes_per_launch": alg_bytes,
+                     "launch_ms": launch_ms},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": args.e2e_steps},
+        "gpu_launches": args.steps * PREFILL_LAUNCHES,
+        "clocks": clk.summary(),
+        "decode": {"workload": "kda_decode_step: 256 sequences x 1 token, 64 heads x 128, fp32 state in place",
+                   "state_gbs": dec_state_gbs, "ms_per_step": dec_ms,
+                   "roofline": {"kernel": "kda_decode", "bound": "hbm", "achieved": dec_alg_gbs,
+                                "peak": hbm_peak, "unit": "GB/s", "frac": dec_alg_gbs / hbm_peak,
+                                "state_frac": dec_state_gbs / hbm_peak, "traffic": dec_traffic,
+                                "algorithmic_bytes_per_launch": npairs * DEC_BYTES_PER_PAIR},
+                   "gpu_launches": args.steps * DECODE_LAUNCHES},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

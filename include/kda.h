@@ -1,0 +1,152 @@
+/*
+ * kda.h -- C ABI of libkda.so, the B200 (sm_100a) KDA sequence-mixing library.
+ *
+ * Operation (page "GLM-5.3-Flash im Detail", section "Sequenz-Mixing:
+ * 34 KDA-Schichten mit festem Zustand"; dimensions from "GLM-5.3-Flash
+ * Internals - a measured profile", section "Anatomy"): per head, q, k and v pass a
+ * causal depthwise convolution of width 4; q and k are L2-normalised; a
+ * channel-wise forget gate alpha_t = exp(max(g_t, -5)) decays the state; a
+ * scalar beta_t drives a delta-rule write; the query reads the updated state:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t                    (S_t: 128 x 128 fp32 per head)
+ *
+ * Prefill evaluates many tokens per call (chunk-parallel inside, state handed
+ * from chunk to chunk); decode applies one recurrent update per sequence.  The
+ * same section states that prefill and decode use different kernel shapes, and
+ * "GLM-5.3-Flash im Detail", section "FP8-Checkpoint und Betriebsgrenzen", that
+ * disaggregated prefill and decode share identical KDA layouts: the final state
+ * and conv tail written by kda_prefill are exactly the state and conv cache that
+ * kda_decode_step consumes.
+ *
+ * Conventions for every entry point:
+ *  - All pointers are caller-owned.  Tensor pointers are DEVICE pointers unless
+ *    a parameter name ends in _host.  The library never allocates or frees.
+ *  - Head dims are fixed at d_k = d_v = 128 (KDA_HEAD_DIM).
+ *  - Per-token tensors are packed token-major, channel contiguous:
+ *      q, k, v, g, o : [total_T, H, 128]   beta : [total_T, H]
+ *    element type per `dt` (fp32 or bf16).  conv_w is always fp32:
+ *      conv_w : [3, H*128, 4]  (q, k, v taps; tap 3 multiplies the current
+ *               token, tap 0 the token three steps back; no bias)
+ *  - States are fp32 [N, H, 128, 128], row = key channel, column = value
+ *    channel (value index contiguous).  Conv history / tail / cache is
+ *    [N, 3 (q,k,v), 3 (time, oldest first), H*128] in the input dtype.
+ *  - L2 norm: x / sqrt(sum x^2 + 1e-6).  No query scale.  Conv activation:
+ *    KDA_CONV_NONE (default) or KDA_CONV_SILU (y * sigmoid(y)).
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).  Argument errors are detected on the host before
+ *    anything is launched and returned as a status; nothing aborts.
+ *  - Alignment: q, k, v, g, o, states, conv tensors and workspace must be
+ *    16-byte aligned; beta aligned to its element size.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_HEAD_DIM 128
+#define KDA_CHUNK 64
+#define KDA_CONV_WIDTH 4
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad cu_seqlens, bad enum   */
+  KDA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement         */
+  KDA_ERR_ALIGNMENT = 3,    /* a pointer violates the alignment rule above         */
+  KDA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required          */
+  KDA_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute, ...) */
+  KDA_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up (async status)   */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+typedef enum { KDA_CONV_NONE = 0, KDA_CONV_SILU = 1 } kda_conv_act;
+
+/* Bytes of device workspace kda_prefill needs for this problem (0 if none).
+ * Pure host function; never fails (returns 0 for invalid sizes). */
+size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_heads,
+                                  int max_seqlen, kda_dtype dt);
+
+/*
+ * kda_prefill -- one KDA mixing step over N packed segments (varlen prefill).
+ *   q, k, v, g, beta : inputs as laid out above; segment n is rows
+ *                      [cu_seqlens[n], cu_seqlens[n+1]).  May be NULL only when
+ *                      total_T == 0.
+ *   conv_w           : [3, H*128, 4] fp32 conv taps.
+ *   init_state       : [N, H, 128, 128] fp32, or NULL for zero states.
+ *   init_conv        : [N, 3, 3, H*128] raw q/k/v of the 3 tokens before each
+ *                      segment (oldest first), or NULL for zeros.
+ *   cu_seqlens_dev   : [N+1] int32 device copy of the segment offsets.
+ *   cu_seqlens_host  : [N+1] int32 host copy (used for scheduling; must equal
+ *                      the device copy).  cu[0] == 0, non-decreasing.
+ *   o                : out [total_T, H, 128] (dt).  Must not alias inputs.
+ *   final_state      : out [N, H, 128, 128] fp32; may equal init_state (in place).
+ *   conv_tail        : out [N, 3, 3, H*128] (dt): last 3 raw tokens of
+ *                      concat(init_conv, segment); may equal init_conv.
+ *   workspace        : device scratch of kda_prefill_workspace_size() bytes
+ *                      (may be NULL when that size is 0).
+ * Returns KDA_OK once all work is enqueued.  bf16 inputs run the chunked
+ * tensor-core path; fp32 inputs run the fp32 recurrent path.
+ */
+kda_status kda_prefill(const void* q, const void* k, const void* v, const void* g,
+                       const void* beta, const float* conv_w, const float* init_state,
+                       const void* init_conv, const int32_t* cu_seqlens_dev,
+                       const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                       kda_dtype dt, kda_conv_act act, void* o, float* final_state,
+                       void* conv_tail, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
+ * kda_prefill_recurrent -- same contract as kda_prefill, always evaluated by
+ * the token-by-token fp32 kernel (one thread block per (segment, head), the
+ * state held in registers).  Exact to fp32 rounding for any dtype; slower.
+ * Needs no workspace (pass NULL, 0).
+ */
+kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, const void* g,
+                                 const void* beta, const float* conv_w,
+                                 const float* init_state, const void* init_conv,
+                                 const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                                 int num_seqs, int num_heads, kda_dtype dt, kda_conv_act act,
+                                 void* o, float* final_state, void* conv_tail, void* stream);
+
+/*
+ * kda_decode_step -- one recurrent update per sequence (page "GLM-5.3-Flash im
+ * Detail", section "Sequenz-Mixing: ...": decode of a single token performs a
+ * recurrent update), in place.
+ *   state      : [N, H, 128, 128] fp32, read and overwritten with S_t.
+ *   conv_cache : [N, 3, 3, H*128] (dt), read (3 previous raw tokens) and
+ *                shifted in place so that it ends with this step's raw token.
+ *   q, k, v, g : [N, H, 128] raw inputs of the new token (dt); beta : [N, H].
+ *   conv_w     : [3, H*128, 4] fp32.
+ *   o          : out [N, H, 128] (dt).
+ * Each (sequence, head) state is streamed through registers exactly once.
+ */
+kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const void* k,
+                           const void* v, const void* g, const void* beta,
+                           const float* conv_w, int num_seqs, int num_heads, kda_dtype dt,
+                           kda_conv_act act, void* o, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* kda_status_string(kda_status s);
+
+/*
+ * Synchronises `stream`, then returns and clears the library's device status
+ * word on the current device: KDA_OK, or KDA_ERR_TIMEOUT if a bounded
+ * device-side wait gave up since the last call (the kernel that gave up
+ * stopped early, so its outputs are invalid), or KDA_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+kda_status kda_check_async_status(void* stream);
+
+/* Library ABI version: (major << 16) | minor. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -54,20 +54,25 @@ def _threads() -> int:
     return max(1, min(32, os.cpu_count() or 1))
 
 
-def _draw(shape, seed: int, stream: int, kind: str) -> torch.Tensor:
-    """float32 tensor of N(0,1) ('n') or U[0,1) ('u') draws, generated in fixed
-    blocks with their own seeds so the result does not depend on thread count."""
+def _draw(shape, seed: int, stream: int, kind: str, dtype: torch.dtype = torch.float32,
+          scale: float = 1.0, fn=None) -> torch.Tensor:
+    """Tensor of N(0,1) ('n') or U[0,1) ('u') draws, optionally mapped by
+    fn(x, first_index), then scaled; generated in fp32 blocks with their own
+    seeds (the result does not depend on the thread count) and stored as
+    `dtype` (round-to-nearest-even for bf16) block by block."""
     n = int(np.prod(shape)) if len(shape) else 1
-    out = torch.empty(n, dtype=torch.float32)
+    out = torch.empty(n, dtype=dtype)
     nblocks = (n + _BLOCK - 1) // _BLOCK
 
     def fill(b: int) -> None:
         gen = torch.Generator().manual_seed(_mix(seed, stream, b))
         lo, hi = b * _BLOCK, min(n, (b + 1) * _BLOCK)
-        if kind == "n":
-            out[lo:hi] = torch.randn(hi - lo, generator=gen)
-        else:
-            out[lo:hi] = torch.rand(hi - lo, generator=gen)
+        x = torch.randn(hi - lo, generator=gen) if kind == "n" else torch.rand(hi - lo, generator=gen)
+        if fn is not None:
+            x = fn(x, lo)
+        if scale != 1.0:
+            x = x * scale
+        out[lo:hi] = x
 
     if nblocks <= 1:
         for b in range(nblocks):
@@ -78,19 +83,21 @@ def _draw(shape, seed: int, stream: int, kind: str) -> torch.Tensor:
     return out.view(*shape)
 
 
-def randn(shape, seed: int, stream: int, std: float = 1.0) -> torch.Tensor:
-    x = _draw(shape, seed, stream, "n")
-    if std != 1.0:
-        x.mul_(std)
-    return x
+def randn(shape, seed: int, stream: int, std: float = 1.0,
+          dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    return _draw(shape, seed, stream, "n", dtype, std)
 
 
 def rand(shape, seed: int, stream: int) -> torch.Tensor:
     return _draw(shape, seed, stream, "u")
 
 
-def _cast(x: torch.Tensor, dtype: torch.dtype) -> torch.Tensor:
-    return x if dtype == torch.float32 else x.to(dtype)
+def _sigmoid(x: torch.Tensor, lo: int) -> torch.Tensor:
+    return torch.sigmoid(x)
+
+
+def _neg5_sigmoid(x: torch.Tensor, lo: int) -> torch.Tensor:
+    return torch.sigmoid(x).mul_(-5.0)
 
 
 @dataclasses.dataclass
@@ -148,21 +155,27 @@ class DecodeInputs:
         return self.q.dtype
 
 
-def gate_sigmoid(shape, seed: int) -> torch.Tensor:
-    """g = -5 * sigmoid(N(0,1)), fp32."""
-    return torch.sigmoid(randn(shape, seed, _G)).mul_(-5.0)
+def gate_sigmoid(shape, seed: int, dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    """g = -5 * sigmoid(N(0,1))."""
+    return _draw(shape, seed, _G, "n", dtype, fn=_neg5_sigmoid)
 
 
-def gate_bimodal(total_t: int, H: int, D: int, seed: int, frac: float = 0.1) -> torch.Tensor:
+def gate_bimodal(total_t: int, H: int, D: int, seed: int, frac: float = 0.1,
+                 dtype: torch.dtype = torch.float32) -> torch.Tensor:
     """Long-context gate mix: a seeded `frac` of (head, key channel) pairs get
     g = -5 + 0.1 U(0,1) for every token, the rest g = -0.05 U(0,1)."""
     rng = np.random.default_rng(_mix(seed, _GSEL, 0))
-    nsel = int(round(frac * H * D))
-    sel = np.zeros(H * D, dtype=bool)
-    sel[rng.permutation(H * D)[:nsel]] = True
-    u = rand((total_t, H, D), seed, _GU)
-    sel_t = torch.from_numpy(sel.reshape(1, H, D))
-    return torch.where(sel_t, -5.0 + 0.1 * u, -0.05 * u)
+    HD = H * D
+    nsel = int(round(frac * HD))
+    sel = np.zeros(HD, dtype=bool)
+    sel[rng.permutation(HD)[:nsel]] = True
+    sel_t = torch.from_numpy(sel)
+
+    def mix(u: torch.Tensor, lo: int) -> torch.Tensor:
+        chan = (torch.arange(lo, lo + u.numel(), dtype=torch.int64) % HD)
+        return torch.where(sel_t[chan], -5.0 + 0.1 * u, -0.05 * u)
+
+    return _draw((total_t, H, D), seed, _GU, "u", dtype, fn=mix)
 
 
 def make_prefill(seqlens: Sequence[int], H: int, dtype: torch.dtype, seed: int, *,
@@ -173,32 +186,31 @@ def make_prefill(seqlens: Sequence[int], H: int, dtype: torch.dtype, seed: int, 
     cu = np.zeros(N + 1, dtype=np.int32)
     cu[1:] = np.cumsum(seqlens)
     T = int(cu[-1])
-    q = _cast(randn((T, H, D), seed, _Q), dtype)
-    k = _cast(randn((T, H, D), seed, _K), dtype)
-    v = _cast(randn((T, H, D), seed, _V), dtype)
+    q = randn((T, H, D), seed, _Q, dtype=dtype)
+    k = randn((T, H, D), seed, _K, dtype=dtype)
+    v = randn((T, H, D), seed, _V, dtype=dtype)
     if gate == "sigmoid":
-        g = gate_sigmoid((T, H, D), seed)
+        g = gate_sigmoid((T, H, D), seed, dtype)
     elif gate == "bimodal":
-        g = gate_bimodal(T, H, D, seed)
+        g = gate_bimodal(T, H, D, seed, dtype=dtype)
     else:
         raise ValueError(gate)
-    g = _cast(g, dtype)
-    beta = _cast(torch.sigmoid(randn((T, H), seed, _BETA)), dtype)
+    beta = _draw((T, H), seed, _BETA, "n", dtype, fn=_sigmoid)
     conv_w = randn((3, H * D, 4), seed, _CONVW, std=0.5)
     init_state = randn((N, H, D, D), seed, _STATE, std=state_std) if state_std else None
-    init_conv = _cast(randn((N, 3, 3, H * D), seed, _CONV), dtype) if conv_history else None
+    init_conv = randn((N, 3, 3, H * D), seed, _CONV, dtype=dtype) if conv_history else None
     return PrefillInputs(q, k, v, g, beta, conv_w, init_state, init_conv, cu, name)
 
 
 def make_decode(N: int, H: int, dtype: torch.dtype, seed: int, *, D: int = D_HEAD,
                 state_std: float = 0.02, name: str = "") -> DecodeInputs:
     state = randn((N, H, D, D), seed, _STATE, std=state_std)
-    conv_cache = _cast(randn((N, 3, 3, H * D), seed, _CONV), dtype)
-    q = _cast(randn((N, H, D), seed, _Q), dtype)
-    k = _cast(randn((N, H, D), seed, _K), dtype)
-    v = _cast(randn((N, H, D), seed, _V), dtype)
-    g = _cast(gate_sigmoid((N, H, D), seed), dtype)
-    beta = _cast(torch.sigmoid(randn((N, H), seed, _BETA)), dtype)
+    conv_cache = randn((N, 3, 3, H * D), seed, _CONV, dtype=dtype)
+    q = randn((N, H, D), seed, _Q, dtype=dtype)
+    k = randn((N, H, D), seed, _K, dtype=dtype)
+    v = randn((N, H, D), seed, _V, dtype=dtype)
+    g = gate_sigmoid((N, H, D), seed, dtype)
+    beta = _draw((N, H), seed, _BETA, "n", dtype, fn=_sigmoid)
     conv_w = randn((3, H * D, 4), seed, _CONVW, std=0.5)
     return DecodeInputs(state, conv_cache, q, k, v, g, beta, conv_w, name)
 

@@ -1,0 +1,140 @@
+"""Python binding of libkda.so (the B200 KDA sequence-mixing library).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI of ``include/kda.h``.  PyTorch is used for device
+memory, streams and dtype plumbing.  If ``libkda.so`` has not been built the
+import fails loudly; there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkda.so")
+HEAD_DIM = 128
+CHUNK = 64
+
+KDA_F32, KDA_BF16 = 0, 1
+KDA_CONV_NONE, KDA_CONV_SILU = 0, 1
+STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "KDA_ERR_ALIGNMENT",
+          4: "KDA_ERR_WORKSPACE", 5: "KDA_ERR_CUDA", 6: "KDA_ERR_TIMEOUT"}
+
+# every entry point declared in include/kda.h
+EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
+           "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m "
+                      "linear_attention_sequence_kda_b200.build` (nvcc, sm_100a)")
+
+_vp, _i32p, _f32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+lib = ctypes.CDLL(LIB_PATH)
+lib.kda_prefill_workspace_size.restype = ctypes.c_size_t
+lib.kda_prefill_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_int]
+_PREFILL_ARGS = [_vp, _vp, _vp, _vp, _vp, _f32p, _f32p, _vp, _i32p, _i32p, ctypes.c_int, ctypes.c_int,
+                 ctypes.c_int, ctypes.c_int, _vp, _f32p, _vp]
+lib.kda_prefill.restype = ctypes.c_int
+lib.kda_prefill.argtypes = _PREFILL_ARGS + [_vp, ctypes.c_size_t, _vp]
+lib.kda_prefill_recurrent.restype = ctypes.c_int
+lib.kda_prefill_recurrent.argtypes = _PREFILL_ARGS + [_vp]
+lib.kda_decode_step.restype = ctypes.c_int
+lib.kda_decode_step.argtypes = [_f32p, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
+                                ctypes.c_int, ctypes.c_int, _vp, _vp]
+lib.kda_status_string.restype = ctypes.c_char_p
+lib.kda_status_string.argtypes = [ctypes.c_int]
+lib.kda_check_async_status.restype = ctypes.c_int
+lib.kda_check_async_status.argtypes = [_vp]
+lib.kda_version.restype = ctypes.c_int
+
+
+class KdaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({lib.kda_status_string(code).decode()})")
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise KdaError(code, where)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KDA_F32
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def workspace_size(num_seqs: int, total_tokens: int, num_heads: int, max_seqlen: int,
+                   dtype: torch.dtype = torch.bfloat16) -> int:
+    return int(lib.kda_prefill_workspace_size(num_seqs, total_tokens, num_heads, max_seqlen,
+                                              KDA_F32 if dtype == torch.float32 else KDA_BF16))
+
+
+def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init_state=None,
+            init_conv=None, act: int = KDA_CONV_NONE, o=None, final_state=None, conv_tail=None,
+            workspace=None, stream=None, recurrent: bool = False):
+    """kda_prefill (or kda_prefill_recurrent) on device tensors.  Returns
+    (o, final_state, conv_tail); outputs are allocated when not given."""
+    cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
+    N = len(cu_h) - 1
+    T, H = q.shape[0], q.shape[1]
+    dev = q.device
+    if cu_seqlens_dev is None:
+        cu_seqlens_dev = torch.from_numpy(cu_h).to(dev)
+    if o is None:
+        o = torch.empty_like(q)
+    if final_state is None:
+        final_state = torch.empty((N, H, HEAD_DIM, HEAD_DIM), dtype=torch.float32, device=dev)
+    if conv_tail is None:
+        conv_tail = torch.empty((N, 3, 3, H * HEAD_DIM), dtype=q.dtype, device=dev)
+    dt = _dtype_code(q)
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(conv_w), _ptr(init_state),
+            _ptr(init_conv), _ptr(cu_seqlens_dev), _ptr(cu_h), N, H, dt, int(act), _ptr(o),
+            _ptr(final_state), _ptr(conv_tail)]
+    if recurrent:
+        _check(lib.kda_prefill_recurrent(*args, _stream(stream)), "kda_prefill_recurrent")
+    else:
+        need = workspace_size(N, int(cu_h[-1]), H, int(np.diff(cu_h).max()) if N else 0, q.dtype)
+        if workspace is None and need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        _check(lib.kda_prefill(*args, _ptr(workspace), wbytes, _stream(stream)), "kda_prefill")
+    return o, final_state, conv_tail
+
+
+def decode_step(state, conv_cache, q, k, v, g, beta, conv_w, act: int = KDA_CONV_NONE, o=None,
+                stream=None):
+    """kda_decode_step in place on `state` and `conv_cache`; returns o."""
+    N, H = q.shape[0], q.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    _check(lib.kda_decode_step(_ptr(state), _ptr(conv_cache), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                               _ptr(beta), _ptr(conv_w), N, H, _dtype_code(q), int(act), _ptr(o),
+                               _stream(stream)), "kda_decode_step")
+    return o
+
+
+def check_async_status(stream=None) -> int:
+    return int(lib.kda_check_async_status(_stream(stream)))

@@ -1,0 +1,203 @@
+// libkda.so: the C ABI declared in include/kda.h.  Host-side argument
+// validation, then asynchronous launches on the caller's stream.
+#include <stdio.h>
+
+#include "kda_common.cuh"
+#include "kda_decode.cuh"
+#include "kda_recurrent.cuh"
+#include "kda_tail.cuh"
+#include "kda_chunked.cuh"
+
+using namespace kda;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t esize(kda_dtype dt) { return dt == KDA_F32 ? 4 : 2; }
+
+struct PrefillArgs {
+  const void *q, *k, *v, *g, *beta;
+  const float* conv_w;
+  const float* init_state;
+  const void* init_conv;
+  const int32_t *cu_dev, *cu_host;
+  int N, H;
+  kda_dtype dt;
+  kda_conv_act act;
+  void* o;
+  float* final_state;
+  void* conv_tail;
+  cudaStream_t stream;
+  int64_t total_T;
+  int max_len;
+};
+
+kda_status validate_prefill(PrefillArgs& a) {
+  if (a.N < 0 || a.H < 1) return KDA_ERR_INVALID_ARG;
+  if (a.dt != KDA_F32 && a.dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (a.act != KDA_CONV_NONE && a.act != KDA_CONV_SILU) return KDA_ERR_INVALID_ARG;
+  if (a.N == 0) { a.total_T = 0; a.max_len = 0; return KDA_OK; }
+  if (!a.cu_host || !a.cu_dev) return KDA_ERR_INVALID_ARG;
+  if (a.cu_host[0] != 0) return KDA_ERR_INVALID_ARG;
+  int max_len = 0;
+  for (int n = 0; n < a.N; ++n) {
+    const int64_t len = (int64_t)a.cu_host[n + 1] - a.cu_host[n];
+    if (len < 0) return KDA_ERR_INVALID_ARG;
+    if (len > max_len) max_len = (int)len;
+  }
+  a.total_T = a.cu_host[a.N];
+  a.max_len = max_len;
+  if (a.N > 65535) return KDA_ERR_UNSUPPORTED;
+  if (!a.final_state || !a.conv_tail || !a.conv_w) return KDA_ERR_INVALID_ARG;
+  if (a.total_T > 0 && (!a.q || !a.k || !a.v || !a.g || !a.beta || !a.o)) return KDA_ERR_INVALID_ARG;
+  const void* al16[] = {a.q, a.k, a.v, a.g, a.o, a.conv_w, a.init_state, a.final_state,
+                        a.init_conv, a.conv_tail};
+  for (const void* p : al16)
+    if (p && !aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+  if (a.beta && !aligned(a.beta, esize(a.dt))) return KDA_ERR_ALIGNMENT;
+  if (a.total_T > 0 && (a.o == a.q || a.o == a.k || a.o == a.v || a.o == a.g))
+    return KDA_ERR_INVALID_ARG;
+  return KDA_OK;
+}
+
+template <typename Tin>
+kda_status launch_tail(const PrefillArgs& a) {
+  const int64_t total = (int64_t)a.N * 3 * a.H * D;
+  if (total == 0) return KDA_OK;
+  const int64_t want = (total + 255) / 256;
+  const int64_t blocks = want < 148 * 16 ? want : 148 * 16;
+  conv_tail_kernel<Tin><<<(unsigned)blocks, 256, 0, a.stream>>>(
+      (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.init_conv, a.cu_dev, a.N,
+      a.H, (Tin*)a.conv_tail);
+  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+template <typename Tin>
+kda_status launch_recurrent(const PrefillArgs& a) {
+  dim3 grid(a.H, a.N);
+  if (a.act == KDA_CONV_SILU)
+    recurrent_prefill_kernel<Tin, KDA_CONV_SILU><<<grid, 128, 0, a.stream>>>(
+        (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.g, (const Tin*)a.beta,
+        a.conv_w, a.init_state, (const Tin*)a.init_conv, a.cu_dev, a.H, (Tin*)a.o, a.final_state);
+  else
+    recurrent_prefill_kernel<Tin, KDA_CONV_NONE><<<grid, 128, 0, a.stream>>>(
+        (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.g, (const Tin*)a.beta,
+        a.conv_w, a.init_state, (const Tin*)a.init_conv, a.cu_dev, a.H, (Tin*)a.o, a.final_state);
+  if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+  return launch_tail<Tin>(a);
+}
+
+kda_status run_recurrent(PrefillArgs& a) {
+  if (a.N == 0) return KDA_OK;
+  return a.dt == KDA_F32 ? launch_recurrent<float>(a) : launch_recurrent<__nv_bfloat16>(a);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_heads,
+                                  int max_seqlen, kda_dtype dt) {
+  if (num_seqs < 0 || total_tokens < 0 || num_heads < 1 || max_seqlen < 0) return 0;
+  if (dt != KDA_BF16) return 0;
+  return chunked_workspace_bytes(num_seqs, num_heads);
+}
+
+kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, const void* g,
+                                 const void* beta, const float* conv_w,
+                                 const float* init_state, const void* init_conv,
+                                 const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
+                                 int num_seqs, int num_heads, kda_dtype dt, kda_conv_act act,
+                                 void* o, float* final_state, void* conv_tail, void* stream) {
+  PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o, final_state, conv_tail,
+                (cudaStream_t)stream, 0, 0};
+  kda_status st = validate_prefill(a);
+  if (st != KDA_OK) return st;
+  return run_recurrent(a);
+}
+
+kda_status kda_prefill(const void* q, const void* k, const void* v, const void* g,
+                       const void* beta, const float* conv_w, const float* init_state,
+                       const void* init_conv, const int32_t* cu_seqlens_dev,
+                       const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                       kda_dtype dt, kda_conv_act act, void* o, float* final_state,
+                       void* conv_tail, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o, final_state, conv_tail,
+                (cudaStream_t)stream, 0, 0};
+  kda_status st = validate_prefill(a);
+  if (st != KDA_OK) return st;
+  if (a.N == 0) return KDA_OK;
+  if (dt == KDA_F32) return run_recurrent(a);
+  const size_t need = chunked_workspace_bytes(a.N, a.H);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 16)) return KDA_ERR_ALIGNMENT;
+  st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
+                      a.cu_host, a.N, a.H, a.act, a.o, a.final_state, workspace, a.stream);
+  if (st != KDA_OK) return st;
+  return launch_tail<__nv_bfloat16>(a);
+}
+
+kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const void* k,
+                           const void* v, const void* g, const void* beta,
+                           const float* conv_w, int num_seqs, int num_heads, kda_dtype dt,
+                           kda_conv_act act, void* o, void* stream) {
+  if (num_seqs < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (act != KDA_CONV_NONE && act != KDA_CONV_SILU) return KDA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KDA_OK;
+  if (num_seqs > 65535) return KDA_ERR_UNSUPPORTED;
+  if (!state || !conv_cache || !q || !k || !v || !g || !beta || !conv_w || !o)
+    return KDA_ERR_INVALID_ARG;
+  const void* al16[] = {state, conv_cache, q, k, v, g, conv_w, o};
+  for (const void* p : al16)
+    if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+  if (!aligned(beta, esize(dt))) return KDA_ERR_ALIGNMENT;
+  if (o == q || o == k || o == v || o == g) return KDA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  dim3 grid(num_heads, num_seqs);
+#define KDA_DECODE_LAUNCH(T, A)                                                               \
+  decode_kernel<T, A><<<grid, 256, 0, s>>>(state, (T*)conv_cache, (const T*)q, (const T*)k,   \
+                                           (const T*)v, (const T*)g, (const T*)beta, conv_w, \
+                                           num_heads, (T*)o)
+  if (dt == KDA_F32) {
+    if (act == KDA_CONV_SILU) KDA_DECODE_LAUNCH(float, KDA_CONV_SILU);
+    else KDA_DECODE_LAUNCH(float, KDA_CONV_NONE);
+  } else {
+    if (act == KDA_CONV_SILU) KDA_DECODE_LAUNCH(__nv_bfloat16, KDA_CONV_SILU);
+    else KDA_DECODE_LAUNCH(__nv_bfloat16, KDA_CONV_NONE);
+  }
+#undef KDA_DECODE_LAUNCH
+  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+const char* kda_status_string(kda_status s) {
+  switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_INVALID_ARG: return "invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "unsupported request";
+    case KDA_ERR_ALIGNMENT: return "misaligned pointer";
+    case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+    case KDA_ERR_CUDA: return "CUDA runtime error";
+    case KDA_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+kda_status kda_check_async_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KDA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  return (kda_status)v;
+}
+
+int kda_version(void) { return (1 << 16) | 0; }
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Shared device helpers for the KDA kernels (sm_100a).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+constexpr int D = KDA_HEAD_DIM;   // d_k = d_v = 128
+constexpr float LOG_DECAY_FLOOR = -5.0f;
+constexpr float NORM_EPS = 1e-6f;
+
+// Device status word (one per device per process): kernels that give up on a
+// bounded wait write a nonzero kda_status here; kda_check_async_status reads it.
+__device__ int g_status;
+
+__device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// ---- element loads/stores in either dtype, converted to/from fp32 ----------
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// 4 consecutive elements -> float4 (pointer 8/16-byte aligned).
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  uint2 u = *reinterpret_cast<const uint2*>(p);
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x);
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+  float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+__device__ __forceinline__ float silu(float y) { return y / (1.0f + __expf(-y)); }
+
+// Causal width-4 conv tap sum: w.x = w0*x_{t-3} + w1*x_{t-2} + w2*x_{t-1} + w3*x_t
+__device__ __forceinline__ float conv4(float4 w, float xm3, float xm2, float xm1, float x0) {
+  return fmaf(w.w, x0, fmaf(w.z, xm1, fmaf(w.y, xm2, w.x * xm3)));
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Streaming (evict-first) 16-byte global load/store for data touched once.
+__device__ __forceinline__ float4 ld_stream(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ void st_stream(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
+
+}  // namespace kda

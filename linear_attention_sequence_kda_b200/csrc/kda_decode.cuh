@@ -1,0 +1,126 @@
+// Single-token KDA decode, in place, bound by streaming the fp32 states.
+//
+// Page "GLM-5.3-Flash im Detail", section "Sequenz-Mixing: 34 KDA-Schichten mit
+// festem Zustand": decoding one token is one recurrent update of the per-head
+// state.  Per (sequence, head), with S the 128 x 128 state (row = key channel):
+//     y = conv4(cache, x) for q, k, v;  q, k L2-normalised;  a = exp(max(g,-5))
+//     r = S^T (a * k),  u = beta (v - r),  o = S^T (a * q) + u (k . q)
+//     S <- Diag(a) S + k u^T,  cache <- shift(cache, x)
+// so S is read once and written once (single pass).
+//
+// Block = 256 threads = 8 warps per (sequence, head).  Warp w owns rows
+// [16w, 16w+16); lane l owns columns [4l, 4l+4): 16 float4 registers per
+// thread.  The 64 KiB state is loaded with streaming 16-byte loads issued
+// before the prologue so the loads overlap it; reductions over rows are
+// finished through shared memory; the updated rows are written with
+// streaming stores.
+#pragma once
+#include "kda_common.cuh"
+
+namespace kda {
+
+template <typename Tin, int ACT>
+__global__ void __launch_bounds__(256, 2)
+decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
+              const Tin* __restrict__ k, const Tin* __restrict__ v, const Tin* __restrict__ g,
+              const Tin* __restrict__ beta, const float* __restrict__ conv_w, int H,
+              Tin* __restrict__ o) {
+  __shared__ __align__(16) float sh_kh[D], sh_ka[D], sh_qa[D], sh_al[D], sh_v[D], sh_u[D];
+  __shared__ __align__(16) float sh_r[8][D], sh_y[8][D];
+  __shared__ float sh_red[4][3];
+
+  const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int64_t HD = (int64_t)H * D;
+  float* S = state + ((int64_t)n * H + h) * D * D;
+
+  // 1. issue the state loads first
+  float4 s[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) s[i] = ld_stream(S + (warp * 16 + i) * D + lane * 4);
+
+  // 2. prologue: threads 0..127 -> q and k of channel c; 128..255 -> v and g
+  const int c = tid & (D - 1);
+  const int64_t ch = (int64_t)h * D + c;
+  const int64_t tok = (int64_t)n * HD + ch;   // [N, H, D] index
+  Tin* cb = cache + (int64_t)n * 9 * HD + ch; // [3 x][3 t] stride HD
+  float yq = 0.f, yk = 0.f;
+  if (tid < D) {
+    const float4 wq = load4(conv_w + (0 * HD + ch) * 4);
+    const float4 wk = load4(conv_w + (1 * HD + ch) * 4);
+    const float q0 = to_f(cb[0 * HD]), q1 = to_f(cb[1 * HD]), q2 = to_f(cb[2 * HD]);
+    const float k0 = to_f(cb[3 * HD]), k1 = to_f(cb[4 * HD]), k2 = to_f(cb[5 * HD]);
+    const Tin xq = q[tok], xk = k[tok];
+    yq = conv4(wq, q0, q1, q2, to_f(xq));
+    yk = conv4(wk, k0, k1, k2, to_f(xk));
+    if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
+    // shift the cache (all reads of this channel's history are done above)
+    cb[0 * HD] = cb[1 * HD]; cb[1 * HD] = cb[2 * HD]; cb[2 * HD] = xq;
+    cb[3 * HD] = cb[4 * HD]; cb[4 * HD] = cb[5 * HD]; cb[5 * HD] = xk;
+    float nq = warp_sum(yq * yq), nk = warp_sum(yk * yk), qk = warp_sum(yq * yk);
+    if (lane == 0) { sh_red[warp][0] = nq; sh_red[warp][1] = nk; sh_red[warp][2] = qk; }
+  } else {
+    const float4 wv = load4(conv_w + (2 * HD + ch) * 4);
+    const float v0 = to_f(cb[6 * HD]), v1 = to_f(cb[7 * HD]), v2 = to_f(cb[8 * HD]);
+    const Tin xv = v[tok];
+    float yv = conv4(wv, v0, v1, v2, to_f(xv));
+    if (ACT == KDA_CONV_SILU) yv = silu(yv);
+    cb[6 * HD] = cb[7 * HD]; cb[7 * HD] = cb[8 * HD]; cb[8 * HD] = xv;
+    sh_v[c] = yv;
+    sh_al[c] = __expf(fmaxf(to_f(g[tok]), LOG_DECAY_FLOOR));
+  }
+  __syncthreads();
+  const float nq = sh_red[0][0] + sh_red[1][0] + sh_red[2][0] + sh_red[3][0];
+  const float nk = sh_red[0][1] + sh_red[1][1] + sh_red[2][1] + sh_red[3][1];
+  const float qk = sh_red[0][2] + sh_red[1][2] + sh_red[2][2] + sh_red[3][2];
+  const float rq = rsqrtf(nq + NORM_EPS), rk = rsqrtf(nk + NORM_EPS);
+  const float kq = qk * rq * rk;
+  if (tid < D) {
+    const float a = sh_al[c];
+    const float kh = yk * rk;
+    sh_kh[c] = kh;
+    sh_ka[c] = a * kh;
+    sh_qa[c] = a * yq * rq;
+  }
+  __syncthreads();
+
+  // 3. partial reductions over this warp's 16 rows, 4 columns per lane
+  float4 r = make_float4(0.f, 0.f, 0.f, 0.f), y = r;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float ka = sh_ka[warp * 16 + i], qa = sh_qa[warp * 16 + i];
+    r.x = fmaf(s[i].x, ka, r.x); r.y = fmaf(s[i].y, ka, r.y);
+    r.z = fmaf(s[i].z, ka, r.z); r.w = fmaf(s[i].w, ka, r.w);
+    y.x = fmaf(s[i].x, qa, y.x); y.y = fmaf(s[i].y, qa, y.y);
+    y.z = fmaf(s[i].z, qa, y.z); y.w = fmaf(s[i].w, qa, y.w);
+  }
+  *reinterpret_cast<float4*>(&sh_r[warp][lane * 4]) = r;
+  *reinterpret_cast<float4*>(&sh_y[warp][lane * 4]) = y;
+  __syncthreads();
+  if (tid < D) {
+    float rr = 0.f, yy = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) { rr += sh_r[w][tid]; yy += sh_y[w][tid]; }
+    const float b = to_f(beta[(int64_t)n * H + h]);
+    const float u = b * (sh_v[tid] - rr);
+    sh_u[tid] = u;
+    o[tok] = from_f<Tin>(yy + u * kq);
+  }
+  __syncthreads();
+
+  // 4. S <- Diag(a) S + k u^T, written once
+  const float4 u4 = *reinterpret_cast<const float4*>(&sh_u[lane * 4]);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int row = warp * 16 + i;
+    const float a = sh_al[row], kh = sh_kh[row];
+    float4 t;
+    t.x = fmaf(a, s[i].x, kh * u4.x);
+    t.y = fmaf(a, s[i].y, kh * u4.y);
+    t.z = fmaf(a, s[i].z, kh * u4.z);
+    t.w = fmaf(a, s[i].w, kh * u4.w);
+    st_stream(S + row * D + lane * 4, t);
+  }
+}
+
+}  // namespace kda

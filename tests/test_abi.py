@@ -1,0 +1,98 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/kda.h declares, and rejects bad arguments on the host before any launch
+(fake device addresses are never dereferenced on these paths)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import linear_attention_sequence_kda_b200 as kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+# distinct, 16-byte aligned fake device addresses
+Q, K, V, G, B, W, O, FS, CT, CU, WS = [(i + 1) << 20 for i in range(11)]
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", txt)))
+
+
+def test_header_declarations_are_exported():
+    names = _declared()
+    assert set(names) == set(kda.EXPORTS), names
+    out = subprocess.run(["nm", "-D", "--defined-only", kda.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for n in names:
+        assert n in exported, n
+        assert hasattr(kda.lib, n)
+
+
+def test_version_and_status_strings():
+    assert kda.lib.kda_version() >> 16 == 1
+    for code in range(7):
+        s = kda.lib.kda_status_string(code)
+        assert s and s.decode()
+    assert kda.lib.kda_status_string(99).decode() == "unknown status"
+
+
+def test_workspace_size_invalid_is_zero():
+    assert kda.lib.kda_prefill_workspace_size(-1, 10, 4, 10, 1) == 0
+    assert kda.lib.kda_prefill_workspace_size(1, 10, 0, 10, 1) == 0
+    assert kda.lib.kda_prefill_workspace_size(1, 10, 4, 10, 0) == 0  # fp32 path needs none
+
+
+def _prefill(cu, H=4, dt=1, act=0, q=Q, o=O, final=FS, tail=CT, ws=WS, wsb=1 << 40, beta=B,
+             recurrent=False):
+    cu = np.ascontiguousarray(np.asarray(cu, dtype=np.int32))
+    args = [q, K, V, G, beta, W, None, None, CU, cu.ctypes.data, len(cu) - 1, H, dt, act, o, final, tail]
+    if recurrent:
+        return kda.lib.kda_prefill_recurrent(*args, None)
+    return kda.lib.kda_prefill(*args, ws, wsb, None)
+
+
+@pytest.mark.parametrize("recurrent", [False, True])
+def test_prefill_argument_validation(recurrent):
+    p = lambda *a, **kw: _prefill(*a, recurrent=recurrent, **kw)  # noqa: E731
+    assert p([0, 5], H=0) == 1
+    assert p([0, 5], dt=7) == 1
+    assert p([0, 5], act=5) == 1
+    assert p([1, 5]) == 1          # cu[0] != 0
+    assert p([0, 5, 3]) == 1       # decreasing offsets
+    assert p([0, 5], q=Q + 2) == 3  # misaligned
+    assert p([0, 5], beta=B + 1) == 3
+    assert p([0, 5], final=None) == 1
+    assert p([0, 5], tail=None) == 1
+    assert p([0, 5], q=None) == 1
+    assert p([0, 5], o=Q) == 1     # output aliases an input
+    assert p([0] * 70001) == 2     # more segments than the grid allows
+    assert p([0]) == 0             # no segments: nothing to do, no launch
+
+
+def test_prefill_workspace_check():
+    need = kda.lib.kda_prefill_workspace_size(2, 10, 4, 5, 1)
+    if need == 0:
+        pytest.skip("the bf16 path needs no workspace")
+    assert _prefill([0, 5, 10], ws=None, wsb=0) == 4
+    assert _prefill([0, 5, 10], wsb=need - 1) == 4
+    assert _prefill([0, 5, 10], ws=WS + 8) == 3
+
+
+def test_decode_argument_validation():
+    d = kda.lib.kda_decode_step
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 0, 1, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 3, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 9, O, None) == 1
+    assert d(FS + 4, CT, Q, K, V, G, B, W, 4, 2, 1, 0, O, None) == 3
+    assert d(FS, CT, Q, K, V, G, B + 1, W, 4, 2, 1, 0, O, None) == 3
+    assert d(None, CT, Q, K, V, G, B, W, 4, 2, 1, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, Q, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 70000, 2, 1, 0, O, None) == 2
+    assert d(FS, CT, Q, K, V, G, B, W, 0, 2, 1, 0, O, None) == 0
