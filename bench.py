@@ -36,16 +36,16 @@ sys.path.insert(0, ROOT)
 import kda_inputs as ki  # noqa: E402
 
 METRIC = "KDA prefill tokens/s (64 heads, T=64k) and decode state GB/s vs HBM peak"
-WORKLOAD = "kda_prefill long-context: 1 x T=65536, 64 heads x 128, bf16 in / fp32 state, chunk 64"
+WORKLOAD = "kda_prefill long-context: 1 x T=65536, 64 heads x 128, bf16 in / fp32 state / fp32 out, chunk 64"
 H, D, T_LONG = 64, 128, 65536
 # algorithmic bytes (what the method must move): per token-head q,k,v,g (4 x 256 B bf16)
-# + beta (2 B) + o (256 B); per (sequence, head) the final state (64 KiB; no initial
-# state in this workload).
-BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 2 + D * 2
+# + beta (2 B) + o (512 B fp32); per (sequence, head) the final state (64 KiB; no
+# initial state in this workload).
+BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 2 + D * 4
 STATE_BYTES = D * D * 4
-# decode: per (sequence, head) the state read + written, q/k/v/g in, o out, beta,
+# decode: per (sequence, head) the state read + written, q/k/v/g in, o out (fp32), beta,
 # the conv cache (3 tokens x q/k/v read, 3 written)
-DEC_BYTES_PER_PAIR = 2 * STATE_BYTES + 4 * D * 2 + D * 2 + 2 + 2 * 9 * D * 2
+DEC_BYTES_PER_PAIR = 2 * STATE_BYTES + 4 * D * 2 + D * 4 + 2 + 2 * 9 * D * 2
 # kernels launched per call: kda_prefill bf16 = main kernel + conv-tail kernel
 PREFILL_LAUNCHES = 2
 DECODE_LAUNCHES = 1
@@ -248,7 +248,7 @@ def main():
     inp = ki.workload(2)
     d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "g", "beta", "conv_w")}
     cu_dev = torch.from_numpy(inp.cu_seqlens).to(dev)
-    o = torch.empty_like(d["q"])
+    o = torch.empty(d["q"].shape, dtype=torch.float32, device=dev)
     S = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
     tail = torch.empty((1, 3, 3, H * D), dtype=torch.bfloat16, device=dev)
     ws_bytes = kda.workspace_size(1, T_LONG, H, T_LONG)
@@ -291,7 +291,7 @@ def main():
     # ---------------- decode step: 256 sequences, state in place ----------------
     dec = ki.workload(4)
     dd = {n: getattr(dec, n).to(dev) for n in ("state", "conv_cache", "q", "k", "v", "g", "beta", "conv_w")}
-    o_dec = torch.empty_like(dd["q"])
+    o_dec = torch.empty(dd["q"].shape, dtype=torch.float32, device=dev)
 
     def dstep():
         kda.decode_step(dd["state"], dd["conv_cache"], dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],

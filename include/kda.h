@@ -33,6 +33,10 @@
  *    [N, 3 (q,k,v), 3 (time, oldest first), H*128] in the input dtype.
  *  - L2 norm: x / sqrt(sum x^2 + 1e-6).  No query scale.  Conv activation:
  *    KDA_CONV_NONE (default) or KDA_CONV_SILU (y * sigmoid(y)).
+ *  - The output o has its own element type `o_dt` (fp32 or bf16).  Outputs of
+ *    this layer are heavy-tailed (an aligned q_t, k_t pair makes |o_t| many
+ *    times its rms), so rounding o to bf16 alone moves the largest elements
+ *    by several percent of rms; fp32 keeps the full result.
  *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream).  Argument errors are detected on the host before
  *    anything is launched and returned as a status; nothing aborts.
@@ -83,7 +87,8 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_he
  *   cu_seqlens_dev   : [N+1] int32 device copy of the segment offsets.
  *   cu_seqlens_host  : [N+1] int32 host copy (used for scheduling; must equal
  *                      the device copy).  cu[0] == 0, non-decreasing.
- *   o                : out [total_T, H, 128] (dt).  Must not alias inputs.
+ *   o_dt             : element type of o (KDA_F32 or KDA_BF16).
+ *   o                : out [total_T, H, 128] (o_dt).  Must not alias inputs.
  *   final_state      : out [N, H, 128, 128] fp32; may equal init_state (in place).
  *   conv_tail        : out [N, 3, 3, H*128] (dt): last 3 raw tokens of
  *                      concat(init_conv, segment); may equal init_conv.
@@ -96,9 +101,9 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
                        const void* beta, const float* conv_w, const float* init_state,
                        const void* init_conv, const int32_t* cu_seqlens_dev,
                        const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
-                       kda_dtype dt, kda_conv_act act, void* o, float* final_state,
-                       void* conv_tail, void* workspace, size_t workspace_bytes,
-                       void* stream);
+                       kda_dtype dt, kda_conv_act act, kda_dtype o_dt, void* o,
+                       float* final_state, void* conv_tail, void* workspace,
+                       size_t workspace_bytes, void* stream);
 
 /*
  * kda_prefill_recurrent -- same contract as kda_prefill, always evaluated by
@@ -111,7 +116,8 @@ kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, co
                                  const float* init_state, const void* init_conv,
                                  const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
                                  int num_seqs, int num_heads, kda_dtype dt, kda_conv_act act,
-                                 void* o, float* final_state, void* conv_tail, void* stream);
+                                 kda_dtype o_dt, void* o, float* final_state, void* conv_tail,
+                                 void* stream);
 
 /*
  * kda_decode_step -- one recurrent update per sequence (page "GLM-5.3-Flash im
@@ -122,13 +128,13 @@ kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, co
  *                shifted in place so that it ends with this step's raw token.
  *   q, k, v, g : [N, H, 128] raw inputs of the new token (dt); beta : [N, H].
  *   conv_w     : [3, H*128, 4] fp32.
- *   o          : out [N, H, 128] (dt).
+ *   o_dt, o    : out [N, H, 128] with element type o_dt.
  * Each (sequence, head) state is streamed through registers exactly once.
  */
 kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const void* k,
                            const void* v, const void* g, const void* beta,
                            const float* conv_w, int num_seqs, int num_heads, kda_dtype dt,
-                           kda_conv_act act, void* o, void* stream);
+                           kda_conv_act act, kda_dtype o_dt, void* o, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* kda_status_string(kda_status s);

@@ -38,14 +38,14 @@ lib.kda_prefill_workspace_size.restype = ctypes.c_size_t
 lib.kda_prefill_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int]
 _PREFILL_ARGS = [_vp, _vp, _vp, _vp, _vp, _f32p, _f32p, _vp, _i32p, _i32p, ctypes.c_int, ctypes.c_int,
-                 ctypes.c_int, ctypes.c_int, _vp, _f32p, _vp]
+                 ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _f32p, _vp]
 lib.kda_prefill.restype = ctypes.c_int
 lib.kda_prefill.argtypes = _PREFILL_ARGS + [_vp, ctypes.c_size_t, _vp]
 lib.kda_prefill_recurrent.restype = ctypes.c_int
 lib.kda_prefill_recurrent.argtypes = _PREFILL_ARGS + [_vp]
 lib.kda_decode_step.restype = ctypes.c_int
 lib.kda_decode_step.argtypes = [_f32p, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
-                                ctypes.c_int, ctypes.c_int, _vp, _vp]
+                                ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp]
 lib.kda_status_string.restype = ctypes.c_char_p
 lib.kda_status_string.argtypes = [ctypes.c_int]
 lib.kda_check_async_status.restype = ctypes.c_int
@@ -94,9 +94,10 @@ def workspace_size(num_seqs: int, total_tokens: int, num_heads: int, max_seqlen:
 
 def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init_state=None,
             init_conv=None, act: int = KDA_CONV_NONE, o=None, final_state=None, conv_tail=None,
-            workspace=None, stream=None, recurrent: bool = False):
+            workspace=None, stream=None, recurrent: bool = False, o_dtype=torch.float32):
     """kda_prefill (or kda_prefill_recurrent) on device tensors.  Returns
-    (o, final_state, conv_tail); outputs are allocated when not given."""
+    (o, final_state, conv_tail); outputs are allocated when not given (o in
+    `o_dtype`, fp32 by default)."""
     cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
     N = len(cu_h) - 1
     T, H = q.shape[0], q.shape[1]
@@ -104,15 +105,15 @@ def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init
     if cu_seqlens_dev is None:
         cu_seqlens_dev = torch.from_numpy(cu_h).to(dev)
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=o_dtype, device=dev)
     if final_state is None:
         final_state = torch.empty((N, H, HEAD_DIM, HEAD_DIM), dtype=torch.float32, device=dev)
     if conv_tail is None:
         conv_tail = torch.empty((N, 3, 3, H * HEAD_DIM), dtype=q.dtype, device=dev)
     dt = _dtype_code(q)
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(conv_w), _ptr(init_state),
-            _ptr(init_conv), _ptr(cu_seqlens_dev), _ptr(cu_h), N, H, dt, int(act), _ptr(o),
-            _ptr(final_state), _ptr(conv_tail)]
+            _ptr(init_conv), _ptr(cu_seqlens_dev), _ptr(cu_h), N, H, dt, int(act), _dtype_code(o),
+            _ptr(o), _ptr(final_state), _ptr(conv_tail)]
     if recurrent:
         _check(lib.kda_prefill_recurrent(*args, _stream(stream)), "kda_prefill_recurrent")
     else:
@@ -125,14 +126,15 @@ def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init
 
 
 def decode_step(state, conv_cache, q, k, v, g, beta, conv_w, act: int = KDA_CONV_NONE, o=None,
-                stream=None):
-    """kda_decode_step in place on `state` and `conv_cache`; returns o."""
+                stream=None, o_dtype=torch.float32):
+    """kda_decode_step in place on `state` and `conv_cache`; returns o
+    (allocated in `o_dtype` when not given)."""
     N, H = q.shape[0], q.shape[1]
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
     _check(lib.kda_decode_step(_ptr(state), _ptr(conv_cache), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                               _ptr(beta), _ptr(conv_w), N, H, _dtype_code(q), int(act), _ptr(o),
-                               _stream(stream)), "kda_decode_step")
+                               _ptr(beta), _ptr(conv_w), N, H, _dtype_code(q), int(act), _dtype_code(o),
+                               _ptr(o), _stream(stream)), "kda_decode_step")
     return o
 
 

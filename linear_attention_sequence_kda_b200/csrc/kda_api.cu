@@ -25,6 +25,7 @@ struct PrefillArgs {
   int N, H;
   kda_dtype dt;
   kda_conv_act act;
+  kda_dtype o_dt;
   void* o;
   float* final_state;
   void* conv_tail;
@@ -37,6 +38,7 @@ kda_status validate_prefill(PrefillArgs& a) {
   if (a.N < 0 || a.H < 1) return KDA_ERR_INVALID_ARG;
   if (a.dt != KDA_F32 && a.dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (a.act != KDA_CONV_NONE && a.act != KDA_CONV_SILU) return KDA_ERR_INVALID_ARG;
+  if (a.o_dt != KDA_F32 && a.o_dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (a.N == 0) { a.total_T = 0; a.max_len = 0; return KDA_OK; }
   if (!a.cu_host || !a.cu_dev) return KDA_ERR_INVALID_ARG;
   if (a.cu_host[0] != 0) return KDA_ERR_INVALID_ARG;
@@ -73,17 +75,23 @@ kda_status launch_tail(const PrefillArgs& a) {
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+template <typename Tin, typename Tout, int ACT>
+void launch_recurrent_t(const PrefillArgs& a) {
+  recurrent_prefill_kernel<Tin, Tout, ACT><<<dim3(a.H, a.N), 128, 0, a.stream>>>(
+      (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.g, (const Tin*)a.beta,
+      a.conv_w, a.init_state, (const Tin*)a.init_conv, a.cu_dev, a.H, (Tout*)a.o, a.final_state);
+}
+
 template <typename Tin>
 kda_status launch_recurrent(const PrefillArgs& a) {
-  dim3 grid(a.H, a.N);
-  if (a.act == KDA_CONV_SILU)
-    recurrent_prefill_kernel<Tin, KDA_CONV_SILU><<<grid, 128, 0, a.stream>>>(
-        (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.g, (const Tin*)a.beta,
-        a.conv_w, a.init_state, (const Tin*)a.init_conv, a.cu_dev, a.H, (Tin*)a.o, a.final_state);
-  else
-    recurrent_prefill_kernel<Tin, KDA_CONV_NONE><<<grid, 128, 0, a.stream>>>(
-        (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.g, (const Tin*)a.beta,
-        a.conv_w, a.init_state, (const Tin*)a.init_conv, a.cu_dev, a.H, (Tin*)a.o, a.final_state);
+  const bool silu = a.act == KDA_CONV_SILU;
+  if (a.o_dt == KDA_F32) {
+    if (silu) launch_recurrent_t<Tin, float, KDA_CONV_SILU>(a);
+    else launch_recurrent_t<Tin, float, KDA_CONV_NONE>(a);
+  } else {
+    if (silu) launch_recurrent_t<Tin, __nv_bfloat16, KDA_CONV_SILU>(a);
+    else launch_recurrent_t<Tin, __nv_bfloat16, KDA_CONV_NONE>(a);
+  }
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
   return launch_tail<Tin>(a);
 }
@@ -91,6 +99,29 @@ kda_status launch_recurrent(const PrefillArgs& a) {
 kda_status run_recurrent(PrefillArgs& a) {
   if (a.N == 0) return KDA_OK;
   return a.dt == KDA_F32 ? launch_recurrent<float>(a) : launch_recurrent<__nv_bfloat16>(a);
+}
+
+template <typename Tin, typename Tout, int ACT>
+void launch_decode_t(float* state, void* cache, const void* q, const void* k, const void* v,
+                     const void* g, const void* beta, const float* conv_w, int N, int H, void* o,
+                     cudaStream_t s) {
+  decode_kernel<Tin, Tout, ACT><<<dim3(H, N), 256, 0, s>>>(
+      state, (Tin*)cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)g,
+      (const Tin*)beta, conv_w, H, (Tout*)o);
+}
+
+template <typename Tin>
+void launch_decode(kda_conv_act act, kda_dtype o_dt, float* state, void* cache, const void* q,
+                   const void* k, const void* v, const void* g, const void* beta,
+                   const float* conv_w, int N, int H, void* o, cudaStream_t s) {
+  const bool silu = act == KDA_CONV_SILU;
+  if (o_dt == KDA_F32) {
+    if (silu) launch_decode_t<Tin, float, KDA_CONV_SILU>(state, cache, q, k, v, g, beta, conv_w, N, H, o, s);
+    else launch_decode_t<Tin, float, KDA_CONV_NONE>(state, cache, q, k, v, g, beta, conv_w, N, H, o, s);
+  } else {
+    if (silu) launch_decode_t<Tin, __nv_bfloat16, KDA_CONV_SILU>(state, cache, q, k, v, g, beta, conv_w, N, H, o, s);
+    else launch_decode_t<Tin, __nv_bfloat16, KDA_CONV_NONE>(state, cache, q, k, v, g, beta, conv_w, N, H, o, s);
+  }
 }
 
 }  // namespace
@@ -109,9 +140,10 @@ kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, co
                                  const float* init_state, const void* init_conv,
                                  const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
                                  int num_seqs, int num_heads, kda_dtype dt, kda_conv_act act,
-                                 void* o, float* final_state, void* conv_tail, void* stream) {
+                                 kda_dtype o_dt, void* o, float* final_state, void* conv_tail,
+                                 void* stream) {
   PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
-                cu_seqlens_host, num_seqs, num_heads, dt, act, o, final_state, conv_tail,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, o, final_state, conv_tail,
                 (cudaStream_t)stream, 0, 0};
   kda_status st = validate_prefill(a);
   if (st != KDA_OK) return st;
@@ -122,11 +154,11 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
                        const void* beta, const float* conv_w, const float* init_state,
                        const void* init_conv, const int32_t* cu_seqlens_dev,
                        const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
-                       kda_dtype dt, kda_conv_act act, void* o, float* final_state,
-                       void* conv_tail, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+                       kda_dtype dt, kda_conv_act act, kda_dtype o_dt, void* o,
+                       float* final_state, void* conv_tail, void* workspace,
+                       size_t workspace_bytes, void* stream) {
   PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
-                cu_seqlens_host, num_seqs, num_heads, dt, act, o, final_state, conv_tail,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, o, final_state, conv_tail,
                 (cudaStream_t)stream, 0, 0};
   kda_status st = validate_prefill(a);
   if (st != KDA_OK) return st;
@@ -136,7 +168,8 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
   if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
   if (workspace && !aligned(workspace, 16)) return KDA_ERR_ALIGNMENT;
   st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
-                      a.cu_host, a.N, a.H, a.act, a.o, a.final_state, workspace, a.stream);
+                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.o, a.final_state, workspace,
+                      workspace_bytes, a.max_len, a.stream);
   if (st != KDA_OK) return st;
   return launch_tail<__nv_bfloat16>(a);
 }
@@ -144,9 +177,10 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
 kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const void* k,
                            const void* v, const void* g, const void* beta,
                            const float* conv_w, int num_seqs, int num_heads, kda_dtype dt,
-                           kda_conv_act act, void* o, void* stream) {
+                           kda_conv_act act, kda_dtype o_dt, void* o, void* stream) {
   if (num_seqs < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
   if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (o_dt != KDA_F32 && o_dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
   if (act != KDA_CONV_NONE && act != KDA_CONV_SILU) return KDA_ERR_INVALID_ARG;
   if (num_seqs == 0) return KDA_OK;
   if (num_seqs > 65535) return KDA_ERR_UNSUPPORTED;
@@ -158,19 +192,12 @@ kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const 
   if (!aligned(beta, esize(dt))) return KDA_ERR_ALIGNMENT;
   if (o == q || o == k || o == v || o == g) return KDA_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  dim3 grid(num_heads, num_seqs);
-#define KDA_DECODE_LAUNCH(T, A)                                                               \
-  decode_kernel<T, A><<<grid, 256, 0, s>>>(state, (T*)conv_cache, (const T*)q, (const T*)k,   \
-                                           (const T*)v, (const T*)g, (const T*)beta, conv_w, \
-                                           num_heads, (T*)o)
-  if (dt == KDA_F32) {
-    if (act == KDA_CONV_SILU) KDA_DECODE_LAUNCH(float, KDA_CONV_SILU);
-    else KDA_DECODE_LAUNCH(float, KDA_CONV_NONE);
-  } else {
-    if (act == KDA_CONV_SILU) KDA_DECODE_LAUNCH(__nv_bfloat16, KDA_CONV_SILU);
-    else KDA_DECODE_LAUNCH(__nv_bfloat16, KDA_CONV_NONE);
-  }
-#undef KDA_DECODE_LAUNCH
+  if (dt == KDA_F32)
+    launch_decode<float>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w, num_seqs,
+                         num_heads, o, s);
+  else
+    launch_decode<__nv_bfloat16>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w,
+                                 num_seqs, num_heads, o, s);
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

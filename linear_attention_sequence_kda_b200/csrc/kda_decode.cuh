@@ -19,12 +19,12 @@
 
 namespace kda {
 
-template <typename Tin, int ACT>
+template <typename Tin, typename Tout, int ACT>
 __global__ void __launch_bounds__(256, 2)
 decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
               const Tin* __restrict__ k, const Tin* __restrict__ v, const Tin* __restrict__ g,
               const Tin* __restrict__ beta, const float* __restrict__ conv_w, int H,
-              Tin* __restrict__ o) {
+              Tout* __restrict__ o) {
   __shared__ __align__(16) float sh_kh[D], sh_ka[D], sh_qa[D], sh_al[D], sh_v[D], sh_u[D];
   __shared__ __align__(16) float sh_r[8][D], sh_y[8][D];
   __shared__ float sh_red[4][3];
@@ -104,7 +104,7 @@ decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __r
     const float b = to_f(beta[(int64_t)n * H + h]);
     const float u = b * (sh_v[tid] - rr);
     sh_u[tid] = u;
-    o[tok] = from_f<Tin>(yy + u * kq);
+    o[tok] = from_f<Tout>(yy + u * kq);
   }
   __syncthreads();
 

@@ -17,13 +17,13 @@ namespace kda {
 
 constexpr int REC_TB = 16;  // tokens per prologue block
 
-template <typename Tin, int ACT>
+template <typename Tin, typename Tout, int ACT>
 __global__ void __launch_bounds__(128)
 recurrent_prefill_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                          const Tin* __restrict__ v, const Tin* __restrict__ g,
                          const Tin* __restrict__ beta, const float* __restrict__ conv_w,
                          const float* init_state, const Tin* __restrict__ init_conv,
-                         const int32_t* __restrict__ cu, int H, Tin* __restrict__ o,
+                         const int32_t* __restrict__ cu, int H, Tout* __restrict__ o,
                          float* final_state) {
   __shared__ __align__(16) float sh_kh[REC_TB][D];    // k_hat
   __shared__ __align__(16) float sh_ka[REC_TB][D];    // alpha * k_hat
@@ -132,7 +132,7 @@ recurrent_prefill_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
         S[i + 2] = fmaf(al.z, S[i + 2], kh.z * u);
         S[i + 3] = fmaf(al.w, S[i + 3], kh.w * u);
       }
-      o[(tb + t) * HD + ch] = from_f<Tin>(out);
+      o[(tb + t) * HD + ch] = from_f<Tout>(out);
     }
     __syncthreads();  // before the next prologue overwrites shared memory
   }

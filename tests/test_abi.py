@@ -50,9 +50,10 @@ def test_workspace_size_invalid_is_zero():
 
 
 def _prefill(cu, H=4, dt=1, act=0, q=Q, o=O, final=FS, tail=CT, ws=WS, wsb=1 << 40, beta=B,
-             recurrent=False):
+             recurrent=False, odt=0):
     cu = np.ascontiguousarray(np.asarray(cu, dtype=np.int32))
-    args = [q, K, V, G, beta, W, None, None, CU, cu.ctypes.data, len(cu) - 1, H, dt, act, o, final, tail]
+    args = [q, K, V, G, beta, W, None, None, CU, cu.ctypes.data, len(cu) - 1, H, dt, act, odt, o, final,
+            tail]
     if recurrent:
         return kda.lib.kda_prefill_recurrent(*args, None)
     return kda.lib.kda_prefill(*args, ws, wsb, None)
@@ -64,6 +65,7 @@ def test_prefill_argument_validation(recurrent):
     assert p([0, 5], H=0) == 1
     assert p([0, 5], dt=7) == 1
     assert p([0, 5], act=5) == 1
+    assert p([0, 5], odt=3) == 1
     assert p([1, 5]) == 1          # cu[0] != 0
     assert p([0, 5, 3]) == 1       # decreasing offsets
     assert p([0, 5], q=Q + 2) == 3  # misaligned
@@ -87,12 +89,13 @@ def test_prefill_workspace_check():
 
 def test_decode_argument_validation():
     d = kda.lib.kda_decode_step
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 0, 1, 0, O, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 3, 0, O, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 9, O, None) == 1
-    assert d(FS + 4, CT, Q, K, V, G, B, W, 4, 2, 1, 0, O, None) == 3
-    assert d(FS, CT, Q, K, V, G, B + 1, W, 4, 2, 1, 0, O, None) == 3
-    assert d(None, CT, Q, K, V, G, B, W, 4, 2, 1, 0, O, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, Q, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 70000, 2, 1, 0, O, None) == 2
-    assert d(FS, CT, Q, K, V, G, B, W, 0, 2, 1, 0, O, None) == 0
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 0, 1, 0, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 3, 0, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 9, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 5, O, None) == 1
+    assert d(FS + 4, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, O, None) == 3
+    assert d(FS, CT, Q, K, V, G, B + 1, W, 4, 2, 1, 0, 0, O, None) == 3
+    assert d(None, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, Q, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 70000, 2, 1, 0, 0, O, None) == 2
+    assert d(FS, CT, Q, K, V, G, B, W, 0, 2, 1, 0, 0, O, None) == 0

@@ -48,6 +48,17 @@ def test_decode_fp32(act):
     assert _compare(inp, _run(inp, act), act) <= 1e-4
 
 
+def test_decode_bf16_output_is_rounded_fp32_output():
+    inp = ki.make_decode(6, 4, torch.bfloat16, 23)
+    outs = []
+    for od in (torch.float32, torch.bfloat16):
+        state = inp.state.clone().cuda()
+        cache = inp.conv_cache.clone().cuda()
+        outs.append(kda.decode_step(state, cache, inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), inp.g.cuda(),
+                                    inp.beta.cuda(), inp.conv_w.cuda(), o_dtype=od))
+    assert torch.equal(outs[1], outs[0].to(torch.bfloat16))
+
+
 def test_decode_bf16_silu_single_head():
     inp = ki.make_decode(7, 1, torch.bfloat16, 22)
     _compare(inp, _run(inp, 1), 1)

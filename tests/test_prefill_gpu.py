@@ -60,6 +60,16 @@ def test_gate_floor_and_beta_extremes():
     compare_prefill(inp, run_prefill(inp))
 
 
+def test_bf16_output_is_rounded_fp32_output():
+    """o_dt = bf16 gives exactly the fp32 result rounded to bf16."""
+    inp = ki.make_prefill([130, 7], 2, torch.bfloat16, 15, state_std=0.02, conv_history=True)
+    d = to_dev(inp)
+    o32 = run_prefill(inp, dev_inputs=d)[0]
+    o16 = run_prefill(inp, dev_inputs=d, o_dtype=torch.bfloat16)[0]
+    assert o16.dtype == torch.bfloat16
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+
+
 def test_all_segments_empty():
     inp = ki.make_prefill([0, 0], 2, torch.bfloat16, 10, state_std=0.02, conv_history=True)
     o, S, tail = run_prefill(inp)
