@@ -46,8 +46,8 @@ STATE_BYTES = D * D * 4
 # decode: per (sequence, head) the state read + written, q/k/v/g in, o out (fp32), beta,
 # the conv cache (3 tokens x q/k/v read, 3 written)
 DEC_BYTES_PER_PAIR = 2 * STATE_BYTES + 4 * D * 2 + D * 4 + 2 + 2 * 9 * D * 2
-# kernels launched per call: kda_prefill bf16 = main kernel + conv-tail kernel
-PREFILL_LAUNCHES = 2
+# kernels launched per call: kda_prefill bf16 = chunk_prep + chunk_scan + conv tail
+PREFILL_LAUNCHES = 3
 DECODE_LAUNCHES = 1
 
 
@@ -267,7 +267,7 @@ def main():
     alg_bytes = T_LONG * H * BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
     launch_ms = statistics.mean(per_step)
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
-    kernel_name = "kda_chunked_prefill"
+    kernel_name = "kda_prefill (chunk_prep_kernel + chunk_scan_kernel)"
     traffic = recorded_traffic(kernel_name)
 
     # ---------------- end to end: host buffers through the C ABI ----------------

@@ -132,7 +132,7 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_he
                                   int max_seqlen, kda_dtype dt) {
   if (num_seqs < 0 || total_tokens < 0 || num_heads < 1 || max_seqlen < 0) return 0;
   if (dt != KDA_BF16) return 0;
-  return chunked_workspace_bytes(num_seqs, num_heads);
+  return chunked_workspace_bytes(num_seqs, num_heads, total_tokens);
 }
 
 kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, const void* g,
@@ -164,7 +164,7 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
   if (st != KDA_OK) return st;
   if (a.N == 0) return KDA_OK;
   if (dt == KDA_F32) return run_recurrent(a);
-  const size_t need = chunked_workspace_bytes(a.N, a.H);
+  const size_t need = chunked_workspace_bytes(a.N, a.H, a.total_T);
   if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
   if (workspace && !aligned(workspace, 16)) return KDA_ERR_ALIGNMENT;
   st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,

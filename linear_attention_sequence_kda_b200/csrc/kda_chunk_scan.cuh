@@ -1,0 +1,251 @@
+// Chunk scan (the state-dependent half of the chunked KDA prefill): one thread
+// block per (segment, head), serial over the segment's chunks, the 128 x 128
+// fp32 state held in tensor memory the whole time (page "GLM-5.3-Flash im
+// Detail", section "Sequenz-Mixing: 34 KDA-Schichten mit festem Zustand": a
+// state is handed from chunk to chunk).
+//
+// Thread v (of 128) owns value column v: TMEM lane v holds row v of
+//   V^T (cols 0..63) | S^T (cols 64..191) | U^T (192..255) | O^T (256..319).
+// Per chunk, with the record written by chunk_prep_kernel:
+//   MMA1  U^T = [V^T | S^T] [T_s | -W]^T        (K = 64 + 128)
+//         O^T = S^T Q~^T                          (K = 128)
+//   fp32  U^T += beta * V^T (diagonal of T);  S^T <- S^T diag(e^{Gamma_C})
+//   MMA2  O^T += U^T P_s^T;   S^T += U^T K-bar    (K = 64, A = U^T from TMEM)
+//   fp32  o = O + P_tt u (diagonal of P), written to HBM.
+// A operands are read from TMEM as tf32; the state itself stays fp32.
+#pragma once
+#include "kda_chunk_prep.cuh"
+#include "kda_common.cuh"
+#include "kda_tc.cuh"
+
+namespace kda {
+
+constexpr uint32_t SCAN_A0 = 0;                      // stage A buffer 0: B1 | QT (81920 B)
+constexpr uint32_t SCAN_A1 = REC_TILES_A;            // stage A buffer 1
+constexpr uint32_t SCAN_B = 2 * REC_TILES_A;         // stage B: PS | KB | SC (50176 B)
+constexpr uint32_t SCAN_SMEM = 2 * REC_TILES_A + REC_TILES_B + 1024;
+constexpr int TM_V = 0, TM_S = 64, TM_U = 192, TM_O = 256;
+
+template <typename Tout, int ACT>
+__global__ void __launch_bounds__(128, 1)
+chunk_scan_kernel(const __nv_bfloat16* __restrict__ v, const float* __restrict__ conv_w,
+                  const float* init_state, const __nv_bfloat16* __restrict__ init_conv,
+                  const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
+                  const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
+                  Tout* __restrict__ o, float* final_state) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ uint64_t bar_a[2], bar_b, bar_m1, bar_m2;
+  __shared__ uint32_t tmem_base;
+  __shared__ float sc[256];  // this chunk's beta[64], P_tt[64], e^{Gamma_C}[128]
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int n = seq_order[blockIdx.x / H], h = blockIdx.x % H;
+  const int64_t seg0 = cu[n], T = cu[n + 1] - seg0;
+  const int nchunks = (int)((T + CH - 1) / CH);
+  const int64_t HD = (int64_t)H * D;
+  const int64_t chan = (int64_t)h * D + tid;
+  const uint8_t* rec0 = records + (int64_t)chunk_base[n] * H * REC_BYTES + (int64_t)h * REC_BYTES;
+  const int64_t rec_stride = (int64_t)H * REC_BYTES;  // next chunk of the same head
+
+  if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
+  if (tid == 0) {
+    tc::bar_init(&bar_a[0], 1); tc::bar_init(&bar_a[1], 1); tc::bar_init(&bar_b, 1);
+    tc::bar_init(&bar_m1, 1); tc::bar_init(&bar_m2, 1);
+    tc::bar_init_fence();
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tm = tmem_base;
+  const uint32_t lane_base = tm + ((uint32_t)(32 * warp) << 16);
+
+  // initial state: row v of S^T = column v of S
+  {
+    const float* Si = init_state ? init_state + ((int64_t)n * H + h) * D * D + tid : nullptr;
+    for (int g16 = 0; g16 < 8; ++g16) {
+      float s[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) s[i] = Si ? Si[(int64_t)(16 * g16 + i) * D] : 0.f;
+      tc::st16(lane_base + TM_S + 16 * g16, s);
+    }
+  }
+  // value conv taps and history for channel tid
+  const float4 wv = load4(conv_w + (2 * HD + chan) * 4);
+  float hv0 = 0.f, hv1 = 0.f, hv2 = 0.f;
+  if (init_conv) {
+    const __nv_bfloat16* c = init_conv + ((int64_t)n * 9 + 6) * HD + chan;
+    hv0 = to_f(c[0]); hv1 = to_f(c[HD]); hv2 = to_f(c[2 * HD]);
+  }
+
+  // issued / waited counts per barrier (uniform across the block), so the exit
+  // path can wait for any copy or MMA still in flight before freeing TMEM
+  int a_iss[2] = {0, 0}, b_iss = 0, m1 = 0, m2 = 0;
+  auto load_a = [&](int i) {
+    const uint8_t* r = rec0 + (int64_t)i * rec_stride;
+    uint8_t* dst = sm + ((i & 1) ? SCAN_A1 : SCAN_A0);
+    tc::bar_expect_tx(&bar_a[i & 1], REC_TILES_A);
+    tc::bulk_g2s(dst, r, REC_TILES_A, &bar_a[i & 1]);
+  };
+  auto load_b = [&](int i) {
+    const uint8_t* r = rec0 + (int64_t)i * rec_stride + REC_PS;
+    tc::bar_expect_tx(&bar_b, REC_TILES_B);
+    tc::bulk_g2s(sm + SCAN_B, r, REC_TILES_B, &bar_b);
+  };
+  if (nchunks > 0) {
+    if (tid == 0) {
+      load_a(0);
+      if (nchunks > 1) load_a(1);
+      load_b(0);
+    }
+    a_iss[0] = 1; a_iss[1] = nchunks > 1; b_iss = 1;
+  }
+
+  bool ok = true;
+  for (int i = 0; i < nchunks && ok; ++i) {
+    const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
+    const int64_t t0 = seg0 + (int64_t)CH * i;
+    uint8_t* sa = sm + ((i & 1) ? SCAN_A1 : SCAN_A0);
+    uint8_t* sb = sm + SCAN_B;
+
+    // (a) causal conv of v for this chunk; V^T row into TMEM (tf32)
+    float vv[CH];
+#pragma unroll
+    for (int t = 0; t < CH; ++t) {
+      float y = 0.f;
+      if (t < L) {
+        const float x = to_f(v[(t0 + t) * HD + chan]);
+        y = conv4(wv, hv0, hv1, hv2, x);
+        if (ACT == KDA_CONV_SILU) y = silu(y);
+        hv0 = hv1; hv1 = hv2; hv2 = x;
+      }
+      vv[t] = y;
+    }
+#pragma unroll
+    for (int g16 = 0; g16 < 4; ++g16) {
+      float r[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) r[j] = tc::to_tf32(vv[16 * g16 + j]);
+      tc::st16(lane_base + TM_V + 16 * g16, r);
+    }
+    tc::st_wait();
+    // (b) this chunk's tiles
+    ok &= tc::bar_wait(&bar_a[i & 1], (i >> 1) & 1);
+    ok &= tc::bar_wait(&bar_b, i & 1);
+    sc[tid] = reinterpret_cast<const float*>(sb + (REC_SC - REC_PS))[tid];
+    sc[tid + 128] = reinterpret_cast<const float*>(sb + (REC_SC - REC_PS))[tid + 128];
+    tc::fence_before();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    // (c) MMA group 1
+    if (tid == 0) {
+      tc::fence_after();
+      const uint32_t b1 = tc::smem_u32(sa), qt = tc::smem_u32(sa + REC_QT);
+#pragma unroll
+      for (int ks = 0; ks < 24; ++ks)
+        tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, tc::desc_k(b1, 64, ks), tc::idesc_tf32(128, 64), ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks)
+        tc::mma_ts(tm + TM_O, tm + TM_S + 8 * ks, tc::desc_k(qt, 64, ks), tc::idesc_tf32(128, 64), ks > 0);
+      tc::commit(&bar_m1);
+    }
+    ++m1;
+    ok &= tc::bar_wait(&bar_m1, i & 1);
+    tc::fence_after();
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    if (i + 2 < nchunks) {  // stage A buffer is free again
+      if (tid == 0) load_a(i + 2);
+      a_iss[i & 1]++;
+    }
+    // (d) U += beta V (exact diagonal of T V), S^T <- S^T diag(gamma)
+    float uu[CH];
+#pragma unroll
+    for (int g16 = 0; g16 < 4; ++g16) {
+      float r[16];
+      tc::ld16(lane_base + TM_U + 16 * g16, r);
+      tc::ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int t = 16 * g16 + j;
+        uu[t] = fmaf(sc[t], vv[t], r[j]);
+        r[j] = tc::to_tf32(uu[t]);
+      }
+      tc::st16(lane_base + TM_U + 16 * g16, r);
+    }
+#pragma unroll
+    for (int g16 = 0; g16 < 8; ++g16) {
+      float r[16];
+      tc::ld16(lane_base + TM_S + 16 * g16, r);
+      tc::ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) r[j] *= sc[128 + 16 * g16 + j];
+      tc::st16(lane_base + TM_S + 16 * g16, r);
+    }
+    tc::st_wait();
+    tc::fence_before();
+    __syncthreads();
+    // (e) MMA group 2
+    if (tid == 0) {
+      tc::fence_after();
+      const uint32_t ps = tc::smem_u32(sb), kb = tc::smem_u32(sb + (REC_KB - REC_PS));
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        tc::mma_ts(tm + TM_O, tm + TM_U + 8 * ks, tc::desc_k(ps, 64, ks), tc::idesc_tf32(128, 64), 1);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, tc::desc_k(kb, 128, ks), tc::idesc_tf32(128, 128), 1);
+      tc::commit(&bar_m2);
+    }
+    ++m2;
+    ok &= tc::bar_wait(&bar_m2, i & 1);
+    tc::fence_after();
+    if (!__syncthreads_and(ok)) { ok = false; break; }
+    if (i + 1 < nchunks) {  // stage B is free again
+      if (tid == 0) load_b(i + 1);
+      b_iss++;
+    }
+    // (f) o = O + P_tt u
+#pragma unroll
+    for (int g16 = 0; g16 < 4; ++g16) {
+      float r[16];
+      tc::ld16(lane_base + TM_O + 16 * g16, r);
+      tc::ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int t = 16 * g16 + j;
+        if (t < L) o[(t0 + t) * HD + chan] = from_f<Tout>(fmaf(sc[64 + t], uu[t], r[j]));
+      }
+    }
+    tc::fence_before();
+    __syncthreads();  // sc and TMEM O are rewritten by the next chunk
+    tc::fence_after();
+  }
+
+  if (!ok) {
+    // a wait gave up (status already recorded): drain what is still in flight
+    // (each bounded) so that TMEM and shared memory are idle before exit
+    if (tid == 0) tc::commit(&bar_m2);
+    tc::bar_wait(&bar_m2, m2 & 1);
+    // waiting on the parity of the last issued phase returns at once if it
+    // already completed
+    for (int b = 0; b < 2; ++b)
+      if (a_iss[b] > 0) tc::bar_wait(&bar_a[b], (a_iss[b] - 1) & 1);
+    if (b_iss > 0) tc::bar_wait(&bar_b, (b_iss - 1) & 1);
+  }
+  // final state: column v of S = row v of S^T
+  if (ok) {
+    float* Sf = final_state + ((int64_t)n * H + h) * D * D + tid;
+    for (int g16 = 0; g16 < 8; ++g16) {
+      float s[16];
+      tc::ld16(lane_base + TM_S + 16 * g16, s);
+      tc::ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) Sf[(int64_t)(16 * g16 + i) * D] = s[i];
+    }
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+}  // namespace kda

@@ -1,33 +1,106 @@
-// Chunked bf16 prefill entry (interim: evaluated by the recurrent kernel).
+// Chunked bf16 prefill on the tensor cores: host-side scheduling and launches.
+// Two kernels on the caller's stream: chunk_prep_kernel (every chunk of every
+// (segment, head) in parallel) writes one operand record per chunk-head into
+// the workspace; chunk_scan_kernel (one block per (segment, head), longest
+// segments first) carries the state across the segment's chunks.
 #pragma once
+#include <algorithm>
+#include <numeric>
+#include <vector>
+
+#include "kda_chunk_prep.cuh"
+#include "kda_chunk_scan.cuh"
 #include "kda_common.cuh"
-#include "kda_recurrent.cuh"
 
 namespace kda {
 
-inline size_t chunked_workspace_bytes(int /*N*/, int /*H*/) { return 0; }
+// workspace = header (chunk table, per-segment first chunk, segment order),
+// then REC_BYTES per (chunk, head)
+inline int64_t chunk_bound(int N, int64_t total_tokens) { return total_tokens / CH + N; }
+inline size_t chunk_header_bytes(int N, int64_t nchunks) {
+  const size_t b = (size_t)nchunks * sizeof(int2) + (size_t)(N + 1) * 4 + (size_t)N * 4;
+  return (b + 1023) & ~(size_t)1023;
+}
+inline size_t chunked_workspace_bytes(int N, int H, int64_t total_tokens) {
+  const int64_t nc = chunk_bound(N, total_tokens);
+  return chunk_header_bytes(N, nc) + (size_t)nc * H * REC_BYTES;
+}
+
+template <int ACT>
+inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, const void* g,
+                                   const void* beta, const float* conv_w, const float* init_state,
+                                   const void* init_conv, const int32_t* cu_dev,
+                                   const int32_t* cu_host, int N, int H, kda_dtype o_dt, void* o,
+                                   float* final_state, void* workspace, cudaStream_t stream) {
+  using T = __nv_bfloat16;
+  // chunk table and longest-first segment order
+  std::vector<int64_t> nch(N);
+  int64_t total = 0;
+  for (int n = 0; n < N; ++n) {
+    nch[n] = ((int64_t)cu_host[n + 1] - cu_host[n] + CH - 1) / CH;
+    total += nch[n];
+  }
+  const size_t hdr = chunk_header_bytes(N, total);
+  std::vector<uint8_t> host(hdr, 0);
+  int2* tab = reinterpret_cast<int2*>(host.data());
+  int32_t* base = reinterpret_cast<int32_t*>(host.data() + (size_t)total * sizeof(int2));
+  int32_t* order = base + (N + 1);
+  int64_t c = 0;
+  for (int n = 0; n < N; ++n) {
+    base[n] = (int32_t)c;
+    for (int64_t i = 0; i < nch[n]; ++i) tab[c++] = make_int2(n, (int)i);
+  }
+  base[N] = (int32_t)c;
+  std::iota(order, order + N, 0);
+  std::stable_sort(order, order + N, [&](int a, int b) { return nch[a] > nch[b]; });
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // pageable source: the call returns after the bytes are staged, so `host`
+  // may be released right after
+  if (cudaMemcpyAsync(ws, host.data(), hdr, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  const int2* d_tab = reinterpret_cast<const int2*>(ws);
+  const int32_t* d_base = reinterpret_cast<const int32_t*>(ws + (size_t)total * sizeof(int2));
+  const int32_t* d_order = d_base + (N + 1);
+  uint8_t* records = ws + hdr;
+
+  if (total > 0) {
+    auto prep = chunk_prep_kernel<ACT>;
+    if (cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    prep<<<dim3((unsigned)total, H), 256, PREP_SMEM, stream>>>(
+        (const T*)q, (const T*)k, (const T*)g, (const T*)beta, conv_w, (const T*)init_conv, cu_dev,
+        d_tab, H, records);
+    if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  if (o_dt == KDA_F32) {
+    auto scan = chunk_scan_kernel<float, ACT>;
+    if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    scan<<<(unsigned)N * H, 128, SCAN_SMEM, stream>>>((const T*)v, conv_w, init_state, (const T*)init_conv,
+                                                      cu_dev, d_base, d_order, H, records, (float*)o,
+                                                      final_state);
+  } else {
+    auto scan = chunk_scan_kernel<T, ACT>;
+    if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    scan<<<(unsigned)N * H, 128, SCAN_SMEM, stream>>>((const T*)v, conv_w, init_state, (const T*)init_conv,
+                                                      cu_dev, d_base, d_order, H, records, (T*)o,
+                                                      final_state);
+  }
+  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
 
 inline kda_status launch_chunked(const void* q, const void* k, const void* v, const void* g,
                                  const void* beta, const float* conv_w, const float* init_state,
                                  const void* init_conv, const int32_t* cu_dev,
-                                 const int32_t* /*cu_host*/, int N, int H, kda_conv_act act,
-                                 kda_dtype o_dt, void* o, float* final_state,
-                                 void* /*workspace*/, size_t /*workspace_bytes*/, int /*max_len*/,
-                                 cudaStream_t stream) {
-  using T = __nv_bfloat16;
-  dim3 grid(H, N);
-  const bool silu = act == KDA_CONV_SILU;
-#define KDA_REC(TO, A)                                                                          \
-  recurrent_prefill_kernel<T, TO, A><<<grid, 128, 0, stream>>>(                                  \
-      (const T*)q, (const T*)k, (const T*)v, (const T*)g, (const T*)beta, conv_w, init_state,   \
-      (const T*)init_conv, cu_dev, H, (TO*)o, final_state)
-  if (o_dt == KDA_F32) {
-    if (silu) KDA_REC(float, KDA_CONV_SILU); else KDA_REC(float, KDA_CONV_NONE);
-  } else {
-    if (silu) KDA_REC(T, KDA_CONV_SILU); else KDA_REC(T, KDA_CONV_NONE);
-  }
-#undef KDA_REC
-  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+                                 const int32_t* cu_host, int N, int H, kda_conv_act act,
+                                 kda_dtype o_dt, void* o, float* final_state, void* workspace,
+                                 size_t /*workspace_bytes*/, int /*max_len*/, cudaStream_t stream) {
+  if (act == KDA_CONV_SILU)
+    return launch_chunked_t<KDA_CONV_SILU>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
+                                           cu_host, N, H, o_dt, o, final_state, workspace, stream);
+  return launch_chunked_t<KDA_CONV_NONE>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
+                                         cu_host, N, H, o_dt, o, final_state, workspace, stream);
 }
 
 }  // namespace kda
