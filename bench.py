@@ -227,8 +227,13 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode leg")
+    ap.add_argument("--heads", type=int, default=H,
+                    help="reduced head count (profiling only; the reported workload uses 64)")
+    ap.add_argument("--seq-len", type=int, default=T_LONG,
+                    help="reduced length (profiling only; the reported workload uses 65536)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -245,13 +250,17 @@ def main():
     hbm_peak, bf16_peak, peak_src = peaks()
 
     # ---------------- prefill: long-context workload, resident in HBM ----------
-    inp = ki.workload(2)
+    heads, T_run = args.heads, args.seq_len
+    if (heads, T_run) == (H, T_LONG):
+        inp = ki.workload(2)
+    else:  # same recipe, reduced size (for profiler captures)
+        inp = ki.make_prefill([T_run], heads, torch.bfloat16, ki.BASE_SEED + 2, gate="bimodal")
     d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "g", "beta", "conv_w")}
     cu_dev = torch.from_numpy(inp.cu_seqlens).to(dev)
     o = torch.empty(d["q"].shape, dtype=torch.float32, device=dev)
-    S = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
-    tail = torch.empty((1, 3, 3, H * D), dtype=torch.bfloat16, device=dev)
-    ws_bytes = kda.workspace_size(1, T_LONG, H, T_LONG)
+    S = torch.empty((1, heads, D, D), dtype=torch.float32, device=dev)
+    tail = torch.empty((1, 3, 3, heads * D), dtype=torch.bfloat16, device=dev)
+    ws_bytes = kda.workspace_size(1, T_run, heads, T_run)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
 
     def step():
@@ -262,15 +271,55 @@ def main():
         total_ms, per_step = timed(step, args.steps, args.warmup, world, stream)
     assert kda.check_async_status(stream) == 0
     ms = total_ms / args.steps
-    tokens_per_rank = T_LONG
+    tokens_per_rank = T_run
     value = world * tokens_per_rank * args.steps / (total_ms / 1e3)
-    alg_bytes = T_LONG * H * BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+    alg_bytes = T_run * heads * BYTES_PER_TOKEN_HEAD + heads * STATE_BYTES
     launch_ms = statistics.mean(per_step)
     achieved = alg_bytes / (launch_ms / 1e3) / 1e9
     kernel_name = "kda_prefill (chunk_prep_kernel + chunk_scan_kernel)"
     traffic = recorded_traffic(kernel_name)
 
     # ---------------- end to end: host buffers through the C ABI ----------------
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e = run_e2e(args, world, stream, inp, d, o, S, step, tokens_per_rank)
+
+    # ---------------- decode step: 256 sequences, state in place ----------------
+    dec_line = None
+    if not args.no_decode:
+        dec_line = run_decode(args, world, dev, stream, kda, hbm_peak)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "heads": heads, "head_dim": D, "seq_len": T_run, "batch_per_gpu": 1,
+                   "chunk": 64, "parallelism": f"dp{world} (independent sequences per GPU)",
+                   "l2": "inputs larger than L2 (4.3 GB read per step), no flush"},
+        "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst)",
+                     "traffic": traffic, "algorithmic_bytes_per_launch": alg_bytes,
+                     "launch_ms": launch_ms},
+        "e2e": e2e,
+        "gpu_launches": args.steps * PREFILL_LAUNCHES,
+        "clocks": clk.summary(),
+        "decode": dec_line,
+    }
+    if (heads, T_run) != (H, T_LONG):
+        line["config"]["note"] = "reduced profiling size, not the reported workload"
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(args, world, stream, inp, d, o, S, step, tokens_per_rank):
+    """Same metric through the C ABI with host buffers: each step copies the
+    inputs from pinned host memory, runs kda_prefill, and reads o and the final
+    state back to pinned host memory."""
     pin = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "g", "beta")}
     o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     S_host = torch.empty(S.shape, dtype=S.dtype, pin_memory=True)
@@ -285,10 +334,13 @@ def main():
         S_host.copy_(S, non_blocking=True)
 
     e2e_ms, _ = timed(e2e_step, args.e2e_steps, 1, world, stream)
-    e2e_value = world * tokens_per_rank * args.e2e_steps / (e2e_ms / 1e3)
-    del pin, o_host, S_host
+    value = world * tokens_per_rank * args.e2e_steps / (e2e_ms / 1e3)
+    return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": args.e2e_steps}
 
-    # ---------------- decode step: 256 sequences, state in place ----------------
+
+def run_decode(args, world, dev, stream, kda, hbm_peak):
+    """kda_decode_step on the decode workload (256 sequences, state in place)."""
     dec = ki.workload(4)
     dd = {n: getattr(dec, n).to(dev) for n in ("state", "conv_cache", "q", "k", "v", "g", "beta", "conv_w")}
     o_dec = torch.empty(dd["q"].shape, dtype=torch.float32, device=dev)
@@ -297,43 +349,18 @@ def main():
         kda.decode_step(dd["state"], dd["conv_cache"], dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
                         dd["conv_w"], o=o_dec, stream=stream)
 
-    dec_total, dec_steps = timed(dstep, args.steps, args.warmup, world, stream)
+    _, dec_steps = timed(dstep, args.steps, args.warmup, world, stream)
     npairs = dec.num_seqs * H
     dec_ms = statistics.mean(dec_steps)
     dec_state_gbs = npairs * 2 * STATE_BYTES / (dec_ms / 1e3) / 1e9
     dec_alg_gbs = npairs * DEC_BYTES_PER_PAIR / (dec_ms / 1e3) / 1e9
-    dec_traffic = recorded_traffic("kda_decode")
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "heads": H, "head_dim": D, "seq_len": T_LONG, "batch_per_gpu": 1,
-                   "chunk": 64, "parallelism": f"dp{world} (independent sequences per GPU)",
-                   "l2": "inputs larger than L2 (4.3 GB read per step), no flush"},
-        "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst)",
-                     "traffic": traffic, "algorithmic_bytes_per_launch": alg_bytes,
-                     "launch_ms": launch_ms},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": args.e2e_steps},
-        "gpu_launches": args.steps * PREFILL_LAUNCHES,
-        "clocks": clk.summary(),
-        "decode": {"workload": "kda_decode_step: 256 sequences x 1 token, 64 heads x 128, fp32 state in place",
-                   "state_gbs": dec_state_gbs, "ms_per_step": dec_ms,
-                   "roofline": {"kernel": "kda_decode", "bound": "hbm", "achieved": dec_alg_gbs,
-                                "peak": hbm_peak, "unit": "GB/s", "frac": dec_alg_gbs / hbm_peak,
-                                "state_frac": dec_state_gbs / hbm_peak, "traffic": dec_traffic,
-                                "algorithmic_bytes_per_launch": npairs * DEC_BYTES_PER_PAIR},
-                   "gpu_launches": args.steps * DECODE_LAUNCHES},
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    return {"workload": "kda_decode_step: 256 sequences x 1 token, 64 heads x 128, fp32 state in place",
+            "state_gbs": dec_state_gbs, "ms_per_step": dec_ms,
+            "roofline": {"kernel": "kda_decode", "bound": "hbm", "achieved": dec_alg_gbs, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": dec_alg_gbs / hbm_peak, "state_frac": dec_state_gbs / hbm_peak,
+                         "traffic": recorded_traffic("kda_decode"),
+                         "algorithmic_bytes_per_launch": npairs * DEC_BYTES_PER_PAIR},
+            "gpu_launches": args.steps * DECODE_LAUNCHES}
 
 
 if __name__ == "__main__":

@@ -70,10 +70,14 @@ constexpr int SV_XD = 0 /*4x16x16*/, SV_YB = 1024 /*3x16x16*/;
 
 __device__ __forceinline__ int zidx(int I, int J) { return (I * (I - 1)) / 2 + J; }  // J < I
 
+// raw input tiles: 3 halo rows + 64 chunk rows of one head (128 bf16 = 256 B)
+constexpr int RAW_ROWS = CH + 3;
+constexpr uint32_t RAW_BYTES = RAW_ROWS * D * 2;  // 17152
+
 template <int ACT>
 __global__ void __launch_bounds__(256, 1)
-chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                  const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ beta,
+chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16* __restrict__ beta,
                   const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int2* __restrict__ chunk_tab, int H,
                   uint8_t* __restrict__ records) {
@@ -105,24 +109,39 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
   const int64_t chan = (int64_t)h * D + ch;
   uint8_t* rec = records + ((int64_t)cid * H + h) * REC_BYTES;
 
+  // raw tiles land in the region the Gram operands and M/P use later
+  const __nv_bfloat16* rq_t = reinterpret_cast<const __nv_bfloat16*>(sm + PREP_OPA);
+  const __nv_bfloat16* rk_t = reinterpret_cast<const __nv_bfloat16*>(sm + PREP_OPA + RAW_BYTES);
+  const __nv_bfloat16* rg_t = reinterpret_cast<const __nv_bfloat16*>(sm + PREP_OPA + 2 * RAW_BYTES);
   if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
-  if (tid == 0) { tc::bar_init(&bar, 1); tc::bar_init_fence(); }
+  if (tid == 0) {
+    tc::bar_init(&bar, 1);
+    tc::bar_init_fence();
+    // rows t0-3 .. t0+63 of head h (rows outside the tensor read as zero)
+    tc::bar_expect_tx(&bar, 3 * RAW_BYTES);
+    tc::tma_load_2d(sm + PREP_OPA, &tm_q, h * D, (int)(t0 - 3), &bar);
+    tc::tma_load_2d(sm + PREP_OPA + RAW_BYTES, &tm_k, h * D, (int)(t0 - 3), &bar);
+    tc::tma_load_2d(sm + PREP_OPA + 2 * RAW_BYTES, &tm_g, h * D, (int)(t0 - 3), &bar);
+  }
+  if (tid < CH) ms[MS_BETA + tid] = tid < L ? to_f(beta[(t0 + tid) * H + h]) : 0.f;
+  const float4 wq = load4(conv_w + (0 * HD + chan) * 4);
+  const float4 wk = load4(conv_w + (1 * HD + chan) * 4);
+  __syncthreads();
+  uint32_t phase = 0;
+  tc::bar_wait(&bar, phase);
+  phase ^= 1;
 
   // ---- 1. causal conv of q and k, clamped log-decay, half-local cumsum ------
   {
-    const float4 wq = load4(conv_w + (0 * HD + chan) * 4);
-    const float4 wk = load4(conv_w + (1 * HD + chan) * 4);
     const int r0 = 32 * half;
     float hq[3], hk[3];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
-      const int64_t p = t0 + r0 - 3 + j;  // absolute token index of the halo row
-      float a = 0.f, b = 0.f;
-      if (r0 - 3 + j < L) {
-        if (p >= seg0) {
-          a = to_f(q[p * HD + chan]);
-          b = to_f(k[p * HD + chan]);
-        } else if (init_conv) {
+      const int64_t p = t0 + r0 - 3 + j;  // absolute token of the halo row (tile row r0 + j)
+      float a = to_f(rq_t[(r0 + j) * D + ch]), b = to_f(rk_t[(r0 + j) * D + ch]);
+      if (p < seg0) {  // before the segment: conv history (or zeros)
+        a = b = 0.f;
+        if (init_conv) {
           const int slot = (int)(3 + (p - seg0));
           a = to_f(init_conv[((int64_t)n * 9 + 0 * 3 + slot) * HD + chan]);
           b = to_f(init_conv[((int64_t)n * 9 + 1 * 3 + slot) * HD + chan]);
@@ -131,26 +150,22 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
       hq[j] = a; hk[j] = b;
     }
     float cum = 0.f;
-#pragma unroll 4
+#pragma unroll 8
     for (int r = 0; r < 32; ++r) {
       const int t = r0 + r;
-      float yq = 0.f, yk = 0.f, gl = 0.f;
-      if (t < L) {
-        const int64_t row = (t0 + t) * HD + chan;
-        const float xq = to_f(q[row]), xk = to_f(k[row]);
-        gl = fmaxf(to_f(g[row]), LOG_DECAY_FLOOR);
-        yq = conv4(wq, hq[0], hq[1], hq[2], xq);
-        yk = conv4(wk, hk[0], hk[1], hk[2], xk);
-        if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
-        hq[0] = hq[1]; hq[1] = hq[2]; hq[2] = xq;
-        hk[0] = hk[1]; hk[1] = hk[2]; hk[2] = xk;
-      }
+      const float xq = to_f(rq_t[(t + 3) * D + ch]), xk = to_f(rk_t[(t + 3) * D + ch]);
+      float yq = conv4(wq, hq[0], hq[1], hq[2], xq);
+      float yk = conv4(wk, hk[0], hk[1], hk[2], xk);
+      if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
+      hq[0] = hq[1]; hq[1] = hq[2]; hq[2] = xq;
+      hk[0] = hk[1]; hk[1] = hk[2]; hk[2] = xk;
+      const bool valid = t < L;
+      const float gl = valid ? fmaxf(to_f(rg_t[(t + 3) * D + ch]), LOG_DECAY_FLOOR) : 0.f;
       cum += gl;
-      Yq[t * D + ch] = yq;
-      Yk[t * D + ch] = yk;
+      Yq[t * D + ch] = valid ? yq : 0.f;
+      Yk[t * D + ch] = valid ? yk : 0.f;
       E1[t * D + ch] = cum;
     }
-    if (tid < CH) ms[MS_BETA + tid] = tid < L ? to_f(beta[(t0 + tid) * H + h]) : 0.f;
   }
   __syncthreads();
 
@@ -234,7 +249,6 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 
   // ---- 5. gated Gram blocks on the tensor core, 4 slabs of 32 channels -------
   const uint32_t tm = tmem_base;
-  uint32_t phase = 0;
   for (int kp = 0; kp < 4; ++kp) {
     // A_I: 4 x 64 rows x 32 channels (8192 elements), B_I: 4 x 32 rows x 32 (4096)
     for (int e = tid; e < 4 * 64 * 32; e += 256) {
@@ -258,12 +272,13 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     __syncthreads();
     if (tid == 0) {
       tc::fence_after();
+      const uint64_t da = tc::desc(tc::smem_u32(opA)), db = tc::desc(tc::smem_u32(opB));
 #pragma unroll
       for (int I = 0; I < 4; ++I)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          tc::mma_ss(tm + 32 * I, tc::desc_k(tc::smem_u32(opA + I * 8192), 64, ks),
-                     tc::desc_k(tc::smem_u32(opB + I * 4096), 32, ks), tc::idesc_tf32(64, 32),
+          tc::mma_ss(tm + 32 * I, da + ((I * 8192) >> 4) + tc::desc_step(64, ks),
+                     db + ((I * 4096) >> 4) + tc::desc_step(32, ks), tc::idesc_tf32(64, 32),
                      (kp > 0 || ks > 0) ? 1 : 0);
       tc::commit(&bar);
     }
@@ -367,10 +382,11 @@ chunk_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
   __syncthreads();
   if (tid == 0) {
     tc::fence_after();
+    const uint64_t dt = tc::desc(tc::smem_u32(tT)), dk = tc::desc(tc::smem_u32(tK));
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks)
-      tc::mma_ss(tm + 128, tc::desc_k(tc::smem_u32(tT), 64, ks), tc::desc_k(tc::smem_u32(tK), 128, ks),
-                 tc::idesc_tf32(64, 128), ks > 0 ? 1 : 0);
+      tc::mma_ss(tm + 128, dt + tc::desc_step(64, ks), dk + tc::desc_step(128, ks), tc::idesc_tf32(64, 128),
+                 ks > 0 ? 1 : 0);
     tc::commit(&bar);
   }
   tc::bar_wait(&bar, phase);

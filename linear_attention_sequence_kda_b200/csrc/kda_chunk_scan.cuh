@@ -5,7 +5,8 @@
 // state is handed from chunk to chunk).
 //
 // Thread v (of 128) owns value column v: TMEM lane v holds row v of
-//   V^T (cols 0..63) | S^T (cols 64..191) | U^T (192..255) | O^T (256..319).
+//   V^T (cols 0..63) | S^T (cols 64..191) | U^T (192..255) | O^T (256..319)
+// (tf32 MMA operands) and, in fp32, V^T (320..383) and U^T (384..447).
 // Per chunk, with the record written by chunk_prep_kernel:
 //   MMA1  U^T = [V^T | S^T] [T_s | -W]^T        (K = 64 + 128)
 //         O^T = S^T Q~^T                          (K = 128)
@@ -13,6 +14,10 @@
 //   MMA2  O^T += U^T P_s^T;   S^T += U^T K-bar    (K = 64, A = U^T from TMEM)
 //   fp32  o = O + P_tt u (diagonal of P), written to HBM.
 // A operands are read from TMEM as tf32; the state itself stays fp32.
+//
+// Data movement: the raw value tile of chunk i+2 (TMA, 64 rows x 256 B) and the
+// record halves of chunk i+1 (bulk copies) are in flight while chunk i runs;
+// each record half is refilled as soon as the MMA group that reads it is done.
 #pragma once
 #include "kda_chunk_prep.cuh"
 #include "kda_common.cuh"
@@ -20,22 +25,25 @@
 
 namespace kda {
 
-constexpr uint32_t SCAN_A0 = 0;                      // stage A buffer 0: B1 | QT (81920 B)
-constexpr uint32_t SCAN_A1 = REC_TILES_A;            // stage A buffer 1
-constexpr uint32_t SCAN_B = 2 * REC_TILES_A;         // stage B: PS | KB | SC (50176 B)
-constexpr uint32_t SCAN_SMEM = 2 * REC_TILES_A + REC_TILES_B + 1024;
+constexpr uint32_t VT_BYTES = CH * D * 2;            // raw value tile (bf16)
+constexpr uint32_t SCAN_A = 0;                       // record part A: B1 | QT (81920 B)
+constexpr uint32_t SCAN_B = REC_TILES_A;             // record part B: PS | KB | SC (50176 B)
+constexpr uint32_t SCAN_V0 = REC_TILES_A + REC_TILES_B;
+constexpr uint32_t SCAN_V1 = SCAN_V0 + VT_BYTES;
+constexpr uint32_t SCAN_SMEM = SCAN_V1 + VT_BYTES + 1024;
 constexpr int TM_V = 0, TM_S = 64, TM_U = 192, TM_O = 256;
+constexpr int TM_VX = 320, TM_UX = 384;  // exact fp32 V and U for the diagonal terms
 
 template <typename Tout, int ACT>
 __global__ void __launch_bounds__(128, 1)
-chunk_scan_kernel(const __nv_bfloat16* __restrict__ v, const float* __restrict__ conv_w,
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ conv_w,
                   const float* init_state, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
                   Tout* __restrict__ o, float* final_state) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t bar_a[2], bar_b, bar_m1, bar_m2;
+  __shared__ uint64_t bar_a, bar_b, bar_v[2], bar_m1, bar_m2;
   __shared__ uint32_t tmem_base;
   __shared__ float sc[256];  // this chunk's beta[64], P_tt[64], e^{Gamma_C}[128]
 
@@ -50,7 +58,8 @@ chunk_scan_kernel(const __nv_bfloat16* __restrict__ v, const float* __restrict__
 
   if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
   if (tid == 0) {
-    tc::bar_init(&bar_a[0], 1); tc::bar_init(&bar_a[1], 1); tc::bar_init(&bar_b, 1);
+    tc::bar_init(&bar_a, 1); tc::bar_init(&bar_b, 1);
+    tc::bar_init(&bar_v[0], 1); tc::bar_init(&bar_v[1], 1);
     tc::bar_init(&bar_m1, 1); tc::bar_init(&bar_m2, 1);
     tc::bar_init_fence();
   }
@@ -78,108 +87,118 @@ chunk_scan_kernel(const __nv_bfloat16* __restrict__ v, const float* __restrict__
     hv0 = to_f(c[0]); hv1 = to_f(c[HD]); hv2 = to_f(c[2 * HD]);
   }
 
-  // issued / waited counts per barrier (uniform across the block), so the exit
-  // path can wait for any copy or MMA still in flight before freeing TMEM
-  int a_iss[2] = {0, 0}, b_iss = 0, m1 = 0, m2 = 0;
+  // issued counts per barrier (uniform across the block) for the exit drain
+  int a_iss = 0, b_iss = 0, v_iss[2] = {0, 0}, m2 = 0;
   auto load_a = [&](int i) {
-    const uint8_t* r = rec0 + (int64_t)i * rec_stride;
-    uint8_t* dst = sm + ((i & 1) ? SCAN_A1 : SCAN_A0);
-    tc::bar_expect_tx(&bar_a[i & 1], REC_TILES_A);
-    tc::bulk_g2s(dst, r, REC_TILES_A, &bar_a[i & 1]);
+    tc::bar_expect_tx(&bar_a, REC_TILES_A);
+    tc::bulk_g2s(sm + SCAN_A, rec0 + (int64_t)i * rec_stride, REC_TILES_A, &bar_a);
   };
   auto load_b = [&](int i) {
-    const uint8_t* r = rec0 + (int64_t)i * rec_stride + REC_PS;
     tc::bar_expect_tx(&bar_b, REC_TILES_B);
-    tc::bulk_g2s(sm + SCAN_B, r, REC_TILES_B, &bar_b);
+    tc::bulk_g2s(sm + SCAN_B, rec0 + (int64_t)i * rec_stride + REC_PS, REC_TILES_B, &bar_b);
+  };
+  auto load_v = [&](int i) {
+    tc::bar_expect_tx(&bar_v[i & 1], VT_BYTES);
+    tc::tma_load_2d(sm + ((i & 1) ? SCAN_V1 : SCAN_V0), &tm_v, h * D, (int)(seg0 + (int64_t)CH * i),
+                    &bar_v[i & 1]);
   };
   if (nchunks > 0) {
     if (tid == 0) {
       load_a(0);
-      if (nchunks > 1) load_a(1);
       load_b(0);
+      load_v(0);
+      if (nchunks > 1) load_v(1);
     }
-    a_iss[0] = 1; a_iss[1] = nchunks > 1; b_iss = 1;
+    a_iss = b_iss = 1; v_iss[0] = 1; v_iss[1] = nchunks > 1;
   }
+  const uint64_t d_b1 = tc::desc(tc::smem_u32(sm + SCAN_A));
+  const uint64_t d_qt = tc::desc(tc::smem_u32(sm + SCAN_A + REC_QT));
+  const uint64_t d_ps = tc::desc(tc::smem_u32(sm + SCAN_B));
+  const uint64_t d_kb = tc::desc(tc::smem_u32(sm + SCAN_B + (REC_KB - REC_PS)));
 
   bool ok = true;
   for (int i = 0; i < nchunks && ok; ++i) {
     const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
     const int64_t t0 = seg0 + (int64_t)CH * i;
-    uint8_t* sa = sm + ((i & 1) ? SCAN_A1 : SCAN_A0);
-    uint8_t* sb = sm + SCAN_B;
 
-    // (a) causal conv of v for this chunk; V^T row into TMEM (tf32)
-    float vv[CH];
+    // (a) causal conv of v for this chunk; V^T row into TMEM (tf32 and fp32)
+    ok &= tc::bar_wait(&bar_v[i & 1], (i >> 1) & 1);
+    {
+      const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + ((i & 1) ? SCAN_V1 : SCAN_V0));
 #pragma unroll
-    for (int t = 0; t < CH; ++t) {
-      float y = 0.f;
-      if (t < L) {
-        const float x = to_f(v[(t0 + t) * HD + chan]);
-        y = conv4(wv, hv0, hv1, hv2, x);
-        if (ACT == KDA_CONV_SILU) y = silu(y);
-        hv0 = hv1; hv1 = hv2; hv2 = x;
+      for (int g16 = 0; g16 < 4; ++g16) {
+        float vv[16], r[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = 16 * g16 + j;
+          const float x = to_f(vt[t * D + tid]);
+          float y = conv4(wv, hv0, hv1, hv2, x);
+          if (ACT == KDA_CONV_SILU) y = silu(y);
+          hv0 = hv1; hv1 = hv2; hv2 = x;
+          vv[j] = t < L ? y : 0.f;
+          r[j] = tc::to_tf32(vv[j]);
+        }
+        tc::st16(lane_base + TM_V + 16 * g16, r);
+        tc::st16(lane_base + TM_VX + 16 * g16, vv);
       }
-      vv[t] = y;
-    }
-#pragma unroll
-    for (int g16 = 0; g16 < 4; ++g16) {
-      float r[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) r[j] = tc::to_tf32(vv[16 * g16 + j]);
-      tc::st16(lane_base + TM_V + 16 * g16, r);
     }
     tc::st_wait();
-    // (b) this chunk's tiles
-    ok &= tc::bar_wait(&bar_a[i & 1], (i >> 1) & 1);
+    // (b) this chunk's record
+    ok &= tc::bar_wait(&bar_a, i & 1);
     ok &= tc::bar_wait(&bar_b, i & 1);
-    sc[tid] = reinterpret_cast<const float*>(sb + (REC_SC - REC_PS))[tid];
-    sc[tid + 128] = reinterpret_cast<const float*>(sb + (REC_SC - REC_PS))[tid + 128];
+    sc[tid] = reinterpret_cast<const float*>(sm + SCAN_B + (REC_SC - REC_PS))[tid];
+    sc[tid + 128] = reinterpret_cast<const float*>(sm + SCAN_B + (REC_SC - REC_PS))[tid + 128];
     tc::fence_before();
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    // (c) MMA group 1
+    // (c) MMA group 1; the value tile buffer is free again
     if (tid == 0) {
       tc::fence_after();
-      const uint32_t b1 = tc::smem_u32(sa), qt = tc::smem_u32(sa + REC_QT);
 #pragma unroll
       for (int ks = 0; ks < 24; ++ks)
-        tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, tc::desc_k(b1, 64, ks), tc::idesc_tf32(128, 64), ks > 0);
+        tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, d_b1 + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), ks > 0);
 #pragma unroll
       for (int ks = 0; ks < 16; ++ks)
-        tc::mma_ts(tm + TM_O, tm + TM_S + 8 * ks, tc::desc_k(qt, 64, ks), tc::idesc_tf32(128, 64), ks > 0);
+        tc::mma_ts(tm + TM_O, tm + TM_S + 8 * ks, d_qt + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), ks > 0);
       tc::commit(&bar_m1);
+      if (i + 2 < nchunks) load_v(i + 2);
     }
-    ++m1;
+    if (i + 2 < nchunks) v_iss[i & 1]++;
     ok &= tc::bar_wait(&bar_m1, i & 1);
     tc::fence_after();
     if (!__syncthreads_and(ok)) { ok = false; break; }
-    if (i + 2 < nchunks) {  // stage A buffer is free again
-      if (tid == 0) load_a(i + 2);
-      a_iss[i & 1]++;
+    if (i + 1 < nchunks) {  // record part A is free again
+      if (tid == 0) load_a(i + 1);
+      a_iss++;
     }
     // (d) U += beta V (exact diagonal of T V), S^T <- S^T diag(gamma)
-    float uu[CH];
 #pragma unroll
     for (int g16 = 0; g16 < 4; ++g16) {
-      float r[16];
+      float r[16], vx[16], ux[16];
       tc::ld16(lane_base + TM_U + 16 * g16, r);
+      tc::ld16(lane_base + TM_VX + 16 * g16, vx);
       tc::ld_wait();
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int t = 16 * g16 + j;
-        uu[t] = fmaf(sc[t], vv[t], r[j]);
-        r[j] = tc::to_tf32(uu[t]);
+        ux[j] = fmaf(sc[16 * g16 + j], vx[j], r[j]);
+        r[j] = tc::to_tf32(ux[j]);
       }
       tc::st16(lane_base + TM_U + 16 * g16, r);
+      tc::st16(lane_base + TM_UX + 16 * g16, ux);
     }
 #pragma unroll
-    for (int g16 = 0; g16 < 8; ++g16) {
-      float r[16];
-      tc::ld16(lane_base + TM_S + 16 * g16, r);
+    for (int g16 = 0; g16 < 8; g16 += 2) {
+      float r0[16], r1[16];
+      tc::ld16(lane_base + TM_S + 16 * g16, r0);
+      tc::ld16(lane_base + TM_S + 16 * g16 + 16, r1);
       tc::ld_wait();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) r[j] *= sc[128 + 16 * g16 + j];
-      tc::st16(lane_base + TM_S + 16 * g16, r);
+      for (int j = 0; j < 16; ++j) {
+        r0[j] *= sc[128 + 16 * g16 + j];
+        r1[j] *= sc[128 + 16 * g16 + 16 + j];
+      }
+      tc::st16(lane_base + TM_S + 16 * g16, r0);
+      tc::st16(lane_base + TM_S + 16 * g16 + 16, r1);
     }
     tc::st_wait();
     tc::fence_before();
@@ -187,34 +206,33 @@ chunk_scan_kernel(const __nv_bfloat16* __restrict__ v, const float* __restrict__
     // (e) MMA group 2
     if (tid == 0) {
       tc::fence_after();
-      const uint32_t ps = tc::smem_u32(sb), kb = tc::smem_u32(sb + (REC_KB - REC_PS));
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        tc::mma_ts(tm + TM_O, tm + TM_U + 8 * ks, tc::desc_k(ps, 64, ks), tc::idesc_tf32(128, 64), 1);
+        tc::mma_ts(tm + TM_O, tm + TM_U + 8 * ks, d_ps + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, tc::desc_k(kb, 128, ks), tc::idesc_tf32(128, 128), 1);
+        tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, d_kb + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), 1);
       tc::commit(&bar_m2);
     }
     ++m2;
     ok &= tc::bar_wait(&bar_m2, i & 1);
     tc::fence_after();
     if (!__syncthreads_and(ok)) { ok = false; break; }
-    if (i + 1 < nchunks) {  // stage B is free again
+    if (i + 1 < nchunks) {  // record part B is free again
       if (tid == 0) load_b(i + 1);
       b_iss++;
     }
     // (f) o = O + P_tt u
 #pragma unroll
     for (int g16 = 0; g16 < 4; ++g16) {
-      float r[16];
+      float r[16], ux[16];
       tc::ld16(lane_base + TM_O + 16 * g16, r);
+      tc::ld16(lane_base + TM_UX + 16 * g16, ux);
       tc::ld_wait();
+      Tout* orow = o + (t0 + 16 * g16) * HD + chan;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int t = 16 * g16 + j;
-        if (t < L) o[(t0 + t) * HD + chan] = from_f<Tout>(fmaf(sc[64 + t], uu[t], r[j]));
-      }
+      for (int j = 0; j < 16; ++j)
+        if (16 * g16 + j < L) orow[j * HD] = from_f<Tout>(fmaf(sc[64 + 16 * g16 + j], ux[j], r[j]));
     }
     tc::fence_before();
     __syncthreads();  // sc and TMEM O are rewritten by the next chunk
@@ -223,14 +241,14 @@ chunk_scan_kernel(const __nv_bfloat16* __restrict__ v, const float* __restrict__
 
   if (!ok) {
     // a wait gave up (status already recorded): drain what is still in flight
-    // (each bounded) so that TMEM and shared memory are idle before exit
+    // (each wait bounded; waiting on the parity of a completed phase returns at
+    // once) so that TMEM and shared memory are idle before exit
     if (tid == 0) tc::commit(&bar_m2);
     tc::bar_wait(&bar_m2, m2 & 1);
-    // waiting on the parity of the last issued phase returns at once if it
-    // already completed
-    for (int b = 0; b < 2; ++b)
-      if (a_iss[b] > 0) tc::bar_wait(&bar_a[b], (a_iss[b] - 1) & 1);
+    if (a_iss > 0) tc::bar_wait(&bar_a, (a_iss - 1) & 1);
     if (b_iss > 0) tc::bar_wait(&bar_b, (b_iss - 1) & 1);
+    for (int b = 0; b < 2; ++b)
+      if (v_iss[b] > 0) tc::bar_wait(&bar_v[b], (v_iss[b] - 1) & 1);
   }
   // final state: column v of S = row v of S^T
   if (ok) {

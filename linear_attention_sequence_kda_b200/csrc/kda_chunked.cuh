@@ -11,6 +11,7 @@
 #include "kda_chunk_prep.cuh"
 #include "kda_chunk_scan.cuh"
 #include "kda_common.cuh"
+#include "kda_tmap.cuh"
 
 namespace kda {
 
@@ -63,29 +64,34 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   const int32_t* d_order = d_base + (N + 1);
   uint8_t* records = ws + hdr;
 
+  // TMA descriptors over the packed [total_T, H*128] inputs: 67-row boxes
+  // (3 halo rows + one chunk) for q, k, g; 64-row boxes for v
+  const uint64_t rows = (uint64_t)cu_host[N], cols = (uint64_t)H * D;
+  CUtensorMap tq, tk, tg, tv;
+  if (!make_tmap_bf16_2d(&tq, q, rows, cols, RAW_ROWS, D) || !make_tmap_bf16_2d(&tk, k, rows, cols, RAW_ROWS, D) ||
+      !make_tmap_bf16_2d(&tg, g, rows, cols, RAW_ROWS, D) || !make_tmap_bf16_2d(&tv, v, rows, cols, CH, D))
+    return KDA_ERR_CUDA;
+
   if (total > 0) {
     auto prep = chunk_prep_kernel<ACT>;
     if (cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess)
       return KDA_ERR_CUDA;
-    prep<<<dim3((unsigned)total, H), 256, PREP_SMEM, stream>>>(
-        (const T*)q, (const T*)k, (const T*)g, (const T*)beta, conv_w, (const T*)init_conv, cu_dev,
-        d_tab, H, records);
+    prep<<<dim3((unsigned)total, H), 256, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w,
+                                                               (const T*)init_conv, cu_dev, d_tab, H, records);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
   }
   if (o_dt == KDA_F32) {
     auto scan = chunk_scan_kernel<float, ACT>;
     if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
       return KDA_ERR_CUDA;
-    scan<<<(unsigned)N * H, 128, SCAN_SMEM, stream>>>((const T*)v, conv_w, init_state, (const T*)init_conv,
-                                                      cu_dev, d_base, d_order, H, records, (float*)o,
-                                                      final_state);
+    scan<<<(unsigned)N * H, 128, SCAN_SMEM, stream>>>(tv, conv_w, init_state, (const T*)init_conv, cu_dev,
+                                                      d_base, d_order, H, records, (float*)o, final_state);
   } else {
     auto scan = chunk_scan_kernel<T, ACT>;
     if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
       return KDA_ERR_CUDA;
-    scan<<<(unsigned)N * H, 128, SCAN_SMEM, stream>>>((const T*)v, conv_w, init_state, (const T*)init_conv,
-                                                      cu_dev, d_base, d_order, H, records, (T*)o,
-                                                      final_state);
+    scan<<<(unsigned)N * H, 128, SCAN_SMEM, stream>>>(tv, conv_w, init_state, (const T*)init_conv, cu_dev,
+                                                      d_base, d_order, H, records, (T*)o, final_state);
   }
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

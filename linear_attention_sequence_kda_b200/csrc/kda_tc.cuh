@@ -10,6 +10,7 @@
 // hardware applies that XOR on address bits [4,7) ^ [7,10), so a descriptor
 // may start at slab base + 32 * kstep bytes for the kstep-th 8-column step.
 #pragma once
+#include <cuda.h>
 #include <stdint.h>
 
 #include "kda_common.cuh"
@@ -38,6 +39,12 @@ __device__ __forceinline__ uint64_t desc(uint32_t saddr) {
 // descriptor of k-step `ks` (8 columns) of a tile with R rows at `base`
 __device__ __forceinline__ uint64_t desc_k(uint32_t base, int R, int ks) {
   return desc(base + (uint32_t)((ks >> 2) * R * 128 + (ks & 3) * 32));
+}
+// the same as a constant added to desc(base): k-step ks of an R-row tile
+// starts (ks / 4) slabs and (ks % 4) * 32 bytes further (address field is in
+// 16-byte units and never overflows for shared-memory addresses)
+__host__ __device__ constexpr uint64_t desc_step(int R, int ks) {
+  return (uint64_t)(((ks >> 2) * R * 128 + (ks & 3) * 32) >> 4);
 }
 
 // instruction descriptor, kind::tf32, fp32 accumulate, both operands K-major
@@ -137,6 +144,18 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
   }
   set_status(KDA_ERR_TIMEOUT);
   return false;
+}
+
+// 2D tiled tensor copy global -> shared through a tensor map (TMA); (x, y) =
+// (inner column, row) of the box origin, x * element size a multiple of 16 B.
+// Rows outside the tensor (including negative y) are filled with zeros.
+__device__ __forceinline__ void tma_load_2d(void* dst_smem, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // bulk async copy global -> shared, completion signalled on `bar` (tx bytes)
