@@ -10,6 +10,15 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # (re)build libkda.so and the oracle before any test module imports them
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_kda_build", os.path.join(ROOT, "linear_attention_sequence_kda_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import oracle
+    oracle.build()
 
 
 def pytest_collection_modifyitems(config, items):
