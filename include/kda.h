@@ -136,6 +136,39 @@ kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const 
                            const float* conv_w, int num_seqs, int num_heads, kda_dtype dt,
                            kda_conv_act act, kda_dtype o_dt, void* o, void* stream);
 
+/*
+ * kda_prefill_noalloc -- kda_prefill for callers that cannot allocate device
+ * memory.  (Not an operation of the method: the pages have no counterpart; it
+ * only changes where the scratch lives.)
+ *
+ * Some callers cannot call cudaMalloc or hand the library a workspace: an
+ * inference server that has carved all device memory into its own pools
+ * before serving starts, or a plugin whose host application owns every device
+ * allocation.  This entry point takes the same arguments as kda_prefill
+ * without the workspace and allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library call).  Its scratch is one static device array of
+ * KDA_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads it,
+ * until the process exits.
+ *   - Problems whose kda_prefill_workspace_size() exceeds
+ *     KDA_NOALLOC_SCRATCH_BYTES are rejected with KDA_ERR_WORKSPACE before any
+ *     launch (about 1000 chunk-heads: (sum over segments of ceil(T_n / 64))
+ *     x num_heads <= 1000 fits).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (every byte a call reads is written earlier in that same call, so
+ *     nothing needs clearing).  Calls whose work overlaps on the GPU (other
+ *     streams, other host threads) race on it: serialise them.
+ *   - fp32 inputs use the recurrent path, which needs no scratch.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)128 << 20)
+kda_status kda_prefill_noalloc(const void* q, const void* k, const void* v, const void* g,
+                               const void* beta, const float* conv_w, const float* init_state,
+                               const void* init_conv, const int32_t* cu_seqlens_dev,
+                               const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                               kda_dtype dt, kda_conv_act act, kda_dtype o_dt, void* o,
+                               float* final_state, void* conv_tail, void* stream);
+
 /* Static description of a status code (never NULL). */
 const char* kda_status_string(kda_status s);
 

@@ -26,11 +26,12 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 
 # every entry point declared in include/kda.h
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
-           "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version")
+           "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version",
+           "kda_prefill_noalloc")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m "
-                      "linear_attention_sequence_kda_b200.build` (nvcc, sm_100a)")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python "
+                      "linear_attention_sequence_kda_b200/build.py` (nvcc, sm_100a)")
 
 _vp, _i32p, _f32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
 lib = ctypes.CDLL(LIB_PATH)
@@ -43,6 +44,9 @@ lib.kda_prefill.restype = ctypes.c_int
 lib.kda_prefill.argtypes = _PREFILL_ARGS + [_vp, ctypes.c_size_t, _vp]
 lib.kda_prefill_recurrent.restype = ctypes.c_int
 lib.kda_prefill_recurrent.argtypes = _PREFILL_ARGS + [_vp]
+lib.kda_prefill_noalloc.restype = ctypes.c_int
+lib.kda_prefill_noalloc.argtypes = _PREFILL_ARGS + [_vp]
+NOALLOC_SCRATCH_BYTES = 128 << 20  # KDA_NOALLOC_SCRATCH_BYTES
 lib.kda_decode_step.restype = ctypes.c_int
 lib.kda_decode_step.argtypes = [_f32p, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
                                 ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp]
@@ -122,6 +126,30 @@ def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
         _check(lib.kda_prefill(*args, _ptr(workspace), wbytes, _stream(stream)), "kda_prefill")
+    return o, final_state, conv_tail
+
+
+def prefill_noalloc(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init_state=None,
+                    init_conv=None, act: int = KDA_CONV_NONE, o=None, final_state=None, conv_tail=None,
+                    stream=None, o_dtype=torch.float32):
+    """kda_prefill_noalloc: like prefill() but the library uses its own static
+    device scratch instead of a workspace.  Returns (o, final_state, conv_tail)."""
+    cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
+    N = len(cu_h) - 1
+    H = q.shape[1]
+    dev = q.device
+    if cu_seqlens_dev is None:
+        cu_seqlens_dev = torch.from_numpy(cu_h).to(dev)
+    if o is None:
+        o = torch.empty(q.shape, dtype=o_dtype, device=dev)
+    if final_state is None:
+        final_state = torch.empty((N, H, HEAD_DIM, HEAD_DIM), dtype=torch.float32, device=dev)
+    if conv_tail is None:
+        conv_tail = torch.empty((N, 3, 3, H * HEAD_DIM), dtype=q.dtype, device=dev)
+    _check(lib.kda_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(conv_w),
+                                   _ptr(init_state), _ptr(init_conv), _ptr(cu_seqlens_dev), _ptr(cu_h), N, H,
+                                   _dtype_code(q), int(act), _dtype_code(o), _ptr(o), _ptr(final_state),
+                                   _ptr(conv_tail), _stream(stream)), "kda_prefill_noalloc")
     return o, final_state, conv_tail
 
 

@@ -2,6 +2,8 @@
 // validation, then asynchronous launches on the caller's stream.
 #include <stdio.h>
 
+#include <mutex>
+
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
 #include "kda_recurrent.cuh"
@@ -228,3 +230,59 @@ kda_status kda_check_async_status(void* stream) {
 int kda_version(void) { return (1 << 16) | 0; }
 
 }  // extern "C"
+
+// ---- prefill for callers that cannot allocate device memory ------------------
+// The chunked path's scratch (chunk table + one operand record per chunk and
+// head) lives in this file-scope device array instead of a caller workspace.
+// In host code the name below is only a stand-in for the symbol; the device
+// address is obtained with cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char kda_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// device address of kda_noalloc_scratch on the current device (looked up on
+// the first call for that device, with that device current)
+kda_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, kda_noalloc_scratch) != cudaSuccess || !p) return KDA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return KDA_OK;
+}
+}  // namespace
+
+extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const void* v, const void* g,
+                                          const void* beta, const float* conv_w,
+                                          const float* init_state, const void* init_conv,
+                                          const int32_t* cu_seqlens_dev,
+                                          const int32_t* cu_seqlens_host, int num_seqs,
+                                          int num_heads, kda_dtype dt, kda_conv_act act,
+                                          kda_dtype o_dt, void* o, float* final_state,
+                                          void* conv_tail, void* stream) {
+  PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, o, final_state, conv_tail,
+                (cudaStream_t)stream, 0, 0};
+  kda_status st = validate_prefill(a);
+  if (st != KDA_OK) return st;
+  if (a.N == 0) return KDA_OK;
+  if (dt == KDA_F32) return run_recurrent(a);  // the fp32 path uses no scratch
+  const size_t need = chunked_workspace_bytes(a.N, a.H, a.total_T);
+  if (need > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != KDA_OK) return st;
+  st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
+                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.o, a.final_state, scratch, need,
+                      a.max_len, a.stream);
+  if (st != KDA_OK) return st;
+  return launch_tail<__nv_bfloat16>(a);
+}
