@@ -31,6 +31,12 @@
 // computes, per block row I, D_I[j][i'] = sum_c A_I[j][c] B_I[i'][c] with
 // A_I[j] = k_j e^{G_{m_I} - G_j} (j in blocks <= I, 0 elsewhere) and
 // B_I = [k_i; q_i] e^{G_i - G_{m_I}} for the 16 i of block I.
+//
+// Block of 512 threads; thread (c, b) owns key/query channel c of token block
+// b (rows 16b..16b+15), so each block's midpoint factors stay in one thread.
+// The B operands of all four block rows are one tile written once (KQX); the
+// A operands are built per 32-channel slab into two alternating buffers while
+// the previous slab's MMAs run.
 #pragma once
 #include "kda_common.cuh"
 #include "kda_tc.cuh"
@@ -47,26 +53,24 @@ constexpr uint32_t REC_BYTES = 132096;
 constexpr uint32_t REC_TILES_A = REC_PS;              // B1 + QT: consumed by the first MMA group
 constexpr uint32_t REC_TILES_B = REC_BYTES - REC_PS;  // PS + KB + SC: second MMA group + scalars
 
-// shared memory plan of the prep kernel (bytes from a 1024-aligned base)
-constexpr uint32_t PREP_YQ = 0;          // [64][128] f32: conv(q) -> q_hat
-constexpr uint32_t PREP_YK = 32768;      // [64][128] f32: conv(k) -> k_hat
-constexpr uint32_t PREP_E1 = 65536;      // [64][128] f32: Gamma -> e^{G_mid(J) - G_t}
-constexpr uint32_t PREP_XF = 98304;      // [64][128] f32: e^{G_t - G_mid(J)}
-constexpr uint32_t PREP_OPA = 131072;    // 4 x 8 KB Gram A (one 32-channel slab); later T tile
-constexpr uint32_t PREP_OPB = 163840;    // 4 x 4 KB Gram B; (OPA+16K .. OPB+16K) later K~^T tile
-constexpr uint32_t PREP_M = 180224;      // [64][64] f32: diag(beta) M strict -> X
-constexpr uint32_t PREP_P = 196608;      // [64][64] f32: P strict
-constexpr uint32_t PREP_MISC = 212992;   // scalars and solve temporaries (8 KB)
-constexpr uint32_t PREP_SMEM = 221184 + 1024;  // + alignment slack
+// shared memory plan (bytes from a 1024-aligned base); regions are reused
+// phase by phase
+constexpr int PREP_THREADS = 512;
+constexpr uint32_t P_RAW = 0;        // step 0-1: raw q, k, g tiles (3 x RAW_BYTES)
+                                     // step 5: Gram A operands, 2 buffers x 32 KB
+                                     // step 7: solve temporaries; step 8: T tile (16 KB) + K~^T tile (32 KB)
+constexpr uint32_t P_KQX = 65536;    // steps 1-3: conv(q), conv(k) row-major fp32 (2 x 32 KB)
+                                     // steps 3-8: KQX tile [128 rows x 128] (rows 32I..32I+15: k e^{G-G_m(I)},
+                                     //            rows 32I+16..32I+31: q e^{G-G_m(I)} of block I)
+constexpr uint32_t P_G = 131072;     // steps 1-3: Gamma row-major; steps 3-5: KE = k e^{G_m - G} row-major
+                                     // steps 6-8: diag(beta) M strict -> X (16 KB), P strict (16 KB)
+constexpr uint32_t P_MISC = 163840;  // scalars (12 KB)
+constexpr uint32_t PREP_SMEM = 176128 + 1024;
 
-// misc region layout (floats; 2048 floats = 8 KB)
-constexpr int MS_BETA = 0, MS_RQ = 64, MS_RK = 128, MS_PD = 192, MS_Z = 256 /*6x128*/,
-              MS_EGM = 1024 /*4x128*/, MS_EGC = 1536 /*4x128*/;
-// short-lived temporaries placed in regions that are idle at the time:
-// block-midpoint Gammas in the Gram A region (steps 3-3b, before the Gram),
-// solve temporaries in the Gram B region (step 7, after the Gram)
-constexpr int GT_GMID = 0 /*4x128*/, GT_GC = 512 /*128*/;
-constexpr int SV_XD = 0 /*4x16x16*/, SV_YB = 1024 /*3x16x16*/;
+// misc region (floats)
+constexpr int MS_BETA = 0, MS_RQ = 64, MS_RK = 128, MS_PD = 192, MS_GMID = 256 /*4x128*/,
+              MS_GC = 768 /*128*/, MS_Z = 896 /*6x128*/, MS_EGM = 1664 /*4x128*/, MS_CARRY = 2176 /*4x128*/;
+// ends at 2688 floats (10752 B) < 12 KB
 
 __device__ __forceinline__ int zidx(int I, int J) { return (I * (I - 1)) / 2 + J; }  // J < I
 
@@ -75,7 +79,7 @@ constexpr int RAW_ROWS = CH + 3;
 constexpr uint32_t RAW_BYTES = RAW_ROWS * D * 2;  // 17152
 
 template <int ACT>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(PREP_THREADS, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16* __restrict__ beta,
                   const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ init_conv,
@@ -83,22 +87,18 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   uint8_t* __restrict__ records) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  float* Yq = (float*)(sm + PREP_YQ);
-  float* Yk = (float*)(sm + PREP_YK);
-  float* E1 = (float*)(sm + PREP_E1);
-  float* Xf = (float*)(sm + PREP_XF);
-  uint8_t* opA = sm + PREP_OPA;
-  uint8_t* opB = sm + PREP_OPB;
-  float* Ms = (float*)(sm + PREP_M);
-  float* Ps = (float*)(sm + PREP_P);
-  float* ms = (float*)(sm + PREP_MISC);
-  float* gt = (float*)(sm + PREP_OPA);  // steps 3-3b only
-  float* sv = (float*)(sm + PREP_OPB);  // step 7 only
-  __shared__ uint64_t bar;
+  float* Yq = (float*)(sm + P_KQX);
+  float* Yk = (float*)(sm + P_KQX + 32768);
+  uint8_t* kqx = sm + P_KQX;
+  float* Gm = (float*)(sm + P_G);  // Gamma, then KE
+  float* Ms = (float*)(sm + P_G);
+  float* Ps = (float*)(sm + P_G + 16384);
+  float* ms = (float*)(sm + P_MISC);
+  __shared__ uint64_t bar_ld, bar_g[2], bar_w;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ch = tid & 127, half = tid >> 7;
+  const int ch = tid & 127, blk = tid >> 7;  // channel, 16-row token block
   const int cid = blockIdx.x, h = blockIdx.y;
   const int2 nc = chunk_tab[cid];
   const int n = nc.x;
@@ -109,35 +109,36 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int64_t chan = (int64_t)h * D + ch;
   uint8_t* rec = records + ((int64_t)cid * H + h) * REC_BYTES;
 
-  // raw tiles land in the region the Gram operands and M/P use later
-  const __nv_bfloat16* rq_t = reinterpret_cast<const __nv_bfloat16*>(sm + PREP_OPA);
-  const __nv_bfloat16* rk_t = reinterpret_cast<const __nv_bfloat16*>(sm + PREP_OPA + RAW_BYTES);
-  const __nv_bfloat16* rg_t = reinterpret_cast<const __nv_bfloat16*>(sm + PREP_OPA + 2 * RAW_BYTES);
+  // ---- 0. TMA loads of the raw q, k, g tiles (rows t0-3 .. t0+63) -----------
+  const __nv_bfloat16* rq_t = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW);
+  const __nv_bfloat16* rk_t = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + RAW_BYTES);
+  const __nv_bfloat16* rg_t = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + 2 * RAW_BYTES);
   if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
   if (tid == 0) {
-    tc::bar_init(&bar, 1);
+    tc::bar_init(&bar_ld, 1); tc::bar_init(&bar_g[0], 1); tc::bar_init(&bar_g[1], 1);
+    tc::bar_init(&bar_w, 1);
     tc::bar_init_fence();
-    // rows t0-3 .. t0+63 of head h (rows outside the tensor read as zero)
-    tc::bar_expect_tx(&bar, 3 * RAW_BYTES);
-    tc::tma_load_2d(sm + PREP_OPA, &tm_q, h * D, (int)(t0 - 3), &bar);
-    tc::tma_load_2d(sm + PREP_OPA + RAW_BYTES, &tm_k, h * D, (int)(t0 - 3), &bar);
-    tc::tma_load_2d(sm + PREP_OPA + 2 * RAW_BYTES, &tm_g, h * D, (int)(t0 - 3), &bar);
+    tc::bar_expect_tx(&bar_ld, 3 * RAW_BYTES);
+    tc::tma_load_2d(sm + P_RAW, &tm_q, h * D, (int)(t0 - 3), &bar_ld);
+    tc::tma_load_2d(sm + P_RAW + RAW_BYTES, &tm_k, h * D, (int)(t0 - 3), &bar_ld);
+    tc::tma_load_2d(sm + P_RAW + 2 * RAW_BYTES, &tm_g, h * D, (int)(t0 - 3), &bar_ld);
   }
   if (tid < CH) ms[MS_BETA + tid] = tid < L ? to_f(beta[(t0 + tid) * H + h]) : 0.f;
   const float4 wq = load4(conv_w + (0 * HD + chan) * 4);
   const float4 wk = load4(conv_w + (1 * HD + chan) * 4);
+  tc::fence_before();
   __syncthreads();
-  uint32_t phase = 0;
-  tc::bar_wait(&bar, phase);
-  phase ^= 1;
+  tc::fence_after();
+  const uint32_t tm = tmem_base;
+  tc::bar_wait(&bar_ld, 0);
 
-  // ---- 1. causal conv of q and k, clamped log-decay, half-local cumsum ------
+  // ---- 1. causal conv of q, k and block-local cumsum of the clamped gate ----
+  const int r0 = 16 * blk;
   {
-    const int r0 = 32 * half;
     float hq[3], hk[3];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
-      const int64_t p = t0 + r0 - 3 + j;  // absolute token of the halo row (tile row r0 + j)
+      const int64_t p = t0 + r0 - 3 + j;  // token of tile row r0 + j
       float a = to_f(rq_t[(r0 + j) * D + ch]), b = to_f(rk_t[(r0 + j) * D + ch]);
       if (p < seg0) {  // before the segment: conv history (or zeros)
         a = b = 0.f;
@@ -150,8 +151,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       hq[j] = a; hk[j] = b;
     }
     float cum = 0.f;
-#pragma unroll 8
-    for (int r = 0; r < 32; ++r) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
       const int t = r0 + r;
       const float xq = to_f(rq_t[(t + 3) * D + ch]), xk = to_f(rk_t[(t + 3) * D + ch]);
       float yq = conv4(wq, hq[0], hq[1], hq[2], xq);
@@ -160,21 +161,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       hq[0] = hq[1]; hq[1] = hq[2]; hq[2] = xq;
       hk[0] = hk[1]; hk[1] = hk[2]; hk[2] = xk;
       const bool valid = t < L;
-      const float gl = valid ? fmaxf(to_f(rg_t[(t + 3) * D + ch]), LOG_DECAY_FLOOR) : 0.f;
-      cum += gl;
+      cum += valid ? fmaxf(to_f(rg_t[(t + 3) * D + ch]), LOG_DECAY_FLOOR) : 0.f;
       Yq[t * D + ch] = valid ? yq : 0.f;
       Yk[t * D + ch] = valid ? yk : 0.f;
-      E1[t * D + ch] = cum;
+      Gm[t * D + ch] = cum;
     }
+    ms[MS_CARRY + blk * D + ch] = cum;  // this block's total
   }
   __syncthreads();
 
-  // ---- 2. cumsum carry into the second half; L2 norms (warp per 8 rows) ----
-  if (half == 1) {
-    const float carry = E1[31 * D + ch];
-    for (int t = 32; t < CH; ++t) E1[t * D + ch] += carry;
-  }
-  for (int t = warp * 8; t < warp * 8 + 8; ++t) {
+  // ---- 2. L2 norms (warp per 4 rows) -----------------------------------------
+  for (int t = warp * 4; t < warp * 4 + 4; ++t) {
     const float4 a = *reinterpret_cast<const float4*>(&Yq[t * D + lane * 4]);
     const float4 b = *reinterpret_cast<const float4*>(&Yk[t * D + lane * 4]);
     float nq = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
@@ -188,128 +185,136 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   __syncthreads();
 
-  // ---- 3. normalise; block-midpoint factors ----------------------------------
+  // ---- 3. normalise; factors about this block's midpoint ---------------------
+  // e_t = e^{G_t - G_mid} within [e^-40, e^40]; KX = k e, QX = q e (B operands),
+  // KE = k / e (A operand base), QT = e^{G_mid} QX (record)
+  float kx[16], qx[16];
   {
-    const int r0 = 32 * half;
-    // midpoints of this half's two blocks, and Gamma_C (row 63) from half 1
-    for (int J = 2 * half; J < 2 * half + 2; ++J) gt[GT_GMID + J * D + ch] = E1[(16 * J + 8) * D + ch];
-    if (half == 1) gt[GT_GC + ch] = E1[63 * D + ch];
-    for (int r = 0; r < 32; ++r) {
+    float carry = 0.f;
+    for (int b = 0; b < blk; ++b) carry += ms[MS_CARRY + b * D + ch];
+    float G[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) G[r] = Gm[(r0 + r) * D + ch] + carry;
+    const float gmid = G[8];
+    ms[MS_GMID + blk * D + ch] = gmid;
+    if (blk == 3) ms[MS_GC + ch] = G[15];
+    const float egm = __expf(gmid);
+    ms[MS_EGM + blk * D + ch] = egm;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
       const int t = r0 + r;
-      Yq[t * D + ch] *= ms[MS_RQ + t];
-      Yk[t * D + ch] *= ms[MS_RK + t];
-      const float d = E1[t * D + ch] - E1[(16 * (t >> 4) + 8) * D + ch];  // G_t - G_mid
-      Xf[t * D + ch] = __expf(d);
+      const float e = __expf(G[r] - gmid);
+      const float kh = Yk[t * D + ch] * ms[MS_RK + t], qh = Yq[t * D + ch] * ms[MS_RQ + t];
+      kx[r] = kh * e;
+      qx[r] = qh * e;
+      Gm[t * D + ch] = kh / e;  // KE (own element)
+      *reinterpret_cast<float*>(rec + REC_QT + tc::sw128(t, ch, 64)) = tc::to_tf32(egm * qx[r]);
     }
   }
-  __syncthreads();
-  {
-    const int r0 = 32 * half;
-    for (int r = 0; r < 32; ++r) {
-      const int t = r0 + r;
-      E1[t * D + ch] = 1.0f / Xf[t * D + ch];  // e^{G_mid - G_t}
-    }
-    // per-(block, channel) factors: e^{G_mid(J)}, e^{G_C - G_mid(J)}, and the
-    // block-to-block factors e^{G_mid(I) - G_mid(J)} for J < I
-    if (half == 0) {
-      const float gc = gt[GT_GC + ch];
-      for (int J = 0; J < 4; ++J) {
-        const float gm = gt[GT_GMID + J * D + ch];
-        ms[MS_EGM + J * D + ch] = __expf(gm);
-        ms[MS_EGC + J * D + ch] = __expf(gc - gm);
-      }
-    } else {
-      for (int I = 1; I < 4; ++I)
-        for (int J = 0; J < I; ++J)
-          ms[MS_Z + zidx(I, J) * D + ch] = __expf(gt[GT_GMID + I * D + ch] - gt[GT_GMID + J * D + ch]);
-    }
+  __syncthreads();  // conv(q), conv(k) are read; the KQX tile may overwrite them
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    *reinterpret_cast<float*>(kqx + tc::sw128(32 * blk + r, ch, 128)) = tc::to_tf32(kx[r]);
+    *reinterpret_cast<float*>(kqx + tc::sw128(32 * blk + 16 + r, ch, 128)) = tc::to_tf32(qx[r]);
   }
   __syncthreads();
 
-  // ---- 4. record tiles that need no solve: QT, KB (thread = channel), scalars
+  // ---- 4. block-to-block factors; record tiles KB and scalars ----------------
   {
-    const int r0 = 32 * half;
-    float kb[32];
-    for (int r = 0; r < 32; ++r) {
-      const int t = r0 + r, J = t >> 4;
-      const float xf = Xf[t * D + ch], e1 = E1[t * D + ch];
-      const float qt = ms[MS_EGM + J * D + ch] * xf * Yq[t * D + ch];
-      *reinterpret_cast<float*>(rec + REC_QT + tc::sw128(t, ch, 64)) = tc::to_tf32(qt);
-      kb[r] = tc::to_tf32(ms[MS_EGC + J * D + ch] * e1 * Yk[t * D + ch]);
-    }
-    // row ch of KB, columns r0..r0+31 = one 128-byte slab row
+    const float gc = ms[MS_GC + ch], gm = ms[MS_GMID + blk * D + ch];
+    for (int J = 0; J < blk; ++J) ms[MS_Z + zidx(blk, J) * D + ch] = __expf(gm - ms[MS_GMID + J * D + ch]);
+    const float egc = __expf(gc - gm);  // e^{G_C - G_mid}
+    float kb[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int r = 0; r < 16; ++r) kb[r] = tc::to_tf32(egc * Gm[(r0 + r) * D + ch]);
+    // row ch of KB, columns r0..r0+15 (half of a 128-byte slab row)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
       *reinterpret_cast<float4*>(rec + REC_KB + tc::sw128(ch, r0 + 4 * j, 128)) =
           make_float4(kb[4 * j], kb[4 * j + 1], kb[4 * j + 2], kb[4 * j + 3]);
     float* sc = reinterpret_cast<float*>(rec + REC_SC);
     if (tid < CH) { sc[tid] = ms[MS_BETA + tid]; sc[64 + tid] = ms[MS_PD + tid]; }
-    if (half == 1) sc[128 + ch] = __expf(gt[GT_GC + ch]);  // gt is intact until step 5
+    if (blk == 0) sc[128 + ch] = __expf(gc);
   }
+  __syncthreads();
 
-  // ---- 5. gated Gram blocks on the tensor core, 4 slabs of 32 channels -------
-  const uint32_t tm = tmem_base;
-  for (int kp = 0; kp < 4; ++kp) {
-    // A_I: 4 x 64 rows x 32 channels (8192 elements), B_I: 4 x 32 rows x 32 (4096)
-    for (int e = tid; e < 4 * 64 * 32; e += 256) {
-      const int cc = e & 31, j = (e >> 5) & 63, I = e >> 11;
-      const int c = kp * 32 + cc, J = j >> 4;
-      float val = 0.f;
-      if (J <= I) {
-        val = Yk[j * D + c] * E1[j * D + c];
-        if (J < I) val *= ms[MS_Z + zidx(I, J) * D + c];
+  // ---- 5. gated Gram blocks on the tensor core --------------------------------
+  // pass kp covers channels 32kp..32kp+31; A_I rows j of blocks J <= I (other
+  // rows are never read back), B_I = rows 32I..32I+31 of KQX
+  auto build_a = [&](int kp) {
+    uint8_t* buf = sm + P_RAW + (kp & 1) * 32768;
+    // (I, j, 4-channel group) with J(j) <= I: 160 rows x 8 groups
+    for (int e = tid; e < 160 * 8; e += PREP_THREADS) {
+      const int c4 = e & 7, rr = e >> 3;  // rr in [0, 160): I-major rows
+      const int I = rr < 16 ? 0 : rr < 48 ? 1 : rr < 96 ? 2 : 3;
+      const int j = rr - (I == 0 ? 0 : I == 1 ? 16 : I == 2 ? 48 : 96);
+      const int J = j >> 4, c = 32 * kp + 4 * c4;
+      float4 v = *reinterpret_cast<const float4*>(&Gm[j * D + c]);
+      if (J < I) {
+        const float4 z = *reinterpret_cast<const float4*>(&ms[MS_Z + zidx(I, J) * D + c]);
+        v.x *= z.x; v.y *= z.y; v.z *= z.z; v.w *= z.w;
       }
-      *reinterpret_cast<float*>(opA + I * 8192 + tc::sw128(j, cc, 64)) = tc::to_tf32(val);
-    }
-    for (int e = tid; e < 4 * 32 * 32; e += 256) {
-      const int cc = e & 31, r = (e >> 5) & 31, I = e >> 10;
-      const int c = kp * 32 + cc, i = 16 * I + (r & 15);
-      const float src = r < 16 ? Yk[i * D + c] : Yq[i * D + c];
-      *reinterpret_cast<float*>(opB + I * 4096 + tc::sw128(r, cc, 32)) = tc::to_tf32(src * Xf[i * D + c]);
+      v = make_float4(tc::to_tf32(v.x), tc::to_tf32(v.y), tc::to_tf32(v.z), tc::to_tf32(v.w));
+      *reinterpret_cast<float4*>(buf + I * 8192 + tc::sw128(j, 4 * c4, 64)) = v;
     }
     tc::fence_async_smem();
-    tc::fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tc::fence_after();
-      const uint64_t da = tc::desc(tc::smem_u32(opA)), db = tc::desc(tc::smem_u32(opB));
-#pragma unroll
-      for (int I = 0; I < 4; ++I)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          tc::mma_ss(tm + 32 * I, da + ((I * 8192) >> 4) + tc::desc_step(64, ks),
-                     db + ((I * 4096) >> 4) + tc::desc_step(32, ks), tc::idesc_tf32(64, 32),
-                     (kp > 0 || ks > 0) ? 1 : 0);
-      tc::commit(&bar);
-    }
-    tc::bar_wait(&bar, phase);
-    phase ^= 1;
+  };
+  auto issue_gram = [&](int kp) {
     tc::fence_after();
-  }
+    const uint64_t da = tc::desc(tc::smem_u32(sm + P_RAW + (kp & 1) * 32768));
+    const uint64_t db = tc::desc(tc::smem_u32(kqx + kp * 16384));
+#pragma unroll
+    for (int I = 0; I < 4; ++I)
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        tc::mma_ss(tm + 32 * I, da + ((I * 8192) >> 4) + tc::desc_step(64, ks),
+                   db + ((I * 32 * 128) >> 4) + tc::desc_step(128, ks), tc::idesc_tf32(64, 32),
+                   (kp > 0 || ks > 0) ? 1 : 0);
+    tc::commit(&bar_g[kp & 1]);
+  };
+  build_a(0);
+  tc::fence_before();
+  __syncthreads();
+  if (tid == 0) issue_gram(0);
+  build_a(1);
+  tc::fence_before();
+  __syncthreads();
+  if (tid == 0) issue_gram(1);
+  tc::bar_wait(&bar_g[0], 0);  // pass 0 done: buffer 0 free
+  build_a(2);
+  tc::fence_before();
+  __syncthreads();
+  if (tid == 0) issue_gram(2);
+  tc::bar_wait(&bar_g[1], 0);  // pass 1 done: buffer 1 free
+  build_a(3);
+  tc::fence_before();
+  __syncthreads();
+  if (tid == 0) issue_gram(3);
+  tc::bar_wait(&bar_g[1], 1);  // pass 3 (and everything before it) done
+  tc::fence_after();
 
   // ---- 6. read D_I (M = 64 layout: row j -> lane j%16 + 32*(j/16)) ---------
-  if (warp < 4) {
-    const int j = 16 * warp + (lane & 15);
-    for (int I = 0; I < 4; ++I) {
-      float mv[16], pv[16];
-      tc::ld16(tm + ((uint32_t)(32 * warp) << 16) + 32 * I, mv);
-      tc::ld16(tm + ((uint32_t)(32 * warp) << 16) + 32 * I + 16, pv);
-      tc::ld_wait();
-      if (lane < 16) {
+  {
+    const int sub = warp & 3, I = warp >> 2;  // warp reads block row I for rows 16sub..16sub+15
+    const int j = 16 * sub + (lane & 15);
+    float mv[16], pv[16];
+    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 32 * I, mv);
+    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 32 * I + 16, pv);
+    tc::ld_wait();
+    if (lane < 16) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          const int i = 16 * I + r;
-          Ms[i * CH + j] = i > j ? ms[MS_BETA + i] * mv[r] : 0.f;  // diag(beta) M, strict
-          Ps[i * CH + j] = i > j ? pv[r] : 0.f;
-        }
+      for (int r = 0; r < 16; ++r) {
+        const int i = 16 * I + r;
+        Ms[i * CH + j] = i > j ? ms[MS_BETA + i] * mv[r] : 0.f;  // diag(beta) M, strict
+        Ps[i * CH + j] = i > j ? pv[r] : 0.f;
       }
     }
   }
   __syncthreads();
 
   // ---- 7. X = (I + diag(beta) M)^-1, blocked forward substitution -------------
-  float* Xd = sv + SV_XD;  // [4][16][16] inverses of the diagonal blocks
-  float* Yb = sv + SV_YB;  // [3][16][16]
+  float* Xd = (float*)(sm + P_RAW);         // [4][16][16] inverses of the diagonal blocks
+  float* Yb = (float*)(sm + P_RAW) + 1024;  // [3][16][16]
   if (tid < 64) {
     const int I = tid >> 4, cc = tid & 15;  // column cc of X_II
     float x[16];
@@ -324,21 +329,24 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int r = 0; r < 16; ++r) Xd[(I * 16 + r) * 16 + cc] = x[r];
   }
   __syncthreads();
+#pragma unroll
   for (int I = 1; I < 4; ++I) {
     // Y_IJ = sum_{K=J}^{I-1} L_IK X_KJ  for J < I (X_KJ already in Ms for K < I)
-    for (int e = tid; e < I * 256; e += 256) {
+    for (int e = tid; e < I * 256; e += PREP_THREADS) {
       const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+      const float* Lrow = Ms + (16 * I + r) * CH;
       float s = 0.f;
-      for (int m = 16 * J; m < 16 * I; ++m) {
-        const float xk = (m >> 4) == J ? Xd[(J * 16 + (m & 15)) * 16 + cc]   // X_JJ
-                                       : Ms[m * CH + 16 * J + cc];           // X_KJ, K > J
-        s += Ms[(16 * I + r) * CH + m] * xk;
+#pragma unroll
+      for (int m = 0; m < 16; ++m) s += Lrow[16 * J + m] * Xd[(J * 16 + m) * 16 + cc];
+      for (int K = J + 1; K < I; ++K) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) s += Lrow[16 * K + m] * Ms[(16 * K + m) * CH + 16 * J + cc];
       }
       Yb[(J * 16 + r) * 16 + cc] = s;
     }
     __syncthreads();
     // X_IJ = -X_II Y_IJ, written over L_IJ
-    for (int e = tid; e < I * 256; e += 256) {
+    for (int e = tid; e < I * 256; e += PREP_THREADS) {
       const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
       float s = 0.f;
 #pragma unroll
@@ -348,32 +356,44 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
   }
   // diagonal blocks into Ms; Ms now holds X (unit lower triangular)
-  for (int e = tid; e < 4 * 256; e += 256) {
+  for (int e = tid; e < 4 * 256; e += PREP_THREADS) {
     const int I = e >> 8, r = (e >> 4) & 15, cc = e & 15;
     Ms[(16 * I + r) * CH + 16 * I + cc] = Xd[(I * 16 + r) * 16 + cc];
   }
   __syncthreads();
 
   // ---- 8. T = X diag(beta); tiles for W = T K~ and the record's T_s, P_s -----
-  uint8_t* tT = opA;          // [64 t][64 t'] tile, 16 KB
-  uint8_t* tK = opA + 16384;  // [128 k][64 t'] tile (K~^T), 32 KB
-  for (int e = tid; e < CH * CH; e += 256) {
-    const int t = e >> 6, tp = e & 63;
-    const float tv = tp <= t ? Ms[t * CH + tp] * ms[MS_BETA + tp] : 0.f;
-    const float tr = tc::to_tf32(tv);
-    *reinterpret_cast<float*>(tT + tc::sw128(t, tp, 64)) = tr;
-    *reinterpret_cast<float*>(rec + REC_B1 + tc::sw128(t, tp, 64)) = tp < t ? tr : 0.f;
-    *reinterpret_cast<float*>(rec + REC_PS + tc::sw128(t, tp, 64)) = tc::to_tf32(Ps[t * CH + tp]);
+  uint8_t* tT = sm + P_RAW;          // [64 t][64 t'] tile, 16 KB
+  uint8_t* tK = sm + P_RAW + 16384;  // [128 k][64 t'] tile (K~^T), 32 KB
+  for (int e = tid; e < CH * 16; e += PREP_THREADS) {  // 4-column groups
+    const int t = e >> 4, tp = 4 * (e & 15);
+    float4 tv, pv;
+    float* tvp = &tv.x;
+    float* pvp = &pv.x;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = tp + u;
+      tvp[u] = tc::to_tf32(c <= t ? Ms[t * CH + c] * ms[MS_BETA + c] : 0.f);
+      pvp[u] = tc::to_tf32(Ps[t * CH + c]);
+    }
+    *reinterpret_cast<float4*>(tT + tc::sw128(t, tp, 64)) = tv;
+    float4 ts = tv;
+    float* tsp = &ts.x;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (tp + u >= t) tsp[u] = 0.f;  // strictly lower part only
+    *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, tp, 64)) = ts;
+    *reinterpret_cast<float4*>(rec + REC_PS + tc::sw128(t, tp, 64)) = pv;
   }
   {
-    const int r0 = 32 * half;
-    float kt[32];
-    for (int r = 0; r < 32; ++r) {
-      const int t = r0 + r;
-      kt[r] = tc::to_tf32(ms[MS_EGM + (t >> 4) * D + ch] * Xf[t * D + ch] * Yk[t * D + ch]);
-    }
+    // K~^T row ch, columns r0..r0+15: e^{G_t} k_t = e^{G_mid} * KX
+    const float egm = ms[MS_EGM + blk * D + ch];
+    float kt[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int r = 0; r < 16; ++r)
+      kt[r] = tc::to_tf32(egm * *reinterpret_cast<const float*>(kqx + tc::sw128(32 * blk + r, ch, 128)));
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
       *reinterpret_cast<float4*>(tK + tc::sw128(ch, r0 + 4 * j, 128)) =
           make_float4(kt[4 * j], kt[4 * j + 1], kt[4 * j + 2], kt[4 * j + 3]);
   }
@@ -387,25 +407,28 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int ks = 0; ks < 8; ++ks)
       tc::mma_ss(tm + 128, dt + tc::desc_step(64, ks), dk + tc::desc_step(128, ks), tc::idesc_tf32(64, 128),
                  ks > 0 ? 1 : 0);
-    tc::commit(&bar);
+    tc::commit(&bar_w);
   }
-  tc::bar_wait(&bar, phase);
-  phase ^= 1;
+  tc::bar_wait(&bar_w, 0);
   tc::fence_after();
 
   // ---- 9. -W rows into the record (columns 64..191 of B1) --------------------
-  if (warp < 4) {
-    const int t = 16 * warp + (lane & 15);
-    for (int cb = 0; cb < 8; ++cb) {
-      float w[16];
-      tc::ld16(tm + ((uint32_t)(32 * warp) << 16) + 128 + 16 * cb, w);
-      tc::ld_wait();
-      if (lane < 16) {
+  {
+    const int sub = warp & 3, cb = warp >> 2;  // rows 16sub.., columns 32cb..32cb+31
+    const int t = 16 * sub + (lane & 15);
+    float w0[16], w1[16];
+    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 128 + 32 * cb, w0);
+    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 128 + 32 * cb + 16, w1);
+    tc::ld_wait();
+    if (lane < 16) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + 16 * cb + 4 * j, 64)) =
-              make_float4(tc::to_tf32(-w[4 * j]), tc::to_tf32(-w[4 * j + 1]), tc::to_tf32(-w[4 * j + 2]),
-                          tc::to_tf32(-w[4 * j + 3]));
+      for (int j = 0; j < 4; ++j) {
+        *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + 32 * cb + 4 * j, 64)) =
+            make_float4(tc::to_tf32(-w0[4 * j]), tc::to_tf32(-w0[4 * j + 1]), tc::to_tf32(-w0[4 * j + 2]),
+                        tc::to_tf32(-w0[4 * j + 3]));
+        *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + 32 * cb + 16 + 4 * j, 64)) =
+            make_float4(tc::to_tf32(-w1[4 * j]), tc::to_tf32(-w1[4 * j + 1]), tc::to_tf32(-w1[4 * j + 2]),
+                        tc::to_tf32(-w1[4 * j + 3]));
       }
     }
   }

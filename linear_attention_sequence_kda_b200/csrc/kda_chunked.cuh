@@ -76,7 +76,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     auto prep = chunk_prep_kernel<ACT>;
     if (cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess)
       return KDA_ERR_CUDA;
-    prep<<<dim3((unsigned)total, H), 256, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w,
+    prep<<<dim3((unsigned)total, H), PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w,
                                                                (const T*)init_conv, cu_dev, d_tab, H, records);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
   }
