@@ -84,7 +84,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16* __restrict__ beta,
                   const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int2* __restrict__ chunk_tab, int H,
-                  uint8_t* __restrict__ records) {
+                  int n_items, uint8_t* __restrict__ records) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* Yq = (float*)(sm + P_KQX);
@@ -99,38 +99,50 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ch = tid & 127, blk = tid >> 7;  // channel, 16-row token block
-  const int cid = blockIdx.x, h = blockIdx.y;
-  const int2 nc = chunk_tab[cid];
-  const int n = nc.x;
-  const int64_t seg0 = cu[n], seg1 = cu[n + 1];
-  const int64_t t0 = seg0 + (int64_t)CH * nc.y;
-  const int L = (int)((seg1 - t0) < CH ? (seg1 - t0) : CH);
   const int64_t HD = (int64_t)H * D;
-  const int64_t chan = (int64_t)h * D + ch;
-  uint8_t* rec = records + ((int64_t)cid * H + h) * REC_BYTES;
-
-  // ---- 0. TMA loads of the raw q, k, g tiles (rows t0-3 .. t0+63) -----------
   const __nv_bfloat16* rq_t = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW);
   const __nv_bfloat16* rk_t = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + RAW_BYTES);
   const __nv_bfloat16* rg_t = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + 2 * RAW_BYTES);
+  // raw q, k, g tiles of work item `it` (rows t0-3 .. t0+63; outside the tensor
+  // reads as zero) into the raw region
+  auto load_raw = [&](int it) {
+    const int2 c = chunk_tab[it / H];
+    const int hh = it % H;
+    const int y = (int)(cu[c.x] + (int64_t)CH * c.y - 3);
+    tc::bar_expect_tx(&bar_ld, 3 * RAW_BYTES);
+    tc::tma_load_2d(sm + P_RAW, &tm_q, hh * D, y, &bar_ld);
+    tc::tma_load_2d(sm + P_RAW + RAW_BYTES, &tm_k, hh * D, y, &bar_ld);
+    tc::tma_load_2d(sm + P_RAW + 2 * RAW_BYTES, &tm_g, hh * D, y, &bar_ld);
+  };
+
+  // ---- 0. once per block: TMEM, barriers, first item's tiles ----------------
   if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
   if (tid == 0) {
     tc::bar_init(&bar_ld, 1); tc::bar_init(&bar_g[0], 1); tc::bar_init(&bar_g[1], 1);
     tc::bar_init(&bar_w, 1);
     tc::bar_init_fence();
-    tc::bar_expect_tx(&bar_ld, 3 * RAW_BYTES);
-    tc::tma_load_2d(sm + P_RAW, &tm_q, h * D, (int)(t0 - 3), &bar_ld);
-    tc::tma_load_2d(sm + P_RAW + RAW_BYTES, &tm_k, h * D, (int)(t0 - 3), &bar_ld);
-    tc::tma_load_2d(sm + P_RAW + 2 * RAW_BYTES, &tm_g, h * D, (int)(t0 - 3), &bar_ld);
+    if ((int)blockIdx.x < n_items) load_raw(blockIdx.x);
   }
-  if (tid < CH) ms[MS_BETA + tid] = tid < L ? to_f(beta[(t0 + tid) * H + h]) : 0.f;
-  const float4 wq = load4(conv_w + (0 * HD + chan) * 4);
-  const float4 wk = load4(conv_w + (1 * HD + chan) * 4);
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
   const uint32_t tm = tmem_base;
-  tc::bar_wait(&bar_ld, 0);
+  uint32_t par = 0;  // phase parity of the per-item barriers (bar_ld, bar_w)
+
+  // persistent loop over (chunk, head) work items, chunk-major
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x, par ^= 1) {
+  const int cid = item / H, h = item % H;
+  const int2 nc = chunk_tab[cid];
+  const int n = nc.x;
+  const int64_t seg0 = cu[n], seg1 = cu[n + 1];
+  const int64_t t0 = seg0 + (int64_t)CH * nc.y;
+  const int L = (int)((seg1 - t0) < CH ? (seg1 - t0) : CH);
+  const int64_t chan = (int64_t)h * D + ch;
+  uint8_t* rec = records + ((int64_t)cid * H + h) * REC_BYTES;
+  if (tid < CH) ms[MS_BETA + tid] = tid < L ? to_f(beta[(t0 + tid) * H + h]) : 0.f;
+  const float4 wq = load4(conv_w + (0 * HD + chan) * 4);
+  const float4 wk = load4(conv_w + (1 * HD + chan) * 4);
+  tc::bar_wait(&bar_ld, par);
 
   // ---- 1. causal conv of q, k and block-local cumsum of the clamped gate ----
   const int r0 = 16 * blk;
@@ -171,6 +183,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
 
   // ---- 2. L2 norms (warp per 4 rows) -----------------------------------------
+#pragma unroll
   for (int t = warp * 4; t < warp * 4 + 4; ++t) {
     const float4 a = *reinterpret_cast<const float4*>(&Yq[t * D + lane * 4]);
     const float4 b = *reinterpret_cast<const float4*>(&Yk[t * D + lane * 4]);
@@ -208,10 +221,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       kx[r] = kh * e;
       qx[r] = qh * e;
       Gm[t * D + ch] = kh / e;  // KE (own element)
-      *reinterpret_cast<float*>(rec + REC_QT + tc::sw128(t, ch, 64)) = tc::to_tf32(egm * qx[r]);
+      // QT tile image staged in the raw region (its tiles were consumed in step 1)
+      *reinterpret_cast<float*>(sm + P_RAW + tc::sw128(t, ch, 64)) = tc::to_tf32(egm * qx[r]);
     }
   }
+  tc::fence_async_smem();
   __syncthreads();  // conv(q), conv(k) are read; the KQX tile may overwrite them
+  if (tid == 0) {
+    tc::bulk_s2g(rec + REC_QT, sm + P_RAW, 32768);
+    tc::bulk_commit();
+  }
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
     *reinterpret_cast<float*>(kqx + tc::sw128(32 * blk + r, ch, 128)) = tc::to_tf32(kx[r]);
@@ -236,6 +255,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid < CH) { sc[tid] = ms[MS_BETA + tid]; sc[64 + tid] = ms[MS_PD + tid]; }
     if (blk == 0) sc[128 + ch] = __expf(gc);
   }
+  if (tid == 0) tc::bulk_wait_read();  // the QT staging may be overwritten after this
   __syncthreads();
 
   // ---- 5. gated Gram blocks on the tensor core --------------------------------
@@ -290,7 +310,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc::fence_before();
   __syncthreads();
   if (tid == 0) issue_gram(3);
-  tc::bar_wait(&bar_g[1], 1);  // pass 3 (and everything before it) done
+  tc::bar_wait(&bar_g[1], 1);  // pass 3 done
+  tc::bar_wait(&bar_g[0], 1);  // pass 2 done (each item uses two phases of each barrier)
   tc::fence_after();
 
   // ---- 6. read D_I (M = 64 layout: row j -> lane j%16 + 32*(j/16)) ---------
@@ -409,8 +430,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                  ks > 0 ? 1 : 0);
     tc::commit(&bar_w);
   }
-  tc::bar_wait(&bar_w, 0);
+  tc::bar_wait(&bar_w, par);
   tc::fence_after();
+  // the raw region (T and K~^T tiles) is free: fetch the next item's tiles
+  // while this item finishes
+  __syncthreads();
+  if (tid == 0 && item + (int)gridDim.x < n_items) load_raw(item + gridDim.x);
 
   // ---- 9. -W rows into the record (columns 64..191 of B1) --------------------
   {
@@ -432,6 +457,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     }
   }
+  tc::fence_before();
+  __syncthreads();  // TMEM columns and shared regions are reused by the next item
+  tc::fence_after();
+  }  // item loop
+  if (tid == 0) tc::bulk_wait_all();
   tc::fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem_base, 256);

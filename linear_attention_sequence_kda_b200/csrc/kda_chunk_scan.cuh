@@ -18,6 +18,8 @@
 // Data movement: the raw value tile of chunk i+2 (TMA, 64 rows x 256 B) and the
 // record halves of chunk i+1 (bulk copies) are in flight while chunk i runs;
 // each record half is refilled as soon as the MMA group that reads it is done.
+// The output rows of a chunk are staged in shared memory and leave with one
+// bulk store per valid row (rows past the segment end are never written).
 #pragma once
 #include "kda_chunk_prep.cuh"
 #include "kda_common.cuh"
@@ -30,7 +32,8 @@ constexpr uint32_t SCAN_A = 0;                       // record part A: B1 | QT (
 constexpr uint32_t SCAN_B = REC_TILES_A;             // record part B: PS | KB | SC (50176 B)
 constexpr uint32_t SCAN_V0 = REC_TILES_A + REC_TILES_B;
 constexpr uint32_t SCAN_V1 = SCAN_V0 + VT_BYTES;
-constexpr uint32_t SCAN_SMEM = SCAN_V1 + VT_BYTES + 1024;
+constexpr uint32_t SCAN_O = SCAN_V1 + VT_BYTES;      // output staging [64 t][128] (fp32 or bf16)
+constexpr uint32_t SCAN_SMEM = SCAN_O + CH * D * 4 + 1024;
 constexpr int TM_V = 0, TM_S = 64, TM_U = 192, TM_O = 256;
 constexpr int TM_VX = 320, TM_UX = 384;  // exact fp32 V and U for the diagonal terms
 
@@ -171,6 +174,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
       if (tid == 0) load_a(i + 1);
       a_iss++;
     }
+    // the previous chunk's output stores must have read the staging buffer
+    // before (f) rewrites it (they were issued a whole chunk earlier)
+    if (tid < 32) tc::bulk_wait_read();
     // (d) U += beta V (exact diagonal of T V), S^T <- S^T diag(gamma)
 #pragma unroll
     for (int g16 = 0; g16 < 4; ++g16) {
@@ -222,21 +228,27 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
       if (tid == 0) load_b(i + 1);
       b_iss++;
     }
-    // (f) o = O + P_tt u
+    // (f) o = O + P_tt u, staged as [t][v] rows, then one bulk store per row
+    Tout* ost = reinterpret_cast<Tout*>(sm + SCAN_O);
 #pragma unroll
     for (int g16 = 0; g16 < 4; ++g16) {
       float r[16], ux[16];
       tc::ld16(lane_base + TM_O + 16 * g16, r);
       tc::ld16(lane_base + TM_UX + 16 * g16, ux);
       tc::ld_wait();
-      Tout* orow = o + (t0 + 16 * g16) * HD + chan;
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        if (16 * g16 + j < L) orow[j * HD] = from_f<Tout>(fmaf(sc[64 + 16 * g16 + j], ux[j], r[j]));
+        ost[(16 * g16 + j) * D + tid] = from_f<Tout>(fmaf(sc[64 + 16 * g16 + j], ux[j], r[j]));
     }
+    tc::fence_async_smem();
     tc::fence_before();
-    __syncthreads();  // sc and TMEM O are rewritten by the next chunk
+    __syncthreads();  // staging complete; sc and TMEM O are rewritten by the next chunk
     tc::fence_after();
+    if (tid < 32) {
+      for (int t = tid; t < L; t += 32)
+        tc::bulk_s2g(o + (t0 + t) * HD + (int64_t)h * D, ost + t * D, D * sizeof(Tout));
+      tc::bulk_commit();
+    }
   }
 
   if (!ok) {
@@ -250,6 +262,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
     for (int b = 0; b < 2; ++b)
       if (v_iss[b] > 0) tc::bar_wait(&bar_v[b], (v_iss[b] - 1) & 1);
   }
+  if (tid < 32) tc::bulk_wait_all();  // output rows are in global memory before exit
   // final state: column v of S = row v of S^T
   if (ok) {
     float* Sf = final_state + ((int64_t)n * H + h) * D * D + tid;
