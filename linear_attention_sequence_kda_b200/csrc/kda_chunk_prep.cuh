@@ -259,8 +259,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
 
   // ---- 5. gated Gram blocks on the tensor core --------------------------------
-  // pass kp covers channels 32kp..32kp+31; A_I rows j of blocks J <= I (other
-  // rows are never read back), B_I = rows 32I..32I+31 of KQX
+  // pass kp covers channels 32kp..32kp+31.  Block rows are paired: pair p
+  // stacks A_{2p} (rows 0..63) over A_{2p+1} (rows 64..127) into one M = 128
+  // operand against B = KQX rows 64p..64p+63 (= B_{2p} | B_{2p+1}, N = 64); the
+  // wanted products are the two diagonal 64 x 32 quadrants.  A_I rows j of
+  // blocks J <= I are written (other rows are never read back).
   auto build_a = [&](int kp) {
     uint8_t* buf = sm + P_RAW + (kp & 1) * 32768;
     // (I, j, 4-channel group) with J(j) <= I: 160 rows x 8 groups
@@ -275,7 +278,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         v.x *= z.x; v.y *= z.y; v.z *= z.z; v.w *= z.w;
       }
       v = make_float4(tc::to_tf32(v.x), tc::to_tf32(v.y), tc::to_tf32(v.z), tc::to_tf32(v.w));
-      *reinterpret_cast<float4*>(buf + I * 8192 + tc::sw128(j, 4 * c4, 64)) = v;
+      *reinterpret_cast<float4*>(buf + (I >> 1) * 16384 + tc::sw128((I & 1) * 64 + j, 4 * c4, 128)) = v;
     }
     tc::fence_async_smem();
   };
@@ -284,11 +287,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint64_t da = tc::desc(tc::smem_u32(sm + P_RAW + (kp & 1) * 32768));
     const uint64_t db = tc::desc(tc::smem_u32(kqx + kp * 16384));
 #pragma unroll
-    for (int I = 0; I < 4; ++I)
+    for (int pr = 0; pr < 2; ++pr)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        tc::mma_ss(tm + 32 * I, da + ((I * 8192) >> 4) + tc::desc_step(64, ks),
-                   db + ((I * 32 * 128) >> 4) + tc::desc_step(128, ks), tc::idesc_tf32(64, 32),
+        tc::mma_ss(tm + 64 * pr, da + ((pr * 16384) >> 4) + tc::desc_step(128, ks),
+                   db + ((pr * 64 * 128) >> 4) + tc::desc_step(128, ks), tc::idesc_tf32(128, 64),
                    (kp > 0 || ks > 0) ? 1 : 0);
     tc::commit(&bar_g[kp & 1]);
   };
@@ -314,21 +317,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc::bar_wait(&bar_g[0], 1);  // pass 2 done (each item uses two phases of each barrier)
   tc::fence_after();
 
-  // ---- 6. read D_I (M = 64 layout: row j -> lane j%16 + 32*(j/16)) ---------
+  // ---- 6. read the diagonal quadrants (M = 128 layout: row m -> lane m) ------
   {
-    const int sub = warp & 3, I = warp >> 2;  // warp reads block row I for rows 16sub..16sub+15
-    const int j = 16 * sub + (lane & 15);
-    float mv[16], pv[16];
-    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 32 * I, mv);
-    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 32 * I + 16, pv);
+    const int sub = warp & 3, pr = (warp >> 2) & 1, part = warp >> 3;  // part 0: M columns, 1: P columns
+    const int m = 32 * sub + lane;       // accumulator row
+    const int I = 2 * pr + (m >> 6);     // block row
+    const int j = m & 63;
+    float v[16];
+    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 64 * pr + 32 * (m >> 6) + 16 * part, v);
     tc::ld_wait();
-    if (lane < 16) {
+    float* dst = part == 0 ? Ms : Ps;
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const int i = 16 * I + r;
-        Ms[i * CH + j] = i > j ? ms[MS_BETA + i] * mv[r] : 0.f;  // diag(beta) M, strict
-        Ps[i * CH + j] = i > j ? pv[r] : 0.f;
-      }
+    for (int r = 0; r < 16; ++r) {
+      const int i = 16 * I + r;
+      dst[i * CH + j] = i > j ? (part == 0 ? ms[MS_BETA + i] * v[r] : v[r]) : 0.f;  // diag(beta) M / P, strict
     }
   }
   __syncthreads();

@@ -6,7 +6,9 @@
 //
 // Thread v (of 128) owns value column v: TMEM lane v holds row v of
 //   V^T (cols 0..63) | S^T (cols 64..191) | U^T (192..255) | O^T (256..319)
-// (tf32 MMA operands) and, in fp32, V^T (320..383) and U^T (384..447).
+// (tf32 MMA operands), in fp32 V^T (320..383) and U^T (384..447), and a second
+// O^T buffer (448..511): chunk i's output is finalised while chunk i+1's first
+// MMA group runs.
 // Per chunk, with the record written by chunk_prep_kernel:
 //   MMA1  U^T = [V^T | S^T] [T_s | -W]^T        (K = 64 + 128)
 //         O^T = S^T Q~^T                          (K = 128)
@@ -19,7 +21,8 @@
 // record halves of chunk i+1 (bulk copies) are in flight while chunk i runs;
 // each record half is refilled as soon as the MMA group that reads it is done.
 // The output rows of a chunk are staged in shared memory and leave with one
-// bulk store per valid row (rows past the segment end are never written).
+// TMA tensor store (full chunks) or one bulk store per valid row (a segment's
+// last, partial chunk: rows past the segment end are never written).
 #pragma once
 #include "kda_chunk_prep.cuh"
 #include "kda_common.cuh"
@@ -34,12 +37,15 @@ constexpr uint32_t SCAN_V0 = REC_TILES_A + REC_TILES_B;
 constexpr uint32_t SCAN_V1 = SCAN_V0 + VT_BYTES;
 constexpr uint32_t SCAN_O = SCAN_V1 + VT_BYTES;      // output staging [64 t][128] (fp32 or bf16)
 constexpr uint32_t SCAN_SMEM = SCAN_O + CH * D * 4 + 1024;
-constexpr int TM_V = 0, TM_S = 64, TM_U = 192, TM_O = 256;
+constexpr int TM_V = 0, TM_S = 64, TM_U = 192;
 constexpr int TM_VX = 320, TM_UX = 384;  // exact fp32 V and U for the diagonal terms
+constexpr int TM_O0 = 256, TM_O1 = 448;  // output accumulators, alternating by chunk
+__device__ __forceinline__ int o_col(int chunk) { return (chunk & 1) ? TM_O1 : TM_O0; }
 
 template <typename Tout, int ACT>
 __global__ void __launch_bounds__(128, 1)
-chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ conv_w,
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const float* __restrict__ conv_w,
                   const float* init_state, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
@@ -48,7 +54,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t bar_a, bar_b, bar_v[2], bar_m1, bar_m2;
   __shared__ uint32_t tmem_base;
-  __shared__ float sc[256];  // this chunk's beta[64], P_tt[64], e^{Gamma_C}[128]
+  __shared__ float scb[2][256];  // per chunk parity: beta[64], P_tt[64], e^{Gamma_C}[128]
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int n = seq_order[blockIdx.x / H], h = blockIdx.x % H;
@@ -119,6 +125,37 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
   const uint64_t d_ps = tc::desc(tc::smem_u32(sm + SCAN_B));
   const uint64_t d_kb = tc::desc(tc::smem_u32(sm + SCAN_B + (REC_KB - REC_PS)));
 
+  // o = O + P_tt u for chunk j (O in its TMEM buffer, exact U still in UX):
+  // staged as [t][v] rows in shared memory, then one tensor store (full chunk)
+  // or one bulk store per valid row
+  Tout* ost = reinterpret_cast<Tout*>(sm + SCAN_O);
+  auto finalize = [&](int j) {
+    const int Lj = (int)((T - (int64_t)CH * j) < CH ? (T - (int64_t)CH * j) : CH);
+    const int64_t tj = seg0 + (int64_t)CH * j;
+    const float* scj = scb[j & 1];
+#pragma unroll
+    for (int g16 = 0; g16 < 4; ++g16) {
+      float r[16], ux[16];
+      tc::ld16(lane_base + o_col(j) + 16 * g16, r);
+      tc::ld16(lane_base + TM_UX + 16 * g16, ux);
+      tc::ld_wait();
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj)
+        ost[(16 * g16 + jj) * D + tid] = from_f<Tout>(fmaf(scj[64 + 16 * g16 + jj], ux[jj], r[jj]));
+    }
+    tc::fence_async_smem();
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    if (tid == 0) {
+      if (Lj == CH)
+        tc::tma_store_2d(&tm_o, h * D, (int)tj, ost);
+      else
+        for (int t = 0; t < Lj; ++t) tc::bulk_s2g(o + (tj + t) * HD + (int64_t)h * D, ost + t * D, D * sizeof(Tout));
+      tc::bulk_commit();
+    }
+  };
+
   bool ok = true;
   for (int i = 0; i < nchunks && ok; ++i) {
     const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
@@ -147,10 +184,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
     }
     tc::st_wait();
     // (b) this chunk's record
+    float* sc = scb[i & 1];
     ok &= tc::bar_wait(&bar_a, i & 1);
     ok &= tc::bar_wait(&bar_b, i & 1);
     sc[tid] = reinterpret_cast<const float*>(sm + SCAN_B + (REC_SC - REC_PS))[tid];
     sc[tid + 128] = reinterpret_cast<const float*>(sm + SCAN_B + (REC_SC - REC_PS))[tid + 128];
+    if (tid == 0) tc::bulk_wait_read();  // the previous output store has read the staging tile
     tc::fence_before();
     ok = __syncthreads_and(ok);
     if (!ok) break;
@@ -162,11 +201,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
         tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, d_b1 + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), ks > 0);
 #pragma unroll
       for (int ks = 0; ks < 16; ++ks)
-        tc::mma_ts(tm + TM_O, tm + TM_S + 8 * ks, d_qt + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), ks > 0);
+        tc::mma_ts(tm + o_col(i), tm + TM_S + 8 * ks, d_qt + tc::desc_step(64, ks), tc::idesc_tf32(128, 64),
+                   ks > 0);
       tc::commit(&bar_m1);
       if (i + 2 < nchunks) load_v(i + 2);
     }
     if (i + 2 < nchunks) v_iss[i & 1]++;
+    // while MMA group 1 runs: finish the previous chunk's output
+    if (i > 0) finalize(i - 1);
     ok &= tc::bar_wait(&bar_m1, i & 1);
     tc::fence_after();
     if (!__syncthreads_and(ok)) { ok = false; break; }
@@ -174,9 +216,6 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
       if (tid == 0) load_a(i + 1);
       a_iss++;
     }
-    // the previous chunk's output stores must have read the staging buffer
-    // before (f) rewrites it (they were issued a whole chunk earlier)
-    if (tid < 32) tc::bulk_wait_read();
     // (d) U += beta V (exact diagonal of T V), S^T <- S^T diag(gamma)
 #pragma unroll
     for (int g16 = 0; g16 < 4; ++g16) {
@@ -214,7 +253,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
       tc::fence_after();
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        tc::mma_ts(tm + TM_O, tm + TM_U + 8 * ks, d_ps + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
+        tc::mma_ts(tm + o_col(i), tm + TM_U + 8 * ks, d_ps + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
         tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, d_kb + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), 1);
@@ -228,28 +267,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
       if (tid == 0) load_b(i + 1);
       b_iss++;
     }
-    // (f) o = O + P_tt u, staged as [t][v] rows, then one bulk store per row
-    Tout* ost = reinterpret_cast<Tout*>(sm + SCAN_O);
-#pragma unroll
-    for (int g16 = 0; g16 < 4; ++g16) {
-      float r[16], ux[16];
-      tc::ld16(lane_base + TM_O + 16 * g16, r);
-      tc::ld16(lane_base + TM_UX + 16 * g16, ux);
-      tc::ld_wait();
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        ost[(16 * g16 + j) * D + tid] = from_f<Tout>(fmaf(sc[64 + 16 * g16 + j], ux[j], r[j]));
-    }
-    tc::fence_async_smem();
-    tc::fence_before();
-    __syncthreads();  // staging complete; sc and TMEM O are rewritten by the next chunk
-    tc::fence_after();
-    if (tid < 32) {
-      for (int t = tid; t < L; t += 32)
-        tc::bulk_s2g(o + (t0 + t) * HD + (int64_t)h * D, ost + t * D, D * sizeof(Tout));
-      tc::bulk_commit();
-    }
   }
+  if (ok && nchunks > 0) finalize(nchunks - 1);
 
   if (!ok) {
     // a wait gave up (status already recorded): drain what is still in flight
@@ -262,7 +281,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
     for (int b = 0; b < 2; ++b)
       if (v_iss[b] > 0) tc::bar_wait(&bar_v[b], (v_iss[b] - 1) & 1);
   }
-  if (tid < 32) tc::bulk_wait_all();  // output rows are in global memory before exit
+  if (tid == 0) tc::bulk_wait_all();  // output rows are in global memory before exit
   // final state: column v of S = row v of S^T
   if (ok) {
     float* Sf = final_state + ((int64_t)n * H + h) * D * D + tid;

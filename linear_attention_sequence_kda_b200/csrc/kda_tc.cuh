@@ -158,6 +158,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst_smem, const CUtensorMap* m
       : "memory");
 }
 
+// 2D tiled tensor store shared -> global through a tensor map (bulk-group
+// completion); the box must lie inside rows the caller owns
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, const void* src_smem) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_u32(src_smem))
+               : "memory");
+}
+
 // bulk async copy shared -> global (bulk-group completion); both addresses
 // 16-byte aligned, size a multiple of 16
 __device__ __forceinline__ void bulk_s2g(void* dst, const void* src_smem, uint32_t bytes) {

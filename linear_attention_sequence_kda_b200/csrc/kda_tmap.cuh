@@ -21,21 +21,28 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
   return fn;
 }
 
-// [rows, cols] bf16 row-major tensor, box of box_rows x box_cols, no swizzle,
-// zero fill outside.  A zero-row tensor gets an all-zero map (never used).
-inline bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                              uint32_t box_rows, uint32_t box_cols) {
+// [rows, cols] row-major tensor of bf16 (esize 2) or fp32 (esize 4), box of
+// box_rows x box_cols, no swizzle, zero fill outside.  A zero-row tensor gets
+// an all-zero map (never used).
+inline bool make_tmap_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows, uint32_t box_cols, int esize) {
   memset(map, 0, sizeof(*map));
   if (rows == 0) return true;
   auto enc = tmap_encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint64_t strides[1] = {cols * (cuuint64_t)esize};
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const CUtensorMapDataType dt = esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                              uint32_t box_rows, uint32_t box_cols) {
+  return make_tmap_2d(map, base, rows, cols, box_rows, box_cols, 2);
 }
 
 }  // namespace kda
