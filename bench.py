@@ -151,12 +151,8 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from linear_attention_sequence_kda_b200.sharding import max_over_ranks as _max
+    return x if world == 1 else _max(x, device="cuda")
 
 
 def timed(fn, steps, warmup, world, stream):
@@ -234,6 +230,9 @@ def main():
                     help="reduced head count (profiling only; the reported workload uses 64)")
     ap.add_argument("--seq-len", type=int, default=T_LONG,
                     help="reduced length (profiling only; the reported workload uses 65536)")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill leg (profiling only)")
+    ap.add_argument("--decode-seqs", type=int, default=256,
+                    help="reduced decode batch (profiling only; the reported workload uses 256)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -248,6 +247,10 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     hbm_peak, bf16_peak, peak_src = peaks()
+
+    if args.no_prefill:  # decode leg only (profiling)
+        print(json.dumps({"decode": run_decode(args, world, dev, stream, kda, hbm_peak)}), flush=True)
+        return
 
     # ---------------- prefill: long-context workload, resident in HBM ----------
     heads, T_run = args.heads, args.seq_len
@@ -341,7 +344,8 @@ def run_e2e(args, world, stream, inp, d, o, S, step, tokens_per_rank):
 
 def run_decode(args, world, dev, stream, kda, hbm_peak):
     """kda_decode_step on the decode workload (256 sequences, state in place)."""
-    dec = ki.workload(4)
+    dec = ki.workload(4) if args.decode_seqs == 256 else \
+        ki.make_decode(args.decode_seqs, H, torch.bfloat16, ki.BASE_SEED + 4)
     dd = {n: getattr(dec, n).to(dev) for n in ("state", "conv_cache", "q", "k", "v", "g", "beta", "conv_w")}
     o_dec = torch.empty(dd["q"].shape, dtype=torch.float32, device=dev)
 
