@@ -23,20 +23,24 @@
 // The diagonal terms beta_t v_t (of T V) and P_tt u_t (of P U) are applied in
 // fp32 by the scan kernel; they carry the largest single-token contributions.
 //
-// Gram blocks without overflow: tokens are grouped in 16-row blocks with
-// midpoint m_J = 16J + 8.  For i in block I and j <= i,
-//   e^{G_i - G_j} = [e^{G_i - G_{m_I}}] * [e^{G_{m_I} - G_{m_J}}] * [e^{G_{m_J} - G_j}]
-// where the outer factors stay within e^{+-40} (|g'| <= 5, <= 8 steps) and the
-// middle one is <= 1, so every operand is finite in fp32/tf32.  The tensor core
-// computes, per block row I, D_I[j][i'] = sum_c A_I[j][c] B_I[i'][c] with
-// A_I[j] = k_j e^{G_{m_I} - G_j} (j in blocks <= I, 0 elsewhere) and
-// B_I = [k_i; q_i] e^{G_i - G_{m_I}} for the 16 i of block I.
+// Gram blocks without overflow: the chunk is split into two 32-row halves b
+// with reference rows m_b = 32b + 16.  For i in half I and j <= i in half J,
+//   e^{G_i - G_j} = e^{G_i - G_{m_I}} * e^{G_{m_I} - G_j}
+// where |G_i - G_{m_I}| <= 5 * 16 = 80 (fp32 and tf32 reach e^88) and
+// e^{G_{m_I} - G_j} <= e^80 for j in half I, <= 1 for j in an earlier half.
+// The tensor core computes one M = 128 product per Gram, rows (A, K-major):
+//   0..31   k_j e^{G_{m_0} - G_j}, j = 0..31      (against half 0's columns)
+//   32..95  k_j e^{G_{m_1} - G_j}, j = 0..63      (against half 1's columns)
+//   96..127 not read back
+// and columns (B) [x_i e^{G_i - G_{m_0}}]_{i<32} | [x_i e^{G_i - G_{m_1}}]_{i>=32}
+// with x = q (the P Gram) or k (the M Gram); the wanted entries are the
+// row-0..31 x column-0..31 and row-32..95 x column-32..63 blocks.
 //
-// Block of 512 threads; thread (c, b) owns key/query channel c of token block
-// b (rows 16b..16b+15), so each block's midpoint factors stay in one thread.
-// The B operands of all four block rows are one tile written once (KQX); the
-// A operands are built per 32-channel slab into two alternating buffers while
-// the previous slab's MMAs run.
+// Two blocks of 256 threads share an SM (88 KB of shared memory and 256 TMEM
+// columns each), so that one block's barrier and tensor-core waits are covered
+// by the other's work.  Thread (c, b) owns key/query channel c of token half b;
+// the short-conv outputs of a chunk live in TMEM (lane = channel) rather than
+// in shared memory, and row norms are reduced with warp shuffles.
 #pragma once
 #include "kda_common.cuh"
 #include "kda_tc.cuh"
@@ -53,33 +57,60 @@ constexpr uint32_t REC_BYTES = 132096;
 constexpr uint32_t REC_TILES_A = REC_PS;              // B1 + QT: consumed by the first MMA group
 constexpr uint32_t REC_TILES_B = REC_BYTES - REC_PS;  // PS + KB + SC: second MMA group + scalars
 
-// shared memory plan (bytes from a 1024-aligned base); regions are reused
-// phase by phase
-constexpr int PREP_THREADS = 512;
-constexpr uint32_t P_RAW = 0;        // step 0-1: raw q, k, g tiles (3 x RAW_BYTES)
-                                     // step 5: Gram A operands, 2 buffers x 32 KB
-                                     // step 7: solve temporaries; step 8: T tile (16 KB) + K~^T tile (32 KB)
-constexpr uint32_t P_KQX = 65536;    // steps 1-3: conv(q), conv(k) row-major fp32 (2 x 32 KB)
-                                     // steps 3-8: KQX tile [128 rows x 128] (rows 32I..32I+15: k e^{G-G_m(I)},
-                                     //            rows 32I+16..32I+31: q e^{G-G_m(I)} of block I)
-constexpr uint32_t P_G = 131072;     // steps 1-3: Gamma row-major; steps 3-5: KE = k e^{G_m - G} row-major
-                                     // steps 6-8: diag(beta) M strict -> X (16 KB), P strict (16 KB)
-constexpr uint32_t P_MISC = 163840;  // scalars (12 KB)
-constexpr uint32_t PREP_SMEM = 176128 + 1024;
-
-// misc region (floats)
-constexpr int MS_BETA = 0, MS_RQ = 64, MS_RK = 128, MS_PD = 192, MS_GMID = 256 /*4x128*/,
-              MS_GC = 768 /*128*/, MS_Z = 896 /*6x128*/, MS_EGM = 1664 /*4x128*/, MS_CARRY = 2176 /*4x128*/;
-// ends at 2688 floats (10752 B) < 12 KB
-
-__device__ __forceinline__ int zidx(int I, int J) { return (I * (I - 1)) / 2 + J; }  // J < I
-
 // raw input tiles: 3 halo rows + 64 chunk rows of one head (128 bf16 = 256 B)
 constexpr int RAW_ROWS = CH + 3;
 constexpr uint32_t RAW_BYTES = RAW_ROWS * D * 2;  // 17152
 
+// shared memory plan (bytes from a 1024-aligned base); regions are reused
+// phase by phase
+constexpr int PREP_THREADS = 256;
+constexpr uint32_t P_RAW = 0;                // steps 0-1: raw q, k, g tiles (3 x RAW_BYTES)
+constexpr uint32_t P_GA = 0;                 // steps 3-5: Gram A tile, 4 slabs x 96 rows
+constexpr uint32_t GA_ROWS = 96;
+constexpr uint32_t P_GB = 49152;             // steps 3-5: Gram B tile, 4 slabs x 64 rows
+constexpr uint32_t MS_LD = 68;               // row stride (floats) of the solve matrix: rows
+                                             // 16-byte aligned, columns spread over all banks
+constexpr uint32_t P_MS = 0;                 // steps 6-7: diag(beta) M strict -> X, [64][68] fp32
+constexpr uint32_t P_TT = 17408;             // step 7: T tile [64 t][64 t'] (16 KB)
+constexpr uint32_t P_KT = 33792;             // step 7: K~^T tile [128 k][64 t] (32 KB)
+constexpr uint32_t P_TMP = 66560;            // step 6: solve temporaries (8 KB)
+constexpr uint32_t P_MISC = 81920;           // scalars (6 KB)
+constexpr uint32_t PREP_SMEM = P_MISC + 6144 + 1024;
+static_assert(P_GA + 3 * GA_ROWS * 128 + 128 * 128 <= P_MISC, "A tile reads past the Gram region");
+static_assert(3 * RAW_BYTES <= P_MISC && P_TMP + 8192 <= P_MISC, "shared regions overlap the scalars");
+static_assert(P_MS + 64 * MS_LD * 4 <= P_TT, "solve matrix overlaps the T tile");
+
+// scalar region (floats)
+constexpr int MB_BETA = 0, MB_RQ = 64, MB_RK = 128, MB_PD = 192, MB_CARRY = 256 /*128*/,
+              MB_G1M = 384 /*128*/, MB_G1T = 512 /*128*/, MB_PART = 640 /*2 x 4 x 3 x 32*/;
+static_assert((MB_PART + 768) * 4 <= 6144, "scalar region");
+
+// TMEM columns: short-conv outputs, then stashes and accumulators
+constexpr int TC_YQ = 0;    // conv(q) -> stash of k e^{G - G_m} (M Gram B operand)
+constexpr int TC_YK = 64;   // conv(k) -> stash of e^{G} k (W operand)
+constexpr int TC_G = 128;   // half-local cumulative gate
+constexpr int TC_DP = 128;  // P Gram accumulator (64 columns)
+constexpr int TC_DM = 192;  // M Gram accumulator (64 columns)
+constexpr int TC_W = 128;   // W accumulator (M = 64, 128 columns)
+
+// Sum over the 32 lanes of a warp of 16 per-lane vectors; lane l returns the
+// total of entry l % 16 (recursive halving: 16 shuffles instead of 16 x 5).
+__device__ __forceinline__ float lane_reduce16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int m = 8; m >= 1; m >>= 1) {
+    const bool up = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < m; ++i) {
+      const float send = up ? v[i] : v[i + m];
+      const float keep = up ? v[i + m] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
+}
+
 template <int ACT>
-__global__ void __launch_bounds__(PREP_THREADS, 1)
+__global__ void __launch_bounds__(PREP_THREADS, 2)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16* __restrict__ beta,
                   const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ init_conv,
@@ -87,18 +118,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   int n_items, uint8_t* __restrict__ records) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  float* Yq = (float*)(sm + P_KQX);
-  float* Yk = (float*)(sm + P_KQX + 32768);
-  uint8_t* kqx = sm + P_KQX;
-  float* Gm = (float*)(sm + P_G);  // Gamma, then KE
-  float* Ms = (float*)(sm + P_G);
-  float* Ps = (float*)(sm + P_G + 16384);
   float* ms = (float*)(sm + P_MISC);
-  __shared__ uint64_t bar_ld, bar_g[2], bar_w;
+  float* Ms = (float*)(sm + P_MS);
+  __shared__ uint64_t bar_ld, bar_p, bar_m, bar_w;
   __shared__ uint32_t tmem_base;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ch = tid & 127, blk = tid >> 7;  // channel, 16-row token block
+  const int ch = tid & 127, hb = tid >> 7;  // channel, 32-row half of the chunk
+  const int q4 = warp & 3;                  // TMEM lane quarter (= ch / 32)
+  const int r0 = 32 * hb;                   // first row of this thread's half
   const int64_t HD = (int64_t)H * D;
   const __nv_bfloat16* rq_t = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW);
   const __nv_bfloat16* rk_t = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + RAW_BYTES);
@@ -118,8 +146,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // ---- 0. once per block: TMEM, barriers, first item's tiles ----------------
   if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
   if (tid == 0) {
-    tc::bar_init(&bar_ld, 1); tc::bar_init(&bar_g[0], 1); tc::bar_init(&bar_g[1], 1);
-    tc::bar_init(&bar_w, 1);
+    tc::bar_init(&bar_ld, 1); tc::bar_init(&bar_p, 1); tc::bar_init(&bar_m, 1); tc::bar_init(&bar_w, 1);
     tc::bar_init_fence();
     if ((int)blockIdx.x < n_items) load_raw(blockIdx.x);
   }
@@ -127,7 +154,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc::fence_after();
   const uint32_t tm = tmem_base;
-  uint32_t par = 0;  // phase parity of the per-item barriers (bar_ld, bar_w)
+  const uint32_t tl = tm + ((uint32_t)(32 * q4) << 16);  // this warp's TMEM lanes
+  uint32_t par = 0;  // phase parity of the per-item barriers
 
   // persistent loop over (chunk, head) work items, chunk-major
   for (int item = blockIdx.x; item < n_items; item += gridDim.x, par ^= 1) {
@@ -139,13 +167,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int L = (int)((seg1 - t0) < CH ? (seg1 - t0) : CH);
   const int64_t chan = (int64_t)h * D + ch;
   uint8_t* rec = records + ((int64_t)cid * H + h) * REC_BYTES;
-  if (tid < CH) ms[MS_BETA + tid] = tid < L ? to_f(beta[(t0 + tid) * H + h]) : 0.f;
+  if (tid < CH) ms[MB_BETA + tid] = tid < L ? to_f(beta[(t0 + tid) * H + h]) : 0.f;
   const float4 wq = load4(conv_w + (0 * HD + chan) * 4);
   const float4 wk = load4(conv_w + (1 * HD + chan) * 4);
   tc::bar_wait(&bar_ld, par);
 
-  // ---- 1. causal conv of q, k and block-local cumsum of the clamped gate ----
-  const int r0 = 16 * blk;
+  // ---- 1. causal conv of q, k; half-local cumsum of the clamped gate; the
+  //         row sums |q|^2, |k|^2, q.k over this warp's 32 channels ----------
+  float gm_loc;  // half-local cumulative gate through row r0 + 16
   {
     float hq[3], hk[3];
 #pragma unroll
@@ -163,299 +192,342 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       hq[j] = a; hk[j] = b;
     }
     float cum = 0.f;
+    gm_loc = 0.f;
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const int t = r0 + r;
-      const float xq = to_f(rq_t[(t + 3) * D + ch]), xk = to_f(rk_t[(t + 3) * D + ch]);
-      float yq = conv4(wq, hq[0], hq[1], hq[2], xq);
-      float yk = conv4(wk, hk[0], hk[1], hk[2], xk);
-      if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
-      hq[0] = hq[1]; hq[1] = hq[2]; hq[2] = xq;
-      hk[0] = hk[1]; hk[1] = hk[2]; hk[2] = xk;
-      const bool valid = t < L;
-      cum += valid ? fmaxf(to_f(rg_t[(t + 3) * D + ch]), LOG_DECAY_FLOOR) : 0.f;
-      Yq[t * D + ch] = valid ? yq : 0.f;
-      Yk[t * D + ch] = valid ? yk : 0.f;
-      Gm[t * D + ch] = cum;
+    for (int g = 0; g < 2; ++g) {
+      float yq[16], yk[16], gl[16], sq[16], sk[16], sx[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const int t = r0 + 16 * g + r;
+        const float xq = to_f(rq_t[(t + 3) * D + ch]), xk = to_f(rk_t[(t + 3) * D + ch]);
+        float a = conv4(wq, hq[0], hq[1], hq[2], xq);
+        float b = conv4(wk, hk[0], hk[1], hk[2], xk);
+        if (ACT == KDA_CONV_SILU) { a = silu(a); b = silu(b); }
+        hq[0] = hq[1]; hq[1] = hq[2]; hq[2] = xq;
+        hk[0] = hk[1]; hk[1] = hk[2]; hk[2] = xk;
+        const bool valid = t < L;
+        cum += valid ? fmaxf(to_f(rg_t[(t + 3) * D + ch]), LOG_DECAY_FLOOR) : 0.f;
+        yq[r] = valid ? a : 0.f;
+        yk[r] = valid ? b : 0.f;
+        gl[r] = cum;
+        sq[r] = yq[r] * yq[r]; sk[r] = yk[r] * yk[r]; sx[r] = yq[r] * yk[r];
+      }
+      if (g == 1) gm_loc = gl[0];
+      tc::st16(tl + TC_YQ + r0 + 16 * g, yq);
+      tc::st16(tl + TC_YK + r0 + 16 * g, yk);
+      tc::st16(tl + TC_G + r0 + 16 * g, gl);
+      const float nq = lane_reduce16(sq, lane), nk = lane_reduce16(sk, lane), nx = lane_reduce16(sx, lane);
+      if (lane < 16) {
+        float* part = ms + MB_PART + (hb * 4 + q4) * 96 + 16 * g + lane;
+        part[0] = nq; part[32] = nk; part[64] = nx;
+      }
     }
-    ms[MS_CARRY + blk * D + ch] = cum;  // this block's total
+    ms[(hb ? MB_G1T : MB_CARRY) + ch] = cum;  // half totals
+    if (hb) ms[MB_G1M + ch] = gm_loc;
+  }
+  tc::st_wait();
+  __syncthreads();
+
+  // ---- 2. inverse row norms and the exact diagonal q_hat . k_hat ------------
+  if (tid < CH) {
+    const int hh = tid >> 5, rr = tid & 31;
+    float nq = 0.f, nk = 0.f, nx = 0.f;
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      const float* part = ms + MB_PART + (hh * 4 + c4) * 96 + rr;
+      nq += part[0]; nk += part[32]; nx += part[64];
+    }
+    const float rq = 1.0f / sqrtf(nq + NORM_EPS), rk = 1.0f / sqrtf(nk + NORM_EPS);
+    ms[MB_RQ + tid] = rq; ms[MB_RK + tid] = rk; ms[MB_PD + tid] = nx * rq * rk;
   }
   __syncthreads();
 
-  // ---- 2. L2 norms (warp per 4 rows) -----------------------------------------
-#pragma unroll
-  for (int t = warp * 4; t < warp * 4 + 4; ++t) {
-    const float4 a = *reinterpret_cast<const float4*>(&Yq[t * D + lane * 4]);
-    const float4 b = *reinterpret_cast<const float4*>(&Yk[t * D + lane * 4]);
-    float nq = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
-    float nk = b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
-    float qk = a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
-    nq = warp_sum(nq); nk = warp_sum(nk); qk = warp_sum(qk);
-    if (lane == 0) {
-      const float rq = 1.0f / sqrtf(nq + NORM_EPS), rk = 1.0f / sqrtf(nk + NORM_EPS);
-      ms[MS_RQ + t] = rq; ms[MS_RK + t] = rk; ms[MS_PD + t] = qk * rq * rk;
-    }
-  }
-  __syncthreads();
-
-  // ---- 3. normalise; factors about this block's midpoint ---------------------
-  // e_t = e^{G_t - G_mid} within [e^-40, e^40]; KX = k e, QX = q e (B operands),
-  // KE = k / e (A operand base), QT = e^{G_mid} QX (record)
-  float kx[16], qx[16];
+  // ---- 3. normalise; Gram operands, record tiles QT and KB, stashes ---------
+  const float carry = hb ? ms[MB_CARRY + ch] : 0.f;         // gate total of half 0
+  const float g1m = ms[MB_CARRY + ch] + ms[MB_G1M + ch];     // G at row 48
+  const float gC = ms[MB_CARRY + ch] + ms[MB_G1T + ch];      // G at the chunk end
   {
-    float carry = 0.f;
-    for (int b = 0; b < blk; ++b) carry += ms[MS_CARRY + b * D + ch];
-    float G[16];
+    const float gm = hb ? g1m : gm_loc;                      // this half's reference G_m
+    const float egcm = __expf(gC - g1m);                     // half 1: e^{G_C - G_m}, <= 1
 #pragma unroll
-    for (int r = 0; r < 16; ++r) G[r] = Gm[(r0 + r) * D + ch] + carry;
-    const float gmid = G[8];
-    ms[MS_GMID + blk * D + ch] = gmid;
-    if (blk == 3) ms[MS_GC + ch] = G[15];
-    const float egm = __expf(gmid);
-    ms[MS_EGM + blk * D + ch] = egm;
+    for (int g = 0; g < 4; ++g) {  // 8-row groups
+      float yq[8], yk[8], gl[8];
+      tc::ld8(tl + TC_YQ + r0 + 8 * g, yq);
+      tc::ld8(tl + TC_YK + r0 + 8 * g, yk);
+      tc::ld8(tl + TC_G + r0 + 8 * g, gl);
+      tc::ld_wait();
+      float kb[8];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const int t = r0 + r;
-      const float e = __expf(G[r] - gmid);
-      const float kh = Yk[t * D + ch] * ms[MS_RK + t], qh = Yq[t * D + ch] * ms[MS_RQ + t];
-      kx[r] = kh * e;
-      qx[r] = qh * e;
-      Gm[t * D + ch] = kh / e;  // KE (own element)
-      // QT tile image staged in the raw region (its tiles were consumed in step 1)
-      *reinterpret_cast<float*>(sm + P_RAW + tc::sw128(t, ch, 64)) = tc::to_tf32(egm * qx[r]);
+      for (int r = 0; r < 8; ++r) {
+        const int t = r0 + 8 * g + r;
+        const float G = gl[r] + carry;
+        const float d = G - gm;
+        const float e1 = __expf(d), e2 = __expf(-d), e3 = __expf(G);
+        const float kh = yk[r] * ms[MB_RK + t], qh = yq[r] * ms[MB_RQ + t];
+        // B operand of the P Gram; A rows (block of the own half, and for
+        // half 0 the rows read against half 1)
+        *reinterpret_cast<float*>(sm + P_GB + tc::sw128(t, ch, 64)) = tc::to_tf32(qh * e1);
+        // e^{G_{m_1} - G_t}: e2 for half 1; <= 1 for half 0
+        const float a1 = hb ? e2 : __expf(g1m - G);
+        *reinterpret_cast<float*>(sm + P_GA + tc::sw128(32 + t, ch, GA_ROWS)) = tc::to_tf32(kh * a1);
+        if (!hb) *reinterpret_cast<float*>(sm + P_GA + tc::sw128(t, ch, GA_ROWS)) = tc::to_tf32(kh * e2);
+        *reinterpret_cast<float*>(rec + REC_QT + tc::sw128(t, ch, 64)) = tc::to_tf32(qh * e3);
+        // e^{G_C - G_t} = e^{G_C - G_{m_1}} e^{G_{m_1} - G_t}: for half 0 both
+        // factors are <= 1 (an underflow only drops what is below fp32 anyway)
+        kb[r] = tc::to_tf32(kh * (egcm * a1));
+        yq[r] = kh * e1;  // stash: M Gram B operand
+        yk[r] = kh * e3;  // stash: e^{G} k for W
+      }
+      tc::st8(tl + TC_YQ + r0 + 8 * g, yq);
+      tc::st8(tl + TC_YK + r0 + 8 * g, yk);
+      // KB row ch, columns r0 + 8g .. +7
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        *reinterpret_cast<float4*>(rec + REC_KB + tc::sw128(ch, r0 + 8 * g + 4 * j, 128)) =
+            make_float4(kb[4 * j], kb[4 * j + 1], kb[4 * j + 2], kb[4 * j + 3]);
     }
   }
   tc::fence_async_smem();
-  __syncthreads();  // conv(q), conv(k) are read; the KQX tile may overwrite them
-  if (tid == 0) {
-    tc::bulk_s2g(rec + REC_QT, sm + P_RAW, 32768);
-    tc::bulk_commit();
-  }
-#pragma unroll
-  for (int r = 0; r < 16; ++r) {
-    *reinterpret_cast<float*>(kqx + tc::sw128(32 * blk + r, ch, 128)) = tc::to_tf32(kx[r]);
-    *reinterpret_cast<float*>(kqx + tc::sw128(32 * blk + 16 + r, ch, 128)) = tc::to_tf32(qx[r]);
-  }
+  tc::st_wait();
+  tc::fence_before();
   __syncthreads();
 
-  // ---- 4. block-to-block factors; record tiles KB and scalars ----------------
-  {
-    const float gc = ms[MS_GC + ch], gm = ms[MS_GMID + blk * D + ch];
-    for (int J = 0; J < blk; ++J) ms[MS_Z + zidx(blk, J) * D + ch] = __expf(gm - ms[MS_GMID + J * D + ch]);
-    const float egc = __expf(gc - gm);  // e^{G_C - G_mid}
-    float kb[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) kb[r] = tc::to_tf32(egc * Gm[(r0 + r) * D + ch]);
-    // row ch of KB, columns r0..r0+15 (half of a 128-byte slab row)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      *reinterpret_cast<float4*>(rec + REC_KB + tc::sw128(ch, r0 + 4 * j, 128)) =
-          make_float4(kb[4 * j], kb[4 * j + 1], kb[4 * j + 2], kb[4 * j + 3]);
-    float* sc = reinterpret_cast<float*>(rec + REC_SC);
-    if (tid < CH) { sc[tid] = ms[MS_BETA + tid]; sc[64 + tid] = ms[MS_PD + tid]; }
-    if (blk == 0) sc[128 + ch] = __expf(gc);
-  }
-  if (tid == 0) tc::bulk_wait_read();  // the QT staging may be overwritten after this
-  __syncthreads();
-
-  // ---- 5. gated Gram blocks on the tensor core --------------------------------
-  // pass kp covers channels 32kp..32kp+31.  Block rows are paired: pair p
-  // stacks A_{2p} (rows 0..63) over A_{2p+1} (rows 64..127) into one M = 128
-  // operand against B = KQX rows 64p..64p+63 (= B_{2p} | B_{2p+1}, N = 64); the
-  // wanted products are the two diagonal 64 x 32 quadrants.  A_I rows j of
-  // blocks J <= I are written (other rows are never read back).
-  auto build_a = [&](int kp) {
-    uint8_t* buf = sm + P_RAW + (kp & 1) * 32768;
-    // (I, j, 4-channel group) with J(j) <= I: 160 rows x 8 groups
-    for (int e = tid; e < 160 * 8; e += PREP_THREADS) {
-      const int c4 = e & 7, rr = e >> 3;  // rr in [0, 160): I-major rows
-      const int I = rr < 16 ? 0 : rr < 48 ? 1 : rr < 96 ? 2 : 3;
-      const int j = rr - (I == 0 ? 0 : I == 1 ? 16 : I == 2 ? 48 : 96);
-      const int J = j >> 4, c = 32 * kp + 4 * c4;
-      float4 v = *reinterpret_cast<const float4*>(&Gm[j * D + c]);
-      if (J < I) {
-        const float4 z = *reinterpret_cast<const float4*>(&ms[MS_Z + zidx(I, J) * D + c]);
-        v.x *= z.x; v.y *= z.y; v.z *= z.z; v.w *= z.w;
-      }
-      v = make_float4(tc::to_tf32(v.x), tc::to_tf32(v.y), tc::to_tf32(v.z), tc::to_tf32(v.w));
-      *reinterpret_cast<float4*>(buf + (I >> 1) * 16384 + tc::sw128((I & 1) * 64 + j, 4 * c4, 128)) = v;
-    }
-    tc::fence_async_smem();
-  };
-  auto issue_gram = [&](int kp) {
+  // ---- 4. P Gram (A = GA, B = q operand) -------------------------------------
+  const uint64_t d_ga = tc::desc(tc::smem_u32(sm + P_GA)), d_gb = tc::desc(tc::smem_u32(sm + P_GB));
+  auto issue_gram = [&](uint32_t dcol, uint64_t* bar) {
     tc::fence_after();
-    const uint64_t da = tc::desc(tc::smem_u32(sm + P_RAW + (kp & 1) * 32768));
-    const uint64_t db = tc::desc(tc::smem_u32(kqx + kp * 16384));
 #pragma unroll
-    for (int pr = 0; pr < 2; ++pr)
+    for (int s = 0; s < 4; ++s)
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
-        tc::mma_ss(tm + 64 * pr, da + ((pr * 16384) >> 4) + tc::desc_step(128, ks),
-                   db + ((pr * 64 * 128) >> 4) + tc::desc_step(128, ks), tc::idesc_tf32(128, 64),
-                   (kp > 0 || ks > 0) ? 1 : 0);
-    tc::commit(&bar_g[kp & 1]);
+        tc::mma_ss(tm + dcol, d_ga + ((s * GA_ROWS * 128) >> 4) + tc::desc_step(0, ks),
+                   d_gb + ((s * 64 * 128) >> 4) + tc::desc_step(0, ks), tc::idesc_tf32(128, 64),
+                   (s | ks) ? 1 : 0);
+    tc::commit(bar);
   };
-  build_a(0);
-  tc::fence_before();
-  __syncthreads();
-  if (tid == 0) issue_gram(0);
-  build_a(1);
-  tc::fence_before();
-  __syncthreads();
-  if (tid == 0) issue_gram(1);
-  tc::bar_wait(&bar_g[0], 0);  // pass 0 done: buffer 0 free
-  build_a(2);
-  tc::fence_before();
-  __syncthreads();
-  if (tid == 0) issue_gram(2);
-  tc::bar_wait(&bar_g[1], 0);  // pass 1 done: buffer 1 free
-  build_a(3);
-  tc::fence_before();
-  __syncthreads();
-  if (tid == 0) issue_gram(3);
-  tc::bar_wait(&bar_g[1], 1);  // pass 3 done
-  tc::bar_wait(&bar_g[0], 1);  // pass 2 done (each item uses two phases of each barrier)
+  if (tid == 0) issue_gram(TC_DP, &bar_p);
+  tc::bar_wait(&bar_p, par);
   tc::fence_after();
-
-  // ---- 6. read the diagonal quadrants (M = 128 layout: row m -> lane m) ------
-  {
-    const int sub = warp & 3, pr = (warp >> 2) & 1, part = warp >> 3;  // part 0: M columns, 1: P columns
-    const int m = 32 * sub + lane;       // accumulator row
-    const int I = 2 * pr + (m >> 6);     // block row
-    const int j = m & 63;
-    float v[16];
-    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 64 * pr + 32 * (m >> 6) + 16 * part, v);
-    tc::ld_wait();
-    float* dst = part == 0 ? Ms : Ps;
+  // the B tile is free: k operand of the M Gram from the stash
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const int i = 16 * I + r;
-      dst[i * CH + j] = i > j ? (part == 0 ? ms[MS_BETA + i] * v[r] : v[r]) : 0.f;  // diag(beta) M / P, strict
+  for (int g = 0; g < 2; ++g) {
+    float kx[16];
+    tc::ld16(tl + TC_YQ + r0 + 16 * g, kx);
+    tc::ld_wait();
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+      *reinterpret_cast<float*>(sm + P_GB + tc::sw128(r0 + 16 * g + r, ch, 64)) = tc::to_tf32(kx[r]);
+  }
+  tc::fence_async_smem();
+  tc::fence_before();
+  __syncthreads();
+  if (tid == 0) issue_gram(TC_DM, &bar_m);
+
+  // ---- 5. P into the record (while the M Gram runs) ---------------------------
+  // accumulator row m = TMEM lane: A row (j = m for m < 32, j = m - 32 for
+  // 32 <= m < 96); column n = query row i.  Warp (q4, hb) reads lanes of
+  // quarter q4, columns 16 hb .. of the half that quarter pairs with.
+  {
+    const int j = q4 == 2 ? 32 + lane : (q4 == 3 ? 32 + lane : lane);
+    const int ib = (q4 == 0 || q4 == 3 ? 0 : 32) + 16 * hb;  // first query row
+    float v[16];
+    if (q4 < 3) {
+      tc::ld16(tl + TC_DP + ib, v);
+      tc::ld_wait();
+    }
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i = ib + c;
+      const float p = (q4 < 3 && i > j) ? v[c] : 0.f;  // strictly lower part; quarter 3 writes the zero block
+      *reinterpret_cast<float*>(rec + REC_PS + tc::sw128(i, j, 64)) = tc::to_tf32(p);
+    }
+  }
+  tc::bar_wait(&bar_m, par);
+  tc::fence_after();
+  // ---- 5b. diag(beta) M (strictly lower) into the solve matrix ----------------
+  if (q4 < 3) {
+    const int j = q4 == 2 ? 32 + lane : lane;
+    const int ib = (q4 == 0 ? 0 : 32) + 16 * hb;
+    float v[16];
+    tc::ld16(tl + TC_DM + ib, v);
+    tc::ld_wait();
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const int i = ib + c;
+      Ms[i * MS_LD + j] = i > j ? ms[MB_BETA + i] * v[c] : 0.f;
     }
   }
   __syncthreads();
 
-  // ---- 7. X = (I + diag(beta) M)^-1, blocked forward substitution -------------
-  float* Xd = (float*)(sm + P_RAW);         // [4][16][16] inverses of the diagonal blocks
-  float* Yb = (float*)(sm + P_RAW) + 1024;  // [3][16][16]
+  // ---- 6. X = (I + diag(beta) M)^-1 (unit lower triangular) ------------------
+  // diagonal 16-blocks by forward substitution, then the off-diagonal 16-blocks
+  // of each 32-half, then the off-diagonal 32-block:
+  //   X_ba = -X_bb L_ba X_aa  for the 2 x 2 block partition at each level.
+  // Every entry above the diagonal inside each 32-half is 0 (written so by the
+  // readout and by the diagonal-block copy), so the products run over full
+  // block widths.
+  float* Xd = (float*)(sm + P_TMP);         // [4][16][16] inverses of the diagonal 16-blocks
+  float* Yt = (float*)(sm + P_TMP) + 1024;  // [32][32] temporary
   if (tid < 64) {
     const int I = tid >> 4, cc = tid & 15;  // column cc of X_II
+    const float* Lb = Ms + (16 * I) * MS_LD + 16 * I;
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
       float s = (r == cc) ? 1.f : 0.f;
 #pragma unroll
-      for (int m = 0; m < r; ++m) s -= Ms[(16 * I + r) * CH + 16 * I + m] * x[m];
+      for (int m4 = 0; m4 < r; m4 += 4) {
+        const float4 l = *reinterpret_cast<const float4*>(Lb + r * MS_LD + m4);
+        s -= l.x * x[m4];
+        if (m4 + 1 < r) s -= l.y * x[m4 + 1];
+        if (m4 + 2 < r) s -= l.z * x[m4 + 2];
+        if (m4 + 3 < r) s -= l.w * x[m4 + 3];
+      }
       x[r] = r < cc ? 0.f : s;
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) Xd[(I * 16 + r) * 16 + cc] = x[r];
   }
   __syncthreads();
+  {  // Y = L_{2P+1,2P} X_{2P,2P} for P = 0, 1 (16 x 16 each)
+    const int r = (tid >> 4) & 15, cc = tid & 15;
 #pragma unroll
-  for (int I = 1; I < 4; ++I) {
-    // Y_IJ = sum_{K=J}^{I-1} L_IK X_KJ  for J < I (X_KJ already in Ms for K < I)
-    for (int e = tid; e < I * 256; e += PREP_THREADS) {
-      const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-      const float* Lrow = Ms + (16 * I + r) * CH;
+    for (int P = 0; P < 2; ++P) {
+      const float* Lr = Ms + (32 * P + 16 + r) * MS_LD + 32 * P;
+      const float* X0 = Xd + (2 * P) * 256;
       float s = 0.f;
 #pragma unroll
-      for (int m = 0; m < 16; ++m) s += Lrow[16 * J + m] * Xd[(J * 16 + m) * 16 + cc];
-      for (int K = J + 1; K < I; ++K) {
-#pragma unroll
-        for (int m = 0; m < 16; ++m) s += Lrow[16 * K + m] * Ms[(16 * K + m) * CH + 16 * J + cc];
+      for (int m4 = 0; m4 < 16; m4 += 4) {
+        const float4 l = *reinterpret_cast<const float4*>(Lr + m4);
+        s += l.x * X0[m4 * 16 + cc] + l.y * X0[(m4 + 1) * 16 + cc] + l.z * X0[(m4 + 2) * 16 + cc] +
+             l.w * X0[(m4 + 3) * 16 + cc];
       }
-      Yb[(J * 16 + r) * 16 + cc] = s;
+      Yt[(P * 16 + r) * 16 + cc] = s;
     }
-    __syncthreads();
-    // X_IJ = -X_II Y_IJ, written over L_IJ
-    for (int e = tid; e < I * 256; e += PREP_THREADS) {
-      const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+  }
+  __syncthreads();
+  {  // X_{2P+1,2P} = -X_{2P+1,2P+1} Y; diagonal blocks copied into the matrix
+    const int r = (tid >> 4) & 15, cc = tid & 15;
+#pragma unroll
+    for (int P = 0; P < 2; ++P) {
+      const float* X1 = Xd + (2 * P + 1) * 256 + r * 16;
       float s = 0.f;
 #pragma unroll
-      for (int m = 0; m < 16; ++m) s += Xd[(I * 16 + r) * 16 + m] * Yb[(J * 16 + m) * 16 + cc];
-      Ms[(16 * I + r) * CH + 16 * J + cc] = -s;
+      for (int m4 = 0; m4 < 16; m4 += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(X1 + m4);
+        s += x.x * Yt[(P * 16 + m4) * 16 + cc] + x.y * Yt[(P * 16 + m4 + 1) * 16 + cc] +
+             x.z * Yt[(P * 16 + m4 + 2) * 16 + cc] + x.w * Yt[(P * 16 + m4 + 3) * 16 + cc];
+      }
+      Ms[(32 * P + 16 + r) * MS_LD + 32 * P + cc] = -s;
     }
-    __syncthreads();
+#pragma unroll
+    for (int I = 0; I < 4; ++I) Ms[(16 * I + r) * MS_LD + 16 * I + cc] = Xd[(I * 16 + r) * 16 + cc];
   }
-  // diagonal blocks into Ms; Ms now holds X (unit lower triangular)
-  for (int e = tid; e < 4 * 256; e += PREP_THREADS) {
-    const int I = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-    Ms[(16 * I + r) * CH + 16 * I + cc] = Xd[(I * 16 + r) * 16 + cc];
+  __syncthreads();
+  // 32-level products: thread (warp, lane) computes rows warp + 8k (k < 4) of
+  // column lane, so each column operand load serves four rows
+  auto prod32 = [&](const float* A, int lda, const float* B, int ldb, float (&s)[4]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s[k] = 0.f;
+#pragma unroll
+    for (int m4 = 0; m4 < 32; m4 += 4) {
+      const float b0 = B[m4 * ldb + lane], b1 = B[(m4 + 1) * ldb + lane], b2 = B[(m4 + 2) * ldb + lane],
+                  b3 = B[(m4 + 3) * ldb + lane];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 a = *reinterpret_cast<const float4*>(A + (warp + 8 * k) * lda + m4);
+        s[k] += a.x * b0 + a.y * b1 + a.z * b2 + a.w * b3;
+      }
+    }
+  };
+  {  // Y = L_{10} X_{00}: rows 32..63, columns 0..31
+    float s[4];
+    prod32(Ms + 32 * MS_LD, MS_LD, Ms, MS_LD, s);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) Yt[(warp + 8 * k) * 32 + lane] = s[k];
+  }
+  __syncthreads();
+  {  // X_{10} = -X_{11} Y
+    float s[4];
+    prod32(Ms + 32 * MS_LD + 32, MS_LD, Yt, 32, s);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) Ms[(32 + warp + 8 * k) * MS_LD + lane] = -s[k];
   }
   __syncthreads();
 
-  // ---- 8. T = X diag(beta); tiles for W = T K~ and the record's T_s, P_s -----
-  uint8_t* tT = sm + P_RAW;          // [64 t][64 t'] tile, 16 KB
-  uint8_t* tK = sm + P_RAW + 16384;  // [128 k][64 t'] tile (K~^T), 32 KB
+  // ---- 7. T = X diag(beta): record T_s, T tile; K~^T tile; W = T K~ ----------
   for (int e = tid; e < CH * 16; e += PREP_THREADS) {  // 4-column groups
     const int t = e >> 4, tp = 4 * (e & 15);
-    float4 tv, pv;
+    float4 tv, ts;
     float* tvp = &tv.x;
-    float* pvp = &pv.x;
+    float* tsp = &ts.x;
+    const float4 xr = *reinterpret_cast<const float4*>(Ms + t * MS_LD + tp);
+    const float* xrp = &xr.x;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = tp + u;
-      tvp[u] = tc::to_tf32(c <= t ? Ms[t * CH + c] * ms[MS_BETA + c] : 0.f);
-      pvp[u] = tc::to_tf32(Ps[t * CH + c]);
+      const float x = c < t ? xrp[u] : (c == t ? 1.f : 0.f);
+      tvp[u] = tc::to_tf32(x * ms[MB_BETA + c]);
+      tsp[u] = c < t ? tvp[u] : 0.f;
     }
-    *reinterpret_cast<float4*>(tT + tc::sw128(t, tp, 64)) = tv;
-    float4 ts = tv;
-    float* tsp = &ts.x;
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (tp + u >= t) tsp[u] = 0.f;  // strictly lower part only
+    *reinterpret_cast<float4*>(sm + P_TT + tc::sw128(t, tp, 64)) = tv;
     *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, tp, 64)) = ts;
-    *reinterpret_cast<float4*>(rec + REC_PS + tc::sw128(t, tp, 64)) = pv;
   }
-  {
-    // K~^T row ch, columns r0..r0+15: e^{G_t} k_t = e^{G_mid} * KX
-    const float egm = ms[MS_EGM + blk * D + ch];
-    float kt[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r)
-      kt[r] = tc::to_tf32(egm * *reinterpret_cast<const float*>(kqx + tc::sw128(32 * blk + r, ch, 128)));
+  for (int g = 0; g < 2; ++g) {  // K~^T row ch, columns r0 + 16g ..
+    float kt[16];
+    tc::ld16(tl + TC_YK + r0 + 16 * g, kt);
+    tc::ld_wait();
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      *reinterpret_cast<float4*>(tK + tc::sw128(ch, r0 + 4 * j, 128)) =
-          make_float4(kt[4 * j], kt[4 * j + 1], kt[4 * j + 2], kt[4 * j + 3]);
+      *reinterpret_cast<float4*>(sm + P_KT + tc::sw128(ch, r0 + 16 * g + 4 * j, 128)) =
+          make_float4(tc::to_tf32(kt[4 * j]), tc::to_tf32(kt[4 * j + 1]), tc::to_tf32(kt[4 * j + 2]),
+                      tc::to_tf32(kt[4 * j + 3]));
   }
   tc::fence_async_smem();
   tc::fence_before();
   __syncthreads();
   if (tid == 0) {
     tc::fence_after();
-    const uint64_t dt = tc::desc(tc::smem_u32(tT)), dk = tc::desc(tc::smem_u32(tK));
+    const uint64_t dt = tc::desc(tc::smem_u32(sm + P_TT)), dk = tc::desc(tc::smem_u32(sm + P_KT));
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks)
-      tc::mma_ss(tm + 128, dt + tc::desc_step(64, ks), dk + tc::desc_step(128, ks), tc::idesc_tf32(64, 128),
+      tc::mma_ss(tm + TC_W, dt + tc::desc_step(64, ks), dk + tc::desc_step(128, ks), tc::idesc_tf32(64, 128),
                  ks > 0 ? 1 : 0);
     tc::commit(&bar_w);
   }
+  {  // scalars of the record
+    float* sc = reinterpret_cast<float*>(rec + REC_SC);
+    if (tid < CH) { sc[tid] = ms[MB_BETA + tid]; sc[64 + tid] = ms[MB_PD + tid]; }
+    if (hb == 0) sc[128 + ch] = __expf(gC);
+  }
   tc::bar_wait(&bar_w, par);
   tc::fence_after();
-  // the raw region (T and K~^T tiles) is free: fetch the next item's tiles
-  // while this item finishes
+  // the shared regions are free: fetch the next item's tiles while this one finishes
   __syncthreads();
   if (tid == 0 && item + (int)gridDim.x < n_items) load_raw(item + gridDim.x);
 
-  // ---- 9. -W rows into the record (columns 64..191 of B1) --------------------
+  // ---- 8. -W rows into the record (columns 64..191 of B1) --------------------
+  // M = 64 accumulator: row t in lane 16 * (t / 16) ... of quarter t / 16
   {
-    const int sub = warp & 3, cb = warp >> 2;  // rows 16sub.., columns 32cb..32cb+31
-    const int t = 16 * sub + (lane & 15);
-    float w0[16], w1[16];
-    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 128 + 32 * cb, w0);
-    tc::ld16(tm + ((uint32_t)(32 * sub) << 16) + 128 + 32 * cb + 16, w1);
-    tc::ld_wait();
-    if (lane < 16) {
+    const int t = 16 * q4 + (lane & 15);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + 32 * cb + 4 * j, 64)) =
-            make_float4(tc::to_tf32(-w0[4 * j]), tc::to_tf32(-w0[4 * j + 1]), tc::to_tf32(-w0[4 * j + 2]),
-                        tc::to_tf32(-w0[4 * j + 3]));
-        *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + 32 * cb + 16 + 4 * j, 64)) =
-            make_float4(tc::to_tf32(-w1[4 * j]), tc::to_tf32(-w1[4 * j + 1]), tc::to_tf32(-w1[4 * j + 2]),
-                        tc::to_tf32(-w1[4 * j + 3]));
+    for (int part = 0; part < 2; ++part) {
+      float w0[16], w1[16];
+      const int c0 = 64 * hb + 32 * part;
+      tc::ld16(tl + TC_W + c0, w0);
+      tc::ld16(tl + TC_W + c0 + 16, w1);
+      tc::ld_wait();
+      if (lane < 16) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + c0 + 4 * j, 64)) =
+              make_float4(tc::to_tf32(-w0[4 * j]), tc::to_tf32(-w0[4 * j + 1]), tc::to_tf32(-w0[4 * j + 2]),
+                          tc::to_tf32(-w0[4 * j + 3]));
+          *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + c0 + 16 + 4 * j, 64)) =
+              make_float4(tc::to_tf32(-w1[4 * j]), tc::to_tf32(-w1[4 * j + 1]), tc::to_tf32(-w1[4 * j + 2]),
+                          tc::to_tf32(-w1[4 * j + 3]));
+        }
       }
     }
   }
@@ -463,7 +535,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();  // TMEM columns and shared regions are reused by the next item
   tc::fence_after();
   }  // item loop
-  if (tid == 0) tc::bulk_wait_all();
   tc::fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem_base, 256);

@@ -77,13 +77,13 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     auto prep = chunk_prep_kernel<ACT>;
     if (cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess)
       return KDA_ERR_CUDA;
-    // persistent blocks, one per SM, over the (chunk, head) items
+    // persistent blocks, two per SM, over the (chunk, head) items
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return KDA_ERR_CUDA;
     const int64_t items = total * H;
-    const unsigned blocks = (unsigned)(items < sms ? items : sms);
+    const unsigned blocks = (unsigned)(items < 2 * sms ? items : 2 * sms);
     prep<<<blocks, PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w, (const T*)init_conv,
                                                         cu_dev, d_tab, H, (int)items, records);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
