@@ -15,10 +15,13 @@
 //
 // Record (REC_BYTES, 1024-aligned), all tiles fp32 values rounded to tf32,
 // K-major 128-byte swizzled (kda_tc.cuh):
-//   B1  [64 t][192]: columns 0..63 = T strictly below the diagonal, 64..191 = -W
-//   QT  [64 t][128]: e^{Gamma_t} * q_hat_t
-//   PS  [64 t][ 64]: P strictly below the diagonal
-//   KB  [128 k][64]: (e^{Gamma_C - Gamma_t} * k_hat_t)^T
+//   RA  [128][128 k]: -W and Q~ = e^{Gamma_t} * q_hat_t stacked by rows, -W
+//                     first for even chunks of a segment, Q~ first for odd ones
+//                     (so that one N = 128 product writes U next to the output
+//                     buffer of the chunk's parity)
+//   TS  [64 t][ 64]:  T strictly below the diagonal
+//   PS  [64 t][ 64]:  P strictly below the diagonal
+//   KB  [128 k][64]:  (e^{Gamma_C - Gamma_t} * k_hat_t)^T
 //   SC  fp32 beta[64], P_tt[64] (exact q_hat_t . k_hat_t), e^{Gamma_C}[128]
 // The diagonal terms beta_t v_t (of T V) and P_tt u_t (of P U) are applied in
 // fp32 by the scan kernel; they carry the largest single-token contributions.
@@ -48,13 +51,13 @@
 namespace kda {
 
 constexpr int CH = 64;  // chunk length
-constexpr uint32_t REC_B1 = 0;           // 6 slabs x (64 rows x 128 B)
-constexpr uint32_t REC_QT = 49152;       // 4 slabs x 8 KB
+constexpr uint32_t REC_RA = 0;           // 4 slabs x (128 rows x 128 B)
+constexpr uint32_t REC_TS = 65536;       // 2 slabs x 8 KB
 constexpr uint32_t REC_PS = 81920;       // 2 slabs x 8 KB
 constexpr uint32_t REC_KB = 98304;       // 2 slabs x (128 rows x 128 B)
 constexpr uint32_t REC_SC = 131072;      // 256 floats
 constexpr uint32_t REC_BYTES = 132096;
-constexpr uint32_t REC_TILES_A = REC_PS;              // B1 + QT: consumed by the first MMA group
+constexpr uint32_t REC_TILES_A = REC_PS;              // RA + TS: consumed by the first MMA group
 constexpr uint32_t REC_TILES_B = REC_BYTES - REC_PS;  // PS + KB + SC: second MMA group + scalars
 
 // raw input tiles: 3 halo rows + 64 chunk rows of one head (128 bf16 = 256 B)
@@ -167,6 +170,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int L = (int)((seg1 - t0) < CH ? (seg1 - t0) : CH);
   const int64_t chan = (int64_t)h * D + ch;
   uint8_t* rec = records + ((int64_t)cid * H + h) * REC_BYTES;
+  const int wrow0 = (nc.y & 1) ? 64 : 0, qrow0 = 64 - wrow0;  // row blocks of -W and Q~ in RA
   if (tid < CH) ms[MB_BETA + tid] = tid < L ? to_f(beta[(t0 + tid) * H + h]) : 0.f;
   const float4 wq = load4(conv_w + (0 * HD + chan) * 4);
   const float4 wk = load4(conv_w + (1 * HD + chan) * 4);
@@ -174,6 +178,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   // ---- 1. causal conv of q, k; half-local cumsum of the clamped gate; the
   //         row sums |q|^2, |k|^2, q.k over this warp's 32 channels ----------
+  // cumulative gates are kept in base-2 units (Gamma * log2 e) so that every
+  // e^x below is one ex2
   float gm_loc;  // half-local cumulative gate through row r0 + 16
   {
     float hq[3], hk[3];
@@ -206,7 +212,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         hq[0] = hq[1]; hq[1] = hq[2]; hq[2] = xq;
         hk[0] = hk[1]; hk[1] = hk[2]; hk[2] = xk;
         const bool valid = t < L;
-        cum += valid ? fmaxf(to_f(rg_t[(t + 3) * D + ch]), LOG_DECAY_FLOOR) : 0.f;
+        cum += valid ? fmaxf(to_f(rg_t[(t + 3) * D + ch]), LOG_DECAY_FLOOR) * LOG2E : 0.f;
         yq[r] = valid ? a : 0.f;
         yk[r] = valid ? b : 0.f;
         gl[r] = cum;
@@ -248,7 +254,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const float gC = ms[MB_CARRY + ch] + ms[MB_G1T + ch];      // G at the chunk end
   {
     const float gm = hb ? g1m : gm_loc;                      // this half's reference G_m
-    const float egcm = __expf(gC - g1m);                     // half 1: e^{G_C - G_m}, <= 1
+    const float egcm = tc::exp2_fast(gC - g1m);              // e^{G_C - G_{m_1}}, <= 1
 #pragma unroll
     for (int g = 0; g < 4; ++g) {  // 8-row groups
       float yq[8], yk[8], gl[8];
@@ -262,16 +268,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int t = r0 + 8 * g + r;
         const float G = gl[r] + carry;
         const float d = G - gm;
-        const float e1 = __expf(d), e2 = __expf(-d), e3 = __expf(G);
+        const float e1 = tc::exp2_fast(d), e2 = tc::exp2_fast(-d), e3 = tc::exp2_fast(G);
         const float kh = yk[r] * ms[MB_RK + t], qh = yq[r] * ms[MB_RQ + t];
         // B operand of the P Gram; A rows (block of the own half, and for
         // half 0 the rows read against half 1)
-        *reinterpret_cast<float*>(sm + P_GB + tc::sw128(t, ch, 64)) = tc::to_tf32(qh * e1);
+        *reinterpret_cast<float*>(sm + P_GB + tc::sw128o(r0 + 8 * g, r, ch, 64)) = tc::to_tf32(qh * e1);
         // e^{G_{m_1} - G_t}: e2 for half 1; <= 1 for half 0
-        const float a1 = hb ? e2 : __expf(g1m - G);
-        *reinterpret_cast<float*>(sm + P_GA + tc::sw128(32 + t, ch, GA_ROWS)) = tc::to_tf32(kh * a1);
-        if (!hb) *reinterpret_cast<float*>(sm + P_GA + tc::sw128(t, ch, GA_ROWS)) = tc::to_tf32(kh * e2);
-        *reinterpret_cast<float*>(rec + REC_QT + tc::sw128(t, ch, 64)) = tc::to_tf32(qh * e3);
+        const float a1 = hb ? e2 : tc::exp2_fast(g1m - G);
+        *reinterpret_cast<float*>(sm + P_GA + tc::sw128o(32 + r0 + 8 * g, r, ch, GA_ROWS)) = tc::to_tf32(kh * a1);
+        if (!hb)
+          *reinterpret_cast<float*>(sm + P_GA + tc::sw128o(r0 + 8 * g, r, ch, GA_ROWS)) = tc::to_tf32(kh * e2);
+        *reinterpret_cast<float*>(rec + REC_RA + tc::sw128o(qrow0 + r0 + 8 * g, r, ch, 128)) = tc::to_tf32(qh * e3);
         // e^{G_C - G_t} = e^{G_C - G_{m_1}} e^{G_{m_1} - G_t}: for half 0 both
         // factors are <= 1 (an underflow only drops what is below fp32 anyway)
         kb[r] = tc::to_tf32(kh * (egcm * a1));
@@ -316,7 +323,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc::ld_wait();
 #pragma unroll
     for (int r = 0; r < 16; ++r)
-      *reinterpret_cast<float*>(sm + P_GB + tc::sw128(r0 + 16 * g + r, ch, 64)) = tc::to_tf32(kx[r]);
+      *reinterpret_cast<float*>(sm + P_GB + tc::sw128o(r0 + 16 * g, r, ch, 64)) = tc::to_tf32(kx[r]);
   }
   tc::fence_async_smem();
   tc::fence_before();
@@ -339,7 +346,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int c = 0; c < 16; ++c) {
       const int i = ib + c;
       const float p = (q4 < 3 && i > j) ? v[c] : 0.f;  // strictly lower part; quarter 3 writes the zero block
-      *reinterpret_cast<float*>(rec + REC_PS + tc::sw128(i, j, 64)) = tc::to_tf32(p);
+      *reinterpret_cast<float*>(rec + REC_PS + tc::sw128o(ib, c, j, 64)) = tc::to_tf32(p);
     }
   }
   tc::bar_wait(&bar_m, par);
@@ -455,7 +462,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   __syncthreads();
 
-  // ---- 7. T = X diag(beta): record T_s, T tile; K~^T tile; W = T K~ ----------
+  // ---- 7. T = X diag(beta): record TS, T tile; K~^T tile; W = T K~ -----------
   for (int e = tid; e < CH * 16; e += PREP_THREADS) {  // 4-column groups
     const int t = e >> 4, tp = 4 * (e & 15);
     float4 tv, ts;
@@ -471,7 +478,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tsp[u] = c < t ? tvp[u] : 0.f;
     }
     *reinterpret_cast<float4*>(sm + P_TT + tc::sw128(t, tp, 64)) = tv;
-    *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, tp, 64)) = ts;
+    *reinterpret_cast<float4*>(rec + REC_TS + tc::sw128(t, tp, 64)) = ts;
   }
 #pragma unroll
   for (int g = 0; g < 2; ++g) {  // K~^T row ch, columns r0 + 16g ..
@@ -499,7 +506,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   {  // scalars of the record
     float* sc = reinterpret_cast<float*>(rec + REC_SC);
     if (tid < CH) { sc[tid] = ms[MB_BETA + tid]; sc[64 + tid] = ms[MB_PD + tid]; }
-    if (hb == 0) sc[128 + ch] = __expf(gC);
+    if (hb == 0) sc[128 + ch] = tc::exp2_fast(gC);
   }
   tc::bar_wait(&bar_w, par);
   tc::fence_after();
@@ -507,7 +514,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   if (tid == 0 && item + (int)gridDim.x < n_items) load_raw(item + gridDim.x);
 
-  // ---- 8. -W rows into the record (columns 64..191 of B1) --------------------
+  // ---- 8. -W rows into the record (row block wrow0 of RA) -------------------
   // M = 64 accumulator: row t in lane 16 * (t / 16) ... of quarter t / 16
   {
     const int t = 16 * q4 + (lane & 15);
@@ -521,10 +528,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (lane < 16) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + c0 + 4 * j, 64)) =
+          *reinterpret_cast<float4*>(rec + REC_RA + tc::sw128(wrow0 + t, c0 + 4 * j, 128)) =
               make_float4(tc::to_tf32(-w0[4 * j]), tc::to_tf32(-w0[4 * j + 1]), tc::to_tf32(-w0[4 * j + 2]),
                           tc::to_tf32(-w0[4 * j + 3]));
-          *reinterpret_cast<float4*>(rec + REC_B1 + tc::sw128(t, 64 + c0 + 16 + 4 * j, 64)) =
+          *reinterpret_cast<float4*>(rec + REC_RA + tc::sw128(wrow0 + t, c0 + 16 + 4 * j, 128)) =
               make_float4(tc::to_tf32(-w1[4 * j]), tc::to_tf32(-w1[4 * j + 1]), tc::to_tf32(-w1[4 * j + 2]),
                           tc::to_tf32(-w1[4 * j + 3]));
         }

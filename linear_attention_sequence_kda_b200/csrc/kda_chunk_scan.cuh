@@ -4,25 +4,32 @@
 // Detail", section "Sequenz-Mixing: 34 KDA-Schichten mit festem Zustand": a
 // state is handed from chunk to chunk).
 //
-// Thread v (of 128) owns value column v: TMEM lane v holds row v of
-//   V^T (cols 0..63) | S^T (cols 64..191) | U^T (192..255) | O^T (256..319)
-// (tf32 MMA operands), in fp32 V^T (320..383) and U^T (384..447), and a second
-// O^T buffer (448..511): chunk i's output is finalised while chunk i+1's first
-// MMA group runs.
-// Per chunk, with the record written by chunk_prep_kernel:
-//   MMA1  U^T = [V^T | S^T] [T_s | -W]^T        (K = 64 + 128)
-//         O^T = S^T Q~^T                          (K = 128)
-//   fp32  U^T += beta * V^T (diagonal of T);  S^T <- S^T diag(e^{Gamma_C})
-//   MMA2  O^T += U^T P_s^T;   S^T += U^T K-bar    (K = 64, A = U^T from TMEM)
-//   fp32  o = O + P_tt u (diagonal of P), written to HBM.
+// TMEM lane v holds row v of (tf32 MMA operands, fp32 where marked)
+//   O^T odd fp32 (cols 0..63) | U^T (64..127) | O^T even fp32 (128..191)
+//   | S^T fp32 (192..319) | V^T (320..383) | V^T fp32 (384..447) | P_tt U^T fp32 (448..511)
+// Per chunk i, with the record written by chunk_prep_kernel:
+//   MMA_A [U^T | O^T] = S^T [-W ; Q~]^T  (N = 128; the record stacks the two
+//         row blocks in the order that puts O^T in the buffer of i's parity),
+//         then U^T += V^T T_s^T
+//   fp32  U^T += beta * V^T (diagonal of T);  keep P_tt * U^T (diagonal of P)
+//   fp32  S^T <- S^T diag(e^{Gamma_C})
+//   MMA2  O^T += U^T P_s^T;   S^T += U^T K-bar    (A = U^T from TMEM)
+//   fp32  o = O + P_tt u, written to HBM (any time before chunk i + 2 reuses O^T).
 // A operands are read from TMEM as tf32; the state itself stays fp32.
 //
-// Data movement: the raw value tile of chunk i+2 (TMA, 64 rows x 256 B) and the
-// record halves of chunk i+1 (bulk copies) are in flight while chunk i runs;
-// each record half is refilled as soon as the MMA group that reads it is done.
-// The output rows of a chunk are staged in shared memory and leave with one
-// TMA tensor store (full chunks) or one bulk store per valid row (a segment's
-// last, partial chunk: rows past the segment end are never written).
+// Warp roles, handing off through mbarriers (no block-wide barrier inside the
+// chunk loop):
+//   warps 0..7  compute: warp w serves TMEM lanes 32 (w % 4) .. (value columns)
+//               and token / key half w / 4 of every per-chunk step: the fp32
+//               updates of chunk i, the short conv of v for chunk i + 1 while
+//               MMA2 of chunk i runs, then the output of chunk i.
+//   warp 8      one thread issues the MMAs.
+//   warp 9      one thread issues the loads: the first record piece
+//               ([-W ; Q~], T_s) is refilled as soon as MMA_A is done; the
+//               second (P_s, K-bar, scalars) is double-buffered and loaded a
+//               chunk ahead, as is the raw value tile.  One SM keeps only a few
+//               bulk copies in flight, so record bytes arrive at a fraction of
+//               HBM speed; the earlier a load is issued, the less it stalls.
 #pragma once
 #include "kda_chunk_prep.cuh"
 #include "kda_common.cuh"
@@ -30,267 +37,312 @@
 
 namespace kda {
 
-constexpr uint32_t VT_BYTES = CH * D * 2;            // raw value tile (bf16)
-constexpr uint32_t SCAN_A = 0;                       // record part A: B1 | QT (81920 B)
-constexpr uint32_t SCAN_B = REC_TILES_A;             // record part B: PS | KB | SC (50176 B)
-constexpr uint32_t SCAN_V0 = REC_TILES_A + REC_TILES_B;
-constexpr uint32_t SCAN_V1 = SCAN_V0 + VT_BYTES;
-constexpr uint32_t SCAN_O = SCAN_V1 + VT_BYTES;      // output staging [64 t][128] (fp32 or bf16)
-constexpr uint32_t SCAN_SMEM = SCAN_O + CH * D * 4 + 1024;
-constexpr int TM_V = 0, TM_S = 64, TM_U = 192;
-constexpr int TM_VX = 320, TM_UX = 384;  // exact fp32 V and U for the diagonal terms
-constexpr int TM_O0 = 256, TM_O1 = 448;  // output accumulators, alternating by chunk
+constexpr int SCAN_THREADS = 320;  // 8 compute warps, an MMA-issuing warp, a load-issuing warp
+constexpr uint32_t SCAN_RA = REC_RA;     // [-W ; Q~] and T_s   (81920 B, one copy)
+constexpr uint32_t SCAN_TS = REC_TS;
+constexpr uint32_t SCAN_PK = REC_PS;     // P_s | K-bar | scalars, 2 buffers (2 x 50176 B)
+constexpr uint32_t PK_BYTES = REC_BYTES - REC_PS;
+constexpr uint32_t SCAN_V0 = SCAN_PK + 2 * PK_BYTES;  // raw value tiles: 3 halo rows + 64 rows (bf16)
+constexpr uint32_t SCAN_V1 = SCAN_V0 + RAW_BYTES;
+constexpr uint32_t SCAN_SMEM = SCAN_V1 + RAW_BYTES + 1024;
+static_assert(SCAN_SMEM <= 232448, "scan shared memory");
+static_assert(PK_BYTES % 1024 == 0, "second record piece keeps 1024-byte tile alignment");
+constexpr int TM_O1 = 0, TM_U = 64, TM_O0 = 128, TM_S = 192, TM_V = 320;
+constexpr int TM_VX = 384, TM_UP = 448;  // exact fp32 V and P_tt * U for the diagonal terms
 __device__ __forceinline__ int o_col(int chunk) { return (chunk & 1) ? TM_O1 : TM_O0; }
 
 template <typename Tout, int ACT>
-__global__ void __launch_bounds__(128, 1)
-chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  const float* __restrict__ conv_w,
+__global__ void __launch_bounds__(SCAN_THREADS, 1)
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ conv_w,
                   const float* init_state, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
                   Tout* __restrict__ o, float* final_state) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  __shared__ uint64_t bar_a, bar_b, bar_v[2], bar_m1, bar_m2;
+  // loads (record pieces, value tiles), MMA commits, compute-warp hand-offs
+  // Every barrier a thread waits on by parity can run at most one phase ahead
+  // of that thread: the loader waits only on per-buffer "free" barriers whose
+  // next phase needs the load it is about to issue.
+  __shared__ uint64_t bar_a, bar_pk[2], bar_v[2], bar_ma, bar_m2, bar_conv, bar_d, bar_drain, bar_pkfree[2],
+      bar_vfree[2];
   __shared__ uint32_t tmem_base;
-  __shared__ float scb[2][256];  // per chunk parity: beta[64], P_tt[64], e^{Gamma_C}[128]
+  __shared__ int s_abort;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = seq_order[blockIdx.x / H], h = blockIdx.x % H;
   const int64_t seg0 = cu[n], T = cu[n + 1] - seg0;
   const int nchunks = (int)((T + CH - 1) / CH);
   const int64_t HD = (int64_t)H * D;
-  const int64_t chan = (int64_t)h * D + tid;
   const uint8_t* rec0 = records + (int64_t)chunk_base[n] * H * REC_BYTES + (int64_t)h * REC_BYTES;
   const int64_t rec_stride = (int64_t)H * REC_BYTES;  // next chunk of the same head
+  const volatile int* abort_flag = &s_abort;
 
   if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
   if (tid == 0) {
-    tc::bar_init(&bar_a, 1); tc::bar_init(&bar_b, 1);
+    tc::bar_init(&bar_a, 1); tc::bar_init(&bar_pk[0], 1); tc::bar_init(&bar_pk[1], 1);
     tc::bar_init(&bar_v[0], 1); tc::bar_init(&bar_v[1], 1);
-    tc::bar_init(&bar_m1, 1); tc::bar_init(&bar_m2, 1);
+    tc::bar_init(&bar_ma, 1); tc::bar_init(&bar_m2, 1);
+    tc::bar_init(&bar_conv, 256); tc::bar_init(&bar_d, 256);
+    tc::bar_init(&bar_pkfree[0], 1); tc::bar_init(&bar_pkfree[1], 1);
+    tc::bar_init(&bar_vfree[0], 256); tc::bar_init(&bar_vfree[1], 256);
+    tc::bar_init(&bar_drain, 1);
+    s_abort = 0;
     tc::bar_init_fence();
   }
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
   const uint32_t tm = tmem_base;
-  const uint32_t lane_base = tm + ((uint32_t)(32 * warp) << 16);
 
-  // initial state: row v of S^T = column v of S
-  {
-    const float* Si = init_state ? init_state + ((int64_t)n * H + h) * D * D + tid : nullptr;
-    for (int g16 = 0; g16 < 8; ++g16) {
-      float s[16];
+  if (warp == 8) {
+    // ======================= MMA-issuing thread =============================
+    if (lane == 0) {
+      const uint64_t d_ra = tc::desc(tc::smem_u32(sm + SCAN_RA));
+      const uint64_t d_ts = tc::desc(tc::smem_u32(sm + SCAN_TS));
+      const uint64_t d_ps = tc::desc(tc::smem_u32(sm + SCAN_PK));
+      const uint64_t d_kb = tc::desc(tc::smem_u32(sm + SCAN_PK + (REC_KB - REC_PS)));
+      constexpr uint64_t d_pk_step = PK_BYTES >> 4;  // second buffer, in descriptor units
+      bool ok = true;
+      for (int i = 0; i < nchunks && ok; ++i) {
+        const uint32_t p = i & 1;
+        // V_i in TMEM (and the output of chunk i - 2 read from the O^T buffer
+        // of this parity), the first record piece of chunk i in shared memory
+        ok = tc::bar_wait_or(&bar_conv, p, abort_flag);
+        ok = ok && tc::bar_wait_or(&bar_a, p, abort_flag);
+        if (!ok) break;
+        tc::fence_after();
+        // [U^T | O^T] = S^T [-W ; Q~]^T, then U^T += V^T T_s^T
+        const uint32_t dA = tm + (p ? TM_O1 : TM_U);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) s[i] = Si ? Si[(int64_t)(16 * g16 + i) * D] : 0.f;
-      tc::st16(lane_base + TM_S + 16 * g16, s);
-    }
-  }
-  // value conv taps and history for channel tid
-  const float4 wv = load4(conv_w + (2 * HD + chan) * 4);
-  float hv0 = 0.f, hv1 = 0.f, hv2 = 0.f;
-  if (init_conv) {
-    const __nv_bfloat16* c = init_conv + ((int64_t)n * 9 + 6) * HD + chan;
-    hv0 = to_f(c[0]); hv1 = to_f(c[HD]); hv2 = to_f(c[2 * HD]);
-  }
-
-  // issued counts per barrier (uniform across the block) for the exit drain
-  int a_iss = 0, b_iss = 0, v_iss[2] = {0, 0}, m2 = 0;
-  auto load_a = [&](int i) {
-    tc::bar_expect_tx(&bar_a, REC_TILES_A);
-    tc::bulk_g2s(sm + SCAN_A, rec0 + (int64_t)i * rec_stride, REC_TILES_A, &bar_a);
-  };
-  auto load_b = [&](int i) {
-    tc::bar_expect_tx(&bar_b, REC_TILES_B);
-    tc::bulk_g2s(sm + SCAN_B, rec0 + (int64_t)i * rec_stride + REC_PS, REC_TILES_B, &bar_b);
-  };
-  auto load_v = [&](int i) {
-    tc::bar_expect_tx(&bar_v[i & 1], VT_BYTES);
-    tc::tma_load_2d(sm + ((i & 1) ? SCAN_V1 : SCAN_V0), &tm_v, h * D, (int)(seg0 + (int64_t)CH * i),
-                    &bar_v[i & 1]);
-  };
-  if (nchunks > 0) {
-    if (tid == 0) {
-      load_a(0);
-      load_b(0);
-      load_v(0);
-      if (nchunks > 1) load_v(1);
-    }
-    a_iss = b_iss = 1; v_iss[0] = 1; v_iss[1] = nchunks > 1;
-  }
-  const uint64_t d_b1 = tc::desc(tc::smem_u32(sm + SCAN_A));
-  const uint64_t d_qt = tc::desc(tc::smem_u32(sm + SCAN_A + REC_QT));
-  const uint64_t d_ps = tc::desc(tc::smem_u32(sm + SCAN_B));
-  const uint64_t d_kb = tc::desc(tc::smem_u32(sm + SCAN_B + (REC_KB - REC_PS)));
-
-  // o = O + P_tt u for chunk j (O in its TMEM buffer, exact U still in UX):
-  // staged as [t][v] rows in shared memory, then one tensor store (full chunk)
-  // or one bulk store per valid row
-  Tout* ost = reinterpret_cast<Tout*>(sm + SCAN_O);
-  auto finalize = [&](int j) {
-    const int Lj = (int)((T - (int64_t)CH * j) < CH ? (T - (int64_t)CH * j) : CH);
-    const int64_t tj = seg0 + (int64_t)CH * j;
-    const float* scj = scb[j & 1];
+        for (int ks = 0; ks < 16; ++ks)
+          tc::mma_ts(dA, tm + TM_S + 8 * ks, d_ra + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), ks > 0);
 #pragma unroll
-    for (int g16 = 0; g16 < 4; ++g16) {
-      float r[16], ux[16];
-      tc::ld16(lane_base + o_col(j) + 16 * g16, r);
-      tc::ld16(lane_base + TM_UX + 16 * g16, ux);
-      tc::ld_wait();
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, d_ts + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
+        tc::commit(&bar_ma);
+        ok = tc::bar_wait_or(&bar_d, p, abort_flag);  // U^T final, S^T diag(gamma) applied
+        ok = ok && tc::bar_wait_or(&bar_pk[p], (uint32_t)((i >> 1) & 1), abort_flag);
+        if (!ok) break;
+        tc::fence_after();
+        const uint32_t dO = tm + o_col(i);
+        const uint64_t pko = p ? d_pk_step : 0;
 #pragma unroll
-      for (int jj = 0; jj < 16; ++jj)
-        ost[(16 * g16 + jj) * D + tid] = from_f<Tout>(fmaf(scj[64 + 16 * g16 + jj], ux[jj], r[jj]));
+        for (int ks = 0; ks < 8; ++ks) {
+          tc::mma_ts(dO, tm + TM_U + 8 * ks, d_ps + pko + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
+          tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, d_kb + pko + tc::desc_step(128, ks), tc::idesc_tf32(128, 128),
+                     1);
+        }
+        tc::commit(&bar_m2);
+        tc::commit(&bar_pkfree[p]);
+        ok = tc::bar_wait_or(&bar_m2, p, abort_flag);  // S^T complete for the next chunk
+      }
+      if (!ok) {
+        s_abort = 1;
+        // every issued MMA completes before TMEM is released (bounded wait)
+        tc::commit(&bar_drain);
+        tc::bar_wait(&bar_drain, 0);
+      }
     }
-    tc::fence_async_smem();
-    tc::fence_before();
-    __syncthreads();
-    tc::fence_after();
-    if (tid == 0) {
-      if (Lj == CH)
-        tc::tma_store_2d(&tm_o, h * D, (int)tj, ost);
-      else
-        for (int t = 0; t < Lj; ++t) tc::bulk_s2g(o + (tj + t) * HD + (int64_t)h * D, ost + t * D, D * sizeof(Tout));
-      tc::bulk_commit();
+  } else if (warp == 9) {
+    // ======================= load-issuing thread ============================
+    // A load issue can stall while the copy engine is busy; a separate thread
+    // keeps that stall off the MMA issue path.
+    if (lane == 0) {
+      int n_a = 0, n_pk[2] = {0, 0}, n_v[2] = {0, 0};  // loads issued per barrier, for the drain
+      auto load_a = [&](int i) {  // [-W ; Q~] and T_s
+        tc::bar_expect_tx(&bar_a, REC_TILES_A);
+        tc::bulk_g2s(sm + SCAN_RA, rec0 + (int64_t)i * rec_stride, REC_TILES_A, &bar_a);
+        ++n_a;
+      };
+      auto load_pk = [&](int i) {  // P_s, K-bar, scalars
+        tc::bar_expect_tx(&bar_pk[i & 1], PK_BYTES);
+        tc::bulk_g2s(sm + SCAN_PK + (i & 1) * PK_BYTES, rec0 + (int64_t)i * rec_stride + REC_PS, PK_BYTES,
+                     &bar_pk[i & 1]);
+        ++n_pk[i & 1];
+      };
+      auto load_v = [&](int i) {  // rows t0 - 3 .. t0 + 63 of this head's value columns
+        tc::bar_expect_tx(&bar_v[i & 1], RAW_BYTES);
+        tc::tma_load_2d(sm + ((i & 1) ? SCAN_V1 : SCAN_V0), &tm_v, h * D, (int)(seg0 + (int64_t)CH * i - 3),
+                        &bar_v[i & 1]);
+        ++n_v[i & 1];
+      };
+      bool ok = true;
+      if (nchunks > 0) {
+        load_a(0); load_v(0); load_pk(0);
+        if (nchunks > 1) { load_v(1); load_pk(1); }
+      }
+      for (int i = 0; i < nchunks && ok; ++i) {
+        const uint32_t p = i & 1, pb = (i >> 1) & 1;
+        if (i + 2 < nchunks) {  // value tile i consumed by the conv
+          ok = tc::bar_wait_or(&bar_vfree[p], pb, abort_flag);
+          if (ok) load_v(i + 2);
+        }
+        if (ok && i + 1 < nchunks) {  // MMA_A of chunk i has read the first piece
+          ok = tc::bar_wait_or(&bar_ma, p, abort_flag);
+          if (ok) load_a(i + 1);
+        }
+        if (ok && i + 2 < nchunks) {  // MMA2 of chunk i has read this second-piece buffer
+          ok = tc::bar_wait_or(&bar_pkfree[p], pb, abort_flag);
+          if (ok) load_pk(i + 2);
+        }
+      }
+      if (!ok) {
+        s_abort = 1;
+        // every issued load lands before shared memory is released (each wait
+        // bounded; awaiting the phase of the last issued load returns at once
+        // if it already completed)
+        if (n_a) tc::bar_wait(&bar_a, (uint32_t)((n_a - 1) & 1));
+        for (int b = 0; b < 2; ++b) {
+          if (n_pk[b]) tc::bar_wait(&bar_pk[b], (uint32_t)((n_pk[b] - 1) & 1));
+          if (n_v[b]) tc::bar_wait(&bar_v[b], (uint32_t)((n_v[b] - 1) & 1));
+        }
+      }
     }
-  };
-
-  bool ok = true;
-  for (int i = 0; i < nchunks && ok; ++i) {
-    const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
-    const int64_t t0 = seg0 + (int64_t)CH * i;
-
-    // (a) causal conv of v for this chunk; V^T row into TMEM (tf32 and fp32)
-    ok &= tc::bar_wait(&bar_v[i & 1], (i >> 1) & 1);
+  } else {
+    // ======================= compute warps ==================================
+    const int q = warp & 3, hf = warp >> 2;  // TMEM lane quarter, token / key half
+    const int v = 32 * q + lane;             // value column
+    const uint32_t tl = tm + ((uint32_t)(32 * q) << 16);
+    const int64_t chan = (int64_t)h * D + v;
+    // initial state: row v of S^T = column v of S (key rows 64 hf ..)
     {
-      const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + ((i & 1) ? SCAN_V1 : SCAN_V0));
+      const float* Si = init_state ? init_state + ((int64_t)n * H + h) * D * D + v : nullptr;
 #pragma unroll
       for (int g16 = 0; g16 < 4; ++g16) {
+        float s[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) s[j] = Si ? Si[(int64_t)(64 * hf + 16 * g16 + j) * D] : 0.f;
+        tc::st16(tl + TM_S + 64 * hf + 16 * g16, s);
+      }
+    }
+    const float4 wv = load4(conv_w + (2 * HD + chan) * 4);
+    const float* scal0 = reinterpret_cast<const float*>(sm + SCAN_PK + (REC_SC - REC_PS));
+    // short conv of v for chunk i, tokens 32 hf .. 32 hf + 31 -> V^T (tf32 and fp32)
+    auto conv_v = [&](int i) -> bool {
+      if (!tc::bar_wait_or(&bar_v[i & 1], (uint32_t)((i >> 1) & 1), abort_flag)) return false;
+      const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + ((i & 1) ? SCAN_V1 : SCAN_V0));
+      const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
+      const int r0 = 32 * hf;
+      float h0, h1, h2;  // tokens r0 - 3 .. r0 - 1 (tile rows r0 .. r0 + 2)
+      {
+        float hh[3];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const int64_t pos = (int64_t)CH * i + r0 - 3 + j;  // position in the segment
+          float x = to_f(vt[(r0 + j) * D + v]);
+          if (pos < 0) {  // before the segment: conv history (or zeros)
+            x = 0.f;
+            if (init_conv) x = to_f(init_conv[((int64_t)n * 9 + 6 + (int)(3 + pos)) * HD + chan]);
+          }
+          hh[j] = x;
+        }
+        h0 = hh[0]; h1 = hh[1]; h2 = hh[2];
+      }
+#pragma unroll
+      for (int g16 = 0; g16 < 2; ++g16) {
         float vv[16], r[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const int t = 16 * g16 + j;
-          const float x = to_f(vt[t * D + tid]);
-          float y = conv4(wv, hv0, hv1, hv2, x);
+          const int t = r0 + 16 * g16 + j;
+          const float x = to_f(vt[(t + 3) * D + v]);
+          float y = conv4(wv, h0, h1, h2, x);
           if (ACT == KDA_CONV_SILU) y = silu(y);
-          hv0 = hv1; hv1 = hv2; hv2 = x;
+          h0 = h1; h1 = h2; h2 = x;
           vv[j] = t < L ? y : 0.f;
           r[j] = tc::to_tf32(vv[j]);
         }
-        tc::st16(lane_base + TM_V + 16 * g16, r);
-        tc::st16(lane_base + TM_VX + 16 * g16, vv);
+        tc::st16(tl + TM_V + r0 + 16 * g16, r);
+        tc::st16(tl + TM_VX + r0 + 16 * g16, vv);
       }
-    }
-    tc::st_wait();
-    // (b) this chunk's record
-    float* sc = scb[i & 1];
-    ok &= tc::bar_wait(&bar_a, i & 1);
-    ok &= tc::bar_wait(&bar_b, i & 1);
-    sc[tid] = reinterpret_cast<const float*>(sm + SCAN_B + (REC_SC - REC_PS))[tid];
-    sc[tid + 128] = reinterpret_cast<const float*>(sm + SCAN_B + (REC_SC - REC_PS))[tid + 128];
-    if (tid == 0) tc::bulk_wait_read();  // the previous output store has read the staging tile
-    tc::fence_before();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    // (c) MMA group 1; the value tile buffer is free again
-    if (tid == 0) {
-      tc::fence_after();
-#pragma unroll
-      for (int ks = 0; ks < 24; ++ks)
-        tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, d_b1 + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < 16; ++ks)
-        tc::mma_ts(tm + o_col(i), tm + TM_S + 8 * ks, d_qt + tc::desc_step(64, ks), tc::idesc_tf32(128, 64),
-                   ks > 0);
-      tc::commit(&bar_m1);
-      if (i + 2 < nchunks) load_v(i + 2);
-    }
-    if (i + 2 < nchunks) v_iss[i & 1]++;
-    // while MMA group 1 runs: finish the previous chunk's output
-    if (i > 0) finalize(i - 1);
-    ok &= tc::bar_wait(&bar_m1, i & 1);
-    tc::fence_after();
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    if (i + 1 < nchunks) {  // record part A is free again
-      if (tid == 0) load_a(i + 1);
-      a_iss++;
-    }
-    // (d) U += beta V (exact diagonal of T V), S^T <- S^T diag(gamma)
-#pragma unroll
-    for (int g16 = 0; g16 < 4; ++g16) {
-      float r[16], vx[16], ux[16];
-      tc::ld16(lane_base + TM_U + 16 * g16, r);
-      tc::ld16(lane_base + TM_VX + 16 * g16, vx);
-      tc::ld_wait();
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        ux[j] = fmaf(sc[16 * g16 + j], vx[j], r[j]);
-        r[j] = tc::to_tf32(ux[j]);
-      }
-      tc::st16(lane_base + TM_U + 16 * g16, r);
-      tc::st16(lane_base + TM_UX + 16 * g16, ux);
-    }
-#pragma unroll
-    for (int g16 = 0; g16 < 8; g16 += 2) {
-      float r0[16], r1[16];
-      tc::ld16(lane_base + TM_S + 16 * g16, r0);
-      tc::ld16(lane_base + TM_S + 16 * g16 + 16, r1);
-      tc::ld_wait();
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        r0[j] *= sc[128 + 16 * g16 + j];
-        r1[j] *= sc[128 + 16 * g16 + 16 + j];
-      }
-      tc::st16(lane_base + TM_S + 16 * g16, r0);
-      tc::st16(lane_base + TM_S + 16 * g16 + 16, r1);
-    }
-    tc::st_wait();
-    tc::fence_before();
-    __syncthreads();
-    // (e) MMA group 2
-    if (tid == 0) {
-      tc::fence_after();
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        tc::mma_ts(tm + o_col(i), tm + TM_U + 8 * ks, d_ps + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, d_kb + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), 1);
-      tc::commit(&bar_m2);
-    }
-    ++m2;
-    ok &= tc::bar_wait(&bar_m2, i & 1);
-    tc::fence_after();
-    if (!__syncthreads_and(ok)) { ok = false; break; }
-    if (i + 1 < nchunks) {  // record part B is free again
-      if (tid == 0) load_b(i + 1);
-      b_iss++;
-    }
-  }
-  if (ok && nchunks > 0) finalize(nchunks - 1);
+      tc::st_wait();
+      tc::fence_before();
+      tc::bar_arrive(&bar_conv);
+      tc::bar_arrive(&bar_vfree[i & 1]);  // value tile i has been read
+      return true;
+    };
 
-  if (!ok) {
-    // a wait gave up (status already recorded): drain what is still in flight
-    // (each wait bounded; waiting on the parity of a completed phase returns at
-    // once) so that TMEM and shared memory are idle before exit
-    if (tid == 0) tc::commit(&bar_m2);
-    tc::bar_wait(&bar_m2, m2 & 1);
-    if (a_iss > 0) tc::bar_wait(&bar_a, (a_iss - 1) & 1);
-    if (b_iss > 0) tc::bar_wait(&bar_b, (b_iss - 1) & 1);
-    for (int b = 0; b < 2; ++b)
-      if (v_iss[b] > 0) tc::bar_wait(&bar_v[b], (v_iss[b] - 1) & 1);
-  }
-  if (tid == 0) tc::bulk_wait_all();  // output rows are in global memory before exit
-  // final state: column v of S = row v of S^T
-  if (ok) {
-    float* Sf = final_state + ((int64_t)n * H + h) * D * D + tid;
-    for (int g16 = 0; g16 < 8; ++g16) {
-      float s[16];
-      tc::ld16(lane_base + TM_S + 16 * g16, s);
-      tc::ld_wait();
+    bool ok = true;
+    if (nchunks > 0) ok = conv_v(0);
+    for (int i = 0; i < nchunks && ok; ++i) {
+      const uint32_t p = i & 1;
+      const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
+      // (a) U^T of this chunk (S^T read by the tensor core) and its scalars
+      ok = tc::bar_wait_or(&bar_ma, p, abort_flag);
+      ok = ok && tc::bar_wait_or(&bar_pk[p], (uint32_t)((i >> 1) & 1), abort_flag);
+      const float* scal = scal0 + p * (PK_BYTES / 4);
+      if (!ok) break;
+      tc::fence_after();
+      // (b) U += beta V (exact diagonal of T V); P_tt U kept in fp32
 #pragma unroll
-      for (int i = 0; i < 16; ++i) Sf[(int64_t)(16 * g16 + i) * D] = s[i];
+      for (int g16 = 0; g16 < 2; ++g16) {
+        const int c0 = 32 * hf + 16 * g16;
+        float r[16], vx[16];
+        tc::ld16(tl + TM_U + c0, r);
+        tc::ld16(tl + TM_VX + c0, vx);
+        tc::ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float u = fmaf(scal[c0 + j], vx[j], r[j]);
+          r[j] = tc::to_tf32(u);
+          vx[j] = scal[64 + c0 + j] * u;
+        }
+        tc::st16(tl + TM_U + c0, r);
+        tc::st16(tl + TM_UP + c0, vx);
+      }
+      // (c) S^T <- S^T diag(gamma)
+#pragma unroll
+      for (int g16 = 0; g16 < 4; g16 += 2) {
+        const int c0 = 64 * hf + 16 * g16;
+        float r0[16], r1[16];
+        tc::ld16(tl + TM_S + c0, r0);
+        tc::ld16(tl + TM_S + c0 + 16, r1);
+        tc::ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          r0[j] *= scal[128 + c0 + j];
+          r1[j] *= scal[128 + c0 + 16 + j];
+        }
+        tc::st16(tl + TM_S + c0, r0);
+        tc::st16(tl + TM_S + c0 + 16, r1);
+      }
+      tc::st_wait();
+      tc::fence_before();
+      tc::bar_arrive(&bar_d);
+      // (d) the next chunk's value conv while MMA2 runs
+      if (i + 1 < nchunks) ok = conv_v(i + 1);
+      // (e) o = O + P_tt u once MMA2 is done
+      ok = ok && tc::bar_wait_or(&bar_m2, p, abort_flag);
+      if (!ok) break;
+      tc::fence_after();
+      {
+        const int64_t tj = seg0 + (int64_t)CH * i;
+        const uint32_t oc = (uint32_t)o_col(i);
+#pragma unroll
+        for (int g16 = 0; g16 < 2; ++g16) {
+          const int c0 = 32 * hf + 16 * g16;
+          float r[16], up[16];
+          tc::ld16(tl + oc + c0, r);
+          tc::ld16(tl + TM_UP + c0, up);
+          tc::ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < L) o[(tj + c0 + j) * HD + chan] = from_f<Tout>(r[j] + up[j]);
+        }
+      }
+    }
+    if (!ok) s_abort = 1;
+    // final state: column v of S = row v of S^T
+    if (ok) {
+      float* Sf = final_state + ((int64_t)n * H + h) * D * D + v;
+#pragma unroll
+      for (int g16 = 0; g16 < 4; ++g16) {
+        float s[16];
+        tc::ld16(tl + TM_S + 64 * hf + 16 * g16, s);
+        tc::ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) Sf[(int64_t)(64 * hf + 16 * g16 + j) * D] = s[j];
+      }
     }
   }
   tc::fence_before();

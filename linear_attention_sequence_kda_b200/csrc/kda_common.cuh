@@ -11,6 +11,7 @@ namespace kda {
 constexpr int D = KDA_HEAD_DIM;   // d_k = d_v = 128
 constexpr float LOG_DECAY_FLOOR = -5.0f;
 constexpr float NORM_EPS = 1e-6f;
+constexpr float LOG2E = 1.4426950408889634f;
 
 // Device status word (one per device per process): kernels that give up on a
 // bounded wait write a nonzero kda_status here; kda_check_async_status reads it.

@@ -31,6 +31,21 @@ __host__ __device__ __forceinline__ uint32_t sw128(int r, int k, int R) {
   return (uint32_t)(slab * (R * 128) + r * 128 + ((c ^ (r & 7)) << 4) + ((kc & 3) << 2));
 }
 
+// the same offset for row rb + r where rb is a multiple of 8, so that the
+// swizzle phase of the row is r % 8: with r a compile-time constant (unrolled
+// loops) the row-dependent part folds into an immediate and one XOR
+__host__ __device__ __forceinline__ uint32_t sw128o(int rb, int r, int k, int R) {
+  const int slab = k >> 5, c = (k >> 2) & 7;
+  return (uint32_t)(slab * (R * 128) + rb * 128 + r * 128 + ((c ^ (r & 7)) << 4) + ((k & 3) << 2));
+}
+
+// 2^x on the special-function unit (PTX ex2.approx, relative error ~2^-22)
+__device__ __forceinline__ float exp2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // shared-memory matrix descriptor: SW128 K-major, SBO = 1024 B (8 rows x 128 B)
 __device__ __forceinline__ uint64_t desc(uint32_t saddr) {
   return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
@@ -164,6 +179,29 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
+// Bounded wait that also gives up (without recording a status) once `*abort`
+// is nonzero: another role of the block has already failed and will not
+// produce what is awaited.
+__device__ __forceinline__ bool bar_wait_or(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  const uint32_t a = smem_u32(bar);
+  for (int it = 0; it < kWaitLimit; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((it & 255) == 255 && *abort) return false;
+  }
+  set_status(KDA_ERR_TIMEOUT);
+  return false;
+}
+// plain arrival (release) on an mbarrier
+__device__ __forceinline__ void bar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // 2D tiled tensor copy global -> shared through a tensor map (TMA); (x, y) =
 // (inner column, row) of the box origin, x * element size a multiple of 16 B.
 // Rows outside the tensor (including negative y) are filled with zeros.
@@ -197,6 +235,11 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // wait until every committed bulk store of this thread is complete
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// hint: bring `bytes` (multiple of 16) of global memory at `src` into L2
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 // bulk async copy global -> shared, completion signalled on `bar` (tx bytes)
 __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
