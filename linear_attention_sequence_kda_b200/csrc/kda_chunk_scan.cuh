@@ -12,9 +12,10 @@
 //         row blocks in the order that puts O^T in the buffer of i's parity),
 //         then U^T += V^T T_s^T
 //   fp32  U^T += beta * V^T (diagonal of T);  keep P_tt * U^T (diagonal of P)
-//   fp32  S^T <- S^T diag(e^{Gamma_C})
-//   MMA2  O^T += U^T P_s^T;   S^T += U^T K-bar    (A = U^T from TMEM)
-//   fp32  o = O + P_tt u, written to HBM (any time before chunk i + 2 reuses O^T).
+//   MMA2o O^T += U^T P_s^T                       (A = U^T from TMEM)
+//   fp32  S^T <- S^T diag(e^{Gamma_C})          (while MMA2o runs)
+//   MMA2s S^T += U^T K-bar
+//   fp32  o = O + P_tt u, staged in shared memory and stored by TMA.
 // A operands are read from TMEM as tf32; the state itself stays fp32.
 //
 // Warp roles, handing off through mbarriers (no block-wide barrier inside the
@@ -22,14 +23,15 @@
 //   warps 0..7  compute: warp w serves TMEM lanes 32 (w % 4) .. (value columns)
 //               and token / key half w / 4 of every per-chunk step: the fp32
 //               updates of chunk i, the short conv of v for chunk i + 1 while
-//               MMA2 of chunk i runs, then the output of chunk i.
+//               MMA2 of chunk i runs, then the output tile of chunk i.
 //   warp 8      one thread issues the MMAs.
-//   warp 9      one thread issues the loads: the first record piece
-//               ([-W ; Q~], T_s) is refilled as soon as MMA_A is done; the
-//               second (P_s, K-bar, scalars) is double-buffered and loaded a
-//               chunk ahead, as is the raw value tile.  One SM keeps only a few
-//               bulk copies in flight, so record bytes arrive at a fraction of
-//               HBM speed; the earlier a load is issued, the less it stalls.
+//   warp 9      one thread issues the loads, each as soon as the step that
+//               read the previous contents of its buffer is done.
+//   warp 10     one thread stores the output tiles (double-buffered staging),
+//               so that global stores never hold up the compute warps.
+// Each thread waits by parity only on barriers that cannot complete two phases
+// ahead of it: the next phase of every barrier it waits on needs an action of
+// its own (or of a role that itself waited on this thread's previous step).
 #pragma once
 #include "kda_chunk_prep.cuh"
 #include "kda_common.cuh"
@@ -37,23 +39,24 @@
 
 namespace kda {
 
-constexpr int SCAN_THREADS = 320;  // 8 compute warps, an MMA-issuing warp, a load-issuing warp
-constexpr uint32_t SCAN_RA = REC_RA;     // [-W ; Q~] and T_s   (81920 B, one copy)
-constexpr uint32_t SCAN_TS = REC_TS;
-constexpr uint32_t SCAN_PK = REC_PS;     // P_s | K-bar | scalars, 2 buffers (2 x 50176 B)
+constexpr int SCAN_THREADS = 352;  // 8 compute warps, MMA, load and store issuing warps
+constexpr uint32_t SCAN_RA = 0;                          // [-W ; Q~] and T_s (81920 B)
+constexpr uint32_t SCAN_PK = REC_TILES_A;                // P_s | K-bar | scalars (50176 B)
 constexpr uint32_t PK_BYTES = REC_BYTES - REC_PS;
-constexpr uint32_t SCAN_V0 = SCAN_PK + 2 * PK_BYTES;  // raw value tiles: 3 halo rows + 64 rows (bf16)
-constexpr uint32_t SCAN_V1 = SCAN_V0 + RAW_BYTES;
-constexpr uint32_t SCAN_SMEM = SCAN_V1 + RAW_BYTES + 1024;
-static_assert(SCAN_SMEM <= 232448, "scan shared memory");
-static_assert(PK_BYTES % 1024 == 0, "second record piece keeps 1024-byte tile alignment");
+constexpr uint32_t SCAN_V = SCAN_PK + PK_BYTES;          // raw value tile: 3 halo rows + 64 rows (bf16)
+constexpr uint32_t SCAN_OST = (SCAN_V + RAW_BYTES + 1023) & ~1023u;  // 2 output tiles [64 t][128] (fp32 at most)
+constexpr uint32_t OST_BYTES = CH * D * 4;
+constexpr uint32_t SCAN_SMEM = SCAN_OST + 2 * OST_BYTES + 1024;
+static_assert(SCAN_SMEM + 256 <= 232448, "scan shared memory (dynamic + the static barriers)");
+static_assert(REC_TILES_A % 1024 == 0 && REC_TS % 1024 == 0, "record tiles stay 1024-byte aligned");
 constexpr int TM_O1 = 0, TM_U = 64, TM_O0 = 128, TM_S = 192, TM_V = 320;
 constexpr int TM_VX = 384, TM_UP = 448;  // exact fp32 V and P_tt * U for the diagonal terms
 __device__ __forceinline__ int o_col(int chunk) { return (chunk & 1) ? TM_O1 : TM_O0; }
 
 template <typename Tout, int ACT>
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
-chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ conv_w,
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const float* __restrict__ conv_w,
                   const float* init_state, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
@@ -61,11 +64,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   // loads (record pieces, value tiles), MMA commits, compute-warp hand-offs
-  // Every barrier a thread waits on by parity can run at most one phase ahead
-  // of that thread: the loader waits only on per-buffer "free" barriers whose
-  // next phase needs the load it is about to issue.
-  __shared__ uint64_t bar_a, bar_pk[2], bar_v[2], bar_ma, bar_m2, bar_conv, bar_d, bar_drain, bar_pkfree[2],
-      bar_vfree[2];
+  // loads; "free" signals for the loader; MMA commits; compute-warp hand-offs;
+  // output staging full / free
+  __shared__ uint64_t bar_a, bar_pk, bar_v, bar_pkfree, bar_vfree, bar_ma, bar_m2, bar_conv, bar_b, bar_d,
+      bar_ost[2], bar_ofree[2], bar_drain;
   __shared__ uint32_t tmem_base;
   __shared__ int s_abort;
 
@@ -80,12 +82,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
 
   if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
   if (tid == 0) {
-    tc::bar_init(&bar_a, 1); tc::bar_init(&bar_pk[0], 1); tc::bar_init(&bar_pk[1], 1);
-    tc::bar_init(&bar_v[0], 1); tc::bar_init(&bar_v[1], 1);
+    tc::bar_init(&bar_a, 1); tc::bar_init(&bar_pk, 1); tc::bar_init(&bar_v, 1);
+    tc::bar_init(&bar_pkfree, 1); tc::bar_init(&bar_vfree, 256);
     tc::bar_init(&bar_ma, 1); tc::bar_init(&bar_m2, 1);
-    tc::bar_init(&bar_conv, 256); tc::bar_init(&bar_d, 256);
-    tc::bar_init(&bar_pkfree[0], 1); tc::bar_init(&bar_pkfree[1], 1);
-    tc::bar_init(&bar_vfree[0], 256); tc::bar_init(&bar_vfree[1], 256);
+    tc::bar_init(&bar_conv, 256); tc::bar_init(&bar_b, 256); tc::bar_init(&bar_d, 256);
+    tc::bar_init(&bar_ost[0], 256); tc::bar_init(&bar_ost[1], 256);
+    tc::bar_init(&bar_ofree[0], 1); tc::bar_init(&bar_ofree[1], 1);
     tc::bar_init(&bar_drain, 1);
     s_abort = 0;
     tc::bar_init_fence();
@@ -99,15 +101,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
     // ======================= MMA-issuing thread =============================
     if (lane == 0) {
       const uint64_t d_ra = tc::desc(tc::smem_u32(sm + SCAN_RA));
-      const uint64_t d_ts = tc::desc(tc::smem_u32(sm + SCAN_TS));
+      const uint64_t d_ts = tc::desc(tc::smem_u32(sm + SCAN_RA + REC_TS));
       const uint64_t d_ps = tc::desc(tc::smem_u32(sm + SCAN_PK));
       const uint64_t d_kb = tc::desc(tc::smem_u32(sm + SCAN_PK + (REC_KB - REC_PS)));
-      constexpr uint64_t d_pk_step = PK_BYTES >> 4;  // second buffer, in descriptor units
       bool ok = true;
       for (int i = 0; i < nchunks && ok; ++i) {
         const uint32_t p = i & 1;
         // V_i in TMEM (and the output of chunk i - 2 read from the O^T buffer
-        // of this parity), the first record piece of chunk i in shared memory
+        // of this parity); the first record piece of chunk i in shared memory
         ok = tc::bar_wait_or(&bar_conv, p, abort_flag);
         ok = ok && tc::bar_wait_or(&bar_a, p, abort_flag);
         if (!ok) break;
@@ -121,20 +122,24 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
         for (int ks = 0; ks < 8; ++ks)
           tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, d_ts + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
         tc::commit(&bar_ma);
-        ok = tc::bar_wait_or(&bar_d, p, abort_flag);  // U^T final, S^T diag(gamma) applied
-        ok = ok && tc::bar_wait_or(&bar_pk[p], (uint32_t)((i >> 1) & 1), abort_flag);
+        // O^T += U^T P_s^T as soon as U^T is final
+        ok = tc::bar_wait_or(&bar_b, p, abort_flag);
+        ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag);
         if (!ok) break;
         tc::fence_after();
         const uint32_t dO = tm + o_col(i);
-        const uint64_t pko = p ? d_pk_step : 0;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          tc::mma_ts(dO, tm + TM_U + 8 * ks, d_ps + pko + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
-          tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, d_kb + pko + tc::desc_step(128, ks), tc::idesc_tf32(128, 128),
-                     1);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_ts(dO, tm + TM_U + 8 * ks, d_ps + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
+        // S^T += U^T K-bar once S^T diag(gamma) is in place
+        ok = tc::bar_wait_or(&bar_d, p, abort_flag);
+        if (!ok) break;
+        tc::fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, d_kb + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), 1);
         tc::commit(&bar_m2);
-        tc::commit(&bar_pkfree[p]);
+        tc::commit(&bar_pkfree);
         ok = tc::bar_wait_or(&bar_m2, p, abort_flag);  // S^T complete for the next chunk
       }
       if (!ok) {
@@ -146,46 +151,34 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
     }
   } else if (warp == 9) {
     // ======================= load-issuing thread ============================
-    // A load issue can stall while the copy engine is busy; a separate thread
-    // keeps that stall off the MMA issue path.
     if (lane == 0) {
-      int n_a = 0, n_pk[2] = {0, 0}, n_v[2] = {0, 0};  // loads issued per barrier, for the drain
+      int n_a = 0, n_pk = 0, n_v = 0;  // loads issued per barrier, for the drain
       auto load_a = [&](int i) {  // [-W ; Q~] and T_s
         tc::bar_expect_tx(&bar_a, REC_TILES_A);
         tc::bulk_g2s(sm + SCAN_RA, rec0 + (int64_t)i * rec_stride, REC_TILES_A, &bar_a);
         ++n_a;
       };
       auto load_pk = [&](int i) {  // P_s, K-bar, scalars
-        tc::bar_expect_tx(&bar_pk[i & 1], PK_BYTES);
-        tc::bulk_g2s(sm + SCAN_PK + (i & 1) * PK_BYTES, rec0 + (int64_t)i * rec_stride + REC_PS, PK_BYTES,
-                     &bar_pk[i & 1]);
-        ++n_pk[i & 1];
+        tc::bar_expect_tx(&bar_pk, PK_BYTES);
+        tc::bulk_g2s(sm + SCAN_PK, rec0 + (int64_t)i * rec_stride + REC_PS, PK_BYTES, &bar_pk);
+        ++n_pk;
       };
       auto load_v = [&](int i) {  // rows t0 - 3 .. t0 + 63 of this head's value columns
-        tc::bar_expect_tx(&bar_v[i & 1], RAW_BYTES);
-        tc::tma_load_2d(sm + ((i & 1) ? SCAN_V1 : SCAN_V0), &tm_v, h * D, (int)(seg0 + (int64_t)CH * i - 3),
-                        &bar_v[i & 1]);
-        ++n_v[i & 1];
+        tc::bar_expect_tx(&bar_v, RAW_BYTES);
+        tc::tma_load_2d(sm + SCAN_V, &tm_v, h * D, (int)(seg0 + (int64_t)CH * i - 3), &bar_v);
+        ++n_v;
       };
       bool ok = true;
-      if (nchunks > 0) {
-        load_a(0); load_v(0); load_pk(0);
-        if (nchunks > 1) { load_v(1); load_pk(1); }
-      }
-      for (int i = 0; i < nchunks && ok; ++i) {
-        const uint32_t p = i & 1, pb = (i >> 1) & 1;
-        if (i + 2 < nchunks) {  // value tile i consumed by the conv
-          ok = tc::bar_wait_or(&bar_vfree[p], pb, abort_flag);
-          if (ok) load_v(i + 2);
-        }
-        if (ok && i + 1 < nchunks) {  // MMA_A of chunk i has read the first piece
-          ok = tc::bar_wait_or(&bar_ma, p, abort_flag);
-          if (ok) load_a(i + 1);
-        }
-        if (ok && i + 2 < nchunks) {  // MMA2 of chunk i has read this second-piece buffer
-          ok = tc::bar_wait_or(&bar_pkfree[p], pb, abort_flag);
-          if (ok) load_pk(i + 2);
-        }
+      if (nchunks > 0) { load_a(0); load_v(0); load_pk(0); }
+      // loads for chunk j, in the order their buffers free up during chunk j - 1
+      for (int j = 1; j < nchunks && ok; ++j) {
+        const uint32_t q = (j - 1) & 1;
+        ok = tc::bar_wait_or(&bar_vfree, q, abort_flag);  // the conv has read value tile j - 1
+        if (ok) load_v(j);
+        ok = ok && tc::bar_wait_or(&bar_ma, q, abort_flag);  // MMA_A of chunk j - 1 has read the first piece
+        if (ok) load_a(j);
+        ok = ok && tc::bar_wait_or(&bar_pkfree, q, abort_flag);  // MMA2 of chunk j - 1 has read the second
+        if (ok) load_pk(j);
       }
       if (!ok) {
         s_abort = 1;
@@ -193,11 +186,33 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
         // bounded; awaiting the phase of the last issued load returns at once
         // if it already completed)
         if (n_a) tc::bar_wait(&bar_a, (uint32_t)((n_a - 1) & 1));
-        for (int b = 0; b < 2; ++b) {
-          if (n_pk[b]) tc::bar_wait(&bar_pk[b], (uint32_t)((n_pk[b] - 1) & 1));
-          if (n_v[b]) tc::bar_wait(&bar_v[b], (uint32_t)((n_v[b] - 1) & 1));
-        }
+        if (n_pk) tc::bar_wait(&bar_pk, (uint32_t)((n_pk - 1) & 1));
+        if (n_v) tc::bar_wait(&bar_v, (uint32_t)((n_v - 1) & 1));
       }
+    }
+  } else if (warp == 10) {
+    // ======================= output-storing thread ==========================
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < nchunks && ok; ++i) {
+        const int b = i & 1;
+        ok = tc::bar_wait_or(&bar_ost[b], (uint32_t)((i >> 1) & 1), abort_flag);
+        if (!ok) break;
+        const Tout* st = reinterpret_cast<const Tout*>(sm + SCAN_OST + b * OST_BYTES);
+        const int64_t tj = seg0 + (int64_t)CH * i;
+        const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
+        if (L == CH) {
+          tc::tma_store_2d(&tm_o, h * D, (int)tj, st);
+        } else {  // a segment's last, partial chunk: rows past its end are not written
+          for (int t = 0; t < L; ++t)
+            tc::bulk_s2g(o + (tj + t) * HD + (int64_t)h * D, st + t * D, D * sizeof(Tout));
+        }
+        tc::bulk_commit();
+        tc::bulk_wait_read();  // the staging tile may be refilled
+        tc::bar_arrive(&bar_ofree[b]);
+      }
+      if (!ok) s_abort = 1;
+      tc::bulk_wait_all();  // output rows are in global memory before exit
     }
   } else {
     // ======================= compute warps ==================================
@@ -220,8 +235,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
     const float* scal0 = reinterpret_cast<const float*>(sm + SCAN_PK + (REC_SC - REC_PS));
     // short conv of v for chunk i, tokens 32 hf .. 32 hf + 31 -> V^T (tf32 and fp32)
     auto conv_v = [&](int i) -> bool {
-      if (!tc::bar_wait_or(&bar_v[i & 1], (uint32_t)((i >> 1) & 1), abort_flag)) return false;
-      const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + ((i & 1) ? SCAN_V1 : SCAN_V0));
+      if (!tc::bar_wait_or(&bar_v, (uint32_t)(i & 1), abort_flag)) return false;
+      const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + SCAN_V);
       const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
       const int r0 = 32 * hf;
       float h0, h1, h2;  // tokens r0 - 3 .. r0 - 1 (tile rows r0 .. r0 + 2)
@@ -258,7 +273,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
       tc::st_wait();
       tc::fence_before();
       tc::bar_arrive(&bar_conv);
-      tc::bar_arrive(&bar_vfree[i & 1]);  // value tile i has been read
+      tc::bar_arrive(&bar_vfree);  // value tile i has been read
       return true;
     };
 
@@ -266,11 +281,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
     if (nchunks > 0) ok = conv_v(0);
     for (int i = 0; i < nchunks && ok; ++i) {
       const uint32_t p = i & 1;
-      const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
       // (a) U^T of this chunk (S^T read by the tensor core) and its scalars
       ok = tc::bar_wait_or(&bar_ma, p, abort_flag);
-      ok = ok && tc::bar_wait_or(&bar_pk[p], (uint32_t)((i >> 1) & 1), abort_flag);
-      const float* scal = scal0 + p * (PK_BYTES / 4);
+      ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag);
+      const float* scal = scal0;
       if (!ok) break;
       tc::fence_after();
       // (b) U += beta V (exact diagonal of T V); P_tt U kept in fp32
@@ -290,7 +304,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
         tc::st16(tl + TM_U + c0, r);
         tc::st16(tl + TM_UP + c0, vx);
       }
-      // (c) S^T <- S^T diag(gamma)
+      tc::st_wait();
+      tc::fence_before();
+      tc::bar_arrive(&bar_b);
+      // (c) S^T <- S^T diag(gamma) while O^T += U^T P_s^T runs
 #pragma unroll
       for (int g16 = 0; g16 < 4; g16 += 2) {
         const int c0 = 64 * hf + 16 * g16;
@@ -311,12 +328,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
       tc::bar_arrive(&bar_d);
       // (d) the next chunk's value conv while MMA2 runs
       if (i + 1 < nchunks) ok = conv_v(i + 1);
-      // (e) o = O + P_tt u once MMA2 is done
+      // (e) o = O + P_tt u once MMA2 is done, into the staging tile of this
+      // parity (free once the store of chunk i - 2 has read it)
       ok = ok && tc::bar_wait_or(&bar_m2, p, abort_flag);
+      if (ok && i >= 2) ok = tc::bar_wait_or(&bar_ofree[p], (uint32_t)(((i >> 1) - 1) & 1), abort_flag);
       if (!ok) break;
       tc::fence_after();
       {
-        const int64_t tj = seg0 + (int64_t)CH * i;
+        Tout* st = reinterpret_cast<Tout*>(sm + SCAN_OST + p * OST_BYTES);
         const uint32_t oc = (uint32_t)o_col(i);
 #pragma unroll
         for (int g16 = 0; g16 < 2; ++g16) {
@@ -326,10 +345,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const float* __restr
           tc::ld16(tl + TM_UP + c0, up);
           tc::ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < L) o[(tj + c0 + j) * HD + chan] = from_f<Tout>(r[j] + up[j]);
+          for (int j = 0; j < 16; ++j) st[(c0 + j) * D + v] = from_f<Tout>(r[j] + up[j]);
         }
       }
+      tc::fence_async_smem();
+      tc::bar_arrive(&bar_ost[p]);
     }
     if (!ok) s_abort = 1;
     // final state: column v of S = row v of S^T

@@ -64,12 +64,13 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   const int32_t* d_order = d_base + (N + 1);
   uint8_t* records = ws + hdr;
 
-  // TMA descriptors over the packed [total_T, H*128] inputs: 67-row boxes
-  // (3 halo rows + one chunk)
+  // TMA descriptors over the packed [total_T, H*128] tensors: 67-row boxes for
+  // the inputs (3 halo rows + one chunk); 64-row boxes for the output tiles
   const uint64_t rows = (uint64_t)cu_host[N], cols = (uint64_t)H * D;
-  CUtensorMap tq, tk, tg, tv;
+  CUtensorMap tq, tk, tg, tv, to;
   if (!make_tmap_bf16_2d(&tq, q, rows, cols, RAW_ROWS, D) || !make_tmap_bf16_2d(&tk, k, rows, cols, RAW_ROWS, D) ||
-      !make_tmap_bf16_2d(&tg, g, rows, cols, RAW_ROWS, D) || !make_tmap_bf16_2d(&tv, v, rows, cols, RAW_ROWS, D))
+      !make_tmap_bf16_2d(&tg, g, rows, cols, RAW_ROWS, D) || !make_tmap_bf16_2d(&tv, v, rows, cols, RAW_ROWS, D) ||
+      !make_tmap_2d(&to, o, rows, cols, CH, D, o_dt == KDA_F32 ? 4 : 2))
     return KDA_ERR_CUDA;
 
   if (total > 0) {
@@ -91,13 +92,13 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     auto scan = chunk_scan_kernel<float, ACT>;
     if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
       return KDA_ERR_CUDA;
-    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, stream>>>(tv, conv_w, init_state, (const T*)init_conv, cu_dev,
+    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, stream>>>(tv, to, conv_w, init_state, (const T*)init_conv, cu_dev,
                                                                d_base, d_order, H, records, (float*)o, final_state);
   } else {
     auto scan = chunk_scan_kernel<T, ACT>;
     if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
       return KDA_ERR_CUDA;
-    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, stream>>>(tv, conv_w, init_state, (const T*)init_conv, cu_dev,
+    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, stream>>>(tv, to, conv_w, init_state, (const T*)init_conv, cu_dev,
                                                                d_base, d_order, H, records, (T*)o, final_state);
   }
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
