@@ -20,14 +20,14 @@
 //
 // Warp roles, handing off through mbarriers (no block-wide barrier inside the
 // chunk loop):
-//   warps 0..7  compute: warp w serves TMEM lanes 32 (w % 4) .. (value columns)
-//               and token / key half w / 4 of every per-chunk step: the fp32
+//   warps 0..15 compute: warp w serves TMEM lanes 32 (w % 4) .. (value columns)
+//               and token / key quarter w / 4 of every per-chunk step: the fp32
 //               updates of chunk i, the short conv of v for chunk i + 1 while
 //               MMA2 of chunk i runs, then the output tile of chunk i.
-//   warp 8      one thread issues the MMAs.
-//   warp 9      one thread issues the loads, each as soon as the step that
+//   warp 16     one thread issues the MMAs.
+//   warp 17     one thread issues the loads, each as soon as the step that
 //               read the previous contents of its buffer is done.
-//   warp 10     one thread stores the output tiles (double-buffered staging),
+//   warp 18     one thread stores the output tiles (double-buffered staging),
 //               so that global stores never hold up the compute warps.
 // Each thread waits by parity only on barriers that cannot complete two phases
 // ahead of it: the next phase of every barrier it waits on needs an action of
@@ -39,7 +39,8 @@
 
 namespace kda {
 
-constexpr int SCAN_THREADS = 352;  // 8 compute warps, MMA, load and store issuing warps
+constexpr int SCAN_THREADS = 608;  // 16 compute warps, MMA, load and store issuing warps
+constexpr int SCAN_COMPUTE = 512;
 constexpr uint32_t SCAN_RA = 0;                          // [-W ; Q~] and T_s (81920 B)
 constexpr uint32_t SCAN_PK = REC_TILES_A;                // P_s | K-bar | scalars (50176 B)
 constexpr uint32_t PK_BYTES = REC_BYTES - REC_PS;
@@ -83,10 +84,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
   if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
   if (tid == 0) {
     tc::bar_init(&bar_a, 1); tc::bar_init(&bar_pk, 1); tc::bar_init(&bar_v, 1);
-    tc::bar_init(&bar_pkfree, 1); tc::bar_init(&bar_vfree, 256);
+    tc::bar_init(&bar_pkfree, 1); tc::bar_init(&bar_vfree, SCAN_COMPUTE);
     tc::bar_init(&bar_ma, 1); tc::bar_init(&bar_m2, 1);
-    tc::bar_init(&bar_conv, 256); tc::bar_init(&bar_b, 256); tc::bar_init(&bar_d, 256);
-    tc::bar_init(&bar_ost[0], 256); tc::bar_init(&bar_ost[1], 256);
+    tc::bar_init(&bar_conv, SCAN_COMPUTE); tc::bar_init(&bar_b, SCAN_COMPUTE); tc::bar_init(&bar_d, SCAN_COMPUTE);
+    tc::bar_init(&bar_ost[0], SCAN_COMPUTE); tc::bar_init(&bar_ost[1], SCAN_COMPUTE);
     tc::bar_init(&bar_ofree[0], 1); tc::bar_init(&bar_ofree[1], 1);
     tc::bar_init(&bar_drain, 1);
     s_abort = 0;
@@ -97,7 +98,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
   tc::fence_after();
   const uint32_t tm = tmem_base;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ======================= MMA-issuing thread =============================
     if (lane == 0) {
       const uint64_t d_ra = tc::desc(tc::smem_u32(sm + SCAN_RA));
@@ -149,7 +150,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         tc::bar_wait(&bar_drain, 0);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ======================= load-issuing thread ============================
     if (lane == 0) {
       int n_a = 0, n_pk = 0, n_v = 0;  // loads issued per barrier, for the drain
@@ -190,7 +191,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         if (n_v) tc::bar_wait(&bar_v, (uint32_t)((n_v - 1) & 1));
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == 18) {
     // ======================= output-storing thread ==========================
     if (lane == 0) {
       bool ok = true;
@@ -216,36 +217,37 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     }
   } else {
     // ======================= compute warps ==================================
-    const int q = warp & 3, hf = warp >> 2;  // TMEM lane quarter, token / key half
-    const int v = 32 * q + lane;             // value column
+    const int q = warp & 3, part = warp >> 2;  // TMEM lane quarter, token / key quarter
+    const int v = 32 * q + lane;               // value column
+    const int t0 = 16 * part;                  // tokens t0 .. t0 + 15
+    const int k0 = 32 * part;                  // keys k0 .. k0 + 31
     const uint32_t tl = tm + ((uint32_t)(32 * q) << 16);
     const int64_t chan = (int64_t)h * D + v;
-    // initial state: row v of S^T = column v of S (key rows 64 hf ..)
+    // initial state: row v of S^T = column v of S (key rows k0 ..)
     {
       const float* Si = init_state ? init_state + ((int64_t)n * H + h) * D * D + v : nullptr;
 #pragma unroll
-      for (int g16 = 0; g16 < 4; ++g16) {
+      for (int g16 = 0; g16 < 2; ++g16) {
         float s[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) s[j] = Si ? Si[(int64_t)(64 * hf + 16 * g16 + j) * D] : 0.f;
-        tc::st16(tl + TM_S + 64 * hf + 16 * g16, s);
+        for (int j = 0; j < 16; ++j) s[j] = Si ? Si[(int64_t)(k0 + 16 * g16 + j) * D] : 0.f;
+        tc::st16(tl + TM_S + k0 + 16 * g16, s);
       }
     }
     const float4 wv = load4(conv_w + (2 * HD + chan) * 4);
-    const float* scal0 = reinterpret_cast<const float*>(sm + SCAN_PK + (REC_SC - REC_PS));
-    // short conv of v for chunk i, tokens 32 hf .. 32 hf + 31 -> V^T (tf32 and fp32)
+    const float* scal = reinterpret_cast<const float*>(sm + SCAN_PK + (REC_SC - REC_PS));
+    // short conv of v for chunk i, tokens t0 .. t0 + 15 -> V^T (tf32 and fp32)
     auto conv_v = [&](int i) -> bool {
       if (!tc::bar_wait_or(&bar_v, (uint32_t)(i & 1), abort_flag)) return false;
       const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + SCAN_V);
       const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
-      const int r0 = 32 * hf;
-      float h0, h1, h2;  // tokens r0 - 3 .. r0 - 1 (tile rows r0 .. r0 + 2)
+      float h0, h1, h2;  // tokens t0 - 3 .. t0 - 1 (tile rows t0 .. t0 + 2)
       {
         float hh[3];
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
-          const int64_t pos = (int64_t)CH * i + r0 - 3 + j;  // position in the segment
-          float x = to_f(vt[(r0 + j) * D + v]);
+          const int64_t pos = (int64_t)CH * i + t0 - 3 + j;  // position in the segment
+          float x = to_f(vt[(t0 + j) * D + v]);
           if (pos < 0) {  // before the segment: conv history (or zeros)
             x = 0.f;
             if (init_conv) x = to_f(init_conv[((int64_t)n * 9 + 6 + (int)(3 + pos)) * HD + chan]);
@@ -254,22 +256,19 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         }
         h0 = hh[0]; h1 = hh[1]; h2 = hh[2];
       }
+      float vv[16], r[16];
 #pragma unroll
-      for (int g16 = 0; g16 < 2; ++g16) {
-        float vv[16], r[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = r0 + 16 * g16 + j;
-          const float x = to_f(vt[(t + 3) * D + v]);
-          float y = conv4(wv, h0, h1, h2, x);
-          if (ACT == KDA_CONV_SILU) y = silu(y);
-          h0 = h1; h1 = h2; h2 = x;
-          vv[j] = t < L ? y : 0.f;
-          r[j] = tc::to_tf32(vv[j]);
-        }
-        tc::st16(tl + TM_V + r0 + 16 * g16, r);
-        tc::st16(tl + TM_VX + r0 + 16 * g16, vv);
+      for (int j = 0; j < 16; ++j) {
+        const int t = t0 + j;
+        const float x = to_f(vt[(t + 3) * D + v]);
+        float y = conv4(wv, h0, h1, h2, x);
+        if (ACT == KDA_CONV_SILU) y = silu(y);
+        h0 = h1; h1 = h2; h2 = x;
+        vv[j] = t < L ? y : 0.f;
+        r[j] = tc::to_tf32(vv[j]);
       }
+      tc::st16(tl + TM_V + t0, r);
+      tc::st16(tl + TM_VX + t0, vv);
       tc::st_wait();
       tc::fence_before();
       tc::bar_arrive(&bar_conv);
@@ -284,44 +283,39 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       // (a) U^T of this chunk (S^T read by the tensor core) and its scalars
       ok = tc::bar_wait_or(&bar_ma, p, abort_flag);
       ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag);
-      const float* scal = scal0;
       if (!ok) break;
       tc::fence_after();
       // (b) U += beta V (exact diagonal of T V); P_tt U kept in fp32
-#pragma unroll
-      for (int g16 = 0; g16 < 2; ++g16) {
-        const int c0 = 32 * hf + 16 * g16;
+      {
         float r[16], vx[16];
-        tc::ld16(tl + TM_U + c0, r);
-        tc::ld16(tl + TM_VX + c0, vx);
+        tc::ld16(tl + TM_U + t0, r);
+        tc::ld16(tl + TM_VX + t0, vx);
         tc::ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float u = fmaf(scal[c0 + j], vx[j], r[j]);
+          const float u = fmaf(scal[t0 + j], vx[j], r[j]);
           r[j] = tc::to_tf32(u);
-          vx[j] = scal[64 + c0 + j] * u;
+          vx[j] = scal[64 + t0 + j] * u;
         }
-        tc::st16(tl + TM_U + c0, r);
-        tc::st16(tl + TM_UP + c0, vx);
+        tc::st16(tl + TM_U + t0, r);
+        tc::st16(tl + TM_UP + t0, vx);
       }
       tc::st_wait();
       tc::fence_before();
       tc::bar_arrive(&bar_b);
       // (c) S^T <- S^T diag(gamma) while O^T += U^T P_s^T runs
-#pragma unroll
-      for (int g16 = 0; g16 < 4; g16 += 2) {
-        const int c0 = 64 * hf + 16 * g16;
+      {
         float r0[16], r1[16];
-        tc::ld16(tl + TM_S + c0, r0);
-        tc::ld16(tl + TM_S + c0 + 16, r1);
+        tc::ld16(tl + TM_S + k0, r0);
+        tc::ld16(tl + TM_S + k0 + 16, r1);
         tc::ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          r0[j] *= scal[128 + c0 + j];
-          r1[j] *= scal[128 + c0 + 16 + j];
+          r0[j] *= scal[128 + k0 + j];
+          r1[j] *= scal[128 + k0 + 16 + j];
         }
-        tc::st16(tl + TM_S + c0, r0);
-        tc::st16(tl + TM_S + c0 + 16, r1);
+        tc::st16(tl + TM_S + k0, r0);
+        tc::st16(tl + TM_S + k0 + 16, r1);
       }
       tc::st_wait();
       tc::fence_before();
@@ -336,17 +330,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       tc::fence_after();
       {
         Tout* st = reinterpret_cast<Tout*>(sm + SCAN_OST + p * OST_BYTES);
-        const uint32_t oc = (uint32_t)o_col(i);
+        float r[16], up[16];
+        tc::ld16(tl + (uint32_t)o_col(i) + t0, r);
+        tc::ld16(tl + TM_UP + t0, up);
+        tc::ld_wait();
 #pragma unroll
-        for (int g16 = 0; g16 < 2; ++g16) {
-          const int c0 = 32 * hf + 16 * g16;
-          float r[16], up[16];
-          tc::ld16(tl + oc + c0, r);
-          tc::ld16(tl + TM_UP + c0, up);
-          tc::ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) st[(c0 + j) * D + v] = from_f<Tout>(r[j] + up[j]);
-        }
+        for (int j = 0; j < 16; ++j) st[(t0 + j) * D + v] = from_f<Tout>(r[j] + up[j]);
       }
       tc::fence_async_smem();
       tc::bar_arrive(&bar_ost[p]);
@@ -356,12 +345,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     if (ok) {
       float* Sf = final_state + ((int64_t)n * H + h) * D * D + v;
 #pragma unroll
-      for (int g16 = 0; g16 < 4; ++g16) {
+      for (int g16 = 0; g16 < 2; ++g16) {
         float s[16];
-        tc::ld16(tl + TM_S + 64 * hf + 16 * g16, s);
+        tc::ld16(tl + TM_S + k0 + 16 * g16, s);
         tc::ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) Sf[(int64_t)(64 * hf + 16 * g16 + j) * D] = s[j];
+        for (int j = 0; j < 16; ++j) Sf[(int64_t)(k0 + 16 * g16 + j) * D] = s[j];
       }
     }
   }
