@@ -73,14 +73,15 @@ constexpr uint32_t GA_ROWS = 96;
 constexpr uint32_t P_GB = 49152;             // steps 3-5: Gram B tile, 4 slabs x 64 rows
 constexpr uint32_t MS_LD = 68;               // row stride (floats) of the solve matrix: rows
                                              // 16-byte aligned, columns spread over all banks
-constexpr uint32_t P_MS = 0;                 // steps 6-7: diag(beta) M strict -> X, [64][68] fp32
+constexpr uint32_t P_MS = 0;                 // step 6: diag(beta) M strict, [64][68] fp32
 constexpr uint32_t P_TT = 17408;             // step 7: T tile [64 t][64 t'] (16 KB)
 constexpr uint32_t P_KT = 33792;             // step 7: K~^T tile [128 k][64 t] (32 KB)
-constexpr uint32_t P_TMP = 66560;            // step 6: solve temporaries (8 KB)
+constexpr uint32_t P_TMP = 66560;            // steps 6-7: blocks of X (12.3 KB)
 constexpr uint32_t P_MISC = 81920;           // scalars (6 KB)
 constexpr uint32_t PREP_SMEM = P_MISC + 6144 + 1024;
 static_assert(P_GA + 3 * GA_ROWS * 128 + 128 * 128 <= P_MISC, "A tile reads past the Gram region");
-static_assert(3 * RAW_BYTES <= P_MISC && P_TMP + 8192 <= P_MISC, "shared regions overlap the scalars");
+static_assert(3 * RAW_BYTES <= P_MISC && P_TMP + (96 * 20 + 32 * 36 + 16) * 4 <= P_MISC,
+              "shared regions overlap the scalars");
 static_assert(P_MS + 64 * MS_LD * 4 <= P_TT, "solve matrix overlaps the T tile");
 
 // scalar region (floats)
@@ -367,14 +368,21 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
 
   // ---- 6. X = (I + diag(beta) M)^-1 (unit lower triangular) ------------------
-  // diagonal 16-blocks by forward substitution, then the off-diagonal 16-blocks
-  // of each 32-half, then the off-diagonal 32-block:
-  //   X_ba = -X_bb L_ba X_aa  for the 2 x 2 block partition at each level.
-  // Every entry above the diagonal inside each 32-half is 0 (written so by the
-  // readout and by the diagonal-block copy), so the products run over full
-  // block widths.
-  float* Xd = (float*)(sm + P_TMP);         // [4][16][16] inverses of the diagonal 16-blocks
-  float* Yt = (float*)(sm + P_TMP) + 1024;  // [32][32] temporary
+  // Blocks of the 2 x 2 partitions, each X_ba = -X_bb L_ba X_aa:
+  //   A  the four diagonal 16-blocks, by forward substitution   -> Xd[I]
+  //   B  the off-diagonal 16-block of each 32-half               -> XB[P]
+  //   C  the off-diagonal 32-block                               -> XC
+  // Results go to their own buffers (nothing is overwritten while another
+  // thread may still read it), so each stage needs one barrier.  Within B and
+  // C a thread group computes a column of the intermediate product L X_aa and
+  // shares it by shuffles before multiplying by X_bb.
+  // Row strides of 20 (36) floats put 8 consecutive rows of a block in 8
+  // distinct 4-bank groups, so the float4 row loads below are conflict-free.
+  constexpr int XS = 20, XCS = 36;
+  float* Xd = (float*)(sm + P_TMP);           // [4][16][XS]
+  float* XB = Xd + 4 * 16 * XS;               // [2][16][XS]
+  float* XC = XB + 2 * 16 * XS;               // [32][XCS]
+  float* Zr = XC + 32 * XCS;                  // [16] zeros
   if (tid < 64) {
     const int I = tid >> 4, cc = tid & 15;  // column cc of X_II
     const float* Lb = Ms + (16 * I) * MS_LD + 16 * I;
@@ -393,72 +401,108 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       x[r] = r < cc ? 0.f : s;
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) Xd[(I * 16 + r) * 16 + cc] = x[r];
+    for (int r = 0; r < 16; ++r) Xd[(I * 16 + r) * XS + cc] = x[r];
+  } else if (tid < 80) {
+    Zr[tid - 64] = 0.f;
   }
   __syncthreads();
-  {  // Y = L_{2P+1,2P} X_{2P,2P} for P = 0, 1 (16 x 16 each)
-    const int r = (tid >> 4) & 15, cc = tid & 15;
+  {  // B: warp w -> half P = w / 4, column cc = 4 (w % 4) + lane / 8, rows k and k + 8 (k = lane % 8)
+    const int P = warp >> 2, cc = 4 * (warp & 3) + (lane >> 3), k = lane & 7;
+    const float* X0 = Xd + (2 * P) * 16 * XS;
+    const float* X1 = Xd + (2 * P + 1) * 16 * XS;
+    float xc[16];  // column cc of X_{2P,2P}
 #pragma unroll
-    for (int P = 0; P < 2; ++P) {
-      const float* Lr = Ms + (32 * P + 16 + r) * MS_LD + 32 * P;
-      const float* X0 = Xd + (2 * P) * 256;
+    for (int m = 0; m < 16; ++m) xc[m] = X0[m * XS + cc];
+    float y[2];  // (L_{2P+1,2P} X_{2P,2P}) rows k, k + 8, column cc
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float* Lr = Ms + (32 * P + 16 + k + 8 * u) * MS_LD + 32 * P;
       float s = 0.f;
 #pragma unroll
       for (int m4 = 0; m4 < 16; m4 += 4) {
-        const float4 l = *reinterpret_cast<const float4*>(Lr + m4);
-        s += l.x * X0[m4 * 16 + cc] + l.y * X0[(m4 + 1) * 16 + cc] + l.z * X0[(m4 + 2) * 16 + cc] +
-             l.w * X0[(m4 + 3) * 16 + cc];
+        const float4 a = *reinterpret_cast<const float4*>(Lr + m4);
+        s += a.x * xc[m4] + a.y * xc[m4 + 1] + a.z * xc[m4 + 2] + a.w * xc[m4 + 3];
       }
-      Yt[(P * 16 + r) * 16 + cc] = s;
+      y[u] = s;
     }
-  }
-  __syncthreads();
-  {  // X_{2P+1,2P} = -X_{2P+1,2P+1} Y; diagonal blocks copied into the matrix
-    const int r = (tid >> 4) & 15, cc = tid & 15;
+    float yc[16];  // the whole column cc, from the 8 lanes that share it
+    const int base = lane & ~7;
 #pragma unroll
-    for (int P = 0; P < 2; ++P) {
-      const float* X1 = Xd + (2 * P + 1) * 256 + r * 16;
+    for (int kk = 0; kk < 8; ++kk) {
+      yc[kk] = __shfl_sync(0xffffffffu, y[0], base + kk);
+      yc[kk + 8] = __shfl_sync(0xffffffffu, y[1], base + kk);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float* xr = X1 + (k + 8 * u) * XS;
       float s = 0.f;
 #pragma unroll
       for (int m4 = 0; m4 < 16; m4 += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(X1 + m4);
-        s += x.x * Yt[(P * 16 + m4) * 16 + cc] + x.y * Yt[(P * 16 + m4 + 1) * 16 + cc] +
-             x.z * Yt[(P * 16 + m4 + 2) * 16 + cc] + x.w * Yt[(P * 16 + m4 + 3) * 16 + cc];
+        const float4 a = *reinterpret_cast<const float4*>(xr + m4);
+        s += a.x * yc[m4] + a.y * yc[m4 + 1] + a.z * yc[m4 + 2] + a.w * yc[m4 + 3];
       }
-      Ms[(32 * P + 16 + r) * MS_LD + 32 * P + cc] = -s;
+      XB[(P * 16 + k + 8 * u) * XS + cc] = -s;
     }
-#pragma unroll
-    for (int I = 0; I < 4; ++I) Ms[(16 * I + r) * MS_LD + 16 * I + cc] = Xd[(I * 16 + r) * 16 + cc];
   }
   __syncthreads();
-  // 32-level products: thread (warp, lane) computes rows warp + 8k (k < 4) of
-  // column lane, so each column operand load serves four rows
-  auto prod32 = [&](const float* A, int lda, const float* B, int ldb, float (&s)[4]) {
+  {  // C: warp w -> column cc = 16 (w / 4) + 4 (w % 4) + lane / 8, rows k + 8u (k = lane % 8, u < 4)
+    const int cc = 16 * (warp >> 2) + 4 * (warp & 3) + (lane >> 3), k = lane & 7;
+    float y[4];
+    if (warp < 4) {  // cc < 16: column of X_00 = [Xd0 ; XB0] column cc
+      float xc[32];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) s[k] = 0.f;
+      for (int m = 0; m < 16; ++m) { xc[m] = Xd[m * XS + cc]; xc[16 + m] = XB[m * XS + cc]; }
 #pragma unroll
-    for (int m4 = 0; m4 < 32; m4 += 4) {
-      const float b0 = B[m4 * ldb + lane], b1 = B[(m4 + 1) * ldb + lane], b2 = B[(m4 + 2) * ldb + lane],
-                  b3 = B[(m4 + 3) * ldb + lane];
+      for (int u = 0; u < 4; ++u) {
+        const float* Lr = Ms + (32 + k + 8 * u) * MS_LD;
+        float s = 0.f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 a = *reinterpret_cast<const float4*>(A + (warp + 8 * k) * lda + m4);
-        s[k] += a.x * b0 + a.y * b1 + a.z * b2 + a.w * b3;
+        for (int m4 = 0; m4 < 32; m4 += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(Lr + m4);
+          s += a.x * xc[m4] + a.y * xc[m4 + 1] + a.z * xc[m4 + 2] + a.w * xc[m4 + 3];
+        }
+        y[u] = s;
+      }
+    } else {  // cc >= 16: column of X_00 = [0 ; Xd1] column cc - 16
+      float xc[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) xc[m] = Xd[(16 + m) * XS + (cc - 16)];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float* Lr = Ms + (32 + k + 8 * u) * MS_LD + 16;
+        float s = 0.f;
+#pragma unroll
+        for (int m4 = 0; m4 < 16; m4 += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(Lr + m4);
+          s += a.x * xc[m4] + a.y * xc[m4 + 1] + a.z * xc[m4 + 2] + a.w * xc[m4 + 3];
+        }
+        y[u] = s;
       }
     }
-  };
-  {  // Y = L_{10} X_{00}: rows 32..63, columns 0..31
-    float s[4];
-    prod32(Ms + 32 * MS_LD, MS_LD, Ms, MS_LD, s);
+    float yc[32];  // column cc of L_10 X_00, from the 8 lanes that share it
+    const int base = lane & ~7;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) Yt[(warp + 8 * k) * 32 + lane] = s[k];
-  }
-  __syncthreads();
-  {  // X_{10} = -X_{11} Y
-    float s[4];
-    prod32(Ms + 32 * MS_LD + 32, MS_LD, Yt, 32, s);
+    for (int kk = 0; kk < 8; ++kk)
 #pragma unroll
-    for (int k = 0; k < 4; ++k) Ms[(32 + warp + 8 * k) * MS_LD + lane] = -s[k];
+      for (int u = 0; u < 4; ++u) yc[kk + 8 * u] = __shfl_sync(0xffffffffu, y[u], base + kk);
+    // X_11 row r = [Xd2 row r, 0] (r < 16) or [XB1 row r - 16, Xd3 row r - 16]
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = k + 8 * u;  // u < 2: r < 16
+      const float* ra = u < 2 ? Xd + (32 + r) * XS : XB + r * XS;  // Xd2 row r / XB1 row r - 16
+      const float* rb = u < 2 ? Zr : Xd + (32 + r) * XS;             // zero / Xd3 row r - 16
+      float s = 0.f;
+#pragma unroll
+      for (int m4 = 0; m4 < 16; m4 += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(ra + m4);
+        s += a.x * yc[m4] + a.y * yc[m4 + 1] + a.z * yc[m4 + 2] + a.w * yc[m4 + 3];
+        if (u >= 2) {
+          const float4 b = *reinterpret_cast<const float4*>(rb + m4);
+          s += b.x * yc[16 + m4] + b.y * yc[16 + m4 + 1] + b.z * yc[16 + m4 + 2] + b.w * yc[16 + m4 + 3];
+        }
+      }
+      XC[r * XCS + cc] = -s;
+    }
   }
   __syncthreads();
 
@@ -468,7 +512,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float4 tv, ts;
     float* tvp = &tv.x;
     float* tsp = &ts.x;
-    const float4 xr = *reinterpret_cast<const float4*>(Ms + t * MS_LD + tp);
+    // X row t, columns tp .. tp + 3 (one 16-block): diagonal block, off-diagonal
+    // 16-block of a 32-half, the off-diagonal 32-block, or zero
+    const int I = t >> 4, J = tp >> 4;
+    const float* src = I == J ? Xd + (I * 16 + (t & 15)) * XS + (tp & 15)
+                     : (I == J + 1 && (I & 1)) ? XB + ((I >> 1) * 16 + (t & 15)) * XS + (tp & 15)
+                     : (I >= 2 && J <= 1) ? XC + (t - 32) * XCS + tp
+                     : Zr;
+    const float4 xr = *reinterpret_cast<const float4*>(src);
     const float* xrp = &xr.x;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
