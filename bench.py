@@ -49,6 +49,14 @@ DEC_BYTES_PER_PAIR = 2 * STATE_BYTES + 4 * D * 2 + D * 4 + 2 + 2 * 9 * D * 2
 # kernels launched per call: kda_prefill bf16 = chunk_prep + chunk_scan + conv tail
 PREFILL_LAUNCHES = 3
 DECODE_LAUNCHES = 1
+# multi-token decode (verify R rows, commit the kept prefix), per (sequence, head):
+# state read by verify, read and written by commit; per row the deltas
+# (k_hat, u, alpha fp32) written and read back, q k v g read, beta, o fp32;
+# the conv cache read by both calls and written by commit
+MTP_ROWS = 6
+MTP_BYTES_PER_PAIR = (3 * STATE_BYTES + MTP_ROWS * (2 * 3 * D * 4 + 4 * D * 2 + 2 + D * 4)
+                      + 3 * 9 * D * 2)
+MTP_LAUNCHES = 2
 
 
 def peaks():
@@ -263,8 +271,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
     hbm_peak, bf16_peak, peak_src = peaks()
 
-    if args.no_prefill:  # decode leg only (profiling)
-        print(json.dumps({"decode": run_decode(args, world, dev, stream, kda, hbm_peak)}), flush=True)
+    if args.no_prefill:  # decode legs only (profiling)
+        print(json.dumps({"decode": run_decode(args, world, dev, stream, kda, hbm_peak),
+                          "mtp": run_mtp(args, world, dev, stream, kda, hbm_peak)}), flush=True)
         return
 
     # ---------------- prefill: long-context workload, resident in HBM ----------
@@ -303,9 +312,10 @@ def main():
         e2e = run_e2e(args, world, stream, inp, d, o, S, step, tokens_per_rank)
 
     # ---------------- decode step: 256 sequences, state in place ----------------
-    dec_line = None
+    dec_line = mtp_line = None
     if not args.no_decode:
         dec_line = run_decode(args, world, dev, stream, kda, hbm_peak)
+        mtp_line = run_mtp(args, world, dev, stream, kda, hbm_peak)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -322,6 +332,7 @@ def main():
         "gpu_launches": args.steps * PREFILL_LAUNCHES,
         "clocks": clk.summary(),
         "decode": dec_line,
+        "mtp": mtp_line,
     }
     if (heads, T_run) != (H, T_LONG):
         line["config"]["note"] = "reduced profiling size, not the reported workload"
@@ -380,6 +391,38 @@ def run_decode(args, world, dev, stream, kda, hbm_peak):
                          "traffic": recorded_traffic("kda_decode"),
                          "algorithmic_bytes_per_launch": npairs * DEC_BYTES_PER_PAIR},
             "gpu_launches": args.steps * DECODE_LAUNCHES}
+
+
+def run_mtp(args, world, dev, stream, kda, hbm_peak):
+    """Multi-token decode for speculative serving: kda_decode_verify of 6 rows
+    (5 drafts + 1) per sequence, then kda_decode_commit of the kept prefix
+    (2..6 rows, about four on average), 256 sequences x 64 heads."""
+    N = args.decode_seqs
+    mt = ki.make_decode_rows(N, MTP_ROWS, H, torch.bfloat16, ki.BASE_SEED + 5, accept=(2, MTP_ROWS))
+    dd = {n: getattr(mt, n).to(dev) for n in ("state", "conv_cache", "q", "k", "v", "g", "beta", "conv_w")}
+    o_m = torch.empty(dd["q"].shape, dtype=torch.float32, device=dev)
+    deltas = torch.empty(kda.deltas_size(N, MTP_ROWS, H) // 4, dtype=torch.float32, device=dev)
+    n_acc = torch.from_numpy(mt.n_accept).to(dev)
+
+    def mstep():
+        kda.decode_verify(dd["state"], dd["conv_cache"], dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
+                          dd["conv_w"], o=o_m, deltas=deltas, stream=stream)
+        kda.decode_commit(dd["state"], dd["conv_cache"], dd["q"], dd["k"], dd["v"], deltas, n_acc, stream=stream)
+
+    _, steps = timed(mstep, args.steps, args.warmup, world, stream)
+    assert kda.check_async_status(stream) == 0
+    ms = statistics.mean(steps)
+    npairs = N * H
+    alg = npairs * MTP_BYTES_PER_PAIR
+    gbs = alg / (ms / 1e3) / 1e9
+    return {"workload": f"kda_decode_verify + kda_decode_commit: {N} sequences x {MTP_ROWS} rows, 64 heads x 128, "
+                        f"{int(mt.n_accept.sum())} rows kept, fp32 state in place",
+            "verified_rows_per_s": N * MTP_ROWS / (ms / 1e3), "kept_tokens_per_s": int(mt.n_accept.sum()) / (ms / 1e3),
+            "ms_per_step": ms, "state_gbs": npairs * 3 * STATE_BYTES / (ms / 1e3) / 1e9,
+            "roofline": {"kernel": "kda_decode_verify + kda_decode_commit", "bound": "hbm", "achieved": gbs,
+                         "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak, "traffic": None,
+                         "algorithmic_bytes_per_launch": alg},
+            "gpu_launches": args.steps * MTP_LAUNCHES}
 
 
 if __name__ == "__main__":

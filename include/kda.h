@@ -137,6 +137,69 @@ kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const 
                            kda_conv_act act, kda_dtype o_dt, void* o, void* stream);
 
 /*
+ * Multi-token decode for speculative serving (page "GLM-5.3-Flash Internals -
+ * a measured profile": the model serves with multi-token prediction, k = 5
+ * drafts, so one verify step carries 6 rows, and about four of them are
+ * accepted).  A step verifies R rows against each sequence's state without
+ * changing it, and a second call keeps the accepted prefix:
+ *
+ *   kda_decode_verify(state, cache, rows 0..R-1) -> o for every row, deltas
+ *   kda_decode_commit(state, cache, rows, deltas, n_accept) -> state and cache
+ *       after the first n_accept[n] rows of sequence n
+ *
+ * Row t of a sequence is decoded exactly as kda_decode_step would decode it
+ * after rows 0..t-1 (same arithmetic in the same order), so verify outputs and
+ * the committed state and cache equal those of n single-token steps, bit for
+ * bit.  The state is read once by verify and read and written once by commit,
+ * instead of once per row.
+ *
+ * Common arguments:
+ *   num_seqs N, num_rows R (1 <= R <= KDA_MAX_VERIFY_ROWS), num_heads H.
+ *   q, k, v, g : [N, R, H, 128] raw rows (dt), row t of sequence n at
+ *                (n * R + t); beta : [N, R, H].
+ *   deltas     : device scratch of kda_decode_deltas_size(N, R, H) bytes,
+ *                [N, H, R, 3, 128] fp32 (k_hat, u, alpha of each row), written
+ *                by verify and read by commit; caller-owned.
+ */
+#define KDA_MAX_VERIFY_ROWS 8
+size_t kda_decode_deltas_size(int num_seqs, int num_rows, int num_heads);
+
+/*
+ * kda_decode_verify -- decode rows 0..R-1 of every sequence in turn from
+ * `state` and `conv_cache`, neither of which is modified.
+ *   state      : [N, H, 128, 128] fp32, read only.
+ *   conv_cache : [N, 3, 3, H*128] (dt), read only.
+ *   conv_w     : [3, H*128, 4] fp32.
+ *   o_dt, o    : out [N, R, H, 128], row t = o of that row.
+ *   deltas     : out, see above.
+ * Errors: KDA_ERR_INVALID_ARG for R outside [1, KDA_MAX_VERIFY_ROWS], a NULL
+ * pointer, or outputs aliasing inputs; KDA_ERR_ALIGNMENT for a pointer that
+ * is not 16-byte aligned (beta: element aligned); KDA_ERR_UNSUPPORTED for
+ * N > 65535.  Nothing is launched on error.
+ */
+kda_status kda_decode_verify(const float* state, const void* conv_cache, const void* q, const void* k,
+                             const void* v, const void* g, const void* beta, const float* conv_w,
+                             int num_seqs, int num_rows, int num_heads, kda_dtype dt, kda_conv_act act,
+                             kda_dtype o_dt, void* o, float* deltas, void* stream);
+
+/*
+ * kda_decode_commit -- apply the first n_accept[n] verified rows of sequence
+ * n: state and conv_cache (same layouts as kda_decode_verify) are updated in
+ * place to what n_accept[n] calls of kda_decode_step would leave.
+ *   q, k, v  : the same raw rows that were verified (the conv cache takes the
+ *              last three raw tokens of [cache, accepted rows]).
+ *   deltas   : as written by kda_decode_verify for these rows and this state.
+ *   n_accept : [N] int32 on the device, each in [0, R]; 0 leaves that
+ *              sequence untouched.  A value outside [0, R] is clamped to it
+ *              and recorded as KDA_ERR_INVALID_ARG in the device status word
+ *              (kda_check_async_status).
+ * Errors as for kda_decode_verify.
+ */
+kda_status kda_decode_commit(float* state, void* conv_cache, const void* q, const void* k, const void* v,
+                             const float* deltas, const int32_t* n_accept, int num_seqs, int num_rows,
+                             int num_heads, kda_dtype dt, void* stream);
+
+/*
  * kda_prefill_noalloc -- kda_prefill for callers that cannot allocate device
  * memory.  (Not an operation of the method: the pages have no counterpart; it
  * only changes where the scratch lives.)
@@ -176,7 +239,8 @@ const char* kda_status_string(kda_status s);
  * Synchronises `stream`, then returns and clears the library's device status
  * word on the current device: KDA_OK, or KDA_ERR_TIMEOUT if a bounded
  * device-side wait gave up since the last call (the kernel that gave up
- * stopped early, so its outputs are invalid), or KDA_ERR_CUDA if the
+ * stopped early, so its outputs are invalid), KDA_ERR_INVALID_ARG if
+ * kda_decode_commit met an n_accept outside [0, R], or KDA_ERR_CUDA if the
  * synchronisation itself failed.
  */
 kda_status kda_check_async_status(void* stream);

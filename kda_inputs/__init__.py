@@ -28,7 +28,7 @@ import dataclasses
 import math
 import os
 from concurrent.futures import ThreadPoolExecutor
-from typing import List, Optional, Sequence
+from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
@@ -38,7 +38,7 @@ BASE_SEED = 20261202
 _BLOCK = 1 << 22  # elements per independently seeded block
 
 # stream ids: each tensor draws from its own substream
-_Q, _K, _V, _G, _BETA, _CONVW, _STATE, _CONV, _GSEL, _GU, _LEN = range(1, 12)
+_Q, _K, _V, _G, _BETA, _CONVW, _STATE, _CONV, _GSEL, _GU, _LEN, _ACC = range(1, 13)
 
 
 def _mix(seed: int, stream: int, block: int) -> int:
@@ -213,6 +213,53 @@ def make_decode(N: int, H: int, dtype: torch.dtype, seed: int, *, D: int = D_HEA
     beta = _draw((N, H), seed, _BETA, "n", dtype, fn=_sigmoid)
     conv_w = randn((3, H * D, 4), seed, _CONVW, std=0.5)
     return DecodeInputs(state, conv_cache, q, k, v, g, beta, conv_w, name)
+
+
+@dataclasses.dataclass
+class DecodeRowsInputs:
+    """R new rows per sequence for a multi-token (verify / commit) decode step,
+    with the number of rows each sequence keeps."""
+    state: torch.Tensor       # [N, H, D, D] fp32
+    conv_cache: torch.Tensor  # [N, 3, 3, H*D]
+    q: torch.Tensor           # [N, R, H, D]
+    k: torch.Tensor
+    v: torch.Tensor
+    g: torch.Tensor
+    beta: torch.Tensor        # [N, R, H]
+    conv_w: torch.Tensor
+    n_accept: np.ndarray      # int32 [N], each in [0, R]
+    name: str = ""
+
+    @property
+    def num_seqs(self) -> int:
+        return self.q.shape[0]
+
+    @property
+    def num_rows(self) -> int:
+        return self.q.shape[1]
+
+    @property
+    def num_heads(self) -> int:
+        return self.q.shape[2]
+
+
+def make_decode_rows(N: int, R: int, H: int, dtype: torch.dtype, seed: int, *, D: int = D_HEAD,
+                     state_std: float = 0.02, accept: Tuple[int, int] = (0, -1),
+                     name: str = "") -> DecodeRowsInputs:
+    """Distributions as the single-token decode workload; n_accept uniform on
+    the integers [accept[0], accept[1]] (accept[1] = -1 means R)."""
+    state = randn((N, H, D, D), seed, _STATE, std=state_std)
+    conv_cache = randn((N, 3, 3, H * D), seed, _CONV, dtype=dtype)
+    q = randn((N, R, H, D), seed, _Q, dtype=dtype)
+    k = randn((N, R, H, D), seed, _K, dtype=dtype)
+    v = randn((N, R, H, D), seed, _V, dtype=dtype)
+    g = gate_sigmoid((N, R, H, D), seed, dtype)
+    beta = _draw((N, R, H), seed, _BETA, "n", dtype, fn=_sigmoid)
+    conv_w = randn((3, H * D, 4), seed, _CONVW, std=0.5)
+    lo, hi = accept[0], (R if accept[1] < 0 else accept[1])
+    rng = np.random.default_rng(_mix(seed, _ACC, 0))
+    n_accept = rng.integers(lo, hi, size=N, endpoint=True).astype(np.int32)
+    return DecodeRowsInputs(state, conv_cache, q, k, v, g, beta, conv_w, n_accept, name)
 
 
 def varlen_lengths(seed: int, n: int = 16, lo: int = 1024, hi: int = 32768) -> List[int]:

@@ -27,7 +27,8 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 # every entry point declared in include/kda.h
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
            "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version",
-           "kda_prefill_noalloc")
+           "kda_prefill_noalloc", "kda_decode_deltas_size", "kda_decode_verify", "kda_decode_commit")
+MAX_VERIFY_ROWS = 8  # KDA_MAX_VERIFY_ROWS
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python "
@@ -50,6 +51,14 @@ NOALLOC_SCRATCH_BYTES = 128 << 20  # KDA_NOALLOC_SCRATCH_BYTES
 lib.kda_decode_step.restype = ctypes.c_int
 lib.kda_decode_step.argtypes = [_f32p, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
                                 ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp]
+lib.kda_decode_deltas_size.restype = ctypes.c_size_t
+lib.kda_decode_deltas_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+lib.kda_decode_verify.restype = ctypes.c_int
+lib.kda_decode_verify.argtypes = [_f32p, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _f32p, _vp]
+lib.kda_decode_commit.restype = ctypes.c_int
+lib.kda_decode_commit.argtypes = [_f32p, _vp, _vp, _vp, _vp, _f32p, _i32p, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int, _vp]
 lib.kda_status_string.restype = ctypes.c_char_p
 lib.kda_status_string.argtypes = [ctypes.c_int]
 lib.kda_check_async_status.restype = ctypes.c_int
@@ -164,6 +173,34 @@ def decode_step(state, conv_cache, q, k, v, g, beta, conv_w, act: int = KDA_CONV
                                _ptr(beta), _ptr(conv_w), N, H, _dtype_code(q), int(act), _dtype_code(o),
                                _ptr(o), _stream(stream)), "kda_decode_step")
     return o
+
+
+def deltas_size(num_seqs: int, num_rows: int, num_heads: int) -> int:
+    return int(lib.kda_decode_deltas_size(num_seqs, num_rows, num_heads))
+
+
+def decode_verify(state, conv_cache, q, k, v, g, beta, conv_w, act: int = KDA_CONV_NONE, o=None,
+                  deltas=None, stream=None, o_dtype=torch.float32):
+    """kda_decode_verify: rows [N, R, H, 128] decoded in turn from `state` and
+    `conv_cache` (neither modified).  Returns (o [N, R, H, 128], deltas)."""
+    N, R, H = q.shape[0], q.shape[1], q.shape[2]
+    if o is None:
+        o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
+    if deltas is None:
+        deltas = torch.empty(deltas_size(N, R, H) // 4, dtype=torch.float32, device=q.device)
+    _check(lib.kda_decode_verify(_ptr(state), _ptr(conv_cache), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 _ptr(conv_w), N, R, H, _dtype_code(q), int(act), _dtype_code(o), _ptr(o),
+                                 _ptr(deltas), _stream(stream)), "kda_decode_verify")
+    return o, deltas
+
+
+def decode_commit(state, conv_cache, q, k, v, deltas, n_accept, stream=None):
+    """kda_decode_commit: keep the first n_accept[n] verified rows of each
+    sequence (n_accept: int32 device tensor [N]); state and conv_cache are
+    updated in place."""
+    N, R, H = q.shape[0], q.shape[1], q.shape[2]
+    _check(lib.kda_decode_commit(_ptr(state), _ptr(conv_cache), _ptr(q), _ptr(k), _ptr(v), _ptr(deltas),
+                                 _ptr(n_accept), N, R, H, _dtype_code(q), _stream(stream)), "kda_decode_commit")
 
 
 def check_async_status(stream=None) -> int:

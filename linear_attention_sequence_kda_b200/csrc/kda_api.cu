@@ -6,6 +6,7 @@
 
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
+#include "kda_decode_multi.cuh"
 #include "kda_recurrent.cuh"
 #include "kda_tail.cuh"
 #include "kda_chunked.cuh"
@@ -126,6 +127,39 @@ void launch_decode(kda_conv_act act, kda_dtype o_dt, float* state, void* cache, 
   }
 }
 
+template <typename Tin, typename Tout, int ACT>
+void launch_verify_t(const float* state, const void* cache, const void* q, const void* k, const void* v,
+                     const void* g, const void* beta, const float* conv_w, int N, int R, int H, void* o,
+                     float* deltas, cudaStream_t s) {
+  decode_verify_kernel<Tin, Tout, ACT><<<dim3(H, N), 256, 0, s>>>(
+      state, (const Tin*)cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)g, (const Tin*)beta,
+      conv_w, R, H, (Tout*)o, deltas);
+}
+
+template <typename Tin>
+void launch_verify(kda_conv_act act, kda_dtype o_dt, const float* state, const void* cache, const void* q,
+                   const void* k, const void* v, const void* g, const void* beta, const float* conv_w, int N,
+                   int R, int H, void* o, float* deltas, cudaStream_t s) {
+  const bool silu = act == KDA_CONV_SILU;
+  if (o_dt == KDA_F32) {
+    if (silu) launch_verify_t<Tin, float, KDA_CONV_SILU>(state, cache, q, k, v, g, beta, conv_w, N, R, H, o, deltas, s);
+    else launch_verify_t<Tin, float, KDA_CONV_NONE>(state, cache, q, k, v, g, beta, conv_w, N, R, H, o, deltas, s);
+  } else {
+    if (silu)
+      launch_verify_t<Tin, __nv_bfloat16, KDA_CONV_SILU>(state, cache, q, k, v, g, beta, conv_w, N, R, H, o, deltas, s);
+    else
+      launch_verify_t<Tin, __nv_bfloat16, KDA_CONV_NONE>(state, cache, q, k, v, g, beta, conv_w, N, R, H, o, deltas, s);
+  }
+}
+
+// shared argument checks of the decode entry points
+kda_status check_decode_common(int num_seqs, int num_heads, kda_dtype dt) {
+  if (num_seqs < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
+  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (num_seqs > 65535) return KDA_ERR_UNSUPPORTED;
+  return KDA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -200,6 +234,62 @@ kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const 
   else
     launch_decode<__nv_bfloat16>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w,
                                  num_seqs, num_heads, o, s);
+  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+size_t kda_decode_deltas_size(int num_seqs, int num_rows, int num_heads) {
+  if (num_seqs < 0 || num_rows < 1 || num_rows > KDA_MAX_VERIFY_ROWS || num_heads < 1) return 0;
+  return (size_t)num_seqs * num_heads * num_rows * 3 * D * sizeof(float);
+}
+
+kda_status kda_decode_verify(const float* state, const void* conv_cache, const void* q, const void* k,
+                             const void* v, const void* g, const void* beta, const float* conv_w,
+                             int num_seqs, int num_rows, int num_heads, kda_dtype dt, kda_conv_act act,
+                             kda_dtype o_dt, void* o, float* deltas, void* stream) {
+  kda_status st = check_decode_common(num_seqs, num_heads, dt);
+  if (st != KDA_OK) return st;
+  if (num_rows < 1 || num_rows > KDA_MAX_VERIFY_ROWS) return KDA_ERR_INVALID_ARG;
+  if (o_dt != KDA_F32 && o_dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (act != KDA_CONV_NONE && act != KDA_CONV_SILU) return KDA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KDA_OK;
+  if (!state || !conv_cache || !q || !k || !v || !g || !beta || !conv_w || !o || !deltas)
+    return KDA_ERR_INVALID_ARG;
+  const void* al16[] = {state, conv_cache, q, k, v, g, conv_w, o, deltas};
+  for (const void* p : al16)
+    if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+  if (!aligned(beta, esize(dt))) return KDA_ERR_ALIGNMENT;
+  if (o == q || o == k || o == v || o == g || (const void*)deltas == (const void*)state) return KDA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (dt == KDA_F32)
+    launch_verify<float>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w, num_seqs, num_rows, num_heads, o,
+                         deltas, s);
+  else
+    launch_verify<__nv_bfloat16>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w, num_seqs, num_rows,
+                                 num_heads, o, deltas, s);
+  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_commit(float* state, void* conv_cache, const void* q, const void* k, const void* v,
+                             const float* deltas, const int32_t* n_accept, int num_seqs, int num_rows,
+                             int num_heads, kda_dtype dt, void* stream) {
+  kda_status st = check_decode_common(num_seqs, num_heads, dt);
+  if (st != KDA_OK) return st;
+  if (num_rows < 1 || num_rows > KDA_MAX_VERIFY_ROWS) return KDA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KDA_OK;
+  if (!state || !conv_cache || !q || !k || !v || !deltas || !n_accept) return KDA_ERR_INVALID_ARG;
+  const void* al16[] = {state, conv_cache, q, k, v, deltas};
+  for (const void* p : al16)
+    if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+  if (!aligned(n_accept, 4)) return KDA_ERR_ALIGNMENT;
+  cudaStream_t s = (cudaStream_t)stream;
+  const dim3 grid(num_heads, num_seqs);
+  if (dt == KDA_F32)
+    decode_commit_kernel<float><<<grid, 256, 0, s>>>(state, (float*)conv_cache, (const float*)q, (const float*)k,
+                                                      (const float*)v, deltas, n_accept, num_rows, num_heads);
+  else
+    decode_commit_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        state, (__nv_bfloat16*)conv_cache, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+        (const __nv_bfloat16*)v, deltas, n_accept, num_rows, num_heads);
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -168,6 +168,19 @@ def decode_problem(inp, n: int, h: int, act: int = 0) -> HeadProblem:
                        [c[0], c[1], c[2]], act)
 
 
+def decode_rows_problem(inp, n: int, h: int, rows: int, act: int = 0) -> HeadProblem:
+    """The first `rows` rows of sequence n, head h of a multi-row decode
+    (DecodeRowsInputs), decoded one after another from the sequence's state
+    and conv cache: the recurrence with T = rows and the cache as history.  Its
+    o holds the outputs of those rows, its final_state and tails the state and
+    cache after them."""
+    D = inp.q.shape[3]
+    w = inp.conv_w.view(3, -1, D, 4)[:, h]
+    c = inp.conv_cache.view(inp.num_seqs, 3, 3, -1, D)[n, :, :, h]
+    return HeadProblem(inp.q[n, :rows, h], inp.k[n, :rows, h], inp.v[n, :rows, h], inp.g[n, :rows, h],
+                       inp.beta[n, :rows, h], w[0], w[1], w[2], inp.state[n, h], [c[0], c[1], c[2]], act)
+
+
 def decode(inp, pairs: Optional[Iterable[Tuple[int, int]]] = None, act: int = 0,
            nthreads: Optional[int] = None) -> Dict[Tuple[int, int], HeadProblem]:
     """One decode step = the recurrence with T = 1 and the conv cache as

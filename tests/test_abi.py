@@ -99,3 +99,35 @@ def test_decode_argument_validation():
     assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, Q, None) == 1
     assert d(FS, CT, Q, K, V, G, B, W, 70000, 2, 1, 0, 0, O, None) == 2
     assert d(FS, CT, Q, K, V, G, B, W, 0, 2, 1, 0, 0, O, None) == 0
+
+
+DL, NA = 12 << 20, 13 << 20  # fake deltas and n_accept addresses
+
+
+def test_decode_rows_argument_validation():
+    assert kda.lib.kda_decode_deltas_size(4, 6, 2) == 4 * 2 * 6 * 3 * 128 * 4
+    assert kda.lib.kda_decode_deltas_size(4, 0, 2) == 0
+    assert kda.lib.kda_decode_deltas_size(4, kda.MAX_VERIFY_ROWS + 1, 2) == 0
+    vf = kda.lib.kda_decode_verify
+    #      state CT Q K V G B W  N  R  H dt act odt o  deltas
+    assert vf(None, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 0, 2, 1, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 9, 2, 1, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 0, 1, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 3, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, O, None, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, O, DL + 8, None) == 3
+    assert vf(FS, CT, Q, K, V, G, B + 1, W, 4, 6, 2, 1, 0, 0, O, DL, None) == 3
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, Q, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 70000, 6, 2, 1, 0, 0, O, DL, None) == 2
+    assert vf(FS, CT, Q, K, V, G, B, W, 0, 6, 2, 1, 0, 0, O, DL, None) == 0
+    cm = kda.lib.kda_decode_commit
+    #      state CT Q K V deltas n_acc N R H dt
+    assert cm(FS, CT, Q, K, V, DL, NA, 4, 0, 2, 1, None) == 1
+    assert cm(FS, CT, Q, K, V, DL, NA, 4, 6, 2, 7, None) == 1
+    assert cm(FS, CT, Q, K, V, None, NA, 4, 6, 2, 1, None) == 1
+    assert cm(FS, CT, Q, K, V, DL, None, 4, 6, 2, 1, None) == 1
+    assert cm(FS, CT, Q, K, V, DL, NA + 2, 4, 6, 2, 1, None) == 3
+    assert cm(FS + 4, CT, Q, K, V, DL, NA, 4, 6, 2, 1, None) == 3
+    assert cm(FS, CT, Q, K, V, DL, NA, 70000, 6, 2, 1, None) == 2
+    assert cm(FS, CT, Q, K, V, DL, NA, 0, 6, 2, 1, None) == 0

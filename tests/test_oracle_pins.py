@@ -326,6 +326,30 @@ def test_workload_zero_decode_matches_prefill():
         assert _rel(p.o, o) < 1e-12 and _rel(p.final_state, S) < 1e-12
 
 
+def test_decode_rows_wrapper_equals_chained_single_steps():
+    """The multi-row decode wrapper (rows of sequence n, head h of [N, R, H, D]
+    inputs, cache as history) keeping r rows equals r single-token steps that
+    carry the state and the conv cache; r = 0 keeps state and cache as given."""
+    inp = ki.make_decode_rows(3, 6, 2, torch.float32, 31)
+    for n in range(3):
+        for h in range(2):
+            c = inp.conv_cache.view(3, 3, 3, 2, D)[n, :, :, h].double().numpy()
+            w = inp.conv_w.view(3, 2, D, 4)[:, h].double().numpy()
+            S, hist, outs = inp.state[n, h].double().numpy(), [c[0], c[1], c[2]], []
+            for r in range(7):
+                p = oracle.decode_rows_problem(inp, n, h, r)
+                _solve(p)
+                assert np.array_equal(p.final_state, S) and np.array_equal(p.o, np.array(outs).reshape(r, D))
+                for x in range(3):
+                    assert np.array_equal(p.tail[x], hist[x])
+                if r < 6:
+                    step = _solve(HeadProblem(inp.q[n, r, h][None], inp.k[n, r, h][None], inp.v[n, r, h][None],
+                                              inp.g[n, r, h][None], inp.beta[n, r, h].reshape(1), w[0], w[1], w[2],
+                                              S, hist))
+                    outs.append(step.o[0])
+                    S, hist = step.final_state, step.tail
+
+
 # ---------------------------------------------------------------- page numbers
 
 def test_page_dimensions():
