@@ -412,17 +412,25 @@ def run_mtp(args, world, dev, stream, kda, hbm_peak):
     _, steps = timed(mstep, args.steps, args.warmup, world, stream)
     assert kda.check_async_status(stream) == 0
     ms = statistics.mean(steps)
+
+    def vstep():
+        kda.decode_verify(dd["state"], dd["conv_cache"], dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
+                          dd["conv_w"], o=o_m, deltas=deltas, stream=stream)
+
+    _, vsteps = timed(vstep, args.steps, args.warmup, world, stream)
+    verify_ms = statistics.mean(vsteps)
     npairs = N * H
     alg = npairs * MTP_BYTES_PER_PAIR
     gbs = alg / (ms / 1e3) / 1e9
     return {"workload": f"kda_decode_verify + kda_decode_commit: {N} sequences x {MTP_ROWS} rows, 64 heads x 128, "
                         f"{int(mt.n_accept.sum())} rows kept, fp32 state in place",
             "verified_rows_per_s": N * MTP_ROWS / (ms / 1e3), "kept_tokens_per_s": int(mt.n_accept.sum()) / (ms / 1e3),
-            "ms_per_step": ms, "state_gbs": npairs * 3 * STATE_BYTES / (ms / 1e3) / 1e9,
+            "ms_per_step": ms, "verify_ms": verify_ms, "commit_ms": ms - verify_ms,
+            "state_gbs": npairs * 3 * STATE_BYTES / (ms / 1e3) / 1e9,
             "roofline": {"kernel": "kda_decode_verify + kda_decode_commit", "bound": "hbm", "achieved": gbs,
                          "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak, "traffic": None,
                          "algorithmic_bytes_per_launch": alg},
-            "gpu_launches": args.steps * MTP_LAUNCHES}
+            "gpu_launches": args.steps * (MTP_LAUNCHES + 1)}
 
 
 if __name__ == "__main__":

@@ -31,9 +31,12 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
                      const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                      const Tin* __restrict__ g, const Tin* __restrict__ beta, const float* __restrict__ conv_w,
                      int R, int H, Tout* __restrict__ o, float* __restrict__ deltas) {
-  __shared__ __align__(16) float sh_kh[D], sh_ka[D], sh_qa[D], sh_al[D], sh_v[D], sh_u[D];
-  __shared__ __align__(16) float sh_r[8][D], sh_y[8][D];
-  __shared__ float sh_red[4][3];
+  // per row: k_hat, alpha * k_hat, alpha * q_hat, alpha, conv(v); the row
+  // prologues do not depend on the state, so all rows are prepared first
+  __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][D], sh_ka[MAX_VERIFY_ROWS][D],
+      sh_qa[MAX_VERIFY_ROWS][D], sh_al[MAX_VERIFY_ROWS][D], sh_v[MAX_VERIFY_ROWS][D];
+  __shared__ __align__(16) float sh_r[8][D], sh_y[8][D], sh_u[D];
+  __shared__ float sh_red[MAX_VERIFY_ROWS][4][3], sh_kq[MAX_VERIFY_ROWS], sh_beta[MAX_VERIFY_ROWS];
 
   const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -43,62 +46,90 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
 #pragma unroll
   for (int i = 0; i < 16; ++i) s[i] = ld_stream(S + (warp * 16 + i) * D + lane * 4);
 
-  // conv taps and history of this thread's channel: threads 0..127 q and k,
-  // threads 128..255 v (history = the cache, then the rows of this call)
+  // 1. prologues of all rows: threads 0..127 q and k of channel c, threads
+  //    128..255 v and the gate (conv history = the cache, then earlier rows)
   const int c = tid & (D - 1);
   const int64_t ch = (int64_t)h * D + c;
   const Tin* cb = cache + (int64_t)n * 9 * HD + ch;  // [3 x][3 t] stride HD
-  float4 w0, w1;
-  float h0[3], h1[3];
+  float yq[MAX_VERIFY_ROWS], yk[MAX_VERIFY_ROWS];
+  // raw inputs of all rows are loaded before any is used, so that their
+  // global-memory latencies overlap instead of adding up row by row
   if (tid < D) {
-    w0 = load4(conv_w + (0 * HD + ch) * 4);
-    w1 = load4(conv_w + (1 * HD + ch) * 4);
-    for (int j = 0; j < 3; ++j) { h0[j] = to_f(cb[j * HD]); h1[j] = to_f(cb[(3 + j) * HD]); }
+    float xqs[MAX_VERIFY_ROWS], xks[MAX_VERIFY_ROWS];
+#pragma unroll
+    for (int t = 0; t < MAX_VERIFY_ROWS; ++t) {
+      const int64_t tok = (((int64_t)n * R + t) * H + h) * D + c;  // [N, R, H, D]
+      xqs[t] = t < R ? to_f(q[tok]) : 0.f;
+      xks[t] = t < R ? to_f(k[tok]) : 0.f;
+    }
+    const float4 wq = load4(conv_w + (0 * HD + ch) * 4), wk = load4(conv_w + (1 * HD + ch) * 4);
+    float hq[3], hk[3];
+    for (int j = 0; j < 3; ++j) { hq[j] = to_f(cb[j * HD]); hk[j] = to_f(cb[(3 + j) * HD]); }
+#pragma unroll
+    for (int t = 0; t < MAX_VERIFY_ROWS; ++t) {
+      if (t < R) {
+        const float xq = xqs[t], xk = xks[t];
+        float a = conv4(wq, hq[0], hq[1], hq[2], xq);
+        float b = conv4(wk, hk[0], hk[1], hk[2], xk);
+        if (ACT == KDA_CONV_SILU) { a = silu(a); b = silu(b); }
+        hq[0] = hq[1]; hq[1] = hq[2]; hq[2] = xq;
+        hk[0] = hk[1]; hk[1] = hk[2]; hk[2] = xk;
+        yq[t] = a; yk[t] = b;
+        const float nq = warp_sum(a * a), nk = warp_sum(b * b), qk = warp_sum(a * b);
+        if (lane == 0) { sh_red[t][warp][0] = nq; sh_red[t][warp][1] = nk; sh_red[t][warp][2] = qk; }
+      }
+    }
   } else {
-    w0 = load4(conv_w + (2 * HD + ch) * 4);
-    w1 = w0;
-    for (int j = 0; j < 3; ++j) { h0[j] = to_f(cb[(6 + j) * HD]); h1[j] = 0.f; }
+    float xvs[MAX_VERIFY_ROWS], xgs[MAX_VERIFY_ROWS];
+#pragma unroll
+    for (int t = 0; t < MAX_VERIFY_ROWS; ++t) {
+      const int64_t tok = (((int64_t)n * R + t) * H + h) * D + c;
+      xvs[t] = t < R ? to_f(v[tok]) : 0.f;
+      xgs[t] = t < R ? to_f(g[tok]) : 0.f;
+    }
+    if (c < R) sh_beta[c] = to_f(beta[((int64_t)n * R + c) * H + h]);
+    const float4 wv = load4(conv_w + (2 * HD + ch) * 4);
+    float hv[3];
+    for (int j = 0; j < 3; ++j) hv[j] = to_f(cb[(6 + j) * HD]);
+#pragma unroll
+    for (int t = 0; t < MAX_VERIFY_ROWS; ++t) {
+      if (t < R) {
+        const float xv = xvs[t];
+        float yv = conv4(wv, hv[0], hv[1], hv[2], xv);
+        if (ACT == KDA_CONV_SILU) yv = silu(yv);
+        hv[0] = hv[1]; hv[1] = hv[2]; hv[2] = xv;
+        sh_v[t][c] = yv;
+        sh_al[t][c] = __expf(fmaxf(xgs[t], LOG_DECAY_FLOOR));
+      }
+    }
   }
-  float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;  // [R][3][D]
+  __syncthreads();
+  if (tid < D) {
+#pragma unroll
+    for (int t = 0; t < MAX_VERIFY_ROWS; ++t) {
+      if (t < R) {
+        const float nq = sh_red[t][0][0] + sh_red[t][1][0] + sh_red[t][2][0] + sh_red[t][3][0];
+        const float nk = sh_red[t][0][1] + sh_red[t][1][1] + sh_red[t][2][1] + sh_red[t][3][1];
+        const float qk = sh_red[t][0][2] + sh_red[t][1][2] + sh_red[t][2][2] + sh_red[t][3][2];
+        const float rq = rsqrtf(nq + NORM_EPS), rk = rsqrtf(nk + NORM_EPS);
+        const float a = sh_al[t][c];
+        const float kh = yk[t] * rk;
+        sh_kh[t][c] = kh;
+        sh_ka[t][c] = a * kh;
+        sh_qa[t][c] = a * yq[t] * rq;
+        if (c == 0) sh_kq[t] = qk * rq * rk;
+      }
+    }
+  }
+  __syncthreads();
 
+  // 2. the rows in turn against the state held in registers
+  float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;  // [R][3][D]
   for (int t = 0; t < R; ++t) {
-    const int64_t tok = (((int64_t)n * R + t) * H + h) * D + c;  // [N, R, H, D]
-    float yq = 0.f, yk = 0.f;
-    if (tid < D) {
-      const float xq = to_f(q[tok]), xk = to_f(k[tok]);
-      yq = conv4(w0, h0[0], h0[1], h0[2], xq);
-      yk = conv4(w1, h1[0], h1[1], h1[2], xk);
-      if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
-      h0[0] = h0[1]; h0[1] = h0[2]; h0[2] = xq;
-      h1[0] = h1[1]; h1[1] = h1[2]; h1[2] = xk;
-      float nq = warp_sum(yq * yq), nk = warp_sum(yk * yk), qk = warp_sum(yq * yk);
-      if (lane == 0) { sh_red[warp][0] = nq; sh_red[warp][1] = nk; sh_red[warp][2] = qk; }
-    } else {
-      const float xv = to_f(v[tok]);
-      float yv = conv4(w0, h0[0], h0[1], h0[2], xv);
-      if (ACT == KDA_CONV_SILU) yv = silu(yv);
-      h0[0] = h0[1]; h0[1] = h0[2]; h0[2] = xv;
-      sh_v[c] = yv;
-      sh_al[c] = __expf(fmaxf(to_f(g[tok]), LOG_DECAY_FLOOR));
-    }
-    __syncthreads();
-    const float nq = sh_red[0][0] + sh_red[1][0] + sh_red[2][0] + sh_red[3][0];
-    const float nk = sh_red[0][1] + sh_red[1][1] + sh_red[2][1] + sh_red[3][1];
-    const float qk = sh_red[0][2] + sh_red[1][2] + sh_red[2][2] + sh_red[3][2];
-    const float rq = rsqrtf(nq + NORM_EPS), rk = rsqrtf(nk + NORM_EPS);
-    const float kq = qk * rq * rk;
-    if (tid < D) {
-      const float a = sh_al[c];
-      const float kh = yk * rk;
-      sh_kh[c] = kh;
-      sh_ka[c] = a * kh;
-      sh_qa[c] = a * yq * rq;
-    }
-    __syncthreads();
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f), y = r;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const float ka = sh_ka[warp * 16 + i], qa = sh_qa[warp * 16 + i];
+      const float ka = sh_ka[t][warp * 16 + i], qa = sh_qa[t][warp * 16 + i];
       r.x = fmaf(s[i].x, ka, r.x); r.y = fmaf(s[i].y, ka, r.y);
       r.z = fmaf(s[i].z, ka, r.z); r.w = fmaf(s[i].w, ka, r.w);
       y.x = fmaf(s[i].x, qa, y.x); y.y = fmaf(s[i].y, qa, y.y);
@@ -111,27 +142,27 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
       float rr = 0.f, yy = 0.f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) { rr += sh_r[w][tid]; yy += sh_y[w][tid]; }
-      const float b = to_f(beta[((int64_t)n * R + t) * H + h]);
-      const float u = b * (sh_v[tid] - rr);
+      const float u = sh_beta[t] * (sh_v[t][tid] - rr);
       sh_u[tid] = u;
-      o[tok] = from_f<Tout>(yy + u * kq);
-      dl[(t * 3 + 0) * D + tid] = sh_kh[tid];
+      o[(((int64_t)n * R + t) * H + h) * D + tid] = from_f<Tout>(yy + u * sh_kq[t]);
+      dl[(t * 3 + 0) * D + tid] = sh_kh[t][tid];
       dl[(t * 3 + 1) * D + tid] = u;
-      dl[(t * 3 + 2) * D + tid] = sh_al[tid];
+      dl[(t * 3 + 2) * D + tid] = sh_al[t][tid];
     }
     __syncthreads();
-    // S <- Diag(a) S + k u^T in registers (the same expression as the single step)
+    // S <- Diag(a) S + k u^T in registers (the same expression as the single
+    // step).  sh_r / sh_y of the next row are written only after every thread
+    // has passed the barrier above, i.e. after they were read.
     const float4 u4 = *reinterpret_cast<const float4*>(&sh_u[lane * 4]);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int row = warp * 16 + i;
-      const float a = sh_al[row], kh = sh_kh[row];
+      const float a = sh_al[t][row], kh = sh_kh[t][row];
       s[i].x = fmaf(a, s[i].x, kh * u4.x);
       s[i].y = fmaf(a, s[i].y, kh * u4.y);
       s[i].z = fmaf(a, s[i].z, kh * u4.z);
       s[i].w = fmaf(a, s[i].w, kh * u4.w);
     }
-    __syncthreads();  // shared rows are rewritten by the next row's prologue
   }
 }
 
