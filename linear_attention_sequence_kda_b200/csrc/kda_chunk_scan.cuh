@@ -21,9 +21,10 @@
 // Warp roles, handing off through mbarriers (no block-wide barrier inside the
 // chunk loop):
 //   warps 0..15 compute: warp w serves TMEM lanes 32 (w % 4) .. (value columns)
-//               and token / key quarter w / 4 of every per-chunk step: the fp32
-//               updates of chunk i, the short conv of v for chunk i + 1 while
-//               MMA2 of chunk i runs, then the output tile of chunk i.
+//               and token / key quarter w / 4 of every per-chunk step: the short
+//               conv of v for chunk i + 1 (into registers) while MMA_A of
+//               chunk i runs, the fp32 updates of chunk i, then the output
+//               tile of chunk i.
 //   warp 16     one thread issues the MMAs.
 //   warp 17     one thread issues the loads, each as soon as the step that
 //               read the previous contents of its buffer is done.
@@ -171,13 +172,21 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       };
       bool ok = true;
       if (nchunks > 0) { load_a(0); load_v(0); load_pk(0); }
-      // loads for chunk j, in the order their buffers free up during chunk j - 1
+      if (nchunks > 1) {  // the conv of chunk 0 has read value tile 0
+        ok = tc::bar_wait_or(&bar_vfree, 0, abort_flag);
+        if (ok) load_v(1);
+      }
+      // record pieces of chunk j as their buffers free up during chunk j - 1;
+      // value tile j + 1 once the conv of chunk j (done early in chunk j - 1)
+      // has read tile j
       for (int j = 1; j < nchunks && ok; ++j) {
         const uint32_t q = (j - 1) & 1;
-        ok = tc::bar_wait_or(&bar_vfree, q, abort_flag);  // the conv has read value tile j - 1
-        if (ok) load_v(j);
-        ok = ok && tc::bar_wait_or(&bar_ma, q, abort_flag);  // MMA_A of chunk j - 1 has read the first piece
+        ok = tc::bar_wait_or(&bar_ma, q, abort_flag);  // MMA_A of chunk j - 1 has read the first piece
         if (ok) load_a(j);
+        if (ok && j + 1 < nchunks) {
+          ok = tc::bar_wait_or(&bar_vfree, j & 1, abort_flag);
+          if (ok) load_v(j + 1);
+        }
         ok = ok && tc::bar_wait_or(&bar_pkfree, q, abort_flag);  // MMA2 of chunk j - 1 has read the second
         if (ok) load_pk(j);
       }
@@ -236,8 +245,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     }
     const float4 wv = load4(conv_w + (2 * HD + chan) * 4);
     const float* scal = reinterpret_cast<const float*>(sm + SCAN_PK + (REC_SC - REC_PS));
-    // short conv of v for chunk i, tokens t0 .. t0 + 15 -> V^T (tf32 and fp32)
-    auto conv_v = [&](int i) -> bool {
+    // short conv of v for chunk i, tokens t0 .. t0 + 15, into registers (the
+    // value tile is released as soon as it has been read)
+    auto conv_v = [&](int i, float (&vv)[16]) -> bool {
       if (!tc::bar_wait_or(&bar_v, (uint32_t)(i & 1), abort_flag)) return false;
       const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + SCAN_V);
       const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
@@ -256,7 +266,6 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         }
         h0 = hh[0]; h1 = hh[1]; h2 = hh[2];
       }
-      float vv[16], r[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int t = t0 + j;
@@ -265,23 +274,37 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         if (ACT == KDA_CONV_SILU) y = silu(y);
         h0 = h1; h1 = h2; h2 = x;
         vv[j] = t < L ? y : 0.f;
-        r[j] = tc::to_tf32(vv[j]);
       }
-      tc::st16(tl + TM_V + t0, r);
-      tc::st16(tl + TM_VX + t0, vv);
-      tc::st_wait();
-      tc::fence_before();
-      tc::bar_arrive(&bar_conv);
       tc::bar_arrive(&bar_vfree);  // value tile i has been read
       return true;
     };
+    // V^T (tf32 MMA operand) and V^T fp32 of a chunk from its conv registers
+    auto store_v = [&](const float (&vv)[16]) {
+      float r[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) r[j] = tc::to_tf32(vv[j]);
+      tc::st16(tl + TM_V + t0, r);
+      tc::st16(tl + TM_VX + t0, vv);
+    };
 
     bool ok = true;
-    if (nchunks > 0) ok = conv_v(0);
+    float vn[16];  // conv of the next chunk's values until its TMEM columns are free
+    if (nchunks > 0) {
+      ok = conv_v(0, vn);
+      if (ok) {
+        store_v(vn);
+        tc::st_wait();
+        tc::fence_before();
+        tc::bar_arrive(&bar_conv);
+      }
+    }
     for (int i = 0; i < nchunks && ok; ++i) {
       const uint32_t p = i & 1;
-      // (a) U^T of this chunk (S^T read by the tensor core) and its scalars
-      ok = tc::bar_wait_or(&bar_ma, p, abort_flag);
+      const bool more = i + 1 < nchunks;
+      // (a) the next chunk's value conv while MMA_A of this chunk runs, then
+      //     U^T of this chunk (S^T read by the tensor core) and its scalars
+      if (more) ok = conv_v(i + 1, vn);
+      ok = ok && tc::bar_wait_or(&bar_ma, p, abort_flag);
       ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag);
       if (!ok) break;
       tc::fence_after();
@@ -303,6 +326,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       tc::st_wait();
       tc::fence_before();
       tc::bar_arrive(&bar_b);
+      // V^T of the next chunk: MMA_A of this chunk has read V^T, and V^T fp32
+      // was read just above
+      if (more) store_v(vn);
       // (c) S^T <- S^T diag(gamma) while O^T += U^T P_s^T runs
       {
         float r0[16], r1[16];
@@ -320,8 +346,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       tc::st_wait();
       tc::fence_before();
       tc::bar_arrive(&bar_d);
-      // (d) the next chunk's value conv while MMA2 runs
-      if (i + 1 < nchunks) ok = conv_v(i + 1);
+      if (more) tc::bar_arrive(&bar_conv);
       // (e) o = O + P_tt u once MMA2 is done, into the staging tile of this
       // parity (free once the store of chunk i - 2 has read it)
       ok = ok && tc::bar_wait_or(&bar_m2, p, abort_flag);

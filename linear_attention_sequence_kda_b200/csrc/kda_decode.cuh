@@ -19,6 +19,51 @@
 
 namespace kda {
 
+// A warp's 16 state rows, lane l holding columns [4l, 4l+4) of each: s[i] is
+// row i.  The two helpers below are the whole state arithmetic of a decode
+// step, shared by the single-token and the multi-token kernels so that both
+// round identically.  Packed f32x2 instructions do two columns at a time; each
+// column is rounded as its scalar fmaf would round it.
+//
+// r = sum_i x_i s_i and y = sum_i z_i s_i over the 16 rows, i ascending
+// (x, z: this warp's 16 entries, shared memory, 16-byte aligned).
+__device__ __forceinline__ void rows_dot2(const float4 (&s)[16], const float* x, const float* z, float4& r,
+                                          float4& y) {
+  float2 r0 = make_float2(0.f, 0.f), r1 = r0, y0 = r0, y1 = r0;
+#pragma unroll
+  for (int i4 = 0; i4 < 4; ++i4) {
+    const float4 x4 = *reinterpret_cast<const float4*>(x + 4 * i4);
+    const float4 z4 = *reinterpret_cast<const float4*>(z + 4 * i4);
+    const float xs[4] = {x4.x, x4.y, x4.z, x4.w}, zs[4] = {z4.x, z4.y, z4.z, z4.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 si = s[4 * i4 + j];
+      r0 = fma2(lo2(si), dup2(xs[j]), r0); r1 = fma2(hi2(si), dup2(xs[j]), r1);
+      y0 = fma2(lo2(si), dup2(zs[j]), y0); y1 = fma2(hi2(si), dup2(zs[j]), y1);
+    }
+  }
+  r = cat2(r0, r1);
+  y = cat2(y0, y1);
+}
+
+// s_i <- a_i s_i + kh_i u (the delta-rule row update Diag(a) S + k u^T; a, kh:
+// this warp's 16 entries in shared memory, u4: this lane's 4 columns of u).
+__device__ __forceinline__ void rows_update(float4 (&s)[16], const float* a, const float* kh, float4 u4) {
+  const float2 u0 = lo2(u4), u1 = hi2(u4);
+#pragma unroll
+  for (int i4 = 0; i4 < 4; ++i4) {
+    const float4 a4 = *reinterpret_cast<const float4*>(a + 4 * i4);
+    const float4 k4 = *reinterpret_cast<const float4*>(kh + 4 * i4);
+    const float as[4] = {a4.x, a4.y, a4.z, a4.w}, ks[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float4& si = s[4 * i4 + j];
+      si = cat2(fma2(dup2(as[j]), lo2(si), mul2(dup2(ks[j]), u0)),
+                fma2(dup2(as[j]), hi2(si), mul2(dup2(ks[j]), u1)));
+    }
+  }
+}
+
 template <typename Tin, typename Tout, int ACT>
 __global__ void __launch_bounds__(256, 2)
 decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
@@ -85,15 +130,8 @@ decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __r
   __syncthreads();
 
   // 3. partial reductions over this warp's 16 rows, 4 columns per lane
-  float4 r = make_float4(0.f, 0.f, 0.f, 0.f), y = r;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float ka = sh_ka[warp * 16 + i], qa = sh_qa[warp * 16 + i];
-    r.x = fmaf(s[i].x, ka, r.x); r.y = fmaf(s[i].y, ka, r.y);
-    r.z = fmaf(s[i].z, ka, r.z); r.w = fmaf(s[i].w, ka, r.w);
-    y.x = fmaf(s[i].x, qa, y.x); y.y = fmaf(s[i].y, qa, y.y);
-    y.z = fmaf(s[i].z, qa, y.z); y.w = fmaf(s[i].w, qa, y.w);
-  }
+  float4 r, y;
+  rows_dot2(s, &sh_ka[warp * 16], &sh_qa[warp * 16], r, y);
   *reinterpret_cast<float4*>(&sh_r[warp][lane * 4]) = r;
   *reinterpret_cast<float4*>(&sh_y[warp][lane * 4]) = y;
   __syncthreads();
@@ -109,18 +147,9 @@ decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __r
   __syncthreads();
 
   // 4. S <- Diag(a) S + k u^T, written once
-  const float4 u4 = *reinterpret_cast<const float4*>(&sh_u[lane * 4]);
+  rows_update(s, &sh_al[warp * 16], &sh_kh[warp * 16], *reinterpret_cast<const float4*>(&sh_u[lane * 4]));
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int row = warp * 16 + i;
-    const float a = sh_al[row], kh = sh_kh[row];
-    float4 t;
-    t.x = fmaf(a, s[i].x, kh * u4.x);
-    t.y = fmaf(a, s[i].y, kh * u4.y);
-    t.z = fmaf(a, s[i].z, kh * u4.z);
-    t.w = fmaf(a, s[i].w, kh * u4.w);
-    st_stream(S + row * D + lane * 4, t);
-  }
+  for (int i = 0; i < 16; ++i) st_stream(S + (warp * 16 + i) * D + lane * 4, s[i]);
 }
 
 }  // namespace kda

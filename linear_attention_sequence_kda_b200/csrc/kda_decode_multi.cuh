@@ -20,6 +20,7 @@
 // cache becomes the last three raw tokens of [cache, accepted rows].
 #pragma once
 #include "kda_common.cuh"
+#include "kda_decode.cuh"
 
 namespace kda {
 
@@ -50,6 +51,7 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
   //    128..255 v and the gate (conv history = the cache, then earlier rows)
   const int c = tid & (D - 1);
   const int64_t ch = (int64_t)h * D + c;
+  float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;  // [R][3 (k_hat, u, alpha)][D]
   const Tin* cb = cache + (int64_t)n * 9 * HD + ch;  // [3 x][3 t] stride HD
   float yq[MAX_VERIFY_ROWS], yk[MAX_VERIFY_ROWS];
   // raw inputs of all rows are loaded before any is used, so that their
@@ -118,51 +120,40 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
         sh_ka[t][c] = a * kh;
         sh_qa[t][c] = a * yq[t] * rq;
         if (c == 0) sh_kq[t] = qk * rq * rk;
+        dl[(t * 3 + 0) * D + c] = kh;  // the parts of the row's update that do
+        dl[(t * 3 + 2) * D + c] = a;   // not depend on the state
       }
     }
   }
   __syncthreads();
 
-  // 2. the rows in turn against the state held in registers
-  float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;  // [R][3][D]
+  // 2. the rows in turn against the state held in registers: threads 0..127
+  //    finish r and u of channel c, threads 128..255 the readout y, which
+  //    they complete with u once it is in shared memory
   for (int t = 0; t < R; ++t) {
-    float4 r = make_float4(0.f, 0.f, 0.f, 0.f), y = r;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float ka = sh_ka[t][warp * 16 + i], qa = sh_qa[t][warp * 16 + i];
-      r.x = fmaf(s[i].x, ka, r.x); r.y = fmaf(s[i].y, ka, r.y);
-      r.z = fmaf(s[i].z, ka, r.z); r.w = fmaf(s[i].w, ka, r.w);
-      y.x = fmaf(s[i].x, qa, y.x); y.y = fmaf(s[i].y, qa, y.y);
-      y.z = fmaf(s[i].z, qa, y.z); y.w = fmaf(s[i].w, qa, y.w);
-    }
+    float4 r, y;
+    rows_dot2(s, &sh_ka[t][warp * 16], &sh_qa[t][warp * 16], r, y);
     *reinterpret_cast<float4*>(&sh_r[warp][lane * 4]) = r;
     *reinterpret_cast<float4*>(&sh_y[warp][lane * 4]) = y;
     __syncthreads();
+    float yy = 0.f;
     if (tid < D) {
-      float rr = 0.f, yy = 0.f;
+      float rr = 0.f;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) { rr += sh_r[w][tid]; yy += sh_y[w][tid]; }
-      const float u = sh_beta[t] * (sh_v[t][tid] - rr);
-      sh_u[tid] = u;
-      o[(((int64_t)n * R + t) * H + h) * D + tid] = from_f<Tout>(yy + u * sh_kq[t]);
-      dl[(t * 3 + 0) * D + tid] = sh_kh[t][tid];
-      dl[(t * 3 + 1) * D + tid] = u;
-      dl[(t * 3 + 2) * D + tid] = sh_al[t][tid];
+      for (int w = 0; w < 8; ++w) rr += sh_r[w][c];
+      const float u = sh_beta[t] * (sh_v[t][c] - rr);
+      sh_u[c] = u;
+      dl[(t * 3 + 1) * D + c] = u;
+    } else {
+#pragma unroll
+      for (int w = 0; w < 8; ++w) yy += sh_y[w][c];
     }
     __syncthreads();
-    // S <- Diag(a) S + k u^T in registers (the same expression as the single
-    // step).  sh_r / sh_y of the next row are written only after every thread
-    // has passed the barrier above, i.e. after they were read.
-    const float4 u4 = *reinterpret_cast<const float4*>(&sh_u[lane * 4]);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int row = warp * 16 + i;
-      const float a = sh_al[t][row], kh = sh_kh[t][row];
-      s[i].x = fmaf(a, s[i].x, kh * u4.x);
-      s[i].y = fmaf(a, s[i].y, kh * u4.y);
-      s[i].z = fmaf(a, s[i].z, kh * u4.z);
-      s[i].w = fmaf(a, s[i].w, kh * u4.w);
-    }
+    // sh_r / sh_y / sh_u of the next row are written only after every thread
+    // has passed the next row's first barrier, i.e. after these reads
+    if (tid >= D) o[(((int64_t)n * R + t) * H + h) * D + c] = from_f<Tout>(yy + sh_u[c] * sh_kq[t]);
+    if (t + 1 < R)
+      rows_update(s, &sh_al[t][warp * 16], &sh_kh[t][warp * 16], *reinterpret_cast<const float4*>(&sh_u[lane * 4]));
   }
 }
 
@@ -207,18 +198,8 @@ decode_commit_kernel(float* __restrict__ state, Tin* __restrict__ cache, const T
     for (int j = 0; j < 3; ++j) cb[j * HD] = nv[j];
   }
   __syncthreads();
-  for (int t = 0; t < na; ++t) {
-    const float4 u4 = *reinterpret_cast<const float4*>(&sh_u[t][lane * 4]);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int row = warp * 16 + i;
-      const float a = sh_al[t][row], kh = sh_kh[t][row];
-      s[i].x = fmaf(a, s[i].x, kh * u4.x);
-      s[i].y = fmaf(a, s[i].y, kh * u4.y);
-      s[i].z = fmaf(a, s[i].z, kh * u4.z);
-      s[i].w = fmaf(a, s[i].w, kh * u4.w);
-    }
-  }
+  for (int t = 0; t < na; ++t)
+    rows_update(s, &sh_al[t][warp * 16], &sh_kh[t][warp * 16], *reinterpret_cast<const float4*>(&sh_u[t][lane * 4]));
 #pragma unroll
   for (int i = 0; i < 16; ++i) st_stream(S + (warp * 16 + i) * D + lane * 4, s[i]);
 }
