@@ -55,7 +55,11 @@ class _Job(ctypes.Structure):
         ("act", ctypes.c_int),
         ("o", _dp), ("final_state", _dp),
         ("tq", _dp), ("tk", _dp), ("tv", _dp),
+        ("state_round", ctypes.c_int),
     ]
+
+# state storage modes of a HeadProblem (how the state is stored, see kda_oracle.c)
+STATE_EXACT, STATE_BF16_EACH_TOKEN, STATE_BF16_AT_END = 0, 1, 2
 
 
 def build(force: bool = False) -> str:
@@ -76,9 +80,19 @@ def _load():
         lib.kda_oracle_run_jobs.argtypes = [ctypes.POINTER(_Job), ctypes.c_int, ctypes.c_int]
         lib.kda_oracle_run_jobs.restype = ctypes.c_int
         lib.kda_oracle_job_size.restype = ctypes.c_int
+        lib.kda_oracle_round_bf16.argtypes = [_dp, _dp, ctypes.c_int64]
         assert lib.kda_oracle_job_size() == ctypes.sizeof(_Job), "oracle job struct mismatch"
         _lib = lib
     return _lib
+
+
+def round_bf16(x) -> np.ndarray:
+    """The oracle's state-storage rounding: each double to the nearest bf16
+    value, ties to even, without passing through float."""
+    a = _f64(x)
+    out = np.empty_like(a)
+    _load().kda_oracle_round_bf16(_ptr(a), _ptr(out), a.size)
+    return out
 
 
 def _f64(x) -> np.ndarray:
@@ -97,7 +111,8 @@ class HeadProblem:
     """One (sequence, head) problem in fp64: raw q/k/v/g/beta, conv taps,
     initial state and conv history; `run` fills o, final_state and the tails."""
 
-    def __init__(self, q, k, v, g, beta, wq, wk, wv, init_state=None, hist=None, act=0):
+    def __init__(self, q, k, v, g, beta, wq, wk, wv, init_state=None, hist=None, act=0,
+                 state_round=STATE_EXACT):
         self.q, self.k, self.v, self.g = _f64(q), _f64(k), _f64(v), _f64(g)
         self.beta = _f64(beta).reshape(-1)
         self.wq, self.wk, self.wv = _f64(wq), _f64(wk), _f64(wv)
@@ -110,6 +125,7 @@ class HeadProblem:
         self.init_state = None if init_state is None else _f64(init_state)
         self.hist = None if hist is None else [_f64(h) for h in hist]  # 3 x [3][d]
         self.act = int(act)
+        self.state_round = int(state_round)
         self.o = np.zeros((self.T, self.dv))
         self.final_state = np.zeros((self.dk, self.dv))
         self.tail = [np.zeros((3, self.dk)), np.zeros((3, self.dk)), np.zeros((3, self.dv))]
@@ -120,7 +136,7 @@ class HeadProblem:
                     _ptr(self.beta), _ptr(self.wq), _ptr(self.wk), _ptr(self.wv), _ptr(self.init_state),
                     _ptr(h[0] if h else None), _ptr(h[1] if h else None), _ptr(h[2] if h else None),
                     self.act, _ptr(self.o), _ptr(self.final_state),
-                    _ptr(self.tail[0]), _ptr(self.tail[1]), _ptr(self.tail[2]))
+                    _ptr(self.tail[0]), _ptr(self.tail[1]), _ptr(self.tail[2]), self.state_round)
 
 
 def run_problems(problems, nthreads: Optional[int] = None) -> int:
@@ -134,7 +150,7 @@ def run_problems(problems, nthreads: Optional[int] = None) -> int:
     return lib.kda_oracle_run_jobs(jobs, len(problems), int(nthreads or os.cpu_count() or 1))
 
 
-def prefill_problem(inp, n: int, h: int, act: int = 0) -> HeadProblem:
+def prefill_problem(inp, n: int, h: int, act: int = 0, state_round: int = STATE_EXACT) -> HeadProblem:
     """Extract (sequence n, head h) of packed PrefillInputs as a HeadProblem."""
     s0, s1 = int(inp.cu_seqlens[n]), int(inp.cu_seqlens[n + 1])
     D = inp.q.shape[2]
@@ -145,30 +161,31 @@ def prefill_problem(inp, n: int, h: int, act: int = 0) -> HeadProblem:
         hist = [c[0], c[1], c[2]]
     st = None if inp.init_state is None else inp.init_state[n, h]
     return HeadProblem(inp.q[s0:s1, h], inp.k[s0:s1, h], inp.v[s0:s1, h], inp.g[s0:s1, h],
-                       inp.beta[s0:s1, h], w[0], w[1], w[2], st, hist, act)
+                       inp.beta[s0:s1, h], w[0], w[1], w[2], st, hist, act, state_round)
 
 
 def prefill(inp, pairs: Optional[Iterable[Tuple[int, int]]] = None, act: int = 0,
-            nthreads: Optional[int] = None) -> Dict[Tuple[int, int], HeadProblem]:
+            nthreads: Optional[int] = None, state_round: int = STATE_EXACT) -> Dict[Tuple[int, int], HeadProblem]:
     """Run the oracle on (sequence, head) pairs of a packed prefill (all pairs
     by default).  Returns {(n, h): solved HeadProblem}."""
     if pairs is None:
         pairs = [(n, h) for n in range(inp.num_seqs) for h in range(inp.num_heads)]
-    probs = {p: prefill_problem(inp, p[0], p[1], act) for p in pairs}
+    probs = {p: prefill_problem(inp, p[0], p[1], act, state_round) for p in pairs}
     run_problems(probs.values(), nthreads)
     return probs
 
 
-def decode_problem(inp, n: int, h: int, act: int = 0) -> HeadProblem:
+def decode_problem(inp, n: int, h: int, act: int = 0, state_round: int = STATE_EXACT) -> HeadProblem:
     D = inp.q.shape[2]
     w = inp.conv_w.view(3, -1, D, 4)[:, h]
     c = inp.conv_cache.view(inp.num_seqs, 3, 3, -1, D)[n, :, :, h]
     return HeadProblem(inp.q[n, h][None], inp.k[n, h][None], inp.v[n, h][None], inp.g[n, h][None],
                        inp.beta[n, h].reshape(1), w[0], w[1], w[2], inp.state[n, h],
-                       [c[0], c[1], c[2]], act)
+                       [c[0], c[1], c[2]], act, state_round)
 
 
-def decode_rows_problem(inp, n: int, h: int, rows: int, act: int = 0) -> HeadProblem:
+def decode_rows_problem(inp, n: int, h: int, rows: int, act: int = 0,
+                        state_round: int = STATE_EXACT) -> HeadProblem:
     """The first `rows` rows of sequence n, head h of a multi-row decode
     (DecodeRowsInputs), decoded one after another from the sequence's state
     and conv cache: the recurrence with T = rows and the cache as history.  Its
@@ -178,15 +195,16 @@ def decode_rows_problem(inp, n: int, h: int, rows: int, act: int = 0) -> HeadPro
     w = inp.conv_w.view(3, -1, D, 4)[:, h]
     c = inp.conv_cache.view(inp.num_seqs, 3, 3, -1, D)[n, :, :, h]
     return HeadProblem(inp.q[n, :rows, h], inp.k[n, :rows, h], inp.v[n, :rows, h], inp.g[n, :rows, h],
-                       inp.beta[n, :rows, h], w[0], w[1], w[2], inp.state[n, h], [c[0], c[1], c[2]], act)
+                       inp.beta[n, :rows, h], w[0], w[1], w[2], inp.state[n, h], [c[0], c[1], c[2]], act,
+                       state_round)
 
 
 def decode(inp, pairs: Optional[Iterable[Tuple[int, int]]] = None, act: int = 0,
-           nthreads: Optional[int] = None) -> Dict[Tuple[int, int], HeadProblem]:
+           nthreads: Optional[int] = None, state_round: int = STATE_EXACT) -> Dict[Tuple[int, int], HeadProblem]:
     """One decode step = the recurrence with T = 1 and the conv cache as
     history; the updated cache is the problem's tail."""
     if pairs is None:
         pairs = [(n, h) for n in range(inp.num_seqs) for h in range(inp.num_heads)]
-    probs = {p: decode_problem(inp, p[0], p[1], act) for p in pairs}
+    probs = {p: decode_problem(inp, p[0], p[1], act, state_round) for p in pairs}
     run_problems(probs.values(), nthreads)
     return probs

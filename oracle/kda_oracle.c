@@ -56,7 +56,24 @@ typedef struct {
     double *final_state;    /* [dk][dv] out                                        */
     double *tq, *tk;        /* [3][dk] out: last 3 raw tokens of history+segment   */
     double *tv;             /* [3][dv] out                                         */
+    int state_round;        /* state storage: 0 = kept exact; 1 = rounded to bf16  */
+                            /* after every token (each token is one decode step    */
+                            /* whose state is stored); 2 = rounded to bf16 once,   */
+                            /* when the final state is stored                      */
 } kda_oracle_job;
+
+/* Round x to the nearest bfloat16 value (8 significant bits, exponent range
+ * of fp32), ties to even, directly from double (no intermediate float, so no
+ * double rounding).  |x| is far below the bf16 overflow threshold for states;
+ * larger values are not handled. */
+static double round_bf16(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    frexp(x, &e);                 /* |x| = m 2^e, 0.5 <= m < 1                   */
+    int shift = 8 - e;            /* 8 significant bits: ulp = 2^(e - 8)         */
+    if (e - 8 < -133) shift = 133;  /* bf16 subnormals: ulp 2^-133               */
+    return ldexp(nearbyint(ldexp(x, shift)), -shift);  /* default mode: ties even */
+}
 
 /* y_t[c] = sum_j w[c][j] * x_{t-3+j}[c], x_{<0} from the 3-token history. */
 static double conv_at(const double *x, const double *hist, const double *w,
@@ -143,7 +160,14 @@ void kda_oracle_run_job(const kda_oracle_job *jb) {
         for (int j = 0; j < dv; ++j) ot[j] = 0.0;
         for (int i = 0; i < dk; ++i)
             for (int j = 0; j < dv; ++j) ot[j] += S[i * dv + j] * qh[i];
+        /* 6. a decode step stores its state: in bf16 storage the next token
+         *    starts from the stored (rounded) values; the readout above used
+         *    the state before storage */
+        if (jb->state_round == 1)
+            for (int i = 0; i < dk * dv; ++i) S[i] = round_bf16(S[i]);
     }
+    if (jb->state_round == 2)
+        for (int i = 0; i < dk * dv; ++i) S[i] = round_bf16(S[i]);
     memcpy(jb->final_state, S, sizeof(double) * (size_t)dk * dv);
     conv_tail(jb->q, jb->cq, jb->T, dk, jb->tq);
     conv_tail(jb->k, jb->ck, jb->T, dk, jb->tk);
@@ -189,3 +213,8 @@ int kda_oracle_run_jobs(const kda_oracle_job *jobs, int njobs, int nthreads) {
 }
 
 int kda_oracle_job_size(void) { return (int)sizeof(kda_oracle_job); }
+
+/* The bf16 rounding above, exposed for its pin tests. */
+void kda_oracle_round_bf16(const double *x, double *y, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) y[i] = round_bf16(x[i]);
+}

@@ -350,6 +350,77 @@ def test_decode_rows_wrapper_equals_chained_single_steps():
                     S, hist = step.final_state, step.tail
 
 
+# ---------------------------------------------------------------- bf16 state storage
+
+def _bf16_neighbours(x):
+    """The two bf16 values around double x (truncation toward zero and the next
+    one away from zero), from frexp: 8 significant bits, fp32 exponent range."""
+    m, e = np.frexp(x)
+    ulp = np.ldexp(1.0, np.maximum(e - 8, -133))
+    lo = np.trunc(x / ulp) * ulp
+    return lo, lo + np.sign(x) * ulp, ulp
+
+
+def test_bf16_rounding_is_nearest_ties_to_even():
+    """Brute force on random doubles of every magnitude (and exact ties): the
+    result is one of the two neighbouring bf16 values, the nearer one, and on a
+    tie the one with an even last mantissa bit; it is representable as bf16
+    (an fp32 whose low 16 bits are zero)."""
+    r = _rng(5)
+    x = r.standard_normal(20000) * np.ldexp(1.0, r.integers(-140, 40, 20000))
+    lo, hi, ulp = _bf16_neighbours(x)
+    ties = lo[:2000] + np.sign(x[:2000]) * ulp[:2000] / 2  # exactly halfway
+    x = np.concatenate([x, ties, [0.0, 1.0, -2.5, 1 + 2 ** -8, 1 + 3 * 2 ** -8]])
+    lo, hi, ulp = _bf16_neighbours(x)
+    y = oracle.round_bf16(x)
+    assert np.all((y == lo) | (y == hi))
+    d_lo, d_hi = np.abs(x - lo), np.abs(x - hi)
+    nearer = np.where(d_lo < d_hi, lo, hi)
+    tie = d_lo == d_hi
+    assert np.array_equal(y[~tie], nearer[~tie])
+    even = np.where(np.round(lo / ulp) % 2 == 0, lo, hi)
+    assert np.array_equal(y[tie], even[tie]) and tie.sum() >= 2000
+    f = y.astype(np.float32)
+    assert np.array_equal(f.astype(np.float64), y) and not np.any(f.view(np.uint32) & 0xFFFF)
+
+
+def test_state_rounded_at_end_changes_only_the_stored_state():
+    """Storage in bf16 at the end of a call: outputs are those of the exact
+    recurrence and the final state is the exact final state rounded once."""
+    for seed, T in ((70, 1), (71, 37)):
+        a, b = _random_problem(seed, T), _random_problem(seed, T)
+        b.state_round = oracle.STATE_BF16_AT_END
+        _solve(a); _solve(b)
+        assert np.array_equal(a.o, b.o)
+        assert np.array_equal(b.final_state, oracle.round_bf16(a.final_state))
+
+
+def test_state_rounded_each_token_equals_chained_stored_steps():
+    """Storage in bf16 after every token = T single-token decode steps, each
+    starting from the previous step's stored (rounded) state and conv cache and
+    rounding its own final state once; the readout of a step uses the state
+    before storage.  The rounding does change the result (it is not a no-op)."""
+    T = 9
+    full = _random_problem(72, T)
+    full.state_round = oracle.STATE_BF16_EACH_TOKEN
+    _solve(full)
+    exact = _random_problem(72, T)
+    _solve(exact)
+    S, hist = full.init_state, full.hist
+    for t in range(T):
+        step = HeadProblem(full.q[t:t + 1], full.k[t:t + 1], full.v[t:t + 1], full.g[t:t + 1], full.beta[t:t + 1],
+                           full.wq, full.wk, full.wv, S, hist, 0, oracle.STATE_BF16_AT_END)
+        _solve(step)
+        assert np.array_equal(step.o[0], full.o[t]), t
+        S, hist = step.final_state, step.tail
+    assert np.array_equal(S, full.final_state)
+    # storage drift from the exact state: rounding moves each stored element by
+    # at most half a bf16 ulp (2^-9 relative) per step, and the largest
+    # elements are several rms, so after 9 steps max|err|/rms is about 2 %
+    drift = _rel(full.final_state, exact.final_state)
+    assert 2 ** -9 < drift < 0.05
+
+
 # ---------------------------------------------------------------- page numbers
 
 def test_page_dimensions():
