@@ -43,9 +43,14 @@ H, D, T_LONG = 64, 128, 65536
 # initial state in this workload).
 BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 2 + D * 4
 STATE_BYTES = D * D * 4
-# decode: per (sequence, head) the state read + written, q/k/v/g in, o out (fp32), beta,
-# the conv cache (3 tokens x q/k/v read, 3 written)
-DEC_BYTES_PER_PAIR = 2 * STATE_BYTES + 4 * D * 2 + D * 4 + 2 + 2 * 9 * D * 2
+
+
+# decode: per (sequence, head) the state read + written (4 or 2 bytes per element), q/k/v/g
+# in, o out (fp32), beta, the conv cache (3 tokens x q/k/v read, 3 written)
+def dec_bytes_per_pair(state_elem_bytes: int) -> int:
+    return 2 * D * D * state_elem_bytes + 4 * D * 2 + D * 4 + 2 + 2 * 9 * D * 2
+
+
 # kernels launched per call: kda_prefill bf16 = chunk_prep + chunk_scan + conv tail
 PREFILL_LAUNCHES = 3
 DECODE_LAUNCHES = 1
@@ -54,8 +59,13 @@ DECODE_LAUNCHES = 1
 # (k_hat, u, alpha fp32) written and read back, q k v g read, beta, o fp32;
 # the conv cache read by both calls and written by commit
 MTP_ROWS = 6
-MTP_BYTES_PER_PAIR = (3 * STATE_BYTES + MTP_ROWS * (2 * 3 * D * 4 + 4 * D * 2 + 2 + D * 4)
-                      + 3 * 9 * D * 2)
+
+
+def mtp_bytes_per_pair(state_elem_bytes: int) -> int:
+    return (3 * D * D * state_elem_bytes + MTP_ROWS * (2 * 3 * D * 4 + 4 * D * 2 + 2 + D * 4)
+            + 3 * 9 * D * 2)
+
+
 MTP_LAUNCHES = 2
 
 
@@ -273,7 +283,12 @@ def main():
 
     if args.no_prefill:  # decode legs only (profiling)
         print(json.dumps({"decode": run_decode(args, world, dev, stream, kda, hbm_peak),
-                          "mtp": run_mtp(args, world, dev, stream, kda, hbm_peak)}), flush=True)
+                          "mtp": run_mtp(args, world, dev, stream, kda, hbm_peak),
+                          "mtp_fused": run_mtp_fused(args, world, dev, stream, kda, hbm_peak),
+                          "decode_bf16_state": run_decode(args, world, dev, stream, kda, hbm_peak, torch.bfloat16),
+                          "mtp_fused_bf16_state": run_mtp_fused(args, world, dev, stream, kda, hbm_peak,
+                                                                torch.bfloat16)}),
+              flush=True)
         return
 
     # ---------------- prefill: long-context workload, resident in HBM ----------
@@ -312,10 +327,13 @@ def main():
         e2e = run_e2e(args, world, stream, inp, d, o, S, step, tokens_per_rank)
 
     # ---------------- decode step: 256 sequences, state in place ----------------
-    dec_line = mtp_line = None
+    dec_line = mtp_line = fused_line = dec16_line = mtp16_line = None
     if not args.no_decode:
         dec_line = run_decode(args, world, dev, stream, kda, hbm_peak)
         mtp_line = run_mtp(args, world, dev, stream, kda, hbm_peak)
+        fused_line = run_mtp_fused(args, world, dev, stream, kda, hbm_peak)
+        dec16_line = run_decode(args, world, dev, stream, kda, hbm_peak, torch.bfloat16)
+        mtp16_line = run_mtp_fused(args, world, dev, stream, kda, hbm_peak, torch.bfloat16)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -333,6 +351,9 @@ def main():
         "clocks": clk.summary(),
         "decode": dec_line,
         "mtp": mtp_line,
+        "mtp_fused": fused_line,
+        "decode_bf16_state": dec16_line,
+        "mtp_fused_bf16_state": mtp16_line,
     }
     if (heads, T_run) != (H, T_LONG):
         line["config"]["note"] = "reduced profiling size, not the reported workload"
@@ -368,11 +389,15 @@ def run_e2e(args, world, stream, inp, d, o, S, step, tokens_per_rank):
             "steps": args.e2e_steps}
 
 
-def run_decode(args, world, dev, stream, kda, hbm_peak):
-    """kda_decode_step on the decode workload (256 sequences, state in place)."""
+def run_decode(args, world, dev, stream, kda, hbm_peak, state_dtype=torch.float32):
+    """kda_decode_step on the decode workload (256 sequences, state in place,
+    stored in `state_dtype`)."""
     dec = ki.workload(4) if args.decode_seqs == 256 else \
         ki.make_decode(args.decode_seqs, H, torch.bfloat16, ki.BASE_SEED + 4)
     dd = {n: getattr(dec, n).to(dev) for n in ("state", "conv_cache", "q", "k", "v", "g", "beta", "conv_w")}
+    dd["state"] = dd["state"].to(state_dtype)
+    sb = dd["state"].element_size()
+    sname = "fp32" if sb == 4 else "bf16"
     o_dec = torch.empty(dd["q"].shape, dtype=torch.float32, device=dev)
 
     def dstep():
@@ -382,24 +407,30 @@ def run_decode(args, world, dev, stream, kda, hbm_peak):
     _, dec_steps = timed(dstep, args.steps, args.warmup, world, stream)
     npairs = dec.num_seqs * H
     dec_ms = statistics.mean(dec_steps)
-    dec_state_gbs = npairs * 2 * STATE_BYTES / (dec_ms / 1e3) / 1e9
-    dec_alg_gbs = npairs * DEC_BYTES_PER_PAIR / (dec_ms / 1e3) / 1e9
-    return {"workload": "kda_decode_step: 256 sequences x 1 token, 64 heads x 128, fp32 state in place",
-            "state_gbs": dec_state_gbs, "ms_per_step": dec_ms,
+    dec_state_gbs = npairs * 2 * D * D * sb / (dec_ms / 1e3) / 1e9
+    alg = npairs * dec_bytes_per_pair(sb)
+    dec_alg_gbs = alg / (dec_ms / 1e3) / 1e9
+    return {"workload": f"kda_decode_step: {dec.num_seqs} sequences x 1 token, 64 heads x 128, "
+                        f"{sname} state in place",
+            "state_gbs": dec_state_gbs, "ms_per_step": dec_ms, "tokens_per_s": dec.num_seqs / (dec_ms / 1e3),
             "roofline": {"kernel": "kda_decode", "bound": "hbm", "achieved": dec_alg_gbs, "peak": hbm_peak,
                          "unit": "GB/s", "frac": dec_alg_gbs / hbm_peak, "state_frac": dec_state_gbs / hbm_peak,
-                         "traffic": recorded_traffic("kda_decode"),
-                         "algorithmic_bytes_per_launch": npairs * DEC_BYTES_PER_PAIR},
+                         "traffic": recorded_traffic("kda_decode") if sb == 4 else None,
+                         "algorithmic_bytes_per_launch": alg},
             "gpu_launches": args.steps * DECODE_LAUNCHES}
 
 
-def run_mtp(args, world, dev, stream, kda, hbm_peak):
+def run_mtp(args, world, dev, stream, kda, hbm_peak, state_dtype=torch.float32):
     """Multi-token decode for speculative serving: kda_decode_verify of 6 rows
     (5 drafts + 1) per sequence, then kda_decode_commit of the kept prefix
-    (2..6 rows, about four on average), 256 sequences x 64 heads."""
+    (2..6 rows, about four on average), 256 sequences x 64 heads, state stored
+    in `state_dtype`."""
     N = args.decode_seqs
     mt = ki.make_decode_rows(N, MTP_ROWS, H, torch.bfloat16, ki.BASE_SEED + 5, accept=(2, MTP_ROWS))
     dd = {n: getattr(mt, n).to(dev) for n in ("state", "conv_cache", "q", "k", "v", "g", "beta", "conv_w")}
+    dd["state"] = dd["state"].to(state_dtype)
+    sb = dd["state"].element_size()
+    sname = "fp32" if sb == 4 else "bf16"
     o_m = torch.empty(dd["q"].shape, dtype=torch.float32, device=dev)
     deltas = torch.empty(kda.deltas_size(N, MTP_ROWS, H) // 4, dtype=torch.float32, device=dev)
     n_acc = torch.from_numpy(mt.n_accept).to(dev)
@@ -420,17 +451,63 @@ def run_mtp(args, world, dev, stream, kda, hbm_peak):
     _, vsteps = timed(vstep, args.steps, args.warmup, world, stream)
     verify_ms = statistics.mean(vsteps)
     npairs = N * H
-    alg = npairs * MTP_BYTES_PER_PAIR
+    alg = npairs * mtp_bytes_per_pair(sb)
     gbs = alg / (ms / 1e3) / 1e9
     return {"workload": f"kda_decode_verify + kda_decode_commit: {N} sequences x {MTP_ROWS} rows, 64 heads x 128, "
-                        f"{int(mt.n_accept.sum())} rows kept, fp32 state in place",
+                        f"{int(mt.n_accept.sum())} rows kept, {sname} state in place",
             "verified_rows_per_s": N * MTP_ROWS / (ms / 1e3), "kept_tokens_per_s": int(mt.n_accept.sum()) / (ms / 1e3),
             "ms_per_step": ms, "verify_ms": verify_ms, "commit_ms": ms - verify_ms,
-            "state_gbs": npairs * 3 * STATE_BYTES / (ms / 1e3) / 1e9,
+            "state_gbs": npairs * 3 * D * D * sb / (ms / 1e3) / 1e9,
             "roofline": {"kernel": "kda_decode_verify + kda_decode_commit", "bound": "hbm", "achieved": gbs,
                          "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak, "traffic": None,
                          "algorithmic_bytes_per_launch": alg},
             "gpu_launches": args.steps * (MTP_LAUNCHES + 1)}
+
+
+def run_mtp_fused(args, world, dev, stream, kda, hbm_peak, state_dtype=torch.float32):
+    """The same speculative serving loop with one kda_decode_commit_verify per
+    step: keep the previous step's accepted rows and verify 6 new rows in one
+    pass over the state (steady state: every step commits the step before)."""
+    N = args.decode_seqs
+    mt = ki.make_decode_rows(N, MTP_ROWS, H, torch.bfloat16, ki.BASE_SEED + 5, accept=(2, MTP_ROWS))
+    dd = {n: getattr(mt, n).to(dev) for n in ("state", "conv_cache", "q", "k", "v", "g", "beta", "conv_w")}
+    dd["state"] = dd["state"].to(state_dtype)
+    sb = dd["state"].element_size()
+    o_m = torch.empty(dd["q"].shape, dtype=torch.float32, device=dev)
+    bufs = [torch.empty(kda.deltas_size(N, MTP_ROWS, H) // 4, dtype=torch.float32, device=dev) for _ in range(2)]
+    n_acc = torch.from_numpy(mt.n_accept).to(dev)
+    kda.decode_verify(dd["state"], dd["conv_cache"], dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["conv_w"],
+                      o=o_m, deltas=bufs[0], stream=stream)
+    cur = [0]
+
+    def fstep():
+        prev, new = bufs[cur[0]], bufs[1 - cur[0]]
+        kda.decode_commit_verify(dd["state"], dd["conv_cache"], (dd["q"], dd["k"], dd["v"], prev, n_acc), dd["q"],
+                                 dd["k"], dd["v"], dd["g"], dd["beta"], dd["conv_w"], o=o_m, deltas=new,
+                                 stream=stream)
+        cur[0] = 1 - cur[0]
+
+    _, steps = timed(fstep, args.steps, args.warmup, world, stream)
+    assert kda.check_async_status(stream) == 0
+    ms = statistics.mean(steps)
+    npairs = N * H
+    kept = float(mt.n_accept.mean())
+    # per (sequence, head): state read + written; per new row deltas written,
+    # q k v g read, beta, o fp32; per kept previous row its deltas read; the
+    # conv cache read and written and the kept raw rows read for it
+    per_pair = (2 * D * D * sb + MTP_ROWS * (3 * D * 4 + 4 * D * 2 + 2 + D * 4) + kept * 3 * D * 4
+                + 2 * 9 * D * 2 + 9 * D * 2)
+    alg = npairs * per_pair
+    gbs = alg / (ms / 1e3) / 1e9
+    return {"workload": f"kda_decode_commit_verify: {N} sequences x {MTP_ROWS} rows, 64 heads x 128, "
+                        f"{int(mt.n_accept.sum())} rows of the previous step kept, "
+                        f"{'fp32' if sb == 4 else 'bf16'} state in place",
+            "verified_rows_per_s": N * MTP_ROWS / (ms / 1e3), "kept_tokens_per_s": int(mt.n_accept.sum()) / (ms / 1e3),
+            "ms_per_step": ms, "state_gbs": npairs * 2 * D * D * sb / (ms / 1e3) / 1e9,
+            "roofline": {"kernel": "kda_decode_commit_verify", "bound": "hbm", "achieved": gbs, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": gbs / hbm_peak, "traffic": None,
+                         "algorithmic_bytes_per_launch": alg},
+            "gpu_launches": args.steps}
 
 
 if __name__ == "__main__":

@@ -28,8 +28,23 @@
  *    element type per `dt` (fp32 or bf16).  conv_w is always fp32:
  *      conv_w : [3, H*128, 4]  (q, k, v taps; tap 3 multiplies the current
  *               token, tap 0 the token three steps back; no bias)
- *  - States are fp32 [N, H, 128, 128], row = key channel, column = value
- *    channel (value index contiguous).  Conv history / tail / cache is
+ *  - States are [N, H, 128, 128], row = key channel, column = value channel
+ *    (value index contiguous), stored with element type `state_dt`:
+ *      KDA_F32  -- the state as computed (fp32);
+ *      KDA_BF16 -- half the bytes.  All state arithmetic is still fp32; the
+ *                  state is rounded to bf16 (nearest, ties to even) wherever
+ *                  it is stored: by every decode step, after every committed
+ *                  verify row, and once at the end of a prefill call (inside
+ *                  a prefill call it stays fp32).  Each stored step moves an
+ *                  element by at most half a bf16 ulp (2^-9 relative); the
+ *                  rounding errors of successive decode steps add up until
+ *                  the gate decays them, so a bf16 state drifts from the fp32
+ *                  one by about 1e-2 of its rms within ten steps.
+ *    The pages give the model's state as fp32 (page "GLM-5.3-Flash im
+ *    Detail", section "Sequenz-Mixing: ...": 128 x 128 fp32 per head); page
+ *    "Reading GLM 5.3 Flash from config.json: 6.0 KB of KV Cache per Token"
+ *    counts a per-request KDA state of about half the fp32 size, i.e. two
+ *    bytes per element.  Conv history / tail / cache is
  *    [N, 3 (q,k,v), 3 (time, oldest first), H*128] in the input dtype.
  *  - L2 norm: x / sqrt(sum x^2 + 1e-6).  No query scale.  Conv activation:
  *    KDA_CONV_NONE (default) or KDA_CONV_SILU (y * sigmoid(y)).
@@ -81,15 +96,17 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_he
  *                      [cu_seqlens[n], cu_seqlens[n+1]).  May be NULL only when
  *                      total_T == 0.
  *   conv_w           : [3, H*128, 4] fp32 conv taps.
- *   init_state       : [N, H, 128, 128] fp32, or NULL for zero states.
+ *   init_state       : [N, H, 128, 128] (state_dt), or NULL for zero states.
  *   init_conv        : [N, 3, 3, H*128] raw q/k/v of the 3 tokens before each
  *                      segment (oldest first), or NULL for zeros.
  *   cu_seqlens_dev   : [N+1] int32 device copy of the segment offsets.
  *   cu_seqlens_host  : [N+1] int32 host copy (used for scheduling; must equal
  *                      the device copy).  cu[0] == 0, non-decreasing.
  *   o_dt             : element type of o (KDA_F32 or KDA_BF16).
+ *   state_dt         : element type of init_state and final_state.
  *   o                : out [total_T, H, 128] (o_dt).  Must not alias inputs.
- *   final_state      : out [N, H, 128, 128] fp32; may equal init_state (in place).
+ *   final_state      : out [N, H, 128, 128] (state_dt); may equal init_state
+ *                      (in place).
  *   conv_tail        : out [N, 3, 3, H*128] (dt): last 3 raw tokens of
  *                      concat(init_conv, segment); may equal init_conv.
  *   workspace        : device scratch of kda_prefill_workspace_size() bytes
@@ -98,11 +115,11 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_he
  * tensor-core path; fp32 inputs run the fp32 recurrent path.
  */
 kda_status kda_prefill(const void* q, const void* k, const void* v, const void* g,
-                       const void* beta, const float* conv_w, const float* init_state,
+                       const void* beta, const float* conv_w, const void* init_state,
                        const void* init_conv, const int32_t* cu_seqlens_dev,
                        const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
-                       kda_dtype dt, kda_conv_act act, kda_dtype o_dt, void* o,
-                       float* final_state, void* conv_tail, void* workspace,
+                       kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                       void* o, void* final_state, void* conv_tail, void* workspace,
                        size_t workspace_bytes, void* stream);
 
 /*
@@ -113,28 +130,34 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
  */
 kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, const void* g,
                                  const void* beta, const float* conv_w,
-                                 const float* init_state, const void* init_conv,
+                                 const void* init_state, const void* init_conv,
                                  const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
                                  int num_seqs, int num_heads, kda_dtype dt, kda_conv_act act,
-                                 kda_dtype o_dt, void* o, float* final_state, void* conv_tail,
-                                 void* stream);
+                                 kda_dtype o_dt, kda_dtype state_dt, void* o, void* final_state,
+                                 void* conv_tail, void* stream);
 
 /*
  * kda_decode_step -- one recurrent update per sequence (page "GLM-5.3-Flash im
  * Detail", section "Sequenz-Mixing: ...": decode of a single token performs a
  * recurrent update), in place.
- *   state      : [N, H, 128, 128] fp32, read and overwritten with S_t.
+ *   state      : [N, H, 128, 128] (state_dt), read and overwritten with S_t.
  *   conv_cache : [N, 3, 3, H*128] (dt), read (3 previous raw tokens) and
  *                shifted in place so that it ends with this step's raw token.
  *   q, k, v, g : [N, H, 128] raw inputs of the new token (dt); beta : [N, H].
  *   conv_w     : [3, H*128, 4] fp32.
  *   o_dt, o    : out [N, H, 128] with element type o_dt.
+ *   state_dt   : element type of state (o reads the loaded state; the
+ *                updated state is rounded when stored).
  * Each (sequence, head) state is streamed through registers exactly once.
+ * Errors: KDA_ERR_INVALID_ARG for a bad size or enum, a NULL pointer, or o
+ * aliasing an input; KDA_ERR_ALIGNMENT for a pointer that is not 16-byte
+ * aligned (beta: element aligned); KDA_ERR_UNSUPPORTED for N > 65535.
  */
-kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const void* k,
+kda_status kda_decode_step(void* state, void* conv_cache, const void* q, const void* k,
                            const void* v, const void* g, const void* beta,
                            const float* conv_w, int num_seqs, int num_heads, kda_dtype dt,
-                           kda_conv_act act, kda_dtype o_dt, void* o, void* stream);
+                           kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt, void* o,
+                           void* stream);
 
 /*
  * Multi-token decode for speculative serving (page "GLM-5.3-Flash Internals -
@@ -167,7 +190,9 @@ size_t kda_decode_deltas_size(int num_seqs, int num_rows, int num_heads);
 /*
  * kda_decode_verify -- decode rows 0..R-1 of every sequence in turn from
  * `state` and `conv_cache`, neither of which is modified.
- *   state      : [N, H, 128, 128] fp32, read only.
+ *   state      : [N, H, 128, 128] (state_dt), read only.  With a bf16 state,
+ *                row t + 1 starts from the state after row t rounded to bf16,
+ *                as the single step of row t would have stored it.
  *   conv_cache : [N, 3, 3, H*128] (dt), read only.
  *   conv_w     : [3, H*128, 4] fp32.
  *   o_dt, o    : out [N, R, H, 128], row t = o of that row.
@@ -177,10 +202,10 @@ size_t kda_decode_deltas_size(int num_seqs, int num_rows, int num_heads);
  * is not 16-byte aligned (beta: element aligned); KDA_ERR_UNSUPPORTED for
  * N > 65535.  Nothing is launched on error.
  */
-kda_status kda_decode_verify(const float* state, const void* conv_cache, const void* q, const void* k,
+kda_status kda_decode_verify(const void* state, const void* conv_cache, const void* q, const void* k,
                              const void* v, const void* g, const void* beta, const float* conv_w,
                              int num_seqs, int num_rows, int num_heads, kda_dtype dt, kda_conv_act act,
-                             kda_dtype o_dt, void* o, float* deltas, void* stream);
+                             kda_dtype o_dt, kda_dtype state_dt, void* o, float* deltas, void* stream);
 
 /*
  * kda_decode_commit -- apply the first n_accept[n] verified rows of sequence
@@ -195,9 +220,42 @@ kda_status kda_decode_verify(const float* state, const void* conv_cache, const v
  *              (kda_check_async_status).
  * Errors as for kda_decode_verify.
  */
-kda_status kda_decode_commit(float* state, void* conv_cache, const void* q, const void* k, const void* v,
+kda_status kda_decode_commit(void* state, void* conv_cache, const void* q, const void* k, const void* v,
                              const float* deltas, const int32_t* n_accept, int num_seqs, int num_rows,
-                             int num_heads, kda_dtype dt, void* stream);
+                             int num_heads, kda_dtype dt, kda_dtype state_dt, void* stream);
+
+/*
+ * kda_decode_commit_verify -- kda_decode_commit of the previous speculative
+ * step followed by kda_decode_verify of the next one, in one pass over each
+ * state: the state is read once and written once (not at all when no row of
+ * the previous step is kept), where the two separate calls read it twice.
+ *   1. The first prev_n_accept[n] rows of the previous step are kept, with
+ *      exactly the arithmetic of kda_decode_commit: state and conv_cache are
+ *      updated in place and stored.
+ *   2. The num_rows new rows are verified from the updated state and cache
+ *      exactly as kda_decode_verify would verify them: o and deltas.
+ * So the results equal kda_decode_commit(prev ...) then kda_decode_verify(...),
+ * bit for bit.
+ *   prev_q, prev_k, prev_v : the previous step's raw rows [N, prev_rows, H, 128]
+ *                            (dt), as given to its verify.
+ *   prev_deltas            : the deltas its verify wrote.
+ *   prev_n_accept          : [N] int32 on the device, each in [0, prev_rows];
+ *                            out-of-range values are clamped and recorded as
+ *                            for kda_decode_commit.
+ *   prev_rows              : rows of the previous step, 1..KDA_MAX_VERIFY_ROWS.
+ *   deltas                 : out, the new rows' deltas; must not overlap
+ *                            prev_deltas (callers alternate two buffers).
+ * Other arguments as for kda_decode_verify.  A first step (no previous step)
+ * is a plain kda_decode_verify.
+ * Errors: as for kda_decode_verify, and KDA_ERR_INVALID_ARG for prev_rows out
+ * of range, a NULL previous-step pointer or overlapping deltas.
+ */
+kda_status kda_decode_commit_verify(void* state, void* conv_cache, const void* prev_q, const void* prev_k,
+                                    const void* prev_v, const float* prev_deltas, const int32_t* prev_n_accept,
+                                    int prev_rows, const void* q, const void* k, const void* v, const void* g,
+                                    const void* beta, const float* conv_w, int num_seqs, int num_rows,
+                                    int num_heads, kda_dtype dt, kda_conv_act act, kda_dtype o_dt,
+                                    kda_dtype state_dt, void* o, float* deltas, void* stream);
 
 /*
  * kda_prefill_noalloc -- kda_prefill for callers that cannot allocate device
@@ -226,11 +284,11 @@ kda_status kda_decode_commit(float* state, void* conv_cache, const void* q, cons
  */
 #define KDA_NOALLOC_SCRATCH_BYTES ((size_t)128 << 20)
 kda_status kda_prefill_noalloc(const void* q, const void* k, const void* v, const void* g,
-                               const void* beta, const float* conv_w, const float* init_state,
+                               const void* beta, const float* conv_w, const void* init_state,
                                const void* init_conv, const int32_t* cu_seqlens_dev,
                                const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
-                               kda_dtype dt, kda_conv_act act, kda_dtype o_dt, void* o,
-                               float* final_state, void* conv_tail, void* stream);
+                               kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                               void* o, void* final_state, void* conv_tail, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* kda_status_string(kda_status s);

@@ -27,7 +27,8 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 # every entry point declared in include/kda.h
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
            "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version",
-           "kda_prefill_noalloc", "kda_decode_deltas_size", "kda_decode_verify", "kda_decode_commit")
+           "kda_prefill_noalloc", "kda_decode_deltas_size", "kda_decode_verify", "kda_decode_commit",
+           "kda_decode_commit_verify")
 MAX_VERIFY_ROWS = 8  # KDA_MAX_VERIFY_ROWS
 
 if not os.path.exists(LIB_PATH):
@@ -39,8 +40,8 @@ lib = ctypes.CDLL(LIB_PATH)
 lib.kda_prefill_workspace_size.restype = ctypes.c_size_t
 lib.kda_prefill_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int]
-_PREFILL_ARGS = [_vp, _vp, _vp, _vp, _vp, _f32p, _f32p, _vp, _i32p, _i32p, ctypes.c_int, ctypes.c_int,
-                 ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _f32p, _vp]
+_PREFILL_ARGS = [_vp, _vp, _vp, _vp, _vp, _f32p, _vp, _vp, _i32p, _i32p, ctypes.c_int, ctypes.c_int,
+                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]
 lib.kda_prefill.restype = ctypes.c_int
 lib.kda_prefill.argtypes = _PREFILL_ARGS + [_vp, ctypes.c_size_t, _vp]
 lib.kda_prefill_recurrent.restype = ctypes.c_int
@@ -49,16 +50,21 @@ lib.kda_prefill_noalloc.restype = ctypes.c_int
 lib.kda_prefill_noalloc.argtypes = _PREFILL_ARGS + [_vp]
 NOALLOC_SCRATCH_BYTES = 128 << 20  # KDA_NOALLOC_SCRATCH_BYTES
 lib.kda_decode_step.restype = ctypes.c_int
-lib.kda_decode_step.argtypes = [_f32p, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
-                                ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp]
+lib.kda_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
+                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp]
 lib.kda_decode_deltas_size.restype = ctypes.c_size_t
 lib.kda_decode_deltas_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
 lib.kda_decode_verify.restype = ctypes.c_int
-lib.kda_decode_verify.argtypes = [_f32p, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
-                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _f32p, _vp]
+lib.kda_decode_verify.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _f32p, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _f32p,
+                                  _vp]
 lib.kda_decode_commit.restype = ctypes.c_int
-lib.kda_decode_commit.argtypes = [_f32p, _vp, _vp, _vp, _vp, _f32p, _i32p, ctypes.c_int, ctypes.c_int,
-                                  ctypes.c_int, ctypes.c_int, _vp]
+lib.kda_decode_commit.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32p, _i32p, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp]
+lib.kda_decode_commit_verify.restype = ctypes.c_int
+lib.kda_decode_commit_verify.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32p, _i32p, ctypes.c_int, _vp, _vp, _vp, _vp,
+                                         _vp, _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _f32p, _vp]
 lib.kda_status_string.restype = ctypes.c_char_p
 lib.kda_status_string.argtypes = [ctypes.c_int]
 lib.kda_check_async_status.restype = ctypes.c_int
@@ -105,12 +111,22 @@ def workspace_size(num_seqs: int, total_tokens: int, num_heads: int, max_seqlen:
                                               KDA_F32 if dtype == torch.float32 else KDA_BF16))
 
 
+def _state_code(final_state, init_state) -> int:
+    """state_dt of a call: the element type of its state tensors (which agree)."""
+    if init_state is not None and init_state.dtype != final_state.dtype:
+        raise ValueError("init_state and final_state must have the same element type")
+    return _dtype_code(final_state)
+
+
 def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init_state=None,
             init_conv=None, act: int = KDA_CONV_NONE, o=None, final_state=None, conv_tail=None,
-            workspace=None, stream=None, recurrent: bool = False, o_dtype=torch.float32):
+            workspace=None, stream=None, recurrent: bool = False, o_dtype=torch.float32,
+            state_dtype=None):
     """kda_prefill (or kda_prefill_recurrent) on device tensors.  Returns
     (o, final_state, conv_tail); outputs are allocated when not given (o in
-    `o_dtype`, fp32 by default)."""
+    `o_dtype`, fp32 by default; the final state in `state_dtype`, default the
+    init state's type, else fp32).  The state element type of the call is that
+    of final_state."""
     cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
     N = len(cu_h) - 1
     T, H = q.shape[0], q.shape[1]
@@ -120,13 +136,14 @@ def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init
     if o is None:
         o = torch.empty(q.shape, dtype=o_dtype, device=dev)
     if final_state is None:
-        final_state = torch.empty((N, H, HEAD_DIM, HEAD_DIM), dtype=torch.float32, device=dev)
+        sdt = state_dtype or (init_state.dtype if init_state is not None else torch.float32)
+        final_state = torch.empty((N, H, HEAD_DIM, HEAD_DIM), dtype=sdt, device=dev)
     if conv_tail is None:
         conv_tail = torch.empty((N, 3, 3, H * HEAD_DIM), dtype=q.dtype, device=dev)
     dt = _dtype_code(q)
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(conv_w), _ptr(init_state),
             _ptr(init_conv), _ptr(cu_seqlens_dev), _ptr(cu_h), N, H, dt, int(act), _dtype_code(o),
-            _ptr(o), _ptr(final_state), _ptr(conv_tail)]
+            _state_code(final_state, init_state), _ptr(o), _ptr(final_state), _ptr(conv_tail)]
     if recurrent:
         _check(lib.kda_prefill_recurrent(*args, _stream(stream)), "kda_prefill_recurrent")
     else:
@@ -140,7 +157,7 @@ def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init
 
 def prefill_noalloc(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init_state=None,
                     init_conv=None, act: int = KDA_CONV_NONE, o=None, final_state=None, conv_tail=None,
-                    stream=None, o_dtype=torch.float32):
+                    stream=None, o_dtype=torch.float32, state_dtype=None):
     """kda_prefill_noalloc: like prefill() but the library uses its own static
     device scratch instead of a workspace.  Returns (o, final_state, conv_tail)."""
     cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
@@ -152,26 +169,28 @@ def prefill_noalloc(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=No
     if o is None:
         o = torch.empty(q.shape, dtype=o_dtype, device=dev)
     if final_state is None:
-        final_state = torch.empty((N, H, HEAD_DIM, HEAD_DIM), dtype=torch.float32, device=dev)
+        sdt = state_dtype or (init_state.dtype if init_state is not None else torch.float32)
+        final_state = torch.empty((N, H, HEAD_DIM, HEAD_DIM), dtype=sdt, device=dev)
     if conv_tail is None:
         conv_tail = torch.empty((N, 3, 3, H * HEAD_DIM), dtype=q.dtype, device=dev)
     _check(lib.kda_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(conv_w),
                                    _ptr(init_state), _ptr(init_conv), _ptr(cu_seqlens_dev), _ptr(cu_h), N, H,
-                                   _dtype_code(q), int(act), _dtype_code(o), _ptr(o), _ptr(final_state),
-                                   _ptr(conv_tail), _stream(stream)), "kda_prefill_noalloc")
+                                   _dtype_code(q), int(act), _dtype_code(o), _state_code(final_state, init_state),
+                                   _ptr(o), _ptr(final_state), _ptr(conv_tail), _stream(stream)),
+           "kda_prefill_noalloc")
     return o, final_state, conv_tail
 
 
 def decode_step(state, conv_cache, q, k, v, g, beta, conv_w, act: int = KDA_CONV_NONE, o=None,
                 stream=None, o_dtype=torch.float32):
-    """kda_decode_step in place on `state` and `conv_cache`; returns o
-    (allocated in `o_dtype` when not given)."""
+    """kda_decode_step in place on `state` (fp32 or bf16 storage) and
+    `conv_cache`; returns o (allocated in `o_dtype` when not given)."""
     N, H = q.shape[0], q.shape[1]
     if o is None:
         o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
     _check(lib.kda_decode_step(_ptr(state), _ptr(conv_cache), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                _ptr(beta), _ptr(conv_w), N, H, _dtype_code(q), int(act), _dtype_code(o),
-                               _ptr(o), _stream(stream)), "kda_decode_step")
+                               _dtype_code(state), _ptr(o), _stream(stream)), "kda_decode_step")
     return o
 
 
@@ -189,8 +208,8 @@ def decode_verify(state, conv_cache, q, k, v, g, beta, conv_w, act: int = KDA_CO
     if deltas is None:
         deltas = torch.empty(deltas_size(N, R, H) // 4, dtype=torch.float32, device=q.device)
     _check(lib.kda_decode_verify(_ptr(state), _ptr(conv_cache), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                 _ptr(conv_w), N, R, H, _dtype_code(q), int(act), _dtype_code(o), _ptr(o),
-                                 _ptr(deltas), _stream(stream)), "kda_decode_verify")
+                                 _ptr(conv_w), N, R, H, _dtype_code(q), int(act), _dtype_code(o),
+                                 _dtype_code(state), _ptr(o), _ptr(deltas), _stream(stream)), "kda_decode_verify")
     return o, deltas
 
 
@@ -200,7 +219,29 @@ def decode_commit(state, conv_cache, q, k, v, deltas, n_accept, stream=None):
     updated in place."""
     N, R, H = q.shape[0], q.shape[1], q.shape[2]
     _check(lib.kda_decode_commit(_ptr(state), _ptr(conv_cache), _ptr(q), _ptr(k), _ptr(v), _ptr(deltas),
-                                 _ptr(n_accept), N, R, H, _dtype_code(q), _stream(stream)), "kda_decode_commit")
+                                 _ptr(n_accept), N, R, H, _dtype_code(q), _dtype_code(state), _stream(stream)),
+           "kda_decode_commit")
+
+
+def decode_commit_verify(state, conv_cache, prev, q, k, v, g, beta, conv_w, act: int = KDA_CONV_NONE, o=None,
+                         deltas=None, stream=None, o_dtype=torch.float32):
+    """kda_decode_commit_verify: keep the first prev.n_accept[n] rows of the
+    previous step (`prev` = (prev_q, prev_k, prev_v, prev_deltas, n_accept) as
+    given to and returned by the previous verify), then verify the new rows
+    [N, R, H, 128] from the updated state and cache.  Returns (o, deltas);
+    `deltas` must not be the previous step's buffer."""
+    pq, pk, pv, pdeltas, pn = prev
+    N, R, H = q.shape[0], q.shape[1], q.shape[2]
+    if o is None:
+        o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
+    if deltas is None:
+        deltas = torch.empty(deltas_size(N, R, H) // 4, dtype=torch.float32, device=q.device)
+    _check(lib.kda_decode_commit_verify(_ptr(state), _ptr(conv_cache), _ptr(pq), _ptr(pk), _ptr(pv), _ptr(pdeltas),
+                                        _ptr(pn), pq.shape[1], _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                        _ptr(conv_w), N, R, H, _dtype_code(q), int(act), _dtype_code(o),
+                                        _dtype_code(state), _ptr(o), _ptr(deltas), _stream(stream)),
+           "kda_decode_commit_verify")
+    return o, deltas
 
 
 def check_async_status(stream=None) -> int:

@@ -3,6 +3,7 @@
 #include <stdio.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
@@ -18,19 +19,33 @@ namespace {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 size_t esize(kda_dtype dt) { return dt == KDA_F32 ? 4 : 2; }
+bool valid_dtype(kda_dtype t) { return t == KDA_F32 || t == KDA_BF16; }
+bool valid_act(kda_conv_act a) { return a == KDA_CONV_NONE || a == KDA_CONV_SILU; }
+
+// Runtime element type / activation -> template argument: f is called with a
+// value of the matching type (float or __nv_bfloat16; an integral_constant
+// holding the activation).
+template <typename F> void by_type(kda_dtype t, F&& f) {
+  if (t == KDA_F32) f(float{});
+  else f(__nv_bfloat16{});
+}
+template <typename F> void by_act(kda_conv_act a, F&& f) {
+  if (a == KDA_CONV_SILU) f(std::integral_constant<int, KDA_CONV_SILU>{});
+  else f(std::integral_constant<int, KDA_CONV_NONE>{});
+}
 
 struct PrefillArgs {
   const void *q, *k, *v, *g, *beta;
   const float* conv_w;
-  const float* init_state;
+  const void* init_state;
   const void* init_conv;
   const int32_t *cu_dev, *cu_host;
   int N, H;
   kda_dtype dt;
   kda_conv_act act;
-  kda_dtype o_dt;
+  kda_dtype o_dt, state_dt;
   void* o;
-  float* final_state;
+  void* final_state;
   void* conv_tail;
   cudaStream_t stream;
   int64_t total_T;
@@ -39,9 +54,8 @@ struct PrefillArgs {
 
 kda_status validate_prefill(PrefillArgs& a) {
   if (a.N < 0 || a.H < 1) return KDA_ERR_INVALID_ARG;
-  if (a.dt != KDA_F32 && a.dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
-  if (a.act != KDA_CONV_NONE && a.act != KDA_CONV_SILU) return KDA_ERR_INVALID_ARG;
-  if (a.o_dt != KDA_F32 && a.o_dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (!valid_dtype(a.dt) || !valid_dtype(a.o_dt) || !valid_dtype(a.state_dt) || !valid_act(a.act))
+    return KDA_ERR_INVALID_ARG;
   if (a.N == 0) { a.total_T = 0; a.max_len = 0; return KDA_OK; }
   if (!a.cu_host || !a.cu_dev) return KDA_ERR_INVALID_ARG;
   if (a.cu_host[0] != 0) return KDA_ERR_INVALID_ARG;
@@ -78,23 +92,19 @@ kda_status launch_tail(const PrefillArgs& a) {
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-template <typename Tin, typename Tout, int ACT>
-void launch_recurrent_t(const PrefillArgs& a) {
-  recurrent_prefill_kernel<Tin, Tout, ACT><<<dim3(a.H, a.N), 128, 0, a.stream>>>(
-      (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.g, (const Tin*)a.beta,
-      a.conv_w, a.init_state, (const Tin*)a.init_conv, a.cu_dev, a.H, (Tout*)a.o, a.final_state);
-}
-
 template <typename Tin>
 kda_status launch_recurrent(const PrefillArgs& a) {
-  const bool silu = a.act == KDA_CONV_SILU;
-  if (a.o_dt == KDA_F32) {
-    if (silu) launch_recurrent_t<Tin, float, KDA_CONV_SILU>(a);
-    else launch_recurrent_t<Tin, float, KDA_CONV_NONE>(a);
-  } else {
-    if (silu) launch_recurrent_t<Tin, __nv_bfloat16, KDA_CONV_SILU>(a);
-    else launch_recurrent_t<Tin, __nv_bfloat16, KDA_CONV_NONE>(a);
-  }
+  by_type(a.o_dt, [&](auto tout) {
+    by_type(a.state_dt, [&](auto ts) {
+      by_act(a.act, [&](auto act) {
+        using Tout = decltype(tout);
+        using Ts = decltype(ts);
+        recurrent_prefill_kernel<Tin, Tout, decltype(act)::value, Ts><<<dim3(a.H, a.N), 128, 0, a.stream>>>(
+            (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.g, (const Tin*)a.beta, a.conv_w,
+            (const Ts*)a.init_state, (const Tin*)a.init_conv, a.cu_dev, a.H, (Tout*)a.o, (Ts*)a.final_state);
+      });
+    });
+  });
   if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
   return launch_tail<Tin>(a);
 }
@@ -104,58 +114,10 @@ kda_status run_recurrent(PrefillArgs& a) {
   return a.dt == KDA_F32 ? launch_recurrent<float>(a) : launch_recurrent<__nv_bfloat16>(a);
 }
 
-template <typename Tin, typename Tout, int ACT>
-void launch_decode_t(float* state, void* cache, const void* q, const void* k, const void* v,
-                     const void* g, const void* beta, const float* conv_w, int N, int H, void* o,
-                     cudaStream_t s) {
-  decode_kernel<Tin, Tout, ACT><<<dim3(H, N), 256, 0, s>>>(
-      state, (Tin*)cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)g,
-      (const Tin*)beta, conv_w, H, (Tout*)o);
-}
-
-template <typename Tin>
-void launch_decode(kda_conv_act act, kda_dtype o_dt, float* state, void* cache, const void* q,
-                   const void* k, const void* v, const void* g, const void* beta,
-                   const float* conv_w, int N, int H, void* o, cudaStream_t s) {
-  const bool silu = act == KDA_CONV_SILU;
-  if (o_dt == KDA_F32) {
-    if (silu) launch_decode_t<Tin, float, KDA_CONV_SILU>(state, cache, q, k, v, g, beta, conv_w, N, H, o, s);
-    else launch_decode_t<Tin, float, KDA_CONV_NONE>(state, cache, q, k, v, g, beta, conv_w, N, H, o, s);
-  } else {
-    if (silu) launch_decode_t<Tin, __nv_bfloat16, KDA_CONV_SILU>(state, cache, q, k, v, g, beta, conv_w, N, H, o, s);
-    else launch_decode_t<Tin, __nv_bfloat16, KDA_CONV_NONE>(state, cache, q, k, v, g, beta, conv_w, N, H, o, s);
-  }
-}
-
-template <typename Tin, typename Tout, int ACT>
-void launch_verify_t(const float* state, const void* cache, const void* q, const void* k, const void* v,
-                     const void* g, const void* beta, const float* conv_w, int N, int R, int H, void* o,
-                     float* deltas, cudaStream_t s) {
-  decode_verify_kernel<Tin, Tout, ACT><<<dim3(H, N), 256, 0, s>>>(
-      state, (const Tin*)cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)g, (const Tin*)beta,
-      conv_w, R, H, (Tout*)o, deltas);
-}
-
-template <typename Tin>
-void launch_verify(kda_conv_act act, kda_dtype o_dt, const float* state, const void* cache, const void* q,
-                   const void* k, const void* v, const void* g, const void* beta, const float* conv_w, int N,
-                   int R, int H, void* o, float* deltas, cudaStream_t s) {
-  const bool silu = act == KDA_CONV_SILU;
-  if (o_dt == KDA_F32) {
-    if (silu) launch_verify_t<Tin, float, KDA_CONV_SILU>(state, cache, q, k, v, g, beta, conv_w, N, R, H, o, deltas, s);
-    else launch_verify_t<Tin, float, KDA_CONV_NONE>(state, cache, q, k, v, g, beta, conv_w, N, R, H, o, deltas, s);
-  } else {
-    if (silu)
-      launch_verify_t<Tin, __nv_bfloat16, KDA_CONV_SILU>(state, cache, q, k, v, g, beta, conv_w, N, R, H, o, deltas, s);
-    else
-      launch_verify_t<Tin, __nv_bfloat16, KDA_CONV_NONE>(state, cache, q, k, v, g, beta, conv_w, N, R, H, o, deltas, s);
-  }
-}
-
 // shared argument checks of the decode entry points
-kda_status check_decode_common(int num_seqs, int num_heads, kda_dtype dt) {
+kda_status check_decode_common(int num_seqs, int num_heads, kda_dtype dt, kda_dtype state_dt) {
   if (num_seqs < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
-  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
+  if (!valid_dtype(dt) || !valid_dtype(state_dt)) return KDA_ERR_INVALID_ARG;
   if (num_seqs > 65535) return KDA_ERR_UNSUPPORTED;
   return KDA_OK;
 }
@@ -173,13 +135,13 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_he
 
 kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, const void* g,
                                  const void* beta, const float* conv_w,
-                                 const float* init_state, const void* init_conv,
+                                 const void* init_state, const void* init_conv,
                                  const int32_t* cu_seqlens_dev, const int32_t* cu_seqlens_host,
                                  int num_seqs, int num_heads, kda_dtype dt, kda_conv_act act,
-                                 kda_dtype o_dt, void* o, float* final_state, void* conv_tail,
-                                 void* stream) {
+                                 kda_dtype o_dt, kda_dtype state_dt, void* o, void* final_state,
+                                 void* conv_tail, void* stream) {
   PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
-                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, o, final_state, conv_tail,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, state_dt, o, final_state, conv_tail,
                 (cudaStream_t)stream, 0, 0};
   kda_status st = validate_prefill(a);
   if (st != KDA_OK) return st;
@@ -187,14 +149,14 @@ kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, co
 }
 
 kda_status kda_prefill(const void* q, const void* k, const void* v, const void* g,
-                       const void* beta, const float* conv_w, const float* init_state,
+                       const void* beta, const float* conv_w, const void* init_state,
                        const void* init_conv, const int32_t* cu_seqlens_dev,
                        const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
-                       kda_dtype dt, kda_conv_act act, kda_dtype o_dt, void* o,
-                       float* final_state, void* conv_tail, void* workspace,
+                       kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                       void* o, void* final_state, void* conv_tail, void* workspace,
                        size_t workspace_bytes, void* stream) {
   PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
-                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, o, final_state, conv_tail,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, state_dt, o, final_state, conv_tail,
                 (cudaStream_t)stream, 0, 0};
   kda_status st = validate_prefill(a);
   if (st != KDA_OK) return st;
@@ -204,22 +166,21 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
   if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
   if (workspace && !aligned(workspace, 16)) return KDA_ERR_ALIGNMENT;
   st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
-                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.o, a.final_state, workspace,
-                      workspace_bytes, a.max_len, a.stream);
+                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.state_dt, a.o, a.final_state, workspace,
+                      a.stream);
   if (st != KDA_OK) return st;
   return launch_tail<__nv_bfloat16>(a);
 }
 
-kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const void* k,
+kda_status kda_decode_step(void* state, void* conv_cache, const void* q, const void* k,
                            const void* v, const void* g, const void* beta,
                            const float* conv_w, int num_seqs, int num_heads, kda_dtype dt,
-                           kda_conv_act act, kda_dtype o_dt, void* o, void* stream) {
-  if (num_seqs < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
-  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
-  if (o_dt != KDA_F32 && o_dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
-  if (act != KDA_CONV_NONE && act != KDA_CONV_SILU) return KDA_ERR_INVALID_ARG;
+                           kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt, void* o,
+                           void* stream) {
+  kda_status st = check_decode_common(num_seqs, num_heads, dt, state_dt);
+  if (st != KDA_OK) return st;
+  if (!valid_dtype(o_dt) || !valid_act(act)) return KDA_ERR_INVALID_ARG;
   if (num_seqs == 0) return KDA_OK;
-  if (num_seqs > 65535) return KDA_ERR_UNSUPPORTED;
   if (!state || !conv_cache || !q || !k || !v || !g || !beta || !conv_w || !o)
     return KDA_ERR_INVALID_ARG;
   const void* al16[] = {state, conv_cache, q, k, v, g, conv_w, o};
@@ -228,12 +189,19 @@ kda_status kda_decode_step(float* state, void* conv_cache, const void* q, const 
   if (!aligned(beta, esize(dt))) return KDA_ERR_ALIGNMENT;
   if (o == q || o == k || o == v || o == g) return KDA_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  if (dt == KDA_F32)
-    launch_decode<float>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w, num_seqs,
-                         num_heads, o, s);
-  else
-    launch_decode<__nv_bfloat16>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w,
-                                 num_seqs, num_heads, o, s);
+  by_type(dt, [&](auto tin) {
+    by_type(o_dt, [&](auto tout) {
+      by_type(state_dt, [&](auto ts) {
+        by_act(act, [&](auto a) {
+          using Tin = decltype(tin);
+          using Ts = decltype(ts);
+          decode_kernel<Tin, decltype(tout), decltype(a)::value, Ts><<<dim3(num_heads, num_seqs), 256, 0, s>>>(
+              (Ts*)state, (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)g,
+              (const Tin*)beta, conv_w, num_heads, (decltype(tout)*)o);
+        });
+      });
+    });
+  });
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -242,15 +210,14 @@ size_t kda_decode_deltas_size(int num_seqs, int num_rows, int num_heads) {
   return (size_t)num_seqs * num_heads * num_rows * 3 * D * sizeof(float);
 }
 
-kda_status kda_decode_verify(const float* state, const void* conv_cache, const void* q, const void* k,
+kda_status kda_decode_verify(const void* state, const void* conv_cache, const void* q, const void* k,
                              const void* v, const void* g, const void* beta, const float* conv_w,
                              int num_seqs, int num_rows, int num_heads, kda_dtype dt, kda_conv_act act,
-                             kda_dtype o_dt, void* o, float* deltas, void* stream) {
-  kda_status st = check_decode_common(num_seqs, num_heads, dt);
+                             kda_dtype o_dt, kda_dtype state_dt, void* o, float* deltas, void* stream) {
+  kda_status st = check_decode_common(num_seqs, num_heads, dt, state_dt);
   if (st != KDA_OK) return st;
   if (num_rows < 1 || num_rows > KDA_MAX_VERIFY_ROWS) return KDA_ERR_INVALID_ARG;
-  if (o_dt != KDA_F32 && o_dt != KDA_BF16) return KDA_ERR_INVALID_ARG;
-  if (act != KDA_CONV_NONE && act != KDA_CONV_SILU) return KDA_ERR_INVALID_ARG;
+  if (!valid_dtype(o_dt) || !valid_act(act)) return KDA_ERR_INVALID_ARG;
   if (num_seqs == 0) return KDA_OK;
   if (!state || !conv_cache || !q || !k || !v || !g || !beta || !conv_w || !o || !deltas)
     return KDA_ERR_INVALID_ARG;
@@ -258,21 +225,76 @@ kda_status kda_decode_verify(const float* state, const void* conv_cache, const v
   for (const void* p : al16)
     if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
   if (!aligned(beta, esize(dt))) return KDA_ERR_ALIGNMENT;
-  if (o == q || o == k || o == v || o == g || (const void*)deltas == (const void*)state) return KDA_ERR_INVALID_ARG;
+  if (o == q || o == k || o == v || o == g || (const void*)deltas == state) return KDA_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  if (dt == KDA_F32)
-    launch_verify<float>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w, num_seqs, num_rows, num_heads, o,
-                         deltas, s);
-  else
-    launch_verify<__nv_bfloat16>(act, o_dt, state, conv_cache, q, k, v, g, beta, conv_w, num_seqs, num_rows,
-                                 num_heads, o, deltas, s);
+  by_type(dt, [&](auto tin) {
+    by_type(o_dt, [&](auto tout) {
+      by_type(state_dt, [&](auto ts) {
+        by_act(act, [&](auto a) {
+          using Tin = decltype(tin);
+          using Ts = decltype(ts);
+          // no previous step: state and cache are only read
+          decode_verify_kernel<Tin, decltype(tout), decltype(a)::value, Ts, false>
+              <<<dim3(num_heads, num_seqs), 256, 0, s>>>((Ts*)state, (Tin*)conv_cache, (const Tin*)q, (const Tin*)k,
+                                                         (const Tin*)v, (const Tin*)g, (const Tin*)beta, conv_w,
+                                                         num_rows, num_heads, (decltype(tout)*)o, deltas, nullptr,
+                                                         nullptr, nullptr, nullptr, nullptr, 0);
+        });
+      });
+    });
+  });
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-kda_status kda_decode_commit(float* state, void* conv_cache, const void* q, const void* k, const void* v,
+kda_status kda_decode_commit_verify(void* state, void* conv_cache, const void* prev_q, const void* prev_k,
+                                    const void* prev_v, const float* prev_deltas, const int32_t* prev_n_accept,
+                                    int prev_rows, const void* q, const void* k, const void* v, const void* g,
+                                    const void* beta, const float* conv_w, int num_seqs, int num_rows,
+                                    int num_heads, kda_dtype dt, kda_conv_act act, kda_dtype o_dt,
+                                    kda_dtype state_dt, void* o, float* deltas, void* stream) {
+  kda_status st = check_decode_common(num_seqs, num_heads, dt, state_dt);
+  if (st != KDA_OK) return st;
+  if (num_rows < 1 || num_rows > KDA_MAX_VERIFY_ROWS) return KDA_ERR_INVALID_ARG;
+  if (prev_rows < 1 || prev_rows > KDA_MAX_VERIFY_ROWS) return KDA_ERR_INVALID_ARG;
+  if (!valid_dtype(o_dt) || !valid_act(act)) return KDA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KDA_OK;
+  if (!state || !conv_cache || !prev_q || !prev_k || !prev_v || !prev_deltas || !prev_n_accept || !q || !k ||
+      !v || !g || !beta || !conv_w || !o || !deltas)
+    return KDA_ERR_INVALID_ARG;
+  const void* al16[] = {state, conv_cache, prev_q, prev_k, prev_v, prev_deltas, q, k, v, g, conv_w, o, deltas};
+  for (const void* p : al16)
+    if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+  if (!aligned(beta, esize(dt)) || !aligned(prev_n_accept, 4)) return KDA_ERR_ALIGNMENT;
+  if (o == q || o == k || o == v || o == g || (const void*)deltas == state) return KDA_ERR_INVALID_ARG;
+  {  // the new deltas may not overlap the previous step's (other blocks still read those)
+    const uintptr_t d0 = (uintptr_t)deltas, d1 = d0 + kda_decode_deltas_size(num_seqs, num_rows, num_heads);
+    const uintptr_t p0 = (uintptr_t)prev_deltas, p1 = p0 + kda_decode_deltas_size(num_seqs, prev_rows, num_heads);
+    if (d0 < p1 && p0 < d1) return KDA_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  by_type(dt, [&](auto tin) {
+    by_type(o_dt, [&](auto tout) {
+      by_type(state_dt, [&](auto ts) {
+        by_act(act, [&](auto a) {
+          using Tin = decltype(tin);
+          using Ts = decltype(ts);
+          decode_verify_kernel<Tin, decltype(tout), decltype(a)::value, Ts, true>
+              <<<dim3(num_heads, num_seqs), 256, 0, s>>>((Ts*)state, (Tin*)conv_cache, (const Tin*)q, (const Tin*)k,
+                                                         (const Tin*)v, (const Tin*)g, (const Tin*)beta, conv_w,
+                                                         num_rows, num_heads, (decltype(tout)*)o, deltas,
+                                                         (const Tin*)prev_q, (const Tin*)prev_k, (const Tin*)prev_v,
+                                                         prev_deltas, prev_n_accept, prev_rows);
+        });
+      });
+    });
+  });
+  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_decode_commit(void* state, void* conv_cache, const void* q, const void* k, const void* v,
                              const float* deltas, const int32_t* n_accept, int num_seqs, int num_rows,
-                             int num_heads, kda_dtype dt, void* stream) {
-  kda_status st = check_decode_common(num_seqs, num_heads, dt);
+                             int num_heads, kda_dtype dt, kda_dtype state_dt, void* stream) {
+  kda_status st = check_decode_common(num_seqs, num_heads, dt, state_dt);
   if (st != KDA_OK) return st;
   if (num_rows < 1 || num_rows > KDA_MAX_VERIFY_ROWS) return KDA_ERR_INVALID_ARG;
   if (num_seqs == 0) return KDA_OK;
@@ -282,14 +304,15 @@ kda_status kda_decode_commit(float* state, void* conv_cache, const void* q, cons
     if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
   if (!aligned(n_accept, 4)) return KDA_ERR_ALIGNMENT;
   cudaStream_t s = (cudaStream_t)stream;
-  const dim3 grid(num_heads, num_seqs);
-  if (dt == KDA_F32)
-    decode_commit_kernel<float><<<grid, 256, 0, s>>>(state, (float*)conv_cache, (const float*)q, (const float*)k,
-                                                      (const float*)v, deltas, n_accept, num_rows, num_heads);
-  else
-    decode_commit_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        state, (__nv_bfloat16*)conv_cache, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-        (const __nv_bfloat16*)v, deltas, n_accept, num_rows, num_heads);
+  by_type(dt, [&](auto tin) {
+    by_type(state_dt, [&](auto ts) {
+      using Tin = decltype(tin);
+      using Ts = decltype(ts);
+      decode_commit_kernel<Tin, Ts><<<dim3(num_heads, num_seqs), 256, 0, s>>>(
+          (Ts*)state, (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, deltas, n_accept, num_rows,
+          num_heads);
+    });
+  });
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -317,7 +340,7 @@ kda_status kda_check_async_status(void* stream) {
   return (kda_status)v;
 }
 
-int kda_version(void) { return (1 << 16) | 0; }
+int kda_version(void) { return (2 << 16) | 0; }
 
 }  // extern "C"
 
@@ -352,14 +375,14 @@ kda_status noalloc_scratch(void** out) {
 
 extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const void* v, const void* g,
                                           const void* beta, const float* conv_w,
-                                          const float* init_state, const void* init_conv,
+                                          const void* init_state, const void* init_conv,
                                           const int32_t* cu_seqlens_dev,
                                           const int32_t* cu_seqlens_host, int num_seqs,
                                           int num_heads, kda_dtype dt, kda_conv_act act,
-                                          kda_dtype o_dt, void* o, float* final_state,
-                                          void* conv_tail, void* stream) {
+                                          kda_dtype o_dt, kda_dtype state_dt, void* o,
+                                          void* final_state, void* conv_tail, void* stream) {
   PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
-                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, o, final_state, conv_tail,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, state_dt, o, final_state, conv_tail,
                 (cudaStream_t)stream, 0, 0};
   kda_status st = validate_prefill(a);
   if (st != KDA_OK) return st;
@@ -371,8 +394,8 @@ extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const vo
   st = noalloc_scratch(&scratch);
   if (st != KDA_OK) return st;
   st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
-                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.o, a.final_state, scratch, need,
-                      a.max_len, a.stream);
+                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.state_dt, a.o, a.final_state, scratch,
+                      a.stream);
   if (st != KDA_OK) return st;
   return launch_tail<__nv_bfloat16>(a);
 }

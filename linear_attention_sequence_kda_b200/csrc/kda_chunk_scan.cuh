@@ -55,14 +55,14 @@ constexpr int TM_O1 = 0, TM_U = 64, TM_O0 = 128, TM_S = 192, TM_V = 320;
 constexpr int TM_VX = 384, TM_UP = 448;  // exact fp32 V and P_tt * U for the diagonal terms
 __device__ __forceinline__ int o_col(int chunk) { return (chunk & 1) ? TM_O1 : TM_O0; }
 
-template <typename Tout, int ACT>
+template <typename Tout, int ACT, typename Ts>
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                   const float* __restrict__ conv_w,
-                  const float* init_state, const __nv_bfloat16* __restrict__ init_conv,
+                  const Ts* init_state, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
-                  Tout* __restrict__ o, float* final_state) {
+                  Tout* __restrict__ o, Ts* final_state) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   // loads (record pieces, value tiles), MMA commits, compute-warp hand-offs
@@ -234,12 +234,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     const int64_t chan = (int64_t)h * D + v;
     // initial state: row v of S^T = column v of S (key rows k0 ..)
     {
-      const float* Si = init_state ? init_state + ((int64_t)n * H + h) * D * D + v : nullptr;
+      const Ts* Si = init_state ? init_state + ((int64_t)n * H + h) * D * D + v : nullptr;
 #pragma unroll
       for (int g16 = 0; g16 < 2; ++g16) {
         float s[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) s[j] = Si ? Si[(int64_t)(k0 + 16 * g16 + j) * D] : 0.f;
+        for (int j = 0; j < 16; ++j) s[j] = Si ? to_f(Si[(int64_t)(k0 + 16 * g16 + j) * D]) : 0.f;
         tc::st16(tl + TM_S + k0 + 16 * g16, s);
       }
     }
@@ -368,14 +368,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     if (!ok) s_abort = 1;
     // final state: column v of S = row v of S^T
     if (ok) {
-      float* Sf = final_state + ((int64_t)n * H + h) * D * D + v;
+      Ts* Sf = final_state + ((int64_t)n * H + h) * D * D + v;
 #pragma unroll
       for (int g16 = 0; g16 < 2; ++g16) {
         float s[16];
         tc::ld16(tl + TM_S + k0 + 16 * g16, s);
         tc::ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) Sf[(int64_t)(k0 + 16 * g16 + j) * D] = s[j];
+        for (int j = 0; j < 16; ++j) Sf[(int64_t)(k0 + 16 * g16 + j) * D] = from_f<Ts>(s[j]);
       }
     }
   }

@@ -29,10 +29,11 @@ inline size_t chunked_workspace_bytes(int N, int H, int64_t total_tokens) {
 
 template <int ACT>
 inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, const void* g,
-                                   const void* beta, const float* conv_w, const float* init_state,
+                                   const void* beta, const float* conv_w, const void* init_state,
                                    const void* init_conv, const int32_t* cu_dev,
-                                   const int32_t* cu_host, int N, int H, kda_dtype o_dt, void* o,
-                                   float* final_state, void* workspace, cudaStream_t stream) {
+                                   const int32_t* cu_host, int N, int H, kda_dtype o_dt,
+                                   kda_dtype state_dt, void* o, void* final_state, void* workspace,
+                                   cudaStream_t stream) {
   using T = __nv_bfloat16;
   // chunk table and longest-first segment order
   std::vector<int64_t> nch(N);
@@ -88,33 +89,38 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
                                                         cu_dev, d_tab, H, (int)items, records);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
   }
-  if (o_dt == KDA_F32) {
-    auto scan = chunk_scan_kernel<float, ACT>;
+  // the scan, instantiated for the output and state element types
+  auto launch_scan = [&](auto tout, auto ts) -> bool {
+    using Tout = decltype(tout);
+    using Ts = decltype(ts);
+    auto scan = chunk_scan_kernel<Tout, ACT, Ts>;
     if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
-      return KDA_ERR_CUDA;
-    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, stream>>>(tv, to, conv_w, init_state, (const T*)init_conv, cu_dev,
-                                                               d_base, d_order, H, records, (float*)o, final_state);
-  } else {
-    auto scan = chunk_scan_kernel<T, ACT>;
-    if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
-      return KDA_ERR_CUDA;
-    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, stream>>>(tv, to, conv_w, init_state, (const T*)init_conv, cu_dev,
-                                                               d_base, d_order, H, records, (T*)o, final_state);
-  }
+      return false;
+    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, stream>>>(tv, to, conv_w, (const Ts*)init_state,
+                                                               (const T*)init_conv, cu_dev, d_base, d_order, H,
+                                                               records, (Tout*)o, (Ts*)final_state);
+    return true;
+  };
+  bool ok;
+  if (o_dt == KDA_F32)
+    ok = state_dt == KDA_F32 ? launch_scan(float{}, float{}) : launch_scan(float{}, T{});
+  else
+    ok = state_dt == KDA_F32 ? launch_scan(T{}, float{}) : launch_scan(T{}, T{});
+  if (!ok) return KDA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 inline kda_status launch_chunked(const void* q, const void* k, const void* v, const void* g,
-                                 const void* beta, const float* conv_w, const float* init_state,
+                                 const void* beta, const float* conv_w, const void* init_state,
                                  const void* init_conv, const int32_t* cu_dev,
                                  const int32_t* cu_host, int N, int H, kda_conv_act act,
-                                 kda_dtype o_dt, void* o, float* final_state, void* workspace,
-                                 size_t /*workspace_bytes*/, int /*max_len*/, cudaStream_t stream) {
+                                 kda_dtype o_dt, kda_dtype state_dt, void* o, void* final_state,
+                                 void* workspace, cudaStream_t stream) {
   if (act == KDA_CONV_SILU)
     return launch_chunked_t<KDA_CONV_SILU>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
-                                           cu_host, N, H, o_dt, o, final_state, workspace, stream);
+                                           cu_host, N, H, o_dt, state_dt, o, final_state, workspace, stream);
   return launch_chunked_t<KDA_CONV_NONE>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
-                                         cu_host, N, H, o_dt, o, final_state, workspace, stream);
+                                         cu_host, N, H, o_dt, state_dt, o, final_state, workspace, stream);
 }
 
 }  // namespace kda

@@ -79,4 +79,31 @@ __device__ __forceinline__ float2 dup2(float x) { return make_float2(x, x); }
 __device__ __forceinline__ float4 ld_stream(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
 __device__ __forceinline__ void st_stream(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
 
+// State storage: fp32, or bf16 (rounded to nearest, ties to even, when
+// stored).  Arithmetic on the state is always fp32; a bf16 state element reads
+// back as the fp32 value it was rounded to.  Four consecutive elements per
+// call, streaming (the states are touched once per step).
+__device__ __forceinline__ float4 ld_state4(const float* p) { return ld_stream(p); }
+__device__ __forceinline__ float4 ld_state4(const __nv_bfloat16* p) {
+  const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));  // element 2j in the low half of word j
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xFFFF0000u));
+}
+__device__ __forceinline__ void st_state4(float* p, float4 v) { st_stream(p, v); }
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+__device__ __forceinline__ void st_state4(__nv_bfloat16* p, float4 v) {
+  __stcs(reinterpret_cast<uint2*>(p), make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w)));
+}
+// The value an element has after a store and a load in storage type Ts.
+template <typename Ts> __device__ __forceinline__ float4 as_stored4(float4 v);
+template <> __device__ __forceinline__ float4 as_stored4<float>(float4 v) { return v; }
+template <> __device__ __forceinline__ float4 as_stored4<__nv_bfloat16>(float4 v) {
+  const uint32_t a = pack_bf16x2(v.x, v.y), b = pack_bf16x2(v.z, v.w);  // one convert per pair
+  return make_float4(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u), __uint_as_float(b << 16),
+                     __uint_as_float(b & 0xFFFF0000u));
+}
+
 }  // namespace kda

@@ -64,9 +64,9 @@ __device__ __forceinline__ void rows_update(float4 (&s)[16], const float* a, con
   }
 }
 
-template <typename Tin, typename Tout, int ACT>
+template <typename Tin, typename Tout, int ACT, typename Ts>
 __global__ void __launch_bounds__(256, 2)
-decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
+decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
               const Tin* __restrict__ k, const Tin* __restrict__ v, const Tin* __restrict__ g,
               const Tin* __restrict__ beta, const float* __restrict__ conv_w, int H,
               Tout* __restrict__ o) {
@@ -77,12 +77,12 @@ decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __r
   const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t HD = (int64_t)H * D;
-  float* S = state + ((int64_t)n * H + h) * D * D;
+  Ts* S = state + ((int64_t)n * H + h) * D * D;
 
   // 1. issue the state loads first
   float4 s[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) s[i] = ld_stream(S + (warp * 16 + i) * D + lane * 4);
+  for (int i = 0; i < 16; ++i) s[i] = ld_state4(S + (warp * 16 + i) * D + lane * 4);
 
   // 2. prologue: threads 0..127 -> q and k of channel c; 128..255 -> v and g
   const int c = tid & (D - 1);
@@ -149,7 +149,7 @@ decode_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __r
   // 4. S <- Diag(a) S + k u^T, written once
   rows_update(s, &sh_al[warp * 16], &sh_kh[warp * 16], *reinterpret_cast<const float4*>(&sh_u[lane * 4]));
 #pragma unroll
-  for (int i = 0; i < 16; ++i) st_stream(S + (warp * 16 + i) * D + lane * 4, s[i]);
+  for (int i = 0; i < 16; ++i) st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
 }
 
 }  // namespace kda

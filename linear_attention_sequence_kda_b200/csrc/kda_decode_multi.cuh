@@ -26,33 +26,70 @@ namespace kda {
 
 constexpr int MAX_VERIFY_ROWS = KDA_MAX_VERIFY_ROWS;
 
-template <typename Tin, typename Tout, int ACT>
+// COMMIT = false: kda_decode_verify.  COMMIT = true: kda_decode_commit_verify,
+// which first keeps the first n_accept rows of the previous step (its raw rows
+// pq/pk/pv, PR of them per sequence, and its deltas) exactly as
+// decode_commit_kernel would, stores the state and the conv cache, and then
+// verifies the new rows from them: one pass over the state per step.
+template <typename Tin, typename Tout, int ACT, typename Ts, bool COMMIT>
 __global__ void __launch_bounds__(256, 2)
-decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ cache,
+decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
                      const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                      const Tin* __restrict__ g, const Tin* __restrict__ beta, const float* __restrict__ conv_w,
-                     int R, int H, Tout* __restrict__ o, float* __restrict__ deltas) {
+                     int R, int H, Tout* __restrict__ o, float* __restrict__ deltas,
+                     const Tin* __restrict__ pq, const Tin* __restrict__ pk, const Tin* __restrict__ pv,
+                     const float* __restrict__ pdeltas, const int32_t* __restrict__ pn_accept, int PR) {
   // per row: k_hat, alpha * k_hat, alpha * q_hat, alpha, conv(v); the row
   // prologues do not depend on the state, so all rows are prepared first
   __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][D], sh_ka[MAX_VERIFY_ROWS][D],
       sh_qa[MAX_VERIFY_ROWS][D], sh_al[MAX_VERIFY_ROWS][D], sh_v[MAX_VERIFY_ROWS][D];
   __shared__ __align__(16) float sh_r[8][D], sh_y[8][D], sh_u[D];
   __shared__ float sh_red[MAX_VERIFY_ROWS][4][3], sh_kq[MAX_VERIFY_ROWS], sh_beta[MAX_VERIFY_ROWS];
+  // the previous step's deltas, [row][k_hat, u, alpha][D] (commit only)
+  __shared__ __align__(16) float sh_prev[COMMIT ? 3 * MAX_VERIFY_ROWS : 1][D];
 
   const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t HD = (int64_t)H * D;
-  const float* S = state + ((int64_t)n * H + h) * D * D;
+  Ts* S = state + ((int64_t)n * H + h) * D * D;
   float4 s[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) s[i] = ld_stream(S + (warp * 16 + i) * D + lane * 4);
+  for (int i = 0; i < 16; ++i) s[i] = ld_state4(S + (warp * 16 + i) * D + lane * 4);
+  int na = 0;  // rows of the previous step kept
+  if (COMMIT) {
+    na = pn_accept[n];
+    if (na < 0 || na > PR) {  // out of range: record it and keep what can be kept
+      if (tid == 0 && h == 0) set_status(KDA_ERR_INVALID_ARG);
+      na = na < 0 ? 0 : PR;
+    }
+    const float* pdl = pdeltas + ((int64_t)n * H + h) * PR * 3 * D;
+    for (int e = tid; e < na * 3 * D; e += 256) sh_prev[e / D][e % D] = pdl[e];
+  }
 
   // 1. prologues of all rows: threads 0..127 q and k of channel c, threads
-  //    128..255 v and the gate (conv history = the cache, then earlier rows)
+  //    128..255 v and the gate (conv history = the cache, advanced by the
+  //    kept rows of the previous step, then earlier rows)
   const int c = tid & (D - 1);
   const int64_t ch = (int64_t)h * D + c;
   float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;  // [R][3 (k_hat, u, alpha)][D]
-  const Tin* cb = cache + (int64_t)n * 9 * HD + ch;  // [3 x][3 t] stride HD
+  Tin* cb = cache + (int64_t)n * 9 * HD + ch;  // [3 x][3 t] stride HD
+  // conv history of tensor x for channel c: the last three raw tokens of
+  // [cache, kept rows of the previous step], written back as the committed
+  // cache (this thread alone reads and writes these three entries)
+  auto history = [&](int x, const Tin* prev, float (&hh)[3]) {
+    Tin nv[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int idx = na + j;  // position in [cache rows 0..2, kept rows]
+      nv[j] = idx < 3 ? cb[(3 * x + idx) * HD] : prev[(((int64_t)n * PR + (idx - 3)) * H + h) * D + c];
+    }
+    if (COMMIT && na > 0) {
+#pragma unroll
+      for (int j = 0; j < 3; ++j) cb[(3 * x + j) * HD] = nv[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 3; ++j) hh[j] = to_f(nv[j]);
+  };
   float yq[MAX_VERIFY_ROWS], yk[MAX_VERIFY_ROWS];
   // raw inputs of all rows are loaded before any is used, so that their
   // global-memory latencies overlap instead of adding up row by row
@@ -66,7 +103,8 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
     }
     const float4 wq = load4(conv_w + (0 * HD + ch) * 4), wk = load4(conv_w + (1 * HD + ch) * 4);
     float hq[3], hk[3];
-    for (int j = 0; j < 3; ++j) { hq[j] = to_f(cb[j * HD]); hk[j] = to_f(cb[(3 + j) * HD]); }
+    history(0, pq, hq);
+    history(1, pk, hk);
 #pragma unroll
     for (int t = 0; t < MAX_VERIFY_ROWS; ++t) {
       if (t < R) {
@@ -92,7 +130,7 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
     if (c < R) sh_beta[c] = to_f(beta[((int64_t)n * R + c) * H + h]);
     const float4 wv = load4(conv_w + (2 * HD + ch) * 4);
     float hv[3];
-    for (int j = 0; j < 3; ++j) hv[j] = to_f(cb[(6 + j) * HD]);
+    history(2, pv, hv);
 #pragma unroll
     for (int t = 0; t < MAX_VERIFY_ROWS; ++t) {
       if (t < R) {
@@ -127,6 +165,25 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
   }
   __syncthreads();
 
+  // the kept rows of the previous step, as decode_commit_kernel applies them;
+  // the committed state is stored, and verification starts from its stored
+  // value (the commit's deltas reached shared memory before the barriers above)
+  if (COMMIT && na > 0) {
+    for (int t = 0; t < na; ++t) {
+      rows_update(s, &sh_prev[3 * t + 2][warp * 16], &sh_prev[3 * t][warp * 16],
+                  *reinterpret_cast<const float4*>(&sh_prev[3 * t + 1][lane * 4]));
+      if (t + 1 < na) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s[i] = as_stored4<Ts>(s[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
+      s[i] = as_stored4<Ts>(s[i]);
+    }
+  }
+
   // 2. the rows in turn against the state held in registers: threads 0..127
   //    finish r and u of channel c, threads 128..255 the readout y, which
   //    they complete with u once it is in shared memory
@@ -152,14 +209,18 @@ decode_verify_kernel(const float* __restrict__ state, const Tin* __restrict__ ca
     // sh_r / sh_y / sh_u of the next row are written only after every thread
     // has passed the next row's first barrier, i.e. after these reads
     if (tid >= D) o[(((int64_t)n * R + t) * H + h) * D + c] = from_f<Tout>(yy + sh_u[c] * sh_kq[t]);
-    if (t + 1 < R)
+    if (t + 1 < R) {
       rows_update(s, &sh_al[t][warp * 16], &sh_kh[t][warp * 16], *reinterpret_cast<const float4*>(&sh_u[lane * 4]));
+      // the next row starts from the state as a single step would have stored it
+#pragma unroll
+      for (int i = 0; i < 16; ++i) s[i] = as_stored4<Ts>(s[i]);
+    }
   }
 }
 
-template <typename Tin>
+template <typename Tin, typename Ts>
 __global__ void __launch_bounds__(256, 2)
-decode_commit_kernel(float* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
+decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
                      const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ deltas,
                      const int32_t* __restrict__ n_accept, int R, int H) {
   __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][D], sh_u[MAX_VERIFY_ROWS][D], sh_al[MAX_VERIFY_ROWS][D];
@@ -172,10 +233,10 @@ decode_commit_kernel(float* __restrict__ state, Tin* __restrict__ cache, const T
     na = na < 0 ? 0 : R;
   }
   if (na == 0) return;  // nothing accepted: state and cache stay as they are
-  float* S = state + ((int64_t)n * H + h) * D * D;
+  Ts* S = state + ((int64_t)n * H + h) * D * D;
   float4 s[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) s[i] = ld_stream(S + (warp * 16 + i) * D + lane * 4);
+  for (int i = 0; i < 16; ++i) s[i] = ld_state4(S + (warp * 16 + i) * D + lane * 4);
   const float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;
   for (int e = tid; e < na * D; e += 256) {
     const int t = e / D, cc = e % D;
@@ -198,10 +259,15 @@ decode_commit_kernel(float* __restrict__ state, Tin* __restrict__ cache, const T
     for (int j = 0; j < 3; ++j) cb[j * HD] = nv[j];
   }
   __syncthreads();
-  for (int t = 0; t < na; ++t)
+  for (int t = 0; t < na; ++t) {
     rows_update(s, &sh_al[t][warp * 16], &sh_kh[t][warp * 16], *reinterpret_cast<const float4*>(&sh_u[t][lane * 4]));
+    if (t + 1 < na) {  // every kept row stores its state (the last one below)
 #pragma unroll
-  for (int i = 0; i < 16; ++i) st_stream(S + (warp * 16 + i) * D + lane * 4, s[i]);
+      for (int i = 0; i < 16; ++i) s[i] = as_stored4<Ts>(s[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
 }
 
 }  // namespace kda

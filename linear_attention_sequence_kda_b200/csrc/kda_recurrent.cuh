@@ -17,14 +17,14 @@ namespace kda {
 
 constexpr int REC_TB = 16;  // tokens per prologue block
 
-template <typename Tin, typename Tout, int ACT>
+template <typename Tin, typename Tout, int ACT, typename Ts>
 __global__ void __launch_bounds__(128)
 recurrent_prefill_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                          const Tin* __restrict__ v, const Tin* __restrict__ g,
                          const Tin* __restrict__ beta, const float* __restrict__ conv_w,
-                         const float* init_state, const Tin* __restrict__ init_conv,
+                         const Ts* init_state, const Tin* __restrict__ init_conv,
                          const int32_t* __restrict__ cu, int H, Tout* __restrict__ o,
-                         float* final_state) {
+                         Ts* final_state) {
   __shared__ __align__(16) float sh_kh[REC_TB][D];    // k_hat
   __shared__ __align__(16) float sh_ka[REC_TB][D];    // alpha * k_hat
   __shared__ __align__(16) float sh_qa[REC_TB][D];    // alpha * q_hat
@@ -55,11 +55,11 @@ recurrent_prefill_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 
   // state column tid
   float S[D];
-  float* Sg = final_state + ((int64_t)n * H + h) * D * D + tid;
+  Ts* Sg = final_state + ((int64_t)n * H + h) * D * D + tid;
   if (init_state) {
-    const float* Si = init_state + ((int64_t)n * H + h) * D * D + tid;
+    const Ts* Si = init_state + ((int64_t)n * H + h) * D * D + tid;
 #pragma unroll
-    for (int i = 0; i < D; ++i) S[i] = Si[(int64_t)i * D];
+    for (int i = 0; i < D; ++i) S[i] = to_f(Si[(int64_t)i * D]);
   } else {
 #pragma unroll
     for (int i = 0; i < D; ++i) S[i] = 0.f;
@@ -137,7 +137,7 @@ recurrent_prefill_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     __syncthreads();  // before the next prologue overwrites shared memory
   }
 #pragma unroll
-  for (int i = 0; i < D; ++i) Sg[(int64_t)i * D] = S[i];
+  for (int i = 0; i < D; ++i) Sg[(int64_t)i * D] = from_f<Ts>(S[i]);
 }
 
 }  // namespace kda

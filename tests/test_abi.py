@@ -36,7 +36,7 @@ def test_header_declarations_are_exported():
 
 
 def test_version_and_status_strings():
-    assert kda.lib.kda_version() >> 16 == 1
+    assert kda.lib.kda_version() >> 16 == 2
     for code in range(7):
         s = kda.lib.kda_status_string(code)
         assert s and s.decode()
@@ -50,9 +50,9 @@ def test_workspace_size_invalid_is_zero():
 
 
 def _prefill(cu, H=4, dt=1, act=0, q=Q, o=O, final=FS, tail=CT, ws=WS, wsb=1 << 40, beta=B,
-             recurrent=False, odt=0):
+             recurrent=False, odt=0, sdt=0):
     cu = np.ascontiguousarray(np.asarray(cu, dtype=np.int32))
-    args = [q, K, V, G, beta, W, None, None, CU, cu.ctypes.data, len(cu) - 1, H, dt, act, odt, o, final,
+    args = [q, K, V, G, beta, W, None, None, CU, cu.ctypes.data, len(cu) - 1, H, dt, act, odt, sdt, o, final,
             tail]
     if recurrent:
         return kda.lib.kda_prefill_recurrent(*args, None)
@@ -66,6 +66,7 @@ def test_prefill_argument_validation(recurrent):
     assert p([0, 5], dt=7) == 1
     assert p([0, 5], act=5) == 1
     assert p([0, 5], odt=3) == 1
+    assert p([0, 5], sdt=2) == 1   # state element type
     assert p([1, 5]) == 1          # cu[0] != 0
     assert p([0, 5, 3]) == 1       # decreasing offsets
     assert p([0, 5], q=Q + 2) == 3  # misaligned
@@ -89,16 +90,17 @@ def test_prefill_workspace_check():
 
 def test_decode_argument_validation():
     d = kda.lib.kda_decode_step
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 0, 1, 0, 0, O, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 3, 0, 0, O, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 9, 0, O, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 5, O, None) == 1
-    assert d(FS + 4, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, O, None) == 3
-    assert d(FS, CT, Q, K, V, G, B + 1, W, 4, 2, 1, 0, 0, O, None) == 3
-    assert d(None, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, O, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, Q, None) == 1
-    assert d(FS, CT, Q, K, V, G, B, W, 70000, 2, 1, 0, 0, O, None) == 2
-    assert d(FS, CT, Q, K, V, G, B, W, 0, 2, 1, 0, 0, O, None) == 0
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 0, 1, 0, 0, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 3, 0, 0, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 9, 0, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 5, 0, O, None) == 1
+    assert d(FS + 4, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, 0, O, None) == 3
+    assert d(FS, CT, Q, K, V, G, B + 1, W, 4, 2, 1, 0, 0, 0, O, None) == 3
+    assert d(None, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, 0, O, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, 0, Q, None) == 1
+    assert d(FS, CT, Q, K, V, G, B, W, 70000, 2, 1, 0, 0, 0, O, None) == 2
+    assert d(FS, CT, Q, K, V, G, B, W, 0, 2, 1, 0, 0, 0, O, None) == 0
+    assert d(FS, CT, Q, K, V, G, B, W, 4, 2, 1, 0, 0, 2, O, None) == 1  # state element type
 
 
 DL, NA = 12 << 20, 13 << 20  # fake deltas and n_accept addresses
@@ -109,25 +111,48 @@ def test_decode_rows_argument_validation():
     assert kda.lib.kda_decode_deltas_size(4, 0, 2) == 0
     assert kda.lib.kda_decode_deltas_size(4, kda.MAX_VERIFY_ROWS + 1, 2) == 0
     vf = kda.lib.kda_decode_verify
-    #      state CT Q K V G B W  N  R  H dt act odt o  deltas
-    assert vf(None, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, O, DL, None) == 1
-    assert vf(FS, CT, Q, K, V, G, B, W, 4, 0, 2, 1, 0, 0, O, DL, None) == 1
-    assert vf(FS, CT, Q, K, V, G, B, W, 4, 9, 2, 1, 0, 0, O, DL, None) == 1
-    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 0, 1, 0, 0, O, DL, None) == 1
-    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 3, 0, 0, O, DL, None) == 1
-    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, O, None, None) == 1
-    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, O, DL + 8, None) == 3
-    assert vf(FS, CT, Q, K, V, G, B + 1, W, 4, 6, 2, 1, 0, 0, O, DL, None) == 3
-    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, Q, DL, None) == 1
-    assert vf(FS, CT, Q, K, V, G, B, W, 70000, 6, 2, 1, 0, 0, O, DL, None) == 2
-    assert vf(FS, CT, Q, K, V, G, B, W, 0, 6, 2, 1, 0, 0, O, DL, None) == 0
+    #      state CT Q K V G B W  N  R  H dt act odt sdt o  deltas
+    assert vf(None, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 0, 2, 1, 0, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 9, 2, 1, 0, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 0, 1, 0, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 3, 0, 0, 0, O, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, 0, O, None, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, 0, O, DL + 8, None) == 3
+    assert vf(FS, CT, Q, K, V, G, B + 1, W, 4, 6, 2, 1, 0, 0, 0, O, DL, None) == 3
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, 0, Q, DL, None) == 1
+    assert vf(FS, CT, Q, K, V, G, B, W, 70000, 6, 2, 1, 0, 0, 0, O, DL, None) == 2
+    assert vf(FS, CT, Q, K, V, G, B, W, 0, 6, 2, 1, 0, 0, 0, O, DL, None) == 0
+    assert vf(FS, CT, Q, K, V, G, B, W, 4, 6, 2, 1, 0, 0, 5, O, DL, None) == 1
     cm = kda.lib.kda_decode_commit
-    #      state CT Q K V deltas n_acc N R H dt
-    assert cm(FS, CT, Q, K, V, DL, NA, 4, 0, 2, 1, None) == 1
-    assert cm(FS, CT, Q, K, V, DL, NA, 4, 6, 2, 7, None) == 1
-    assert cm(FS, CT, Q, K, V, None, NA, 4, 6, 2, 1, None) == 1
-    assert cm(FS, CT, Q, K, V, DL, None, 4, 6, 2, 1, None) == 1
-    assert cm(FS, CT, Q, K, V, DL, NA + 2, 4, 6, 2, 1, None) == 3
-    assert cm(FS + 4, CT, Q, K, V, DL, NA, 4, 6, 2, 1, None) == 3
-    assert cm(FS, CT, Q, K, V, DL, NA, 70000, 6, 2, 1, None) == 2
-    assert cm(FS, CT, Q, K, V, DL, NA, 0, 6, 2, 1, None) == 0
+    #      state CT Q K V deltas n_acc N R H dt sdt
+    assert cm(FS, CT, Q, K, V, DL, NA, 4, 0, 2, 1, 0, None) == 1
+    assert cm(FS, CT, Q, K, V, DL, NA, 4, 6, 2, 7, 0, None) == 1
+    assert cm(FS, CT, Q, K, V, None, NA, 4, 6, 2, 1, 0, None) == 1
+    assert cm(FS, CT, Q, K, V, DL, None, 4, 6, 2, 1, 0, None) == 1
+    assert cm(FS, CT, Q, K, V, DL, NA + 2, 4, 6, 2, 1, 0, None) == 3
+    assert cm(FS + 4, CT, Q, K, V, DL, NA, 4, 6, 2, 1, 0, None) == 3
+    assert cm(FS, CT, Q, K, V, DL, NA, 70000, 6, 2, 1, 0, None) == 2
+    assert cm(FS, CT, Q, K, V, DL, NA, 0, 6, 2, 1, 0, None) == 0
+    assert cm(FS, CT, Q, K, V, DL, NA, 4, 6, 2, 1, 3, None) == 1
+
+
+def test_commit_verify_argument_validation():
+    cv = kda.lib.kda_decode_commit_verify
+    PQ, PK, PV, PD = 14 << 20, 15 << 20, 16 << 20, 17 << 20
+    size = kda.lib.kda_decode_deltas_size(4, 6, 2)
+
+    def call(state=FS, pq=PQ, pdl=PD, na=NA, prows=6, rows=6, deltas=DL, sdt=0, n=4):
+        #         state CT  prev q k v  deltas  n_acc prows  Q K V G B W  N rows H dt act odt sdt o deltas
+        return cv(state, CT, pq, PK, PV, pdl, na, prows, Q, K, V, G, B, W, n, rows, 2, 1, 0, 0, sdt, O, deltas, None)
+
+    assert call(n=0) == 0
+    assert call(prows=0) == 1 and call(prows=kda.MAX_VERIFY_ROWS + 1) == 1
+    assert call(rows=0) == 1
+    assert call(pq=None) == 1 and call(pdl=None) == 1 and call(na=None) == 1
+    assert call(na=NA + 2) == 3 and call(pq=PQ + 4) == 3
+    assert call(sdt=4) == 1
+    assert call(deltas=PD) == 1                        # the same buffer
+    assert call(deltas=PD + size - 16) == 1            # overlapping ranges
+    assert call(deltas=PD - size + 16) == 1
+    assert call(n=70000) == 2

@@ -122,3 +122,47 @@ def test_out_of_range_accept_is_clamped_and_reported():
     assert kda.check_async_status() == 0
     assert torch.equal(S[0], snaps[4][0][0]) and torch.equal(S[1], snaps[0][0][1])
     assert torch.equal(S[2], snaps[2][0][2]) and torch.equal(cache[2], snaps[2][1][2])
+
+
+@pytest.mark.parametrize("state_dtype", [torch.float32, torch.bfloat16])
+def test_commit_verify_equals_commit_then_verify(state_dtype):
+    """Three speculative steps of 6, 4 and 6 rows (0..R rows kept, so steps
+    that keep nothing occur): verify, then commit_verify per later step, equals
+    verify / commit / verify / commit / verify bit for bit (outputs of every
+    step, deltas, and the state and cache after committing the last step)."""
+    steps = [ki.make_decode_rows(9, R, 3, torch.bfloat16, 90 + i, accept=(0, R)) for i, R in enumerate((6, 4, 6))]
+    assert any(int(x) == 0 for st in steps for x in st.n_accept)
+    first = steps[0]
+    rows = [{n: getattr(st, n).cuda() for n in ("q", "k", "v", "g", "beta")} for st in steps]
+    accept = [torch.from_numpy(st.n_accept).cuda() for st in steps]
+    conv_w = first.conv_w.cuda()
+
+    def fresh():
+        return first.state.to(state_dtype).cuda(), first.conv_cache.clone().cuda()
+
+    # separate calls
+    S, C = fresh()
+    outs_a = []
+    for i, r in enumerate(rows):
+        o, dl = kda.decode_verify(S, C, r["q"], r["k"], r["v"], r["g"], r["beta"], conv_w)
+        kda.decode_commit(S, C, r["q"], r["k"], r["v"], dl, accept[i])
+        outs_a.append(o)
+    # fused: one pass per step after the first
+    S2, C2 = fresh()
+    r = rows[0]
+    o, dl = kda.decode_verify(S2, C2, r["q"], r["k"], r["v"], r["g"], r["beta"], conv_w)
+    outs_b = [o]
+    bufs = [dl, torch.empty_like(dl)]
+    for i in (1, 2):
+        p, r = rows[i - 1], rows[i]
+        out_buf = torch.empty(kda.deltas_size(9, r["q"].shape[1], 3) // 4, dtype=torch.float32, device="cuda")
+        o, dl_new = kda.decode_commit_verify(S2, C2, (p["q"], p["k"], p["v"], dl, accept[i - 1]), r["q"], r["k"],
+                                             r["v"], r["g"], r["beta"], conv_w, deltas=out_buf)
+        outs_b.append(o)
+        dl = dl_new
+    kda.decode_commit(S2, C2, rows[2]["q"], rows[2]["k"], rows[2]["v"], dl, accept[2])
+    torch.cuda.synchronize()
+    assert kda.check_async_status() == 0
+    for a, b in zip(outs_a, outs_b):
+        assert torch.equal(a, b)
+    assert torch.equal(S, S2) and torch.equal(C, C2)

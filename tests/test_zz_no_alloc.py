@@ -21,8 +21,8 @@ def test_noalloc_rejects_problems_beyond_the_static_scratch():
     cu = np.array([0, T], dtype=np.int32)
     fake = [(i + 1) << 20 for i in range(10)]
     rc = kda.lib.kda_prefill_noalloc(fake[0], fake[1], fake[2], fake[3], fake[4], fake[5], None, None,
-                                     fake[6], cu.ctypes.data, 1, H, kda.KDA_BF16, 0, kda.KDA_F32, fake[7],
-                                     fake[8], fake[9], None)
+                                     fake[6], cu.ctypes.data, 1, H, kda.KDA_BF16, 0, kda.KDA_F32, kda.KDA_F32,
+                                     fake[7], fake[8], fake[9], None)
     assert rc == 4  # KDA_ERR_WORKSPACE
 
 
