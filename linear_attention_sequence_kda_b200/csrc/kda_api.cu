@@ -114,6 +114,15 @@ kda_status run_recurrent(PrefillArgs& a) {
   return a.dt == KDA_F32 ? launch_recurrent<float>(a) : launch_recurrent<__nv_bfloat16>(a);
 }
 
+// number of SMs of the current device (persistent grids)
+kda_status sm_count(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *out < 1)
+    return KDA_ERR_CUDA;
+  return KDA_OK;
+}
+
 // shared argument checks of the decode entry points
 kda_status check_decode_common(int num_seqs, int num_heads, kda_dtype dt, kda_dtype state_dt) {
   if (num_seqs < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
@@ -188,20 +197,34 @@ kda_status kda_decode_step(void* state, void* conv_cache, const void* q, const v
     if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
   if (!aligned(beta, esize(dt))) return KDA_ERR_ALIGNMENT;
   if (o == q || o == k || o == v || o == g) return KDA_ERR_INVALID_ARG;
+  if ((int64_t)num_seqs * num_heads > INT32_MAX) return KDA_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
+  int sms = 0;
+  if (sm_count(&sms) != KDA_OK) return KDA_ERR_CUDA;
+  bool launch_err = false;
   by_type(dt, [&](auto tin) {
     by_type(o_dt, [&](auto tout) {
       by_type(state_dt, [&](auto ts) {
         by_act(act, [&](auto a) {
           using Tin = decltype(tin);
           using Ts = decltype(ts);
-          decode_kernel<Tin, decltype(tout), decltype(a)::value, Ts><<<dim3(num_heads, num_seqs), 256, 0, s>>>(
-              (Ts*)state, (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)g,
-              (const Tin*)beta, conv_w, num_heads, (decltype(tout)*)o);
+          auto kern = decode_kernel<Tin, decltype(tout), decltype(a)::value, Ts>;
+          constexpr uint32_t smem = decode_smem_bytes<Ts>();
+          if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+            launch_err = true;
+            return;
+          }
+          // persistent: two blocks per SM over the (sequence, head) items
+          const int64_t items = (int64_t)num_seqs * num_heads;
+          const int blocks = (int)(items < 2 * sms ? items : 2 * sms);
+          kern<<<blocks, 256, smem, s>>>((Ts*)state, (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v,
+                                         (const Tin*)g, (const Tin*)beta, conv_w, num_seqs, num_heads,
+                                         (decltype(tout)*)o);
         });
       });
     });
   });
+  if (launch_err) return KDA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -97,6 +97,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ void st_state4(__nv_bfloat16* p, float4 v) {
   __stcs(reinterpret_cast<uint2*>(p), make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w)));
 }
+// Four consecutive state elements from shared memory (a prefetched state).
+__device__ __forceinline__ float4 ld_state4_shared(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 ld_state4_shared(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xFFFF0000u));
+}
 // The value an element has after a store and a load in storage type Ts.
 template <typename Ts> __device__ __forceinline__ float4 as_stored4(float4 v);
 template <> __device__ __forceinline__ float4 as_stored4<float>(float4 v) { return v; }

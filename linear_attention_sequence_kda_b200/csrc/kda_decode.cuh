@@ -8,14 +8,16 @@
 //     S <- Diag(a) S + k u^T,  cache <- shift(cache, x)
 // so S is read once and written once (single pass).
 //
-// Block = 256 threads = 8 warps per (sequence, head).  Warp w owns rows
-// [16w, 16w+16); lane l owns columns [4l, 4l+4): 16 float4 registers per
-// thread.  The 64 KiB state is loaded with streaming 16-byte loads issued
-// before the prologue so the loads overlap it; reductions over rows are
-// finished through shared memory; the updated rows are written with
-// streaming stores.
+// Block = 256 threads = 8 warps, persistent (two per SM) over the (sequence,
+// head) items.  Warp w owns rows [16w, 16w+16); lane l owns columns
+// [4l, 4l+4): 16 float4 registers per thread.  While a block computes one item
+// a single bulk copy brings the next item's state (64 KiB, or 32 KiB in bf16)
+// into shared memory, so the state stream from HBM does not wait on the
+// prologue, the reductions or the barriers; reductions over rows are finished
+// through shared memory; the updated rows are written with streaming stores.
 #pragma once
 #include "kda_common.cuh"
+#include "kda_tc.cuh"
 
 namespace kda {
 
@@ -64,92 +66,124 @@ __device__ __forceinline__ void rows_update(float4 (&s)[16], const float* a, con
   }
 }
 
+// Bytes of dynamic shared memory decode_kernel needs (the prefetched state).
+template <typename Ts> __host__ __device__ constexpr uint32_t decode_smem_bytes() { return (uint32_t)(D * D * sizeof(Ts)); }
+
 template <typename Tin, typename Tout, int ACT, typename Ts>
 __global__ void __launch_bounds__(256, 2)
 decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
               const Tin* __restrict__ k, const Tin* __restrict__ v, const Tin* __restrict__ g,
-              const Tin* __restrict__ beta, const float* __restrict__ conv_w, int H,
+              const Tin* __restrict__ beta, const float* __restrict__ conv_w, int N, int H,
               Tout* __restrict__ o) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  Ts* next_state = reinterpret_cast<Ts*>(dsm);  // the state of the block's next item
   __shared__ __align__(16) float sh_kh[D], sh_ka[D], sh_qa[D], sh_al[D], sh_v[D], sh_u[D];
   __shared__ __align__(16) float sh_r[8][D], sh_y[8][D];
   __shared__ float sh_red[4][3];
+  __shared__ uint64_t bar_state;
 
-  const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t HD = (int64_t)H * D;
-  Ts* S = state + ((int64_t)n * H + h) * D * D;
-
-  // 1. issue the state loads first
-  float4 s[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) s[i] = ld_state4(S + (warp * 16 + i) * D + lane * 4);
-
-  // 2. prologue: threads 0..127 -> q and k of channel c; 128..255 -> v and g
-  const int c = tid & (D - 1);
-  const int64_t ch = (int64_t)h * D + c;
-  const int64_t tok = (int64_t)n * HD + ch;   // [N, H, D] index
-  Tin* cb = cache + (int64_t)n * 9 * HD + ch; // [3 x][3 t] stride HD
-  float yq = 0.f, yk = 0.f;
-  if (tid < D) {
-    const float4 wq = load4(conv_w + (0 * HD + ch) * 4);
-    const float4 wk = load4(conv_w + (1 * HD + ch) * 4);
-    const float q0 = to_f(cb[0 * HD]), q1 = to_f(cb[1 * HD]), q2 = to_f(cb[2 * HD]);
-    const float k0 = to_f(cb[3 * HD]), k1 = to_f(cb[4 * HD]), k2 = to_f(cb[5 * HD]);
-    const Tin xq = q[tok], xk = k[tok];
-    yq = conv4(wq, q0, q1, q2, to_f(xq));
-    yk = conv4(wk, k0, k1, k2, to_f(xk));
-    if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
-    // shift the cache (all reads of this channel's history are done above)
-    cb[0 * HD] = cb[1 * HD]; cb[1 * HD] = cb[2 * HD]; cb[2 * HD] = xq;
-    cb[3 * HD] = cb[4 * HD]; cb[4 * HD] = cb[5 * HD]; cb[5 * HD] = xk;
-    float nq = warp_sum(yq * yq), nk = warp_sum(yk * yk), qk = warp_sum(yq * yk);
-    if (lane == 0) { sh_red[warp][0] = nq; sh_red[warp][1] = nk; sh_red[warp][2] = qk; }
-  } else {
-    const float4 wv = load4(conv_w + (2 * HD + ch) * 4);
-    const float v0 = to_f(cb[6 * HD]), v1 = to_f(cb[7 * HD]), v2 = to_f(cb[8 * HD]);
-    const Tin xv = v[tok];
-    float yv = conv4(wv, v0, v1, v2, to_f(xv));
-    if (ACT == KDA_CONV_SILU) yv = silu(yv);
-    cb[6 * HD] = cb[7 * HD]; cb[7 * HD] = cb[8 * HD]; cb[8 * HD] = xv;
-    sh_v[c] = yv;
-    sh_al[c] = __expf(fmaxf(to_f(g[tok]), LOG_DECAY_FLOOR));
-  }
-  __syncthreads();
-  const float nq = sh_red[0][0] + sh_red[1][0] + sh_red[2][0] + sh_red[3][0];
-  const float nk = sh_red[0][1] + sh_red[1][1] + sh_red[2][1] + sh_red[3][1];
-  const float qk = sh_red[0][2] + sh_red[1][2] + sh_red[2][2] + sh_red[3][2];
-  const float rq = rsqrtf(nq + NORM_EPS), rk = rsqrtf(nk + NORM_EPS);
-  const float kq = qk * rq * rk;
-  if (tid < D) {
-    const float a = sh_al[c];
-    const float kh = yk * rk;
-    sh_kh[c] = kh;
-    sh_ka[c] = a * kh;
-    sh_qa[c] = a * yq * rq;
+  const int items = N * H;  // item = n * H + h: consecutive items are adjacent states
+  constexpr uint32_t kStateBytes = decode_smem_bytes<Ts>();
+  auto prefetch = [&](int item) {  // one thread
+    tc::fence_async_smem();  // the buffer's previous contents were read by every thread
+    tc::bar_expect_tx(&bar_state, kStateBytes);
+    tc::bulk_g2s(next_state, state + (int64_t)item * D * D, kStateBytes, &bar_state);
+  };
+  if (tid == 0) {
+    tc::bar_init(&bar_state, 1);
+    tc::bar_init_fence();
+    if ((int)blockIdx.x < items) prefetch(blockIdx.x);
   }
   __syncthreads();
 
-  // 3. partial reductions over this warp's 16 rows, 4 columns per lane
-  float4 r, y;
-  rows_dot2(s, &sh_ka[warp * 16], &sh_qa[warp * 16], r, y);
-  *reinterpret_cast<float4*>(&sh_r[warp][lane * 4]) = r;
-  *reinterpret_cast<float4*>(&sh_y[warp][lane * 4]) = y;
-  __syncthreads();
-  if (tid < D) {
-    float rr = 0.f, yy = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) { rr += sh_r[w][tid]; yy += sh_y[w][tid]; }
-    const float b = to_f(beta[(int64_t)n * H + h]);
-    const float u = b * (sh_v[tid] - rr);
-    sh_u[tid] = u;
-    o[tok] = from_f<Tout>(yy + u * kq);
-  }
-  __syncthreads();
+  uint32_t par = 0;
+  for (int item = blockIdx.x; item < items; item += gridDim.x, par ^= 1) {
+    const int n = item / H, h = item % H;
+    Ts* S = state + (int64_t)item * D * D;
 
-  // 4. S <- Diag(a) S + k u^T, written once
-  rows_update(s, &sh_al[warp * 16], &sh_kh[warp * 16], *reinterpret_cast<const float4*>(&sh_u[lane * 4]));
+    // 1. this item's state, prefetched into shared memory, into registers;
+    //    then the buffer takes the next item's state
+    if (!__syncthreads_and(tc::bar_wait(&bar_state, par))) {
+      if (tid == 0) tc::bar_wait(&bar_state, par);  // the copy in flight lands before the block exits
+      return;
+    }
+    float4 s[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
+    for (int i = 0; i < 16; ++i) s[i] = ld_state4_shared(next_state + (warp * 16 + i) * D + lane * 4);
+    __syncthreads();
+    if (tid == 0 && item + (int)gridDim.x < items) prefetch(item + gridDim.x);
+
+    // 2. prologue: threads 0..127 -> q and k of channel c; 128..255 -> v and g
+    const int c = tid & (D - 1);
+    const int64_t ch = (int64_t)h * D + c;
+    const int64_t tok = (int64_t)n * HD + ch;   // [N, H, D] index
+    Tin* cb = cache + (int64_t)n * 9 * HD + ch; // [3 x][3 t] stride HD
+    float yq = 0.f, yk = 0.f;
+    if (tid < D) {
+      const float4 wq = load4(conv_w + (0 * HD + ch) * 4);
+      const float4 wk = load4(conv_w + (1 * HD + ch) * 4);
+      const float q0 = to_f(cb[0 * HD]), q1 = to_f(cb[1 * HD]), q2 = to_f(cb[2 * HD]);
+      const float k0 = to_f(cb[3 * HD]), k1 = to_f(cb[4 * HD]), k2 = to_f(cb[5 * HD]);
+      const Tin xq = q[tok], xk = k[tok];
+      yq = conv4(wq, q0, q1, q2, to_f(xq));
+      yk = conv4(wk, k0, k1, k2, to_f(xk));
+      if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
+      // shift the cache (all reads of this channel's history are done above)
+      cb[0 * HD] = cb[1 * HD]; cb[1 * HD] = cb[2 * HD]; cb[2 * HD] = xq;
+      cb[3 * HD] = cb[4 * HD]; cb[4 * HD] = cb[5 * HD]; cb[5 * HD] = xk;
+      float nq = warp_sum(yq * yq), nk = warp_sum(yk * yk), qk = warp_sum(yq * yk);
+      if (lane == 0) { sh_red[warp][0] = nq; sh_red[warp][1] = nk; sh_red[warp][2] = qk; }
+    } else {
+      const float4 wv = load4(conv_w + (2 * HD + ch) * 4);
+      const float v0 = to_f(cb[6 * HD]), v1 = to_f(cb[7 * HD]), v2 = to_f(cb[8 * HD]);
+      const Tin xv = v[tok];
+      float yv = conv4(wv, v0, v1, v2, to_f(xv));
+      if (ACT == KDA_CONV_SILU) yv = silu(yv);
+      cb[6 * HD] = cb[7 * HD]; cb[7 * HD] = cb[8 * HD]; cb[8 * HD] = xv;
+      sh_v[c] = yv;
+      sh_al[c] = __expf(fmaxf(to_f(g[tok]), LOG_DECAY_FLOOR));
+    }
+    __syncthreads();
+    const float nq = sh_red[0][0] + sh_red[1][0] + sh_red[2][0] + sh_red[3][0];
+    const float nk = sh_red[0][1] + sh_red[1][1] + sh_red[2][1] + sh_red[3][1];
+    const float qk = sh_red[0][2] + sh_red[1][2] + sh_red[2][2] + sh_red[3][2];
+    const float rq = rsqrtf(nq + NORM_EPS), rk = rsqrtf(nk + NORM_EPS);
+    const float kq = qk * rq * rk;
+    if (tid < D) {
+      const float a = sh_al[c];
+      const float kh = yk * rk;
+      sh_kh[c] = kh;
+      sh_ka[c] = a * kh;
+      sh_qa[c] = a * yq * rq;
+    }
+    __syncthreads();
+
+    // 3. partial reductions over this warp's 16 rows, 4 columns per lane
+    float4 r, y;
+    rows_dot2(s, &sh_ka[warp * 16], &sh_qa[warp * 16], r, y);
+    *reinterpret_cast<float4*>(&sh_r[warp][lane * 4]) = r;
+    *reinterpret_cast<float4*>(&sh_y[warp][lane * 4]) = y;
+    __syncthreads();
+    if (tid < D) {
+      float rr = 0.f, yy = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) { rr += sh_r[w][tid]; yy += sh_y[w][tid]; }
+      const float b = to_f(beta[(int64_t)n * H + h]);
+      const float u = b * (sh_v[tid] - rr);
+      sh_u[tid] = u;
+      o[tok] = from_f<Tout>(yy + u * kq);
+    }
+    __syncthreads();
+
+    // 4. S <- Diag(a) S + k u^T, written once.  The shared vectors are
+    //    rewritten by the next item only after its first barrier, which every
+    //    thread reaches after this update.
+    rows_update(s, &sh_al[warp * 16], &sh_kh[warp * 16], *reinterpret_cast<const float4*>(&sh_u[lane * 4]));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
+  }
 }
 
 }  // namespace kda
