@@ -123,6 +123,20 @@ kda_status sm_count(int* out) {
   return KDA_OK;
 }
 
+// Launch a persistent decode-family kernel (256 threads, the prefetched state
+// in dynamic shared memory) with two blocks per SM over N x H items.
+template <typename Ts, typename Kern, typename... Args>
+kda_status launch_persistent(Kern kern, int64_t items, cudaStream_t s, Args... args) {
+  int sms = 0;
+  if (sm_count(&sms) != KDA_OK) return KDA_ERR_CUDA;
+  constexpr uint32_t smem = decode_smem_bytes<Ts>();
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  const int blocks = (int)(items < 2 * sms ? items : 2 * sms);
+  kern<<<blocks, 256, smem, s>>>(args...);
+  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 // shared argument checks of the decode entry points
 kda_status check_decode_common(int num_seqs, int num_heads, kda_dtype dt, kda_dtype state_dt) {
   if (num_seqs < 0 || num_heads < 1) return KDA_ERR_INVALID_ARG;
@@ -199,33 +213,22 @@ kda_status kda_decode_step(void* state, void* conv_cache, const void* q, const v
   if (o == q || o == k || o == v || o == g) return KDA_ERR_INVALID_ARG;
   if ((int64_t)num_seqs * num_heads > INT32_MAX) return KDA_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
-  int sms = 0;
-  if (sm_count(&sms) != KDA_OK) return KDA_ERR_CUDA;
-  bool launch_err = false;
+  kda_status rc = KDA_OK;
   by_type(dt, [&](auto tin) {
     by_type(o_dt, [&](auto tout) {
       by_type(state_dt, [&](auto ts) {
         by_act(act, [&](auto a) {
           using Tin = decltype(tin);
           using Ts = decltype(ts);
-          auto kern = decode_kernel<Tin, decltype(tout), decltype(a)::value, Ts>;
-          constexpr uint32_t smem = decode_smem_bytes<Ts>();
-          if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
-            launch_err = true;
-            return;
-          }
-          // persistent: two blocks per SM over the (sequence, head) items
-          const int64_t items = (int64_t)num_seqs * num_heads;
-          const int blocks = (int)(items < 2 * sms ? items : 2 * sms);
-          kern<<<blocks, 256, smem, s>>>((Ts*)state, (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v,
-                                         (const Tin*)g, (const Tin*)beta, conv_w, num_seqs, num_heads,
-                                         (decltype(tout)*)o);
+          rc = launch_persistent<Ts>(decode_kernel<Tin, decltype(tout), decltype(a)::value, Ts>,
+                                     (int64_t)num_seqs * num_heads, s, (Ts*)state, (Tin*)conv_cache, (const Tin*)q,
+                                     (const Tin*)k, (const Tin*)v, (const Tin*)g, (const Tin*)beta, conv_w,
+                                     num_seqs, num_heads, (decltype(tout)*)o);
         });
       });
     });
   });
-  if (launch_err) return KDA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return rc;
 }
 
 size_t kda_decode_deltas_size(int num_seqs, int num_rows, int num_heads) {
@@ -250,6 +253,7 @@ kda_status kda_decode_verify(const void* state, const void* conv_cache, const vo
   if (!aligned(beta, esize(dt))) return KDA_ERR_ALIGNMENT;
   if (o == q || o == k || o == v || o == g || (const void*)deltas == state) return KDA_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
+  kda_status rc = KDA_OK;
   by_type(dt, [&](auto tin) {
     by_type(o_dt, [&](auto tout) {
       by_type(state_dt, [&](auto ts) {
@@ -262,11 +266,12 @@ kda_status kda_decode_verify(const void* state, const void* conv_cache, const vo
                                                          (const Tin*)v, (const Tin*)g, (const Tin*)beta, conv_w,
                                                          num_rows, num_heads, (decltype(tout)*)o, deltas, nullptr,
                                                          nullptr, nullptr, nullptr, nullptr, 0);
+          rc = cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
         });
       });
     });
   });
-  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return rc;
 }
 
 kda_status kda_decode_commit_verify(void* state, void* conv_cache, const void* prev_q, const void* prev_k,
@@ -295,6 +300,7 @@ kda_status kda_decode_commit_verify(void* state, void* conv_cache, const void* p
     if (d0 < p1 && p0 < d1) return KDA_ERR_INVALID_ARG;
   }
   cudaStream_t s = (cudaStream_t)stream;
+  kda_status rc = KDA_OK;
   by_type(dt, [&](auto tin) {
     by_type(o_dt, [&](auto tout) {
       by_type(state_dt, [&](auto ts) {
@@ -307,11 +313,12 @@ kda_status kda_decode_commit_verify(void* state, void* conv_cache, const void* p
                                                          num_rows, num_heads, (decltype(tout)*)o, deltas,
                                                          (const Tin*)prev_q, (const Tin*)prev_k, (const Tin*)prev_v,
                                                          prev_deltas, prev_n_accept, prev_rows);
+          rc = cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
         });
       });
     });
   });
-  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return rc;
 }
 
 kda_status kda_decode_commit(void* state, void* conv_cache, const void* q, const void* k, const void* v,
@@ -327,16 +334,17 @@ kda_status kda_decode_commit(void* state, void* conv_cache, const void* q, const
     if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
   if (!aligned(n_accept, 4)) return KDA_ERR_ALIGNMENT;
   cudaStream_t s = (cudaStream_t)stream;
+  kda_status rc = KDA_OK;
   by_type(dt, [&](auto tin) {
     by_type(state_dt, [&](auto ts) {
       using Tin = decltype(tin);
       using Ts = decltype(ts);
-      decode_commit_kernel<Tin, Ts><<<dim3(num_heads, num_seqs), 256, 0, s>>>(
-          (Ts*)state, (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, deltas, n_accept, num_rows,
-          num_heads);
+      rc = launch_persistent<Ts>(decode_commit_kernel<Tin, Ts>, (int64_t)num_seqs * num_heads, s, (Ts*)state,
+                                 (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, deltas, n_accept,
+                                 num_seqs, num_rows, num_heads);
     });
   });
-  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return rc;
 }
 
 const char* kda_status_string(kda_status s) {

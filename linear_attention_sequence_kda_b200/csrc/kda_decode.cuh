@@ -66,8 +66,62 @@ __device__ __forceinline__ void rows_update(float4 (&s)[16], const float* a, con
   }
 }
 
-// Bytes of dynamic shared memory decode_kernel needs (the prefetched state).
+// Bytes of dynamic shared memory the persistent decode kernels need (the
+// prefetched state).
 template <typename Ts> __host__ __device__ constexpr uint32_t decode_smem_bytes() { return (uint32_t)(D * D * sizeof(Ts)); }
+
+// State prefetch of the persistent decode kernels (256 threads, items visited
+// as blockIdx.x, + gridDim.x, ...): while a block computes one (sequence, head)
+// item, one bulk copy brings the next item's state into the dynamic shared
+// memory buffer.  init() is called once by all threads before the item loop
+// (it contains a barrier); take() by all threads at the top of each item.
+template <typename Ts>
+struct StatePrefetch {
+  Ts* buf;
+  const Ts* state;
+  uint64_t* bar;
+  int items;
+  uint32_t par;
+
+  __device__ __forceinline__ void issue(int item) {  // one thread
+    tc::fence_async_smem();  // the buffer's previous contents were read by every thread
+    tc::bar_expect_tx(bar, decode_smem_bytes<Ts>());
+    tc::bulk_g2s(buf, state + (int64_t)item * D * D, decode_smem_bytes<Ts>(), bar);
+  }
+  __device__ __forceinline__ void init(const Ts* st, int n_items) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ uint64_t bar_state;
+    buf = reinterpret_cast<Ts*>(dsm);
+    state = st;
+    bar = &bar_state;
+    items = n_items;
+    par = 0;
+    if (threadIdx.x == 0) {
+      tc::bar_init(bar, 1);
+      tc::bar_init_fence();
+      if ((int)blockIdx.x < items) issue(blockIdx.x);
+    }
+    __syncthreads();
+  }
+  // This item's state into registers (warp w rows [16w, 16w+16), lane l
+  // columns [4l, 4l+4)), then the next item's copy is issued.  Returns false
+  // for the whole block if the copy did not land in time (recorded as
+  // KDA_ERR_TIMEOUT; the copy in flight is awaited once more before the block
+  // gives up, so nothing lands in shared memory after it exits).
+  __device__ __forceinline__ bool take(int item, float4 (&s)[16]) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (!__syncthreads_and(tc::bar_wait(bar, par))) {
+      if (threadIdx.x == 0) tc::bar_wait(bar, par);
+      return false;
+    }
+    par ^= 1;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s[i] = ld_state4_shared(buf + (warp * 16 + i) * D + lane * 4);
+    __syncthreads();
+    if (threadIdx.x == 0 && item + (int)gridDim.x < items) issue(item + gridDim.x);
+    return true;
+  }
+};
 
 template <typename Tin, typename Tout, int ACT, typename Ts>
 __global__ void __launch_bounds__(256, 2)
@@ -75,45 +129,22 @@ decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __rest
               const Tin* __restrict__ k, const Tin* __restrict__ v, const Tin* __restrict__ g,
               const Tin* __restrict__ beta, const float* __restrict__ conv_w, int N, int H,
               Tout* __restrict__ o) {
-  extern __shared__ __align__(128) uint8_t dsm[];
-  Ts* next_state = reinterpret_cast<Ts*>(dsm);  // the state of the block's next item
   __shared__ __align__(16) float sh_kh[D], sh_ka[D], sh_qa[D], sh_al[D], sh_v[D], sh_u[D];
   __shared__ __align__(16) float sh_r[8][D], sh_y[8][D];
   __shared__ float sh_red[4][3];
-  __shared__ uint64_t bar_state;
+  StatePrefetch<Ts> pf;
+  pf.init(state, N * H);  // item = n * H + h: consecutive items are adjacent states
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t HD = (int64_t)H * D;
-  const int items = N * H;  // item = n * H + h: consecutive items are adjacent states
-  constexpr uint32_t kStateBytes = decode_smem_bytes<Ts>();
-  auto prefetch = [&](int item) {  // one thread
-    tc::fence_async_smem();  // the buffer's previous contents were read by every thread
-    tc::bar_expect_tx(&bar_state, kStateBytes);
-    tc::bulk_g2s(next_state, state + (int64_t)item * D * D, kStateBytes, &bar_state);
-  };
-  if (tid == 0) {
-    tc::bar_init(&bar_state, 1);
-    tc::bar_init_fence();
-    if ((int)blockIdx.x < items) prefetch(blockIdx.x);
-  }
-  __syncthreads();
-
-  uint32_t par = 0;
-  for (int item = blockIdx.x; item < items; item += gridDim.x, par ^= 1) {
+  for (int item = blockIdx.x; item < pf.items; item += gridDim.x) {
     const int n = item / H, h = item % H;
     Ts* S = state + (int64_t)item * D * D;
 
     // 1. this item's state, prefetched into shared memory, into registers;
     //    then the buffer takes the next item's state
-    if (!__syncthreads_and(tc::bar_wait(&bar_state, par))) {
-      if (tid == 0) tc::bar_wait(&bar_state, par);  // the copy in flight lands before the block exits
-      return;
-    }
     float4 s[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) s[i] = ld_state4_shared(next_state + (warp * 16 + i) * D + lane * 4);
-    __syncthreads();
-    if (tid == 0 && item + (int)gridDim.x < items) prefetch(item + gridDim.x);
+    if (!pf.take(item, s)) return;
 
     // 2. prologue: threads 0..127 -> q and k of channel c; 128..255 -> v and g
     const int c = tid & (D - 1);

@@ -47,7 +47,8 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
   __shared__ float sh_red[MAX_VERIFY_ROWS][4][3], sh_kq[MAX_VERIFY_ROWS], sh_beta[MAX_VERIFY_ROWS];
   // the previous step's deltas, [row][k_hat, u, alpha][D] (commit only)
   __shared__ __align__(16) float sh_prev[COMMIT ? 3 * MAX_VERIFY_ROWS : 1][D];
-
+  // one block per (sequence, head): the rows' compute dominates, and two
+  // resident blocks per SM overlap one block's state load with the other's rows
   const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t HD = (int64_t)H * D;
@@ -222,21 +223,25 @@ template <typename Tin, typename Ts>
 __global__ void __launch_bounds__(256, 2)
 decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
                      const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ deltas,
-                     const int32_t* __restrict__ n_accept, int R, int H) {
+                     const int32_t* __restrict__ n_accept, int N, int R, int H) {
   __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][D], sh_u[MAX_VERIFY_ROWS][D], sh_al[MAX_VERIFY_ROWS][D];
-  const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
+  StatePrefetch<Ts> pf;
+  pf.init(state, N * H);
+
+  // persistent loop over the (sequence, head) items
+  for (int item = blockIdx.x; item < pf.items; item += gridDim.x) {
+  const int n = item / H, h = item % H, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int64_t HD = (int64_t)H * D;
+  Ts* S = state + (int64_t)item * D * D;
+  float4 s[16];
+  if (!pf.take(item, s)) return;
   int na = n_accept[n];
   if (na < 0 || na > R) {  // out of range: record it and keep what can be kept
     if (tid == 0 && h == 0) set_status(KDA_ERR_INVALID_ARG);
     na = na < 0 ? 0 : R;
   }
-  if (na == 0) return;  // nothing accepted: state and cache stay as they are
-  Ts* S = state + ((int64_t)n * H + h) * D * D;
-  float4 s[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) s[i] = ld_state4(S + (warp * 16 + i) * D + lane * 4);
+  if (na == 0) continue;  // nothing accepted: state and cache stay as they are
   const float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;
   for (int e = tid; e < na * D; e += 256) {
     const int t = e / D, cc = e % D;
@@ -268,6 +273,7 @@ decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin*
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
+  }  // item loop
 }
 
 }  // namespace kda
