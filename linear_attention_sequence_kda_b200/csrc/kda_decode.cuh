@@ -9,33 +9,56 @@
 // so S is read once and written once (single pass).
 //
 // Block = 256 threads = 8 warps, persistent (two per SM) over the (sequence,
-// head) items.  Warp w owns rows [16w, 16w+16); lane l owns columns
-// [4l, 4l+4): 16 float4 registers per thread.  While a block computes one item
-// a single bulk copy brings the next item's state (64 KiB, or 32 KiB in bf16)
-// into shared memory, so the state stream from HBM does not wait on the
-// prologue, the reductions or the barriers; reductions over rows are finished
-// through shared memory; the updated rows are written with streaming stores.
+// head) items.  Warp w owns value columns [16w, 16w+16) of the state (layout
+// below): the column sums r and y finish inside the warp, so after the
+// prologue a row of the recurrence needs no block barrier.  While a block
+// computes one item a single bulk copy brings the next item's state (64 KiB,
+// or 32 KiB in bf16) into shared memory, so the state stream from HBM does not
+// wait on the prologue or the reductions; the updated rows are written with
+// streaming stores.
 #pragma once
 #include "kda_common.cuh"
 #include "kda_tc.cuh"
 
 namespace kda {
 
-// A warp's 16 state rows, lane l holding columns [4l, 4l+4) of each: s[i] is
-// row i.  The two helpers below are the whole state arithmetic of a decode
-// step, shared by the single-token and the multi-token kernels so that both
-// round identically.  Packed f32x2 instructions do two columns at a time; each
+// Register layout of one (sequence, head) state in the decode kernels (256
+// threads): warp w owns value columns [16w, 16w+16); lane l holds the four
+// columns c0 = 16w + 4 (l & 3) .. c0 + 3 of the sixteen rows 16 rg + i,
+// rg = l >> 2, i = 0..15, as s[i].  A warp load of one i touches 8 rows x 64
+// contiguous bytes.
+struct StateLane {
+  int rg;  // row group: rows 16 rg .. 16 rg + 15
+  int c0;  // first of the lane's four value columns
+};
+__device__ __forceinline__ StateLane state_lane() {
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  return {l >> 2, 16 * w + 4 * (l & 3)};
+}
+__device__ __forceinline__ int state_off(StateLane L, int i) { return (16 * L.rg + i) * D + L.c0; }
+
+// Per-row vectors (indexed by key channel = state row) live in shared memory
+// with 4 floats of padding after every 16 rows: row r at rpad(r).  The 8 row
+// groups of a warp then read their 16-byte vectors from 8 distinct bank quads.
+constexpr int ROWV = D + 4 * (D / 16);
+__device__ __forceinline__ int rpad(int r) { return r + 4 * (r >> 4); }
+
+// The helpers below are the whole state arithmetic of a decode step, shared
+// by the single-token and the multi-token kernels so that all of them round
+// identically.  Packed f32x2 instructions do two columns at a time; each
 // column is rounded as its scalar fmaf would round it.
 //
-// r = sum_i x_i s_i and y = sum_i z_i s_i over the 16 rows, i ascending
-// (x, z: this warp's 16 entries, shared memory, 16-byte aligned).
-__device__ __forceinline__ void rows_dot2(const float4 (&s)[16], const float* x, const float* z, float4& r,
-                                          float4& y) {
+// Column sums over all 128 rows: r = sum_row x_row s_row, y likewise with z
+// (x, z: padded row vectors).  Each lane sums its 16 rows (ascending), then
+// the 8 row groups combine by a butterfly over lanes (xor 4, 8, 16), which
+// leaves the same full sums in every lane of a column quad.
+__device__ __forceinline__ void cols_dot2(const float4 (&s)[16], const float* x, const float* z, int rg,
+                                          float4& r, float4& y) {
   float2 r0 = make_float2(0.f, 0.f), r1 = r0, y0 = r0, y1 = r0;
 #pragma unroll
   for (int i4 = 0; i4 < 4; ++i4) {
-    const float4 x4 = *reinterpret_cast<const float4*>(x + 4 * i4);
-    const float4 z4 = *reinterpret_cast<const float4*>(z + 4 * i4);
+    const float4 x4 = *reinterpret_cast<const float4*>(x + 20 * rg + 4 * i4);  // rows 16 rg + 4 i4 ..
+    const float4 z4 = *reinterpret_cast<const float4*>(z + 20 * rg + 4 * i4);
     const float xs[4] = {x4.x, x4.y, x4.z, x4.w}, zs[4] = {z4.x, z4.y, z4.z, z4.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -44,18 +67,24 @@ __device__ __forceinline__ void rows_dot2(const float4 (&s)[16], const float* x,
       y0 = fma2(lo2(si), dup2(zs[j]), y0); y1 = fma2(hi2(si), dup2(zs[j]), y1);
     }
   }
-  r = cat2(r0, r1);
-  y = cat2(y0, y1);
+  float v[8] = {r0.x, r0.y, r1.x, r1.y, y0.x, y0.y, y1.x, y1.y};
+#pragma unroll
+  for (int m = 4; m < 32; m <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] += __shfl_xor_sync(0xffffffffu, v[e], m);
+  }
+  r = make_float4(v[0], v[1], v[2], v[3]);
+  y = make_float4(v[4], v[5], v[6], v[7]);
 }
 
-// s_i <- a_i s_i + kh_i u (the delta-rule row update Diag(a) S + k u^T; a, kh:
-// this warp's 16 entries in shared memory, u4: this lane's 4 columns of u).
-__device__ __forceinline__ void rows_update(float4 (&s)[16], const float* a, const float* kh, float4 u4) {
+// s_row <- a_row s_row + kh_row u (the delta-rule update Diag(a) S + k u^T;
+// a, kh: padded row vectors; u4: the lane's 4 columns of u).
+__device__ __forceinline__ void rows_update(float4 (&s)[16], const float* a, const float* kh, int rg, float4 u4) {
   const float2 u0 = lo2(u4), u1 = hi2(u4);
 #pragma unroll
   for (int i4 = 0; i4 < 4; ++i4) {
-    const float4 a4 = *reinterpret_cast<const float4*>(a + 4 * i4);
-    const float4 k4 = *reinterpret_cast<const float4*>(kh + 4 * i4);
+    const float4 a4 = *reinterpret_cast<const float4*>(a + 20 * rg + 4 * i4);
+    const float4 k4 = *reinterpret_cast<const float4*>(kh + 20 * rg + 4 * i4);
     const float as[4] = {a4.x, a4.y, a4.z, a4.w}, ks[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -64,6 +93,20 @@ __device__ __forceinline__ void rows_update(float4 (&s)[16], const float* a, con
                 fma2(dup2(as[j]), hi2(si), mul2(dup2(ks[j]), u1)));
     }
   }
+}
+
+// u = beta (v - r) and o = y + u kq for the lane's 4 columns (the expressions
+// of the single step, element by element).
+__device__ __forceinline__ float4 delta_u(float b, float4 v, float4 r) {
+  return make_float4(b * (v.x - r.x), b * (v.y - r.y), b * (v.z - r.z), b * (v.w - r.w));
+}
+__device__ __forceinline__ float4 readout_o(float4 y, float4 u, float kq) {
+  return make_float4(y.x + u.x * kq, y.y + u.y * kq, y.z + u.z * kq, y.w + u.w * kq);
+}
+// four consecutive outputs
+__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
 }
 
 // Bytes of dynamic shared memory the persistent decode kernels need (the
@@ -103,20 +146,20 @@ struct StatePrefetch {
     }
     __syncthreads();
   }
-  // This item's state into registers (warp w rows [16w, 16w+16), lane l
-  // columns [4l, 4l+4)), then the next item's copy is issued.  Returns false
+  // This item's state into registers (the StateLane layout), then the next
+  // item's copy is issued.  Returns false
   // for the whole block if the copy did not land in time (recorded as
   // KDA_ERR_TIMEOUT; the copy in flight is awaited once more before the block
   // gives up, so nothing lands in shared memory after it exits).
   __device__ __forceinline__ bool take(int item, float4 (&s)[16]) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const StateLane L = state_lane();
     if (!__syncthreads_and(tc::bar_wait(bar, par))) {
       if (threadIdx.x == 0) tc::bar_wait(bar, par);
       return false;
     }
     par ^= 1;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s[i] = ld_state4_shared(buf + (warp * 16 + i) * D + lane * 4);
+    for (int i = 0; i < 16; ++i) s[i] = ld_state4_shared(buf + state_off(L, i));
     __syncthreads();
     if (threadIdx.x == 0 && item + (int)gridDim.x < items) issue(item + gridDim.x);
     return true;
@@ -129,13 +172,14 @@ decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __rest
               const Tin* __restrict__ k, const Tin* __restrict__ v, const Tin* __restrict__ g,
               const Tin* __restrict__ beta, const float* __restrict__ conv_w, int N, int H,
               Tout* __restrict__ o) {
-  __shared__ __align__(16) float sh_kh[D], sh_ka[D], sh_qa[D], sh_al[D], sh_v[D], sh_u[D];
-  __shared__ __align__(16) float sh_r[8][D], sh_y[8][D];
+  // row vectors (padded, see rpad) and the value column vector
+  __shared__ __align__(16) float sh_kh[ROWV], sh_ka[ROWV], sh_qa[ROWV], sh_al[ROWV], sh_v[D];
   __shared__ float sh_red[4][3];
   StatePrefetch<Ts> pf;
   pf.init(state, N * H);  // item = n * H + h: consecutive items are adjacent states
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const StateLane L = state_lane();
   const int64_t HD = (int64_t)H * D;
   for (int item = blockIdx.x; item < pf.items; item += gridDim.x) {
     const int n = item / H, h = item % H;
@@ -174,7 +218,7 @@ decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __rest
       if (ACT == KDA_CONV_SILU) yv = silu(yv);
       cb[6 * HD] = cb[7 * HD]; cb[7 * HD] = cb[8 * HD]; cb[8 * HD] = xv;
       sh_v[c] = yv;
-      sh_al[c] = __expf(fmaxf(to_f(g[tok]), LOG_DECAY_FLOOR));
+      sh_al[rpad(c)] = __expf(fmaxf(to_f(g[tok]), LOG_DECAY_FLOOR));
     }
     __syncthreads();
     const float nq = sh_red[0][0] + sh_red[1][0] + sh_red[2][0] + sh_red[3][0];
@@ -183,37 +227,27 @@ decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __rest
     const float rq = rsqrtf(nq + NORM_EPS), rk = rsqrtf(nk + NORM_EPS);
     const float kq = qk * rq * rk;
     if (tid < D) {
-      const float a = sh_al[c];
+      const float a = sh_al[rpad(c)];
       const float kh = yk * rk;
-      sh_kh[c] = kh;
-      sh_ka[c] = a * kh;
-      sh_qa[c] = a * yq * rq;
+      sh_kh[rpad(c)] = kh;
+      sh_ka[rpad(c)] = a * kh;
+      sh_qa[rpad(c)] = a * yq * rq;
     }
     __syncthreads();
 
-    // 3. partial reductions over this warp's 16 rows, 4 columns per lane
+    // 3. column sums r = S^T (a k), y = S^T (a q) within each warp; u and o for
+    //    the lane's 4 columns (lanes of row group 0 write o)
     float4 r, y;
-    rows_dot2(s, &sh_ka[warp * 16], &sh_qa[warp * 16], r, y);
-    *reinterpret_cast<float4*>(&sh_r[warp][lane * 4]) = r;
-    *reinterpret_cast<float4*>(&sh_y[warp][lane * 4]) = y;
-    __syncthreads();
-    if (tid < D) {
-      float rr = 0.f, yy = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) { rr += sh_r[w][tid]; yy += sh_y[w][tid]; }
-      const float b = to_f(beta[(int64_t)n * H + h]);
-      const float u = b * (sh_v[tid] - rr);
-      sh_u[tid] = u;
-      o[tok] = from_f<Tout>(yy + u * kq);
-    }
-    __syncthreads();
+    cols_dot2(s, sh_ka, sh_qa, L.rg, r, y);
+    const float4 u4 = delta_u(to_f(beta[(int64_t)n * H + h]), *reinterpret_cast<const float4*>(&sh_v[L.c0]), r);
+    if (L.rg == 0) store4(o + (int64_t)n * HD + (int64_t)h * D + L.c0, readout_o(y, u4, kq));
 
     // 4. S <- Diag(a) S + k u^T, written once.  The shared vectors are
     //    rewritten by the next item only after its first barrier, which every
     //    thread reaches after this update.
-    rows_update(s, &sh_al[warp * 16], &sh_kh[warp * 16], *reinterpret_cast<const float4*>(&sh_u[lane * 4]));
+    rows_update(s, sh_al, sh_kh, L.rg, u4);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
+    for (int i = 0; i < 16; ++i) st_state4(S + state_off(L, i), s[i]);
   }
 }
 

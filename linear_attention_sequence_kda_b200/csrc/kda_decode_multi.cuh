@@ -12,8 +12,9 @@
 // rows leaves exactly the state and conv cache of n single-token steps.
 //
 // decode_verify_kernel: one 256-thread block per (sequence, head).  The state
-// is read once into registers (warp w rows [16w, 16w+16), lane l columns
-// [4l, 4l+4)) and updated there row by row; it is not written back.  Per row t
+// is read once into registers (the StateLane layout of kda_decode.cuh: each
+// warp owns 16 value columns) and updated there row by row without block
+// barriers; it is not written back.  Per row t
 // it writes o_t and the row's update (k_hat_t, u_t, alpha_t) to `deltas`.
 // decode_commit_kernel: per (sequence, head), S <- Diag(alpha_t) S + k_hat_t u_t^T
 // for the first n_accept rows (one read and one write of S), and the conv
@@ -41,21 +42,23 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
                      const float* __restrict__ pdeltas, const int32_t* __restrict__ pn_accept, int PR) {
   // per row: k_hat, alpha * k_hat, alpha * q_hat, alpha, conv(v); the row
   // prologues do not depend on the state, so all rows are prepared first
-  __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][D], sh_ka[MAX_VERIFY_ROWS][D],
-      sh_qa[MAX_VERIFY_ROWS][D], sh_al[MAX_VERIFY_ROWS][D], sh_v[MAX_VERIFY_ROWS][D];
-  __shared__ __align__(16) float sh_r[8][D], sh_y[8][D], sh_u[D];
+  // row vectors padded (rpad), the value column vectors plain
+  __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][ROWV], sh_ka[MAX_VERIFY_ROWS][ROWV],
+      sh_qa[MAX_VERIFY_ROWS][ROWV], sh_al[MAX_VERIFY_ROWS][ROWV], sh_v[MAX_VERIFY_ROWS][D];
   __shared__ float sh_red[MAX_VERIFY_ROWS][4][3], sh_kq[MAX_VERIFY_ROWS], sh_beta[MAX_VERIFY_ROWS];
-  // the previous step's deltas, [row][k_hat, u, alpha][D] (commit only)
-  __shared__ __align__(16) float sh_prev[COMMIT ? 3 * MAX_VERIFY_ROWS : 1][D];
+  // the previous step's deltas, [row][k_hat, u, alpha] (commit only): k_hat and
+  // alpha padded row vectors, u a column vector
+  __shared__ __align__(16) float sh_prev[COMMIT ? 3 * MAX_VERIFY_ROWS : 1][ROWV];
   // one block per (sequence, head): the rows' compute dominates, and two
   // resident blocks per SM overlap one block's state load with the other's rows
   const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const StateLane L = state_lane();
   const int64_t HD = (int64_t)H * D;
   Ts* S = state + ((int64_t)n * H + h) * D * D;
   float4 s[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) s[i] = ld_state4(S + (warp * 16 + i) * D + lane * 4);
+  for (int i = 0; i < 16; ++i) s[i] = ld_state4(S + state_off(L, i));
   int na = 0;  // rows of the previous step kept
   if (COMMIT) {
     na = pn_accept[n];
@@ -64,7 +67,10 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
       na = na < 0 ? 0 : PR;
     }
     const float* pdl = pdeltas + ((int64_t)n * H + h) * PR * 3 * D;
-    for (int e = tid; e < na * 3 * D; e += 256) sh_prev[e / D][e % D] = pdl[e];
+    for (int e = tid; e < na * 3 * D; e += 256) {
+      const int row = e / D, cc = e % D;  // row = 3 t + part
+      sh_prev[row][row % 3 == 1 ? cc : rpad(cc)] = pdl[e];
+    }
   }
 
   // 1. prologues of all rows: threads 0..127 q and k of channel c, threads
@@ -140,7 +146,7 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
         if (ACT == KDA_CONV_SILU) yv = silu(yv);
         hv[0] = hv[1]; hv[1] = hv[2]; hv[2] = xv;
         sh_v[t][c] = yv;
-        sh_al[t][c] = __expf(fmaxf(xgs[t], LOG_DECAY_FLOOR));
+        sh_al[t][rpad(c)] = __expf(fmaxf(xgs[t], LOG_DECAY_FLOOR));
       }
     }
   }
@@ -153,11 +159,11 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
         const float nk = sh_red[t][0][1] + sh_red[t][1][1] + sh_red[t][2][1] + sh_red[t][3][1];
         const float qk = sh_red[t][0][2] + sh_red[t][1][2] + sh_red[t][2][2] + sh_red[t][3][2];
         const float rq = rsqrtf(nq + NORM_EPS), rk = rsqrtf(nk + NORM_EPS);
-        const float a = sh_al[t][c];
+        const float a = sh_al[t][rpad(c)];
         const float kh = yk[t] * rk;
-        sh_kh[t][c] = kh;
-        sh_ka[t][c] = a * kh;
-        sh_qa[t][c] = a * yq[t] * rq;
+        sh_kh[t][rpad(c)] = kh;
+        sh_ka[t][rpad(c)] = a * kh;
+        sh_qa[t][rpad(c)] = a * yq[t] * rq;
         if (c == 0) sh_kq[t] = qk * rq * rk;
         dl[(t * 3 + 0) * D + c] = kh;  // the parts of the row's update that do
         dl[(t * 3 + 2) * D + c] = a;   // not depend on the state
@@ -171,8 +177,8 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
   // value (the commit's deltas reached shared memory before the barriers above)
   if (COMMIT && na > 0) {
     for (int t = 0; t < na; ++t) {
-      rows_update(s, &sh_prev[3 * t + 2][warp * 16], &sh_prev[3 * t][warp * 16],
-                  *reinterpret_cast<const float4*>(&sh_prev[3 * t + 1][lane * 4]));
+      rows_update(s, sh_prev[3 * t + 2], sh_prev[3 * t], L.rg,
+                  *reinterpret_cast<const float4*>(&sh_prev[3 * t + 1][L.c0]));
       if (t + 1 < na) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) s[i] = as_stored4<Ts>(s[i]);
@@ -180,38 +186,25 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
     }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
+      st_state4(S + state_off(L, i), s[i]);
       s[i] = as_stored4<Ts>(s[i]);
     }
   }
 
-  // 2. the rows in turn against the state held in registers: threads 0..127
-  //    finish r and u of channel c, threads 128..255 the readout y, which
-  //    they complete with u once it is in shared memory
+  // 2. the rows in turn against the state held in registers.  Each warp owns
+  //    16 value columns, so the column sums, u, o and the update of a row need
+  //    no block barrier: the row vectors were all written before the barrier
+  //    above, and each warp only touches its own columns afterwards.
   for (int t = 0; t < R; ++t) {
     float4 r, y;
-    rows_dot2(s, &sh_ka[t][warp * 16], &sh_qa[t][warp * 16], r, y);
-    *reinterpret_cast<float4*>(&sh_r[warp][lane * 4]) = r;
-    *reinterpret_cast<float4*>(&sh_y[warp][lane * 4]) = y;
-    __syncthreads();
-    float yy = 0.f;
-    if (tid < D) {
-      float rr = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) rr += sh_r[w][c];
-      const float u = sh_beta[t] * (sh_v[t][c] - rr);
-      sh_u[c] = u;
-      dl[(t * 3 + 1) * D + c] = u;
-    } else {
-#pragma unroll
-      for (int w = 0; w < 8; ++w) yy += sh_y[w][c];
+    cols_dot2(s, sh_ka[t], sh_qa[t], L.rg, r, y);
+    const float4 u4 = delta_u(sh_beta[t], *reinterpret_cast<const float4*>(&sh_v[t][L.c0]), r);
+    if (L.rg == 0) {
+      store4(o + (((int64_t)n * R + t) * H + h) * D + L.c0, readout_o(y, u4, sh_kq[t]));
+      *reinterpret_cast<float4*>(dl + (t * 3 + 1) * D + L.c0) = u4;
     }
-    __syncthreads();
-    // sh_r / sh_y / sh_u of the next row are written only after every thread
-    // has passed the next row's first barrier, i.e. after these reads
-    if (tid >= D) o[(((int64_t)n * R + t) * H + h) * D + c] = from_f<Tout>(yy + sh_u[c] * sh_kq[t]);
     if (t + 1 < R) {
-      rows_update(s, &sh_al[t][warp * 16], &sh_kh[t][warp * 16], *reinterpret_cast<const float4*>(&sh_u[lane * 4]));
+      rows_update(s, sh_al[t], sh_kh[t], L.rg, u4);
       // the next row starts from the state as a single step would have stored it
 #pragma unroll
       for (int i = 0; i < 16; ++i) s[i] = as_stored4<Ts>(s[i]);
@@ -224,14 +217,16 @@ __global__ void __launch_bounds__(256, 2)
 decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
                      const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ deltas,
                      const int32_t* __restrict__ n_accept, int N, int R, int H) {
-  __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][D], sh_u[MAX_VERIFY_ROWS][D], sh_al[MAX_VERIFY_ROWS][D];
+  // row vectors k_hat, alpha padded (rpad); u a column vector
+  __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][ROWV], sh_u[MAX_VERIFY_ROWS][D],
+      sh_al[MAX_VERIFY_ROWS][ROWV];
   StatePrefetch<Ts> pf;
   pf.init(state, N * H);
 
   // persistent loop over the (sequence, head) items
   for (int item = blockIdx.x; item < pf.items; item += gridDim.x) {
   const int n = item / H, h = item % H, tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
+  const StateLane L = state_lane();
   const int64_t HD = (int64_t)H * D;
   Ts* S = state + (int64_t)item * D * D;
   float4 s[16];
@@ -245,9 +240,9 @@ decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin*
   const float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;
   for (int e = tid; e < na * D; e += 256) {
     const int t = e / D, cc = e % D;
-    sh_kh[t][cc] = dl[(t * 3 + 0) * D + cc];
+    sh_kh[t][rpad(cc)] = dl[(t * 3 + 0) * D + cc];
     sh_u[t][cc] = dl[(t * 3 + 1) * D + cc];
-    sh_al[t][cc] = dl[(t * 3 + 2) * D + cc];
+    sh_al[t][rpad(cc)] = dl[(t * 3 + 2) * D + cc];
   }
   // conv cache: the last three raw tokens of [cache (3 rows), accepted rows];
   // all three are read before any is written (the cache is updated in place)
@@ -265,14 +260,14 @@ decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin*
   }
   __syncthreads();
   for (int t = 0; t < na; ++t) {
-    rows_update(s, &sh_al[t][warp * 16], &sh_kh[t][warp * 16], *reinterpret_cast<const float4*>(&sh_u[t][lane * 4]));
+    rows_update(s, sh_al[t], sh_kh[t], L.rg, *reinterpret_cast<const float4*>(&sh_u[t][L.c0]));
     if (t + 1 < na) {  // every kept row stores its state (the last one below)
 #pragma unroll
       for (int i = 0; i < 16; ++i) s[i] = as_stored4<Ts>(s[i]);
     }
   }
 #pragma unroll
-  for (int i = 0; i < 16; ++i) st_state4(S + (warp * 16 + i) * D + lane * 4, s[i]);
+  for (int i = 0; i < 16; ++i) st_state4(S + state_off(L, i), s[i]);
   }  // item loop
 }
 
