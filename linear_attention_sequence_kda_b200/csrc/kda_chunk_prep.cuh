@@ -119,13 +119,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16* __restrict__ beta,
                   const float* __restrict__ conv_w, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int2* __restrict__ chunk_tab, int H,
-                  int n_items, uint8_t* __restrict__ records) {
+                  int n_items, uint8_t* __restrict__ records, int* __restrict__ work_counter,
+                  int* __restrict__ ready, int vacate_below_smid, int vacate_after) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   float* ms = (float*)(sm + P_MISC);
   float* Ms = (float*)(sm + P_MS);
   __shared__ uint64_t bar_ld, bar_p, bar_m, bar_w;
   __shared__ uint32_t tmem_base;
+  __shared__ int s_next;  // the block's next work item (claimed by thread 0)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ch = tid & 127, hb = tid >> 7;  // channel, 32-row half of the chunk
@@ -147,12 +149,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc::tma_load_2d(sm + P_RAW + 2 * RAW_BYTES, &tm_g, hh * D, y, &bar_ld);
   };
 
+  // Work items are claimed in order from a global counter, so the records are
+  // completed roughly chunk by chunk.  A block on an SM below
+  // vacate_below_smid stops claiming once vacate_after items have been
+  // handed out: those SMs then take the scan kernel, which runs concurrently
+  // and consumes records as their ready flags are published.
+  uint32_t smid;
+  asm("mov.u32 %0, %%smid;" : "=r"(smid));
+  const bool vacate = (int)smid < vacate_below_smid;
+  auto claim = [&]() -> int {  // thread 0
+    if (vacate && *reinterpret_cast<volatile int*>(work_counter) >= vacate_after) return n_items;
+    return atomicAdd(work_counter, 1);
+  };
+
   // ---- 0. once per block: TMEM, barriers, first item's tiles ----------------
   if (warp == 0) tc::tmem_alloc(&tmem_base, 256);
   if (tid == 0) {
     tc::bar_init(&bar_ld, 1); tc::bar_init(&bar_p, 1); tc::bar_init(&bar_m, 1); tc::bar_init(&bar_w, 1);
     tc::bar_init_fence();
-    if ((int)blockIdx.x < n_items) load_raw(blockIdx.x);
+    s_next = atomicAdd(work_counter, 1);  // every block takes at least one item
+    if (s_next < n_items) load_raw(s_next);
   }
   tc::fence_before();
   __syncthreads();
@@ -162,7 +178,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint32_t par = 0;  // phase parity of the per-item barriers
 
   // persistent loop over (chunk, head) work items, chunk-major
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x, par ^= 1) {
+  for (int item = s_next; item < n_items; item = s_next, par ^= 1) {
   const int cid = item / H, h = item % H;
   const int2 nc = chunk_tab[cid];
   const int n = nc.x;
@@ -563,7 +579,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc::fence_after();
   // the shared regions are free: fetch the next item's tiles while this one finishes
   __syncthreads();
-  if (tid == 0 && item + (int)gridDim.x < n_items) load_raw(item + gridDim.x);
+  if (tid == 0) {
+    const int nx = claim();
+    s_next = nx;  // read by every thread after the item's last barrier
+    if (nx < n_items) load_raw(nx);
+  }
 
   // ---- 8. -W rows into the record (row block wrow0 of RA) -------------------
   // M = 64 accumulator: row t in lane 16 * (t / 16) ... of quarter t / 16
@@ -592,6 +612,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc::fence_before();
   __syncthreads();  // TMEM columns and shared regions are reused by the next item
   tc::fence_after();
+  if (tid == 0 && ready) {  // publish the record: every thread's stores precede the barrier above
+    __threadfence();
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(ready + item), "r"(1) : "memory");
+  }
   }  // item loop
   tc::fence_before();
   __syncthreads();

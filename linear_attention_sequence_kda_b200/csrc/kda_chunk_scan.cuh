@@ -62,7 +62,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
                   const Ts* init_state, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
-                  Tout* __restrict__ o, Ts* final_state) {
+                  const int* __restrict__ ready, Tout* __restrict__ o, Ts* final_state) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   // loads (record pieces, value tiles), MMA commits, compute-warp hand-offs
@@ -170,9 +170,16 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         tc::tma_load_2d(sm + SCAN_V, &tm_v, h * D, (int)(seg0 + (int64_t)CH * i - 3), &bar_v);
         ++n_v;
       };
+      // with the prep kernel running concurrently, a chunk's record is read
+      // only once its ready flag is published (flag of chunk j at rdy[j * H])
+      const int* rdy = ready ? ready + (int64_t)chunk_base[n] * H + h : nullptr;
+      auto record_ready = [&](int j) -> bool { return !rdy || tc::flag_wait_or(rdy + (int64_t)j * H, abort_flag); };
       bool ok = true;
-      if (nchunks > 0) { load_a(0); load_v(0); load_pk(0); }
-      if (nchunks > 1) {  // the conv of chunk 0 has read value tile 0
+      if (nchunks > 0) {
+        ok = record_ready(0);
+        if (ok) { load_a(0); load_v(0); load_pk(0); }
+      }
+      if (ok && nchunks > 1) {  // the conv of chunk 0 has read value tile 0
         ok = tc::bar_wait_or(&bar_vfree, 0, abort_flag);
         if (ok) load_v(1);
       }
@@ -182,6 +189,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       for (int j = 1; j < nchunks && ok; ++j) {
         const uint32_t q = (j - 1) & 1;
         ok = tc::bar_wait_or(&bar_ma, q, abort_flag);  // MMA_A of chunk j - 1 has read the first piece
+        ok = ok && record_ready(j);
         if (ok) load_a(j);
         if (ok && j + 1 < nchunks) {
           ok = tc::bar_wait_or(&bar_vfree, j & 1, abort_flag);

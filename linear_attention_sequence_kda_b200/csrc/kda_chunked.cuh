@@ -1,10 +1,22 @@
 // Chunked bf16 prefill on the tensor cores: host-side scheduling and launches.
-// Two kernels on the caller's stream: chunk_prep_kernel (every chunk of every
-// (segment, head) in parallel) writes one operand record per chunk-head into
-// the workspace; chunk_scan_kernel (one block per (segment, head), longest
-// segments first) carries the state across the segment's chunks.
+// chunk_prep_kernel (every chunk of every (segment, head) in parallel) writes
+// one operand record per chunk-head into the workspace; chunk_scan_kernel (one
+// block per (segment, head), longest segments first) carries the state across
+// the segment's chunks.
+//
+// When the scan has few chains (at most OVERLAP_MAX_CHAINS (segment, head)
+// pairs, e.g. one long sequence), it leaves most SMs idle, so the two kernels
+// overlap: the scan runs on an internal stream forked from and joined back to
+// the caller's stream, reading each chunk's record once prep publishes its
+// ready flag, and the prep blocks on the first `chains` SMs stop claiming work
+// once a share of the items is handed out, so that the scan blocks get those
+// SMs while prep finishes on the others.  Prep claims items from a counter and
+// never waits for the scan, so the pair cannot deadlock whichever kernel's
+// blocks become resident first; with more chains the two run one after the
+// other on the caller's stream.
 #pragma once
 #include <algorithm>
+#include <mutex>
 #include <numeric>
 #include <vector>
 
@@ -22,9 +34,40 @@ inline size_t chunk_header_bytes(int N, int64_t nchunks) {
   const size_t b = (size_t)nchunks * sizeof(int2) + (size_t)(N + 1) * 4 + (size_t)N * 4;
   return (b + 1023) & ~(size_t)1023;
 }
+// work counter (16 B) and one ready flag per (chunk, head)
+inline size_t chunk_sync_bytes(int64_t nchunks, int H) {
+  return ((size_t)16 + (size_t)nchunks * H * 4 + 1023) & ~(size_t)1023;
+}
 inline size_t chunked_workspace_bytes(int N, int H, int64_t total_tokens) {
   const int64_t nc = chunk_bound(N, total_tokens);
-  return chunk_header_bytes(N, nc) + (size_t)nc * H * REC_BYTES;
+  return chunk_header_bytes(N, nc) + chunk_sync_bytes(nc, H) + (size_t)nc * H * REC_BYTES;
+}
+
+constexpr int OVERLAP_MAX_CHAINS = 96;  // leaves at least 52 of 148 SMs to prep
+// Scan time per chunk relative to prep SM-time per chunk-head (measured on
+// B200: about 3.4 us per chunk of a chain, about 11.7 us of one SM per
+// chunk-head), used to pick when prep hands SMs over to the scan.
+constexpr double PREP_PER_SCAN_CHUNK = 3.4;
+
+// Side stream and fork / join events of the overlapped mode, one set per
+// device, created on first use.
+inline kda_status overlap_stream(cudaStream_t* side, cudaEvent_t* fork, cudaEvent_t* join) {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  static cudaEvent_t forks[64] = {}, joins[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KDA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    if (cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&forks[dev], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&joins[dev], cudaEventDisableTiming) != cudaSuccess)
+      return KDA_ERR_CUDA;
+  }
+  *side = streams[dev];
+  *fork = forks[dev];
+  *join = joins[dev];
+  return KDA_OK;
 }
 
 template <int ACT>
@@ -63,7 +106,12 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   const int2* d_tab = reinterpret_cast<const int2*>(ws);
   const int32_t* d_base = reinterpret_cast<const int32_t*>(ws + (size_t)total * sizeof(int2));
   const int32_t* d_order = d_base + (N + 1);
-  uint8_t* records = ws + hdr;
+  int* work_counter = reinterpret_cast<int*>(ws + hdr);
+  int* ready = work_counter + 4;
+  uint8_t* records = ws + hdr + chunk_sync_bytes(total, H);
+  if (cudaMemsetAsync(work_counter, 0, 16 + (size_t)total * H * 4, stream) != cudaSuccess) return KDA_ERR_CUDA;
+  const int64_t items = total * H;
+  const bool overlap = items > 0 && (int64_t)N * H <= OVERLAP_MAX_CHAINS;
 
   // TMA descriptors over the packed [total_T, H*128] tensors: 67-row boxes for
   // the inputs (3 halo rows + one chunk); 64-row boxes for the output tiles
@@ -74,6 +122,14 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
       !make_tmap_2d(&to, o, rows, cols, CH, D, o_dt == KDA_F32 ? 4 : 2))
     return KDA_ERR_CUDA;
 
+  cudaStream_t scan_stream = stream, side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (overlap) {
+    if (overlap_stream(&side, &fork, &join) != KDA_OK || cudaEventRecord(fork, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(side, fork, 0) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    scan_stream = side;
+  }
   if (total > 0) {
     auto prep = chunk_prep_kernel<ACT>;
     if (cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess)
@@ -83,10 +139,22 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return KDA_ERR_CUDA;
-    const int64_t items = total * H;
     const unsigned blocks = (unsigned)(items < 2 * sms ? items : 2 * sms);
+    int vacate_sms = 0, vacate_after = (int)items;
+    if (overlap) {
+      // prep hands the first `chains` SMs to the scan after a share f of the
+      // items such that the scan's serial chain (longest segment) and prep's
+      // remainder on the other SMs end together
+      const int chains = N * H;
+      const int64_t longest = *std::max_element(nch.begin(), nch.end());
+      double f = 1.0 - (double)longest * (sms - chains) / ((double)items * PREP_PER_SCAN_CHUNK);
+      f = f < 0.0 ? 0.0 : (f > 1.0 ? 1.0 : f);
+      vacate_sms = chains;
+      vacate_after = (int)(f * (double)items);
+    }
     prep<<<blocks, PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w, (const T*)init_conv,
-                                                        cu_dev, d_tab, H, (int)items, records);
+                                                        cu_dev, d_tab, H, (int)items, records, work_counter,
+                                                        overlap ? ready : nullptr, vacate_sms, vacate_after);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
   }
   // the scan, instantiated for the output and state element types
@@ -96,9 +164,9 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     auto scan = chunk_scan_kernel<Tout, ACT, Ts>;
     if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
       return false;
-    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, stream>>>(tv, to, conv_w, (const Ts*)init_state,
-                                                               (const T*)init_conv, cu_dev, d_base, d_order, H,
-                                                               records, (Tout*)o, (Ts*)final_state);
+    scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, scan_stream>>>(
+        tv, to, conv_w, (const Ts*)init_state, (const T*)init_conv, cu_dev, d_base, d_order, H, records,
+        overlap ? ready : nullptr, (Tout*)o, (Ts*)final_state);
     return true;
   };
   bool ok;
@@ -106,8 +174,10 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     ok = state_dt == KDA_F32 ? launch_scan(float{}, float{}) : launch_scan(float{}, T{});
   else
     ok = state_dt == KDA_F32 ? launch_scan(T{}, float{}) : launch_scan(T{}, T{});
-  if (!ok) return KDA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  if (!ok || cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+  if (overlap && (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess))
+    return KDA_ERR_CUDA;
+  return KDA_OK;
 }
 
 inline kda_status launch_chunked(const void* q, const void* k, const void* v, const void* g,

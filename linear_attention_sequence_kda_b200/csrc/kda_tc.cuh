@@ -197,6 +197,34 @@ __device__ __forceinline__ bool bar_wait_or(uint64_t* bar, uint32_t parity, cons
   set_status(KDA_ERR_TIMEOUT);
   return false;
 }
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait until another kernel publishes *flag != 0 (acquire at GPU scope), then
+// order this thread's later bulk copies (async proxy) after that acquire, so
+// that they read what the flag's writer stored before it.  Bounded: gives up
+// after about two seconds (recording KDA_ERR_TIMEOUT), or without a status
+// once `*abort` is set by another role of the block.
+__device__ __forceinline__ bool flag_wait_or(const int* flag, const volatile int* abort) {
+  const uint64_t t0 = globaltimer();
+  for (int it = 0; it < (1 << 26); ++it) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      return true;
+    }
+    if ((it & 63) == 63) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > 2000000000ull) break;
+    }
+    __nanosleep(64);
+  }
+  set_status(KDA_ERR_TIMEOUT);
+  return false;
+}
 // plain arrival (release) on an mbarrier
 __device__ __forceinline__ void bar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
