@@ -122,7 +122,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   int n_items, uint8_t* __restrict__ records, int* __restrict__ work_counter,
                   int* __restrict__ ready, int vacate_below_smid, int vacate_after) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived from the shared array itself so that the
+  // compiler keeps the shared address space (32-bit shared loads and stores)
+  uint8_t* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   float* ms = (float*)(sm + P_MISC);
   float* Ms = (float*)(sm + P_MS);
   __shared__ uint64_t bar_ld, bar_p, bar_m, bar_w;

@@ -64,7 +64,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
                   const int* __restrict__ ready, Tout* __restrict__ o, Ts* final_state) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived from the shared array itself so that the
+  // compiler keeps the shared address space (32-bit shared loads and stores)
+  uint8_t* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   // loads (record pieces, value tiles), MMA commits, compute-warp hand-offs
   // loads; "free" signals for the loader; MMA commits; compute-warp hand-offs;
   // output staging full / free
