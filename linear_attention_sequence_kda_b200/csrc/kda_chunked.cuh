@@ -44,10 +44,11 @@ inline size_t chunked_workspace_bytes(int N, int H, int64_t total_tokens) {
 }
 
 constexpr int OVERLAP_MAX_CHAINS = 96;  // leaves at least 52 of 148 SMs to prep
-// Scan time per chunk relative to prep SM-time per chunk-head (measured on
-// B200: about 3.4 us per chunk of a chain, about 11.7 us of one SM per
-// chunk-head), used to pick when prep hands SMs over to the scan.
-constexpr double PREP_PER_SCAN_CHUNK = 3.4;
+// Prep SM-time per chunk-head relative to the scan's time per chunk of a
+// chain, used to pick when prep hands SMs over to the scan (the ratio that
+// gave the shortest overlapped call on B200, 64 heads x 65,536 tokens, among
+// 2.8 .. 4.4; the model value from the two kernels' separate timings is ~3).
+constexpr double PREP_PER_SCAN_CHUNK = 2.8;
 
 // Side stream and fork / join events of the overlapped mode, one set per
 // device, created on first use.
