@@ -256,7 +256,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the end-to-end leg")
+    ap.add_argument("--e2e-steps", type=int, default=6, help="0 skips the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode leg")
     ap.add_argument("--heads", type=int, default=H,
@@ -305,9 +305,12 @@ def main():
     ws_bytes = kda.workspace_size(1, T_run, heads, T_run)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
 
+    def prefill_into(dd, oo, ss):
+        kda.prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["conv_w"], inp.cu_seqlens, cu_dev,
+                    None, None, o=oo, final_state=ss, conv_tail=tail, workspace=ws, stream=stream)
+
     def step():
-        kda.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["conv_w"], inp.cu_seqlens, cu_dev,
-                    None, None, o=o, final_state=S, conv_tail=tail, workspace=ws, stream=stream)
+        prefill_into(d, o, S)
 
     with ClockSampler(torch.cuda.current_device()) as clk:
         total_ms, per_step = timed(step, args.steps, args.warmup, world, stream)
@@ -324,7 +327,7 @@ def main():
     # ---------------- end to end: host buffers through the C ABI ----------------
     e2e = None
     if args.e2e_steps > 0:
-        e2e = run_e2e(args, world, stream, inp, d, o, S, step, tokens_per_rank)
+        e2e = run_e2e(args, world, stream, inp, d, o, S, prefill_into, tokens_per_rank)
 
     # ---------------- decode step: 256 sequences, state in place ----------------
     dec_line = mtp_line = fused_line = dec16_line = mtp16_line = None
@@ -366,27 +369,66 @@ def main():
         dist.destroy_process_group()
 
 
-def run_e2e(args, world, stream, inp, d, o, S, step, tokens_per_rank):
-    """Same metric through the C ABI with host buffers: each step copies the
+def run_e2e(args, world, stream, inp, d, o, S, prefill_into, tokens_per_rank):
+    """Same metric through the C ABI with host buffers: every step copies its
     inputs from pinned host memory, runs kda_prefill, and reads o and the final
-    state back to pinned host memory."""
+    state back to pinned host memory.  The steps are pipelined as a serving
+    loop would run them: step i+1's inputs travel host-to-device on one copy
+    stream while step i computes and step i-1's results travel back on
+    another (two device buffer sets alternate).  The timed region starts
+    before the first step's input copy and ends after the last step's result
+    has reached the host."""
     pin = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "g", "beta")}
     o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     S_host = torch.empty(S.shape, dtype=S.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = o_host.numel() * o_host.element_size() + S_host.numel() * 4
+    sets = [(d, o, S), ({**d, **{n: torch.empty_like(d[n]) for n in pin}}, torch.empty_like(o), torch.empty_like(S))]
+    up, down = torch.cuda.Stream(device=o.device), torch.cuda.Stream(device=o.device)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, computed, out_read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    issued = [False, False]
 
-    def e2e_step():
-        for n, t in pin.items():
-            d[n].copy_(t, non_blocking=True)
-        step()
-        o_host.copy_(o, non_blocking=True)
-        S_host.copy_(S, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        dd, ob, sb = sets[b]
+        if issued[b]:  # step i - 2 has finished with this buffer set
+            up.wait_event(computed[b])
+        with torch.cuda.stream(up):
+            for n, t in pin.items():
+                dd[n].copy_(t, non_blocking=True)
+            in_ready[b].record(up)
+        stream.wait_event(in_ready[b])
+        if issued[b]:
+            stream.wait_event(out_read[b])
+        prefill_into(dd, ob, sb)
+        computed[b].record(stream)
+        down.wait_event(computed[b])
+        with torch.cuda.stream(down):
+            o_host.copy_(ob, non_blocking=True)
+            S_host.copy_(sb, non_blocking=True)
+            out_read[b].record(down)
+        issued[b] = True
 
-    e2e_ms, _ = timed(e2e_step, args.e2e_steps, 1, world, stream)
+    for i in range(2):  # warm-up
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    up.wait_event(start)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    stream.wait_stream(down)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(start.elapsed_time(stop), world)
     value = world * tokens_per_rank * args.e2e_steps / (e2e_ms / 1e3)
     return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": args.e2e_steps}
+            "steps": args.e2e_steps, "pipelined": "inputs of step i+1 up and results of step i-1 down while step i runs"}
 
 
 def run_decode(args, world, dev, stream, kda, hbm_peak, state_dtype=torch.float32):
