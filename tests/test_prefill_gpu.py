@@ -146,3 +146,27 @@ def test_causality():
     o2 = run_prefill(inp)[0].cpu()
     assert torch.equal(o1[:t0], o2[:t0])
     assert not torch.equal(o1[t0], o2[t0])
+
+
+@pytest.mark.parametrize("heads", [96, 97])
+def test_overlap_threshold_both_schedules(heads):
+    """One sequence with 96 heads takes the overlapped schedule (the scan runs
+    beside the prep and waits for each chunk's record), 97 heads the one after
+    the other; both against the oracle on sampled heads, and both equal to the
+    same heads run in a call of their own (4 heads, always overlapped): the
+    schedule changes when records are read, never what is computed."""
+    inp = ki.make_prefill([700], heads, torch.bfloat16, 91, state_std=0.02, conv_history=True)
+    o, S, tail = run_prefill(inp)
+    compare_prefill(inp, (o, S, tail), [(0, 0), (0, 45), (0, heads - 1)])
+    sub = ki.make_prefill([700], 4, torch.bfloat16, 91, state_std=0.02, conv_history=True)
+    hs = [0, 1, 2, 3]
+    # the same inputs restricted to heads 0..3 (inputs are drawn per tensor, so slice them)
+    D = 128
+    pick = lambda t: t.view(t.shape[0], heads, -1)[:, hs].reshape(t.shape[0], 4, *t.shape[2:]).contiguous()  # noqa: E731
+    sub.q, sub.k, sub.v, sub.g = pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.g)
+    sub.beta = inp.beta[:, hs].contiguous()
+    sub.conv_w = inp.conv_w.view(3, heads, D, 4)[:, hs].reshape(3, 4 * D, 4).contiguous()
+    sub.init_state = inp.init_state[:, hs].contiguous()
+    sub.init_conv = inp.init_conv.view(1, 3, 3, heads, D)[:, :, :, hs].reshape(1, 3, 3, 4 * D).contiguous()
+    o4, S4, _ = run_prefill(sub)
+    assert torch.equal(o4, o[:, hs]) and torch.equal(S4, S[:, hs])
