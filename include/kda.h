@@ -290,6 +290,27 @@ kda_status kda_prefill_noalloc(const void* q, const void* k, const void* v, cons
                                kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
                                void* o, void* final_state, void* conv_tail, void* stream);
 
+/*
+ * kda_state_affine -- S_out = A S_in + B for `count` (sequence, head) states:
+ * the exchange step of one long sequence split into contiguous segments
+ * (context parallelism).  Page "GLM-5.3-Flash im Detail", section
+ * "Sequenz-Mixing: ...": the state is handed from chunk to chunk, and that
+ * hand-over is linear in the state, so a whole segment maps its initial state
+ * as S_out = A S_in + B.  B is the segment's final state from S_in = 0; A
+ * (key x key) is its final state from S_in = I with v = 0 (each value column a
+ * probe; the v part of the conv history zero as well), both from kda_prefill.
+ * A rank composes its segment's initial state from the (A, B) of every
+ * earlier segment, one call per segment.
+ *   A, B        : [count, 128, 128] fp32, row = key channel.
+ *   S_in, S_out : [count, 128, 128] (state_dt); S_out may equal S_in (every
+ *                 state is read before it is written), not A or B.
+ * fp32 arithmetic with a k-ascending sum.  Errors: KDA_ERR_INVALID_ARG for a
+ * NULL pointer, count < 0, a bad state_dt or S_out aliasing A or B;
+ * KDA_ERR_ALIGNMENT for a pointer that is not 16-byte aligned.
+ */
+kda_status kda_state_affine(const float* A, const void* S_in, const float* B, void* S_out, int count,
+                            kda_dtype state_dt, void* stream);
+
 /* Static description of a status code (never NULL). */
 const char* kda_status_string(kda_status s);
 

@@ -28,7 +28,7 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
            "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version",
            "kda_prefill_noalloc", "kda_decode_deltas_size", "kda_decode_verify", "kda_decode_commit",
-           "kda_decode_commit_verify")
+           "kda_decode_commit_verify", "kda_state_affine")
 MAX_VERIFY_ROWS = 8  # KDA_MAX_VERIFY_ROWS
 
 if not os.path.exists(LIB_PATH):
@@ -65,6 +65,8 @@ lib.kda_decode_commit_verify.restype = ctypes.c_int
 lib.kda_decode_commit_verify.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32p, _i32p, ctypes.c_int, _vp, _vp, _vp, _vp,
                                          _vp, _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _f32p, _vp]
+lib.kda_state_affine.restype = ctypes.c_int
+lib.kda_state_affine.argtypes = [_f32p, _vp, _f32p, _vp, ctypes.c_int, ctypes.c_int, _vp]
 lib.kda_status_string.restype = ctypes.c_char_p
 lib.kda_status_string.argtypes = [ctypes.c_int]
 lib.kda_check_async_status.restype = ctypes.c_int
@@ -242,6 +244,18 @@ def decode_commit_verify(state, conv_cache, prev, q, k, v, g, beta, conv_w, act:
                                         _dtype_code(state), _ptr(o), _ptr(deltas), _stream(stream)),
            "kda_decode_commit_verify")
     return o, deltas
+
+
+def state_affine(A, S_in, B, S_out=None, stream=None):
+    """kda_state_affine: S_out = A S_in + B per (sequence, head); A and B fp32
+    [..., 128, 128], S_in in the state storage type (S_out defaults to a new
+    tensor of that type; it may be S_in)."""
+    if S_out is None:
+        S_out = torch.empty_like(S_in)
+    count = S_in.numel() // (HEAD_DIM * HEAD_DIM)
+    _check(lib.kda_state_affine(_ptr(A), _ptr(S_in), _ptr(B), _ptr(S_out), count, _dtype_code(S_in),
+                                _stream(stream)), "kda_state_affine")
+    return S_out
 
 
 def check_async_status(stream=None) -> int:

@@ -11,6 +11,7 @@
 #include "kda_recurrent.cuh"
 #include "kda_tail.cuh"
 #include "kda_chunked.cuh"
+#include "kda_affine.cuh"
 
 using namespace kda;
 
@@ -343,6 +344,30 @@ kda_status kda_decode_commit(void* state, void* conv_cache, const void* q, const
                                  (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, deltas, n_accept,
                                  num_seqs, num_rows, num_heads);
     });
+  });
+  return rc;
+}
+
+kda_status kda_state_affine(const float* A, const void* S_in, const float* B, void* S_out, int count,
+                            kda_dtype state_dt, void* stream) {
+  if (count < 0 || !valid_dtype(state_dt)) return KDA_ERR_INVALID_ARG;
+  if (count == 0) return KDA_OK;
+  if (!A || !S_in || !B || !S_out) return KDA_ERR_INVALID_ARG;
+  const void* al16[] = {A, S_in, B, S_out};
+  for (const void* p : al16)
+    if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+  if (S_out == (const void*)A || S_out == (const void*)B) return KDA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  kda_status rc = KDA_OK;
+  by_type(state_dt, [&](auto ts) {
+    using Ts = decltype(ts);
+    auto kern = state_affine_kernel<Ts>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AFFINE_SMEM) != cudaSuccess) {
+      rc = KDA_ERR_CUDA;
+      return;
+    }
+    kern<<<count, 256, AFFINE_SMEM, s>>>(A, (const Ts*)S_in, B, (Ts*)S_out);
+    rc = cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
   });
   return rc;
 }

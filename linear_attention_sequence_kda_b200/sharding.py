@@ -2,13 +2,28 @@
 
 The KDA mixing step has no exchange between sequences or heads (each
 (sequence, head) state evolves on its own), so a batch spreads over GPUs by
-handing each rank a contiguous block of whole sequences: no collective is needed
-on the data path.  Ranks only meet for timing (a barrier and the max of the
-per-rank device times).
+handing each rank a contiguous block of whole sequences, or each rank its own
+heads: no collective is needed on the data path.  Ranks only meet for timing (a
+barrier and the max of the per-rank device times).
+
+One long sequence split into contiguous segments, one per rank (context
+parallelism), has one exchange step: the state handed from segment to segment.
+Page "GLM-5.3-Flash im Detail", section "Sequenz-Mixing: 34 KDA-Schichten mit
+festem Zustand": the state is handed from chunk to chunk, and the hand-over is
+linear in the state, so segment r maps its initial state as
+S_out = A_r S_in + B_r.  context_parallel_prefill runs, on every rank:
+  1. the conv halo: each rank's last three raw tokens, gathered, give the next
+     rank its conv history;
+  2. the carry: one prefill call over the segment entered twice, from S = 0
+     (final state B_r) and from S = I with v = 0 (final state A_r);
+  3. the exchange: all ranks gather every (A_j, B_j);
+  4. the composition S_in(r) = A_{r-1}(... (A_0 S_0 + B_0) ...) + B_{r-1};
+  5. the segment's prefill from S_in(r): its outputs, and on the last rank the
+     sequence's final state and conv tail.
 """
 from __future__ import annotations
 
-from typing import List, Sequence, Tuple
+from typing import Callable, List, Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -56,3 +71,74 @@ def max_over_ranks(value: float, device=None) -> float:
 def whole_job_rate(units_per_rank: Sequence[int], max_seconds: float) -> float:
     """Units processed by all ranks divided by the slowest rank's time."""
     return float(sum(units_per_rank)) / max_seconds
+
+
+def conv_halo(q, k, v):
+    """[1, 3 (q, k, v), 3 (time, oldest first), H * D]: the segment's last three
+    raw tokens, the conv history of the segment after it (needs >= 3 tokens)."""
+    if q.shape[0] < 3:
+        raise ValueError("every segment but the last needs at least 3 tokens")
+    import torch
+    return torch.stack([x[-3:].reshape(3, -1) for x in (q, k, v)])[None].contiguous()
+
+
+def compose_initial_state(S0, As, Bs, rank: int, affine: Callable):
+    """S_in of segment `rank`: S0 carried through segments 0 .. rank - 1 by
+    S <- A_j S + B_j (affine(A, S, B) computes one step)."""
+    S = S0
+    for j in range(rank):
+        S = affine(As[j], S, Bs[j])
+    return S
+
+
+def segment_carry(lib, q, k, v, g, beta, conv_w, prev_tail, act: int = 0, stream=None):
+    """(A, B) of one segment, [1, H, D, D] fp32 each, from one prefill call over
+    the segment entered twice: from S = 0 with the real inputs (final state B)
+    and from S = I with v = 0 and a zero v history (final state A)."""
+    import torch
+    T, H, D = q.shape
+    two = lambda x, y=None: torch.cat([x, x if y is None else y]).contiguous()  # noqa: E731
+    init = torch.zeros((2, H, D, D), dtype=torch.float32, device=q.device)
+    init[1] = torch.eye(D, dtype=torch.float32, device=q.device)
+    hist0 = prev_tail.clone()
+    hist0[:, 2] = 0
+    cu = np.array([0, T, 2 * T], dtype=np.int32)
+    _, final, _ = lib.prefill(two(q), two(k), two(v, torch.zeros_like(v)), two(g), two(beta), conv_w, cu,
+                              init_state=init, init_conv=torch.cat([prev_tail, hist0]).contiguous(), act=act,
+                              stream=stream)
+    return final[1:2].contiguous(), final[0:1].contiguous()
+
+
+def context_parallel_prefill(lib, q, k, v, g, beta, conv_w, rank: int, world: int,
+                             all_gather: Callable, init_state=None, init_conv=None, act: int = 0,
+                             stream=None, o_dtype=None):
+    """Prefill of segment `rank` of one sequence split over `world` ranks.
+      q, k, v, g : [T_r, H, 128] this rank's tokens; beta [T_r, H].
+      init_state : [1, H, 128, 128] the sequence's initial state (rank 0; None = 0).
+      init_conv  : [1, 3, 3, H * 128] the sequence's conv history (rank 0; None = 0).
+      all_gather : t -> list of every rank's t, in rank order (a collective).
+      lib        : the library binding (prefill, state_affine).
+    Returns (o, final_state, conv_tail) of this segment; on the last rank the
+    final state and conv tail are those of the whole sequence."""
+    import torch
+    T, H, D = q.shape
+    if T >= 3:
+        halo = conv_halo(q, k, v)
+    elif rank == world - 1:  # nobody reads the last segment's halo
+        halo = torch.zeros((1, 3, 3, H * D), dtype=q.dtype, device=q.device)
+    else:
+        raise ValueError("every segment but the last needs at least 3 tokens")
+    halos = all_gather(halo)
+    if rank > 0:
+        prev_tail = halos[rank - 1]
+    elif init_conv is not None:
+        prev_tail = init_conv
+    else:
+        prev_tail = torch.zeros((1, 3, 3, H * D), dtype=q.dtype, device=q.device)
+    A, B = segment_carry(lib, q, k, v, g, beta, conv_w, prev_tail, act, stream)
+    As, Bs = all_gather(A), all_gather(B)
+    S0 = init_state if init_state is not None else torch.zeros((1, H, D, D), dtype=torch.float32, device=q.device)
+    S_in = compose_initial_state(S0, As, Bs, rank, lib.state_affine)
+    kw = {} if o_dtype is None else {"o_dtype": o_dtype}
+    return lib.prefill(q, k, v, g, beta, conv_w, np.array([0, T], dtype=np.int32), init_state=S_in,
+                       init_conv=prev_tail, act=act, stream=stream, **kw)

@@ -156,3 +156,14 @@ def test_commit_verify_argument_validation():
     assert call(deltas=PD + size - 16) == 1            # overlapping ranges
     assert call(deltas=PD - size + 16) == 1
     assert call(n=70000) == 2
+
+
+def test_state_affine_argument_validation():
+    af = kda.lib.kda_state_affine
+    Aa, Ss, Bb, So = 20 << 20, 21 << 20, 22 << 20, 23 << 20
+    assert af(Aa, Ss, Bb, So, 0, 0, None) == 0          # nothing to do
+    assert af(Aa, Ss, Bb, So, -1, 0, None) == 1
+    assert af(None, Ss, Bb, So, 4, 0, None) == 1
+    assert af(Aa, Ss, Bb, So, 4, 3, None) == 1          # state element type
+    assert af(Aa, Ss, Bb, Aa, 4, 0, None) == 1          # output aliases A
+    assert af(Aa + 4, Ss, Bb, So, 4, 0, None) == 3
