@@ -124,13 +124,13 @@ kda_status sm_count(int* out) {
   return KDA_OK;
 }
 
-// Launch a persistent decode-family kernel (256 threads, the prefetched state
-// in dynamic shared memory) with two blocks per SM over N x H items.
-template <typename Ts, typename Kern, typename... Args>
-kda_status launch_persistent(Kern kern, int64_t items, cudaStream_t s, Args... args) {
+// Launch a persistent decode-family kernel (256 threads, the prefetch buffers
+// in `smem` bytes of dynamic shared memory) with two blocks per SM over N x H
+// items.
+template <typename Kern, typename... Args>
+kda_status launch_persistent(Kern kern, uint32_t smem, int64_t items, cudaStream_t s, Args... args) {
   int sms = 0;
   if (sm_count(&sms) != KDA_OK) return KDA_ERR_CUDA;
-  constexpr uint32_t smem = decode_smem_bytes<Ts>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return KDA_ERR_CUDA;
   const int blocks = (int)(items < 2 * sms ? items : 2 * sms);
@@ -221,8 +221,8 @@ kda_status kda_decode_step(void* state, void* conv_cache, const void* q, const v
         by_act(act, [&](auto a) {
           using Tin = decltype(tin);
           using Ts = decltype(ts);
-          rc = launch_persistent<Ts>(decode_kernel<Tin, decltype(tout), decltype(a)::value, Ts>,
-                                     (int64_t)num_seqs * num_heads, s, (Ts*)state, (Tin*)conv_cache, (const Tin*)q,
+          rc = launch_persistent(decode_kernel<Tin, decltype(tout), decltype(a)::value, Ts>,
+                                 DecodePrefetch<Tin, Ts, sizeof(Ts) == 2>::bytes(), (int64_t)num_seqs * num_heads, s, (Ts*)state, (Tin*)conv_cache, (const Tin*)q,
                                      (const Tin*)k, (const Tin*)v, (const Tin*)g, (const Tin*)beta, conv_w,
                                      num_seqs, num_heads, (decltype(tout)*)o);
         });
@@ -340,7 +340,8 @@ kda_status kda_decode_commit(void* state, void* conv_cache, const void* q, const
     by_type(state_dt, [&](auto ts) {
       using Tin = decltype(tin);
       using Ts = decltype(ts);
-      rc = launch_persistent<Ts>(decode_commit_kernel<Tin, Ts>, (int64_t)num_seqs * num_heads, s, (Ts*)state,
+      rc = launch_persistent(decode_commit_kernel<Tin, Ts>, decode_smem_bytes<Ts>(), (int64_t)num_seqs * num_heads, s,
+                             (Ts*)state,
                                  (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, deltas, n_accept,
                                  num_seqs, num_rows, num_heads);
     });

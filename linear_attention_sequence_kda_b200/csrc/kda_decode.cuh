@@ -166,6 +166,93 @@ struct StatePrefetch {
   }
 };
 
+// The prefetch of decode_kernel.  With a bf16 state (INPUTS = true) the inputs
+// of the next item's prologue (the q, k, v, g rows, the nine conv-cache rows,
+// the three tap rows) arrive by bulk copies on the same mbarrier as its state,
+// into one of two input slots (the prologue reads its slot after the next
+// item's copies were issued): with half the state bytes the prologue's global
+// loads would otherwise be exposed.  With an fp32 state the state stream
+// alone keeps HBM busy and the prologue reads global memory.
+template <typename Tin, typename Ts, bool INPUTS>
+struct DecodePrefetch {
+  static constexpr uint32_t kState = D * D * sizeof(Ts);
+  static constexpr uint32_t kRow = D * sizeof(Tin);
+  static constexpr uint32_t kTaps = D * 4 * sizeof(float);   // one tensor's taps
+  static constexpr uint32_t kSlot = INPUTS ? (13 * kRow + 3 * kTaps + 127) & ~127u : 0;
+  __host__ __device__ static constexpr uint32_t bytes() { return kState + 2 * kSlot; }
+
+  uint8_t* base;
+  Ts* sbuf;
+  const Ts* state;
+  const Tin *q, *k, *v, *g, *cache;
+  const float* conv_w;
+  uint64_t* bar;
+  int items, H;
+  uint32_t par, slot;
+
+  // slot layout: rows 0..3 = q, k, v, g; rows 4 + 3 x + t = cache tensor x,
+  // time t; then the taps of q, k, v ([D][4] each)
+  __device__ __forceinline__ const Tin* row(uint32_t sl, int r) const {
+    return reinterpret_cast<const Tin*>(base + kState + sl * kSlot + r * kRow);
+  }
+  __device__ __forceinline__ const float* taps(uint32_t sl, int x) const {
+    return reinterpret_cast<const float*>(base + kState + sl * kSlot + 13 * kRow + x * kTaps);
+  }
+  __device__ __forceinline__ void issue(int item, uint32_t sl) {  // one thread
+    const int64_t n = item / H, h = item % H, HD = (int64_t)H * D;
+    uint8_t* dst = base + kState + sl * kSlot;
+    tc::fence_async_smem();  // the buffers' previous contents were read by every thread
+    tc::bar_expect_tx(bar, INPUTS ? kState + 13 * kRow + 3 * kTaps : kState);
+    tc::bulk_g2s(sbuf, state + (int64_t)item * D * D, kState, bar);
+    if (!INPUTS) return;
+    const Tin* in[4] = {q, k, v, g};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) tc::bulk_g2s(dst + r * kRow, in[r] + n * HD + h * D, kRow, bar);
+#pragma unroll
+    for (int r = 0; r < 9; ++r) tc::bulk_g2s(dst + (4 + r) * kRow, cache + (n * 9 + r) * HD + h * D, kRow, bar);
+#pragma unroll
+    for (int x = 0; x < 3; ++x)
+      tc::bulk_g2s(dst + 13 * kRow + x * kTaps, conv_w + (x * HD + h * D) * 4, kTaps, bar);
+  }
+  __device__ __forceinline__ void init(const Ts* st, const Tin* q_, const Tin* k_, const Tin* v_, const Tin* g_,
+                                       const Tin* cache_, const float* w_, int n_items, int H_) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ uint64_t bar_pf;
+    base = dsm;
+    sbuf = reinterpret_cast<Ts*>(dsm);
+    state = st; q = q_; k = k_; v = v_; g = g_; cache = cache_; conv_w = w_;
+    bar = &bar_pf;
+    items = n_items;
+    H = H_;
+    par = 0;
+    slot = 0;
+    if (threadIdx.x == 0) {
+      tc::bar_init(bar, 1);
+      tc::bar_init_fence();
+      if ((int)blockIdx.x < items) issue(blockIdx.x, 0);
+    }
+    __syncthreads();
+  }
+  // This item's state into registers; *cur = the slot holding its inputs;
+  // then the next item's copies are issued into the other slot.  Bounded as
+  // StatePrefetch::take.
+  __device__ __forceinline__ bool take(int item, float4 (&s)[16], uint32_t* cur) {
+    const StateLane L = state_lane();
+    if (!__syncthreads_and(tc::bar_wait(bar, par))) {
+      if (threadIdx.x == 0) tc::bar_wait(bar, par);
+      return false;
+    }
+    par ^= 1;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s[i] = ld_state4_shared(sbuf + state_off(L, i));
+    *cur = slot;
+    slot ^= 1;
+    __syncthreads();
+    if (threadIdx.x == 0 && item + (int)gridDim.x < items) issue(item + gridDim.x, slot);
+    return true;
+  }
+};
+
 template <typename Tin, typename Tout, int ACT, typename Ts>
 __global__ void __launch_bounds__(256, 2)
 decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
@@ -175,50 +262,88 @@ decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __rest
   // row vectors (padded, see rpad) and the value column vector
   __shared__ __align__(16) float sh_kh[ROWV], sh_ka[ROWV], sh_qa[ROWV], sh_al[ROWV], sh_v[D];
   __shared__ float sh_red[4][3];
-  StatePrefetch<Ts> pf;
-  pf.init(state, N * H);  // item = n * H + h: consecutive items are adjacent states
+  constexpr bool kInputs = sizeof(Ts) == 2;
+  DecodePrefetch<Tin, Ts, kInputs> pf;
+  pf.init(state, q, k, v, g, cache, conv_w, N * H, H);  // item = n * H + h: consecutive items are adjacent
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const StateLane L = state_lane();
   const int64_t HD = (int64_t)H * D;
+  // beta of the item being computed, loaded one item ahead
+  float b_cur = kInputs && (int)blockIdx.x < pf.items ? to_f(beta[blockIdx.x]) : 0.f;
   for (int item = blockIdx.x; item < pf.items; item += gridDim.x) {
     const int n = item / H, h = item % H;
     Ts* S = state + (int64_t)item * D * D;
 
-    // 1. this item's state, prefetched into shared memory, into registers;
-    //    then the buffer takes the next item's state
+    // 1. this item's state and inputs, prefetched into shared memory; the
+    //    state into registers, then the buffers take the next item's
     float4 s[16];
-    if (!pf.take(item, s)) return;
+    uint32_t sl;
+    if (!pf.take(item, s, &sl)) return;
+    float b_next = 0.f;
+    if constexpr (kInputs) b_next = item + (int)gridDim.x < pf.items ? to_f(beta[item + gridDim.x]) : 0.f;
 
-    // 2. prologue: threads 0..127 -> q and k of channel c; 128..255 -> v and g
+    // 2. prologue: threads 0..127 -> q and k of channel c; 128..255 -> v and g.
+    //    With a bf16 state the inputs come from the prefetched slot; with an
+    //    fp32 state straight from global memory (loads issued together)
     const int c = tid & (D - 1);
     const int64_t ch = (int64_t)h * D + c;
-    const int64_t tok = (int64_t)n * HD + ch;   // [N, H, D] index
     Tin* cb = cache + (int64_t)n * 9 * HD + ch; // [3 x][3 t] stride HD
     float yq = 0.f, yk = 0.f;
-    if (tid < D) {
-      const float4 wq = load4(conv_w + (0 * HD + ch) * 4);
-      const float4 wk = load4(conv_w + (1 * HD + ch) * 4);
-      const float q0 = to_f(cb[0 * HD]), q1 = to_f(cb[1 * HD]), q2 = to_f(cb[2 * HD]);
-      const float k0 = to_f(cb[3 * HD]), k1 = to_f(cb[4 * HD]), k2 = to_f(cb[5 * HD]);
-      const Tin xq = q[tok], xk = k[tok];
-      yq = conv4(wq, q0, q1, q2, to_f(xq));
-      yk = conv4(wk, k0, k1, k2, to_f(xk));
-      if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
-      // shift the cache (all reads of this channel's history are done above)
-      cb[0 * HD] = cb[1 * HD]; cb[1 * HD] = cb[2 * HD]; cb[2 * HD] = xq;
-      cb[3 * HD] = cb[4 * HD]; cb[4 * HD] = cb[5 * HD]; cb[5 * HD] = xk;
-      float nq = warp_sum(yq * yq), nk = warp_sum(yk * yk), qk = warp_sum(yq * yk);
-      if (lane == 0) { sh_red[warp][0] = nq; sh_red[warp][1] = nk; sh_red[warp][2] = qk; }
+    if constexpr (kInputs) {
+      // input r (0..3: q, k, v, g of the token; 4 + 3 x + t: cache tensor x,
+      // time t) and the taps of tensor x, for channel c
+      auto input = [&](int r) -> Tin { return pf.row(sl, r)[c]; };
+      auto taps = [&](int x) -> float4 { return *reinterpret_cast<const float4*>(pf.taps(sl, x) + 4 * c); };
+      if (tid < D) {
+        const float4 wq = taps(0), wk = taps(1);
+        const Tin hq0 = input(4), hq1 = input(5), hq2 = input(6);
+        const Tin hk0 = input(7), hk1 = input(8), hk2 = input(9);
+        const Tin xq = input(0), xk = input(1);
+        yq = conv4(wq, to_f(hq0), to_f(hq1), to_f(hq2), to_f(xq));
+        yk = conv4(wk, to_f(hk0), to_f(hk1), to_f(hk2), to_f(xk));
+        if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
+        // the shifted cache (its old contents were read from the prefetched copy)
+        cb[0 * HD] = hq1; cb[1 * HD] = hq2; cb[2 * HD] = xq;
+        cb[3 * HD] = hk1; cb[4 * HD] = hk2; cb[5 * HD] = xk;
+        float nq = warp_sum(yq * yq), nk = warp_sum(yk * yk), qk = warp_sum(yq * yk);
+        if (lane == 0) { sh_red[warp][0] = nq; sh_red[warp][1] = nk; sh_red[warp][2] = qk; }
+      } else {
+        const float4 wv = taps(2);
+        const Tin hv0 = input(10), hv1 = input(11), hv2 = input(12);
+        const Tin xv = input(2);
+        float yv = conv4(wv, to_f(hv0), to_f(hv1), to_f(hv2), to_f(xv));
+        if (ACT == KDA_CONV_SILU) yv = silu(yv);
+        cb[6 * HD] = hv1; cb[7 * HD] = hv2; cb[8 * HD] = xv;
+        sh_v[c] = yv;
+        sh_al[rpad(c)] = __expf(fmaxf(to_f(input(3)), LOG_DECAY_FLOOR));
+      }
     } else {
-      const float4 wv = load4(conv_w + (2 * HD + ch) * 4);
-      const float v0 = to_f(cb[6 * HD]), v1 = to_f(cb[7 * HD]), v2 = to_f(cb[8 * HD]);
-      const Tin xv = v[tok];
-      float yv = conv4(wv, v0, v1, v2, to_f(xv));
-      if (ACT == KDA_CONV_SILU) yv = silu(yv);
-      cb[6 * HD] = cb[7 * HD]; cb[7 * HD] = cb[8 * HD]; cb[8 * HD] = xv;
-      sh_v[c] = yv;
-      sh_al[rpad(c)] = __expf(fmaxf(to_f(g[tok]), LOG_DECAY_FLOOR));
+      const int64_t tok = (int64_t)n * HD + ch;  // [N, H, D] index
+      if (tid < D) {
+        const float4 wq = load4(conv_w + (0 * HD + ch) * 4);
+        const float4 wk = load4(conv_w + (1 * HD + ch) * 4);
+        const float q0 = to_f(cb[0 * HD]), q1 = to_f(cb[1 * HD]), q2 = to_f(cb[2 * HD]);
+        const float k0 = to_f(cb[3 * HD]), k1 = to_f(cb[4 * HD]), k2 = to_f(cb[5 * HD]);
+        const Tin xq = q[tok], xk = k[tok];
+        yq = conv4(wq, q0, q1, q2, to_f(xq));
+        yk = conv4(wk, k0, k1, k2, to_f(xk));
+        if (ACT == KDA_CONV_SILU) { yq = silu(yq); yk = silu(yk); }
+        // shift the cache (all reads of this channel's history are done above)
+        cb[0 * HD] = cb[1 * HD]; cb[1 * HD] = cb[2 * HD]; cb[2 * HD] = xq;
+        cb[3 * HD] = cb[4 * HD]; cb[4 * HD] = cb[5 * HD]; cb[5 * HD] = xk;
+        float nq = warp_sum(yq * yq), nk = warp_sum(yk * yk), qk = warp_sum(yq * yk);
+        if (lane == 0) { sh_red[warp][0] = nq; sh_red[warp][1] = nk; sh_red[warp][2] = qk; }
+      } else {
+        const float4 wv = load4(conv_w + (2 * HD + ch) * 4);
+        const float v0 = to_f(cb[6 * HD]), v1 = to_f(cb[7 * HD]), v2 = to_f(cb[8 * HD]);
+        const Tin xv = v[tok];
+        float yv = conv4(wv, v0, v1, v2, to_f(xv));
+        if (ACT == KDA_CONV_SILU) yv = silu(yv);
+        cb[6 * HD] = cb[7 * HD]; cb[7 * HD] = cb[8 * HD]; cb[8 * HD] = xv;
+        sh_v[c] = yv;
+        sh_al[rpad(c)] = __expf(fmaxf(to_f(g[tok]), LOG_DECAY_FLOOR));
+      }
     }
     __syncthreads();
     const float nq = sh_red[0][0] + sh_red[1][0] + sh_red[2][0] + sh_red[3][0];
@@ -239,8 +364,10 @@ decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __rest
     //    the lane's 4 columns (lanes of row group 0 write o)
     float4 r, y;
     cols_dot2(s, sh_ka, sh_qa, L.rg, r, y);
-    const float4 u4 = delta_u(to_f(beta[(int64_t)n * H + h]), *reinterpret_cast<const float4*>(&sh_v[L.c0]), r);
+    const float b = kInputs ? b_cur : to_f(beta[(int64_t)n * H + h]);
+    const float4 u4 = delta_u(b, *reinterpret_cast<const float4*>(&sh_v[L.c0]), r);
     if (L.rg == 0) store4(o + (int64_t)n * HD + (int64_t)h * D + L.c0, readout_o(y, u4, kq));
+    b_cur = b_next;
 
     // 4. S <- Diag(a) S + k u^T, written once.  The shared vectors are
     //    rewritten by the next item only after its first barrier, which every
