@@ -113,6 +113,14 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_he
  *                      (may be NULL when that size is 0).
  * Returns KDA_OK once all work is enqueued.  bf16 inputs run the chunked
  * tensor-core path; fp32 inputs run the fp32 recurrent path.
+ *
+ * Scheduling of the chunked path: when N * H <= 96 (one long sequence, say),
+ * its two kernels overlap.  The second runs on a library-owned stream of the
+ * current device that is forked from `stream` after the workspace is set up
+ * and joined back to it with events before the call's last launch, so all work
+ * is still ordered on `stream` as seen from the caller (CUDA-graph capture of
+ * `stream` records the fork and join).  Calls from several host threads at
+ * once share that stream: correct, but their second kernels serialise.
  */
 kda_status kda_prefill(const void* q, const void* k, const void* v, const void* g,
                        const void* beta, const float* conv_w, const void* init_state,
