@@ -332,6 +332,23 @@ const char* kda_status_string(kda_status s);
  */
 kda_status kda_check_async_status(void* stream);
 
+/*
+ * Host-side fault injection, for tests of the failure path only.
+ *   KDA_FAULT_DROP_READY : the next kda_prefill / kda_prefill_noalloc call
+ *       that takes the overlapped chunked mode (at most 96 (sequence, head)
+ *       pairs) launches its preparation kernel without the per-chunk ready
+ *       flags, so the flags the scan waits on are never published.  The scan's
+ *       bounded wait gives up (about 2 s), every block drains its own copies
+ *       and tensor-core work, frees its tensor memory and returns; the call's
+ *       outputs are invalid and kda_check_async_status reports
+ *       KDA_ERR_TIMEOUT.  The context stays usable.
+ *   KDA_FAULT_NONE       : clears a pending fault.
+ * A fault is pending until one call applies it (one-shot); process-wide.
+ * Errors: KDA_ERR_INVALID_ARG for an unknown kind.  Pure host function.
+ */
+typedef enum { KDA_FAULT_NONE = 0, KDA_FAULT_DROP_READY = 1 } kda_fault;
+kda_status kda_inject_fault(kda_fault kind);
+
 /* Library ABI version: (major << 16) | minor. */
 int kda_version(void);
 

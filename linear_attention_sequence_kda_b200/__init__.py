@@ -28,7 +28,7 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
            "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version",
            "kda_prefill_noalloc", "kda_decode_deltas_size", "kda_decode_verify", "kda_decode_commit",
-           "kda_decode_commit_verify", "kda_state_affine")
+           "kda_decode_commit_verify", "kda_state_affine", "kda_inject_fault")
 MAX_VERIFY_ROWS = 8  # KDA_MAX_VERIFY_ROWS
 
 if not os.path.exists(LIB_PATH):
@@ -72,6 +72,9 @@ lib.kda_status_string.argtypes = [ctypes.c_int]
 lib.kda_check_async_status.restype = ctypes.c_int
 lib.kda_check_async_status.argtypes = [_vp]
 lib.kda_version.restype = ctypes.c_int
+lib.kda_inject_fault.restype = ctypes.c_int
+lib.kda_inject_fault.argtypes = [ctypes.c_int]
+KDA_FAULT_NONE, KDA_FAULT_DROP_READY = 0, 1
 
 
 class KdaError(RuntimeError):
@@ -260,3 +263,9 @@ def state_affine(A, S_in, B, S_out=None, stream=None):
 
 def check_async_status(stream=None) -> int:
     return int(lib.kda_check_async_status(_stream(stream)))
+
+
+def inject_fault(kind: int) -> None:
+    """Test hook: arm a host-side fault for the next call that can apply it
+    (KDA_FAULT_DROP_READY) or clear a pending one (KDA_FAULT_NONE)."""
+    _check(lib.kda_inject_fault(int(kind)), "kda_inject_fault")

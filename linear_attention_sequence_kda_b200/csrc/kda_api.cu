@@ -397,7 +397,13 @@ kda_status kda_check_async_status(void* stream) {
   return (kda_status)v;
 }
 
-int kda_version(void) { return (2 << 16) | 0; }
+kda_status kda_inject_fault(kda_fault kind) {
+  if (kind != KDA_FAULT_NONE && kind != KDA_FAULT_DROP_READY) return KDA_ERR_INVALID_ARG;
+  kda::pending_fault().store(kind);
+  return KDA_OK;
+}
+
+int kda_version(void) { return (2 << 16) | 1; }
 
 }  // extern "C"
 

@@ -16,6 +16,7 @@
 // other on the caller's stream.
 #pragma once
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <numeric>
 #include <vector>
@@ -49,6 +50,17 @@ constexpr int OVERLAP_MAX_CHAINS = 96;  // leaves at least 52 of 148 SMs to prep
 // gave the shortest overlapped call on B200, 64 heads x 65,536 tokens, among
 // 2.8 .. 4.4; the model value from the two kernels' separate timings is ~3).
 constexpr double PREP_PER_SCAN_CHUNK = 2.8;
+
+// Pending host-side fault (kda_inject_fault), taken by the first call that
+// applies it.
+inline std::atomic<int>& pending_fault() {
+  static std::atomic<int> fault{KDA_FAULT_NONE};
+  return fault;
+}
+inline bool take_fault(kda_fault kind) {
+  int expected = kind;
+  return pending_fault().compare_exchange_strong(expected, KDA_FAULT_NONE);
+}
 
 // Side stream and fork / join events of the overlapped mode, one set per
 // device, created on first use.
@@ -153,9 +165,12 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
       vacate_sms = chains;
       vacate_after = (int)(f * (double)items);
     }
+    // an injected KDA_FAULT_DROP_READY drops the publication of the flags the
+    // scan waits on
+    int* publish = overlap && !take_fault(KDA_FAULT_DROP_READY) ? ready : nullptr;
     prep<<<blocks, PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w, (const T*)init_conv,
                                                         cu_dev, d_tab, H, (int)items, records, work_counter,
-                                                        overlap ? ready : nullptr, vacate_sms, vacate_after);
+                                                        publish, vacate_sms, vacate_after);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
   }
   // the scan, instantiated for the output and state element types

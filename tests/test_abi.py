@@ -43,6 +43,15 @@ def test_version_and_status_strings():
     assert kda.lib.kda_status_string(99).decode() == "unknown status"
 
 
+def test_inject_fault_host_validation():
+    """Arming and clearing the host-side fault is pure host work; an unknown
+    kind is rejected."""
+    assert kda.lib.kda_inject_fault(7) == 1
+    assert kda.lib.kda_inject_fault(-1) == 1
+    assert kda.lib.kda_inject_fault(kda.KDA_FAULT_DROP_READY) == 0
+    assert kda.lib.kda_inject_fault(kda.KDA_FAULT_NONE) == 0
+
+
 def test_workspace_size_invalid_is_zero():
     assert kda.lib.kda_prefill_workspace_size(-1, 10, 4, 10, 1) == 0
     assert kda.lib.kda_prefill_workspace_size(1, 10, 0, 10, 1) == 0
