@@ -338,7 +338,7 @@ kda_status kda_check_async_status(void* stream);
  *       that takes the overlapped chunked mode (at most 96 (sequence, head)
  *       pairs) launches its preparation kernel without the per-chunk ready
  *       flags, so the flags the scan waits on are never published.  The scan's
- *       bounded wait gives up (about 2 s), every block drains its own copies
+ *       bounded waits give up (well under 2 s), every block drains its own copies
  *       and tensor-core work, frees its tensor memory and returns; the call's
  *       outputs are invalid and kda_check_async_status reports
  *       KDA_ERR_TIMEOUT.  The context stays usable.

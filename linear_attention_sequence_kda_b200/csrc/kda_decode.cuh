@@ -109,9 +109,37 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
   *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
 }
 
+// Shared-memory image of a prefetched state: its 8 row groups (16 rows each,
+// StateLane::rg) as separate pieces.  One load instruction of a warp reads the
+// same 4 columns of 8 rows 16 apart; with a 256-byte row pitch (bf16) those
+// rows all start on the same bank, so a bf16 state's pieces are placed 32
+// bytes further apart than their size, which spreads the 8 rows over all 32
+// banks.  An fp32 state is kept as one unpadded piece.
+template <typename Ts>
+struct StateImage {
+  static constexpr uint32_t kGroup = 16 * D * sizeof(Ts);  // bytes of one row group
+  static constexpr uint32_t kPitch = kGroup + (sizeof(Ts) == 2 ? 32 : 0);
+  static constexpr uint32_t kBytes = 8 * kPitch;           // shared memory taken
+  static constexpr uint32_t kCopied = 8 * kGroup;          // bytes a copy transfers
+  // one thread: the state at `src` into the image at `dst` (16-byte aligned),
+  // completing on `bar`
+  static __device__ __forceinline__ void copy(uint8_t* dst, const Ts* src, uint64_t* bar) {
+    if constexpr (kPitch == kGroup) {
+      tc::bulk_g2s(dst, src, kCopied, bar);
+    } else {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) tc::bulk_g2s(dst + r * kPitch, src + r * 16 * D, kGroup, bar);
+    }
+  }
+  // row 16 rg + i, columns c0 .. c0 + 3 of the lane
+  static __device__ __forceinline__ float4 load(const uint8_t* img, StateLane L, int i) {
+    return ld_state4_shared(reinterpret_cast<const Ts*>(img + L.rg * kPitch) + i * D + L.c0);
+  }
+};
+
 // Bytes of dynamic shared memory the persistent decode kernels need (the
 // prefetched state).
-template <typename Ts> __host__ __device__ constexpr uint32_t decode_smem_bytes() { return (uint32_t)(D * D * sizeof(Ts)); }
+template <typename Ts> __host__ __device__ constexpr uint32_t decode_smem_bytes() { return StateImage<Ts>::kBytes; }
 
 // State prefetch of the persistent decode kernels (256 threads, items visited
 // as blockIdx.x, + gridDim.x, ...): while a block computes one (sequence, head)
@@ -120,7 +148,7 @@ template <typename Ts> __host__ __device__ constexpr uint32_t decode_smem_bytes(
 // (it contains a barrier); take() by all threads at the top of each item.
 template <typename Ts>
 struct StatePrefetch {
-  Ts* buf;
+  uint8_t* buf;
   const Ts* state;
   uint64_t* bar;
   int items;
@@ -128,13 +156,13 @@ struct StatePrefetch {
 
   __device__ __forceinline__ void issue(int item) {  // one thread
     tc::fence_async_smem();  // the buffer's previous contents were read by every thread
-    tc::bar_expect_tx(bar, decode_smem_bytes<Ts>());
-    tc::bulk_g2s(buf, state + (int64_t)item * D * D, decode_smem_bytes<Ts>(), bar);
+    tc::bar_expect_tx(bar, StateImage<Ts>::kCopied);
+    StateImage<Ts>::copy(buf, state + (int64_t)item * D * D, bar);
   }
   __device__ __forceinline__ void init(const Ts* st, int n_items) {
     extern __shared__ __align__(128) uint8_t dsm[];
     __shared__ uint64_t bar_state;
-    buf = reinterpret_cast<Ts*>(dsm);
+    buf = dsm;
     state = st;
     bar = &bar_state;
     items = n_items;
@@ -159,7 +187,7 @@ struct StatePrefetch {
     }
     par ^= 1;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s[i] = ld_state4_shared(buf + state_off(L, i));
+    for (int i = 0; i < 16; ++i) s[i] = StateImage<Ts>::load(buf, L, i);
     __syncthreads();
     if (threadIdx.x == 0 && item + (int)gridDim.x < items) issue(item + gridDim.x);
     return true;
@@ -175,14 +203,13 @@ struct StatePrefetch {
 // alone keeps HBM busy and the prologue reads global memory.
 template <typename Tin, typename Ts, bool INPUTS>
 struct DecodePrefetch {
-  static constexpr uint32_t kState = D * D * sizeof(Ts);
+  static constexpr uint32_t kState = StateImage<Ts>::kBytes;  // the state image, then the input slots
   static constexpr uint32_t kRow = D * sizeof(Tin);
   static constexpr uint32_t kTaps = D * 4 * sizeof(float);   // one tensor's taps
   static constexpr uint32_t kSlot = INPUTS ? (13 * kRow + 3 * kTaps + 127) & ~127u : 0;
   __host__ __device__ static constexpr uint32_t bytes() { return kState + 2 * kSlot; }
 
   uint8_t* base;
-  Ts* sbuf;
   const Ts* state;
   const Tin *q, *k, *v, *g, *cache;
   const float* conv_w;
@@ -202,8 +229,9 @@ struct DecodePrefetch {
     const int64_t n = item / H, h = item % H, HD = (int64_t)H * D;
     uint8_t* dst = base + kState + sl * kSlot;
     tc::fence_async_smem();  // the buffers' previous contents were read by every thread
-    tc::bar_expect_tx(bar, INPUTS ? kState + 13 * kRow + 3 * kTaps : kState);
-    tc::bulk_g2s(sbuf, state + (int64_t)item * D * D, kState, bar);
+    constexpr uint32_t kCopied = StateImage<Ts>::kCopied;
+    tc::bar_expect_tx(bar, INPUTS ? kCopied + 13 * kRow + 3 * kTaps : kCopied);
+    StateImage<Ts>::copy(base, state + (int64_t)item * D * D, bar);
     if (!INPUTS) return;
     const Tin* in[4] = {q, k, v, g};
 #pragma unroll
@@ -219,7 +247,6 @@ struct DecodePrefetch {
     extern __shared__ __align__(128) uint8_t dsm[];
     __shared__ uint64_t bar_pf;
     base = dsm;
-    sbuf = reinterpret_cast<Ts*>(dsm);
     state = st; q = q_; k = k_; v = v_; g = g_; cache = cache_; conv_w = w_;
     bar = &bar_pf;
     items = n_items;
@@ -244,7 +271,7 @@ struct DecodePrefetch {
     }
     par ^= 1;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) s[i] = ld_state4_shared(sbuf + state_off(L, i));
+    for (int i = 0; i < 16; ++i) s[i] = StateImage<Ts>::load(base, L, i);
     *cur = slot;
     slot ^= 1;
     __syncthreads();

@@ -43,7 +43,7 @@ def test_dropped_ready_flags_time_out_and_context_recovers():
     finally:
         kda.inject_fault(kda.KDA_FAULT_NONE)
     assert status == 6, kda.STATUS.get(status, status)  # KDA_ERR_TIMEOUT
-    assert elapsed < 60.0  # bounded: about two seconds of waiting
+    assert elapsed < 60.0  # bounded: the scan's waits give up well within two seconds
     assert kda.check_async_status() == 0  # the status word was read and cleared
     # the fault was taken by the call that applied it: the next call is whole
     for _ in range(2):
