@@ -340,10 +340,9 @@ kda_status kda_decode_commit(void* state, void* conv_cache, const void* q, const
     by_type(state_dt, [&](auto ts) {
       using Tin = decltype(tin);
       using Ts = decltype(ts);
-      rc = launch_persistent(decode_commit_kernel<Tin, Ts>, decode_smem_bytes<Ts>(), (int64_t)num_seqs * num_heads, s,
-                             (Ts*)state,
-                                 (Tin*)conv_cache, (const Tin*)q, (const Tin*)k, (const Tin*)v, deltas, n_accept,
-                                 num_seqs, num_rows, num_heads);
+      rc = launch_persistent(decode_commit_kernel<Tin, Ts>, CommitPrefetch<Ts>::bytes(num_rows),
+                             (int64_t)num_seqs * num_heads, s, (Ts*)state, (Tin*)conv_cache, (const Tin*)q,
+                             (const Tin*)k, (const Tin*)v, deltas, n_accept, num_seqs, num_rows, num_heads);
     });
   });
   return rc;

@@ -137,63 +137,6 @@ struct StateImage {
   }
 };
 
-// Bytes of dynamic shared memory the persistent decode kernels need (the
-// prefetched state).
-template <typename Ts> __host__ __device__ constexpr uint32_t decode_smem_bytes() { return StateImage<Ts>::kBytes; }
-
-// State prefetch of the persistent decode kernels (256 threads, items visited
-// as blockIdx.x, + gridDim.x, ...): while a block computes one (sequence, head)
-// item, one bulk copy brings the next item's state into the dynamic shared
-// memory buffer.  init() is called once by all threads before the item loop
-// (it contains a barrier); take() by all threads at the top of each item.
-template <typename Ts>
-struct StatePrefetch {
-  uint8_t* buf;
-  const Ts* state;
-  uint64_t* bar;
-  int items;
-  uint32_t par;
-
-  __device__ __forceinline__ void issue(int item) {  // one thread
-    tc::fence_async_smem();  // the buffer's previous contents were read by every thread
-    tc::bar_expect_tx(bar, StateImage<Ts>::kCopied);
-    StateImage<Ts>::copy(buf, state + (int64_t)item * D * D, bar);
-  }
-  __device__ __forceinline__ void init(const Ts* st, int n_items) {
-    extern __shared__ __align__(128) uint8_t dsm[];
-    __shared__ uint64_t bar_state;
-    buf = dsm;
-    state = st;
-    bar = &bar_state;
-    items = n_items;
-    par = 0;
-    if (threadIdx.x == 0) {
-      tc::bar_init(bar, 1);
-      tc::bar_init_fence();
-      if ((int)blockIdx.x < items) issue(blockIdx.x);
-    }
-    __syncthreads();
-  }
-  // This item's state into registers (the StateLane layout), then the next
-  // item's copy is issued.  Returns false
-  // for the whole block if the copy did not land in time (recorded as
-  // KDA_ERR_TIMEOUT; the copy in flight is awaited once more before the block
-  // gives up, so nothing lands in shared memory after it exits).
-  __device__ __forceinline__ bool take(int item, float4 (&s)[16]) {
-    const StateLane L = state_lane();
-    if (!__syncthreads_and(tc::bar_wait(bar, par))) {
-      if (threadIdx.x == 0) tc::bar_wait(bar, par);
-      return false;
-    }
-    par ^= 1;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) s[i] = StateImage<Ts>::load(buf, L, i);
-    __syncthreads();
-    if (threadIdx.x == 0 && item + (int)gridDim.x < items) issue(item + gridDim.x);
-    return true;
-  }
-};
-
 // The prefetch of decode_kernel.  With a bf16 state (INPUTS = true) the inputs
 // of the next item's prologue (the q, k, v, g rows, the nine conv-cache rows,
 // the three tap rows) arrive by bulk copies on the same mbarrier as its state,
@@ -260,9 +203,13 @@ struct DecodePrefetch {
     }
     __syncthreads();
   }
-  // This item's state into registers; *cur = the slot holding its inputs;
-  // then the next item's copies are issued into the other slot.  Bounded as
-  // StatePrefetch::take.
+  // Called by all threads at the top of each item (init() once before the
+  // item loop; both contain a barrier).  This item's state into registers
+  // (the StateLane layout); *cur = the slot holding its inputs; then the next
+  // item's copies are issued into the other slot.  Returns false for the
+  // whole block if the copies did not land in time (recorded as
+  // KDA_ERR_TIMEOUT; the copies in flight are awaited once more before the
+  // block gives up, so nothing lands in shared memory after it exits).
   __device__ __forceinline__ bool take(int item, float4 (&s)[16], uint32_t* cur) {
     const StateLane L = state_lane();
     if (!__syncthreads_and(tc::bar_wait(bar, par))) {

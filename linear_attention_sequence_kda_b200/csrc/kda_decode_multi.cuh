@@ -20,6 +20,8 @@
 // for the first n_accept rows (one read and one write of S), and the conv
 // cache becomes the last three raw tokens of [cache, accepted rows].
 #pragma once
+#include <type_traits>
+
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
 
@@ -212,6 +214,70 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
   }
 }
 
+// The prefetch of decode_commit_kernel: the next item's state (StateImage) and
+// its R rows of deltas ([R][3][D] fp32, one bulk copy) arrive on one mbarrier,
+// the deltas into one of two slots, so that neither waits for global memory
+// while an item is committed.  All R rows are copied, whatever the item keeps.
+template <typename Ts>
+struct CommitPrefetch {
+  static constexpr uint32_t kState = StateImage<Ts>::kBytes;
+  __host__ __device__ static constexpr uint32_t slot_bytes(int R) { return (uint32_t)R * 3 * D * sizeof(float); }
+  __host__ __device__ static constexpr uint32_t bytes(int R) { return kState + 2 * slot_bytes(R); }
+
+  uint8_t* base;
+  const Ts* state;
+  const float* deltas;
+  uint64_t* bar;
+  int items, R;
+  uint32_t par, slot;
+
+  __device__ __forceinline__ const float* rows(uint32_t sl) const {
+    return reinterpret_cast<const float*>(base + kState + sl * slot_bytes(R));
+  }
+  __device__ __forceinline__ void issue(int item, uint32_t sl) {  // one thread
+    tc::fence_async_smem();  // the buffers' previous contents were read by every thread
+    tc::bar_expect_tx(bar, StateImage<Ts>::kCopied + slot_bytes(R));
+    StateImage<Ts>::copy(base, state + (int64_t)item * D * D, bar);
+    tc::bulk_g2s(base + kState + sl * slot_bytes(R), deltas + (int64_t)item * R * 3 * D, slot_bytes(R), bar);
+  }
+  __device__ __forceinline__ void init(const Ts* st, const float* dl, int n_items, int R_) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ uint64_t bar_cp;
+    base = dsm;
+    state = st;
+    deltas = dl;
+    bar = &bar_cp;
+    items = n_items;
+    R = R_;
+    par = 0;
+    slot = 0;
+    if (threadIdx.x == 0) {
+      tc::bar_init(bar, 1);
+      tc::bar_init_fence();
+      if ((int)blockIdx.x < items) issue(blockIdx.x, 0);
+    }
+    __syncthreads();
+  }
+  // This item's state into registers; *cur = the slot holding its deltas; then
+  // the next item's copies are issued into the other slot.  Bounded as
+  // DecodePrefetch::take.
+  __device__ __forceinline__ bool take(int item, float4 (&s)[16], uint32_t* cur) {
+    const StateLane L = state_lane();
+    if (!__syncthreads_and(tc::bar_wait(bar, par))) {
+      if (threadIdx.x == 0) tc::bar_wait(bar, par);
+      return false;
+    }
+    par ^= 1;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) s[i] = StateImage<Ts>::load(base, L, i);
+    *cur = slot;
+    slot ^= 1;
+    __syncthreads();
+    if (threadIdx.x == 0 && item + (int)gridDim.x < items) issue(item + gridDim.x, slot);
+    return true;
+  }
+};
+
 template <typename Tin, typename Ts>
 __global__ void __launch_bounds__(256, 2)
 decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __restrict__ q,
@@ -220,43 +286,56 @@ decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin*
   // row vectors k_hat, alpha padded (rpad); u a column vector
   __shared__ __align__(16) float sh_kh[MAX_VERIFY_ROWS][ROWV], sh_u[MAX_VERIFY_ROWS][D],
       sh_al[MAX_VERIFY_ROWS][ROWV];
-  StatePrefetch<Ts> pf;
-  pf.init(state, N * H);
+  // new conv-cache rows [3][3 x 128] (each thread its own channel pairs)
+  __shared__ __align__(16) uint8_t sh_cc_raw[3 * 3 * D * sizeof(Tin)];
+  auto sh_cc = reinterpret_cast<Tin(*)[3 * D]>(sh_cc_raw);
+  CommitPrefetch<Ts> pf;
+  pf.init(state, deltas, N * H, R);
+  const int tid = threadIdx.x;
+  const StateLane L = state_lane();
+  const int64_t HD = (int64_t)H * D;
+  // n_accept of the item being committed, loaded one item ahead
+  int na_next = (int)blockIdx.x < pf.items ? n_accept[blockIdx.x / H] : 0;
 
   // persistent loop over the (sequence, head) items
   for (int item = blockIdx.x; item < pf.items; item += gridDim.x) {
-  const int n = item / H, h = item % H, tid = threadIdx.x;
-  const StateLane L = state_lane();
-  const int64_t HD = (int64_t)H * D;
+  const int n = item / H, h = item % H;
   Ts* S = state + (int64_t)item * D * D;
   float4 s[16];
-  if (!pf.take(item, s)) return;
-  int na = n_accept[n];
+  uint32_t sl;
+  if (!pf.take(item, s, &sl)) return;
+  int na = na_next;
+  na_next = item + (int)gridDim.x < pf.items ? n_accept[(item + gridDim.x) / H] : 0;
   if (na < 0 || na > R) {  // out of range: record it and keep what can be kept
     if (tid == 0 && h == 0) set_status(KDA_ERR_INVALID_ARG);
     na = na < 0 ? 0 : R;
   }
   if (na == 0) continue;  // nothing accepted: state and cache stay as they are
-  const float* dl = deltas + ((int64_t)n * H + h) * R * 3 * D;
+  // conv cache: the last three raw tokens of [cache (3 rows), accepted rows].
+  // Thread tid < 192 takes the channel pair (x, cc .. cc + 1) of the 3 x 128
+  // (tensor, channel) columns: its three values are copied asynchronously into
+  // its own shared slots now and stored back after the state update, so the
+  // loads' latency is hidden and no registers are held across the update.
+  const bool cache_thread = tid < 3 * D / 2;
+  const int cx = tid / (D / 2), ccp = 2 * (tid % (D / 2));
+  if (cache_thread) {
+    const Tin* cb = cache + ((int64_t)n * 9 + 3 * cx) * HD + (int64_t)h * D + ccp;
+    const Tin* src = cx == 0 ? q : (cx == 1 ? k : v);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int idx = na + j;  // position in [cache rows 0..2, accepted rows]
+      const Tin* from = idx < 3 ? cb + idx * HD : src + (((int64_t)n * R + (idx - 3)) * H + h) * D + ccp;
+      tc::async_copy<2 * sizeof(Tin)>(&sh_cc[j][cx * D + ccp], from);
+    }
+    tc::async_commit();
+  }
+  // the kept rows' deltas from the prefetched slot into the padded row vectors
+  const float* dl = pf.rows(sl);
   for (int e = tid; e < na * D; e += 256) {
     const int t = e / D, cc = e % D;
     sh_kh[t][rpad(cc)] = dl[(t * 3 + 0) * D + cc];
     sh_u[t][cc] = dl[(t * 3 + 1) * D + cc];
     sh_al[t][rpad(cc)] = dl[(t * 3 + 2) * D + cc];
-  }
-  // conv cache: the last three raw tokens of [cache (3 rows), accepted rows];
-  // all three are read before any is written (the cache is updated in place)
-  for (int e = tid; e < 3 * D; e += 256) {
-    const int x = e / D, cc = e % D;  // tensor (q, k, v), channel
-    const int64_t ch = (int64_t)h * D + cc;
-    Tin* cb = cache + ((int64_t)n * 9 + 3 * x) * HD + ch;
-    const Tin* src = x == 0 ? q : (x == 1 ? k : v);
-    Tin nv[3];
-    for (int j = 0; j < 3; ++j) {
-      const int idx = na + j;  // position in [cache rows 0..2, accepted rows]
-      nv[j] = idx < 3 ? cb[idx * HD] : src[(((int64_t)n * R + (idx - 3)) * H + h) * D + cc];
-    }
-    for (int j = 0; j < 3; ++j) cb[j * HD] = nv[j];
   }
   __syncthreads();
   for (int t = 0; t < na; ++t) {
@@ -268,6 +347,14 @@ decode_commit_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin*
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) st_state4(S + state_off(L, i), s[i]);
+  if (cache_thread) {  // the thread's own copies: no barrier needed
+    tc::async_wait_all();
+    Tin* cb = cache + ((int64_t)(item / H) * 9 + 3 * cx) * HD + (int64_t)(item % H) * D + ccp;
+    using Pair = typename std::conditional<sizeof(Tin) == 2, uint32_t, uint2>::type;
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+      *reinterpret_cast<Pair*>(cb + j * HD) = *reinterpret_cast<const Pair*>(&sh_cc[j][cx * D + ccp]);
+  }
   }  // item loop
 }
 

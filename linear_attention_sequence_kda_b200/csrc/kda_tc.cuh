@@ -258,6 +258,17 @@ __device__ __forceinline__ void bulk_s2g(void* dst, const void* src_smem, uint32
                "r"(smem_u32(src_smem)), "r"(bytes)
                : "memory");
 }
+// Per-thread asynchronous copy global -> shared of 4 or 8 bytes (both
+// addresses aligned to the size); completion is awaited by the same thread
+// with async_wait_all.
+template <int BYTES>
+__device__ __forceinline__ void async_copy(void* dst_smem, const void* src) {
+  static_assert(BYTES == 4 || BYTES == 8, "cp.async.ca copies 4, 8 or 16 bytes");
+  asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_u32(dst_smem)), "l"(src), "n"(BYTES)
+               : "memory");
+}
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until every committed bulk store of this thread has finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
