@@ -48,12 +48,24 @@ __device__ __forceinline__ int rpad(int r) { return r + 4 * (r >> 4); }
 // identically.  Packed f32x2 instructions do two columns at a time; each
 // column is rounded as its scalar fmaf would round it.
 //
-// Column sums over all 128 rows: r = sum_row x_row s_row, y likewise with z
-// (x, z: padded row vectors).  Each lane sums its 16 rows (ascending), then
-// the 8 row groups combine by a butterfly over lanes (xor 4, 8, 16), which
-// leaves the same full sums in every lane of a column quad.
-__device__ __forceinline__ void cols_dot2(const float4 (&s)[16], const float* x, const float* z, int rg,
-                                          float4& r, float4& y) {
+// The column step of a row: the column sums r = sum_row x_row s_row and
+// y = sum_row z_row s_row over all 128 rows (x, z: padded row vectors), then
+// u = beta (v - r) and o = y + u kq.  Each lane sums its 16 rows (ascending);
+// the 8 row groups of a column quad then combine by recursive halving over
+// lanes xor 4, 8, 16: at each stage a lane adds its partner's value of the
+// half it keeps, so every sum is formed from the same pairs in the same order
+// as a full butterfly would form it, with 7 shuffles instead of 24.  This
+// leaves each of the quad's 8 sums (r and y of its 4 columns) in one lane: the
+// lane of row group rg holds sum number 4 (rg & 1) + 2 ((rg >> 1) & 1) +
+// (rg >> 2), an r for even rg and a y for odd rg.  u is formed where r is and
+// gathered into every lane of the quad; o is formed where y is.
+struct ColStep {
+  float4 u;  // u of the lane's 4 columns (every lane)
+  float o;   // o of column c0 + oc (lanes of odd row groups)
+  int oc;
+};
+__device__ __forceinline__ ColStep col_step(const float4 (&s)[16], const float* x, const float* z, int rg,
+                                            float beta, const float* vcols, float kq) {
   float2 r0 = make_float2(0.f, 0.f), r1 = r0, y0 = r0, y1 = r0;
 #pragma unroll
   for (int i4 = 0; i4 < 4; ++i4) {
@@ -68,13 +80,29 @@ __device__ __forceinline__ void cols_dot2(const float4 (&s)[16], const float* x,
     }
   }
   float v[8] = {r0.x, r0.y, r1.x, r1.y, y0.x, y0.y, y1.x, y1.y};
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int m = 4; m < 32; m <<= 1) {
+  for (int st = 0; st < 3; ++st) {
+    const int m = 4 << st, n = 4 >> st;  // partner lane xor m; values kept after this stage
+    const bool up = (lane & m) != 0;     // keeps the upper half
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] += __shfl_xor_sync(0xffffffffu, v[e], m);
+    for (int i = 0; i < n; ++i) {
+      const float send = up ? v[i] : v[i + n];
+      const float keep = up ? v[i + n] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+    }
   }
-  r = make_float4(v[0], v[1], v[2], v[3]);
-  y = make_float4(v[4], v[5], v[6], v[7]);
+  const int idx = 4 * (rg & 1) + 2 * ((rg >> 1) & 1) + (rg >> 2);  // the sum this lane holds
+  const float um = beta * (vcols[idx & 3] - v[0]);                 // meaningful for even rg
+  // u of column c0 + j sits in the lane of row group 0, 4, 2, 6 for j = 0 .. 3
+  const int q = lane & 3;
+  ColStep cs;
+  cs.u = make_float4(__shfl_sync(0xffffffffu, um, q), __shfl_sync(0xffffffffu, um, q + 16),
+                     __shfl_sync(0xffffffffu, um, q + 8), __shfl_sync(0xffffffffu, um, q + 24));
+  cs.oc = idx & 3;
+  const float uo = cs.oc == 0 ? cs.u.x : (cs.oc == 1 ? cs.u.y : (cs.oc == 2 ? cs.u.z : cs.u.w));
+  cs.o = v[0] + uo * kq;
+  return cs;
 }
 
 // s_row <- a_row s_row + kh_row u (the delta-rule update Diag(a) S + k u^T;
@@ -95,19 +123,8 @@ __device__ __forceinline__ void rows_update(float4 (&s)[16], const float* a, con
   }
 }
 
-// u = beta (v - r) and o = y + u kq for the lane's 4 columns (the expressions
-// of the single step, element by element).
-__device__ __forceinline__ float4 delta_u(float b, float4 v, float4 r) {
-  return make_float4(b * (v.x - r.x), b * (v.y - r.y), b * (v.z - r.z), b * (v.w - r.w));
-}
-__device__ __forceinline__ float4 readout_o(float4 y, float4 u, float kq) {
-  return make_float4(y.x + u.x * kq, y.y + u.y * kq, y.z + u.z * kq, y.w + u.w * kq);
-}
-// four consecutive outputs
-__device__ __forceinline__ void store4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
-__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
-  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-}
+// one output element
+template <typename T> __device__ __forceinline__ void store1(T* p, float v) { *p = from_f<T>(v); }
 
 // Shared-memory image of a prefetched state: its 8 row groups (16 rows each,
 // StateLane::rg) as separate pieces.  One load instruction of a warp reads the
@@ -336,17 +353,15 @@ decode_kernel(Ts* __restrict__ state, Tin* __restrict__ cache, const Tin* __rest
 
     // 3. column sums r = S^T (a k), y = S^T (a q) within each warp; u and o for
     //    the lane's 4 columns (lanes of row group 0 write o)
-    float4 r, y;
-    cols_dot2(s, sh_ka, sh_qa, L.rg, r, y);
     const float b = kInputs ? b_cur : to_f(beta[(int64_t)n * H + h]);
-    const float4 u4 = delta_u(b, *reinterpret_cast<const float4*>(&sh_v[L.c0]), r);
-    if (L.rg == 0) store4(o + (int64_t)n * HD + (int64_t)h * D + L.c0, readout_o(y, u4, kq));
+    const ColStep cs = col_step(s, sh_ka, sh_qa, L.rg, b, &sh_v[L.c0], kq);
+    if (L.rg & 1) store1(o + (int64_t)n * HD + (int64_t)h * D + L.c0 + cs.oc, cs.o);
     b_cur = b_next;
 
     // 4. S <- Diag(a) S + k u^T, written once.  The shared vectors are
     //    rewritten by the next item only after its first barrier, which every
     //    thread reaches after this update.
-    rows_update(s, sh_al, sh_kh, L.rg, u4);
+    rows_update(s, sh_al, sh_kh, L.rg, cs.u);
 #pragma unroll
     for (int i = 0; i < 16; ++i) st_state4(S + state_off(L, i), s[i]);
   }

@@ -198,15 +198,11 @@ decode_verify_kernel(Ts* __restrict__ state, Tin* __restrict__ cache,
   //    no block barrier: the row vectors were all written before the barrier
   //    above, and each warp only touches its own columns afterwards.
   for (int t = 0; t < R; ++t) {
-    float4 r, y;
-    cols_dot2(s, sh_ka[t], sh_qa[t], L.rg, r, y);
-    const float4 u4 = delta_u(sh_beta[t], *reinterpret_cast<const float4*>(&sh_v[t][L.c0]), r);
-    if (L.rg == 0) {
-      store4(o + (((int64_t)n * R + t) * H + h) * D + L.c0, readout_o(y, u4, sh_kq[t]));
-      *reinterpret_cast<float4*>(dl + (t * 3 + 1) * D + L.c0) = u4;
-    }
+    const ColStep cs = col_step(s, sh_ka[t], sh_qa[t], L.rg, sh_beta[t], &sh_v[t][L.c0], sh_kq[t]);
+    if (L.rg & 1) store1(o + (((int64_t)n * R + t) * H + h) * D + L.c0 + cs.oc, cs.o);
+    if (L.rg == 0) *reinterpret_cast<float4*>(dl + (t * 3 + 1) * D + L.c0) = cs.u;
     if (t + 1 < R) {
-      rows_update(s, sh_al[t], sh_kh[t], L.rg, u4);
+      rows_update(s, sh_al[t], sh_kh[t], L.rg, cs.u);
       // the next row starts from the state as a single step would have stored it
 #pragma unroll
       for (int i = 0; i < 16; ++i) s[i] = as_stored4<Ts>(s[i]);
