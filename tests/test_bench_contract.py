@@ -1,0 +1,70 @@
+"""The benchmark's contract on the host (no GPU): the algorithmic byte counts
+behind every roofline figure, written out term by term from what each step must
+move, and the JSON line of the reference arm (the fp64 oracle on host cores)."""
+import json
+import os
+import subprocess
+import sys
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+KIB = 1024
+
+
+def test_prefill_bytes_per_token_head():
+    # q, k, v, g rows in bf16 (4 x 256 B), beta in bf16, o in fp32 (512 B)
+    assert bench.BYTES_PER_TOKEN_HEAD == 4 * 256 + 2 + 512
+    assert bench.STATE_BYTES == 64 * KIB
+    # the long-context workload: 65,536 tokens x 64 heads, one final state per head
+    assert 65536 * 64 * bench.BYTES_PER_TOKEN_HEAD + 64 * bench.STATE_BYTES == 6_455_033_856
+
+
+def test_decode_bytes_per_pair():
+    rows_in = 4 * 256            # q, k, v, g of the token, bf16
+    o_out = 512                  # fp32
+    beta = 2
+    cache = 2 * 9 * 256          # 3 tensors x 3 tokens, read and written
+    assert bench.dec_bytes_per_pair(4) == 2 * 64 * KIB + rows_in + o_out + beta + cache == 137_218
+    assert bench.dec_bytes_per_pair(2) == 2 * 32 * KIB + rows_in + o_out + beta + cache == 71_682
+
+
+def test_mtp_bytes_per_pair():
+    per_row = 2 * 3 * 512 + 4 * 256 + 2 + 512  # deltas written and read back, q k v g, beta, o
+    cache = 3 * 9 * 256                         # read by verify and commit, written by commit
+    assert bench.MTP_ROWS == 6
+    assert bench.mtp_bytes_per_pair(4) == 3 * 64 * KIB + 6 * per_row + cache == 231_180
+    assert bench.mtp_bytes_per_pair(2) == 3 * 32 * KIB + 6 * per_row + cache == 132_876
+
+
+def _run(args, env_extra=None):
+    env = dict(os.environ, **(env_extra or {}))
+    return subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, capture_output=True, text=True,
+                          timeout=600, env=env)
+
+
+def test_reference_arm_json_line():
+    r = _run(["--impl", "reference", "--steps", "1", "--warmup", "0"], {"RANK": "0", "WORLD_SIZE": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    for key in ("metric", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config"):
+        assert key in line, key
+    assert line["value"] > 0 and line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["steps"] == 1 and line["warmup"] == 0 and line["n_gpus"] == 1
+    assert line["vs_baseline"] is None and line["data"] == "synthetic"
+    assert "workload" in line["config"]
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    r = _run(["--impl", "reference", "--steps", "1", "--warmup", "0"], {"RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
