@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -101,15 +102,69 @@ def recorded_traffic(kernel: str):
 
 
 class ClockSampler:
+    """SM clock and clock-event (throttle) reasons of one GPU, sampled while a
+    timed region runs: NVML polled every `period_s` from a background thread
+    (reads only), or, where NVML cannot be used, nvidia-smi's 200 ms loop.
+    `nvml` may be given a stand-in module (tests)."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, nvml=None, period_s: float = 0.01):
         self.idx = device_index
+        self.nvml = nvml
+        self.period = period_s
+        self.rows = []      # (sm MHz, max sm MHz, [active reasons])
         self.proc = None
+        self.thread = None
+        self.out = ""
+        self.source = None
+
+    def _start_nvml(self):
+        nv = self.nvml
+        if nv is None:
+            import pynvml as nv
+        nv.nvmlInit()
+        self.nvml = nv
+        try:  # the CUDA device's own GPU, whatever devices this process sees
+            h = nv.nvmlDeviceGetHandleByUUID("GPU-" + str(torch.cuda.get_device_properties(self.idx).uuid))
+        except Exception:
+            h = nv.nvmlDeviceGetHandleByIndex(self.idx)
+        max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        read_mask = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        bits = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+
+        def sample():
+            mhz, mask = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), int(read_mask(h))
+            self.rows.append((mhz, max_mhz, [name for name, b in bits if mask & b]))
+
+        sample()  # a first read here, so that an NVML that cannot sample falls back now
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.wait(self.period):
+                try:
+                    sample()
+                except Exception:
+                    return
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+        self.source = "nvml"
 
     def __enter__(self):
+        try:
+            self._start_nvml()
+            return self
+        except Exception:
+            self.thread = None
+            self.rows = []
+        self.source = "nvidia-smi"
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -120,7 +175,14 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=2)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
+            return
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -128,23 +190,25 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 self.out, _ = self.proc.communicate()
-
-    def summary(self):
-        rows = []
+        names = [name for name, _ in self.REASONS]
         for line in (self.out or "").splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                self.rows.append((float(parts[1]), float(parts[2]),
+                                  [names[i] for i, x in enumerate(parts[5:9]) if x.lower() == "active"]))
             except ValueError:
                 continue
+
+    def summary(self):
+        rows = list(self.rows)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, x in enumerate(r) if x.lower() == "active"})
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0,
+                    "source": self.source}
         return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": sorted({n for r in rows for n in r[2]}), "samples": len(rows),
+                "source": self.source}
 
 
 def dist_setup():

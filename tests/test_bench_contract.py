@@ -68,3 +68,63 @@ def test_reference_arm_other_ranks_do_no_work():
     r = _run(["--impl", "reference", "--steps", "1", "--warmup", "0"], {"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+class FakeNvml:
+    """Stand-in for the NVML binding: a fixed sequence of SM clocks and one
+    active clock-event reason (the power cap)."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+
+    def __init__(self, clocks=(1965, 1900, 1965, 1950)):
+        self.clocks, self.n, self.shut = clocks, 0, False
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlShutdown(self):
+        self.shut = True
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        raise RuntimeError("no such device")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("gpu", i)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        assert h == ("gpu", 0) and kind == self.NVML_CLOCK_SM
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.n += 1
+        return self.clocks[(self.n - 1) % len(self.clocks)]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.nvmlClocksEventReasonSwPowerCap
+
+
+def test_clock_sampler_polls_nvml_during_the_region():
+    import time as _time
+    fake = FakeNvml()
+    with bench.ClockSampler(0, nvml=fake, period_s=0.002) as clk:
+        _time.sleep(0.05)
+    s = clk.summary()
+    assert s["source"] == "nvml" and s["samples"] >= 5 and fake.shut
+    assert s["sm_max_mhz"] == 1965 and 1900 <= s["sm_mhz"] <= 1965
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_falls_back_when_nvml_fails():
+    class Broken(FakeNvml):
+        def nvmlInit(self):
+            raise RuntimeError("NVML library not found")
+
+    with bench.ClockSampler(0, nvml=Broken()) as clk:
+        pass
+    s = clk.summary()
+    assert s["source"] == "nvidia-smi"
+    if s["samples"] == 0:  # no nvidia-smi on this host
+        assert s["reasons"] == ["unavailable"]
