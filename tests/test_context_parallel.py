@@ -9,6 +9,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -83,14 +84,28 @@ def _worker(rank, world, port, bounds, result_path):
         dist.destroy_process_group()
 
 
-def test_two_segments_over_gloo_equal_the_whole_sequence(tmp_path):
-    """Segments of 150 and 130 tokens (partial chunks at both ends of the
-    boundary) with a nonzero initial state and conv history."""
+@pytest.mark.parametrize("bounds", [[0, 150, 280], [0, 70, 73, 230]])
+def test_segments_over_gloo_equal_the_whole_sequence(tmp_path, bounds):
+    """Two segments of 150 and 130 tokens (partial chunks at both ends of the
+    boundary); three segments whose middle one has the minimum of 3 tokens, so
+    that the last segment's conv history is that segment alone.  Nonzero
+    initial state and conv history."""
     path = str(tmp_path / "cp.txt")
-    mp.start_processes(_worker, args=(2, _free_port(), [0, 150, 280], path), nprocs=2, start_method="spawn",
+    world = len(bounds) - 1
+    mp.start_processes(_worker, args=(world, _free_port(), bounds, path), nprocs=world, start_method="spawn",
                        join=True)
     err_o, err_s, tail_ok = open(path).read().split()
     assert float(err_o) < 1e-9 and float(err_s) < 1e-9 and tail_ok == "1"
+
+
+def test_conv_halo_needs_three_tokens():
+    """A segment followed by another must hand over three raw tokens."""
+    from linear_attention_sequence_kda_b200.sharding import conv_halo
+    x = torch.zeros((2, 1, D))
+    with pytest.raises(ValueError):
+        conv_halo(x, x, x)
+    halo = conv_halo(*(torch.arange(3 * D, dtype=torch.float32).view(3, 1, D) + 1000 * i for i in range(3)))
+    assert halo.shape == (1, 3, 3, D) and halo[0, 2, 0, 0] == 2000 and halo[0, 0, 2, D - 1] == 3 * D - 1
 
 
 def test_compose_order():
