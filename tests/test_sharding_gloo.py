@@ -5,6 +5,8 @@ takes the max over ranks."""
 import os
 import socket
 
+from hypothesis import given, settings
+from hypothesis import strategies as st
 import numpy as np
 import pytest
 import torch
@@ -76,3 +78,21 @@ def test_sequence_sharding_over_two_gloo_ranks_matches_single_process(tmp_path):
     ok, slowest = open(path).read().split()
     assert ok == "1"
     assert float(slowest) == 2.0
+
+
+@given(st.lists(st.integers(0, 300), min_size=1, max_size=40), st.integers(1, 10))
+@settings(max_examples=200, deadline=None)
+def test_split_varlen_properties(lengths, world):
+    """Any batch (empty segments included) and any rank count: the blocks are
+    contiguous and cover every segment once, and block r ends at the first
+    segment boundary at or past (r + 1) / world of the tokens."""
+    cu = np.cumsum([0] + lengths)
+    blocks = split_varlen(cu, world)
+    assert len(blocks) == world and blocks[0][0] == 0 and blocks[-1][1] == len(lengths)
+    for (a, b), (c, d) in zip(blocks, blocks[1:]):
+        assert b == c and a <= b
+    total = int(cu[-1])
+    for r, (_, end) in enumerate(blocks[:-1]):
+        target = total * (r + 1) / world
+        assert cu[end] >= target
+        assert end == 0 or cu[end - 1] < target
