@@ -176,3 +176,21 @@ def test_state_affine_argument_validation():
     assert af(Aa, Ss, Bb, So, 4, 3, None) == 1          # state element type
     assert af(Aa, Ss, Bb, Aa, 4, 0, None) == 1          # output aliases A
     assert af(Aa + 4, Ss, Bb, So, 4, 0, None) == 3
+
+
+def test_binding_constants_match_the_header():
+    """The binding's copies of the header's constants and enum values."""
+    txt = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    defines = dict(re.findall(r"#define\s+(KDA_[A-Z_]+)\s+(\d+)\s*$", txt, flags=re.M))
+    assert int(defines["KDA_HEAD_DIM"]) == kda.HEAD_DIM
+    assert int(defines["KDA_CHUNK"]) == kda.CHUNK
+    assert int(defines["KDA_MAX_VERIFY_ROWS"]) == kda.MAX_VERIFY_ROWS
+    m = re.search(r"#define\s+KDA_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", txt)
+    assert m and int(m.group(1)) << int(m.group(2)) == kda.NOALLOC_SCRATCH_BYTES
+    enums = {name: int(v) for name, v in re.findall(r"\b(KDA_[A-Z0-9_]+)\s*=\s*(\d+)", txt)}
+    statuses = {k: v for k, v in enums.items() if k == "KDA_OK" or k.startswith("KDA_ERR_")}
+    assert {name: code for code, name in kda.STATUS.items()} == statuses
+    assert (enums["KDA_F32"], enums["KDA_BF16"]) == (kda.KDA_F32, kda.KDA_BF16)
+    assert (enums["KDA_CONV_NONE"], enums["KDA_CONV_SILU"]) == (kda.KDA_CONV_NONE, kda.KDA_CONV_SILU)
+    assert (enums["KDA_FAULT_NONE"], enums["KDA_FAULT_DROP_READY"]) == \
+        (kda.KDA_FAULT_NONE, kda.KDA_FAULT_DROP_READY)
