@@ -7,7 +7,9 @@ floor on 10 % of channels).  `value` is prefill tokens/s over the whole job
 (all ranks), timed on the device with CUDA events, inputs resident in HBM.
 The same line carries the decode-step state bandwidth (256 sequences x 64
 heads, 1 GiB of fp32 state read and written in place) with its own roofline,
-the end-to-end number through the C ABI with host buffers, the oracle's CPU
+the multi-token decode legs (verify + commit of 6 rows, and the fused
+commit + verify), the same decode legs with bf16 state storage, the
+end-to-end number through the C ABI with host buffers, the oracle's CPU
 throughput, and the SM clocks sampled during the timed region.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own
