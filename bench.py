@@ -213,6 +213,27 @@ class ClockSampler:
                 "source": self.source}
 
 
+def device_info(dev_index: int) -> dict:
+    """The GPU's name, its driver version and the CUDA runtime in use (reads
+    only; a field that cannot be read stays None)."""
+    info = {"name": None, "driver": None, "cuda_runtime": torch.version.cuda}
+    try:
+        info["name"] = torch.cuda.get_device_name(dev_index)
+    except Exception:
+        pass
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            v = pynvml.nvmlSystemGetDriverVersion()
+            info["driver"] = v.decode() if isinstance(v, bytes) else str(v)
+        finally:
+            pynvml.nvmlShutdown()
+    except Exception:
+        pass
+    return info
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -418,6 +439,7 @@ def main():
         "e2e": e2e,
         "gpu_launches": args.steps * PREFILL_LAUNCHES,
         "clocks": clk.summary(),
+        "device": device_info(local),
         "decode": dec_line,
         "mtp": mtp_line,
         "mtp_fused": fused_line,

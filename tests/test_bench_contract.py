@@ -6,6 +6,8 @@ import os
 import subprocess
 import sys
 
+import torch
+
 import bench
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -128,3 +130,10 @@ def test_clock_sampler_falls_back_when_nvml_fails():
     assert s["source"] == "nvidia-smi"
     if s["samples"] == 0:  # no nvidia-smi on this host
         assert s["reasons"] == ["unavailable"]
+
+
+def test_device_info_never_raises():
+    """Without a GPU (or NVML) every field it cannot read stays None."""
+    info = bench.device_info(0)
+    assert set(info) == {"name", "driver", "cuda_runtime"}
+    assert info["cuda_runtime"] == torch.version.cuda
