@@ -22,6 +22,9 @@ Parity status: the recurrence is pinned by closed forms and invariants in
 orthonormal keys, last-write recall at beta = 1, linearity, column
 permutation, conv impulse response, causality, varlen isolation, split and
 decode equivalence, chunked == recurrent, literal == expanded).
+``tests/test_oracle_mutants.py`` plants plausible mistakes in a copy of
+``kda_oracle.c`` (wrong sign, dropped term, wrong operand, transposed index,
+reversed order, wrong rounding) and checks that a pin catches each one.
 """
 from __future__ import annotations
 
