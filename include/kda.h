@@ -118,9 +118,13 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_he
  * its two kernels overlap.  The second runs on a library-owned stream of the
  * current device that is forked from `stream` after the workspace is set up
  * and joined back to it with events before the call's last launch, so all work
- * is still ordered on `stream` as seen from the caller (CUDA-graph capture of
- * `stream` records the fork and join).  Calls from several host threads at
- * once share that stream: correct, but their second kernels serialise.
+ * is still ordered on `stream` as seen from the caller.  Calls from several
+ * host threads at once are correct (each fork and join is recorded and
+ * awaited under one lock) and their second kernels serialise on that stream.
+ * The chunked path stages a chunk table from host memory owned by the call, so
+ * it cannot be captured into a CUDA graph: a call on a capturing stream returns
+ * KDA_ERR_UNSUPPORTED and enqueues nothing.  The fp32 recurrent path and the
+ * decode entry points copy nothing from the host.
  */
 kda_status kda_prefill(const void* q, const void* k, const void* v, const void* g,
                        const void* beta, const float* conv_w, const void* init_state,
@@ -282,8 +286,8 @@ kda_status kda_decode_commit_verify(void* state, void* conv_cache, const void* p
  *     KDA_NOALLOC_SCRATCH_BYTES are rejected with KDA_ERR_WORKSPACE before any
  *     launch (about 1000 chunk-heads: (sum over segments of ceil(T_n / 64))
  *     x num_heads <= 1000 fits).
- *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress; no allocation).
  *   - All calls share the one array and it keeps the last call's contents
  *     (every byte a call reads is written earlier in that same call, so
  *     nothing needs clearing).  Calls whose work overlaps on the GPU (other
@@ -338,7 +342,8 @@ kda_status kda_check_async_status(void* stream);
  *       that takes the overlapped chunked mode (at most 96 (sequence, head)
  *       pairs) launches its preparation kernel without the per-chunk ready
  *       flags, so the flags the scan waits on are never published.  The scan's
- *       bounded waits give up (well under 2 s), every block drains its own copies
+ *       bounded waits give up (after 2 s plus 1 us per (chunk, head) work
+ *       item of the call, timed by %globaltimer), every block drains its own copies
  *       and tensor-core work, frees its tensor memory and returns; the call's
  *       outputs are invalid and kda_check_async_status reports
  *       KDA_ERR_TIMEOUT.  The context stays usable.

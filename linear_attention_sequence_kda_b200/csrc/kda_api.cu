@@ -410,27 +410,17 @@ int kda_version(void) { return (2 << 16) | 1; }
 // The chunked path's scratch (chunk table + one operand record per chunk and
 // head) lives in this file-scope device array instead of a caller workspace.
 // In host code the name below is only a stand-in for the symbol; the device
-// address is obtained with cudaGetSymbolAddress, once per device.
+// address is obtained with cudaGetSymbolAddress, with the device current.
 static __device__ __align__(256) unsigned char kda_noalloc_scratch[KDA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// device address of kda_noalloc_scratch on the current device (looked up on
-// the first call for that device, with that device current)
+// device address of kda_noalloc_scratch on the current device, looked up on
+// every call (cheap), so that a context torn down and created again never
+// leaves a stale address behind
 kda_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, kda_noalloc_scratch) != cudaSuccess || !p) return KDA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, kda_noalloc_scratch) != cudaSuccess || !p) return KDA_ERR_CUDA;
+  *out = p;
   return KDA_OK;
 }
 }  // namespace

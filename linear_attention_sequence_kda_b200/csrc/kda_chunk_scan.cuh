@@ -62,7 +62,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
                   const Ts* init_state, const __nv_bfloat16* __restrict__ init_conv,
                   const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
-                  const int* __restrict__ ready, Tout* __restrict__ o, Ts* final_state) {
+                  const int* __restrict__ ready, Tout* __restrict__ o, Ts* final_state,
+                  uint64_t wait_ns) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (32-bit shared loads and stores)
@@ -113,8 +114,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         const uint32_t p = i & 1;
         // V_i in TMEM (and the output of chunk i - 2 read from the O^T buffer
         // of this parity); the first record piece of chunk i in shared memory
-        ok = tc::bar_wait_or(&bar_conv, p, abort_flag);
-        ok = ok && tc::bar_wait_or(&bar_a, p, abort_flag);
+        ok = tc::bar_wait_or(&bar_conv, p, abort_flag, wait_ns);
+        ok = ok && tc::bar_wait_or(&bar_a, p, abort_flag, wait_ns);
         if (!ok) break;
         tc::fence_after();
         // [U^T | O^T] = S^T [-W ; Q~]^T, then U^T += V^T T_s^T
@@ -127,8 +128,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
           tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, d_ts + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
         tc::commit(&bar_ma);
         // O^T += U^T P_s^T as soon as U^T is final
-        ok = tc::bar_wait_or(&bar_b, p, abort_flag);
-        ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag);
+        ok = tc::bar_wait_or(&bar_b, p, abort_flag, wait_ns);
+        ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag, wait_ns);
         if (!ok) break;
         tc::fence_after();
         const uint32_t dO = tm + o_col(i);
@@ -136,7 +137,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         for (int ks = 0; ks < 8; ++ks)
           tc::mma_ts(dO, tm + TM_U + 8 * ks, d_ps + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
         // S^T += U^T K-bar once S^T diag(gamma) is in place
-        ok = tc::bar_wait_or(&bar_d, p, abort_flag);
+        ok = tc::bar_wait_or(&bar_d, p, abort_flag, wait_ns);
         if (!ok) break;
         tc::fence_after();
 #pragma unroll
@@ -144,7 +145,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
           tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, d_kb + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), 1);
         tc::commit(&bar_m2);
         tc::commit(&bar_pkfree);
-        ok = tc::bar_wait_or(&bar_m2, p, abort_flag);  // S^T complete for the next chunk
+        ok = tc::bar_wait_or(&bar_m2, p, abort_flag, wait_ns);  // S^T complete for the next chunk
       }
       if (!ok) {
         s_abort = 1;
@@ -175,14 +176,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       // with the prep kernel running concurrently, a chunk's record is read
       // only once its ready flag is published (flag of chunk j at rdy[j * H])
       const int* rdy = ready ? ready + (int64_t)chunk_base[n] * H + h : nullptr;
-      auto record_ready = [&](int j) -> bool { return !rdy || tc::flag_wait_or(rdy + (int64_t)j * H, abort_flag); };
+      auto record_ready = [&](int j) -> bool { return !rdy || tc::flag_wait_or(rdy + (int64_t)j * H, abort_flag, wait_ns); };
       bool ok = true;
       if (nchunks > 0) {
         ok = record_ready(0);
         if (ok) { load_a(0); load_v(0); load_pk(0); }
       }
       if (ok && nchunks > 1) {  // the conv of chunk 0 has read value tile 0
-        ok = tc::bar_wait_or(&bar_vfree, 0, abort_flag);
+        ok = tc::bar_wait_or(&bar_vfree, 0, abort_flag, wait_ns);
         if (ok) load_v(1);
       }
       // record pieces of chunk j as their buffers free up during chunk j - 1;
@@ -190,14 +191,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       // has read tile j
       for (int j = 1; j < nchunks && ok; ++j) {
         const uint32_t q = (j - 1) & 1;
-        ok = tc::bar_wait_or(&bar_ma, q, abort_flag);  // MMA_A of chunk j - 1 has read the first piece
+        ok = tc::bar_wait_or(&bar_ma, q, abort_flag, wait_ns);  // MMA_A of chunk j - 1 has read the first piece
         ok = ok && record_ready(j);
         if (ok) load_a(j);
         if (ok && j + 1 < nchunks) {
-          ok = tc::bar_wait_or(&bar_vfree, j & 1, abort_flag);
+          ok = tc::bar_wait_or(&bar_vfree, j & 1, abort_flag, wait_ns);
           if (ok) load_v(j + 1);
         }
-        ok = ok && tc::bar_wait_or(&bar_pkfree, q, abort_flag);  // MMA2 of chunk j - 1 has read the second
+        ok = ok && tc::bar_wait_or(&bar_pkfree, q, abort_flag, wait_ns);  // MMA2 of chunk j - 1 has read the second
         if (ok) load_pk(j);
       }
       if (!ok) {
@@ -216,7 +217,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       bool ok = true;
       for (int i = 0; i < nchunks && ok; ++i) {
         const int b = i & 1;
-        ok = tc::bar_wait_or(&bar_ost[b], (uint32_t)((i >> 1) & 1), abort_flag);
+        ok = tc::bar_wait_or(&bar_ost[b], (uint32_t)((i >> 1) & 1), abort_flag, wait_ns);
         if (!ok) break;
         const Tout* st = reinterpret_cast<const Tout*>(sm + SCAN_OST + b * OST_BYTES);
         const int64_t tj = seg0 + (int64_t)CH * i;
@@ -258,7 +259,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     // short conv of v for chunk i, tokens t0 .. t0 + 15, into registers (the
     // value tile is released as soon as it has been read)
     auto conv_v = [&](int i, float (&vv)[16]) -> bool {
-      if (!tc::bar_wait_or(&bar_v, (uint32_t)(i & 1), abort_flag)) return false;
+      if (!tc::bar_wait_or(&bar_v, (uint32_t)(i & 1), abort_flag, wait_ns)) return false;
       const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(sm + SCAN_V);
       const int L = (int)((T - (int64_t)CH * i) < CH ? (T - (int64_t)CH * i) : CH);
       float h0, h1, h2;  // tokens t0 - 3 .. t0 - 1 (tile rows t0 .. t0 + 2)
@@ -314,8 +315,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       // (a) the next chunk's value conv while MMA_A of this chunk runs, then
       //     U^T of this chunk (S^T read by the tensor core) and its scalars
       if (more) ok = conv_v(i + 1, vn);
-      ok = ok && tc::bar_wait_or(&bar_ma, p, abort_flag);
-      ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag);
+      ok = ok && tc::bar_wait_or(&bar_ma, p, abort_flag, wait_ns);
+      ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag, wait_ns);
       if (!ok) break;
       tc::fence_after();
       // (b) U += beta V (exact diagonal of T V); P_tt U kept in fp32
@@ -359,8 +360,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       if (more) tc::bar_arrive(&bar_conv);
       // (e) o = O + P_tt u once MMA2 is done, into the staging tile of this
       // parity (free once the store of chunk i - 2 has read it)
-      ok = ok && tc::bar_wait_or(&bar_m2, p, abort_flag);
-      if (ok && i >= 2) ok = tc::bar_wait_or(&bar_ofree[p], (uint32_t)(((i >> 1) - 1) & 1), abort_flag);
+      ok = ok && tc::bar_wait_or(&bar_m2, p, abort_flag, wait_ns);
+      if (ok && i >= 2) ok = tc::bar_wait_or(&bar_ofree[p], (uint32_t)(((i >> 1) - 1) & 1), abort_flag, wait_ns);
       if (!ok) break;
       tc::fence_after();
       {

@@ -63,25 +63,49 @@ inline bool take_fault(kda_fault kind) {
 }
 
 // Side stream and fork / join events of the overlapped mode, one set per
-// device, created on first use.
-inline kda_status overlap_stream(cudaStream_t* side, cudaEvent_t* fork, cudaEvent_t* join) {
-  static std::mutex mu;
-  static cudaStream_t streams[64] = {};
-  static cudaEvent_t forks[64] = {}, joins[64] = {};
+// device, created on first use.  fork_side() records the fork on `stream` and
+// makes the side stream wait for it under one lock, so that two host threads
+// forking at once cannot make a scan wait on the other thread's stream.
+struct OverlapStreams {
+  std::mutex mu;
+  cudaStream_t streams[64] = {};
+  cudaEvent_t forks[64] = {}, joins[64] = {};
+};
+inline OverlapStreams& overlap_streams() {
+  static OverlapStreams o;
+  return o;
+}
+inline kda_status fork_side(cudaStream_t stream, cudaStream_t* side, cudaEvent_t* join) {
+  OverlapStreams& o = overlap_streams();
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KDA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!streams[dev]) {
-    if (cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&forks[dev], cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&joins[dev], cudaEventDisableTiming) != cudaSuccess)
+  std::lock_guard<std::mutex> lock(o.mu);
+  if (!o.streams[dev]) {
+    if (cudaStreamCreateWithFlags(&o.streams[dev], cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&o.forks[dev], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&o.joins[dev], cudaEventDisableTiming) != cudaSuccess)
       return KDA_ERR_CUDA;
   }
-  *side = streams[dev];
-  *fork = forks[dev];
-  *join = joins[dev];
+  if (cudaEventRecord(o.forks[dev], stream) != cudaSuccess ||
+      cudaStreamWaitEvent(o.streams[dev], o.forks[dev], 0) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  *side = o.streams[dev];
+  *join = o.joins[dev];
   return KDA_OK;
 }
+// The join is recorded and awaited under the same lock for the same reason.
+inline kda_status join_side(cudaStream_t stream, cudaStream_t side, cudaEvent_t join) {
+  std::lock_guard<std::mutex> lock(overlap_streams().mu);
+  if (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  return KDA_OK;
+}
+
+// Bound of the scan's waits on the preparation kernel's progress: two seconds
+// plus a microsecond per work item (prep publishes tens of items per
+// microsecond on the whole GPU, so the bound is far above a legitimate wait
+// even on a shared, time-sliced device).
+inline uint64_t scan_wait_ns(int64_t items) { return 2000000000ull + (uint64_t)items * 1000ull; }
 
 template <int ACT>
 inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, const void* g,
@@ -91,6 +115,12 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
                                    kda_dtype state_dt, void* o, void* final_state, void* workspace,
                                    cudaStream_t stream) {
   using T = __nv_bfloat16;
+  // The chunk table below is staged from host memory that this call owns and
+  // releases on return; a captured graph would read it again on every replay,
+  // long after it is gone, so stream capture is refused.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cap != cudaStreamCaptureStatusNone) return KDA_ERR_UNSUPPORTED;
   // chunk table and longest-first segment order
   std::vector<int64_t> nch(N);
   int64_t total = 0;
@@ -136,11 +166,9 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     return KDA_ERR_CUDA;
 
   cudaStream_t scan_stream = stream, side = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t join = nullptr;
   if (overlap) {
-    if (overlap_stream(&side, &fork, &join) != KDA_OK || cudaEventRecord(fork, stream) != cudaSuccess ||
-        cudaStreamWaitEvent(side, fork, 0) != cudaSuccess)
-      return KDA_ERR_CUDA;
+    if (fork_side(stream, &side, &join) != KDA_OK) return KDA_ERR_CUDA;
     scan_stream = side;
   }
   if (total > 0) {
@@ -182,7 +210,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
       return false;
     scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, scan_stream>>>(
         tv, to, conv_w, (const Ts*)init_state, (const T*)init_conv, cu_dev, d_base, d_order, H, records,
-        overlap ? ready : nullptr, (Tout*)o, (Ts*)final_state);
+        overlap ? ready : nullptr, (Tout*)o, (Ts*)final_state, scan_wait_ns(items));
     return true;
   };
   bool ok;
@@ -191,8 +219,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   else
     ok = state_dt == KDA_F32 ? launch_scan(T{}, float{}) : launch_scan(T{}, T{});
   if (!ok || cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
-  if (overlap && (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess))
-    return KDA_ERR_CUDA;
+  if (overlap && join_side(stream, side, join) != KDA_OK) return KDA_ERR_CUDA;
   return KDA_OK;
 }
 

@@ -18,8 +18,10 @@
 namespace kda {
 namespace tc {
 
-// Upper bound on mbarrier polls before a wait gives up and reports a timeout.
-constexpr int kWaitLimit = 1 << 24;
+// Default bound of a device-side wait, in nanoseconds of %globaltimer: four
+// seconds.  Waits on another kernel's progress take a bound computed by the
+// host for the problem at hand instead.
+constexpr uint64_t kWaitNs = 4000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -162,18 +164,30 @@ __device__ __forceinline__ void bar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ bool try_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait on phase parity.  Returns false (and records KDA_ERR_TIMEOUT in
-// the device status word) if the phase did not complete within the limit.
-__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
+// the device status word) if the phase did not complete within `limit_ns`
+// nanoseconds.
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitNs) {
   const uint32_t a = smem_u32(bar);
-  for (int it = 0; it < kWaitLimit; ++it) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return true;
+  if (try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (try_wait(a, parity)) return true;
+    if ((it & 255) == 0 && globaltimer() - t0 > limit_ns) break;
   }
   set_status(KDA_ERR_TIMEOUT);
   return false;
@@ -182,34 +196,29 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait that also gives up (without recording a status) once `*abort`
 // is nonzero: another role of the block has already failed and will not
 // produce what is awaited.
-__device__ __forceinline__ bool bar_wait_or(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+__device__ __forceinline__ bool bar_wait_or(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                            uint64_t limit_ns = kWaitNs) {
   const uint32_t a = smem_u32(bar);
-  for (int it = 0; it < kWaitLimit; ++it) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if ((it & 255) == 255 && *abort) return false;
+  if (try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (try_wait(a, parity)) return true;
+    if ((it & 255) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > limit_ns) break;
+    }
   }
   set_status(KDA_ERR_TIMEOUT);
   return false;
 }
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 // Wait until another kernel publishes *flag != 0 (acquire at GPU scope), then
 // order this thread's later bulk copies (async proxy) after that acquire, so
 // that they read what the flag's writer stored before it.  Bounded: gives up
-// after about two seconds (recording KDA_ERR_TIMEOUT), or without a status
-// once `*abort` is set by another role of the block.
-__device__ __forceinline__ bool flag_wait_or(const int* flag, const volatile int* abort) {
+// after `limit_ns` nanoseconds (recording KDA_ERR_TIMEOUT), or without a
+// status once `*abort` is set by another role of the block.
+__device__ __forceinline__ bool flag_wait_or(const int* flag, const volatile int* abort, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer();
-  for (int it = 0; it < (1 << 26); ++it) {
+  for (uint32_t it = 0;; ++it) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
     if (v) {
@@ -218,7 +227,7 @@ __device__ __forceinline__ bool flag_wait_or(const int* flag, const volatile int
     }
     if ((it & 63) == 63) {
       if (*abort) return false;
-      if (globaltimer() - t0 > 2000000000ull) break;
+      if (globaltimer() - t0 > limit_ns) break;
     }
     __nanosleep(64);
   }

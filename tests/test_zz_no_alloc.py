@@ -9,7 +9,7 @@ import torch
 
 import kda_inputs as ki
 import linear_attention_sequence_kda_b200 as kda
-from parity import TOL, rel_err, to_dev
+from parity import to_dev
 
 
 def test_noalloc_rejects_problems_beyond_the_static_scratch():
@@ -28,24 +28,27 @@ def test_noalloc_rejects_problems_beyond_the_static_scratch():
 
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row():
+    """Both entry points run the same kernels on the same inputs, and the
+    chunked path is deterministic, so the results must be equal bit for bit.
+    The cases cover both schedules of the chunked path: at most 96 (sequence,
+    head) chains (the scan overlaps the preparation kernel) and more (the two
+    run one after the other), all through the one static scratch array."""
     cases = [ki.make_prefill([200, 37], 4, torch.bfloat16, 31, state_std=0.02, conv_history=True),
-             ki.make_prefill([65, 1, 300], 2, torch.bfloat16, 32, state_std=0.02, conv_history=True)]
-    for inp in cases:  # two different problems back to back through the same scratch
+             ki.make_prefill([65, 1, 300], 2, torch.bfloat16, 32, state_std=0.02, conv_history=True),
+             ki.make_prefill([64, 200, 130, 77, 1, 128, 190, 65], 16, torch.bfloat16, 33, state_std=0.02,
+                             conv_history=True)]
+    assert cases[2].num_seqs * cases[2].num_heads > 96
+    for inp in cases:  # different problems back to back through the same scratch
         assert kda.workspace_size(inp.num_seqs, inp.total_tokens, inp.num_heads,
                                   int(np.diff(inp.cu_seqlens).max())) <= kda.NOALLOC_SCRATCH_BYTES
         d = to_dev(inp)
         args = (d["q"], d["k"], d["v"], d["g"], d["beta"], d["conv_w"], inp.cu_seqlens, d["cu_dev"],
                 d["init_state"], d["init_conv"])
-        o_ref, s_ref, t_ref = kda.prefill(*args)
-        o_na, s_na, t_na = kda.prefill_noalloc(*args)
-        torch.cuda.synchronize()
-        assert kda.check_async_status() == 0
-        tol = TOL[torch.bfloat16]
-        for n in range(inp.num_seqs):
-            s0, s1 = int(inp.cu_seqlens[n]), int(inp.cu_seqlens[n + 1])
-            for h in range(inp.num_heads):
-                if s1 > s0:
-                    assert rel_err(o_na[s0:s1, h].double().cpu().numpy(),
-                                   o_ref[s0:s1, h].double().cpu().numpy()) <= tol
-                assert rel_err(s_na[n, h].double().cpu().numpy(), s_ref[n, h].double().cpu().numpy()) <= tol
-        assert torch.equal(t_na, t_ref)
+        for _ in range(2):  # two calls in a row of each entry point
+            o_ref, s_ref, t_ref = kda.prefill(*args)
+            o_na, s_na, t_na = kda.prefill_noalloc(*args)
+            torch.cuda.synchronize()
+            assert kda.check_async_status() == 0
+            assert torch.equal(o_na, o_ref)
+            assert torch.equal(s_na, s_ref)
+            assert torch.equal(t_na, t_ref)
