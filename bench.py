@@ -41,11 +41,20 @@ import kda_inputs as ki  # noqa: E402
 METRIC = "KDA prefill tokens/s (64 heads, T=64k) and decode state GB/s vs HBM peak"
 WORKLOAD = "kda_prefill long-context: 1 x T=65536, 64 heads x 128, bf16 in / fp32 state / fp32 out, chunk 64"
 H, D, T_LONG = 64, 128, 65536
-# algorithmic bytes (what the method must move): per token-head q,k,v,g (4 x 256 B bf16)
-# + beta (2 B) + o (512 B fp32); per (sequence, head) the final state (64 KiB; no
-# initial state in this workload).
-BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 2 + D * 4
+# Algorithmic bytes of a prefill (what the method must move, bf16 workloads):
+# per token-head q, k, v, g (4 x 256 B) + beta (2 B) + o (256 B in the input
+# dtype) = 1,282 B, plus per (sequence, head) the initial and the final state
+# (2 x 64 KiB fp32).  The library writes o in fp32 (512 B per token-head);
+# that variant is reported beside it, labelled.
+BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 2 + D * 2
+BYTES_PER_TOKEN_HEAD_O32 = 4 * D * 2 + 2 + D * 4
 STATE_BYTES = D * D * 4
+# Useful tensor work of the chunked prefill per token-head: the state products
+# (6 K V) and the intra-chunk products (7 C K), C = 64.
+FLOP_PER_TOKEN_HEAD = 6 * D * D + 7 * 64 * D
+# Every contraction runs as tcgen05 kind::tf32, whose nominal dense rate is
+# half the bf16 rate (1.1 of 2.25 PFLOP/s): the tf32 peak is bf16_tflops / 2.
+TF32_PER_BF16 = 0.5
 
 
 # decode: per (sequence, head) the state read + written (4 or 2 bytes per element), q/k/v/g
@@ -345,6 +354,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=6, help="0 skips the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-prefill", action="store_true",
+                    help="skip the 4 x 4096 and varlen prefill legs")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode leg")
     ap.add_argument("--heads", type=int, default=H,
                     help="reduced head count (profiling only; the reported workload uses 64)")
@@ -384,32 +395,13 @@ def main():
         inp = ki.workload(2)
     else:  # same recipe, reduced size (for profiler captures)
         inp = ki.make_prefill([T_run], heads, torch.bfloat16, ki.BASE_SEED + 2, gate="bimodal")
-    d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "g", "beta", "conv_w")}
-    cu_dev = torch.from_numpy(inp.cu_seqlens).to(dev)
-    o = torch.empty(d["q"].shape, dtype=torch.float32, device=dev)
-    S = torch.empty((1, heads, D, D), dtype=torch.float32, device=dev)
-    tail = torch.empty((1, 3, 3, heads * D), dtype=torch.bfloat16, device=dev)
-    ws_bytes = kda.workspace_size(1, T_run, heads, T_run)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-
-    def prefill_into(dd, oo, ss):
-        kda.prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["conv_w"], inp.cu_seqlens, cu_dev,
-                    None, None, o=oo, final_state=ss, conv_tail=tail, workspace=ws, stream=stream)
-
-    def step():
-        prefill_into(d, o, S)
-
     with ClockSampler(torch.cuda.current_device()) as clk:
-        total_ms, per_step = timed(step, args.steps, args.warmup, world, stream)
-    assert kda.check_async_status(stream) == 0
-    ms = total_ms / args.steps
+        head_leg, ctx = run_prefill_leg(args, world, dev, stream, kda, inp, args.steps, hbm_peak, bf16_peak,
+                                        peak_src, keep=True)
+    d, o, S, prefill_into = ctx
+    ms = head_leg["ms_per_step"]
     tokens_per_rank = T_run
-    value = world * tokens_per_rank * args.steps / (total_ms / 1e3)
-    alg_bytes = T_run * heads * BYTES_PER_TOKEN_HEAD + heads * STATE_BYTES
-    launch_ms = statistics.mean(per_step)
-    achieved = alg_bytes / (launch_ms / 1e3) / 1e9
-    kernel_name = "kda_prefill (chunk_prep_kernel + chunk_scan_kernel)"
-    traffic = recorded_traffic(kernel_name)
+    value = world * tokens_per_rank * args.steps / (head_leg["total_ms"] / 1e3)
 
     # ---------------- end to end: host buffers through the C ABI ----------------
     e2e = None
@@ -425,6 +417,14 @@ def main():
         dec16_line = run_decode(args, world, dev, stream, kda, hbm_peak, torch.bfloat16)
         mtp16_line = run_mtp_fused(args, world, dev, stream, kda, hbm_peak, torch.bfloat16)
 
+    # ---------------- the other prefill workloads (multi-sequence schedules) ----
+    other_legs = {}
+    if not args.no_other_prefill and (heads, T_run) == (H, T_LONG):
+        other_legs["prefill_4x4096"] = run_prefill_leg(args, world, dev, stream, kda, ki.workload(1),
+                                                       args.steps, hbm_peak, bf16_peak, peak_src)[0]
+        other_legs["prefill_varlen"] = run_prefill_leg(args, world, dev, stream, kda, ki.workload(3),
+                                                       max(3, args.steps // 2), hbm_peak, bf16_peak, peak_src)[0]
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -432,10 +432,8 @@ def main():
         "config": {"workload": WORKLOAD, "heads": heads, "head_dim": D, "seq_len": T_run, "batch_per_gpu": 1,
                    "chunk": 64, "parallelism": f"dp{world} (independent sequences per GPU)",
                    "l2": "inputs larger than L2 (4.3 GB read per step), no flush"},
-        "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": hbm_peak,
-                     "unit": "GB/s", "frac": achieved / hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst)",
-                     "traffic": traffic, "algorithmic_bytes_per_launch": alg_bytes,
-                     "launch_ms": launch_ms},
+        "roofline": head_leg["roofline"],
+        "tensor": head_leg["tensor"],
         "e2e": e2e,
         "gpu_launches": args.steps * PREFILL_LAUNCHES,
         "clocks": clk.summary(),
@@ -445,16 +443,133 @@ def main():
         "mtp_fused": fused_line,
         "decode_bf16_state": dec16_line,
         "mtp_fused_bf16_state": mtp16_line,
+        **other_legs,
     }
     if (heads, T_run) != (H, T_LONG):
         line["config"]["note"] = "reduced profiling size, not the reported workload"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
+        line["oracle_per_workload"] = oracle_per_workload()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def prefill_roofline(inp, launch_ms, hbm_peak, bf16_peak, peak_src, traffic, kernel_name):
+    """HBM roofline of one kda_prefill on the method's bytes (1,282 B per
+    token-head + initial and final state per (sequence, head)), the variant
+    with o as the library writes it (fp32), and the tensor-pipe fraction of the
+    useful chunked work against the tf32 peak."""
+    tok_heads = inp.total_tokens * inp.num_heads
+    pairs = inp.num_seqs * inp.num_heads
+    alg = tok_heads * BYTES_PER_TOKEN_HEAD + pairs * 2 * STATE_BYTES
+    alg32 = tok_heads * BYTES_PER_TOKEN_HEAD_O32 + pairs * 2 * STATE_BYTES
+    sec = launch_ms / 1e3
+    achieved = alg / sec / 1e9
+    flops = tok_heads * FLOP_PER_TOKEN_HEAD
+    tf32_peak = bf16_peak * TF32_PER_BF16
+    roof = {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst)", "traffic": traffic,
+            "algorithmic_bytes_per_launch": alg, "launch_ms": launch_ms,
+            "o_fp32_variant": {"algorithmic_bytes_per_launch": alg32, "achieved": alg32 / sec / 1e9,
+                               "frac": alg32 / sec / 1e9 / hbm_peak,
+                               "note": "same call, o counted as written (fp32, 512 B per token-head)"}}
+    tensor = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": tf32_peak, "unit": "TFLOP/s",
+              "frac": flops / sec / 1e12 / tf32_peak, "flop_per_launch": flops,
+              "peak_source": f"{peak_src} bf16_tflops x {TF32_PER_BF16} (nominal tf32 : bf16)"}
+    return roof, tensor
+
+
+def run_prefill_leg(args, world, dev, stream, kda, inp, steps, hbm_peak, bf16_peak, peak_src, keep=False):
+    """Times kda_prefill on one workload with its inputs resident in HBM:
+    W warm-up calls, then `steps` calls between barrier + synchronize, a CUDA
+    event pair per call on the launching stream."""
+    d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "g", "beta", "conv_w")}
+    init_state = None if inp.init_state is None else inp.init_state.to(dev)
+    init_conv = None if inp.init_conv is None else inp.init_conv.to(dev)
+    cu_dev = torch.from_numpy(inp.cu_seqlens).to(dev)
+    N, Hh = inp.num_seqs, inp.num_heads
+    o = torch.empty(d["q"].shape, dtype=torch.float32, device=dev)
+    S = torch.empty((N, Hh, D, D), dtype=torch.float32, device=dev)
+    tail = torch.empty((N, 3, 3, Hh * D), dtype=torch.bfloat16, device=dev)
+    max_len = int(np.diff(inp.cu_seqlens).max()) if N else 0
+    ws_bytes = kda.workspace_size(N, inp.total_tokens, Hh, max_len)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+    def prefill_into(dd, oo, ss):
+        kda.prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["conv_w"], inp.cu_seqlens, cu_dev,
+                    init_state, init_conv, o=oo, final_state=ss, conv_tail=tail, workspace=ws, stream=stream)
+
+    total_ms, per_step = timed(lambda: prefill_into(d, o, S), steps, args.warmup, world, stream)
+    assert kda.check_async_status(stream) == 0
+    launch_ms = statistics.mean(per_step)
+    kernel_name = "kda_prefill (chunk_prep_kernel + chunk_scan_kernel)"
+    chains = N * Hh
+    label = "prefill_long" if (N, inp.total_tokens) == (1, T_LONG) else (
+        "prefill_4x4096" if (N, inp.total_tokens) == (4, 16384) else "prefill_varlen")
+    roof, tensor = prefill_roofline(inp, launch_ms, hbm_peak, bf16_peak, peak_src,
+                                    recorded_traffic(f"{kernel_name} {label}"), kernel_name)
+    leg = {"workload": f"kda_prefill: {N} sequence(s), {inp.total_tokens} tokens, {Hh} heads x 128, bf16 in / "
+                       f"fp32 state / fp32 out, {chains} (sequence, head) chains "
+                       f"({'overlapped' if chains <= 96 else 'one after the other'} schedule)",
+           "tokens_per_s": world * inp.total_tokens * steps / (total_ms / 1e3), "ms_per_step": total_ms / steps,
+           "total_ms": total_ms, "steps": steps, "roofline": roof, "tensor": tensor,
+           "gpu_launches": steps * PREFILL_LAUNCHES}
+    if keep:
+        return leg, (d, o, S, prefill_into)
+    del d, o, S, ws
+    torch.cuda.empty_cache()
+    return leg, None
+
+
+def oracle_per_workload():
+    """The fp64 oracle as it stands, timed on this host's cores for every
+    workload (a bounded sample of the large ones), with the thread count, and
+    on one core for the tiny and the decode workloads."""
+    import oracle  # test infrastructure; only the baseline legs run it
+    cores = os.cpu_count() or 1
+    out = {}
+
+    def time_probs(probs, threads):
+        t0 = time.perf_counter()
+        used = oracle.run_problems(probs, threads)
+        return time.perf_counter() - t0, used
+
+    def prefill_sample(i, inp, tokens_note):
+        probs = [oracle.prefill_problem(inp, n, h) for n in range(inp.num_seqs) for h in range(inp.num_heads)]
+        toks = inp.total_tokens
+        dt, used = time_probs(probs, cores)
+        rec = {"tokens_per_s": toks / dt, "cores": used, "seconds": dt, "sample": tokens_note}
+        if i == 0:
+            dt1, _ = time_probs([oracle.prefill_problem(inp, n, h) for n in range(inp.num_seqs)
+                                 for h in range(inp.num_heads)], 1)
+            rec["one_core_tokens_per_s"] = toks / dt1
+        return rec
+
+    out["tiny_fp32"] = prefill_sample(0, ki.workload(0), "whole workload (1 x 256 tokens, 2 heads)")
+    w1 = ki.workload(1)
+    out["prefill_4x4096"] = prefill_sample(1, w1, "whole workload (4 x 4096 tokens, 64 heads)")
+    del w1
+    w2 = ki.make_prefill([4096], H, torch.bfloat16, ki.BASE_SEED + 2, gate="bimodal")
+    out["prefill_long"] = prefill_sample(2, w2, "first 4096 tokens x 64 heads of the T=65536 workload")
+    del w2
+    lens = ki.varlen_lengths(ki.BASE_SEED + 3)
+    w3 = ki.make_prefill([min(lens[0], 4096)], H, torch.bfloat16, ki.BASE_SEED + 3, state_std=0.02,
+                         conv_history=True)
+    out["prefill_varlen"] = prefill_sample(3, w3, f"first {min(lens[0], 4096)} tokens of segment 0 x 64 heads "
+                                                  f"of the varlen workload (same recipe)")
+    del w3
+    dec = ki.workload(4)
+    probs = [oracle.decode_problem(dec, n, h) for n in range(dec.num_seqs) for h in range(H)]
+    dt, used = time_probs(probs, cores)
+    probs1 = [oracle.decode_problem(dec, n, h) for n in range(16) for h in range(H)]
+    dt1, _ = time_probs(probs1, 1)
+    out["decode"] = {"tokens_per_s": dec.num_seqs / dt, "cores": used, "seconds": dt,
+                     "one_core_tokens_per_s": 16 / dt1,
+                     "sample": "whole workload (256 sequences x 64 heads, one step); one core on 16 sequences"}
+    return out
 
 
 def run_e2e(args, world, stream, inp, d, o, S, prefill_into, tokens_per_rank):

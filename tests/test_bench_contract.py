@@ -15,11 +15,33 @@ KIB = 1024
 
 
 def test_prefill_bytes_per_token_head():
-    # q, k, v, g rows in bf16 (4 x 256 B), beta in bf16, o in fp32 (512 B)
-    assert bench.BYTES_PER_TOKEN_HEAD == 4 * 256 + 2 + 512
+    # the method's bytes: q, k, v, g rows in bf16 (4 x 256 B), beta in bf16, o in
+    # the input dtype (256 B); the library's fp32 o (512 B) is the labelled variant
+    assert bench.BYTES_PER_TOKEN_HEAD == 4 * 256 + 2 + 256 == 1282
+    assert bench.BYTES_PER_TOKEN_HEAD_O32 == 4 * 256 + 2 + 512
     assert bench.STATE_BYTES == 64 * KIB
-    # the long-context workload: 65,536 tokens x 64 heads, one final state per head
-    assert 65536 * 64 * bench.BYTES_PER_TOKEN_HEAD + 64 * bench.STATE_BYTES == 6_455_033_856
+    # the long-context workload: 65,536 tokens x 64 heads, initial and final
+    # state per head
+    assert 65536 * 64 * bench.BYTES_PER_TOKEN_HEAD + 64 * 2 * bench.STATE_BYTES == 5_385_486_336
+
+
+def test_prefill_flop_per_token_head():
+    # state products 6 K V plus intra-chunk products 7 C K (K = V = 128, C = 64)
+    assert bench.FLOP_PER_TOKEN_HEAD == 6 * 128 * 128 + 7 * 64 * 128 == 155_648
+
+
+class _Inp:
+    def __init__(self, n, t, h):
+        self.num_seqs, self.total_tokens, self.num_heads = n, t, h
+
+
+def test_prefill_roofline_fractions():
+    roof, tensor = bench.prefill_roofline(_Inp(1, 65536, 64), 6.0, 6500.0, 1600.0, "measured", None, "k")
+    assert abs(roof["achieved"] - 5_385_486_336 / 6e-3 / 1e9) < 1e-6
+    assert abs(roof["frac"] - roof["achieved"] / 6500.0) < 1e-12
+    assert abs(tensor["peak"] - 800.0) < 1e-9
+    assert abs(tensor["achieved"] - 65536 * 64 * 155_648 / 6e-3 / 1e12) < 1e-9
+    assert roof["o_fp32_variant"]["algorithmic_bytes_per_launch"] == 65536 * 64 * 1538 + 64 * 2 * 65536
 
 
 def test_decode_bytes_per_pair():
