@@ -354,6 +354,13 @@ kda_status kda_check_async_status(void* stream);
 typedef enum { KDA_FAULT_NONE = 0, KDA_FAULT_DROP_READY = 1 } kda_fault;
 kda_status kda_inject_fault(kda_fault kind);
 
+/*
+ * The cudaError_t value behind the last KDA_ERR_CUDA that an entry point
+ * returned on the calling host thread (0 if none has been returned yet).  Pure
+ * host function; the value is not cleared by later successful calls.
+ */
+int kda_last_cuda_error(void);
+
 /* Library ABI version: (major << 16) | minor. */
 int kda_version(void);
 

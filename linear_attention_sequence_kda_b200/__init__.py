@@ -28,7 +28,7 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
            "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version",
            "kda_prefill_noalloc", "kda_decode_deltas_size", "kda_decode_verify", "kda_decode_commit",
-           "kda_decode_commit_verify", "kda_state_affine", "kda_inject_fault")
+           "kda_decode_commit_verify", "kda_state_affine", "kda_inject_fault", "kda_last_cuda_error")
 MAX_VERIFY_ROWS = 8  # KDA_MAX_VERIFY_ROWS
 
 if not os.path.exists(LIB_PATH):
@@ -37,6 +37,8 @@ if not os.path.exists(LIB_PATH):
 
 _vp, _i32p, _f32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
 lib = ctypes.CDLL(LIB_PATH)
+lib.kda_last_cuda_error.restype = ctypes.c_int
+lib.kda_last_cuda_error.argtypes = []
 lib.kda_prefill_workspace_size.restype = ctypes.c_size_t
 lib.kda_prefill_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int]
@@ -80,7 +82,11 @@ KDA_FAULT_NONE, KDA_FAULT_DROP_READY = 0, 1
 class KdaError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {STATUS.get(code, code)} ({lib.kda_status_string(code).decode()})")
+        msg = f"{where}: {STATUS.get(code, code)} ({lib.kda_status_string(code).decode()})"
+        if code == 5:  # KDA_ERR_CUDA: name the CUDA runtime error behind it
+            self.cuda_error = int(lib.kda_last_cuda_error())
+            msg += f" [cudaError_t {self.cuda_error}]"
+        super().__init__(msg)
 
 
 def _check(code: int, where: str) -> None:

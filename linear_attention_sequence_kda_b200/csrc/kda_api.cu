@@ -90,7 +90,7 @@ kda_status launch_tail(const PrefillArgs& a) {
   conv_tail_kernel<Tin><<<(unsigned)blocks, 256, 0, a.stream>>>(
       (const Tin*)a.q, (const Tin*)a.k, (const Tin*)a.v, (const Tin*)a.init_conv, a.cu_dev, a.N,
       a.H, (Tin*)a.conv_tail);
-  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return cuda_ok(cudaGetLastError()) ? KDA_OK : KDA_ERR_CUDA;
 }
 
 template <typename Tin>
@@ -106,7 +106,7 @@ kda_status launch_recurrent(const PrefillArgs& a) {
       });
     });
   });
-  if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+  if (!cuda_ok(cudaGetLastError())) return KDA_ERR_CUDA;
   return launch_tail<Tin>(a);
 }
 
@@ -118,8 +118,8 @@ kda_status run_recurrent(PrefillArgs& a) {
 // number of SMs of the current device (persistent grids)
 kda_status sm_count(int* out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || *out < 1)
+  if (!cuda_ok(cudaGetDevice(&dev)) ||
+      !cuda_ok(cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev)) || *out < 1)
     return KDA_ERR_CUDA;
   return KDA_OK;
 }
@@ -131,11 +131,11 @@ template <typename Kern, typename... Args>
 kda_status launch_persistent(Kern kern, uint32_t smem, int64_t items, cudaStream_t s, Args... args) {
   int sms = 0;
   if (sm_count(&sms) != KDA_OK) return KDA_ERR_CUDA;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (!cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)))
     return KDA_ERR_CUDA;
   const int blocks = (int)(items < 2 * sms ? items : 2 * sms);
   kern<<<blocks, 256, smem, s>>>(args...);
-  return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return cuda_ok(cudaGetLastError()) ? KDA_OK : KDA_ERR_CUDA;
 }
 
 // shared argument checks of the decode entry points
@@ -267,7 +267,7 @@ kda_status kda_decode_verify(const void* state, const void* conv_cache, const vo
                                                          (const Tin*)v, (const Tin*)g, (const Tin*)beta, conv_w,
                                                          num_rows, num_heads, (decltype(tout)*)o, deltas, nullptr,
                                                          nullptr, nullptr, nullptr, nullptr, 0);
-          rc = cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+          rc = cuda_ok(cudaGetLastError()) ? KDA_OK : KDA_ERR_CUDA;
         });
       });
     });
@@ -314,7 +314,7 @@ kda_status kda_decode_commit_verify(void* state, void* conv_cache, const void* p
                                                          num_rows, num_heads, (decltype(tout)*)o, deltas,
                                                          (const Tin*)prev_q, (const Tin*)prev_k, (const Tin*)prev_v,
                                                          prev_deltas, prev_n_accept, prev_rows);
-          rc = cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+          rc = cuda_ok(cudaGetLastError()) ? KDA_OK : KDA_ERR_CUDA;
         });
       });
     });
@@ -362,12 +362,12 @@ kda_status kda_state_affine(const float* A, const void* S_in, const float* B, vo
   by_type(state_dt, [&](auto ts) {
     using Ts = decltype(ts);
     auto kern = state_affine_kernel<Ts>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AFFINE_SMEM) != cudaSuccess) {
+    if (!cuda_ok(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AFFINE_SMEM))) {
       rc = KDA_ERR_CUDA;
       return;
     }
     kern<<<count, 256, AFFINE_SMEM, s>>>(A, (const Ts*)S_in, B, (Ts*)S_out);
-    rc = cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    rc = cuda_ok(cudaGetLastError()) ? KDA_OK : KDA_ERR_CUDA;
   });
   return rc;
 }
@@ -386,12 +386,12 @@ const char* kda_status_string(kda_status s) {
 }
 
 kda_status kda_check_async_status(void* stream) {
-  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KDA_ERR_CUDA;
+  if (!cuda_ok(cudaStreamSynchronize((cudaStream_t)stream))) return KDA_ERR_CUDA;
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+  if (!cuda_ok(cudaMemcpyFromSymbol(&v, g_status, sizeof(int)))) return KDA_ERR_CUDA;
   if (v != 0) {
     const int zero = 0;
-    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+    if (!cuda_ok(cudaMemcpyToSymbol(g_status, &zero, sizeof(int)))) return KDA_ERR_CUDA;
   }
   return (kda_status)v;
 }
@@ -402,7 +402,9 @@ kda_status kda_inject_fault(kda_fault kind) {
   return KDA_OK;
 }
 
-int kda_version(void) { return (2 << 16) | 1; }
+int kda_version(void) { return (2 << 16) | 2; }
+
+int kda_last_cuda_error(void) { return kda::t_last_cuda_error; }
 
 }  // extern "C"
 
@@ -419,7 +421,7 @@ namespace {
 // leaves a stale address behind
 kda_status noalloc_scratch(void** out) {
   void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, kda_noalloc_scratch) != cudaSuccess || !p) return KDA_ERR_CUDA;
+  if (!cuda_ok(cudaGetSymbolAddress(&p, kda_noalloc_scratch)) || !p) return KDA_ERR_CUDA;
   *out = p;
   return KDA_OK;
 }

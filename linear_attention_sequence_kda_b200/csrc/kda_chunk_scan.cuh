@@ -2,58 +2,67 @@
 // block per (segment, head), serial over the segment's chunks, the 128 x 128
 // fp32 state held in tensor memory the whole time (page "GLM-5.3-Flash im
 // Detail", section "Sequenz-Mixing: 34 KDA-Schichten mit festem Zustand": a
-// state is handed from chunk to chunk).
+// state is handed from chunk to chunk).  The record of each chunk (kda_record.cuh)
+// holds everything that does not depend on the state.
 //
 // TMEM lane v holds row v of (tf32 MMA operands, fp32 where marked)
-//   O^T odd fp32 (cols 0..63) | U^T (64..127) | O^T even fp32 (128..191)
-//   | S^T fp32 (192..319) | V^T (320..383) | V^T fp32 (384..447) | P_tt U^T fp32 (448..511)
-// Per chunk i, with the record written by chunk_prep_kernel:
-//   MMA_A [U^T | O^T] = S^T [-W ; Q~]^T  (N = 128; the record stacks the two
-//         row blocks in the order that puts O^T in the buffer of i's parity),
-//         then U^T += V^T T_s^T
-//   fp32  U^T += beta * V^T (diagonal of T);  keep P_tt * U^T (diagonal of P)
-//   MMA2o O^T += U^T P_s^T                       (A = U^T from TMEM)
-//   fp32  S^T <- S^T diag(e^{Gamma_C})          (while MMA2o runs)
-//   MMA2s S^T += U^T K-bar
-//   fp32  o = O + P_tt u, staged in shared memory and stored by TMA.
-// A operands are read from TMEM as tf32; the state itself stays fp32.
+//   S0 fp32 (cols 0..127) | O^T odd fp32 (128..191) | U'^T (192..255)
+//   | O^T even fp32 (256..319) | S1 fp32 (320..447) | V^T (448..511)
+// The state S^T of chunk i lives in buffer S(i % 2).  Per chunk i, p = i % 2:
+//   MMA_A  [U'^T | O^T] (p = 0) or [O^T | U'^T] (p = 1) = S(p) RA^T   (N = 128)
+//          then U'^T += V^T TS^T                                      (N = 64)
+//   fp32   S(1-p) <- S(p) diag(gamma)          (while MMA_A reads S(p))
+//   fp32   U'^T += b * V^T (the diagonal of Dk T); keep d * U' (of p)
+//   MMA2   [O^T | S(1)] (p = 0) or [S(0) | O^T] (p = 1) += U'^T B2     (N = 192)
+//   fp32   o = r * (O + d u'), staged in shared memory and stored by TMA.
+// So the serial chain from one state to the next is MMA_A, the U' update and
+// MMA2; the decay and the output run beside the tensor core.  A operands are
+// read from TMEM as tf32; the state itself stays fp32.
 //
 // Warp roles, handing off through mbarriers (no block-wide barrier inside the
 // chunk loop):
-//   warps 0..15 compute: warp w serves TMEM lanes 32 (w % 4) .. (value columns)
-//               and token / key quarter w / 4 of every per-chunk step: the short
-//               conv of v for chunk i + 1 (into registers) while MMA_A of
-//               chunk i runs, the fp32 updates of chunk i, then the output
-//               tile of chunk i.
+//   warps 0..15 compute: warp w serves TMEM lanes 32 (w % 4) .. (value columns),
+//               tokens 16 (w / 4) .. and keys 32 (w / 4) .. of every per-chunk
+//               step: the output of chunk i - 1 and the decay of chunk i while
+//               MMA_A of chunk i runs, the U' update of chunk i, then the short
+//               conv of v for chunk i + 1 while MMA2 of chunk i runs.
 //   warp 16     one thread issues the MMAs.
-//   warp 17     one thread issues the loads, each as soon as the step that
-//               read the previous contents of its buffer is done.
+//   warp 17     issues the loads (one thread), each as soon as the product that
+//               read the previous contents of its buffer is done, and drops the
+//               consumed record from L2 (all lanes), so that a record read soon
+//               after it was written never reaches HBM.
 //   warp 18     one thread stores the output tiles (double-buffered staging),
 //               so that global stores never hold up the compute warps.
 // Each thread waits by parity only on barriers that cannot complete two phases
 // ahead of it: the next phase of every barrier it waits on needs an action of
 // its own (or of a role that itself waited on this thread's previous step).
 #pragma once
-#include "kda_chunk_prep.cuh"
 #include "kda_common.cuh"
+#include "kda_record.cuh"
 #include "kda_tc.cuh"
 
 namespace kda {
 
 constexpr int SCAN_THREADS = 608;  // 16 compute warps, MMA, load and store issuing warps
 constexpr int SCAN_COMPUTE = 512;
-constexpr uint32_t SCAN_RA = 0;                          // [-W ; Q~] and T_s (81920 B)
-constexpr uint32_t SCAN_PK = REC_TILES_A;                // P_s | K-bar | scalars (50176 B)
-constexpr uint32_t PK_BYTES = REC_BYTES - REC_PS;
-constexpr uint32_t SCAN_V = SCAN_PK + PK_BYTES;          // raw value tile: 3 halo rows + 64 rows (bf16)
+constexpr uint32_t SCAN_A = 0;                              // RA and TS (81920 B)
+constexpr uint32_t SCAN_B = REC_PIECE_A;                    // B2 (49152 B)
+constexpr uint32_t B2_BYTES = REC_SC - REC_B2;
+constexpr uint32_t SC_BYTES = REC_BYTES - REC_SC;           // the scalars (1280 B), double-buffered
+constexpr uint32_t SCAN_SC = SCAN_B + B2_BYTES;
+constexpr uint32_t SCAN_V = (SCAN_SC + 2 * SC_BYTES + 1023) & ~1023u;  // raw value tile (bf16)
 constexpr uint32_t SCAN_OST = (SCAN_V + RAW_BYTES + 1023) & ~1023u;  // 2 output tiles [64 t][128] (fp32 at most)
 constexpr uint32_t OST_BYTES = CH * D * 4;
 constexpr uint32_t SCAN_SMEM = SCAN_OST + 2 * OST_BYTES + 1024;
 static_assert(SCAN_SMEM + 256 <= 232448, "scan shared memory (dynamic + the static barriers)");
-static_assert(REC_TILES_A % 1024 == 0 && REC_TS % 1024 == 0, "record tiles stay 1024-byte aligned");
-constexpr int TM_O1 = 0, TM_U = 64, TM_O0 = 128, TM_S = 192, TM_V = 320;
-constexpr int TM_VX = 384, TM_UP = 448;  // exact fp32 V and P_tt * U for the diagonal terms
+constexpr int TM_S0 = 0, TM_O1 = 128, TM_U = 192, TM_O0 = 256, TM_S1 = 320, TM_V = 448;
+__device__ __forceinline__ int s_col(int chunk) { return (chunk & 1) ? TM_S1 : TM_S0; }
 __device__ __forceinline__ int o_col(int chunk) { return (chunk & 1) ? TM_O1 : TM_O0; }
+
+// drop one 128-byte line of dead data from L2 without writing it back
+__device__ __forceinline__ void discard_l2(const void* p) {
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
 
 template <typename Tout, int ACT, typename Ts>
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
@@ -68,10 +77,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (32-bit shared loads and stores)
   uint8_t* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-  // loads (record pieces, value tiles), MMA commits, compute-warp hand-offs
-  // loads; "free" signals for the loader; MMA commits; compute-warp hand-offs;
-  // output staging full / free
-  __shared__ uint64_t bar_a, bar_pk, bar_v, bar_pkfree, bar_vfree, bar_ma, bar_m2, bar_conv, bar_b, bar_d,
+  // loads (record pieces, value tiles); "free" signals for the loader; MMA
+  // commits; compute-warp hand-offs; output staging full / free
+  __shared__ uint64_t bar_a, bar_pk, bar_sc[2], bar_v, bar_pkfree, bar_vfree, bar_ma, bar_m2, bar_conv, bar_b,
       bar_ost[2], bar_ofree[2], bar_drain;
   __shared__ uint32_t tmem_base;
   __shared__ int s_abort;
@@ -88,9 +96,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
   if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
   if (tid == 0) {
     tc::bar_init(&bar_a, 1); tc::bar_init(&bar_pk, 1); tc::bar_init(&bar_v, 1);
+    tc::bar_init(&bar_sc[0], 1); tc::bar_init(&bar_sc[1], 1);
     tc::bar_init(&bar_pkfree, 1); tc::bar_init(&bar_vfree, SCAN_COMPUTE);
     tc::bar_init(&bar_ma, 1); tc::bar_init(&bar_m2, 1);
-    tc::bar_init(&bar_conv, SCAN_COMPUTE); tc::bar_init(&bar_b, SCAN_COMPUTE); tc::bar_init(&bar_d, SCAN_COMPUTE);
+    tc::bar_init(&bar_conv, SCAN_COMPUTE); tc::bar_init(&bar_b, SCAN_COMPUTE);
     tc::bar_init(&bar_ost[0], SCAN_COMPUTE); tc::bar_init(&bar_ost[1], SCAN_COMPUTE);
     tc::bar_init(&bar_ofree[0], 1); tc::bar_init(&bar_ofree[1], 1);
     tc::bar_init(&bar_drain, 1);
@@ -105,47 +114,41 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
   if (warp == 16) {
     // ======================= MMA-issuing thread =============================
     if (lane == 0) {
-      const uint64_t d_ra = tc::desc(tc::smem_u32(sm + SCAN_RA));
-      const uint64_t d_ts = tc::desc(tc::smem_u32(sm + SCAN_RA + REC_TS));
-      const uint64_t d_ps = tc::desc(tc::smem_u32(sm + SCAN_PK));
-      const uint64_t d_kb = tc::desc(tc::smem_u32(sm + SCAN_PK + (REC_KB - REC_PS)));
+      const uint64_t d_ra = tc::desc(tc::smem_u32(sm + SCAN_A + REC_RA));
+      const uint64_t d_ts = tc::desc(tc::smem_u32(sm + SCAN_A + REC_TS));
+      const uint64_t d_b2 = tc::desc(tc::smem_u32(sm + SCAN_B));
       bool ok = true;
       for (int i = 0; i < nchunks && ok; ++i) {
         const uint32_t p = i & 1;
         // V_i in TMEM (and the output of chunk i - 2 read from the O^T buffer
-        // of this parity); the first record piece of chunk i in shared memory
+        // of this parity); the first record piece of chunk i in shared memory;
+        // the state of chunk i complete (MMA2 of chunk i - 1 done)
         ok = tc::bar_wait_or(&bar_conv, p, abort_flag, wait_ns);
         ok = ok && tc::bar_wait_or(&bar_a, p, abort_flag, wait_ns);
+        if (i > 0) ok = ok && tc::bar_wait_or(&bar_m2, p ^ 1, abort_flag, wait_ns);
         if (!ok) break;
         tc::fence_after();
-        // [U^T | O^T] = S^T [-W ; Q~]^T, then U^T += V^T T_s^T
         const uint32_t dA = tm + (p ? TM_O1 : TM_U);
+        const uint32_t sA = tm + s_col(i);
 #pragma unroll
         for (int ks = 0; ks < 16; ++ks)
-          tc::mma_ts(dA, tm + TM_S + 8 * ks, d_ra + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), ks > 0);
+          tc::mma_ts(dA, sA + 8 * ks, d_ra + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, d_ts + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
         tc::commit(&bar_ma);
-        // O^T += U^T P_s^T as soon as U^T is final
+        // [O^T | S(1)] or [S(0) | O^T] += U'^T B2 once U' is final and the
+        // decayed state is in place
         ok = tc::bar_wait_or(&bar_b, p, abort_flag, wait_ns);
         ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag, wait_ns);
         if (!ok) break;
         tc::fence_after();
-        const uint32_t dO = tm + o_col(i);
+        const uint32_t d2 = tm + (p ? TM_S0 : TM_O0);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          tc::mma_ts(dO, tm + TM_U + 8 * ks, d_ps + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
-        // S^T += U^T K-bar once S^T diag(gamma) is in place
-        ok = tc::bar_wait_or(&bar_d, p, abort_flag, wait_ns);
-        if (!ok) break;
-        tc::fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          tc::mma_ts(tm + TM_S, tm + TM_U + 8 * ks, d_kb + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), 1);
+          tc::mma_ts(d2, tm + TM_U + 8 * ks, d_b2 + tc::desc_step(B2_ROWS, ks), tc::idesc_tf32(128, 192), 1);
         tc::commit(&bar_m2);
         tc::commit(&bar_pkfree);
-        ok = tc::bar_wait_or(&bar_m2, p, abort_flag, wait_ns);  // S^T complete for the next chunk
       }
       if (!ok) {
         s_abort = 1;
@@ -155,61 +158,90 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       }
     }
   } else if (warp == 17) {
-    // ======================= load-issuing thread ============================
-    if (lane == 0) {
-      int n_a = 0, n_pk = 0, n_v = 0;  // loads issued per barrier, for the drain
-      auto load_a = [&](int i) {  // [-W ; Q~] and T_s
-        tc::bar_expect_tx(&bar_a, REC_TILES_A);
-        tc::bulk_g2s(sm + SCAN_RA, rec0 + (int64_t)i * rec_stride, REC_TILES_A, &bar_a);
-        ++n_a;
-      };
-      auto load_pk = [&](int i) {  // P_s, K-bar, scalars
-        tc::bar_expect_tx(&bar_pk, PK_BYTES);
-        tc::bulk_g2s(sm + SCAN_PK, rec0 + (int64_t)i * rec_stride + REC_PS, PK_BYTES, &bar_pk);
-        ++n_pk;
-      };
-      auto load_v = [&](int i) {  // rows t0 - 3 .. t0 + 63 of this head's value columns
+    // ======================= loads and L2 drops =============================
+    // Every lane runs the loop (waits are read-only polls); lane 0 issues the
+    // loads, all lanes drop consumed record lines.
+    const bool leader = lane == 0;
+    int n_a = 0, n_pk = 0, n_v = 0;  // loads issued per barrier, for the drain
+    auto load_a = [&](int i) {  // RA and TS; the scalars into their buffer of i's parity
+      if (leader) {
+        const uint8_t* r = rec0 + (int64_t)i * rec_stride;
+        tc::bar_expect_tx(&bar_a, REC_PIECE_A);
+        tc::bulk_g2s(sm + SCAN_A, r, REC_PIECE_A, &bar_a);
+        tc::bar_expect_tx(&bar_sc[i & 1], SC_BYTES);
+        tc::bulk_g2s(sm + SCAN_SC + (i & 1) * SC_BYTES, r + REC_SC, SC_BYTES, &bar_sc[i & 1]);
+      }
+      ++n_a;
+    };
+    auto load_pk = [&](int i) {  // B2
+      if (leader) {
+        tc::bar_expect_tx(&bar_pk, B2_BYTES);
+        tc::bulk_g2s(sm + SCAN_B, rec0 + (int64_t)i * rec_stride + REC_B2, B2_BYTES, &bar_pk);
+      }
+      ++n_pk;
+    };
+    auto load_v = [&](int i) {  // rows t0 - 3 .. t0 + 63 of this head's value columns
+      if (leader) {
         tc::bar_expect_tx(&bar_v, RAW_BYTES);
         tc::tma_load_2d(sm + SCAN_V, &tm_v, h * D, (int)(seg0 + (int64_t)CH * i - 3), &bar_v);
-        ++n_v;
-      };
-      // with the prep kernel running concurrently, a chunk's record is read
-      // only once its ready flag is published (flag of chunk j at rdy[j * H])
-      const int* rdy = ready ? ready + (int64_t)chunk_base[n] * H + h : nullptr;
-      auto record_ready = [&](int j) -> bool { return !rdy || tc::flag_wait_or(rdy + (int64_t)j * H, abort_flag, wait_ns); };
-      bool ok = true;
-      if (nchunks > 0) {
-        ok = record_ready(0);
-        if (ok) { load_a(0); load_v(0); load_pk(0); }
       }
-      if (ok && nchunks > 1) {  // the conv of chunk 0 has read value tile 0
-        ok = tc::bar_wait_or(&bar_vfree, 0, abort_flag, wait_ns);
-        if (ok) load_v(1);
+      ++n_v;
+    };
+    // a record piece that the tensor core has read is dead: drop its lines
+    auto drop = [&](const uint8_t* base, uint32_t bytes) {
+      for (uint32_t off = 128u * lane; off < bytes; off += 128u * 32u) discard_l2(base + off);
+    };
+    // with the prep kernel running concurrently, a chunk's record is read
+    // only once its ready flag is published (flag of chunk j at rdy[j * H])
+    const int* rdy = ready ? ready + (int64_t)chunk_base[n] * H + h : nullptr;
+    auto record_ready = [&](int j) -> bool {
+      return !rdy || tc::flag_wait_or(rdy + (int64_t)j * H, abort_flag, wait_ns);
+    };
+    auto all = [](bool x) { return __all_sync(0xffffffffu, x) != 0; };
+    bool ok = true;
+    if (nchunks > 0) {
+      ok = all(record_ready(0));
+      if (ok) { load_a(0); load_v(0); load_pk(0); }
+    }
+    if (ok && nchunks > 1) {  // the conv of chunk 0 has read value tile 0
+      ok = all(tc::bar_wait_or(&bar_vfree, 0, abort_flag, wait_ns));
+      if (ok) load_v(1);
+    }
+    // record pieces of chunk j as their buffers free up during chunk j - 1;
+    // value tile j + 1 once the conv of chunk j (done early in chunk j - 1)
+    // has read tile j
+    for (int j = 1; j < nchunks && ok; ++j) {
+      const uint32_t q = (j - 1) & 1;
+      const uint8_t* prev = rec0 + (int64_t)(j - 1) * rec_stride;
+      ok = all(tc::bar_wait_or(&bar_ma, q, abort_flag, wait_ns));  // MMA_A of chunk j - 1 read piece A
+      if (ok) drop(prev, REC_PIECE_A);
+      ok = ok && all(record_ready(j));
+      if (ok) load_a(j);
+      if (ok && j + 1 < nchunks) {
+        ok = all(tc::bar_wait_or(&bar_vfree, j & 1, abort_flag, wait_ns));
+        if (ok) load_v(j + 1);
       }
-      // record pieces of chunk j as their buffers free up during chunk j - 1;
-      // value tile j + 1 once the conv of chunk j (done early in chunk j - 1)
-      // has read tile j
-      for (int j = 1; j < nchunks && ok; ++j) {
-        const uint32_t q = (j - 1) & 1;
-        ok = tc::bar_wait_or(&bar_ma, q, abort_flag, wait_ns);  // MMA_A of chunk j - 1 has read the first piece
-        ok = ok && record_ready(j);
-        if (ok) load_a(j);
-        if (ok && j + 1 < nchunks) {
-          ok = tc::bar_wait_or(&bar_vfree, j & 1, abort_flag, wait_ns);
-          if (ok) load_v(j + 1);
-        }
-        ok = ok && tc::bar_wait_or(&bar_pkfree, q, abort_flag, wait_ns);  // MMA2 of chunk j - 1 has read the second
-        if (ok) load_pk(j);
+      ok = ok && all(tc::bar_wait_or(&bar_pkfree, q, abort_flag, wait_ns));  // MMA2 of chunk j - 1 read piece B
+      if (ok) {
+        drop(prev + REC_B2, REC_PIECE_B);
+        load_pk(j);
       }
-      if (!ok) {
-        s_abort = 1;
-        // every issued load lands before shared memory is released (each wait
-        // bounded; awaiting the phase of the last issued load returns at once
-        // if it already completed)
-        if (n_a) tc::bar_wait(&bar_a, (uint32_t)((n_a - 1) & 1));
-        if (n_pk) tc::bar_wait(&bar_pk, (uint32_t)((n_pk - 1) & 1));
-        if (n_v) tc::bar_wait(&bar_v, (uint32_t)((n_v - 1) & 1));
-      }
+    }
+    if (ok && nchunks > 0) {  // the last chunk's record
+      const uint8_t* last = rec0 + (int64_t)(nchunks - 1) * rec_stride;
+      ok = all(tc::bar_wait_or(&bar_pkfree, (nchunks - 1) & 1, abort_flag, wait_ns));
+      if (ok) drop(last, REC_BYTES);
+    }
+    if (!ok && leader) {
+      s_abort = 1;
+      // every issued load lands before shared memory is released (each wait
+      // bounded; awaiting the phase of the last issued load returns at once
+      // if it already completed)
+      if (n_a) tc::bar_wait(&bar_a, (uint32_t)((n_a - 1) & 1));
+      if (n_a) tc::bar_wait(&bar_sc[(n_a - 1) & 1], (uint32_t)(((n_a - 1) >> 1) & 1));
+      if (n_a > 1) tc::bar_wait(&bar_sc[n_a & 1], (uint32_t)(((n_a - 2) >> 1) & 1));
+      if (n_pk) tc::bar_wait(&bar_pk, (uint32_t)((n_pk - 1) & 1));
+      if (n_v) tc::bar_wait(&bar_v, (uint32_t)((n_v - 1) & 1));
     }
   } else if (warp == 18) {
     // ======================= output-storing thread ==========================
@@ -243,7 +275,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     const int k0 = 32 * part;                  // keys k0 .. k0 + 31
     const uint32_t tl = tm + ((uint32_t)(32 * q) << 16);
     const int64_t chan = (int64_t)h * D + v;
-    // initial state: row v of S^T = column v of S (key rows k0 ..)
+    // initial state: row v of S^T = column v of S (key rows k0 ..), into S0
     {
       const Ts* Si = init_state ? init_state + ((int64_t)n * H + h) * D * D + v : nullptr;
 #pragma unroll
@@ -251,11 +283,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         float s[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) s[j] = Si ? to_f(Si[(int64_t)(k0 + 16 * g16 + j) * D]) : 0.f;
-        tc::st16(tl + TM_S + k0 + 16 * g16, s);
+        tc::st16(tl + TM_S0 + k0 + 16 * g16, s);
       }
+      tc::st_wait();
     }
     const float4 wv = load4(conv_w + (2 * HD + chan) * 4);
-    const float* scal = reinterpret_cast<const float*>(sm + SCAN_PK + (REC_SC - REC_PS));
     // short conv of v for chunk i, tokens t0 .. t0 + 15, into registers (the
     // value tile is released as soon as it has been read)
     auto conv_v = [&](int i, float (&vv)[16]) -> bool {
@@ -289,21 +321,37 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       tc::bar_arrive(&bar_vfree);  // value tile i has been read
       return true;
     };
-    // V^T (tf32 MMA operand) and V^T fp32 of a chunk from its conv registers
+    // V^T of a chunk (tf32 MMA operand) from its conv registers
     auto store_v = [&](const float (&vv)[16]) {
       float r[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) r[j] = tc::to_tf32(vv[j]);
       tc::st16(tl + TM_V + t0, r);
-      tc::st16(tl + TM_VX + t0, vv);
+    };
+    // output of chunk c: o = r (O + d u'), into the staging tile of c's parity
+    // (free once the store of chunk c - 2 has read it)
+    auto output = [&](int c, const float (&rr)[16], const float (&du)[16]) -> bool {
+      const int b = c & 1;
+      if (c >= 2 && !tc::bar_wait_or(&bar_ofree[b], (uint32_t)(((c >> 1) - 1) & 1), abort_flag, wait_ns))
+        return false;
+      Tout* st = reinterpret_cast<Tout*>(sm + SCAN_OST + b * OST_BYTES);
+      float r[16];
+      tc::ld16(tl + (uint32_t)o_col(c) + t0, r);
+      tc::ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) st[(t0 + j) * D + v] = from_f<Tout>(rr[j] * (r[j] + du[j]));
+      tc::fence_async_smem();
+      tc::bar_arrive(&bar_ost[b]);
+      return true;
     };
 
     bool ok = true;
-    float vn[16];  // conv of the next chunk's values until its TMEM columns are free
+    float vcur[16];        // exact conv outputs of this chunk's values
+    float rr[16], du[16];  // r_t and d_t u'_t of the previous chunk, for its output
     if (nchunks > 0) {
-      ok = conv_v(0, vn);
+      ok = conv_v(0, vcur);
       if (ok) {
-        store_v(vn);
+        store_v(vcur);
         tc::st_wait();
         tc::fence_before();
         tc::bar_arrive(&bar_conv);
@@ -311,79 +359,77 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     }
     for (int i = 0; i < nchunks && ok; ++i) {
       const uint32_t p = i & 1;
-      const bool more = i + 1 < nchunks;
-      // (a) the next chunk's value conv while MMA_A of this chunk runs, then
-      //     U^T of this chunk (S^T read by the tensor core) and its scalars
-      if (more) ok = conv_v(i + 1, vn);
-      ok = ok && tc::bar_wait_or(&bar_ma, p, abort_flag, wait_ns);
-      ok = ok && tc::bar_wait_or(&bar_pk, p, abort_flag, wait_ns);
+      // (a) the previous chunk's output once MMA2 of it is done (its state
+      //     update, which is this chunk's state, is then complete too)
+      if (i > 0) {
+        ok = tc::bar_wait_or(&bar_m2, p ^ 1, abort_flag, wait_ns);
+        if (ok) {
+          tc::fence_after();
+          ok = output(i - 1, rr, du);
+        }
+      }
+      // (b) the decay into the other state buffer, S(1-p) = S(p) diag(gamma),
+      //     while MMA_A reads S(p); the chunk's scalars arrive with its first
+      //     record piece, in a buffer of their own
+      ok = ok && tc::bar_wait_or(&bar_sc[p], (uint32_t)((i >> 1) & 1), abort_flag, wait_ns);
+      if (!ok) break;
+      const float* scal = reinterpret_cast<const float*>(sm + SCAN_SC + p * SC_BYTES);
+#pragma unroll
+      for (int g16 = 0; g16 < 2; ++g16) {
+        float r[16];
+        tc::ld16(tl + (uint32_t)s_col(i) + k0 + 16 * g16, r);
+        tc::ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) r[j] *= scal[SC_G + k0 + 16 * g16 + j];
+        tc::st16(tl + (uint32_t)s_col(i + 1) + k0 + 16 * g16, r);
+      }
+      // (c) U' += b V (the exact diagonal of Dk T V); keep d u' and r
+      ok = tc::bar_wait_or(&bar_ma, p, abort_flag, wait_ns);
       if (!ok) break;
       tc::fence_after();
-      // (b) U += beta V (exact diagonal of T V); P_tt U kept in fp32
       {
-        float r[16], vx[16];
+        float r[16];
         tc::ld16(tl + TM_U + t0, r);
-        tc::ld16(tl + TM_VX + t0, vx);
         tc::ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float u = fmaf(scal[t0 + j], vx[j], r[j]);
+          const float u = fmaf(scal[SC_B + t0 + j], vcur[j], r[j]);
           r[j] = tc::to_tf32(u);
-          vx[j] = scal[64 + t0 + j] * u;
+          du[j] = scal[SC_D + t0 + j] * u;
+          rr[j] = scal[SC_R + t0 + j];
         }
         tc::st16(tl + TM_U + t0, r);
-        tc::st16(tl + TM_UP + t0, vx);
       }
       tc::st_wait();
       tc::fence_before();
       tc::bar_arrive(&bar_b);
-      // V^T of the next chunk: MMA_A of this chunk has read V^T, and V^T fp32
-      // was read just above
-      if (more) store_v(vn);
-      // (c) S^T <- S^T diag(gamma) while O^T += U^T P_s^T runs
-      {
-        float r0[16], r1[16];
-        tc::ld16(tl + TM_S + k0, r0);
-        tc::ld16(tl + TM_S + k0 + 16, r1);
-        tc::ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          r0[j] *= scal[128 + k0 + j];
-          r1[j] *= scal[128 + k0 + 16 + j];
-        }
-        tc::st16(tl + TM_S + k0, r0);
-        tc::st16(tl + TM_S + k0 + 16, r1);
+      // (d) the next chunk's value conv and V^T while MMA2 runs (MMA_A of this
+      //     chunk has read V^T)
+      if (i + 1 < nchunks) {
+        ok = conv_v(i + 1, vcur);
+        if (!ok) break;
+        store_v(vcur);
+        tc::st_wait();
+        tc::fence_before();
+        tc::bar_arrive(&bar_conv);
       }
-      tc::st_wait();
-      tc::fence_before();
-      tc::bar_arrive(&bar_d);
-      if (more) tc::bar_arrive(&bar_conv);
-      // (e) o = O + P_tt u once MMA2 is done, into the staging tile of this
-      // parity (free once the store of chunk i - 2 has read it)
-      ok = ok && tc::bar_wait_or(&bar_m2, p, abort_flag, wait_ns);
-      if (ok && i >= 2) ok = tc::bar_wait_or(&bar_ofree[p], (uint32_t)(((i >> 1) - 1) & 1), abort_flag, wait_ns);
-      if (!ok) break;
-      tc::fence_after();
-      {
-        Tout* st = reinterpret_cast<Tout*>(sm + SCAN_OST + p * OST_BYTES);
-        float r[16], up[16];
-        tc::ld16(tl + (uint32_t)o_col(i) + t0, r);
-        tc::ld16(tl + TM_UP + t0, up);
-        tc::ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) st[(t0 + j) * D + v] = from_f<Tout>(r[j] + up[j]);
+    }
+    // the last chunk's output; then the final state S(nchunks % 2)
+    if (ok && nchunks > 0) {
+      ok = tc::bar_wait_or(&bar_m2, (nchunks - 1) & 1, abort_flag, wait_ns);
+      if (ok) {
+        tc::fence_after();
+        ok = output(nchunks - 1, rr, du);
       }
-      tc::fence_async_smem();
-      tc::bar_arrive(&bar_ost[p]);
     }
     if (!ok) s_abort = 1;
-    // final state: column v of S = row v of S^T
     if (ok) {
+      // column v of S = row v of S^T
       Ts* Sf = final_state + ((int64_t)n * H + h) * D * D + v;
 #pragma unroll
       for (int g16 = 0; g16 < 2; ++g16) {
         float s[16];
-        tc::ld16(tl + TM_S + k0 + 16 * g16, s);
+        tc::ld16(tl + (uint32_t)s_col(nchunks) + k0 + 16 * g16, s);
         tc::ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) Sf[(int64_t)(k0 + 16 * g16 + j) * D] = from_f<Ts>(s[j]);

@@ -39,9 +39,12 @@ inline size_t chunk_header_bytes(int N, int64_t nchunks) {
 inline size_t chunk_sync_bytes(int64_t nchunks, int H) {
   return ((size_t)16 + (size_t)nchunks * H * 4 + 1023) & ~(size_t)1023;
 }
+// (+128: the records start on a 128-byte line whatever the workspace's
+// 16-byte alignment, so that the scan can drop whole lines of a consumed
+// record from L2)
 inline size_t chunked_workspace_bytes(int N, int H, int64_t total_tokens) {
   const int64_t nc = chunk_bound(N, total_tokens);
-  return chunk_header_bytes(N, nc) + chunk_sync_bytes(nc, H) + (size_t)nc * H * REC_BYTES;
+  return chunk_header_bytes(N, nc) + chunk_sync_bytes(nc, H) + 128 + (size_t)nc * H * REC_BYTES;
 }
 
 constexpr int OVERLAP_MAX_CHAINS = 96;  // leaves at least 52 of 148 SMs to prep
@@ -78,16 +81,16 @@ inline OverlapStreams& overlap_streams() {
 inline kda_status fork_side(cudaStream_t stream, cudaStream_t* side, cudaEvent_t* join) {
   OverlapStreams& o = overlap_streams();
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KDA_ERR_CUDA;
+  if (!cuda_ok(cudaGetDevice(&dev)) || dev < 0 || dev >= 64) return KDA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(o.mu);
   if (!o.streams[dev]) {
-    if (cudaStreamCreateWithFlags(&o.streams[dev], cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&o.forks[dev], cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&o.joins[dev], cudaEventDisableTiming) != cudaSuccess)
+    if (!cuda_ok(cudaStreamCreateWithFlags(&o.streams[dev], cudaStreamNonBlocking)) ||
+        !cuda_ok(cudaEventCreateWithFlags(&o.forks[dev], cudaEventDisableTiming)) ||
+        !cuda_ok(cudaEventCreateWithFlags(&o.joins[dev], cudaEventDisableTiming)))
       return KDA_ERR_CUDA;
   }
-  if (cudaEventRecord(o.forks[dev], stream) != cudaSuccess ||
-      cudaStreamWaitEvent(o.streams[dev], o.forks[dev], 0) != cudaSuccess)
+  if (!cuda_ok(cudaEventRecord(o.forks[dev], stream)) ||
+      !cuda_ok(cudaStreamWaitEvent(o.streams[dev], o.forks[dev], 0)))
     return KDA_ERR_CUDA;
   *side = o.streams[dev];
   *join = o.joins[dev];
@@ -96,7 +99,7 @@ inline kda_status fork_side(cudaStream_t stream, cudaStream_t* side, cudaEvent_t
 // The join is recorded and awaited under the same lock for the same reason.
 inline kda_status join_side(cudaStream_t stream, cudaStream_t side, cudaEvent_t join) {
   std::lock_guard<std::mutex> lock(overlap_streams().mu);
-  if (cudaEventRecord(join, side) != cudaSuccess || cudaStreamWaitEvent(stream, join, 0) != cudaSuccess)
+  if (!cuda_ok(cudaEventRecord(join, side)) || !cuda_ok(cudaStreamWaitEvent(stream, join, 0)))
     return KDA_ERR_CUDA;
   return KDA_OK;
 }
@@ -119,7 +122,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   // releases on return; a captured graph would read it again on every replay,
   // long after it is gone, so stream capture is refused.
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return KDA_ERR_CUDA;
+  if (!cuda_ok(cudaStreamIsCapturing(stream, &cap))) return KDA_ERR_CUDA;
   if (cap != cudaStreamCaptureStatusNone) return KDA_ERR_UNSUPPORTED;
   // chunk table and longest-first segment order
   std::vector<int64_t> nch(N);
@@ -144,7 +147,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   // pageable source: the call returns after the bytes are staged, so `host`
   // may be released right after
-  if (cudaMemcpyAsync(ws, host.data(), hdr, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+  if (!cuda_ok(cudaMemcpyAsync(ws, host.data(), hdr, cudaMemcpyHostToDevice, stream)))
     return KDA_ERR_CUDA;
   const int2* d_tab = reinterpret_cast<const int2*>(ws);
   const int32_t* d_base = reinterpret_cast<const int32_t*>(ws + (size_t)total * sizeof(int2));
@@ -152,7 +155,8 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   int* work_counter = reinterpret_cast<int*>(ws + hdr);
   int* ready = work_counter + 4;
   uint8_t* records = ws + hdr + chunk_sync_bytes(total, H);
-  if (cudaMemsetAsync(work_counter, 0, 16 + (size_t)total * H * 4, stream) != cudaSuccess) return KDA_ERR_CUDA;
+  records += (128 - (reinterpret_cast<uintptr_t>(records) & 127)) & 127;
+  if (!cuda_ok(cudaMemsetAsync(work_counter, 0, 16 + (size_t)total * H * 4, stream))) return KDA_ERR_CUDA;
   const int64_t items = total * H;
   const bool overlap = items > 0 && (int64_t)N * H <= OVERLAP_MAX_CHAINS;
 
@@ -173,12 +177,12 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   }
   if (total > 0) {
     auto prep = chunk_prep_kernel<ACT>;
-    if (cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM) != cudaSuccess)
+    if (!cuda_ok(cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM)))
       return KDA_ERR_CUDA;
     // persistent blocks, two per SM, over the (chunk, head) items
     int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    if (!cuda_ok(cudaGetDevice(&dev)) ||
+        !cuda_ok(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)))
       return KDA_ERR_CUDA;
     const unsigned blocks = (unsigned)(items < 2 * sms ? items : 2 * sms);
     int vacate_sms = 0, vacate_after = (int)items;
@@ -196,17 +200,18 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     // an injected KDA_FAULT_DROP_READY drops the publication of the flags the
     // scan waits on
     int* publish = overlap && !take_fault(KDA_FAULT_DROP_READY) ? ready : nullptr;
-    prep<<<blocks, PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w, (const T*)init_conv,
-                                                        cu_dev, d_tab, H, (int)items, records, work_counter,
-                                                        publish, vacate_sms, vacate_after);
-    if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    prep<<<blocks, PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)q, (const T*)k, (const T*)g,
+                                                        (const T*)beta, conv_w, (const T*)init_conv, cu_dev, d_tab,
+                                                        H, (int)items, records, work_counter, publish, vacate_sms,
+                                                        vacate_after);
+    if (!cuda_ok(cudaGetLastError())) return KDA_ERR_CUDA;
   }
   // the scan, instantiated for the output and state element types
   auto launch_scan = [&](auto tout, auto ts) -> bool {
     using Tout = decltype(tout);
     using Ts = decltype(ts);
     auto scan = chunk_scan_kernel<Tout, ACT, Ts>;
-    if (cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM) != cudaSuccess)
+    if (!cuda_ok(cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM)))
       return false;
     scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, scan_stream>>>(
         tv, to, conv_w, (const Ts*)init_state, (const T*)init_conv, cu_dev, d_base, d_order, H, records,
@@ -218,7 +223,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     ok = state_dt == KDA_F32 ? launch_scan(float{}, float{}) : launch_scan(float{}, T{});
   else
     ok = state_dt == KDA_F32 ? launch_scan(T{}, float{}) : launch_scan(T{}, T{});
-  if (!ok || cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+  if (!ok || !cuda_ok(cudaGetLastError())) return KDA_ERR_CUDA;
   if (overlap && join_side(stream, side, join) != KDA_OK) return KDA_ERR_CUDA;
   return KDA_OK;
 }

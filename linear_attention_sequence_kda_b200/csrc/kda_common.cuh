@@ -19,6 +19,15 @@ __device__ int g_status;
 
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// The CUDA error behind the last KDA_ERR_CUDA returned on this host thread
+// (kda_last_cuda_error); every host-side CUDA call is checked through cuda_ok.
+inline thread_local int t_last_cuda_error = 0;
+inline bool cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return true;
+  t_last_cuda_error = (int)e;
+  return false;
+}
+
 // ---- element loads/stores in either dtype, converted to/from fp32 ----------
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -66,6 +75,14 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   float2 d;
   asm("{\n.reg .b64 a, b, d;\nmov.b64 a, {%2, %3};\nmov.b64 b, {%4, %5};\n"
       "mul.rn.f32x2 d, a, b;\nmov.b64 {%0, %1}, d;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n.reg .b64 a, b, d;\nmov.b64 a, {%2, %3};\nmov.b64 b, {%4, %5};\n"
+      "add.rn.f32x2 d, a, b;\nmov.b64 {%0, %1}, d;\n}"
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
