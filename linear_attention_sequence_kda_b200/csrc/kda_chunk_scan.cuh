@@ -79,8 +79,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
   uint8_t* sm = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   // loads (record pieces, value tiles); "free" signals for the loader; MMA
   // commits; compute-warp hand-offs; output staging full / free
-  __shared__ uint64_t bar_a, bar_pk, bar_sc[2], bar_v, bar_pkfree, bar_vfree, bar_ma, bar_m2, bar_conv, bar_b,
-      bar_ost[2], bar_ofree[2], bar_drain;
+  // bar_ra[s]: slab s of the first record piece (s < 4: 32 key columns of RA,
+  // s = 4: TS) has landed; bar_rafree[s]: the products that read it are done
+  __shared__ uint64_t bar_ra[5], bar_rafree[5], bar_pk, bar_sc[2], bar_v, bar_pkfree, bar_vfree, bar_ma, bar_m2,
+      bar_conv, bar_b, bar_ost[2], bar_ofree[2], bar_drain;
   __shared__ uint32_t tmem_base;
   __shared__ int s_abort;
 
@@ -95,7 +97,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
 
   if (warp == 0) tc::tmem_alloc(&tmem_base, 512);
   if (tid == 0) {
-    tc::bar_init(&bar_a, 1); tc::bar_init(&bar_pk, 1); tc::bar_init(&bar_v, 1);
+    for (int j = 0; j < 5; ++j) { tc::bar_init(&bar_ra[j], 1); tc::bar_init(&bar_rafree[j], 1); }
+    tc::bar_init(&bar_pk, 1); tc::bar_init(&bar_v, 1);
     tc::bar_init(&bar_sc[0], 1); tc::bar_init(&bar_sc[1], 1);
     tc::bar_init(&bar_pkfree, 1); tc::bar_init(&bar_vfree, SCAN_COMPUTE);
     tc::bar_init(&bar_ma, 1); tc::bar_init(&bar_m2, 1);
@@ -124,18 +127,31 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         // of this parity); the first record piece of chunk i in shared memory;
         // the state of chunk i complete (MMA2 of chunk i - 1 done)
         ok = tc::bar_wait_or(&bar_conv, p, abort_flag, wait_ns);
-        ok = ok && tc::bar_wait_or(&bar_a, p, abort_flag, wait_ns);
         if (i > 0) ok = ok && tc::bar_wait_or(&bar_m2, p ^ 1, abort_flag, wait_ns);
         if (!ok) break;
-        tc::fence_after();
         const uint32_t dA = tm + (p ? TM_O1 : TM_U);
         const uint32_t sA = tm + s_col(i);
+        // slab by slab as the record arrives; each slab is handed back to the
+        // loader as soon as the products that read it are done
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks)
-          tc::mma_ts(dA, sA + 8 * ks, d_ra + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), ks > 0);
+        for (int sl = 0; sl < 4 && ok; ++sl) {
+          ok = tc::bar_wait_or(&bar_ra[sl], p, abort_flag, wait_ns);
+          if (!ok) break;
+          tc::fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int ks = 4 * sl + kk;
+            tc::mma_ts(dA, sA + 8 * ks, d_ra + tc::desc_step(128, ks), tc::idesc_tf32(128, 128), ks > 0);
+          }
+          tc::commit(&bar_rafree[sl]);
+        }
+        ok = ok && tc::bar_wait_or(&bar_ra[4], p, abort_flag, wait_ns);
+        if (!ok) break;
+        tc::fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           tc::mma_ts(tm + TM_U, tm + TM_V + 8 * ks, d_ts + tc::desc_step(64, ks), tc::idesc_tf32(128, 64), 1);
+        tc::commit(&bar_rafree[4]);
         tc::commit(&bar_ma);
         // [O^T | S(1)] or [S(0) | O^T] += U'^T B2 once U' is final and the
         // decayed state is in place
@@ -162,16 +178,20 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     // Every lane runs the loop (waits are read-only polls); lane 0 issues the
     // loads, all lanes drop consumed record lines.
     const bool leader = lane == 0;
-    int n_a = 0, n_pk = 0, n_v = 0;  // loads issued per barrier, for the drain
-    auto load_a = [&](int i) {  // RA and TS; the scalars into their buffer of i's parity
+    int n_sl[5] = {0, 0, 0, 0, 0}, n_pk = 0, n_v = 0;  // loads issued per barrier, for the drain
+    // slab sl (16 KB) of the first record piece of chunk i: RA columns
+    // 32 sl .. (sl < 4) or TS (sl = 4); the scalars travel with slab 0
+    auto load_slab = [&](int i, int sl) {
       if (leader) {
         const uint8_t* r = rec0 + (int64_t)i * rec_stride;
-        tc::bar_expect_tx(&bar_a, REC_PIECE_A);
-        tc::bulk_g2s(sm + SCAN_A, r, REC_PIECE_A, &bar_a);
-        tc::bar_expect_tx(&bar_sc[i & 1], SC_BYTES);
-        tc::bulk_g2s(sm + SCAN_SC + (i & 1) * SC_BYTES, r + REC_SC, SC_BYTES, &bar_sc[i & 1]);
+        tc::bar_expect_tx(&bar_ra[sl], 16384);
+        tc::bulk_g2s(sm + SCAN_A + sl * 16384, r + sl * 16384, 16384, &bar_ra[sl]);
+        if (sl == 0) {
+          tc::bar_expect_tx(&bar_sc[i & 1], SC_BYTES);
+          tc::bulk_g2s(sm + SCAN_SC + (i & 1) * SC_BYTES, r + REC_SC, SC_BYTES, &bar_sc[i & 1]);
+        }
       }
-      ++n_a;
+      ++n_sl[sl];
     };
     auto load_pk = [&](int i) {  // B2
       if (leader) {
@@ -198,25 +218,43 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       return !rdy || tc::flag_wait_or(rdy + (int64_t)j * H, abort_flag, wait_ns);
     };
     auto all = [](bool x) { return __all_sync(0xffffffffu, x) != 0; };
+    // start the record of chunk j on its way into L2 (two chunks ahead of its
+    // load), so that its bulk copies wait on L2 rather than HBM; a record the
+    // preparation kernel has not published yet is left alone
+    auto warm = [&](int j) {
+      if (leader && j < nchunks && (!rdy || *reinterpret_cast<const volatile int*>(rdy + (int64_t)j * H)))
+        tc::prefetch_l2(rec0 + (int64_t)j * rec_stride, REC_BYTES);
+    };
     bool ok = true;
     if (nchunks > 0) {
       ok = all(record_ready(0));
-      if (ok) { load_a(0); load_v(0); load_pk(0); }
+      if (ok) {
+        for (int sl = 0; sl < 5; ++sl) load_slab(0, sl);
+        load_v(0);
+        load_pk(0);
+        warm(1);
+        warm(2);
+      }
     }
     if (ok && nchunks > 1) {  // the conv of chunk 0 has read value tile 0
       ok = all(tc::bar_wait_or(&bar_vfree, 0, abort_flag, wait_ns));
       if (ok) load_v(1);
     }
-    // record pieces of chunk j as their buffers free up during chunk j - 1;
-    // value tile j + 1 once the conv of chunk j (done early in chunk j - 1)
-    // has read tile j
+    // the slabs of chunk j's first piece one by one as the products of chunk
+    // j - 1 release them; value tile j + 1 once the conv of chunk j has read
+    // tile j; the second piece once MMA2 of chunk j - 1 has read it
     for (int j = 1; j < nchunks && ok; ++j) {
       const uint32_t q = (j - 1) & 1;
       const uint8_t* prev = rec0 + (int64_t)(j - 1) * rec_stride;
-      ok = all(tc::bar_wait_or(&bar_ma, q, abort_flag, wait_ns));  // MMA_A of chunk j - 1 read piece A
-      if (ok) drop(prev, REC_PIECE_A);
-      ok = ok && all(record_ready(j));
-      if (ok) load_a(j);
+      ok = all(record_ready(j));
+      for (int sl = 0; sl < 5 && ok; ++sl) {
+        ok = all(tc::bar_wait_or(&bar_rafree[sl], q, abort_flag, wait_ns));
+        if (ok) load_slab(j, sl);
+      }
+      if (ok) {
+        drop(prev, REC_PIECE_A);
+        warm(j + 2);
+      }
       if (ok && j + 1 < nchunks) {
         ok = all(tc::bar_wait_or(&bar_vfree, j & 1, abort_flag, wait_ns));
         if (ok) load_v(j + 1);
@@ -237,9 +275,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       // every issued load lands before shared memory is released (each wait
       // bounded; awaiting the phase of the last issued load returns at once
       // if it already completed)
-      if (n_a) tc::bar_wait(&bar_a, (uint32_t)((n_a - 1) & 1));
-      if (n_a) tc::bar_wait(&bar_sc[(n_a - 1) & 1], (uint32_t)(((n_a - 1) >> 1) & 1));
-      if (n_a > 1) tc::bar_wait(&bar_sc[n_a & 1], (uint32_t)(((n_a - 2) >> 1) & 1));
+      for (int sl = 0; sl < 5; ++sl)
+        if (n_sl[sl]) tc::bar_wait(&bar_ra[sl], (uint32_t)((n_sl[sl] - 1) & 1));
+      if (n_sl[0]) tc::bar_wait(&bar_sc[(n_sl[0] - 1) & 1], (uint32_t)(((n_sl[0] - 1) >> 1) & 1));
+      if (n_sl[0] > 1) tc::bar_wait(&bar_sc[n_sl[0] & 1], (uint32_t)(((n_sl[0] - 2) >> 1) & 1));
       if (n_pk) tc::bar_wait(&bar_pk, (uint32_t)((n_pk - 1) & 1));
       if (n_v) tc::bar_wait(&bar_v, (uint32_t)((n_v - 1) & 1));
     }

@@ -52,7 +52,7 @@ constexpr int OVERLAP_MAX_CHAINS = 96;  // leaves at least 52 of 148 SMs to prep
 // chain, used to pick when prep hands SMs over to the scan (the ratio that
 // gave the shortest overlapped call on B200, 64 heads x 65,536 tokens, among
 // 2.8 .. 4.4; the model value from the two kernels' separate timings is ~3).
-constexpr double PREP_PER_SCAN_CHUNK = 2.8;
+constexpr double PREP_PER_SCAN_CHUNK = 3.2;
 
 // Pending host-side fault (kda_inject_fault), taken by the first call that
 // applies it.
@@ -200,10 +200,9 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     // an injected KDA_FAULT_DROP_READY drops the publication of the flags the
     // scan waits on
     int* publish = overlap && !take_fault(KDA_FAULT_DROP_READY) ? ready : nullptr;
-    prep<<<blocks, PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)q, (const T*)k, (const T*)g,
-                                                        (const T*)beta, conv_w, (const T*)init_conv, cu_dev, d_tab,
-                                                        H, (int)items, records, work_counter, publish, vacate_sms,
-                                                        vacate_after);
+    prep<<<blocks, PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w, (const T*)init_conv,
+                                                        cu_dev, d_tab, H, (int)items, records, work_counter,
+                                                        publish, vacate_sms, vacate_after);
     if (!cuda_ok(cudaGetLastError())) return KDA_ERR_CUDA;
   }
   // the scan, instantiated for the output and state element types
