@@ -36,6 +36,7 @@ from typing import Dict, Iterable, Optional, Tuple
 import numpy as np
 import torch
 
+from . import epilogue  # noqa: F401  (re-exported)
 from . import forms  # noqa: F401  (re-exported)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
