@@ -49,6 +49,7 @@ H, D, T_LONG = 64, 128, 65536
 BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 2 + D * 2
 BYTES_PER_TOKEN_HEAD_O32 = 4 * D * 2 + 2 + D * 4
 STATE_BYTES = D * D * 4
+GATE_BYTES_PER_TOKEN_HEAD = D * 2  # the output epilogue's gate z (bf16)
 # Useful tensor work of the chunked prefill per token-head: the state products
 # (6 K V) and the intra-chunk products (7 C K), C = 64.
 FLOP_PER_TOKEN_HEAD = 6 * D * D + 7 * 64 * D
@@ -424,6 +425,8 @@ def main():
                                                        args.steps, hbm_peak, bf16_peak, peak_src)[0]
         other_legs["prefill_varlen"] = run_prefill_leg(args, world, dev, stream, kda, ki.workload(3),
                                                        max(3, args.steps // 2), hbm_peak, bf16_peak, peak_src)[0]
+        other_legs["prefill_long_gated"] = run_prefill_leg(args, world, dev, stream, kda, inp, args.steps,
+                                                           hbm_peak, bf16_peak, peak_src, gated=True)[0]
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -457,15 +460,18 @@ def main():
         dist.destroy_process_group()
 
 
-def prefill_roofline(inp, launch_ms, hbm_peak, bf16_peak, peak_src, traffic, kernel_name):
+def prefill_roofline(inp, launch_ms, hbm_peak, bf16_peak, peak_src, traffic, kernel_name, gated=False):
     """HBM roofline of one kda_prefill on the method's bytes (1,282 B per
     token-head + initial and final state per (sequence, head)), the variant
     with o as the library writes it (fp32), and the tensor-pipe fraction of the
-    useful chunked work against the tf32 peak."""
+    useful chunked work against the tf32 peak.  With the fused output
+    epilogue the gate adds 256 B per token-head and o is written in bf16, as
+    the method's bytes already count it."""
     tok_heads = inp.total_tokens * inp.num_heads
     pairs = inp.num_seqs * inp.num_heads
-    alg = tok_heads * BYTES_PER_TOKEN_HEAD + pairs * 2 * STATE_BYTES
-    alg32 = tok_heads * BYTES_PER_TOKEN_HEAD_O32 + pairs * 2 * STATE_BYTES
+    extra = GATE_BYTES_PER_TOKEN_HEAD if gated else 0
+    alg = tok_heads * (BYTES_PER_TOKEN_HEAD + extra) + pairs * 2 * STATE_BYTES
+    alg32 = alg if gated else tok_heads * BYTES_PER_TOKEN_HEAD_O32 + pairs * 2 * STATE_BYTES
     sec = launch_ms / 1e3
     achieved = alg / sec / 1e9
     flops = tok_heads * FLOP_PER_TOKEN_HEAD
@@ -473,26 +479,33 @@ def prefill_roofline(inp, launch_ms, hbm_peak, bf16_peak, peak_src, traffic, ker
     roof = {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
             "frac": achieved / hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst)", "traffic": traffic,
             "algorithmic_bytes_per_launch": alg, "launch_ms": launch_ms,
-            "o_fp32_variant": {"algorithmic_bytes_per_launch": alg32, "achieved": alg32 / sec / 1e9,
-                               "frac": alg32 / sec / 1e9 / hbm_peak,
-                               "note": "same call, o counted as written (fp32, 512 B per token-head)"}}
+            "o_fp32_variant": None if gated else {
+                "algorithmic_bytes_per_launch": alg32, "achieved": alg32 / sec / 1e9,
+                "frac": alg32 / sec / 1e9 / hbm_peak,
+                "note": "same call, o counted as written (fp32, 512 B per token-head)"}}
     tensor = {"bound": "tensor", "achieved": flops / sec / 1e12, "peak": tf32_peak, "unit": "TFLOP/s",
               "frac": flops / sec / 1e12 / tf32_peak, "flop_per_launch": flops,
               "peak_source": f"{peak_src} bf16_tflops x {TF32_PER_BF16} (nominal tf32 : bf16)"}
     return roof, tensor
 
 
-def run_prefill_leg(args, world, dev, stream, kda, inp, steps, hbm_peak, bf16_peak, peak_src, keep=False):
-    """Times kda_prefill on one workload with its inputs resident in HBM:
-    W warm-up calls, then `steps` calls between barrier + synchronize, a CUDA
-    event pair per call on the launching stream."""
+def run_prefill_leg(args, world, dev, stream, kda, inp, steps, hbm_peak, bf16_peak, peak_src, keep=False,
+                    gated=False):
+    """Times kda_prefill (kda_prefill_gated with `gated`: the output epilogue
+    fused, synthetic gate and norm weight, bf16 output) on one workload with
+    its inputs resident in HBM: W warm-up calls, then `steps` calls between
+    barrier + synchronize, a CUDA event pair per call on the launching stream."""
     d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "g", "beta", "conv_w")}
     init_state = None if inp.init_state is None else inp.init_state.to(dev)
     init_conv = None if inp.init_conv is None else inp.init_conv.to(dev)
     cu_dev = torch.from_numpy(inp.cu_seqlens).to(dev)
     N, Hh = inp.num_seqs, inp.num_heads
-    o = torch.empty(d["q"].shape, dtype=torch.float32, device=dev)
+    o = torch.empty(d["q"].shape, dtype=torch.bfloat16 if gated else torch.float32, device=dev)
     S = torch.empty((N, Hh, D, D), dtype=torch.float32, device=dev)
+    norm = {}
+    if gated:
+        z, w = ki.make_output_norm(inp.total_tokens, Hh, ki.BASE_SEED + 2)
+        norm = {"gate": z.to(dev), "norm_weight": w.to(dev), "norm_eps": 1e-6}
     tail = torch.empty((N, 3, 3, Hh * D), dtype=torch.bfloat16, device=dev)
     max_len = int(np.diff(inp.cu_seqlens).max()) if N else 0
     ws_bytes = kda.workspace_size(N, inp.total_tokens, Hh, max_len)
@@ -500,19 +513,21 @@ def run_prefill_leg(args, world, dev, stream, kda, inp, steps, hbm_peak, bf16_pe
 
     def prefill_into(dd, oo, ss):
         kda.prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["conv_w"], inp.cu_seqlens, cu_dev,
-                    init_state, init_conv, o=oo, final_state=ss, conv_tail=tail, workspace=ws, stream=stream)
+                    init_state, init_conv, o=oo, final_state=ss, conv_tail=tail, workspace=ws, stream=stream,
+                    **norm)
 
     total_ms, per_step = timed(lambda: prefill_into(d, o, S), steps, args.warmup, world, stream)
     assert kda.check_async_status(stream) == 0
     launch_ms = statistics.mean(per_step)
-    kernel_name = "kda_prefill (chunk_prep_kernel + chunk_scan_kernel)"
+    kernel_name = ("kda_prefill_gated" if gated else "kda_prefill") + " (chunk_prep_kernel + chunk_scan_kernel)"
     chains = N * Hh
     label = "prefill_long" if (N, inp.total_tokens) == (1, T_LONG) else (
         "prefill_4x4096" if (N, inp.total_tokens) == (4, 16384) else "prefill_varlen")
     roof, tensor = prefill_roofline(inp, launch_ms, hbm_peak, bf16_peak, peak_src,
-                                    recorded_traffic(f"{kernel_name} {label}"), kernel_name)
+                                    recorded_traffic(f"{kernel_name} {label}"), kernel_name, gated)
+    out_desc = "bf16 out through the fused gated RMS normalisation" if gated else "fp32 out"
     leg = {"workload": f"kda_prefill: {N} sequence(s), {inp.total_tokens} tokens, {Hh} heads x 128, bf16 in / "
-                       f"fp32 state / fp32 out, {chains} (sequence, head) chains "
+                       f"fp32 state / {out_desc}, {chains} (sequence, head) chains "
                        f"({'overlapped' if chains <= 96 else 'one after the other'} schedule)",
            "tokens_per_s": world * inp.total_tokens * steps / (total_ms / 1e3), "ms_per_step": total_ms / steps,
            "total_ms": total_ms, "steps": steps, "roofline": roof, "tensor": tensor,

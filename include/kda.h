@@ -149,6 +149,50 @@ kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, co
                                  void* conv_tail, void* stream);
 
 /*
+ * kda_prefill_gated -- kda_prefill followed by the output epilogue, fused into
+ * the chunked path's output store, so that the unnormalised o never reaches
+ * HBM.  Page "GLM-5.3-Flash Internals - a measured profile", section
+ * "Findings": the mixer output passes o_norm, gated by the g_b_proj output,
+ * before o_proj.  The pages name these modules only; the reading taken is a
+ * gated RMS normalisation over each head's 128 value channels:
+ *     o[t, h, :] = x / sqrt(mean_c x_c^2 + norm_eps) * norm_weight * sigmoid(gate[t, h, :])
+ * where x is the mixer output kda_prefill would write for (t, h).
+ *   gate        : [total_T, H, 128] bf16, the g_b_proj output; must not alias o.
+ *   norm_weight : [128] fp32 (shared by the heads), 16-byte aligned.
+ *   norm_eps    : >= 0 and finite.
+ *   o_dt        : must be KDA_BF16 (the epilogue writes bf16).
+ * Every other argument, the workspace and the scheduling are those of
+ * kda_prefill.  Errors: as kda_prefill; KDA_ERR_INVALID_ARG for a NULL gate or
+ * weight, gate == o, o_dt != KDA_BF16 or a negative / non-finite eps;
+ * KDA_ERR_UNSUPPORTED for fp32 inputs (the recurrent path has no fused
+ * epilogue: run kda_prefill and then kda_output_norm).
+ */
+kda_status kda_prefill_gated(const void* q, const void* k, const void* v, const void* g,
+                             const void* beta, const float* conv_w, const void* init_state,
+                             const void* init_conv, const int32_t* cu_seqlens_dev,
+                             const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                             kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                             void* o, void* final_state, void* conv_tail, void* workspace,
+                             size_t workspace_bytes, const void* gate, const float* norm_weight,
+                             float norm_eps, void* stream);
+
+/*
+ * kda_output_norm -- the same output epilogue on its own, for mixer outputs
+ * produced by the decode entry points or the recurrent path:
+ *     y[r, h, :] = o[r, h, :] / sqrt(mean_c o[r, h, c]^2 + norm_eps) * norm_weight * sigmoid(gate[r, h, :])
+ *   o           : [rows, H, 128] of element type o_dt.
+ *   gate        : [rows, H, 128] bf16.
+ *   norm_weight : [128] fp32.
+ *   y           : out [rows, H, 128] bf16; may equal o when o_dt is KDA_BF16,
+ *                 must not alias gate.
+ * All pointers 16-byte aligned (KDA_ERR_ALIGNMENT otherwise).  rows == 0
+ * enqueues nothing.  Errors: KDA_ERR_INVALID_ARG for a bad size, enum or eps,
+ * a NULL pointer or a forbidden alias.
+ */
+kda_status kda_output_norm(const void* o, kda_dtype o_dt, const void* gate, const float* norm_weight,
+                           float norm_eps, void* y, int64_t rows, int num_heads, void* stream);
+
+/*
  * kda_decode_step -- one recurrent update per sequence (page "GLM-5.3-Flash im
  * Detail", section "Sequenz-Mixing: ...": decode of a single token performs a
  * recurrent update), in place.

@@ -38,7 +38,7 @@ BASE_SEED = 20261202
 _BLOCK = 1 << 22  # elements per independently seeded block
 
 # stream ids: each tensor draws from its own substream
-_Q, _K, _V, _G, _BETA, _CONVW, _STATE, _CONV, _GSEL, _GU, _LEN, _ACC = range(1, 13)
+_Q, _K, _V, _G, _BETA, _CONVW, _STATE, _CONV, _GSEL, _GU, _LEN, _ACC, _Z, _NW = range(1, 15)
 
 
 def _mix(seed: int, stream: int, block: int) -> int:
@@ -295,3 +295,12 @@ def workload(i: int, heads: Optional[int] = None):
     if i == 4:
         return make_decode(256, heads or 64, torch.bfloat16, seed, name="decode_bf16_256")
     raise ValueError(i)
+
+
+def make_output_norm(rows: int, H: int, seed: int, D: int = D_HEAD):
+    """Synthetic inputs of the output epilogue (no trained weights exist here):
+    the gate z [rows, H, D] bf16 ~ N(0, 2^2), as logits of a sigmoid gate that
+    spans closed to open; the norm weight w [D] fp32 ~ 1 + 0.25 N(0, 1)."""
+    z = randn((rows, H, D), seed, _Z, std=2.0, dtype=torch.bfloat16)
+    w = 1.0 + randn((D,), seed, _NW, std=0.25)
+    return z, w

@@ -28,7 +28,8 @@ STATUS = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED", 3: "K
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
            "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version",
            "kda_prefill_noalloc", "kda_decode_deltas_size", "kda_decode_verify", "kda_decode_commit",
-           "kda_decode_commit_verify", "kda_state_affine", "kda_inject_fault", "kda_last_cuda_error")
+           "kda_decode_commit_verify", "kda_state_affine", "kda_inject_fault", "kda_last_cuda_error",
+           "kda_prefill_gated", "kda_output_norm")
 MAX_VERIFY_ROWS = 8  # KDA_MAX_VERIFY_ROWS
 
 if not os.path.exists(LIB_PATH):
@@ -48,6 +49,11 @@ lib.kda_prefill.restype = ctypes.c_int
 lib.kda_prefill.argtypes = _PREFILL_ARGS + [_vp, ctypes.c_size_t, _vp]
 lib.kda_prefill_recurrent.restype = ctypes.c_int
 lib.kda_prefill_recurrent.argtypes = _PREFILL_ARGS + [_vp]
+lib.kda_prefill_gated.restype = ctypes.c_int
+lib.kda_prefill_gated.argtypes = _PREFILL_ARGS + [_vp, ctypes.c_size_t, _vp, _f32p, ctypes.c_float, _vp]
+lib.kda_output_norm.restype = ctypes.c_int
+lib.kda_output_norm.argtypes = [_vp, ctypes.c_int, _vp, _f32p, ctypes.c_float, _vp, ctypes.c_int64, ctypes.c_int,
+                                _vp]
 lib.kda_prefill_noalloc.restype = ctypes.c_int
 lib.kda_prefill_noalloc.argtypes = _PREFILL_ARGS + [_vp]
 NOALLOC_SCRATCH_BYTES = 128 << 20  # KDA_NOALLOC_SCRATCH_BYTES
@@ -132,12 +138,18 @@ def _state_code(final_state, init_state) -> int:
 def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init_state=None,
             init_conv=None, act: int = KDA_CONV_NONE, o=None, final_state=None, conv_tail=None,
             workspace=None, stream=None, recurrent: bool = False, o_dtype=torch.float32,
-            state_dtype=None):
+            state_dtype=None, gate=None, norm_weight=None, norm_eps: float = 1e-6):
     """kda_prefill (or kda_prefill_recurrent) on device tensors.  Returns
     (o, final_state, conv_tail); outputs are allocated when not given (o in
     `o_dtype`, fp32 by default; the final state in `state_dtype`, default the
     init state's type, else fp32).  The state element type of the call is that
-    of final_state."""
+    of final_state.  With `gate` ([T, H, 128] bf16) and `norm_weight` ([128]
+    fp32) the call is kda_prefill_gated: o holds the gated RMS-normalised
+    output, in bf16."""
+    if gate is not None:
+        if recurrent:
+            raise ValueError("the fused output epilogue runs on the chunked path only")
+        o_dtype = torch.bfloat16
     cu_h = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
     N = len(cu_h) - 1
     T, H = q.shape[0], q.shape[1]
@@ -162,8 +174,24 @@ def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init
         if workspace is None and need > 0:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-        _check(lib.kda_prefill(*args, _ptr(workspace), wbytes, _stream(stream)), "kda_prefill")
+        if gate is not None:
+            _check(lib.kda_prefill_gated(*args, _ptr(workspace), wbytes, _ptr(gate), _ptr(norm_weight),
+                                         float(norm_eps), _stream(stream)), "kda_prefill_gated")
+        else:
+            _check(lib.kda_prefill(*args, _ptr(workspace), wbytes, _stream(stream)), "kda_prefill")
     return o, final_state, conv_tail
+
+
+def output_norm(o, gate, norm_weight, norm_eps: float = 1e-6, y=None, stream=None):
+    """kda_output_norm: y = o / sqrt(mean o^2 + eps) * norm_weight * sigmoid(gate)
+    over each head's 128 channels; o [rows, H, 128] fp32 or bf16, gate bf16,
+    y bf16 (allocated when not given; may be o itself when o is bf16)."""
+    rows, H = o.shape[0], o.shape[1]
+    if y is None:
+        y = torch.empty(o.shape, dtype=torch.bfloat16, device=o.device)
+    _check(lib.kda_output_norm(_ptr(o), _dtype_code(o), _ptr(gate), _ptr(norm_weight), float(norm_eps),
+                               _ptr(y), rows, H, _stream(stream)), "kda_output_norm")
+    return y
 
 
 def prefill_noalloc(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init_state=None,

@@ -12,6 +12,7 @@
 #include "kda_tail.cuh"
 #include "kda_chunked.cuh"
 #include "kda_affine.cuh"
+#include "kda_output_norm.cuh"
 
 using namespace kda;
 
@@ -194,6 +195,64 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
                       a.stream);
   if (st != KDA_OK) return st;
   return launch_tail<__nv_bfloat16>(a);
+}
+
+kda_status kda_prefill_gated(const void* q, const void* k, const void* v, const void* g,
+                             const void* beta, const float* conv_w, const void* init_state,
+                             const void* init_conv, const int32_t* cu_seqlens_dev,
+                             const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                             kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                             void* o, void* final_state, void* conv_tail, void* workspace,
+                             size_t workspace_bytes, const void* gate, const float* norm_weight,
+                             float norm_eps, void* stream) {
+  PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, state_dt, o, final_state, conv_tail,
+                (cudaStream_t)stream, 0, 0};
+  kda_status st = validate_prefill(a);
+  if (st != KDA_OK) return st;
+  if (o_dt != KDA_BF16 || !norm_weight || !(norm_eps >= 0.f) || norm_eps > 3.0e38f) return KDA_ERR_INVALID_ARG;
+  if (a.total_T > 0 && (!gate || gate == o)) return KDA_ERR_INVALID_ARG;
+  if ((gate && !aligned(gate, 16)) || !aligned(norm_weight, 16)) return KDA_ERR_ALIGNMENT;
+  if (dt != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+  if (a.N == 0) return KDA_OK;
+  const size_t need = chunked_workspace_bytes(a.N, a.H, a.total_T);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 16)) return KDA_ERR_ALIGNMENT;
+  OutputNorm norm;
+  norm.gate = gate;
+  norm.weight = norm_weight;
+  norm.eps = norm_eps;
+  st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
+                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.state_dt, a.o, a.final_state, workspace,
+                      a.stream, norm);
+  if (st != KDA_OK) return st;
+  return launch_tail<__nv_bfloat16>(a);
+}
+
+kda_status kda_output_norm(const void* o, kda_dtype o_dt, const void* gate, const float* norm_weight,
+                           float norm_eps, void* y, int64_t rows, int num_heads, void* stream) {
+  if (rows < 0 || num_heads < 1 || !valid_dtype(o_dt)) return KDA_ERR_INVALID_ARG;
+  if (!norm_weight || !(norm_eps >= 0.f) || norm_eps > 3.0e38f) return KDA_ERR_INVALID_ARG;
+  if (rows == 0) return KDA_OK;
+  if (!o || !gate || !y || gate == y || (y == o && o_dt != KDA_BF16)) return KDA_ERR_INVALID_ARG;
+  const void* al16[] = {o, gate, y, norm_weight};
+  for (const void* p : al16)
+    if (!aligned(p, 16)) return KDA_ERR_ALIGNMENT;
+  const int64_t row_heads = rows * num_heads;
+  int sms = 0;
+  kda_status st = sm_count(&sms);
+  if (st != KDA_OK) return st;
+  const int64_t want = (row_heads + NORM_THREADS / 32 - 1) / (NORM_THREADS / 32);
+  const unsigned blocks = (unsigned)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  cudaStream_t s = (cudaStream_t)stream;
+  if (o_dt == KDA_F32)
+    output_norm_kernel<float><<<blocks, NORM_THREADS, 0, s>>>(
+        (const float*)o, (const __nv_bfloat16*)gate, norm_weight, norm_eps, (__nv_bfloat16*)y, row_heads);
+  else
+    output_norm_kernel<__nv_bfloat16><<<blocks, NORM_THREADS, 0, s>>>(
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)gate, norm_weight, norm_eps, (__nv_bfloat16*)y,
+        row_heads);
+  return cuda_ok(cudaGetLastError()) ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_decode_step(void* state, void* conv_cache, const void* q, const void* k,
@@ -402,7 +461,7 @@ kda_status kda_inject_fault(kda_fault kind) {
   return KDA_OK;
 }
 
-int kda_version(void) { return (2 << 16) | 2; }
+int kda_version(void) { return (2 << 16) | 3; }
 
 int kda_last_cuda_error(void) { return kda::t_last_cuda_error; }
 

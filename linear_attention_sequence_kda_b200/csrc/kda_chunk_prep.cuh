@@ -64,12 +64,16 @@ constexpr uint32_t P_MS = 0;                 // step 6: diag(beta) M strict, [64
 constexpr uint32_t P_TT = 17408;             // step 7: T tile [64 t][64 t'] (16 KB)
 constexpr uint32_t P_KT = 33792;             // step 7: K~^T tile [128 k][64 t] (32 KB)
 constexpr uint32_t P_TMP = 66560;            // steps 6-7: blocks of X (12.3 KB)
-constexpr uint32_t P_MISC = 81920;           // scalars (6 KB)
+constexpr uint32_t P_WST = 52224;            // step 8: -W staged in its record image (32 KB), read by
+                                             // bulk copies until the next item's step 3
+constexpr uint32_t P_MISC = 84992;           // scalars (6 KB)
 constexpr uint32_t PREP_SMEM = P_MISC + 6144 + 1024;
 static_assert(P_GA + 3 * GA_ROWS * 128 + 128 * 128 <= P_MISC, "A tile reads past the Gram region");
 static_assert(3 * RAW_BYTES <= P_MISC && P_TMP + (96 * 20 + 32 * 36 + 16) * 4 <= P_MISC,
               "shared regions overlap the scalars");
 static_assert(P_MS + 64 * MS_LD * 4 <= P_TT, "solve matrix overlaps the T tile");
+static_assert(P_WST >= 3 * RAW_BYTES && P_WST + 4 * 64 * 128 <= P_MISC && P_WST % 1024 == 0,
+              "the -W staging overlaps the next item's raw tiles or the scalars");
 
 // scalar region (floats)
 constexpr int MB_BETA = 0, MB_RQ = 64, MB_RK = 128, MB_PD = 192, MB_CARRY = 256 /*128*/,
@@ -165,6 +169,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t tm = tmem_base;
   const uint32_t tl = tm + ((uint32_t)(32 * q4) << 16);  // this warp's TMEM lanes
   uint32_t par = 0;  // phase parity of the per-item barriers
+  // thread 0: the item whose -W bulk copies are in flight; its record is
+  // published once they are complete (during the next item, or at exit)
+  int pending = -1;
+  auto publish = [&](int it) {
+    tc::bulk_wait_all();
+    tc::fence_async_global();
+    if (ready) {  // every thread's stores of the item precede a barrier thread 0 has passed
+      __threadfence();
+      asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(ready + it), "r"(1) : "memory");
+    }
+  };
 
   // persistent loop over (chunk, head) work items, chunk-major
   for (int item = s_next; item < n_items; item = s_next, par ^= 1) {
@@ -254,6 +269,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const float rq = 1.0f / sqrtf(nq + NORM_EPS), rk = 1.0f / sqrtf(nk + NORM_EPS);
     ms[MB_RQ + tid] = rq; ms[MB_RK + tid] = rk; ms[MB_PD + tid] = nx * rq * rk;
   }
+  if (tid == 0 && pending >= 0) tc::bulk_wait_read();  // step 3 overwrites the previous -W staging
   __syncthreads();
 
   // ---- 3. normalise; Gram operands, record tiles QT and KB, stashes ---------
@@ -269,15 +285,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tc::ld8(tl + TC_YQ + r0 + 8 * g, yq);
       tc::ld8(tl + TC_YK + r0 + 8 * g, yk);
       tc::ld8(tl + TC_G + r0 + 8 * g, gl);
+      const float4 rk0 = *reinterpret_cast<const float4*>(ms + MB_RK + r0 + 8 * g);
+      const float4 rk1 = *reinterpret_cast<const float4*>(ms + MB_RK + r0 + 8 * g + 4);
+      const float4 rq0 = *reinterpret_cast<const float4*>(ms + MB_RQ + r0 + 8 * g);
+      const float4 rq1 = *reinterpret_cast<const float4*>(ms + MB_RQ + r0 + 8 * g + 4);
+      const float rkv[8] = {rk0.x, rk0.y, rk0.z, rk0.w, rk1.x, rk1.y, rk1.z, rk1.w};
+      const float rqv[8] = {rq0.x, rq0.y, rq0.z, rq0.w, rq1.x, rq1.y, rq1.z, rq1.w};
       tc::ld_wait();
       float kb[8];
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const int t = r0 + 8 * g + r;
         const float G = gl[r] + carry;
         const float d = G - gm;
         const float e1 = tc::exp2_fast(d), e2 = tc::exp2_fast(-d), e3 = tc::exp2_fast(G);
-        const float kh = yk[r] * ms[MB_RK + t], qh = yq[r] * ms[MB_RQ + t];
+        const float kh = yk[r] * rkv[r], qh = yq[r] * rqv[r];
         // B operand of the P Gram; A rows (block of the own half, and for
         // half 0 the rows read against half 1)
         *reinterpret_cast<float*>(sm + P_GB + tc::sw128o(r0 + 8 * g, r, ch, 64)) = tc::to_tf32(qh * e1);
@@ -514,6 +535,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
 
   // ---- 7. T = X diag(beta): record TS, T tile; K~^T tile; W = T K~ -----------
+  if (tid == 0 && pending >= 0) {
+    publish(pending);
+    pending = -1;
+  }
   for (int e = tid; e < CH * 16; e += PREP_THREADS) {  // 4-column groups
     const int t = e >> 4, tp = 4 * (e & 15);
     float4 tv, ts;
@@ -577,7 +602,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
 
   // ---- 8. -W rows into the record (row block wrow0 of RA) -------------------
-  // M = 64 accumulator: row t in lane 16 * (t / 16) ... of quarter t / 16
+  // M = 64 accumulator: row t in lane 16 * (t / 16) ... of quarter t / 16.
+  // The rows are staged in their record image (the swizzle phase of row
+  // wrow0 + t is that of t) and leave in four 8 KB bulk copies, one per slab,
+  // instead of one scattered 16-byte store per row and column group.
   {
     const int t = 16 * q4 + (lane & 15);
 #pragma unroll
@@ -590,24 +618,29 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (lane < 16) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          *reinterpret_cast<float4*>(rec + REC_RA + tc::sw128(wrow0 + t, c0 + 4 * j, 128)) =
+          *reinterpret_cast<float4*>(sm + P_WST + tc::sw128(t, c0 + 4 * j, 64)) =
               make_float4(tc::to_tf32(-w0[4 * j]), tc::to_tf32(-w0[4 * j + 1]), tc::to_tf32(-w0[4 * j + 2]),
                           tc::to_tf32(-w0[4 * j + 3]));
-          *reinterpret_cast<float4*>(rec + REC_RA + tc::sw128(wrow0 + t, c0 + 16 + 4 * j, 128)) =
+          *reinterpret_cast<float4*>(sm + P_WST + tc::sw128(t, c0 + 16 + 4 * j, 64)) =
               make_float4(tc::to_tf32(-w1[4 * j]), tc::to_tf32(-w1[4 * j + 1]), tc::to_tf32(-w1[4 * j + 2]),
                           tc::to_tf32(-w1[4 * j + 3]));
         }
       }
     }
   }
+  tc::fence_async_smem();
   tc::fence_before();
   __syncthreads();  // TMEM columns and shared regions are reused by the next item
   tc::fence_after();
-  if (tid == 0 && ready) {  // publish the record: every thread's stores precede the barrier above
-    __threadfence();
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(ready + item), "r"(1) : "memory");
+  if (tid == 0) {
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl)
+      tc::bulk_s2g(rec + REC_RA + sl * 16384 + wrow0 * 128, sm + P_WST + sl * 8192, 8192);
+    tc::bulk_commit();
+    pending = item;
   }
   }  // item loop
+  if (tid == 0 && pending >= 0) publish(pending);
   tc::fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem_base, 256);

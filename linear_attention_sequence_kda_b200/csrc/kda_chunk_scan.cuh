@@ -15,6 +15,15 @@
 //   fp32   U'^T += b * V^T (the diagonal of Dk T); keep d * U' (of p)
 //   MMA2   [O^T | S(1)] (p = 0) or [S(0) | O^T] (p = 1) += U'^T B2     (N = 192)
 //   fp32   o = r * (O + d u'), staged in shared memory and stored by TMA.
+// With the output epilogue (EPI, bf16 output) the stored rows are
+//          y = o / sqrt(mean_v o^2 + eps) * w * sigmoid(z)
+// per token over the head's 128 value columns (the gated RMS normalisation of
+// the mixer output, page "GLM-5.3-Flash Internals -- a measured profile",
+// section "Findings": o_norm gated by the g_b_proj output z), so that o never
+// reaches HBM unnormalised.  The compute warps that share a token quarter
+// exchange their rows' partial sums of o^2 through shared memory; the gate
+// tile comes in by TMA two chunks ahead, behind the bf16 output tile of the
+// same staging buffer.
 // So the serial chain from one state to the next is MMA_A, the U' update and
 // MMA2; the decay and the output run beside the tensor core.  A operands are
 // read from TMEM as tf32; the state itself stays fp32.
@@ -32,7 +41,9 @@
 //               consumed record from L2 (all lanes), so that a record read soon
 //               after it was written never reaches HBM.
 //   warp 18     one thread stores the output tiles (double-buffered staging),
-//               so that global stores never hold up the compute warps.
+//               so that global stores never hold up the compute warps (with
+//               the epilogue it also loads the gate tile of chunk i + 2 once
+//               the store of chunk i has read the staging buffer).
 // Each thread waits by parity only on barriers that cannot complete two phases
 // ahead of it: the next phase of every barrier it waits on needs an action of
 // its own (or of a role that itself waited on this thread's previous step).
@@ -53,8 +64,9 @@ constexpr uint32_t SCAN_SC = SCAN_B + B2_BYTES;
 constexpr uint32_t SCAN_V = (SCAN_SC + 2 * SC_BYTES + 1023) & ~1023u;  // raw value tile (bf16)
 constexpr uint32_t SCAN_OST = (SCAN_V + RAW_BYTES + 1023) & ~1023u;  // 2 output tiles [64 t][128] (fp32 at most)
 constexpr uint32_t OST_BYTES = CH * D * 4;
+constexpr uint32_t OST_Z = CH * D * 2;  // epilogue: gate tile [64 t][128] bf16 behind the bf16 output tile
 constexpr uint32_t SCAN_SMEM = SCAN_OST + 2 * OST_BYTES + 1024;
-static_assert(SCAN_SMEM + 256 <= 232448, "scan shared memory (dynamic + the static barriers)");
+static_assert(SCAN_SMEM + 2560 <= 232448, "scan shared memory (dynamic + the static barriers and epilogue sums)");
 constexpr int TM_S0 = 0, TM_O1 = 128, TM_U = 192, TM_O0 = 256, TM_S1 = 320, TM_V = 448;
 __device__ __forceinline__ int s_col(int chunk) { return (chunk & 1) ? TM_S1 : TM_S0; }
 __device__ __forceinline__ int o_col(int chunk) { return (chunk & 1) ? TM_O1 : TM_O0; }
@@ -64,7 +76,7 @@ __device__ __forceinline__ void discard_l2(const void* p) {
   asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 
-template <typename Tout, int ACT, typename Ts>
+template <typename Tout, int ACT, typename Ts, bool EPI>
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                   const float* __restrict__ conv_w,
@@ -72,7 +84,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
                   const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_base,
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
                   const int* __restrict__ ready, Tout* __restrict__ o, Ts* final_state,
-                  uint64_t wait_ns) {
+                  uint64_t wait_ns, const __grid_constant__ CUtensorMap tm_z,
+                  const float* __restrict__ norm_w, float norm_eps) {
+  static_assert(!EPI || sizeof(Tout) == 2, "the output epilogue writes bf16");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that the
   // compiler keeps the shared address space (32-bit shared loads and stores)
@@ -83,6 +97,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
   // s = 4: TS) has landed; bar_rafree[s]: the products that read it are done
   __shared__ uint64_t bar_ra[5], bar_rafree[5], bar_pk, bar_sc[2], bar_v, bar_pkfree, bar_vfree, bar_ma, bar_m2,
       bar_conv, bar_b, bar_ost[2], bar_ofree[2], bar_drain;
+  // epilogue: gate tiles landed (by staging buffer); per-row partial sums of
+  // o^2 of the four warps that share a token quarter (by chunk parity)
+  constexpr int NR = EPI ? 2 : 1;
+  __shared__ uint64_t bar_z[NR], bar_red[NR][4];
+  __shared__ float s_red[NR][4][EPI ? 16 : 1][4];
   __shared__ uint32_t tmem_base;
   __shared__ int s_abort;
 
@@ -106,6 +125,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     tc::bar_init(&bar_ost[0], SCAN_COMPUTE); tc::bar_init(&bar_ost[1], SCAN_COMPUTE);
     tc::bar_init(&bar_ofree[0], 1); tc::bar_init(&bar_ofree[1], 1);
     tc::bar_init(&bar_drain, 1);
+    if (EPI) {
+      for (int j = 0; j < NR; ++j) {
+        tc::bar_init(&bar_z[j], 1);
+        for (int pq = 0; pq < 4; ++pq) tc::bar_init(&bar_red[j][pq], 64);
+      }
+    }
     s_abort = 0;
     tc::bar_init_fence();
   }
@@ -286,6 +311,16 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     // ======================= output-storing thread ==========================
     if (lane == 0) {
       bool ok = true;
+      int n_z[2] = {0, 0};  // gate loads issued per buffer, for the drain
+      auto load_z = [&](int i) {
+        const int b = i & 1;
+        tc::bar_expect_tx(&bar_z[b & (NR - 1)], OST_Z);
+        tc::tma_load_2d(sm + SCAN_OST + b * OST_BYTES + OST_Z, &tm_z, h * D, (int)(seg0 + (int64_t)CH * i),
+                        &bar_z[b & (NR - 1)]);
+        ++n_z[b];
+      };
+      if (EPI)
+        for (int i = 0; i < 2 && i < nchunks; ++i) load_z(i);
       for (int i = 0; i < nchunks && ok; ++i) {
         const int b = i & 1;
         ok = tc::bar_wait_or(&bar_ost[b], (uint32_t)((i >> 1) & 1), abort_flag, wait_ns);
@@ -301,9 +336,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
         }
         tc::bulk_commit();
         tc::bulk_wait_read();  // the staging tile may be refilled
+        if (EPI && i + 2 < nchunks) load_z(i + 2);  // the gate of chunk i + 2 (output(i) has read z(i))
         tc::bar_arrive(&bar_ofree[b]);
       }
-      if (!ok) s_abort = 1;
+      if (!ok) {
+        s_abort = 1;
+        for (int b = 0; b < 2; ++b)  // issued gate loads land before shared memory is released
+          if (n_z[b]) tc::bar_wait(&bar_z[b & (NR - 1)], (uint32_t)((n_z[b] - 1) & 1));
+      }
       tc::bulk_wait_all();  // output rows are in global memory before exit
     }
   } else {
@@ -367,6 +407,50 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       for (int j = 0; j < 16; ++j) r[j] = tc::to_tf32(vv[j]);
       tc::st16(tl + TM_V + t0, r);
     };
+    // epilogue of the 16 output rows t0 .. t0 + 15 (column v) of chunk c, in
+    // place: the sum of squares of each row over this warp's 32 columns by a
+    // reduce-scatter across the lanes (row m ends in lanes 2m and 2m + 1),
+    // then over the four warps of the token quarter through shared memory
+    float wn = 0.f;
+    if constexpr (EPI) wn = norm_w[v];
+    auto epilogue = [&](int c, float (&y)[16]) -> bool {
+      const int b = c & 1 & (NR - 1);
+      const uint32_t ph = (uint32_t)((c >> 1) & 1);
+      float s8[8], s4[4], s2[2];
+      const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float lo = y[j] * y[j], hi = y[j + 8] * y[j + 8];
+        s8[j] = (b4 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b4 ? lo : hi, 16);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        s4[j] = (b3 ? s8[j + 4] : s8[j]) + __shfl_xor_sync(0xffffffffu, b3 ? s8[j] : s8[j + 4], 8);
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        s2[j] = (b2 ? s4[j + 2] : s4[j]) + __shfl_xor_sync(0xffffffffu, b2 ? s4[j] : s4[j + 2], 4);
+      float s1 = (b1 ? s2[1] : s2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? s2[0] : s2[1], 2);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 1);  // row t0 + lane / 2, over the warp's 32 columns
+      if (!(lane & 1)) {
+        s_red[b][part][(lane >> 1) & (EPI ? 15 : 0)][q] = s1;
+        tc::bar_arrive(&bar_red[b][part]);
+      }
+      if (!tc::bar_wait_or(&bar_red[b][part], ph, abort_flag, wait_ns)) return false;
+      float rs = 0.f;
+      if (lane < 16) {
+        const float* pr = s_red[b][part][lane & (EPI ? 15 : 0)];
+        rs = rsqrtf((pr[0] + pr[1] + pr[2] + pr[3]) * (1.f / D) + norm_eps);
+      }
+      if (!tc::bar_wait_or(&bar_z[b], ph, abort_flag, wait_ns)) return false;
+      const __nv_bfloat16* zt =
+          reinterpret_cast<const __nv_bfloat16*>(sm + SCAN_OST + (c & 1) * OST_BYTES + OST_Z);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float gate = __fdividef(1.f, 1.f + __expf(-to_f(zt[(t0 + j) * D + v])));
+        y[j] *= __shfl_sync(0xffffffffu, rs, j) * wn * gate;
+      }
+      return true;
+    };
     // output of chunk c: o = r (O + d u'), into the staging tile of c's parity
     // (free once the store of chunk c - 2 has read it)
     auto output = [&](int c, const float (&rr)[16], const float (&du)[16]) -> bool {
@@ -377,8 +461,16 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       float r[16];
       tc::ld16(tl + (uint32_t)o_col(c) + t0, r);
       tc::ld_wait();
+      if constexpr (EPI) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) st[(t0 + j) * D + v] = from_f<Tout>(rr[j] * (r[j] + du[j]));
+        for (int j = 0; j < 16; ++j) r[j] = rr[j] * (r[j] + du[j]);
+        if (!epilogue(c, r)) return false;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) st[(t0 + j) * D + v] = from_f<Tout>(r[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) st[(t0 + j) * D + v] = from_f<Tout>(rr[j] * (r[j] + du[j]));
+      }
       tc::fence_async_smem();
       tc::bar_arrive(&bar_ost[b]);
       return true;

@@ -15,6 +15,7 @@
 // blocks become resident first; with more chains the two run one after the
 // other on the caller's stream.
 #pragma once
+#include <type_traits>
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -46,6 +47,14 @@ inline size_t chunked_workspace_bytes(int N, int H, int64_t total_tokens) {
   const int64_t nc = chunk_bound(N, total_tokens);
   return chunk_header_bytes(N, nc) + chunk_sync_bytes(nc, H) + 128 + (size_t)nc * H * REC_BYTES;
 }
+
+// The optional output epilogue: the gated RMS normalisation of each head's
+// output row, y = o / sqrt(mean o^2 + eps) * weight * sigmoid(gate).
+struct OutputNorm {
+  const void* gate = nullptr;    // [total_T, H, 128] bf16, or null for plain o
+  const float* weight = nullptr;  // [128] fp32
+  float eps = 0.f;
+};
 
 constexpr int OVERLAP_MAX_CHAINS = 96;  // leaves at least 52 of 148 SMs to prep
 // Prep SM-time per chunk-head relative to the scan's time per chunk of a
@@ -116,7 +125,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
                                    const void* init_conv, const int32_t* cu_dev,
                                    const int32_t* cu_host, int N, int H, kda_dtype o_dt,
                                    kda_dtype state_dt, void* o, void* final_state, void* workspace,
-                                   cudaStream_t stream) {
+                                   const OutputNorm& norm, cudaStream_t stream) {
   using T = __nv_bfloat16;
   // The chunk table below is staged from host memory that this call owns and
   // releases on return; a captured graph would read it again on every replay,
@@ -163,10 +172,11 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   // TMA descriptors over the packed [total_T, H*128] tensors: 67-row boxes for
   // the inputs (3 halo rows + one chunk); 64-row boxes for the output tiles
   const uint64_t rows = (uint64_t)cu_host[N], cols = (uint64_t)H * D;
-  CUtensorMap tq, tk, tg, tv, to;
+  CUtensorMap tq, tk, tg, tv, to, tz;
   if (!make_tmap_bf16_2d(&tq, q, rows, cols, RAW_ROWS, D) || !make_tmap_bf16_2d(&tk, k, rows, cols, RAW_ROWS, D) ||
       !make_tmap_bf16_2d(&tg, g, rows, cols, RAW_ROWS, D) || !make_tmap_bf16_2d(&tv, v, rows, cols, RAW_ROWS, D) ||
-      !make_tmap_2d(&to, o, rows, cols, CH, D, o_dt == KDA_F32 ? 4 : 2))
+      !make_tmap_2d(&to, o, rows, cols, CH, D, o_dt == KDA_F32 ? 4 : 2) ||
+      !make_tmap_bf16_2d(&tz, norm.gate ? norm.gate : v, rows, cols, CH, D))
     return KDA_ERR_CUDA;
 
   cudaStream_t scan_stream = stream, side = nullptr;
@@ -206,22 +216,28 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     if (!cuda_ok(cudaGetLastError())) return KDA_ERR_CUDA;
   }
   // the scan, instantiated for the output and state element types
-  auto launch_scan = [&](auto tout, auto ts) -> bool {
+  auto launch_scan = [&](auto tout, auto ts, auto epi) -> bool {
     using Tout = decltype(tout);
     using Ts = decltype(ts);
-    auto scan = chunk_scan_kernel<Tout, ACT, Ts>;
+    constexpr bool E = decltype(epi)::value;
+    auto scan = chunk_scan_kernel<Tout, ACT, Ts, E>;
     if (!cuda_ok(cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM)))
       return false;
     scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, scan_stream>>>(
         tv, to, conv_w, (const Ts*)init_state, (const T*)init_conv, cu_dev, d_base, d_order, H, records,
-        overlap ? ready : nullptr, (Tout*)o, (Ts*)final_state, scan_wait_ns(items));
+        overlap ? ready : nullptr, (Tout*)o, (Ts*)final_state, scan_wait_ns(items), tz, norm.weight,
+        norm.eps);
     return true;
   };
+  using Plain = std::false_type;
+  using Epi = std::true_type;
   bool ok;
-  if (o_dt == KDA_F32)
-    ok = state_dt == KDA_F32 ? launch_scan(float{}, float{}) : launch_scan(float{}, T{});
+  if (norm.gate)  // the epilogue writes bf16 (checked by the caller)
+    ok = state_dt == KDA_F32 ? launch_scan(T{}, float{}, Epi{}) : launch_scan(T{}, T{}, Epi{});
+  else if (o_dt == KDA_F32)
+    ok = state_dt == KDA_F32 ? launch_scan(float{}, float{}, Plain{}) : launch_scan(float{}, T{}, Plain{});
   else
-    ok = state_dt == KDA_F32 ? launch_scan(T{}, float{}) : launch_scan(T{}, T{});
+    ok = state_dt == KDA_F32 ? launch_scan(T{}, float{}, Plain{}) : launch_scan(T{}, T{}, Plain{});
   if (!ok || !cuda_ok(cudaGetLastError())) return KDA_ERR_CUDA;
   if (overlap && join_side(stream, side, join) != KDA_OK) return KDA_ERR_CUDA;
   return KDA_OK;
@@ -232,12 +248,15 @@ inline kda_status launch_chunked(const void* q, const void* k, const void* v, co
                                  const void* init_conv, const int32_t* cu_dev,
                                  const int32_t* cu_host, int N, int H, kda_conv_act act,
                                  kda_dtype o_dt, kda_dtype state_dt, void* o, void* final_state,
-                                 void* workspace, cudaStream_t stream) {
+                                 void* workspace, cudaStream_t stream,
+                                 const OutputNorm& norm = OutputNorm{}) {
   if (act == KDA_CONV_SILU)
     return launch_chunked_t<KDA_CONV_SILU>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
-                                           cu_host, N, H, o_dt, state_dt, o, final_state, workspace, stream);
+                                           cu_host, N, H, o_dt, state_dt, o, final_state, workspace, norm,
+                                           stream);
   return launch_chunked_t<KDA_CONV_NONE>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
-                                         cu_host, N, H, o_dt, state_dt, o, final_state, workspace, stream);
+                                         cu_host, N, H, o_dt, state_dt, o, final_state, workspace, norm,
+                                         stream);
 }
 
 }  // namespace kda

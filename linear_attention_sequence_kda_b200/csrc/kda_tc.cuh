@@ -283,6 +283,14 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // wait until every committed bulk store of this thread is complete
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// order completed bulk (async-proxy) global writes before this thread's later generic accesses
+__device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// hint: a tile of a tensor map into L2 (x, y: innermost and outer coordinates)
+__device__ __forceinline__ void prefetch_tile_l2(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
+}
 
 // hint: bring `bytes` (multiple of 16) of global memory at `src` into L2
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {

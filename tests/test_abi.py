@@ -97,6 +97,46 @@ def test_prefill_workspace_check():
     assert _prefill([0, 5, 10], ws=WS + 8) == 3
 
 
+ZG, NW = 12 << 20, 13 << 20  # gate and norm weight
+
+
+def _gated(cu, dt=1, odt=1, gate=ZG, nw=NW, eps=1e-6, o=O, **kw):
+    cu = np.ascontiguousarray(np.asarray(cu, dtype=np.int32))
+    args = [Q, K, V, G, B, W, None, None, CU, cu.ctypes.data, len(cu) - 1, 4, dt, 0, odt, 0, o, FS, CT]
+    return kda.lib.kda_prefill_gated(*args, WS, 1 << 40, gate, nw, eps, None)
+
+
+def test_prefill_gated_argument_validation():
+    """The fused epilogue writes bf16 and needs a gate and a weight; fp32
+    inputs have no fused epilogue.  Every case returns before any launch."""
+    assert _gated([0, 5], odt=0) == 1           # fp32 output
+    assert _gated([0, 5], gate=None) == 1
+    assert _gated([0, 5], nw=None) == 1
+    assert _gated([0, 5], eps=-1.0) == 1
+    assert _gated([0, 5], eps=float("nan")) == 1
+    assert _gated([0, 5], eps=float("inf")) == 1
+    assert _gated([0, 5], gate=O) == 1          # gate aliases the output
+    assert _gated([0, 5], gate=ZG + 8) == 3     # misaligned
+    assert _gated([0, 5], nw=NW + 4) == 3
+    assert _gated([0, 5], dt=0) == 2            # fp32 inputs: recurrent path, no fused epilogue
+    assert _gated([1, 5]) == 1                  # the prefill checks still apply
+    assert _gated([0]) == 0                     # no segments: nothing to do
+
+
+def test_output_norm_argument_validation():
+    f = kda.lib.kda_output_norm
+    assert f(O, 1, ZG, NW, 1e-6, O, 0, 4, None) == 0        # no rows: nothing enqueued
+    assert f(O, 1, ZG, NW, 1e-6, O, -1, 4, None) == 1
+    assert f(O, 1, ZG, NW, 1e-6, O, 5, 0, None) == 1
+    assert f(O, 5, ZG, NW, 1e-6, O, 5, 4, None) == 1        # bad dtype
+    assert f(O, 1, ZG, None, 1e-6, O, 5, 4, None) == 1
+    assert f(O, 1, ZG, NW, -1.0, O, 5, 4, None) == 1
+    assert f(None, 1, ZG, NW, 1e-6, O, 5, 4, None) == 1
+    assert f(O, 1, ZG, NW, 1e-6, ZG, 5, 4, None) == 1       # y aliases the gate
+    assert f(O, 0, ZG, NW, 1e-6, O, 5, 4, None) == 1        # in place needs a bf16 o
+    assert f(O + 8, 1, ZG, NW, 1e-6, Q, 5, 4, None) == 3
+
+
 def test_decode_argument_validation():
     d = kda.lib.kda_decode_step
     assert d(FS, CT, Q, K, V, G, B, W, 4, 0, 1, 0, 0, 0, O, None) == 1

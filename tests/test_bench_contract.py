@@ -44,6 +44,14 @@ def test_prefill_roofline_fractions():
     assert roof["o_fp32_variant"]["algorithmic_bytes_per_launch"] == 65536 * 64 * 1538 + 64 * 2 * 65536
 
 
+def test_gated_prefill_roofline_counts_the_gate():
+    """With the fused output epilogue the gate z (256 B per token-head) is read
+    and o is written in bf16, as the method's 1,282 B already count it."""
+    roof, _ = bench.prefill_roofline(_Inp(1, 65536, 64), 6.0, 6500.0, 1600.0, "measured", None, "k", gated=True)
+    assert roof["algorithmic_bytes_per_launch"] == 65536 * 64 * (1282 + 256) + 64 * 2 * 65536
+    assert roof["o_fp32_variant"] is None
+
+
 def test_decode_bytes_per_pair():
     rows_in = 4 * 256            # q, k, v, g of the token, bf16
     o_out = 512                  # fp32
