@@ -88,6 +88,14 @@ constexpr int TC_DP = 128;  // P Gram accumulator (64 columns)
 constexpr int TC_DM = 192;  // M Gram accumulator (64 columns)
 constexpr int TC_W = 128;   // W accumulator (M = 64, 128 columns)
 
+// one 32-byte (256-bit) global store; dst 32-byte aligned
+__device__ __forceinline__ void st_global_v8(float* dst, float a0, float a1, float a2, float a3, float a4, float a5,
+                                             float a6, float a7) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "f"(a0), "f"(a1), "f"(a2),
+               "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7)
+               : "memory");
+}
+
 // Sum over the 32 lanes of a warp of 16 per-lane vectors; lane l returns the
 // total of entry l % 16 (recursive halving: 16 shuffles instead of 16 x 5).
 __device__ __forceinline__ float lane_reduce16(float (&v)[16], int lane) {
@@ -316,11 +324,18 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       tc::st8(tl + TC_YQ + r0 + 8 * g, yq);
       tc::st8(tl + TC_YK + r0 + 8 * g, yk);
-      // K-bar^T row ch (B2 row krow0 + ch), columns r0 + 8g .. +7
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-        *reinterpret_cast<float4*>(rec + REC_B2 + tc::sw128(krow0 + ch, r0 + 8 * g + 4 * j, B2_ROWS)) =
-            make_float4(kb[4 * j], kb[4 * j + 1], kb[4 * j + 2], kb[4 * j + 3]);
+      // K-bar^T row ch (B2 row krow0 + ch), columns r0 + 8g .. +7: the two
+      // 16-byte chunks (2g and 2g + 1 before the swizzle) fill one aligned
+      // 32-byte sector, in swapped order on rows of odd swizzle phase; one
+      // 256-bit store writes it
+      {
+        const bool swap = (ch & 1) != 0;  // swizzle phase of row krow0 + ch is ch % 8
+        float* dst = reinterpret_cast<float*>(rec + REC_B2 + (tc::sw128(krow0 + ch, r0 + 8 * g, B2_ROWS) & ~16u));
+        if (swap)
+          st_global_v8(dst, kb[4], kb[5], kb[6], kb[7], kb[0], kb[1], kb[2], kb[3]);
+        else
+          st_global_v8(dst, kb[0], kb[1], kb[2], kb[3], kb[4], kb[5], kb[6], kb[7]);
+      }
     }
   }
   tc::fence_async_smem();
