@@ -149,6 +149,49 @@ kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, co
                                  void* conv_tail, void* stream);
 
 /*
+ * kda_prefill_records / kda_prefill_scan -- the chunked prefill in two halves,
+ * for callers that run several scans over the same chunks with different
+ * values or initial states (context parallelism: one prefill from S = 0 and
+ * one from S = I with v = 0 give a segment's affine carry S_out = A S_in + B,
+ * and a third from the carried-in state gives its outputs; page
+ * "GLM-5.3-Flash im Detail", section "Sequenz-Mixing: ...": a state is handed
+ * from chunk to chunk, linearly).  The chunk records (everything the scan
+ * reads that does not involve v or the state) depend on q, k, g, beta, the
+ * segments, the heads, conv_w's q and k taps and the q and k rows of
+ * init_conv only.
+ *   kda_prefill_records : exactly kda_prefill, and the records stay valid in
+ *                         `workspace` after the call (kda_prefill drops them
+ *                         from L2 without writing them back as they are read).
+ *   kda_prefill_scan    : the scan half only: o, final_state and conv_tail of
+ *                         a kda_prefill with these arguments, provided that
+ *                         `workspace` holds the records of a kda_prefill_records
+ *                         call with the same q, k, g, beta, cu_seqlens,
+ *                         num_heads, act, conv_w and q/k conv history (v,
+ *                         init_state, the v history and the output types may
+ *                         differ).  Results are then bit-identical to
+ *                         kda_prefill's; with other records they are
+ *                         meaningless but every access stays inside
+ *                         `workspace`.  Any number of scans may follow one
+ *                         records call, until the workspace is reused.
+ * Arguments, workspace size and errors are kda_prefill's; fp32 inputs (the
+ * recurrent path, which keeps no records) return KDA_ERR_UNSUPPORTED.
+ */
+kda_status kda_prefill_records(const void* q, const void* k, const void* v, const void* g,
+                               const void* beta, const float* conv_w, const void* init_state,
+                               const void* init_conv, const int32_t* cu_seqlens_dev,
+                               const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                               kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                               void* o, void* final_state, void* conv_tail, void* workspace,
+                               size_t workspace_bytes, void* stream);
+kda_status kda_prefill_scan(const void* q, const void* k, const void* v, const void* g,
+                            const void* beta, const float* conv_w, const void* init_state,
+                            const void* init_conv, const int32_t* cu_seqlens_dev,
+                            const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                            kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                            void* o, void* final_state, void* conv_tail, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
  * kda_prefill_gated -- kda_prefill followed by the output epilogue, fused into
  * the chunked path's output store, so that the unnormalised o never reaches
  * HBM.  Page "GLM-5.3-Flash Internals - a measured profile", section

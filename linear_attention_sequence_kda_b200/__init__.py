@@ -29,7 +29,7 @@ EXPORTS = ("kda_prefill_workspace_size", "kda_prefill", "kda_prefill_recurrent",
            "kda_decode_step", "kda_status_string", "kda_check_async_status", "kda_version",
            "kda_prefill_noalloc", "kda_decode_deltas_size", "kda_decode_verify", "kda_decode_commit",
            "kda_decode_commit_verify", "kda_state_affine", "kda_inject_fault", "kda_last_cuda_error",
-           "kda_prefill_gated", "kda_output_norm")
+           "kda_prefill_gated", "kda_output_norm", "kda_prefill_records", "kda_prefill_scan")
 MAX_VERIFY_ROWS = 8  # KDA_MAX_VERIFY_ROWS
 
 if not os.path.exists(LIB_PATH):
@@ -47,6 +47,9 @@ _PREFILL_ARGS = [_vp, _vp, _vp, _vp, _vp, _f32p, _vp, _vp, _i32p, _i32p, ctypes.
                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, _vp, _vp]
 lib.kda_prefill.restype = ctypes.c_int
 lib.kda_prefill.argtypes = _PREFILL_ARGS + [_vp, ctypes.c_size_t, _vp]
+for _name in ("kda_prefill_records", "kda_prefill_scan"):
+    getattr(lib, _name).restype = ctypes.c_int
+    getattr(lib, _name).argtypes = _PREFILL_ARGS + [_vp, ctypes.c_size_t, _vp]
 lib.kda_prefill_recurrent.restype = ctypes.c_int
 lib.kda_prefill_recurrent.argtypes = _PREFILL_ARGS + [_vp]
 lib.kda_prefill_gated.restype = ctypes.c_int
@@ -138,14 +141,22 @@ def _state_code(final_state, init_state) -> int:
 def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init_state=None,
             init_conv=None, act: int = KDA_CONV_NONE, o=None, final_state=None, conv_tail=None,
             workspace=None, stream=None, recurrent: bool = False, o_dtype=torch.float32,
-            state_dtype=None, gate=None, norm_weight=None, norm_eps: float = 1e-6):
+            state_dtype=None, gate=None, norm_weight=None, norm_eps: float = 1e-6, mode: str = "full"):
     """kda_prefill (or kda_prefill_recurrent) on device tensors.  Returns
     (o, final_state, conv_tail); outputs are allocated when not given (o in
     `o_dtype`, fp32 by default; the final state in `state_dtype`, default the
     init state's type, else fp32).  The state element type of the call is that
     of final_state.  With `gate` ([T, H, 128] bf16) and `norm_weight` ([128]
     fp32) the call is kda_prefill_gated: o holds the gated RMS-normalised
-    output, in bf16."""
+    output, in bf16.  `mode` "records" calls kda_prefill_records (the chunk
+    records stay valid in `workspace`), "scan" kda_prefill_scan (the scan over
+    records a "records" call left in `workspace`; see include/kda.h)."""
+    if mode not in ("full", "records", "scan"):
+        raise ValueError(f"unknown prefill mode {mode!r}")
+    if mode != "full" and (recurrent or gate is not None):
+        raise ValueError("record-keeping and scan-only calls run the plain chunked path")
+    if mode == "scan" and workspace is None:
+        raise ValueError("a scan-only call reads the records of an earlier call from its workspace")
     if gate is not None:
         if recurrent:
             raise ValueError("the fused output epilogue runs on the chunked path only")
@@ -177,6 +188,9 @@ def prefill(q, k, v, g, beta, conv_w, cu_seqlens_host, cu_seqlens_dev=None, init
         if gate is not None:
             _check(lib.kda_prefill_gated(*args, _ptr(workspace), wbytes, _ptr(gate), _ptr(norm_weight),
                                          float(norm_eps), _stream(stream)), "kda_prefill_gated")
+        elif mode != "full":
+            name = "kda_prefill_records" if mode == "records" else "kda_prefill_scan"
+            _check(getattr(lib, name)(*args, _ptr(workspace), wbytes, _stream(stream)), name)
         else:
             _check(lib.kda_prefill(*args, _ptr(workspace), wbytes, _stream(stream)), "kda_prefill")
     return o, final_state, conv_tail

@@ -173,6 +173,33 @@ kda_status kda_prefill_recurrent(const void* q, const void* k, const void* v, co
   return run_recurrent(a);
 }
 
+namespace {
+// kda_prefill and its record-keeping / scan-only forms
+kda_status prefill_mode(const PrefillArgs& args, void* workspace, size_t workspace_bytes, ChunkedMode mode) {
+  PrefillArgs a = args;
+  kda_status st = validate_prefill(a);
+  if (st != KDA_OK) return st;
+  if (a.N == 0) return KDA_OK;
+  if (a.dt == KDA_F32) {
+    if (mode != ChunkedMode::kFull) return KDA_ERR_UNSUPPORTED;  // the recurrent path keeps no records
+    return run_recurrent(a);
+  }
+  const size_t need = chunked_workspace_bytes(a.N, a.H, a.total_T);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 16)) return KDA_ERR_ALIGNMENT;
+  st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
+                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.state_dt, a.o, a.final_state, workspace,
+                      a.stream, OutputNorm{}, mode);
+  if (st != KDA_OK) return st;
+  return launch_tail<__nv_bfloat16>(a);
+}
+}  // namespace
+
+#define KDA_PREFILL_ARGS_STRUCT                                                                          \
+  PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,                        \
+                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, state_dt, o, final_state, conv_tail, \
+                (cudaStream_t)stream, 0, 0}
+
 kda_status kda_prefill(const void* q, const void* k, const void* v, const void* g,
                        const void* beta, const float* conv_w, const void* init_state,
                        const void* init_conv, const int32_t* cu_seqlens_dev,
@@ -180,22 +207,32 @@ kda_status kda_prefill(const void* q, const void* k, const void* v, const void* 
                        kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
                        void* o, void* final_state, void* conv_tail, void* workspace,
                        size_t workspace_bytes, void* stream) {
-  PrefillArgs a{q, k, v, g, beta, conv_w, init_state, init_conv, cu_seqlens_dev,
-                cu_seqlens_host, num_seqs, num_heads, dt, act, o_dt, state_dt, o, final_state, conv_tail,
-                (cudaStream_t)stream, 0, 0};
-  kda_status st = validate_prefill(a);
-  if (st != KDA_OK) return st;
-  if (a.N == 0) return KDA_OK;
-  if (dt == KDA_F32) return run_recurrent(a);
-  const size_t need = chunked_workspace_bytes(a.N, a.H, a.total_T);
-  if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
-  if (workspace && !aligned(workspace, 16)) return KDA_ERR_ALIGNMENT;
-  st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
-                      a.cu_host, a.N, a.H, a.act, a.o_dt, a.state_dt, a.o, a.final_state, workspace,
-                      a.stream);
-  if (st != KDA_OK) return st;
-  return launch_tail<__nv_bfloat16>(a);
+  KDA_PREFILL_ARGS_STRUCT;
+  return prefill_mode(a, workspace, workspace_bytes, ChunkedMode::kFull);
 }
+
+kda_status kda_prefill_records(const void* q, const void* k, const void* v, const void* g,
+                               const void* beta, const float* conv_w, const void* init_state,
+                               const void* init_conv, const int32_t* cu_seqlens_dev,
+                               const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                               kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                               void* o, void* final_state, void* conv_tail, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  KDA_PREFILL_ARGS_STRUCT;
+  return prefill_mode(a, workspace, workspace_bytes, ChunkedMode::kKeepRecords);
+}
+
+kda_status kda_prefill_scan(const void* q, const void* k, const void* v, const void* g,
+                            const void* beta, const float* conv_w, const void* init_state,
+                            const void* init_conv, const int32_t* cu_seqlens_dev,
+                            const int32_t* cu_seqlens_host, int num_seqs, int num_heads,
+                            kda_dtype dt, kda_conv_act act, kda_dtype o_dt, kda_dtype state_dt,
+                            void* o, void* final_state, void* conv_tail, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  KDA_PREFILL_ARGS_STRUCT;
+  return prefill_mode(a, workspace, workspace_bytes, ChunkedMode::kScanOnly);
+}
+#undef KDA_PREFILL_ARGS_STRUCT
 
 kda_status kda_prefill_gated(const void* q, const void* k, const void* v, const void* g,
                              const void* beta, const float* conv_w, const void* init_state,

@@ -85,7 +85,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
                   const int32_t* __restrict__ seq_order, int H, const uint8_t* __restrict__ records,
                   const int* __restrict__ ready, Tout* __restrict__ o, Ts* final_state,
                   uint64_t wait_ns, const __grid_constant__ CUtensorMap tm_z,
-                  const float* __restrict__ norm_w, float norm_eps) {
+                  const float* __restrict__ norm_w, float norm_eps, int keep_records) {
   static_assert(!EPI || sizeof(Tout) == 2, "the output epilogue writes bf16");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array itself so that the
@@ -233,7 +233,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       ++n_v;
     };
     // a record piece that the tensor core has read is dead: drop its lines
+    // (unless the records are kept for another scan over them)
     auto drop = [&](const uint8_t* base, uint32_t bytes) {
+      if (keep_records) return;
       for (uint32_t off = 128u * lane; off < bytes; off += 128u * 32u) discard_l2(base + off);
     };
     // with the prep kernel running concurrently, a chunk's record is read

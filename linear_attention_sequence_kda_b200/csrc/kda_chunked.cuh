@@ -56,6 +56,11 @@ struct OutputNorm {
   float eps = 0.f;
 };
 
+// What a chunked call runs: both kernels (the records are dropped from L2 as
+// the scan consumes them), both keeping the records in the workspace, or the
+// scan alone over records a keeping call left there.
+enum class ChunkedMode { kFull, kKeepRecords, kScanOnly };
+
 constexpr int OVERLAP_MAX_CHAINS = 96;  // leaves at least 52 of 148 SMs to prep
 // Prep SM-time per chunk-head relative to the scan's time per chunk of a
 // chain, used to pick when prep hands SMs over to the scan (the ratio that
@@ -125,7 +130,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
                                    const void* init_conv, const int32_t* cu_dev,
                                    const int32_t* cu_host, int N, int H, kda_dtype o_dt,
                                    kda_dtype state_dt, void* o, void* final_state, void* workspace,
-                                   const OutputNorm& norm, cudaStream_t stream) {
+                                   const OutputNorm& norm, ChunkedMode mode, cudaStream_t stream) {
   using T = __nv_bfloat16;
   // The chunk table below is staged from host memory that this call owns and
   // releases on return; a captured graph would read it again on every replay,
@@ -165,9 +170,11 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   int* ready = work_counter + 4;
   uint8_t* records = ws + hdr + chunk_sync_bytes(total, H);
   records += (128 - (reinterpret_cast<uintptr_t>(records) & 127)) & 127;
-  if (!cuda_ok(cudaMemsetAsync(work_counter, 0, 16 + (size_t)total * H * 4, stream))) return KDA_ERR_CUDA;
+  const bool scan_only = mode == ChunkedMode::kScanOnly;
+  if (!scan_only && !cuda_ok(cudaMemsetAsync(work_counter, 0, 16 + (size_t)total * H * 4, stream)))
+    return KDA_ERR_CUDA;
   const int64_t items = total * H;
-  const bool overlap = items > 0 && (int64_t)N * H <= OVERLAP_MAX_CHAINS;
+  const bool overlap = !scan_only && items > 0 && (int64_t)N * H <= OVERLAP_MAX_CHAINS;
 
   // TMA descriptors over the packed [total_T, H*128] tensors: 67-row boxes for
   // the inputs (3 halo rows + one chunk); 64-row boxes for the output tiles
@@ -185,7 +192,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     if (fork_side(stream, &side, &join) != KDA_OK) return KDA_ERR_CUDA;
     scan_stream = side;
   }
-  if (total > 0) {
+  if (total > 0 && !scan_only) {
     auto prep = chunk_prep_kernel<ACT>;
     if (!cuda_ok(cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM)))
       return KDA_ERR_CUDA;
@@ -226,7 +233,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, scan_stream>>>(
         tv, to, conv_w, (const Ts*)init_state, (const T*)init_conv, cu_dev, d_base, d_order, H, records,
         overlap ? ready : nullptr, (Tout*)o, (Ts*)final_state, scan_wait_ns(items), tz, norm.weight,
-        norm.eps);
+        norm.eps, mode == ChunkedMode::kFull ? 0 : 1);
     return true;
   };
   using Plain = std::false_type;
@@ -249,14 +256,15 @@ inline kda_status launch_chunked(const void* q, const void* k, const void* v, co
                                  const int32_t* cu_host, int N, int H, kda_conv_act act,
                                  kda_dtype o_dt, kda_dtype state_dt, void* o, void* final_state,
                                  void* workspace, cudaStream_t stream,
-                                 const OutputNorm& norm = OutputNorm{}) {
+                                 const OutputNorm& norm = OutputNorm{},
+                                 ChunkedMode mode = ChunkedMode::kFull) {
   if (act == KDA_CONV_SILU)
     return launch_chunked_t<KDA_CONV_SILU>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
                                            cu_host, N, H, o_dt, state_dt, o, final_state, workspace, norm,
-                                           stream);
+                                           mode, stream);
   return launch_chunked_t<KDA_CONV_NONE>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
                                          cu_host, N, H, o_dt, state_dt, o, final_state, workspace, norm,
-                                         stream);
+                                         mode, stream);
 }
 
 }  // namespace kda

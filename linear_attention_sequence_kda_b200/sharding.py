@@ -14,8 +14,12 @@ linear in the state, so segment r maps its initial state as
 S_out = A_r S_in + B_r.  context_parallel_prefill runs, on every rank:
   1. the conv halo: each rank's last three raw tokens, gathered, give the next
      rank its conv history;
-  2. the carry: one prefill call over the segment entered twice, from S = 0
-     (final state B_r) and from S = I with v = 0 (final state A_r);
+  2. the carry: the segment entered from S = 0 (final state B_r) and from
+     S = I with v = 0 (final state A_r).  On the chunked (bf16) path the chunk
+     records, which depend on q, k, g and beta only, are prepared once: a
+     record-keeping prefill gives B_r and two scans over the same records give
+     A_r and, in step 5, the outputs.  On the fp32 path one prefill call runs
+     the segment twice;
   3. the exchange: all ranks gather every (A_j, B_j);
   4. the composition S_in(r) = A_{r-1}(... (A_0 S_0 + B_0) ...) + B_{r-1};
   5. the segment's prefill from S_in(r): its outputs, and on the last rank the
@@ -91,12 +95,37 @@ def compose_initial_state(S0, As, Bs, rank: int, affine: Callable):
     return S
 
 
-def segment_carry(lib, q, k, v, g, beta, conv_w, prev_tail, act: int = 0, stream=None):
-    """(A, B) of one segment, [1, H, D, D] fp32 each, from one prefill call over
-    the segment entered twice: from S = 0 with the real inputs (final state B)
-    and from S = I with v = 0 and a zero v history (final state A)."""
+def segment_workspace(lib, q):
+    """A workspace for the segment's chunk records (None where the call
+    needs none: fp32 inputs)."""
+    import torch
+    T, H, _ = q.shape
+    if q.dtype != torch.bfloat16:
+        return None
+    need = lib.workspace_size(1, T, H, T)
+    return torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if need > 0 else None
+
+
+def segment_carry(lib, q, k, v, g, beta, conv_w, prev_tail, act: int = 0, stream=None, workspace=None):
+    """(A, B) of one segment, [1, H, D, D] fp32 each: the segment entered from
+    S = 0 with the real inputs (final state B) and from S = I with v = 0 and a
+    zero v history (final state A).  With a `workspace` (bf16 inputs) the chunk
+    records are prepared once (a record-keeping prefill gives B, a scan over
+    the same records A) and stay in `workspace` for the segment's final scan;
+    otherwise one prefill call runs the segment twice."""
     import torch
     T, H, D = q.shape
+    if workspace is not None:
+        cu = np.array([0, T], dtype=np.int32)
+        zero = torch.zeros((1, H, D, D), dtype=torch.float32, device=q.device)
+        eye = torch.eye(D, dtype=torch.float32, device=q.device).expand(1, H, D, D).contiguous()
+        hist0 = prev_tail.clone()
+        hist0[:, 2] = 0
+        _, B, _ = lib.prefill(q, k, v, g, beta, conv_w, cu, init_state=zero, init_conv=prev_tail, act=act,
+                              stream=stream, workspace=workspace, mode="records")
+        _, A, _ = lib.prefill(q, k, torch.zeros_like(v), g, beta, conv_w, cu, init_state=eye, init_conv=hist0,
+                              act=act, stream=stream, workspace=workspace, mode="scan")
+        return A, B
     two = lambda x, y=None: torch.cat([x, x if y is None else y]).contiguous()  # noqa: E731
     init = torch.zeros((2, H, D, D), dtype=torch.float32, device=q.device)
     init[1] = torch.eye(D, dtype=torch.float32, device=q.device)
@@ -135,10 +164,13 @@ def context_parallel_prefill(lib, q, k, v, g, beta, conv_w, rank: int, world: in
         prev_tail = init_conv
     else:
         prev_tail = torch.zeros((1, 3, 3, H * D), dtype=q.dtype, device=q.device)
-    A, B = segment_carry(lib, q, k, v, g, beta, conv_w, prev_tail, act, stream)
+    ws = segment_workspace(lib, q)
+    A, B = segment_carry(lib, q, k, v, g, beta, conv_w, prev_tail, act, stream, workspace=ws)
     As, Bs = all_gather(A), all_gather(B)
     S0 = init_state if init_state is not None else torch.zeros((1, H, D, D), dtype=torch.float32, device=q.device)
     S_in = compose_initial_state(S0, As, Bs, rank, lib.state_affine)
     kw = {} if o_dtype is None else {"o_dtype": o_dtype}
+    if ws is not None:  # the segment's records are in ws: its scan alone
+        kw.update(workspace=ws, mode="scan")
     return lib.prefill(q, k, v, g, beta, conv_w, np.array([0, T], dtype=np.int32), init_state=S_in,
                        init_conv=prev_tail, act=act, stream=stream, **kw)

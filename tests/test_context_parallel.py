@@ -19,12 +19,17 @@ D = 128
 
 class OracleLib:
     """prefill / state_affine of the library's binding, evaluated by the fp64
-    oracle on the CPU (test stand-in)."""
+    oracle on the CPU (test stand-in).  Record-keeping and scan-only calls
+    (`mode`, `workspace`) give what the library gives for them, the prefill of
+    their arguments, so the oracle recomputes it; each call is logged, so that
+    the driver's use of the modes can be checked."""
+    calls = []
 
     @staticmethod
     def prefill(q, k, v, g, beta, conv_w, cu, init_state=None, init_conv=None, act=0, stream=None, **kw):
         import kda_inputs as ki
         import oracle
+        OracleLib.calls.append(kw.get("mode", "full"))
         cu = np.asarray(cu, dtype=np.int32)
         N, (T, H, _) = len(cu) - 1, q.shape
         inp = ki.PrefillInputs(q, k, v, g, beta, conv_w, init_state, init_conv, cu)
@@ -40,6 +45,10 @@ class OracleLib:
         return o, S, tail
 
     @staticmethod
+    def workspace_size(num_seqs, total_tokens, num_heads, max_seqlen, dtype=None):
+        return 16  # a token workspace: the oracle keeps no records
+
+    @staticmethod
     def state_affine(A, S, B, S_out=None, stream=None):
         return A.double() @ S.double() + B.double()
 
@@ -50,13 +59,13 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, bounds, result_path):
+def _worker(rank, world, port, bounds, result_path, dtype=torch.float32):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         import kda_inputs as ki
         from linear_attention_sequence_kda_b200.sharding import context_parallel_prefill
-        inp = ki.make_prefill([bounds[-1]], 2, torch.float32, 93, state_std=0.02, conv_history=True)
+        inp = ki.make_prefill([bounds[-1]], 2, dtype, 93, state_std=0.02, conv_history=True)
         t0, t1 = bounds[rank], bounds[rank + 1]
 
         def gather(t):
@@ -79,23 +88,26 @@ def _worker(rank, world, port, bounds, result_path):
             tail_ok = all(np.array_equal(outs[-1][2][0, x, :, h * D:(h + 1) * D], full[(0, h)].tail[x])
                           for h in range(2) for x in range(3))
             with open(result_path, "w") as f:
-                f.write(f"{err_o} {err_s} {int(tail_ok)}")
+                f.write(f"{err_o} {err_s} {int(tail_ok)} {','.join(OracleLib.calls)}")
     finally:
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("bounds", [[0, 150, 280], [0, 70, 73, 230]])
-def test_segments_over_gloo_equal_the_whole_sequence(tmp_path, bounds):
+def test_segments_over_gloo_equal_the_whole_sequence(tmp_path, bounds, dtype):
     """Two segments of 150 and 130 tokens (partial chunks at both ends of the
     boundary); three segments whose middle one has the minimum of 3 tokens, so
     that the last segment's conv history is that segment alone.  Nonzero
-    initial state and conv history."""
+    initial state and conv history.  With bf16 inputs the driver prepares each
+    segment's records once: one record-keeping call, then two scans."""
     path = str(tmp_path / "cp.txt")
     world = len(bounds) - 1
-    mp.start_processes(_worker, args=(world, _free_port(), bounds, path), nprocs=world, start_method="spawn",
-                       join=True)
-    err_o, err_s, tail_ok = open(path).read().split()
+    mp.start_processes(_worker, args=(world, _free_port(), bounds, path, dtype), nprocs=world,
+                       start_method="spawn", join=True)
+    err_o, err_s, tail_ok, calls = open(path).read().split()
     assert float(err_o) < 1e-9 and float(err_s) < 1e-9 and tail_ok == "1"
+    assert calls == ("records,scan,scan" if dtype == torch.bfloat16 else "full,full")
 
 
 def test_conv_halo_needs_three_tokens():

@@ -10,8 +10,9 @@ import torch
 import kda_inputs as ki
 import linear_attention_sequence_kda_b200 as kda
 import oracle
-from linear_attention_sequence_kda_b200.sharding import compose_initial_state, conv_halo, segment_carry
-from parity import TOL, rel_err, run_prefill
+from linear_attention_sequence_kda_b200.sharding import (compose_initial_state, conv_halo, segment_carry,
+                                                         segment_workspace)
+from parity import TOL, rel_err, run_prefill, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -34,8 +35,8 @@ def test_state_affine_matches_fp64_product():
     assert ((got16.double() - want16).abs() <= 2.0 ** -7 * want16.abs() + 1e-6).all()
 
 
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_four_segments_equal_one_call(dtype):
+@pytest.mark.parametrize("dtype,records", [(torch.bfloat16, False), (torch.bfloat16, True), (torch.float32, False)])
+def test_four_segments_equal_one_call(dtype, records):
     bounds = [0, 700, 1100, 1950, 2300]  # segments of 700, 400, 850, 350 tokens
     H = 4
     inp = ki.make_prefill([bounds[-1]], H, dtype, 95, state_std=0.02, conv_history=True)
@@ -44,19 +45,22 @@ def test_four_segments_equal_one_call(dtype):
     seg = [{n: dev[n][t0:t1].contiguous() for n in ("q", "k", "v", "g", "beta")}
            for t0, t1 in zip(bounds[:-1], bounds[1:])]
     halos = [conv_halo(s["q"], s["k"], s["v"]) for s in seg]
-    As, Bs = [], []
+    As, Bs, wss = [], [], []
     for r, s in enumerate(seg):
         prev = dev["init_conv"] if r == 0 else halos[r - 1]
-        A, B = segment_carry(kda, s["q"], s["k"], s["v"], s["g"], s["beta"], dev["conv_w"], prev)
+        ws = segment_workspace(kda, s["q"]) if records else None  # records prepared once per segment
+        A, B = segment_carry(kda, s["q"], s["k"], s["v"], s["g"], s["beta"], dev["conv_w"], prev, workspace=ws)
         As.append(A)
         Bs.append(B)
+        wss.append(ws)
     outs = []
     for r, s in enumerate(seg):
         S_in = compose_initial_state(dev["init_state"], As, Bs, r, kda.state_affine)
         prev = dev["init_conv"] if r == 0 else halos[r - 1]
         T = s["q"].shape[0]
+        kw = {"workspace": wss[r], "mode": "scan"} if records else {}
         outs.append(kda.prefill(s["q"], s["k"], s["v"], s["g"], s["beta"], dev["conv_w"],
-                                np.array([0, T], dtype=np.int32), init_state=S_in, init_conv=prev))
+                                np.array([0, T], dtype=np.int32), init_state=S_in, init_conv=prev, **kw))
     torch.cuda.synchronize()
     assert kda.check_async_status() == 0
     o = torch.cat([x[0] for x in outs]).cpu()
@@ -70,3 +74,34 @@ def test_four_segments_equal_one_call(dtype):
         assert rel_err(S[0, h].double().numpy(), ref[(0, h)].final_state) <= tol, h
         # against one call on the GPU
         assert rel_err(o[:, h].double().numpy(), whole_o[:, h].cpu().double().numpy()) <= tol, h
+
+
+@pytest.mark.parametrize("lens,H", [([700, 130, 5], 4), ([300, 300], 64)])
+def test_scan_over_kept_records_equals_prefill(lens, H):
+    """kda_prefill_scan over the records of a kda_prefill_records call equals
+    kda_prefill of its own arguments bit for bit, with other values, initial
+    states, v history and output type, and again on a second scan; the
+    records call itself equals kda_prefill.  12 chains (the overlapped
+    schedule) and 128 chains (prep, then the scan)."""
+    inp = ki.make_prefill(lens, H, torch.bfloat16, 96, state_std=0.02, conv_history=True)
+    d = to_dev(inp)
+    ws = torch.empty(kda.workspace_size(len(lens), sum(lens), H, max(lens)), dtype=torch.uint8, device="cuda")
+    cu = inp.cu_seqlens
+    args = lambda dd: (dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["conv_w"], cu, dd["cu_dev"])  # noqa: E731
+    o1, S1, t1 = kda.prefill(*args(d), d["init_state"], d["init_conv"], workspace=ws, mode="records")
+    o1f, S1f, t1f = kda.prefill(*args(d), d["init_state"], d["init_conv"])
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o1f) and torch.equal(S1, S1f) and torch.equal(t1, t1f)
+    # other v, v history and initial state: the records do not depend on them
+    d2 = dict(d)
+    d2["v"] = ki.randn(tuple(inp.v.shape), 97, 1, dtype=torch.bfloat16).cuda()
+    hist = d["init_conv"].clone()
+    hist[:, 2] = ki.randn(tuple(hist[:, 2].shape), 97, 2, dtype=torch.bfloat16).cuda()
+    S0 = ki.randn(tuple(inp.init_state.shape), 97, 3, std=0.05).cuda()
+    want = kda.prefill(*args(d2), S0, hist, o_dtype=torch.bfloat16)
+    for _ in range(2):
+        got = kda.prefill(*args(d2), S0, hist, workspace=ws, mode="scan", o_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert kda.check_async_status() == 0
+        for x, y in zip(got, want):
+            assert torch.equal(x, y)
