@@ -365,6 +365,10 @@ def main():
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill leg (profiling only)")
     ap.add_argument("--decode-seqs", type=int, default=256,
                     help="reduced decode batch (profiling only; the reported workload uses 256)")
+    ap.add_argument("--workload", default="long", choices=["long", "4x4096"],
+                    help="the prefill leg's workload (profiling only; the reported workload is long)")
+    ap.add_argument("--gated", action="store_true",
+                    help="run the prefill leg with the fused output epilogue (profiling only)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -392,13 +396,17 @@ def main():
 
     # ---------------- prefill: long-context workload, resident in HBM ----------
     heads, T_run = args.heads, args.seq_len
-    if (heads, T_run) == (H, T_LONG):
+    profiling = args.workload != "long" or args.gated
+    if args.workload == "4x4096":
+        inp = ki.workload(1, heads)
+        T_run = inp.total_tokens
+    elif (heads, T_run) == (H, T_LONG):
         inp = ki.workload(2)
     else:  # same recipe, reduced size (for profiler captures)
         inp = ki.make_prefill([T_run], heads, torch.bfloat16, ki.BASE_SEED + 2, gate="bimodal")
     with ClockSampler(torch.cuda.current_device()) as clk:
         head_leg, ctx = run_prefill_leg(args, world, dev, stream, kda, inp, args.steps, hbm_peak, bf16_peak,
-                                        peak_src, keep=True)
+                                        peak_src, keep=True, gated=args.gated)
     d, o, S, prefill_into = ctx
     ms = head_leg["ms_per_step"]
     tokens_per_rank = T_run
@@ -420,7 +428,7 @@ def main():
 
     # ---------------- the other prefill workloads (multi-sequence schedules) ----
     other_legs = {}
-    if not args.no_other_prefill and (heads, T_run) == (H, T_LONG):
+    if not args.no_other_prefill and (heads, T_run) == (H, T_LONG) and not profiling:
         other_legs["prefill_4x4096"] = run_prefill_leg(args, world, dev, stream, kda, ki.workload(1),
                                                        args.steps, hbm_peak, bf16_peak, peak_src)[0]
         other_legs["prefill_varlen"] = run_prefill_leg(args, world, dev, stream, kda, ki.workload(3),
@@ -448,8 +456,8 @@ def main():
         "mtp_fused_bf16_state": mtp16_line,
         **other_legs,
     }
-    if (heads, T_run) != (H, T_LONG):
-        line["config"]["note"] = "reduced profiling size, not the reported workload"
+    if (heads, T_run) != (H, T_LONG) or profiling:
+        line["config"]["note"] = "profiling run, not the reported workload"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
         line["oracle_per_workload"] = oracle_per_workload()
@@ -675,7 +683,7 @@ def run_decode(args, world, dev, stream, kda, hbm_peak, state_dtype=torch.float3
             "state_gbs": dec_state_gbs, "ms_per_step": dec_ms, "tokens_per_s": dec.num_seqs / (dec_ms / 1e3),
             "roofline": {"kernel": "kda_decode", "bound": "hbm", "achieved": dec_alg_gbs, "peak": hbm_peak,
                          "unit": "GB/s", "frac": dec_alg_gbs / hbm_peak, "state_frac": dec_state_gbs / hbm_peak,
-                         "traffic": recorded_traffic("kda_decode") if sb == 4 else None,
+                         "traffic": recorded_traffic("kda_decode" if sb == 4 else "kda_decode bf16_state"),
                          "algorithmic_bytes_per_launch": alg},
             "gpu_launches": args.steps * DECODE_LAUNCHES}
 
@@ -719,7 +727,9 @@ def run_mtp(args, world, dev, stream, kda, hbm_peak, state_dtype=torch.float32):
             "ms_per_step": ms, "verify_ms": verify_ms, "commit_ms": ms - verify_ms,
             "state_gbs": npairs * 3 * D * D * sb / (ms / 1e3) / 1e9,
             "roofline": {"kernel": "kda_decode_verify + kda_decode_commit", "bound": "hbm", "achieved": gbs,
-                         "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak, "traffic": None,
+                         "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "traffic": recorded_traffic("kda_decode_verify + kda_decode_commit"
+                                                     + ("" if sb == 4 else " bf16_state")),
                          "algorithmic_bytes_per_launch": alg},
             "gpu_launches": args.steps * (MTP_LAUNCHES + 1)}
 
@@ -765,7 +775,8 @@ def run_mtp_fused(args, world, dev, stream, kda, hbm_peak, state_dtype=torch.flo
             "verified_rows_per_s": N * MTP_ROWS / (ms / 1e3), "kept_tokens_per_s": int(mt.n_accept.sum()) / (ms / 1e3),
             "ms_per_step": ms, "state_gbs": npairs * 2 * D * D * sb / (ms / 1e3) / 1e9,
             "roofline": {"kernel": "kda_decode_commit_verify", "bound": "hbm", "achieved": gbs, "peak": hbm_peak,
-                         "unit": "GB/s", "frac": gbs / hbm_peak, "traffic": None,
+                         "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "traffic": recorded_traffic("kda_decode_commit_verify" + ("" if sb == 4 else " bf16_state")),
                          "algorithmic_bytes_per_launch": alg},
             "gpu_launches": args.steps}
 
