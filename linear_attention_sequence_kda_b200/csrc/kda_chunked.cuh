@@ -67,6 +67,10 @@ constexpr int OVERLAP_MAX_CHAINS = 96;  // leaves at least 52 of 148 SMs to prep
 // gave the shortest overlapped call on B200, 64 heads x 65,536 tokens, among
 // 2.8 .. 4.4; the model value from the two kernels' separate timings is ~3).
 constexpr double PREP_PER_SCAN_CHUNK = 3.2;
+// The same with the output epilogue fused into the scan, whose chain is slower
+// per chunk, so the scan takes its SMs earlier (best among 2.0 .. 3.6: 2.0 and
+// 2.4 within noise of each other, 0.3-0.5 ms shorter than at 3.2).
+constexpr double PREP_PER_SCAN_CHUNK_GATED = 2.2;
 
 // Pending host-side fault (kda_inject_fault), taken by the first call that
 // applies it.
@@ -209,7 +213,8 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
       // remainder on the other SMs end together
       const int chains = N * H;
       const int64_t longest = *std::max_element(nch.begin(), nch.end());
-      double f = 1.0 - (double)longest * (sms - chains) / ((double)items * PREP_PER_SCAN_CHUNK);
+      const double r = norm.gate ? PREP_PER_SCAN_CHUNK_GATED : PREP_PER_SCAN_CHUNK;
+      double f = 1.0 - (double)longest * (sms - chains) / ((double)items * r);
       f = f < 0.0 ? 0.0 : (f > 1.0 ? 1.0 : f);
       vacate_sms = chains;
       vacate_after = (int)(f * (double)items);
