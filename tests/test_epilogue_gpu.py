@@ -103,7 +103,7 @@ def test_gated_prefill_long_context_full_size():
 
 
 def test_gated_prefill_extreme_gates():
-    """Gates far in both tails (sigmoid 0 and 1 in fp32) and a zero eps."""
+    """Gates far in both tails (sigmoid 1 in fp32, and all but closed) and a zero eps."""
     inp = ki.make_prefill([130], 2, torch.bfloat16, 35, state_std=0.02, conv_history=True)
     d = to_dev(inp)
     T, H = inp.q.shape[0], inp.q.shape[1]
@@ -116,7 +116,8 @@ def test_gated_prefill_extreme_gates():
     for (n, h), p in ref.items():
         yr = epilogue.gated_rmsnorm(p.o, z[:, h].double().numpy(), w.double().numpy(), 0.0)
         _check(y[:, h].float().cpu().numpy(), yr, 2e-2, f"head {h}")
-    assert torch.all(y[::2].float() == 0)
+    # a closed gate: sigmoid(-100) = 3.7e-44 (the kernel's sigmoid saturates at 2^-64 there)
+    assert torch.all(y[::2].float().abs() < 1e-15)
 
 
 @pytest.mark.parametrize("odt", [torch.float32, torch.bfloat16])
