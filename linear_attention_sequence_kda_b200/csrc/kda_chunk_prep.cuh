@@ -13,16 +13,19 @@
 // (segment, head) in parallel, and stored as a record of operand tiles already
 // in the shared-memory layout the scan kernel's tensor-core instructions read.
 //
-// Record (REC_BYTES, 1024-aligned), all tiles fp32 values rounded to tf32,
-// K-major 128-byte swizzled (kda_tc.cuh):
+// The record (kda_record.cuh), in the plainly normalised form (q_hat, k_hat;
+// r = 1), all tiles fp32 values rounded to tf32, K-major 128-byte swizzled
+// (kda_tc.cuh):
 //   RA  [128][128 k]: -W and Q~ = e^{Gamma_t} * q_hat_t stacked by rows, -W
 //                     first for even chunks of a segment, Q~ first for odd ones
 //                     (so that one N = 128 product writes U next to the output
 //                     buffer of the chunk's parity)
 //   TS  [64 t][ 64]:  T strictly below the diagonal
-//   PS  [64 t][ 64]:  P strictly below the diagonal
-//   KB  [128 k][64]:  (e^{Gamma_C - Gamma_t} * k_hat_t)^T
-//   SC  fp32 beta[64], P_tt[64] (exact q_hat_t . k_hat_t), e^{Gamma_C}[128]
+//   B2  [192][64 t]:  P strictly below the diagonal and
+//                     (e^{Gamma_C - Gamma_t} * k_hat_t)^T, in the same parity
+//                     order
+//   SC  fp32 b = beta[64], d = P_tt[64] (exact q_hat_t . k_hat_t), r = 1,
+//       e^{Gamma_C}[128]
 // The diagonal terms beta_t v_t (of T V) and P_tt u_t (of P U) are applied in
 // fp32 by the scan kernel; they carry the largest single-token contributions.
 //
@@ -39,7 +42,7 @@
 // with x = q (the P Gram) or k (the M Gram); the wanted entries are the
 // row-0..31 x column-0..31 and row-32..95 x column-32..63 blocks.
 //
-// Two blocks of 256 threads share an SM (88 KB of shared memory and 256 TMEM
+// Two blocks of 256 threads share an SM (90 KB of shared memory and 256 TMEM
 // columns each), so that one block's barrier and tensor-core waits are covered
 // by the other's work.  Thread (c, b) owns key/query channel c of token half b;
 // the short-conv outputs of a chunk live in TMEM (lane = channel) rather than
@@ -280,7 +283,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (tid == 0 && pending >= 0) tc::bulk_wait_read();  // step 3 overwrites the previous -W staging
   __syncthreads();
 
-  // ---- 3. normalise; Gram operands, record tiles QT and KB, stashes ---------
+  // ---- 3. normalise; Gram operands, record tiles Q~ and K-bar^T, stashes ----
   const float carry = hb ? ms[MB_CARRY + ch] : 0.f;         // gate total of half 0
   const float g1m = ms[MB_CARRY + ch] + ms[MB_G1M + ch];     // G at row 48
   const float gC = ms[MB_CARRY + ch] + ms[MB_G1T + ch];      // G at the chunk end
