@@ -152,3 +152,23 @@ def test_output_norm_after_decode():
     for (n, h), p in ref.items():
         yr = epilogue.gated_rmsnorm(p.o[0], z[n, h].double().numpy(), w.double().numpy(), EPS)
         _check(yc[n, h], yr, 1e-4, f"seq {n} head {h}")
+
+
+@pytest.mark.parametrize("silu", [0, 1])
+def test_gated_prefill_bf16_state(silu):
+    """The epilogue instance with bf16 state storage and both conv activations:
+    the final state equals the plain call's bit for bit, and the output the
+    plain call's output through the standalone epilogue within 2^-7."""
+    inp = ki.make_prefill([400, 90], 3, torch.bfloat16, 38 + silu, state_std=0.02, conv_history=True)
+    d = to_dev(inp)
+    d["init_state"] = d["init_state"].to(torch.bfloat16)
+    T, H = inp.q.shape[0], inp.q.shape[1]
+    z, w = ki.make_output_norm(T, H, 38)
+    zd, wd = z.cuda(), w.cuda()
+    y, S, tail = run_prefill(inp, dev_inputs=d, act=silu, gate=zd, norm_weight=wd, norm_eps=EPS)
+    o, S0, tail0 = run_prefill(inp, dev_inputs=d, act=silu)
+    assert S.dtype == torch.bfloat16 and torch.equal(S, S0) and torch.equal(tail, tail0)
+    y2 = kda.output_norm(o, zd, wd, EPS)
+    torch.cuda.synchronize()
+    a, b = y.float(), y2.float()
+    assert torch.all((a - b).abs() <= 2.0 ** -7 * b.abs() + 1e-6), float((a - b).abs().max())
