@@ -76,8 +76,9 @@ def test_four_segments_equal_one_call(dtype, records):
         assert rel_err(o[:, h].double().numpy(), whole_o[:, h].cpu().double().numpy()) <= tol, h
 
 
-@pytest.mark.parametrize("lens,H", [([700, 130, 5], 4), ([300, 300], 64)])
-def test_scan_over_kept_records_equals_prefill(lens, H):
+@pytest.mark.parametrize("lens,H,sdt", [([700, 130, 5], 4, torch.float32), ([300, 300], 64, torch.float32),
+                                        ([500, 64], 4, torch.bfloat16)])
+def test_scan_over_kept_records_equals_prefill(lens, H, sdt):
     """kda_prefill_scan over the records of a kda_prefill_records call equals
     kda_prefill of its own arguments bit for bit, with other values, initial
     states, v history and output type, and again on a second scan; the
@@ -85,6 +86,7 @@ def test_scan_over_kept_records_equals_prefill(lens, H):
     schedule) and 128 chains (prep, then the scan)."""
     inp = ki.make_prefill(lens, H, torch.bfloat16, 96, state_std=0.02, conv_history=True)
     d = to_dev(inp)
+    d["init_state"] = d["init_state"].to(sdt)
     ws = torch.empty(kda.workspace_size(len(lens), sum(lens), H, max(lens)), dtype=torch.uint8, device="cuda")
     cu = inp.cu_seqlens
     args = lambda dd: (dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["conv_w"], cu, dd["cu_dev"])  # noqa: E731
@@ -97,7 +99,7 @@ def test_scan_over_kept_records_equals_prefill(lens, H):
     d2["v"] = ki.randn(tuple(inp.v.shape), 97, 1, dtype=torch.bfloat16).cuda()
     hist = d["init_conv"].clone()
     hist[:, 2] = ki.randn(tuple(hist[:, 2].shape), 97, 2, dtype=torch.bfloat16).cuda()
-    S0 = ki.randn(tuple(inp.init_state.shape), 97, 3, std=0.05).cuda()
+    S0 = ki.randn(tuple(inp.init_state.shape), 97, 3, std=0.05).cuda().to(sdt)
     want = kda.prefill(*args(d2), S0, hist, o_dtype=torch.bfloat16)
     for _ in range(2):
         got = kda.prefill(*args(d2), S0, hist, workspace=ws, mode="scan", o_dtype=torch.bfloat16)
