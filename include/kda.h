@@ -100,8 +100,12 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int num_he
  *   init_conv        : [N, 3, 3, H*128] raw q/k/v of the 3 tokens before each
  *                      segment (oldest first), or NULL for zeros.
  *   cu_seqlens_dev   : [N+1] int32 device copy of the segment offsets.
- *   cu_seqlens_host  : [N+1] int32 host copy (used for scheduling; must equal
- *                      the device copy).  cu[0] == 0, non-decreasing.
+ *   cu_seqlens_host  : [N+1] int32 host copy; must equal the device copy.
+ *                      cu[0] == 0, non-decreasing.  The chunked (bf16) path
+ *                      validates and schedules from this copy and stages it
+ *                      in the workspace with its chunk table, and its kernels
+ *                      read only that staged copy; the fp32 recurrent path's
+ *                      kernels read cu_seqlens_dev.
  *   o_dt             : element type of o (KDA_F32 or KDA_BF16).
  *   state_dt         : element type of init_state and final_state.
  *   o                : out [total_T, H, 128] (o_dt).  Must not alias inputs.

@@ -187,10 +187,12 @@ kda_status prefill_mode(const PrefillArgs& args, void* workspace, size_t workspa
   const size_t need = chunked_workspace_bytes(a.N, a.H, a.total_T);
   if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
   if (workspace && !aligned(workspace, 16)) return KDA_ERR_ALIGNMENT;
+  const int32_t* cu_used = nullptr;
   st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
                       a.cu_host, a.N, a.H, a.act, a.o_dt, a.state_dt, a.o, a.final_state, workspace,
-                      a.stream, OutputNorm{}, mode);
+                      a.stream, OutputNorm{}, mode, &cu_used);
   if (st != KDA_OK) return st;
+  a.cu_dev = cu_used;  // the staged host offsets, as the chunked kernels used
   return launch_tail<__nv_bfloat16>(a);
 }
 }  // namespace
@@ -259,10 +261,12 @@ kda_status kda_prefill_gated(const void* q, const void* k, const void* v, const 
   norm.gate = gate;
   norm.weight = norm_weight;
   norm.eps = norm_eps;
+  const int32_t* cu_used = nullptr;
   st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
                       a.cu_host, a.N, a.H, a.act, a.o_dt, a.state_dt, a.o, a.final_state, workspace,
-                      a.stream, norm);
+                      a.stream, norm, ChunkedMode::kFull, &cu_used);
   if (st != KDA_OK) return st;
+  a.cu_dev = cu_used;
   return launch_tail<__nv_bfloat16>(a);
 }
 
@@ -543,9 +547,11 @@ extern "C" kda_status kda_prefill_noalloc(const void* q, const void* k, const vo
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != KDA_OK) return st;
+  const int32_t* cu_used = nullptr;
   st = launch_chunked(a.q, a.k, a.v, a.g, a.beta, a.conv_w, a.init_state, a.init_conv, a.cu_dev,
                       a.cu_host, a.N, a.H, a.act, a.o_dt, a.state_dt, a.o, a.final_state, scratch,
-                      a.stream);
+                      a.stream, OutputNorm{}, ChunkedMode::kFull, &cu_used);
   if (st != KDA_OK) return st;
+  a.cu_dev = cu_used;
   return launch_tail<__nv_bfloat16>(a);
 }

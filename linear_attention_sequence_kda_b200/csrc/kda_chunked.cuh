@@ -33,7 +33,7 @@ namespace kda {
 // then REC_BYTES per (chunk, head)
 inline int64_t chunk_bound(int N, int64_t total_tokens) { return total_tokens / CH + N; }
 inline size_t chunk_header_bytes(int N, int64_t nchunks) {
-  const size_t b = (size_t)nchunks * sizeof(int2) + (size_t)(N + 1) * 4 + (size_t)N * 4;
+  const size_t b = (size_t)nchunks * sizeof(int2) + (size_t)(N + 1) * 4 + (size_t)N * 4 + (size_t)(N + 1) * 4;
   return (b + 1023) & ~(size_t)1023;
 }
 // work counter (16 B) and one ready flag per (chunk, head)
@@ -134,8 +134,10 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
                                    const void* init_conv, const int32_t* cu_dev,
                                    const int32_t* cu_host, int N, int H, kda_dtype o_dt,
                                    kda_dtype state_dt, void* o, void* final_state, void* workspace,
-                                   const OutputNorm& norm, ChunkedMode mode, cudaStream_t stream) {
+                                   const OutputNorm& norm, ChunkedMode mode, cudaStream_t stream,
+                                   const int32_t** cu_used) {
   using T = __nv_bfloat16;
+  (void)cu_dev;  // the kernels read the host offsets staged below, never the caller's device copy
   // The chunk table below is staged from host memory that this call owns and
   // releases on return; a captured graph would read it again on every replay,
   // long after it is gone, so stream capture is refused.
@@ -154,6 +156,11 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   int2* tab = reinterpret_cast<int2*>(host.data());
   int32_t* base = reinterpret_cast<int32_t*>(host.data() + (size_t)total * sizeof(int2));
   int32_t* order = base + (N + 1);
+  // the segment offsets the kernels read: the host copy, staged with the chunk
+  // table, so that the schedule and every kernel see the same segments even
+  // if the caller's device copy differs from it
+  int32_t* cu_stage = order + N;
+  std::copy(cu_host, cu_host + N + 1, cu_stage);
   int64_t c = 0;
   for (int n = 0; n < N; ++n) {
     base[n] = (int32_t)c;
@@ -170,6 +177,8 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
   const int2* d_tab = reinterpret_cast<const int2*>(ws);
   const int32_t* d_base = reinterpret_cast<const int32_t*>(ws + (size_t)total * sizeof(int2));
   const int32_t* d_order = d_base + (N + 1);
+  const int32_t* d_cu = d_order + N;
+  if (cu_used) *cu_used = d_cu;
   int* work_counter = reinterpret_cast<int*>(ws + hdr);
   int* ready = work_counter + 4;
   uint8_t* records = ws + hdr + chunk_sync_bytes(total, H);
@@ -223,7 +232,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     // scan waits on
     int* publish = overlap && !take_fault(KDA_FAULT_DROP_READY) ? ready : nullptr;
     prep<<<blocks, PREP_THREADS, PREP_SMEM, stream>>>(tq, tk, tg, (const T*)beta, conv_w, (const T*)init_conv,
-                                                        cu_dev, d_tab, H, (int)items, records, work_counter,
+                                                        d_cu, d_tab, H, (int)items, records, work_counter,
                                                         publish, vacate_sms, vacate_after);
     if (!cuda_ok(cudaGetLastError())) return KDA_ERR_CUDA;
   }
@@ -236,7 +245,7 @@ inline kda_status launch_chunked_t(const void* q, const void* k, const void* v, 
     if (!cuda_ok(cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM)))
       return false;
     scan<<<(unsigned)N * H, SCAN_THREADS, SCAN_SMEM, scan_stream>>>(
-        tv, to, conv_w, (const Ts*)init_state, (const T*)init_conv, cu_dev, d_base, d_order, H, records,
+        tv, to, conv_w, (const Ts*)init_state, (const T*)init_conv, d_cu, d_base, d_order, H, records,
         overlap ? ready : nullptr, (Tout*)o, (Ts*)final_state, scan_wait_ns(items), tz, norm.weight,
         norm.eps, mode == ChunkedMode::kFull ? 0 : 1);
     return true;
@@ -262,14 +271,15 @@ inline kda_status launch_chunked(const void* q, const void* k, const void* v, co
                                  kda_dtype o_dt, kda_dtype state_dt, void* o, void* final_state,
                                  void* workspace, cudaStream_t stream,
                                  const OutputNorm& norm = OutputNorm{},
-                                 ChunkedMode mode = ChunkedMode::kFull) {
+                                 ChunkedMode mode = ChunkedMode::kFull,
+                                 const int32_t** cu_used = nullptr) {
   if (act == KDA_CONV_SILU)
     return launch_chunked_t<KDA_CONV_SILU>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
                                            cu_host, N, H, o_dt, state_dt, o, final_state, workspace, norm,
-                                           mode, stream);
+                                           mode, stream, cu_used);
   return launch_chunked_t<KDA_CONV_NONE>(q, k, v, g, beta, conv_w, init_state, init_conv, cu_dev,
                                          cu_host, N, H, o_dt, state_dt, o, final_state, workspace, norm,
-                                         mode, stream);
+                                         mode, stream, cu_used);
 }
 
 }  // namespace kda
