@@ -28,6 +28,8 @@ MUTANTS = {
     "q not normalised": ("qh[c] *= nq;", "qh[c] *= 1.0;"),
     "norm without the square root": ("nk = 1.0 / sqrt(nk + KDA_ORACLE_NORM_EPS);",
                                      "nk = 1.0 / (nk + KDA_ORACLE_NORM_EPS);"),
+    "SiLU with the sigmoid of -y": ("y = y / (1.0 + exp(-y));", "y = y / (1.0 + exp(y));"),
+    "SiLU without the factor y": ("y = y / (1.0 + exp(-y));", "y = 1.0 / (1.0 + exp(-y));"),
     "bf16 storage truncates": ("ldexp(nearbyint(ldexp(x, shift)), -shift)", "ldexp(floor(ldexp(x, shift)), -shift)"),
 }
 

@@ -146,6 +146,28 @@ def test_conv_matches_numpy_convolve_and_tap_order():
     assert np.abs(np.delete(p.o, 5, axis=1)).max() < 1e-9
 
 
+def test_silu_closed_form_through_recall():
+    """The SiLU activation of the conv (act = 1), pinned by values rather than by
+    its formula: with identity taps, beta = 1 and q = k of norm ~1e3, o_t = v'_t,
+    the activated value.  At x = ln a the sigmoid is a / (1 + a), so
+    SiLU(ln a) = ln a * a / (1 + a); and SiLU(x) - SiLU(-x) = x,
+    SiLU(x) + SiLU(-x) = x tanh(x / 2) (numpy's tanh)."""
+    r = _rng(41)
+    T = 8
+    x = r.standard_normal((T, D)) * 1e3
+    a = np.exp(r.uniform(-4.0, 4.0, (T, D)))
+    lv = np.log(a)
+    lv[:, 0] = 0.0  # SiLU(0) = 0
+    outs = []
+    for sign in (1.0, -1.0):
+        p = _solve(HeadProblem(x, x, sign * lv, np.zeros((T, D)), np.ones(T), IDENT, IDENT, IDENT, None, None, 1))
+        outs.append(p.o)
+    assert np.abs(outs[0] - lv * a / (1.0 + a)).max() < 1e-9
+    assert np.abs(outs[0][:, 0]).max() < 1e-12
+    assert np.abs((outs[0] - outs[1]) - lv).max() < 1e-9
+    assert np.abs((outs[0] + outs[1]) - lv * np.tanh(lv / 2.0)).max() < 1e-9
+
+
 def test_key_conv_and_single_write():
     """One write at t = 0 (beta = 1, S_0 = 0, g = 0), then beta = 0: o_t =
     v_0 * (k_hat_0 . q_hat_t), with k_hat_0, q_hat_t, v_0 from numpy.convolve."""
