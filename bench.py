@@ -353,7 +353,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=6, help="0 skips the end-to-end leg")
+    ap.add_argument("--e2e-steps", type=int, default=16,
+                    help="timed steps of the pipelined end-to-end loop (its fill and drain are spread over them); 0 skips it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-other-prefill", action="store_true",
                     help="skip the 4 x 4096 and varlen prefill legs")
@@ -653,8 +654,52 @@ def run_e2e(args, world, stream, inp, d, o, S, prefill_into, tokens_per_rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(start.elapsed_time(stop), world)
     value = world * tokens_per_rank * args.e2e_steps / (e2e_ms / 1e3)
+
+    # the host link alone: the same copies with nothing else on the device, each
+    # direction timed on its own stream (max over ranks)
+    def link_gbs(copy_stream, copies, nbytes, reps=3):
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        with torch.cuda.stream(copy_stream):
+            a.record(copy_stream)
+            for _ in range(reps):
+                copies()
+            z.record(copy_stream)
+        torch.cuda.synchronize()
+        return nbytes * reps / (max_over_ranks(a.elapsed_time(z), world) / 1e3) / 1e9
+
+    dd0, ob0, sb0 = sets[0]
+    ups = lambda: [dd0[n].copy_(t, non_blocking=True) for n, t in pin.items()]  # noqa: E731
+    downs = lambda: (o_host.copy_(ob0, non_blocking=True), S_host.copy_(sb0, non_blocking=True))  # noqa: E731
+    h2d_alone = link_gbs(up, ups, h2d)
+    d2h_alone = link_gbs(down, downs, d2h)
+    # both directions at once, as the pipelined loop runs them: the copy-only step time
+    reps = 3
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    a.record(stream)
+    up.wait_event(a)
+    down.wait_event(a)
+    for _ in range(reps):
+        with torch.cuda.stream(up):
+            ups()
+        with torch.cuda.stream(down):
+            downs()
+    stream.wait_stream(up)
+    stream.wait_stream(down)
+    z.record(stream)
+    torch.cuda.synchronize()
+    copy_ms = max_over_ranks(a.elapsed_time(z), world) / reps
+    ceiling = world * tokens_per_rank / (copy_ms / 1e3)
     return {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": args.e2e_steps, "pipelined": "inputs of step i+1 up and results of step i-1 down while step i runs"}
+            "steps": args.e2e_steps, "pipelined": "inputs of step i+1 up and results of step i-1 down while step i runs",
+            "link": {"bound": "host link", "h2d_gbs_alone": h2d_alone, "d2h_gbs_alone": d2h_alone,
+                     "copy_ms_per_step": copy_ms, "ceiling": ceiling, "frac": value / ceiling,
+                     "h2d_gbs_in_e2e": h2d * args.e2e_steps / (e2e_ms / 1e3) / 1e9,
+                     "note": "ceiling = the step's copies alone (pinned host memory, same tensors, both "
+                             "directions at once, 3 repeats), no kernel"}}
 
 
 def run_decode(args, world, dev, stream, kda, hbm_peak, state_dtype=torch.float32):

@@ -421,9 +421,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       float s8[8], s4[4], s2[2];
       const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float lo = y[j] * y[j], hi = y[j + 8] * y[j + 8];
-        s8[j] = (b4 ? hi : lo) + __shfl_xor_sync(0xffffffffu, b4 ? lo : hi, 16);
+      for (int j = 0; j < 8; ++j) {  // the squares of rows j and j + 8 in one packed multiply
+        const float2 sq = mul2(make_float2(y[j], y[j + 8]), make_float2(y[j], y[j + 8]));
+        s8[j] = (b4 ? sq.y : sq.x) + __shfl_xor_sync(0xffffffffu, b4 ? sq.x : sq.y, 16);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -447,16 +447,25 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       const __nv_bfloat16* zt =
           reinterpret_cast<const __nv_bfloat16*>(sm + SCAN_OST + (c & 1) * OST_BYTES + OST_Z);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < 16; j += 2) {
         // sigmoid(z) = 1 / (1 + 2^t), t = -z log2 e (capped at 64, where sigmoid < 2^-64): one ex2 on
         // the special-function pipe, the reciprocal by three Newton steps on the FMA pipe from a
-        // bit-pattern estimate (relative error below 2^-22 for 1 <= d <= 2^64 + 1)
-        const float d = 1.f + tc::exp2_fast(fminf(-to_f(zt[(t0 + j) * D + v]) * 1.4426950408889634f, 64.f));
-        float rc = __int_as_float(0x7EF311C3 - __float_as_int(d));
-        rc = fmaf(rc, fmaf(-d, rc, 1.f), rc);
-        rc = fmaf(rc, fmaf(-d, rc, 1.f), rc);
-        const float gate = fmaf(rc, fmaf(-d, rc, 1.f), rc);
-        y[j] *= __shfl_sync(0xffffffffu, rs, j) * wn * gate;
+        // bit-pattern estimate (relative error below 2^-22 for 1 <= d <= 2^64 + 1); rows j and
+        // j + 1 share each packed instruction, every lane rounded as the scalar form would be
+        const float2 t = mul2(make_float2(to_f(zt[(t0 + j) * D + v]), to_f(zt[(t0 + j + 1) * D + v])),
+                              dup2(-1.4426950408889634f));
+        const float2 d = add2(dup2(1.f), make_float2(tc::exp2_fast(fminf(t.x, 64.f)), tc::exp2_fast(fminf(t.y, 64.f))));
+        const float2 nd = mul2(d, dup2(-1.f));
+        float2 rc = make_float2(__int_as_float(0x7EF311C3 - __float_as_int(d.x)),
+                                __int_as_float(0x7EF311C3 - __float_as_int(d.y)));
+        rc = fma2(rc, fma2(nd, rc, dup2(1.f)), rc);
+        rc = fma2(rc, fma2(nd, rc, dup2(1.f)), rc);
+        rc = fma2(rc, fma2(nd, rc, dup2(1.f)), rc);
+        const float2 sc = mul2(mul2(make_float2(__shfl_sync(0xffffffffu, rs, j), __shfl_sync(0xffffffffu, rs, j + 1)),
+                                    dup2(wn)), rc);
+        const float2 yy = mul2(make_float2(y[j], y[j + 1]), sc);
+        y[j] = yy.x;
+        y[j + 1] = yy.y;
       }
       return true;
     };
@@ -472,7 +481,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       tc::ld_wait();
       if constexpr (EPI) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) r[j] = rr[j] * (r[j] + du[j]);
+        for (int j = 0; j < 16; j += 2) {
+          const float2 a = mul2(make_float2(rr[j], rr[j + 1]), add2(make_float2(r[j], r[j + 1]), make_float2(du[j], du[j + 1])));
+          r[j] = a.x;
+          r[j + 1] = a.y;
+        }
         if (!epilogue(c, r)) return false;
 #pragma unroll
         for (int j = 0; j < 16; ++j) st[(t0 + j) * D + v] = from_f<Tout>(r[j]);
