@@ -304,26 +304,41 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float rqv[8] = {rq0.x, rq0.y, rq0.z, rq0.w, rq1.x, rq1.y, rq1.z, rq1.w};
       tc::ld_wait();
       float kb[8];
+      // rows r and r + 1 share each packed multiply and add (every lane rounded
+      // as the scalar form rounds it); exponentials and tf32 roundings are per row
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const float G = gl[r] + carry;
-        const float d = G - gm;
-        const float e1 = tc::exp2_fast(d), e2 = tc::exp2_fast(-d), e3 = tc::exp2_fast(G);
-        const float kh = yk[r] * rkv[r], qh = yq[r] * rqv[r];
-        // B operand of the P Gram; A rows (block of the own half, and for
-        // half 0 the rows read against half 1)
-        *reinterpret_cast<float*>(sm + P_GB + tc::sw128o(r0 + 8 * g, r, ch, 64)) = tc::to_tf32(qh * e1);
+      for (int r = 0; r < 8; r += 2) {
+        const float2 G = add2(make_float2(gl[r], gl[r + 1]), dup2(carry));
+        const float2 d = add2(G, dup2(-gm));
+        const float2 e1 = make_float2(tc::exp2_fast(d.x), tc::exp2_fast(d.y));
+        const float2 e2 = make_float2(tc::exp2_fast(-d.x), tc::exp2_fast(-d.y));
+        const float2 e3 = make_float2(tc::exp2_fast(G.x), tc::exp2_fast(G.y));
+        const float2 kh = mul2(make_float2(yk[r], yk[r + 1]), make_float2(rkv[r], rkv[r + 1]));
+        const float2 qh = mul2(make_float2(yq[r], yq[r + 1]), make_float2(rqv[r], rqv[r + 1]));
         // e^{G_{m_1} - G_t}: e2 for half 1; <= 1 for half 0
-        const float a1 = hb ? e2 : tc::exp2_fast(g1m - G);
-        *reinterpret_cast<float*>(sm + P_GA + tc::sw128o(32 + r0 + 8 * g, r, ch, GA_ROWS)) = tc::to_tf32(kh * a1);
-        if (!hb)
-          *reinterpret_cast<float*>(sm + P_GA + tc::sw128o(r0 + 8 * g, r, ch, GA_ROWS)) = tc::to_tf32(kh * e2);
-        *reinterpret_cast<float*>(rec + REC_RA + tc::sw128o(qrow0 + r0 + 8 * g, r, ch, 128)) = tc::to_tf32(qh * e3);
+        const float2 a1 = hb ? e2 : make_float2(tc::exp2_fast(g1m - G.x), tc::exp2_fast(g1m - G.y));
+        const float2 pb = mul2(qh, e1), pa = mul2(kh, a1), pq = mul2(qh, e3);
         // e^{G_C - G_t} = e^{G_C - G_{m_1}} e^{G_{m_1} - G_t}: for half 0 both
         // factors are <= 1 (an underflow only drops what is below fp32 anyway)
-        kb[r] = tc::to_tf32(kh * (egcm * a1));
-        yq[r] = kh * e1;  // stash: M Gram B operand
-        yk[r] = kh * e3;  // stash: e^{G} k for W
+        const float2 kbr = mul2(kh, mul2(dup2(egcm), a1));
+        const float2 ke1 = mul2(kh, e1), ke3 = mul2(kh, e3);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int rr = r + u;
+          // B operand of the P Gram; A rows (block of the own half, and for
+          // half 0 the rows read against half 1)
+          *reinterpret_cast<float*>(sm + P_GB + tc::sw128o(r0 + 8 * g, rr, ch, 64)) = tc::to_tf32(u ? pb.y : pb.x);
+          *reinterpret_cast<float*>(sm + P_GA + tc::sw128o(32 + r0 + 8 * g, rr, ch, GA_ROWS)) =
+              tc::to_tf32(u ? pa.y : pa.x);
+          if (!hb)
+            *reinterpret_cast<float*>(sm + P_GA + tc::sw128o(r0 + 8 * g, rr, ch, GA_ROWS)) =
+                tc::to_tf32((u ? kh.y : kh.x) * (u ? e2.y : e2.x));
+          *reinterpret_cast<float*>(rec + REC_RA + tc::sw128o(qrow0 + r0 + 8 * g, rr, ch, 128)) =
+              tc::to_tf32(u ? pq.y : pq.x);
+          kb[rr] = tc::to_tf32(u ? kbr.y : kbr.x);
+        }
+        yq[r] = ke1.x; yq[r + 1] = ke1.y;  // stash: M Gram B operand
+        yk[r] = ke3.x; yk[r + 1] = ke3.y;  // stash: e^{G} k for W
       }
       tc::st8(tl + TC_YQ + r0 + 8 * g, yq);
       tc::st8(tl + TC_YK + r0 + 8 * g, yk);
