@@ -95,6 +95,30 @@ def test_gated_prefill_several_chunks(silu):
         _check(y[s0:s1, h].float().cpu().numpy(), yr, 2e-2, f"seq {n} head {h}")
 
 
+@pytest.mark.parametrize("silu", [0, 1])
+def test_gated_prefill_many_chains(silu):
+    """More than 96 (segment, head) chains: the preparation and the scan run one
+    after the other (the schedule of the multi-sequence workloads), with the
+    epilogue instance of the scan; ragged lengths, conv history and initial
+    states.  Every pair against the oracle; state and conv tails bit-identical
+    to the plain call."""
+    lens = [300, 64, 1, 190, 65, 7, 128, 250]
+    inp = ki.make_prefill(lens, 16, torch.bfloat16, 39 + silu, state_std=0.02, conv_history=True)
+    assert inp.num_seqs * inp.num_heads > 96
+    d = to_dev(inp)
+    T, H = inp.q.shape[0], inp.q.shape[1]
+    z, w = ki.make_output_norm(T, H, 39)
+    y, S, tail = run_prefill(inp, dev_inputs=d, act=silu, gate=z.cuda(), norm_weight=w.cuda(), norm_eps=EPS)
+    _, S0, tail0 = run_prefill(inp, dev_inputs=d, act=silu)
+    assert torch.equal(S, S0) and torch.equal(tail, tail0)
+    ref = oracle.prefill(inp, act=silu)
+    yc, zc = y.float().cpu().numpy(), z.double().numpy()
+    for (n, h), p in ref.items():
+        s0, s1 = int(inp.cu_seqlens[n]), int(inp.cu_seqlens[n + 1])
+        yr = epilogue.gated_rmsnorm(p.o, zc[s0:s1, h], w.double().numpy(), EPS)
+        _check(yc[s0:s1, h], yr, 2e-2, f"seq {n} head {h}")
+
+
 def test_gated_prefill_long_context_full_size():
     """1 x 65,536 tokens, 64 heads, with the epilogue: every head against the
     oracle, in the launch configuration the benchmark times (overlapped)."""
