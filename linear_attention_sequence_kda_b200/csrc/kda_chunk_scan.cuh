@@ -247,9 +247,13 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
     auto all = [](bool x) { return __all_sync(0xffffffffu, x) != 0; };
     // start the record of chunk j on its way into L2 (two chunks ahead of its
     // load), so that its bulk copies wait on L2 rather than HBM; a record the
-    // preparation kernel has not published yet is left alone
+    // preparation kernel has not published yet is left alone.  Only beside a
+    // running preparation kernel and without the output epilogue: there the
+    // chain waits on its record loads.  With every chain streaming records
+    // from HBM at once (preparation done first), or with the epilogue's longer
+    // compute step, the extra prefetch traffic made the call slower.
     auto warm = [&](int j) {
-      if (leader && j < nchunks && (!rdy || *reinterpret_cast<const volatile int*>(rdy + (int64_t)j * H)))
+      if (!EPI && rdy && leader && j < nchunks && *reinterpret_cast<const volatile int*>(rdy + (int64_t)j * H))
         tc::prefetch_l2(rec0 + (int64_t)j * rec_stride, REC_BYTES);
     };
     bool ok = true;
