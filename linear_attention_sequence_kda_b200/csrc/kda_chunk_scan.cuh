@@ -232,10 +232,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constan
       }
       ++n_v;
     };
-    // a record piece that the tensor core has read is dead: drop its lines
-    // (unless the records are kept for another scan over them)
+    // a record piece that the tensor core has read is dead: drop its lines, so
+    // that a record written moments ago by the concurrently running
+    // preparation kernel is never written back to HBM (not when the records
+    // are kept for another scan over them, and not after a preparation kernel
+    // that ran first: its records have long left L2, and the discards only
+    // cost time)
     auto drop = [&](const uint8_t* base, uint32_t bytes) {
-      if (keep_records) return;
+      if (keep_records || !ready) return;
       for (uint32_t off = 128u * lane; off < bytes; off += 128u * 32u) discard_l2(base + off);
     };
     // with the prep kernel running concurrently, a chunk's record is read
