@@ -436,6 +436,7 @@ def main():
                                                        max(3, args.steps // 2), hbm_peak, bf16_peak, peak_src)[0]
         other_legs["prefill_long_gated"] = run_prefill_leg(args, world, dev, stream, kda, inp, args.steps,
                                                            hbm_peak, bf16_peak, peak_src, gated=True)[0]
+        other_legs["prefill_long_scan_only"] = run_scan_only(args, world, dev, stream, kda, inp, args.steps)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -546,6 +547,39 @@ def run_prefill_leg(args, world, dev, stream, kda, inp, steps, hbm_peak, bf16_pe
     del d, o, S, ws
     torch.cuda.empty_cache()
     return leg, None
+
+
+def run_scan_only(args, world, dev, stream, kda, inp, steps):
+    """The state scan alone on the long-context workload: one record-keeping
+    call (kda_prefill_records) prepares every chunk record, then `steps`
+    kda_prefill_scan calls over those records are timed like the prefill leg.
+    With every record ready, the call is the 64 serial chains: its time over
+    the chunk count is the chain's time per chunk."""
+    d = {n: getattr(inp, n).to(dev) for n in ("q", "k", "v", "g", "beta", "conv_w")}
+    cu_dev = torch.from_numpy(inp.cu_seqlens).to(dev)
+    N, Hh = inp.num_seqs, inp.num_heads
+    o = torch.empty(d["q"].shape, dtype=torch.float32, device=dev)
+    S = torch.empty((N, Hh, D, D), dtype=torch.float32, device=dev)
+    tail = torch.empty((N, 3, 3, Hh * D), dtype=torch.bfloat16, device=dev)
+    max_len = int(np.diff(inp.cu_seqlens).max())
+    ws = torch.empty(kda.workspace_size(N, inp.total_tokens, Hh, max_len), dtype=torch.uint8, device=dev)
+
+    def call(mode):
+        kda.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["conv_w"], inp.cu_seqlens, cu_dev, None, None,
+                    o=o, final_state=S, conv_tail=tail, workspace=ws, stream=stream, mode=mode)
+
+    call("records")
+    total_ms, per_step = timed(lambda: call("scan"), steps, args.warmup, world, stream)
+    assert kda.check_async_status(stream) == 0
+    chunks = -(-max_len // 64)
+    ms = total_ms / steps
+    out = {"workload": f"kda_prefill_scan over kept records: {N} x {inp.total_tokens} tokens, {Hh} heads x 128 "
+                       f"({N * Hh} chains of {chunks} chunks)",
+           "ms_per_step": ms, "steps": steps, "us_per_chunk": ms * 1e3 / chunks,
+           "gpu_launches": steps * 2}
+    del d, o, S, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def oracle_per_workload():
