@@ -37,9 +37,10 @@
 //               conv of v for chunk i + 1 while MMA2 of chunk i runs.
 //   warp 16     one thread issues the MMAs.
 //   warp 17     issues the loads (one thread), each as soon as the product that
-//               read the previous contents of its buffer is done, and drops the
-//               consumed record from L2 (all lanes), so that a record read soon
-//               after it was written never reaches HBM.
+//               read the previous contents of its buffer is done; beside a
+//               running preparation kernel it also drops the consumed record
+//               from L2 (all lanes), so that a record read soon after it was
+//               written never reaches HBM.
 //   warp 18     one thread stores the output tiles (double-buffered staging),
 //               so that global stores never hold up the compute warps (with
 //               the epilogue it also loads the gate tile of chunk i + 2 once
